@@ -1,0 +1,407 @@
+"""CPU oracle for the SmoothQuant W8A8 linear layer.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+``bench.py`` (its ``cpu_baseline`` leg and ``--impl reference`` arm) may import
+this package.  The product package never imports it, and it never imports the
+product package: the two share no code.  Inputs come from ``synth`` (seeded
+generators only, none of the method's arithmetic).
+
+The scalar work lives in ``sq_oracle.c`` (plain C, fp32 operations written out
+one by one, ``-ffp-contract=off``); this module compiles it, wraps it with
+ctypes/numpy and adds the fp64 numpy checks and the per-workload pipelines.
+
+Sources (the five pages on SmoothQuant):
+  [KWKR]  kwkr.cn blog on SmoothQuant W8A8 (sections 1.2, 2.1-2.3, 3.1-3.3, 5.2)
+  [TBR8]  tbr8.org article on activation outliers (PyTorch toy example)
+  [PWWT]  pwwt.cn "SmoothQuant技术解析：LLM模型INT8无损量化实践" (2.2, 3.1)
+  [AIU]   aiunderstanding.org "SmoothQuant 和激活量化" (technical insight)
+  [ADR10] blog.yoooo.fun "010. SmoothQuant Integration" (context, key design
+          points 1-6, consequences)
+
+Parity pins (tests/test_oracle_pins.py; tests/golden/ fixtures):
+  f16/bf16 conversions  -- exhaustive / random vs numpy and torch CPU casts
+  quant rule            -- [KWKR] 1.2 worked numbers (golden), RNE ties
+  calib_absmax          -- numpy reduction, running-max == concatenated max,
+                           outlier channel reads back exactly 100.0
+  smooth_scales         -- alpha = 0.5 / 1 / 0 closed forms, clamp at 1e-5
+  static_scale          -- brute force over every smoothed calibration value
+                           (bit-exact: fl() is monotone)
+  quant_weight          -- row argmax -> +-127, |w' - q*scale| <= scale/2
+  smooth_quant_act      -- same bounds, static and per-token
+  gemm_s32              -- numpy int64 matmul (ragged shapes)
+  dequant               -- fp64 product within one fp32 rounding + one output
+                           rounding
+  rmsnorm_quant         -- fp64 unfused RMSNorm then x/s, within rounding
+  silu_mul_bf16         -- math.exp closed form; silu(0) = 0, silu(g) -> g
+  mse_f16, gemm_f16_ref -- numpy fp64 mean / matmul
+  identity              -- fp64 XW^T == (X diag(s)^-1)(W diag(s))^T, 1e-9
+  quality gain          -- [ADR10] consequences: ~10x lower error with
+                           smoothing on the outlier layer; not worse on normal
+                           activations; smoothing after quantisation gives no
+                           gain ([KWKR] 5.2).  The exact factor is
+                           "parity unpinned" (the page gives only "about an
+                           order of magnitude"); the test bounds it below.
+  alpha_search          -- argmin over the grid equals an fp64 numpy
+                           re-evaluation; the chosen MSE is <= both extremes.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sq_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_SO = os.path.join(_BUILD, "libsq_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+F32, F16, BF16 = 0, 1, 2
+STATIC, PER_TOKEN = 0, 1
+ALPHA_GRID = (0.25, 0.5, 0.75, 1.0)   # [ADR10] key design point 2
+ALPHA_DEFAULT = 0.5                    # [KWKR] 2.2, [AIU], [ADR10] key design point 2
+CLAMP_MIN = 1e-5                       # [TBR8] s.clamp(min=1e-5)
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+
+
+def build(force: bool = False) -> str:
+    """Compile sq_oracle.c into oracle/_build/libsq_oracle.so (gcc, OpenMP)."""
+    os.makedirs(_BUILD, exist_ok=True)
+    if (not force and os.path.exists(_SO)
+            and os.path.getmtime(_SO) >= os.path.getmtime(_SRC)):
+        return _SO
+    tmp = _SO + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
+           "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _SO)
+    return _SO
+
+
+def lib():
+    global _lib
+    with _lock:
+        if _lib is None:
+            L = ctypes.CDLL(build())
+            L.oracle_f16_to_f32.restype = ctypes.c_float
+            L.oracle_f16_to_f32.argtypes = [ctypes.c_uint16]
+            L.oracle_bf16_to_f32.restype = ctypes.c_float
+            L.oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
+            L.oracle_f32_to_f16.restype = ctypes.c_uint16
+            L.oracle_f32_to_f16.argtypes = [ctypes.c_float]
+            L.oracle_f32_to_bf16.restype = ctypes.c_uint16
+            L.oracle_f32_to_bf16.argtypes = [ctypes.c_float]
+            L.oracle_recip.restype = ctypes.c_float
+            L.oracle_recip.argtypes = [ctypes.c_float]
+            L.oracle_quant.restype = ctypes.c_int8
+            L.oracle_quant.argtypes = [ctypes.c_float]
+            L.oracle_calib_absmax.argtypes = [_P, ctypes.c_int, _I64, _I64, _I64, _P]
+            L.oracle_smooth_scales.argtypes = [_P, _P, _I64, ctypes.c_float, _P]
+            L.oracle_static_scale.restype = ctypes.c_float
+            L.oracle_static_scale.argtypes = [_P, _P, _I64]
+            L.oracle_quant_weight.argtypes = [_P, ctypes.c_int, _I64, _I64, _P, _P, _P]
+            L.oracle_smooth_quant_act.argtypes = [_P, ctypes.c_int, _I64, _I64, _P, ctypes.c_int, _P, _P]
+            L.oracle_gemm_s32.argtypes = [_P, _P, _I64, _I64, _I64, _P]
+            L.oracle_dequant.argtypes = [_P, _I64, _I64, _P, ctypes.c_int, _P, _P, ctypes.c_int, _P]
+            L.oracle_dequant_f32.argtypes = [_P, _I64, _I64, _P, ctypes.c_int, _P, _P]
+            L.oracle_rmsnorm_quant.argtypes = [_P, ctypes.c_int, _I64, _I64, _P, _P, ctypes.c_float,
+                                               _P, _P, _P, _P]
+            L.oracle_silu_mul_bf16.argtypes = [_P, _P, _I64, _P]
+            L.oracle_mse_f16.restype = ctypes.c_double
+            L.oracle_mse_f16.argtypes = [_P, _P, _I64]
+            L.oracle_gemm_f16_ref.argtypes = [_P, _P, _I64, _I64, _I64, _P]
+            L.oracle_to_f32_array.argtypes = [_P, ctypes.c_int, _I64, _P]
+            L.oracle_from_f32_array.argtypes = [_P, _I64, ctypes.c_int, _P]
+            _lib = L
+    return _lib
+
+
+# --------------------------------------------------------------------------
+# numpy helpers.  16-bit tensors travel as uint16 bit patterns (bf16 has no
+# numpy dtype); fp16 arrays are accepted and viewed as uint16.
+# --------------------------------------------------------------------------
+
+def _dtcode(a: np.ndarray, dt: int | None) -> tuple[np.ndarray, int]:
+    if dt is None:
+        if a.dtype == np.float32:
+            dt = F32
+        elif a.dtype == np.float16:
+            dt = F16
+        else:
+            raise TypeError("bf16 data is passed as uint16 with dt=BF16")
+    if dt == F32:
+        a = np.ascontiguousarray(a, dtype=np.float32)
+    else:
+        a = np.ascontiguousarray(a).view(np.uint16)
+    return a, dt
+
+
+def _ptr(a: np.ndarray | None):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def to_f32(a: np.ndarray, dt: int) -> np.ndarray:
+    """Widen a 16-bit bit-pattern array (or an fp32 array) to fp32, exactly."""
+    if dt == F32:
+        return np.array(a, dtype=np.float32)
+    bits = np.ascontiguousarray(a).view(np.uint16)
+    out = np.empty(bits.shape, np.float32)
+    lib().oracle_to_f32_array(_ptr(bits), dt, bits.size, _ptr(out))
+    return out
+
+
+def from_f32(a: np.ndarray, dt: int) -> np.ndarray:
+    """Round fp32 values to dt (RNE); 16-bit results are uint16 bit patterns."""
+    a = np.ascontiguousarray(a, np.float32)
+    if dt == F32:
+        return a.copy()
+    out = np.empty(a.shape, np.uint16)
+    lib().oracle_from_f32_array(_ptr(a), a.size, dt, _ptr(out))
+    return out
+
+
+def quant(v: float) -> int:
+    """[KWKR] 1.2: x_q = round(x / s); RNE, saturate to +-127."""
+    return int(lib().oracle_quant(float(v)))
+
+
+def recip(v: float) -> float:
+    return float(lib().oracle_recip(float(v)))
+
+
+def calib_absmax(x: np.ndarray, dt: int | None = None, absmax: np.ndarray | None = None) -> np.ndarray:
+    """a1/a2 -- running per-column max|x| ([KWKR] 3.1; [ADR10] add_batch)."""
+    x, dt = _dtcode(x, dt)
+    rows, cols = x.shape
+    out = np.zeros(cols, np.float32) if absmax is None else absmax
+    assert out.dtype == np.float32 and out.flags.c_contiguous
+    lib().oracle_calib_absmax(_ptr(x), dt, rows, cols, cols, _ptr(out))
+    return out
+
+
+def smooth_scales(act_max: np.ndarray, w_max: np.ndarray, alpha: float = ALPHA_DEFAULT) -> np.ndarray:
+    """a3 -- s_j = max|X_j|^a / max|W_j|^(1-a) ([KWKR] 2.2; [AIU]; [ADR10] step 1)."""
+    a = np.ascontiguousarray(act_max, np.float32)
+    w = np.ascontiguousarray(w_max, np.float32)
+    s = np.empty_like(a)
+    lib().oracle_smooth_scales(_ptr(a), _ptr(w), len(a), float(alpha), _ptr(s))
+    return s
+
+
+def static_scale(act_max: np.ndarray, s: np.ndarray) -> np.float32:
+    """a3 -- closed-form per-tensor scale max_j(act_max_j/s_j)/127 ([ADR10] point 1)."""
+    a = np.ascontiguousarray(act_max, np.float32)
+    s = np.ascontiguousarray(s, np.float32)
+    return np.float32(lib().oracle_static_scale(_ptr(a), _ptr(s), len(a)))
+
+
+def quant_weight(w: np.ndarray, s: np.ndarray, dt: int | None = None):
+    """a4 -- W' = W diag(s), per-row INT8 ([KWKR] 3.2-3.3; [ADR10] step 3)."""
+    w, dt = _dtcode(w, dt)
+    N, K = w.shape
+    s = np.ascontiguousarray(s, np.float32)
+    wq = np.empty((N, K), np.int8)
+    ws = np.empty(N, np.float32)
+    lib().oracle_quant_weight(_ptr(w), dt, N, K, _ptr(s), _ptr(wq), _ptr(ws))
+    return wq, ws
+
+
+def smooth_quant_act(x: np.ndarray, s: np.ndarray, mode: int, a_scale=None, dt: int | None = None):
+    """a5/a5' -- x/s then INT8 ([KWKR] 3.2, 5.2: smoothing precedes quantisation).
+
+    static: ``a_scale`` is the per-tensor scale; per-token: returns (xq, a[M]).
+    """
+    x, dt = _dtcode(x, dt)
+    M, K = x.shape
+    s = np.ascontiguousarray(s, np.float32)
+    xq = np.empty((M, K), np.int8)
+    if mode == STATIC:
+        a = np.array([a_scale], np.float32).ravel()[:1].copy()
+    else:
+        a = np.empty(M, np.float32)
+    lib().oracle_smooth_quant_act(_ptr(x), dt, M, K, _ptr(s), mode, _ptr(a), _ptr(xq))
+    return xq, a
+
+
+def gemm_s32(xq: np.ndarray, wq: np.ndarray) -> np.ndarray:
+    """a6 -- acc = xq . wq^T in exact int32."""
+    xq = np.ascontiguousarray(xq, np.int8)
+    wq = np.ascontiguousarray(wq, np.int8)
+    M, K = xq.shape
+    N, K2 = wq.shape
+    assert K == K2
+    acc = np.empty((M, N), np.int32)
+    lib().oracle_gemm_s32(_ptr(xq), _ptr(wq), M, N, K, _ptr(acc))
+    return acc
+
+
+def dequant(acc: np.ndarray, a_scale: np.ndarray, mode: int, w_scale: np.ndarray,
+            out_dt: int, bias: np.ndarray | None = None) -> np.ndarray:
+    """a6 epilogue -- fmaf((float)acc, fl(a_m*w_n), bias_n) rounded to out_dt.
+
+    Returns fp32 values (out_dt F32) or uint16 bit patterns (F16/BF16).
+    """
+    acc = np.ascontiguousarray(acc, np.int32)
+    M, N = acc.shape
+    a = np.ascontiguousarray(a_scale, np.float32).ravel()
+    ws = np.ascontiguousarray(w_scale, np.float32)
+    if bias is not None:
+        bias, _ = _dtcode(bias, out_dt)
+    y = np.empty((M, N), np.float32 if out_dt == F32 else np.uint16)
+    lib().oracle_dequant(_ptr(acc), M, N, _ptr(a), mode, _ptr(ws), _ptr(bias), out_dt, _ptr(y))
+    return y
+
+
+def dequant_f32(acc, a_scale, mode, w_scale) -> np.ndarray:
+    acc = np.ascontiguousarray(acc, np.int32)
+    M, N = acc.shape
+    a = np.ascontiguousarray(a_scale, np.float32).ravel()
+    ws = np.ascontiguousarray(w_scale, np.float32)
+    y = np.empty((M, N), np.float32)
+    lib().oracle_dequant_f32(_ptr(acc), M, N, _ptr(a), mode, _ptr(ws), _ptr(y))
+    return y
+
+
+def rmsnorm_quant(x, gamma, s, eps, a_static, dt: int | None = None, r_given=None):
+    """a8 -- RMSNorm with 1/s folded into gamma, then INT8 ([KWKR] 2.3, 3.2; [AIU]).
+
+    Returns (xq, r) where r[m] = 1/sqrt(mean x^2 + eps) (or ``r_given``).
+    """
+    x, dt = _dtcode(x, dt)
+    M, d = x.shape
+    g = np.ascontiguousarray(gamma, np.float32)
+    s = np.ascontiguousarray(s, np.float32)
+    a = np.array([a_static], np.float32).ravel()[:1].copy()
+    rg = None if r_given is None else np.ascontiguousarray(r_given, np.float32)
+    xq = np.empty((M, d), np.int8)
+    r = np.empty(M, np.float32)
+    lib().oracle_rmsnorm_quant(_ptr(x), dt, M, d, _ptr(g), _ptr(s), float(eps), _ptr(a),
+                               _ptr(rg), _ptr(xq), _ptr(r))
+    return xq, r
+
+
+def silu_mul_bf16(g: np.ndarray, u: np.ndarray) -> np.ndarray:
+    """a9 -- h = silu(g) * u, rounded to bf16 (uint16 bits)."""
+    g = np.ascontiguousarray(g, np.float32)
+    u = np.ascontiguousarray(u, np.float32)
+    h = np.empty(g.shape, np.uint16)
+    lib().oracle_silu_mul_bf16(_ptr(g), _ptr(u), g.size, _ptr(h))
+    return h
+
+
+def mse_f16(y_bits: np.ndarray, yref_bits: np.ndarray) -> float:
+    """a7 -- mean((y - y_ref)^2) in fp64 ([ADR10] point 2: output reconstruction error)."""
+    y = np.ascontiguousarray(y_bits).view(np.uint16)
+    r = np.ascontiguousarray(yref_bits).view(np.uint16)
+    return float(lib().oracle_mse_f16(_ptr(y), _ptr(r), y.size))
+
+
+def gemm_f16_ref(x_bits: np.ndarray, w_bits: np.ndarray) -> np.ndarray:
+    """a7 -- unquantised fp16 product, fp64-accumulated, rounded to fp16 (bits)."""
+    x = np.ascontiguousarray(x_bits).view(np.uint16)
+    w = np.ascontiguousarray(w_bits).view(np.uint16)
+    M, K = x.shape
+    N, _ = w.shape
+    y = np.empty((M, N), np.uint16)
+    lib().oracle_gemm_f16_ref(_ptr(x), _ptr(w), M, N, K, _ptr(y))
+    return y
+
+
+# --------------------------------------------------------------------------
+# fp64 numpy checks of the mathematics
+# --------------------------------------------------------------------------
+
+def identity_residual(X: np.ndarray, W: np.ndarray, s: np.ndarray) -> float:
+    """[KWKR] 2.1: Y = XW = (X diag(s)^-1)(diag(s) W); relative Frobenius residual in fp64.
+
+    W is [N,K] (out x in), so diag(s) scales its columns.
+    """
+    X = np.asarray(X, np.float64)
+    W = np.asarray(W, np.float64)
+    s = np.asarray(s, np.float64)
+    Y = X @ W.T
+    Ys = (X / s[None, :]) @ (W * s[None, :]).T
+    return float(np.linalg.norm(Y - Ys) / np.linalg.norm(Y))
+
+
+# --------------------------------------------------------------------------
+# Pipelines (the same sequence of steps the GPU path runs)
+# --------------------------------------------------------------------------
+
+@dataclass
+class LinearState:
+    act_max: np.ndarray
+    w_max: np.ndarray
+    s: np.ndarray
+    a_static: np.float32
+    wq: np.ndarray
+    w_scale: np.ndarray
+
+
+def calibrate_and_quantize(calib_batches, W, alpha=ALPHA_DEFAULT, x_dt=None, w_dt=None) -> LinearState:
+    """a1 -> a2 -> a3 -> a4 for one linear layer."""
+    K = W.shape[1]
+    act_max = np.zeros(K, np.float32)
+    for xb in calib_batches:
+        calib_absmax(xb, x_dt, act_max)
+    w_max = calib_absmax(W, w_dt)
+    s = smooth_scales(act_max, w_max, alpha)
+    a = static_scale(act_max, s)
+    wq, ws = quant_weight(W, s, w_dt)
+    return LinearState(act_max, w_max, s, a, wq, ws)
+
+
+def linear_forward(st: LinearState, X, mode: int, out_dt: int, x_dt=None, bias=None):
+    """a5/a5' -> a6: returns (xq, a_scale, acc, y)."""
+    if mode == STATIC:
+        xq, a = smooth_quant_act(X, st.s, STATIC, st.a_static, x_dt)
+    else:
+        xq, a = smooth_quant_act(X, st.s, PER_TOKEN, None, x_dt)
+    acc = gemm_s32(xq, st.wq)
+    y = dequant(acc, a, mode, st.w_scale, out_dt, bias)
+    return xq, a, acc, y
+
+
+def w8a8_output_f64(X, W, s, a_mode=STATIC, act_max=None):
+    """fp64 value of the dequantised W8A8 product (for the quality checks)."""
+    if a_mode == STATIC:
+        a = static_scale(act_max, s)
+        xq, av = smooth_quant_act(X, s, STATIC, a)
+    else:
+        xq, av = smooth_quant_act(X, s, PER_TOKEN)
+    wq, ws = quant_weight(W, s)
+    acc = gemm_s32(xq, wq).astype(np.float64)
+    av = av.astype(np.float64)
+    am = av[0] if a_mode == STATIC else av[:, None]
+    return acc * am * ws.astype(np.float64)[None, :]
+
+
+def alpha_search(x_held_bits, w_bits, act_max, w_max, grid=ALPHA_GRID, rel_tie=1e-6):
+    """a7 -- per-layer alpha grid search ([ADR10] point 2, honest search).
+
+    For each alpha: s -> static a -> weight quant -> held-batch quant -> INT8
+    GEMM -> fp16 output; MSE against the unquantised fp16 product.  Ties
+    within ``rel_tie`` go to the smaller alpha.  Returns (alpha, mses, y_ref).
+    """
+    y_ref = gemm_f16_ref(x_held_bits, w_bits)
+    mses = []
+    for al in grid:
+        s = smooth_scales(act_max, w_max, al)
+        a = static_scale(act_max, s)
+        wq, ws = quant_weight(w_bits, s, F16)
+        xq, av = smooth_quant_act(x_held_bits, s, STATIC, a, F16)
+        acc = gemm_s32(xq, wq)
+        y = dequant(acc, av, STATIC, ws, F16)
+        mses.append(mse_f16(y, y_ref))
+    best = 0
+    for i in range(1, len(grid)):
+        if mses[i] < mses[best] * (1.0 - rel_tie):
+            best = i
+    return grid[best], mses, y_ref
