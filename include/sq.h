@@ -1,0 +1,269 @@
+/*
+ * sq.h -- C ABI of libsq, the B200 (sm_100a) SmoothQuant W8A8 linear layer.
+ *
+ * The layer has four parts, each one or two calls below:
+ *   (1) per-input-channel calibration statistic max|X_j|       sq_calib_absmax
+ *   (2) smoothing factors, offline weight transform + INT8     sq_smooth_scales, sq_quant_weight
+ *   (3) runtime smoothing x/s + INT8 activation quantisation   sq_smooth_quant_act, sq_rmsnorm_quant
+ *   (4) INT8 x INT8 -> INT32 GEMM with a dequant epilogue       sq_linear_w8a8 (+ fused variants)
+ *
+ * Sources (the pages this layer is built from):
+ *   kwkr.cn blog on SmoothQuant W8A8 ("kwkr"), sections 1.2, 2.1-2.3, 3.1-3.3, 5.2
+ *   tbr8.org article on activation outliers ("tbr8"), PyTorch toy example
+ *   pwwt.cn "SmoothQuant技术解析：LLM模型INT8无损量化实践" ("pwwt"), 3.1
+ *   aiunderstanding.org "SmoothQuant 和激活量化" ("aiu"), technical insight
+ *   blog.yoooo.fun "010. SmoothQuant Integration" ("adr-010"), context and key design points
+ *
+ * Conventions for every call:
+ *   - Layouts are row-major.  X is [M, K] (tokens x input channels), W is [N, K]
+ *     (output x input channels, the nn.Linear layout), Y = X W^T is [M, N].
+ *     "Channel j" is the K index.
+ *   - Every pointer is DEVICE memory owned by the caller, unless a parameter
+ *     says "host".  The library allocates no device memory; calls that need
+ *     scratch take a caller-provided workspace.
+ *   - Calls are asynchronous and stream-ordered on `stream` (a cudaStream_t;
+ *     NULL is the legacy default stream) on the current CUDA device.
+ *   - Arguments are validated before any launch: null pointers, sizes, 16-byte
+ *     alignment where vector or TMA access needs it, dtype support.  A bad
+ *     argument returns an error status and launches nothing.  No call aborts,
+ *     prints, or throws across the ABI.
+ *   - Kernels that wait on on-chip barriers give up after a bounded time and
+ *     record SQ_ERR_TIMEOUT in a device-side error word instead of hanging;
+ *     sq_sync_status() synchronises a stream and reports (and clears) it.
+ *   - Quantised codes are symmetric INT8 in [-127, 127] (zero point 0; -128 is
+ *     never produced), rounded half to even.  Scales are fp32.
+ *   - Canonical fp32 order (bit-exact contract with the CPU oracle):
+ *       recip(v)      = v > 0 ? fl(1/v) : 0
+ *       act code      = q(fl(fl(x * recip(s_j)) * recip(a)))
+ *       weight code   = q(fl(fl(w * s_j) * recip(w_scale_n)))
+ *       absmax scale  = fl(max |value| / 127)
+ *       dequant       = fmaf((float)acc, fl(a_m * w_scale_n), bias_n)
+ *                       (fl((float)acc * fl(a_m * w_scale_n)) without bias),
+ *                       then one rounding to the output dtype.
+ */
+#ifndef SQ_H_
+#define SQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SQ_OK = 0,
+    SQ_ERR_INVALID_ARG = 1,   /* null pointer, bad size/dtype/mode, alpha outside [0,1] */
+    SQ_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement (shape limits) */
+    SQ_ERR_MISALIGNED = 3,    /* pointer or leading dimension not 16-byte aligned */
+    SQ_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed (see sq_last_cuda_error) */
+    SQ_ERR_TIMEOUT = 5,       /* a kernel's bounded barrier wait expired */
+    SQ_ERR_WORKSPACE = 6      /* workspace missing or smaller than required */
+} sq_status;
+
+typedef enum { SQ_F32 = 0, SQ_F16 = 1, SQ_BF16 = 2 } sq_dtype;
+
+typedef enum {
+    SQ_ACT_STATIC = 0,        /* one per-tensor scale a (adr-010 context step 3) */
+    SQ_ACT_PER_TOKEN = 1      /* one scale per row of X, computed at run time */
+} sq_act_mode;
+
+typedef void *sq_stream;      /* cudaStream_t */
+
+/* Human-readable name of a status.  Never NULL. */
+const char *sq_status_string(sq_status st);
+
+/* Last CUDA error code (cudaError_t as int) seen by this thread's calls, 0 if none. */
+int sq_last_cuda_error(void);
+
+/* Upper bound, in nanoseconds, on any single on-chip barrier wait inside this
+ * library's kernels (default 2e9 = 2 s; 0 restores the default).  A wait that
+ * runs out records SQ_ERR_TIMEOUT and the kernel returns without hanging. */
+void sq_set_wait_timeout_ns(unsigned long long ns);
+
+/* Synchronises `stream`, then returns SQ_ERR_TIMEOUT if any kernel of this
+ * library recorded a barrier timeout on the current device since the last
+ * check (and clears the record), SQ_ERR_CUDA if the stream reported an error,
+ * else SQ_OK. */
+sq_status sq_sync_status(sq_stream stream);
+
+/* -------------------------------------------------------------------------
+ * (1) Calibration statistic.  kwkr 3.1: per layer, per channel max of the
+ * activations (and of the weights); adr-010 key design point 1: the running
+ * per-channel max-abs is the only state calibration keeps (O(K) memory).
+ *
+ *   absmax[j] = max(absmax[j], max_{r < rows} |x[r * ld + j]|),  j < cols
+ *
+ * x: [rows, ld] of `dt` (fp32/fp16/bf16), ld >= cols (elements).  absmax:
+ * fp32 [cols], read and written (a running max: the caller zeroes it once and
+ * calls once per calibration batch).  The same call gives max|W_j| when x is
+ * the weight [N, K] (a column max over output rows).  Exact (a max of exactly
+ * widened values), so the result does not depend on launch order.  NaN inputs
+ * are not supported.  rows == 0 is a no-op.
+ * ------------------------------------------------------------------------- */
+sq_status sq_calib_absmax(const void *x, sq_dtype dt, int64_t rows, int64_t cols, int64_t ld,
+                          float *absmax, sq_stream stream);
+
+/* -------------------------------------------------------------------------
+ * (2a) Smoothing factors.  kwkr 2.2, aiu, adr-010 context step 1:
+ *
+ *   s_j = max(act_max_j, 1e-5)^alpha / max(w_max_j, 1e-5)^(1 - alpha)
+ *
+ * evaluated in fp64 and rounded once to fp32 (the clamp at 1e-5 follows tbr8's
+ * example).  If a_static != NULL it also receives the closed-form per-tensor
+ * activation scale of adr-010 key design point 1:
+ *
+ *   a_static[0] = fl(max_j fl(act_max_j * recip(s_j)) / 127)
+ *
+ * act_max, w_max, s: fp32 [K].  a_static: fp32 [1] or NULL.  0 <= alpha <= 1.
+ * ------------------------------------------------------------------------- */
+sq_status sq_smooth_scales(const float *act_max, const float *w_max, int64_t K, float alpha,
+                           float *s, float *a_static, sq_stream stream);
+
+/* -------------------------------------------------------------------------
+ * (2b) Offline weight transform and per-output-row INT8 quantisation.
+ * kwkr 3.2-3.3 (W' = W diag(s) stored as INT8, one scale per output channel),
+ * adr-010 context steps 2-3 (weights per row):
+ *
+ *   W'[n,j]    = fl(W[n,j] * s_j)
+ *   w_scale[n] = fl(max_j |W'[n,j]| / 127)
+ *   wq[n,j]    = q(fl(W'[n,j] * recip(w_scale[n])))
+ *
+ * w: [N, K] of `dt`, contiguous.  s: fp32 [K].  wq: int8 [N, K] (K-major: the
+ * GEMM's B operand as is).  w_scale: fp32 [N].  An all-zero row gets scale 0
+ * and codes 0.  w and wq 16-byte aligned; K*sizeof(dt) and K multiples of 16
+ * bytes are not required (ragged K is handled).
+ * ------------------------------------------------------------------------- */
+sq_status sq_quant_weight(const void *w, sq_dtype dt, int64_t N, int64_t K, const float *s,
+                          int8_t *wq, float *w_scale, sq_stream stream);
+
+/* The same transform for a gate/up pair that share one s (both read the same
+ * normalised input), written in the interleaved row order that
+ * sq_linear_w8a8_gateup_silu consumes: output rows are blocks of 64, block b
+ * holding gate rows 32b..32b+31 then up rows 32b..32b+31.
+ * w_gate, w_up: [N_h, K] of `dt`.  wq_gu: int8 [2*N_h, K].  w_scale_gu: fp32
+ * [2*N_h], same order.  N_h must be a multiple of 32. */
+sq_status sq_quant_weight_gateup(const void *w_gate, const void *w_up, sq_dtype dt, int64_t N_h,
+                                 int64_t K, const float *s, int8_t *wq_gu, float *w_scale_gu,
+                                 sq_stream stream);
+
+/* -------------------------------------------------------------------------
+ * (3a) Runtime smoothing + INT8 activation quantisation.  The 1/s scaling
+ * happens strictly before quantisation (kwkr 3.2 and 5.2):
+ *
+ *   x'[m,j] = fl(x[m,j] * recip(s_j))
+ *   static:    a = a_scale[0] (read);                       xq = q(fl(x' * recip(a)))
+ *   per-token: a_scale[m] = fl(max_j |x'[m,j]| / 127) (written); xq = q(fl(x' * recip(a_scale[m])))
+ *
+ * x: [M, K] of `dt`, contiguous, 16-byte aligned.  s: fp32 [K].  a_scale: fp32
+ * [1] (static, input) or [M] (per-token, output).  xq: int8 [M, K] (K-major:
+ * the GEMM's A operand as is), 16-byte aligned.
+ * ------------------------------------------------------------------------- */
+sq_status sq_smooth_quant_act(const void *x, sq_dtype dt, int64_t M, int64_t K, const float *s,
+                              sq_act_mode mode, float *a_scale, int8_t *xq, sq_stream stream);
+
+/* (3b) RMSNorm with 1/s folded into its gain, fused with the static INT8
+ * quantisation (kwkr 2.3 and 3.2: absorb the per-channel scaling into the
+ * preceding norm's gamma so smoothing costs nothing at run time; aiu):
+ *
+ *   r_m  = fl(1 / fl(sqrt(fl(mean + eps))))
+ *   mean = fl32(sum_j x_mj^2 / d), the sum of (exact) squares taken in fp64
+ *   g'_j = fl(gamma_j * recip(s_j))
+ *   xq   = q(fl(fl(fl(x * r_m) * g'_j) * recip(a_scale[0])))
+ *
+ * x: [M, d] of `dt`.  gamma, s: fp32 [d].  a_scale: fp32 [1] (static).
+ * xq: int8 [M, d].  rstd: fp32 [M] receives r_m, or NULL.  The fp64 sum is a
+ * tree sum; its order only matters when the fp64 mean sits within ~1e-15 of
+ * an fp32 rounding boundary. */
+sq_status sq_rmsnorm_quant(const void *x, sq_dtype dt, int64_t M, int64_t d, const float *gamma,
+                           const float *s, float eps, const float *a_scale, int8_t *xq,
+                           float *rstd, sq_stream stream);
+
+/* -------------------------------------------------------------------------
+ * (4) W8A8 GEMM with the dequant epilogue (pwwt 3.1: INT8 matmul with the
+ * scale multiplications merged into it; adr-010 key design points 4-5 name
+ * the real INT8 kernel as the follow-up of its fake-quant layer):
+ *
+ *   acc[m,n] = sum_k xq[m,k] * wq[n,k]           (exact int32; K < 133144)
+ *   y[m,n]   = RN_out(fmaf((float)acc, fl(a_m * w_scale[n]), bias[n]))
+ *
+ * a_m = a_scale[0] (static) or a_scale[m] (per-token).  xq: int8 [M, K],
+ * wq: int8 [N, K], both K-major and 16-byte aligned, K a multiple of 16.
+ * w_scale: fp32 [N].  bias: [N] of out_dt, or NULL.  y: [M, N] of out_dt
+ * (fp32/fp16/bf16), 16-byte aligned, N a multiple of 16.  M >= 1.
+ * Runs on the 5th-generation tensor cores (tcgen05 kind::i8, TMA-fed shared
+ * memory tiles, TMEM int32 accumulators).  Small M (<= 64 by default) takes a
+ * weight-streaming path that may split K across CTAs; it then needs
+ * `workspace` of sq_linear_workspace_size(M, N, K) bytes (16-byte aligned),
+ * which it leaves zeroed for the next call.  The caller zeroes a new
+ * workspace once (e.g. cudaMemsetAsync) before first use.
+ * ------------------------------------------------------------------------- */
+size_t sq_linear_workspace_size(int64_t M, int64_t N, int64_t K);
+
+sq_status sq_linear_w8a8(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, int64_t K,
+                         const float *a_scale, sq_act_mode mode, const float *w_scale,
+                         const void *bias, sq_dtype out_dt, void *y, void *workspace,
+                         size_t workspace_bytes, sq_stream stream);
+
+/* Raw int32 accumulators acc[m,n] = sum_k xq[m,k] * wq[n,k] from the same
+ * tensor-core mainloop (for exact INT32 checks).  acc: int32 [M, N]. */
+sq_status sq_gemm_s32(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, int64_t K,
+                      int32_t *acc, sq_stream stream);
+
+/* Gate/up GEMM with the SiLU*mul epilogue of a decoder MLP block.  wq_gu and
+ * w_scale_gu are in the interleaved order of sq_quant_weight_gateup.  With
+ * g, u the fp32 dequant values (no bias) of the gate and up rows of output
+ * channel c:
+ *
+ *   h[m,c] = RN_bf16(fl(fl(g / fl(1 + expf(-g))) * u))
+ *
+ * h: bf16 [M, N_h] or NULL.  If hq != NULL the epilogue also smooths and
+ * quantises h for the next linear with a static scale:
+ *   hq[m,c] = q(fl(fl(h[m,c] * recip(s2_c)) * recip(a2[0])))
+ * using the bf16-rounded h (so it equals sq_smooth_quant_act on h).
+ * s2: fp32 [N_h], a2: fp32 [1] (required with hq).  N_h a multiple of 128.
+ * expf is CUDA's; h matches a correctly rounded SiLU within 2 bf16 ulp. */
+sq_status sq_linear_w8a8_gateup_silu(const int8_t *xq, const int8_t *wq_gu, int64_t M,
+                                     int64_t N_h, int64_t K, const float *a_scale,
+                                     sq_act_mode mode, const float *w_scale_gu, void *h,
+                                     const float *s2, const float *a2, int8_t *hq,
+                                     sq_stream stream);
+
+/* -------------------------------------------------------------------------
+ * Per-layer alpha search (adr-010 key design point 2: pick, per layer, the
+ * alpha of a small grid with the least output reconstruction error, using the
+ * same quantisation math as the final layer).
+ * ------------------------------------------------------------------------- */
+
+/* Unquantised reference product of fp16 inputs on the tensor cores
+ * (tcgen05 kind::f16, fp32 accumulation): y = RN_f16(sum_k x[m,k] w[n,k]).
+ * x: fp16 [M, K], w: fp16 [N, K], y: fp16 [M, N]; K a multiple of 8, N a
+ * multiple of 16, all 16-byte aligned. */
+sq_status sq_gemm_f16_ref(const void *x, const void *w, int64_t M, int64_t N, int64_t K,
+                          void *y, sq_stream stream);
+
+/* Sum of squared differences of two fp16 tensors, added in fp64 to
+ * *sse (device fp64 [1]; the caller zeroes it).  n elements, 16-byte aligned. */
+sq_status sq_sse_f16(const void *y, const void *y_ref, int64_t n, double *sse, sq_stream stream);
+
+/* Bytes of device workspace sq_alpha_search needs. */
+size_t sq_alpha_search_workspace_size(int64_t M_held, int64_t N, int64_t K, int n_alpha);
+
+/* For each alpha in alphas[0..n_alpha) (host array, ascending): s -> static
+ * scale -> weight quant -> quant of the held batch -> INT8 GEMM -> fp16 y ->
+ * mse = mean((y - y_ref)^2), with y_ref = sq_gemm_f16_ref(x_held, w).  The
+ * chosen alpha is the first whose mse is not beaten by more than 1e-6
+ * relative by a later one (ties go to the smaller alpha).
+ * x_held: fp16 [M_held, K]; w: fp16 [N, K]; act_max, w_max: fp32 [K].
+ * best_alpha: HOST float; mse: HOST double [n_alpha] or NULL.  Synchronises
+ * `stream` (the choice is made on the host).  n_alpha in [1, 16]. */
+sq_status sq_alpha_search(const void *x_held, const void *w, int64_t M_held, int64_t N, int64_t K,
+                          const float *act_max, const float *w_max, const float *alphas,
+                          int n_alpha, void *workspace, size_t workspace_bytes,
+                          float *best_alpha, double *mse, sq_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SQ_H_ */

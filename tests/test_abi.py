@@ -1,0 +1,66 @@
+"""The C ABI library loads and exports every entry point declared in include/sq.h (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "sq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(sq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_five_core_calls():
+    names = _declared()
+    for core in ("sq_calib_absmax", "sq_smooth_scales", "sq_quant_weight", "sq_smooth_quant_act",
+                 "sq_linear_w8a8"):
+        assert core in names
+
+
+def test_library_exports_every_declared_symbol():
+    from w8a8_post_quantization_calib_b200 import LIB_PATH, EXPORTS
+    lib = ctypes.CDLL(LIB_PATH)
+    names = _declared()
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+    assert sorted(EXPORTS) == names          # the binding wraps exactly the declared calls
+
+
+def test_host_only_entry_points_without_gpu():
+    import w8a8_post_quantization_calib_b200 as sq
+    lib = sq.lib()
+    assert lib.sq_status_string(0) == b"SQ_OK"
+    assert lib.sq_status_string(5) == b"SQ_ERR_TIMEOUT"
+    # sizes are pure host arithmetic
+    assert sq.linear_workspace_size(16, 4096, 11008) >= 16 * 4096 * 4
+    assert sq.linear_workspace_size(4096, 4096, 11008) == 0
+    assert sq.alpha_search_workspace_size(512, 13824, 5120, 4) > 13824 * 5120
+
+
+@pytest.mark.parametrize("args", [
+    dict(rows=-1), dict(cols=0), dict(ld=3), dict(dt=7),
+])
+def test_argument_validation_rejects_without_launch(args):
+    """Bad arguments return SQ_ERR_INVALID_ARG before any CUDA call (safe without a GPU)."""
+    import w8a8_post_quantization_calib_b200 as sq
+    lib = sq.lib()
+    kw = dict(x=16, dt=1, rows=4, cols=8, ld=8, absmax=32)
+    kw.update(args)
+    st = lib.sq_calib_absmax(kw["x"], kw["dt"], kw["rows"], kw["cols"], kw["ld"], kw["absmax"], None)
+    assert st == 1
+
+
+def test_gemm_validation():
+    import w8a8_post_quantization_calib_b200 as sq
+    lib = sq.lib()
+    # N not a multiple of 16, K not a multiple of 16, null pointers, misaligned operands
+    assert lib.sq_linear_w8a8(16, 16, 4, 24, 64, 16, 0, 16, None, 1, 16, None, 0, None) == 1
+    assert lib.sq_linear_w8a8(16, 16, 4, 32, 40, 16, 0, 16, None, 1, 16, None, 0, None) == 1
+    assert lib.sq_linear_w8a8(None, 16, 4, 32, 64, 16, 0, 16, None, 1, 16, None, 0, None) == 1
+    assert lib.sq_linear_w8a8(17, 16, 4, 32, 64, 16, 0, 16, None, 1, 16, None, 0, None) == 3
+    assert lib.sq_smooth_scales(16, 16, 8, 1.5, 16, None, None) == 1
+    assert lib.sq_smooth_scales(16, 16, 8, -0.1, 16, None, None) == 1

@@ -1,0 +1,325 @@
+"""Kernel-by-kernel parity of the CUDA path (through the C ABI) against the CPU oracle.
+
+Both sides get the same seeded inputs; where a step consumes scales, the
+oracle's scales are uploaded to the GPU, so codes and accumulators are
+compared bit for bit ("given identical fp32 scales, INT8 tensors and INT32
+accumulators are bit-exact").  Shapes span several tiles and ragged tails.
+"""
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from helpers import BF16, F16, F32, bits_equal, dev, host, mismatch_report, rand_x, rel_err
+
+pytestmark = pytest.mark.gpu
+
+sq = pytest.importorskip("w8a8_post_quantization_calib_b200")
+
+
+def _sync():
+    assert sq.sync_status() == 0
+
+
+@functools.lru_cache(maxsize=16)
+def _int8_operands(M, N, K, seed):
+    g = np.random.default_rng(seed)
+    A = g.integers(-127, 128, (M, K), dtype=np.int8)
+    B = g.integers(-127, 128, (N, K), dtype=np.int8)
+    return A, B, oracle.gemm_s32(A, B)
+
+
+# ------------------------------------------------------------------ a1/a2
+@pytest.mark.parametrize("dt", [F32, F16, BF16])
+@pytest.mark.parametrize("rows,cols", [(1, 64), (37, 200), (1000, 4096), (3, 11008), (2049, 520)])
+def test_calib_absmax(dt, rows, cols):
+    b1 = rand_x(rows * 7 + cols, (rows, cols), dt, 3.0, outliers=min(5, cols // 8))
+    b2 = rand_x(rows * 7 + cols + 1, (max(1, rows // 2), cols), dt, 3.0)
+    am = torch.zeros(cols, dtype=torch.float32, device="cuda")
+    sq.calib_absmax(dev(b1, dt), am)
+    sq.calib_absmax(dev(b2, dt), am)
+    _sync()
+    ref = np.zeros(cols, np.float32)
+    oracle.calib_absmax(b1, dt, ref)
+    oracle.calib_absmax(b2, dt, ref)
+    got = host(am)
+    assert bits_equal(got, ref), mismatch_report(got, ref)
+
+
+def test_calib_absmax_strided_rows():
+    x = rand_x(5, (64, 96), F16, 2.0)            # view of the first 80 columns, ld = 96
+    am = torch.zeros(80, dtype=torch.float32, device="cuda")
+    t = dev(x, F16)
+    sq.calib_absmax(t[:, :80], am)
+    _sync()
+    ref = np.abs(oracle.to_f32(x, F16)[:, :80]).max(axis=0)
+    assert bits_equal(host(am), ref)
+
+
+def test_calib_absmax_empty_is_noop():
+    am = torch.full((16,), 3.0, dtype=torch.float32, device="cuda")
+    x = torch.zeros(0, 16, dtype=torch.float16, device="cuda")
+    sq.lib().sq_calib_absmax(x.data_ptr() or 16, 1, 0, 16, 16, am.data_ptr(), None)
+    _sync()
+    assert torch.all(am == 3.0)
+
+
+# ------------------------------------------------------------------ a3
+@pytest.mark.parametrize("alpha", [0.0, 0.25, 0.5, 0.75, 1.0, 0.6])
+@pytest.mark.parametrize("K", [1, 1000, 28672])
+def test_smooth_scales(alpha, K):
+    g = np.random.default_rng(K)
+    a = (np.abs(g.standard_normal(K)) * 5).astype(np.float32)
+    w = (np.abs(g.standard_normal(K)) * 0.05).astype(np.float32)
+    a[::97] = 0.0
+    w[::89] = 0.0
+    a[::13] *= 80
+    s = torch.empty(K, dtype=torch.float32, device="cuda")
+    at = torch.empty(1, dtype=torch.float32, device="cuda")
+    sq.smooth_scales(dev(a), dev(w), alpha, s, at)
+    _sync()
+    s_ref = oracle.smooth_scales(a, w, alpha)
+    a_ref = oracle.static_scale(a, s_ref)
+    got = host(s)
+    assert rel_err(got, s_ref).max() <= 1e-6
+    assert (got != s_ref).mean() < 1e-3            # fp64 pow on both sides: rounding ties only
+    assert rel_err(host(at), [a_ref]).max() <= 1e-6
+
+
+# ------------------------------------------------------------------ a4
+@pytest.mark.parametrize("dt", [F32, F16, BF16])
+@pytest.mark.parametrize("N,K", [(300, 4096), (64, 5120), (3, 40), (17, 28672), (130, 1000)])
+def test_quant_weight(dt, N, K):
+    W = rand_x(N + K, (N, K), dt, 0.02)
+    s = (np.abs(np.random.default_rng(K).standard_normal(K)) + 0.05).astype(np.float32)
+    wq = torch.empty(N, K, dtype=torch.int8, device="cuda")
+    ws = torch.empty(N, dtype=torch.float32, device="cuda")
+    sq.quant_weight(dev(W, dt), dev(s), wq, ws)
+    _sync()
+    wq_ref, ws_ref = oracle.quant_weight(W, s, dt)
+    assert bits_equal(host(ws), ws_ref), mismatch_report(host(ws), ws_ref)
+    assert bits_equal(host(wq), wq_ref), mismatch_report(host(wq), wq_ref)
+
+
+def test_quant_weight_zero_rows():
+    W = np.zeros((40, 64), np.float32)
+    W[7, 3] = 1.5
+    s = np.ones(64, np.float32)
+    wq = torch.empty(40, 64, dtype=torch.int8, device="cuda")
+    ws = torch.empty(40, dtype=torch.float32, device="cuda")
+    sq.quant_weight(dev(W), dev(s), wq, ws)
+    _sync()
+    wq_ref, ws_ref = oracle.quant_weight(W, s, F32)
+    assert bits_equal(host(wq), wq_ref) and bits_equal(host(ws), ws_ref)
+
+
+@pytest.mark.parametrize("dt", [F16, BF16])
+def test_quant_weight_gateup_interleave(dt):
+    Nh, K = 96, 512
+    Wg = rand_x(1, (Nh, K), dt, 0.02)
+    Wu = rand_x(2, (Nh, K), dt, 0.02)
+    s = (np.abs(np.random.default_rng(3).standard_normal(K)) + 0.1).astype(np.float32)
+    wq = torch.empty(2 * Nh, K, dtype=torch.int8, device="cuda")
+    ws = torch.empty(2 * Nh, dtype=torch.float32, device="cuda")
+    sq.quant_weight_gateup(dev(Wg, dt), dev(Wu, dt), dev(s), wq, ws)
+    _sync()
+    # interleaved order: blocks of 64 rows = 32 gate rows then the same 32 up rows
+    order = np.concatenate([np.concatenate([np.arange(b, b + 32), Nh + np.arange(b, b + 32)])
+                            for b in range(0, Nh, 32)])
+    Wcat = np.concatenate([Wg, Wu])[order]
+    wq_ref, ws_ref = oracle.quant_weight(Wcat, s, dt)
+    assert bits_equal(host(wq), wq_ref) and bits_equal(host(ws), ws_ref)
+
+
+# ------------------------------------------------------------------ a5 / a5'
+@pytest.mark.parametrize("dt", [F32, F16, BF16])
+@pytest.mark.parametrize("M,K", [(1, 4096), (300, 4096), (7, 11008), (5, 1024), (3, 40), (129, 5120)])
+@pytest.mark.parametrize("mode", [oracle.STATIC, oracle.PER_TOKEN])
+def test_smooth_quant_act(dt, M, K, mode):
+    X = rand_x(M * 3 + K, (M, K), dt, 2.0, outliers=min(8, K // 10))
+    s = (np.abs(np.random.default_rng(K + 1).standard_normal(K)) + 0.2).astype(np.float32)
+    xq = torch.empty(M, K, dtype=torch.int8, device="cuda")
+    if mode == oracle.STATIC:
+        a = np.float32(30.0 / 127)                 # saturates the outlier columns on purpose
+        at = dev(np.array([a], np.float32))
+        sq.smooth_quant_act(dev(X, dt), dev(s), mode, at, xq)
+        _sync()
+        xq_ref, _ = oracle.smooth_quant_act(X, s, oracle.STATIC, a, dt)
+    else:
+        at = torch.empty(M, dtype=torch.float32, device="cuda")
+        sq.smooth_quant_act(dev(X, dt), dev(s), mode, at, xq)
+        _sync()
+        xq_ref, a_ref = oracle.smooth_quant_act(X, s, oracle.PER_TOKEN, None, dt)
+        assert bits_equal(host(at), a_ref), mismatch_report(host(at), a_ref)
+    assert bits_equal(host(xq), xq_ref), mismatch_report(host(xq), xq_ref)
+
+
+# ------------------------------------------------------------------ a8
+@pytest.mark.parametrize("M,d", [(300, 8192), (5, 1000), (1, 4096)])
+@pytest.mark.parametrize("random_gamma", [False, True])
+def test_rmsnorm_quant(M, d, random_gamma):
+    X = rand_x(M + d, (M, d), BF16, 1.0, outliers=max(1, d // 200))
+    g = np.random.default_rng(d)
+    gamma = g.uniform(0.5, 1.5, d).astype(np.float32) if random_gamma else np.ones(d, np.float32)
+    s = (np.abs(g.standard_normal(d)) + 0.3).astype(np.float32)
+    a = np.float32(0.05)
+    xq = torch.empty(M, d, dtype=torch.int8, device="cuda")
+    r = torch.empty(M, dtype=torch.float32, device="cuda")
+    sq.rmsnorm_quant(dev(X, BF16), dev(gamma), dev(s), 1e-5, dev(np.array([a])), xq, r)
+    _sync()
+    xq_ref, r_ref = oracle.rmsnorm_quant(X, gamma, s, 1e-5, a, BF16)
+    assert bits_equal(host(r), r_ref), mismatch_report(host(r), r_ref)
+    assert bits_equal(host(xq), xq_ref), mismatch_report(host(xq), xq_ref)
+
+
+# ------------------------------------------------------------------ a6
+GEMM_SHAPES = [(1, 16, 32), (16, 48, 48), (100, 272, 1040), (128, 528, 4096), (129, 256, 128),
+               (300, 528, 1040), (64, 4096, 11008), (257, 768, 4096)]
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+def test_gemm_s32(M, N, K):
+    g = np.random.default_rng(M * 131 + N * 7 + K)
+    A = g.integers(-127, 128, (M, K), dtype=np.int8)
+    B = g.integers(-127, 128, (N, K), dtype=np.int8)
+    acc = torch.empty(M, N, dtype=torch.int32, device="cuda")
+    sq.gemm_s32(dev(A), dev(B), acc)
+    _sync()
+    ref = oracle.gemm_s32(A, B)
+    got = host(acc)
+    assert np.array_equal(got, ref), mismatch_report(got, ref)
+
+
+def test_gemm_s32_extremes():
+    K = 8192
+    A = np.full((130, K), -127, np.int8)
+    B = np.full((32, K), 127, np.int8)
+    B[1::2] = -127
+    acc = torch.empty(130, 32, dtype=torch.int32, device="cuda")
+    sq.gemm_s32(dev(A), dev(B), acc)
+    _sync()
+    assert np.array_equal(host(acc), oracle.gemm_s32(A, B))
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 16, 32), (5, 272, 1040), (16, 4096, 11008), (64, 528, 4096),
+                                   (128, 256, 256), (200, 528, 1040), (300, 4096, 512)])
+@pytest.mark.parametrize("out_dt", [F32, F16, BF16])
+@pytest.mark.parametrize("mode", [oracle.STATIC, oracle.PER_TOKEN])
+@pytest.mark.parametrize("with_bias", [False, True])
+@pytest.mark.parametrize("with_ws", [False, True])
+def test_linear_w8a8(M, N, K, out_dt, mode, with_bias, with_ws):
+    if with_ws and M > 128:
+        pytest.skip("workspace only used by the small-M path")
+    A, B, acc_ref = _int8_operands(M, N, K, M * 7 + N * 3 + K)
+    g = np.random.default_rng(M + N + K + out_dt)
+    a = (np.abs(g.standard_normal(1 if mode == oracle.STATIC else M)) * 1e-2 + 1e-3).astype(np.float32)
+    ws = (np.abs(g.standard_normal(N)) * 1e-4 + 1e-5).astype(np.float32)
+    bias = synth.cast(g.standard_normal(N).astype(np.float32), out_dt) if with_bias else None
+    y = torch.empty(M, N, dtype={F32: torch.float32, F16: torch.float16, BF16: torch.bfloat16}[out_dt],
+                    device="cuda")
+    work = None
+    if with_ws:
+        n = sq.linear_workspace_size(M, N, K)
+        work = torch.zeros(n, dtype=torch.uint8, device="cuda")
+    for _ in range(2):      # twice: the split-K workspace must come back zeroed
+        sq.linear_w8a8(dev(A), dev(B), dev(a), mode, dev(ws), y,
+                       bias=dev(bias, out_dt) if with_bias else None, workspace=work)
+    _sync()
+    ref = oracle.dequant(acc_ref, a, mode, ws, out_dt, bias)
+    got = host(y)
+    assert bits_equal(got, ref), mismatch_report(got, ref)
+    if work is not None:
+        assert int(work.count_nonzero()) == 0
+
+
+# ------------------------------------------------------------------ a9
+@pytest.mark.parametrize("M,Nh,K", [(300, 256, 512), (129, 384, 1040)])
+def test_gateup_silu(M, Nh, K):
+    g = np.random.default_rng(M + Nh)
+    A = g.integers(-127, 128, (M, K), dtype=np.int8)
+    Bg = g.integers(-127, 128, (Nh, K), dtype=np.int8)
+    Bu = g.integers(-127, 128, (Nh, K), dtype=np.int8)
+    a = np.array([2e-3], np.float32)
+    wsg = (np.abs(g.standard_normal(Nh)) * 1e-3 + 1e-4).astype(np.float32)
+    wsu = (np.abs(g.standard_normal(Nh)) * 1e-3 + 1e-4).astype(np.float32)
+    order = np.concatenate([np.concatenate([np.arange(b, b + 32), Nh + np.arange(b, b + 32)])
+                            for b in range(0, Nh, 32)])
+    Bgu = np.concatenate([Bg, Bu])[order]
+    wsgu = np.concatenate([wsg, wsu])[order]
+    s2 = (np.abs(g.standard_normal(Nh)) + 0.5).astype(np.float32)
+    a2 = np.array([0.02], np.float32)
+    h = torch.empty(M, Nh, dtype=torch.bfloat16, device="cuda")
+    hq = torch.empty(M, Nh, dtype=torch.int8, device="cuda")
+    sq.linear_w8a8_gateup_silu(dev(A), dev(Bgu), dev(a), oracle.STATIC, dev(wsgu), h=h, s2=dev(s2),
+                               a2=dev(a2), hq=hq)
+    _sync()
+    gv = oracle.dequant_f32(oracle.gemm_s32(A, Bg), a, oracle.STATIC, wsg)
+    uv = oracle.dequant_f32(oracle.gemm_s32(A, Bu), a, oracle.STATIC, wsu)
+    h_ref = oracle.silu_mul_bf16(gv, uv)
+    h_got = host(h)
+    hf_got = oracle.to_f32(h_got, BF16).astype(np.float64)
+    hf_ref = oracle.to_f32(h_ref, BF16).astype(np.float64)
+    ulp = np.maximum(np.abs(hf_ref), 1e-30) * 2.0 ** -7
+    assert np.all(np.abs(hf_got - hf_ref) <= 2 * ulp + 1e-30)
+    assert (h_got != h_ref).mean() < 0.01
+    # requantised h: exactly the oracle's codes wherever h agrees bitwise
+    hq_ref, _ = oracle.smooth_quant_act(h_ref, s2, oracle.STATIC, a2[0], BF16)
+    hq_got = host(hq)
+    same = h_got == h_ref
+    assert np.array_equal(hq_got[same], hq_ref[same])
+    assert np.all(np.abs(hq_got.astype(int) - hq_ref.astype(int)) <= 1)
+    # the h-only and hq-only forms agree with the combined one
+    h2 = torch.empty_like(h)
+    sq.linear_w8a8_gateup_silu(dev(A), dev(Bgu), dev(a), oracle.STATIC, dev(wsgu), h=h2)
+    hq2 = torch.empty_like(hq)
+    sq.linear_w8a8_gateup_silu(dev(A), dev(Bgu), dev(a), oracle.STATIC, dev(wsgu), s2=dev(s2), a2=dev(a2), hq=hq2)
+    _sync()
+    assert torch.equal(h2.view(torch.int16), h.view(torch.int16)) and torch.equal(hq2, hq)
+
+
+# ------------------------------------------------------------------ a7
+@pytest.mark.parametrize("M,N,K", [(200, 272, 520), (64, 512, 1024)])
+def test_gemm_f16_ref(M, N, K):
+    X = rand_x(M, (M, K), F16, 1.0)
+    W = rand_x(N, (N, K), F16, 0.05)
+    y = torch.empty(M, N, dtype=torch.float16, device="cuda")
+    sq.gemm_f16_ref(dev(X, F16), dev(W, F16), y)
+    _sync()
+    ref = oracle.gemm_f16_ref(X, W)
+    got = oracle.to_f32(host(y), F16).astype(np.float64)
+    want = oracle.to_f32(ref, F16).astype(np.float64)
+    # fp32 accumulation (order differs from the fp64 sum) + one fp16 rounding
+    mag = np.abs(oracle.to_f32(X, F16).astype(np.float64)) @ np.abs(oracle.to_f32(W, F16).astype(np.float64)).T
+    tol = np.abs(want) * 2.0 ** -10 + mag * K * 2.0 ** -24 + 2.0 ** -24
+    assert np.all(np.abs(got - want) <= tol)
+
+
+def test_sse_f16():
+    g = np.random.default_rng(0)
+    y = g.standard_normal(100003).astype(np.float16)
+    r = g.standard_normal(100003).astype(np.float16)
+    sse = torch.zeros(1, dtype=torch.float64, device="cuda")
+    yt = torch.from_numpy(y).cuda()
+    rt = torch.from_numpy(r).cuda()
+    sq.sse_f16(yt, rt, sse)
+    _sync()
+    ref = oracle.mse_f16(y.view(np.uint16), r.view(np.uint16)) * y.size
+    assert abs(float(sse.item()) - ref) <= 1e-9 * ref
+
+
+def test_alpha_search_small():
+    wl = synth.heavy_13b(M=64, K=512, N=272, calib_batches=4, calib_rows=128)
+    am = np.zeros(wl.K, np.float32)
+    for b in wl.calib:
+        oracle.calib_absmax(b, F16, am)
+    wm = oracle.calib_absmax(wl.w, F16)
+    best_ref, mse_ref, _ = oracle.alpha_search(wl.calib[0], wl.w, am, wm)
+    held = wl.calib[0]
+    work = torch.zeros(sq.alpha_search_workspace_size(held.shape[0], wl.N, wl.K, 4), dtype=torch.uint8,
+                       device="cuda")
+    best, mses = sq.alpha_search(dev(held, F16), dev(wl.w, F16), dev(am), dev(wm), work)
+    assert best == best_ref
+    assert rel_err(mses, mse_ref).max() < 1e-2

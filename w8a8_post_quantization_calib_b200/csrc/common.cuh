@@ -1,0 +1,140 @@
+// common.cuh -- shared device helpers of libsq (dtype widening, the canonical
+// fp32 quantisation steps, block reductions, the device error word).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace sq {
+
+enum DType : int { DT_F32 = 0, DT_F16 = 1, DT_BF16 = 2 };
+
+__host__ __device__ constexpr int dtype_size(int dt) { return dt == DT_F32 ? 4 : 2; }
+
+// First barrier-timeout code recorded by any kernel of this library on this
+// device (0 = none).  Read and cleared by sq_sync_status.
+__device__ unsigned int g_error_word;
+
+__device__ __forceinline__ void record_error(unsigned code) { atomicCAS(&g_error_word, 0u, code); }
+
+// ---------------------------------------------------------------------------
+// Canonical fp32 steps (round-to-nearest intrinsics so that nvcc never fuses
+// a product into a multiply-add).  Symmetric INT8 quantisation, zero point 0:
+// kwkr.cn blog 1.2 (x_q = round(x / s)) and 3.3; "010. SmoothQuant
+// Integration" key design point 6 (symmetric only).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float recip_or_zero(float v) { return v > 0.0f ? __frcp_rn(v) : 0.0f; }
+
+__device__ __forceinline__ float scale_from_absmax(float m) { return __fdiv_rn(m, 127.0f); }
+
+// round half to even, saturate to [-127, 127]
+__device__ __forceinline__ int quant8(float v)
+{
+    int r = __float2int_rn(v);
+    return min(max(r, -127), 127);
+}
+
+__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d)
+{
+    return (uint32_t)(a & 0xff) | ((uint32_t)(b & 0xff) << 8) | ((uint32_t)(c & 0xff) << 16) |
+           ((uint32_t)(d & 0xff) << 24);
+}
+
+// ---------------------------------------------------------------------------
+// 16-byte vectors: EPV elements of dtype DT, widened exactly to fp32.
+// ---------------------------------------------------------------------------
+template <int DT> struct VecT { static constexpr int EPV = 16 / dtype_size(DT); };
+
+template <int DT>
+__device__ __forceinline__ void widen(const uint4 &v, float (&f)[VecT<DT>::EPV])
+{
+    if constexpr (DT == DT_F32) {
+        f[0] = __uint_as_float(v.x); f[1] = __uint_as_float(v.y);
+        f[2] = __uint_as_float(v.z); f[3] = __uint_as_float(v.w);
+    } else {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            if constexpr (DT == DT_F16) {
+                __half2 h = *reinterpret_cast<const __half2 *>(&w[i]);
+                float2 t = __half22float2(h);
+                f[2 * i] = t.x; f[2 * i + 1] = t.y;
+            } else {
+                f[2 * i] = __uint_as_float(w[i] << 16);
+                f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+            }
+        }
+    }
+}
+
+template <int DT> __device__ __forceinline__ float load_elem(const void *p, int64_t i)
+{
+    if constexpr (DT == DT_F32) return static_cast<const float *>(p)[i];
+    else if constexpr (DT == DT_F16) return __half2float(static_cast<const __half *>(p)[i]);
+    else return __bfloat162float(static_cast<const __nv_bfloat16 *>(p)[i]);
+}
+
+__device__ __forceinline__ float load_elem_dt(const void *p, int dt, int64_t i)
+{
+    if (dt == DT_F32) return load_elem<DT_F32>(p, i);
+    if (dt == DT_F16) return load_elem<DT_F16>(p, i);
+    return load_elem<DT_BF16>(p, i);
+}
+
+// ---------------------------------------------------------------------------
+// Block reductions (blockDim.x a multiple of 32, <= 1024).  `red` holds 32 floats.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float warp_max(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ float block_max(float v, float *red)
+{
+    v = warp_max(v);
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31, nw = blockDim.x >> 5;
+    __syncthreads();                       // protect `red` from the previous use
+    if (l == 0) red[w] = v;
+    __syncthreads();
+    float r = (l < nw) ? red[l] : 0.0f;
+    return warp_max(r);
+}
+
+__device__ __forceinline__ float block_sum(float v, float *red)
+{
+    v = warp_sum(v);
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31, nw = blockDim.x >> 5;
+    __syncthreads();
+    if (l == 0) red[w] = v;
+    __syncthreads();
+    float r = (l < nw) ? red[l] : 0.0f;
+    return warp_sum(r);
+}
+
+__device__ __forceinline__ double block_sum_f64(double v, double *red)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31, nw = blockDim.x >> 5;
+    __syncthreads();
+    if (l == 0) red[w] = v;
+    __syncthreads();
+    double r = (l < nw) ? red[l] : 0.0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
+    return r;
+}
+
+}  // namespace sq

@@ -1,0 +1,501 @@
+// gemm.cuh -- tcgen05 tensor-core GEMM for sm_100a with fused epilogues.
+//
+//   acc[i, j] = sum_k A[i, k] * B[j, k]      (A, B K-major in global memory)
+//
+// kind::i8 (s8 x s8 -> s32) for the W8A8 linear, kind::f16 (f16 x f16 -> f32)
+// for the unquantised reference product of the alpha search.
+//
+// One persistent CTA per SM (192 threads):
+//   warp 0      TMA producer: 128 x 128-byte A tile + BN x 128-byte B tile per
+//               stage, 128-byte swizzle, into a STAGES-deep shared-memory ring
+//   warp 1      MMA issuer: four 128 x BN x 32-byte tcgen05.mma per stage into
+//               a TMEM accumulator; tcgen05.commit frees the stage / hands a
+//               finished accumulator to the epilogue
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
+//               32*(w%4)..+31), dequant / SiLU*mul / requant, global stores
+// TMEM holds two accumulators (2 x BN columns) so the epilogue of tile i
+// overlaps the mainloop of tile i+1.
+//
+// Orientation.  Normal: A = activations xq [M, K], B = weights wq [N, K]; a
+// TMEM lane is a token row, a column an output channel.  Swap (small M): A =
+// weights, B = activations (BN = 16..128 tokens), so the 128-row MMA is filled
+// with weight rows and the kernel streams the weight matrix; a TMEM lane is an
+// output channel, a column a token.  The swap path may split K across CTAs:
+// partial int32 sums are added (exact, order-free) into a workspace, and the
+// last CTA of a tile (a per-tile arrival counter) applies the epilogue and
+// re-zeroes the workspace.
+//
+// Every mbarrier wait is bounded (ptx::wait_bounded): on expiry the kernel
+// records an error code, stops issuing, waits (bounded) for its own TMA loads
+// and MMAs in flight, frees its TMEM and returns.
+#pragma once
+
+#include "common.cuh"
+#include "ptx_sm100.cuh"
+
+namespace sq {
+namespace gemm {
+
+enum Kind : int { KIND_I8 = 0, KIND_F16 = 1 };
+enum Epi : int { EPI_DEQUANT = 0, EPI_S32 = 1, EPI_GATEUP = 2, EPI_F16 = 3 };
+
+constexpr int BM = 128;            // MMA M: rows of the A operand per tile
+constexpr int BKB = 128;           // bytes of K per stage (one swizzle row)
+constexpr int NUM_THREADS = 192;
+constexpr int GROUP_R = 16;        // raster group along A-row tiles (L2 reuse of B)
+constexpr int SMEM_BUDGET = 200 * 1024;
+
+// error codes recorded on a barrier timeout: 0x100 | role << 4 | where
+constexpr unsigned ERR_PRODUCER = 0x110, ERR_MMA = 0x120, ERR_EPI = 0x130, ERR_DRAIN = 0x140;
+
+__host__ __device__ constexpr int pow2_at_least(int v, int lo)
+{
+    int r = lo;
+    while (r < v) r <<= 1;
+    return r;
+}
+
+template <int BN>
+struct TileCfg {
+    static constexpr int A_BYTES = BM * BKB;
+    static constexpr int B_BYTES = BN * BKB;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int STAGES_RAW = SMEM_BUDGET / STAGE_BYTES;
+    static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
+    static constexpr int TMEM_COLS = pow2_at_least(2 * BN, 32);
+    static constexpr int CW = BN < 32 ? BN : 32;   // TMEM columns per epilogue load
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+    static_assert(STAGE_BYTES % 1024 == 0, "stage must keep 1024-byte alignment");
+    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
+};
+
+struct Params {
+    int M, N, K;               // logical problem: out[M, N] from x[M, K], w[N, K]
+    int rows_a, rows_b;        // rows of the A / B operand tensors
+    int num_kb;                // K blocks of 128 bytes
+    int tiles_r, tiles_c;      // tiles along A rows (BM) and B rows (BN)
+    int splits, kb_per_split;  // split-K (swap path only)
+    int num_units;             // tiles_r * tiles_c * splits
+    const float *a_scale;      // [1] or [M]
+    int per_token;
+    const float *w_scale;      // [N]
+    const void *bias;          // [N] of out_dt or null
+    void *out;                 // [M, N] (gate/up: h [M, N/2] or null)
+    int out_dt;
+    int32_t *ws_acc;           // split-K partial sums [M, N]
+    int *ws_cnt;               // split-K arrival counters [tiles]
+    const float *s2;           // gate/up: smoothing of h [N/2]
+    const float *a2;           // gate/up: static scale of h [1]
+    int8_t *hq;                // gate/up: codes of h [M, N/2] or null
+    unsigned long long timeout_ns;
+};
+
+__device__ __forceinline__ void decode_unit(const Params &p, int u, int &tr, int &tc, int &split, int &tile)
+{
+    split = u % p.splits;
+    tile = u / p.splits;
+    const int group = tile / (GROUP_R * p.tiles_c);
+    const int first = group * GROUP_R;
+    const int gsz = min(GROUP_R, p.tiles_r - first);
+    const int r = tile - group * GROUP_R * p.tiles_c;
+    tr = first + r % gsz;
+    tc = r / gsz;
+}
+
+__device__ __forceinline__ void tmem_load_chunk(uint32_t taddr, uint32_t (&r)[32], int cw)
+{
+    if (cw == 32) {
+        ptx::tmem_ld32(taddr, r);
+    } else {
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+            "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+              "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+              "=r"(r[14]), "=r"(r[15])
+            : "r"(taddr)
+            : "memory");
+    }
+}
+
+__device__ __forceinline__ void store_out(void *out, int out_dt, int64_t idx, float v)
+{
+    if (out_dt == DT_F32) static_cast<float *>(out)[idx] = v;
+    else if (out_dt == DT_F16) static_cast<__half *>(out)[idx] = __float2half_rn(v);
+    else static_cast<__nv_bfloat16 *>(out)[idx] = __float2bfloat16_rn(v);
+}
+
+// 8 fp32 values -> 16 bytes of out_dt at out + idx (idx a multiple of 8 / 4)
+__device__ __forceinline__ void store_out8(void *out, int out_dt, int64_t idx, const float *v)
+{
+    if (out_dt == DT_F32) {
+        float4 *o = reinterpret_cast<float4 *>(static_cast<float *>(out) + idx);
+        o[0] = make_float4(v[0], v[1], v[2], v[3]);
+        o[1] = make_float4(v[4], v[5], v[6], v[7]);
+    } else if (out_dt == DT_F16) {
+        uint4 w;
+        __half2 h0 = __floats2half2_rn(v[0], v[1]), h1 = __floats2half2_rn(v[2], v[3]);
+        __half2 h2 = __floats2half2_rn(v[4], v[5]), h3 = __floats2half2_rn(v[6], v[7]);
+        w.x = *reinterpret_cast<uint32_t *>(&h0); w.y = *reinterpret_cast<uint32_t *>(&h1);
+        w.z = *reinterpret_cast<uint32_t *>(&h2); w.w = *reinterpret_cast<uint32_t *>(&h3);
+        *reinterpret_cast<uint4 *>(static_cast<__half *>(out) + idx) = w;
+    } else {
+        uint4 w;
+        __nv_bfloat162 h0 = __floats2bfloat162_rn(v[0], v[1]), h1 = __floats2bfloat162_rn(v[2], v[3]);
+        __nv_bfloat162 h2 = __floats2bfloat162_rn(v[4], v[5]), h3 = __floats2bfloat162_rn(v[6], v[7]);
+        w.x = *reinterpret_cast<uint32_t *>(&h0); w.y = *reinterpret_cast<uint32_t *>(&h1);
+        w.z = *reinterpret_cast<uint32_t *>(&h2); w.w = *reinterpret_cast<uint32_t *>(&h3);
+        *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(out) + idx) = w;
+    }
+}
+
+__device__ __forceinline__ float load_bias(const void *bias, int out_dt, int64_t n)
+{
+    return bias == nullptr ? 0.0f : load_elem_dt(bias, out_dt, n);
+}
+
+// Dequant: fmaf((float)acc, fl(a*w), bias) (plain product without bias).
+__device__ __forceinline__ float dequant(int32_t acc, float c, const void *bias, float b)
+{
+    const float af = __int2float_rn(acc);
+    return bias != nullptr ? __fmaf_rn(af, c, b) : __fmul_rn(af, c);
+}
+
+// ---------------------------------------------------------------------------
+// Epilogue of one tile, normal orientation (TMEM lane = token row m).
+// ---------------------------------------------------------------------------
+template <int BN, int KIND, int EPI>
+__device__ __forceinline__ void epilogue_normal(const Params &p, uint32_t tbase, int tr, int tc, int q,
+                                                int lane)
+{
+    const int m = tr * BM + q * 32 + lane;
+    const bool mok = m < p.M;
+    float am = 0.0f;
+    if constexpr (EPI == EPI_DEQUANT || EPI == EPI_GATEUP)
+        if (mok) am = p.per_token ? p.a_scale[m] : p.a_scale[0];
+
+    if constexpr (EPI == EPI_GATEUP) {
+        // columns: 32 gate channels, then the same 32 channels' up rows, repeated
+        const int Nh = p.N >> 1;
+        const float inv_a2 = p.hq != nullptr ? recip_or_zero(p.a2[0]) : 0.0f;
+#pragma unroll 1
+        for (int c = 0; c < BN / 64; ++c) {
+            uint32_t rg[32], ru[32];
+            ptx::tmem_ld32(tbase + c * 64, rg);
+            ptx::tmem_ld32(tbase + c * 64 + 32, ru);
+            ptx::tmem_ld_wait();
+            const int row0 = tc * BN + c * 64;         // first gate row of this pair of chunks
+            if (row0 >= p.N) continue;
+            const int ch0 = row0 >> 1;
+            float h[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const float g = __fmul_rn(__int2float_rn(static_cast<int32_t>(rg[i])), __fmul_rn(am, p.w_scale[row0 + i]));
+                const float u = __fmul_rn(__int2float_rn(static_cast<int32_t>(ru[i])), __fmul_rn(am, p.w_scale[row0 + 32 + i]));
+                const float sg = __fdiv_rn(g, __fadd_rn(1.0f, expf(-g)));
+                h[i] = __bfloat162float(__float2bfloat16_rn(__fmul_rn(sg, u)));   // h as bf16
+            }
+            if (!mok) continue;
+            const int64_t o = static_cast<int64_t>(m) * Nh + ch0;
+            if (p.out != nullptr) {
+#pragma unroll
+                for (int i = 0; i < 32; i += 8) store_out8(p.out, DT_BF16, o + i, h + i);
+            }
+            if (p.hq != nullptr) {
+                uint32_t w[8];
+#pragma unroll
+                for (int i = 0; i < 32; i += 4) {
+                    int qv[4];
+#pragma unroll
+                    for (int t = 0; t < 4; ++t)
+                        qv[t] = quant8(__fmul_rn(__fmul_rn(h[i + t], recip_or_zero(p.s2[ch0 + i + t])), inv_a2));
+                    w[i / 4] = pack4(qv[0], qv[1], qv[2], qv[3]);
+                }
+                uint4 *dst = reinterpret_cast<uint4 *>(p.hq + o);
+                dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            }
+        }
+        return;
+    }
+
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        ptx::tmem_ld32(tbase + c * 32, r);
+        ptx::tmem_ld_wait();
+        const int n0 = tc * BN + c * 32;
+        if (n0 >= p.N || !mok) continue;
+        const int nval = min(32, p.N - n0);        // 16 or 32 (N is a multiple of 16)
+        const int64_t o = static_cast<int64_t>(m) * p.N + n0;
+        if constexpr (EPI == EPI_S32) {
+            int4 *dst = reinterpret_cast<int4 *>(static_cast<int32_t *>(p.out) + o);
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+                if (i < nval) dst[i / 4] = make_int4(r[i], r[i + 1], r[i + 2], r[i + 3]);
+        } else if constexpr (EPI == EPI_F16) {
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+#pragma unroll
+            for (int i = 0; i < 32; i += 8)
+                if (i < nval) store_out8(p.out, DT_F16, o + i, v + i);
+        } else {
+            float v[32];
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+                if (i < nval) {
+                    const float4 w4 = *reinterpret_cast<const float4 *>(p.w_scale + n0 + i);
+                    const float ws[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const float cc = __fmul_rn(am, ws[t]);
+                        v[i + t] = dequant(static_cast<int32_t>(r[i + t]), cc, p.bias,
+                                           load_bias(p.bias, p.out_dt, n0 + i + t));
+                    }
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 32; i += 8)
+                if (i < nval) store_out8(p.out, p.out_dt, o + i, v + i);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Epilogue of one unit, swap orientation (TMEM lane = output channel n,
+// column = token).  EPI_DEQUANT or EPI_S32 (no split for S32).
+// ---------------------------------------------------------------------------
+template <int BN, int EPI>
+__device__ __forceinline__ void epilogue_swap(const Params &p, uint32_t tbase, int tr, int tc, int tile,
+                                              int q, int lane, int *last_flag)
+{
+    constexpr int CW = TileCfg<BN>::CW;
+    const int n = tr * BM + q * 32 + lane;
+    const bool nok = n < p.N;
+    const float wsn = nok ? p.w_scale[n] : 0.0f;
+    const float bn = (nok && p.bias != nullptr) ? load_bias(p.bias, p.out_dt, n) : 0.0f;
+    const bool split = p.splits > 1;
+
+#pragma unroll 1
+    for (int c = 0; c < BN / CW; ++c) {
+        uint32_t r[32];
+        tmem_load_chunk(tbase + c * CW, r, CW);
+        ptx::tmem_ld_wait();
+        const int m0 = tc * BN + c * CW;
+        if (!nok) continue;
+#pragma unroll
+        for (int i = 0; i < CW; ++i) {
+            const int m = m0 + i;
+            if (m >= p.M) break;
+            const int64_t o = static_cast<int64_t>(m) * p.N + n;
+            if constexpr (EPI == EPI_S32) {
+                static_cast<int32_t *>(p.out)[o] = static_cast<int32_t>(r[i]);
+            } else if (split) {
+                ptx::red_add_s32(p.ws_acc + o, static_cast<int32_t>(r[i]));
+            } else {
+                const float am = p.per_token ? p.a_scale[m] : p.a_scale[0];
+                store_out(p.out, p.out_dt, o, dequant(static_cast<int32_t>(r[i]), __fmul_rn(am, wsn), p.bias, bn));
+            }
+        }
+    }
+    if constexpr (EPI == EPI_DEQUANT) {
+        if (!split) return;
+        // arrival: the last split of this tile applies the epilogue
+        __threadfence();
+        ptx::named_bar_sync(1, 128);
+        if (q == 2 && lane == 0) {       // first epilogue thread (warp 2)
+            __threadfence();
+            const int prev = atomicAdd(p.ws_cnt + tile, 1);
+            *last_flag = (prev == p.splits - 1) ? 1 : 0;
+        }
+        ptx::named_bar_sync(1, 128);
+        if (*last_flag == 0) return;
+        __threadfence();
+        if (nok) {
+            const int mend = min(p.M, tc * BN + BN);
+            for (int m = tc * BN; m < mend; ++m) {
+                const int64_t o = static_cast<int64_t>(m) * p.N + n;
+                const int32_t acc = __ldcg(p.ws_acc + o);
+                p.ws_acc[o] = 0;
+                const float am = p.per_token ? p.a_scale[m] : p.a_scale[0];
+                store_out(p.out, p.out_dt, o, dequant(acc, __fmul_rn(am, wsn), p.bias, bn));
+            }
+        }
+        ptx::named_bar_sync(1, 128);
+        if (q == 2 && lane == 0) {
+            p.ws_cnt[tile] = 0;
+            *last_flag = 0;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// The kernel
+// ---------------------------------------------------------------------------
+template <int BN, int KIND, int EPI, bool SWAP>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    k_gemm(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b, const Params p)
+{
+    using C = TileCfg<BN>;
+    constexpr int S = C::STAGES;
+    constexpr int BKE = (KIND == KIND_I8) ? BKB : BKB / 2;       // K elements per stage
+    constexpr uint32_t IDESC = (KIND == KIND_I8) ? ptx::idesc_i8(BN) : ptx::idesc_f16(BN);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + S * C::STAGE_BYTES);
+    const uint32_t bar0 = ptx::smem_addr(bars);
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
+    auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * S + b); };
+    auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * S + 2 + b); };
+    const uint32_t done_bar = bar0 + 8u * (2 * S + 4);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 5);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    int *last_flag = reinterpret_cast<int *>(tmem_slot + 2);
+    const uint32_t sbase = ptx::smem_addr(smem);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            ptx::mbar_init(full_bar(s), 1);
+            ptx::mbar_init(empty_bar(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(tfull_bar(b), 1);
+            ptx::mbar_init(tempty_bar(b), 4);
+        }
+        ptx::mbar_init(done_bar, 1);
+        *abort_flag = 0;
+        *last_flag = 0;
+        ptx::fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        ptx::tma_prefetch_desc(&map_a);
+        ptx::tma_prefetch_desc(&map_b);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(ptx::smem_addr(tmem_slot), C::TMEM_COLS);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const uint64_t tmo = p.timeout_ns;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0, issued = 0;
+            uint32_t phase = 0;
+            for (int u = blockIdx.x; u < p.num_units && !*abort_flag; u += gridDim.x) {
+                int tr, tc, split, tile;
+                decode_unit(p, u, tr, tc, split, tile);
+                const int kb0 = split * p.kb_per_split;
+                const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+                bool ok = true;
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!ptx::wait_bounded(empty_bar(stage), phase ^ 1u, tmo, abort_flag, ERR_PRODUCER)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::mbar_arrive_expect_tx(full_bar(stage), C::STAGE_BYTES);
+                    const uint32_t sa = sbase + stage * C::STAGE_BYTES;
+                    ptx::tma_load_2d(sa, &map_a, full_bar(stage), kb * BKE, tr * BM);
+                    ptx::tma_load_2d(sa + C::A_BYTES, &map_b, full_bar(stage), kb * BKE, tc * BN);
+                    ++issued;
+                    if (++stage == S) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+            }
+            // drain: every issued load lands before the CTA exits
+            const int n_wait = issued < S ? issued : S;
+            for (int i = 0; i < n_wait; ++i) {
+                int s = stage - 1 - i;
+                uint32_t ph = phase;
+                if (s < 0) { s += S; ph ^= 1u; }
+                volatile int no_abort = 0;
+                ptx::wait_bounded(full_bar(s), ph, tmo, &no_abort, ERR_DRAIN);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0, local = 0;
+            uint32_t phase = 0;
+            for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++local) {
+                int tr, tc, split, tile;
+                decode_unit(p, u, tr, tc, split, tile);
+                const int kb0 = split * p.kb_per_split;
+                const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+                const int b = local & 1;
+                const uint32_t use = static_cast<uint32_t>(local >> 1) & 1u;
+                if (!ptx::wait_bounded(tempty_bar(b), use ^ 1u, tmo, abort_flag, ERR_MMA)) break;
+                ptx::tc_fence_after();
+                const uint32_t d = tmem_base + static_cast<uint32_t>(b * BN);
+                bool ok = true;
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!ptx::wait_bounded(full_bar(stage), phase, tmo, abort_flag, ERR_MMA + 1)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint32_t sa = sbase + stage * C::STAGE_BYTES;
+                    const uint64_t ad = ptx::sdesc_kmajor_sw128(sa);
+                    const uint64_t bd = ptx::sdesc_kmajor_sw128(sa + C::A_BYTES);
+#pragma unroll
+                    for (int k = 0; k < BKB / 32; ++k) {
+                        const uint32_t acc = (kb > kb0 || k > 0) ? 1u : 0u;
+                        if constexpr (KIND == KIND_I8)
+                            ptx::mma_i8(d, ad + 2 * k, bd + 2 * k, IDESC, acc);
+                        else
+                            ptx::mma_f16(d, ad + 2 * k, bd + 2 * k, IDESC, acc);
+                    }
+                    ptx::tc_commit(empty_bar(stage));
+                    if (++stage == S) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                ptx::tc_commit(tfull_bar(b));
+            }
+            // drain: all issued MMAs complete before TMEM is released
+            ptx::tc_commit(done_bar);
+            volatile int no_abort = 0;
+            ptx::wait_bounded(done_bar, 0u, tmo, &no_abort, ERR_DRAIN + 1);
+        }
+    } else {
+        // ------------------------------------------------ epilogue (warps 2..5)
+        const int q = warp & 3;
+        int local = 0;
+        for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++local) {
+            int tr, tc, split, tile;
+            decode_unit(p, u, tr, tc, split, tile);
+            const int b = local & 1;
+            const uint32_t use = static_cast<uint32_t>(local >> 1) & 1u;
+            int ok = 1;
+            if (lane == 0) ok = ptx::wait_bounded(tfull_bar(b), use, tmo, abort_flag, ERR_EPI) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * BN);
+            if constexpr (SWAP)
+                epilogue_swap<BN, EPI>(p, tbase, tr, tc, tile, q, lane, last_flag);
+            else
+                epilogue_normal<BN, KIND, EPI>(p, tbase, tr, tc, q, lane);
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(tempty_bar(b));
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+}  // namespace gemm
+}  // namespace sq

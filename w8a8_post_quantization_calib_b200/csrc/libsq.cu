@@ -1,0 +1,584 @@
+// libsq.cu -- the C ABI of the SmoothQuant W8A8 linear layer for B200
+// (sm_100a).  One translation unit: the kernels live in the included .cuh
+// files; this file validates arguments, sizes grids for the device, encodes
+// TMA tensor maps and launches.  Declarations and the full contract of every
+// entry point are in include/sq.h.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "sq.h"
+#include "common.cuh"
+#include "ptx_sm100.cuh"
+#include "calib.cuh"
+#include "quant.cuh"
+#include "gemm.cuh"
+
+using namespace sq;
+
+namespace {
+
+thread_local int t_last_cuda_error = 0;
+unsigned long long g_timeout_ns = 2000000000ull;   // bounded barrier waits: 2 s
+
+constexpr int kMaxDevices = 64;
+int g_sm_count[kMaxDevices] = {0};
+std::mutex g_mu;
+
+inline cudaStream_t as_stream(sq_stream s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline bool valid_dt(int dt) { return dt == SQ_F32 || dt == SQ_F16 || dt == SQ_BF16; }
+
+inline sq_status cuda_fail(cudaError_t e)
+{
+    t_last_cuda_error = static_cast<int>(e);
+    return SQ_ERR_CUDA;
+}
+
+inline sq_status check_launch()
+{
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SQ_OK : cuda_fail(e);
+}
+
+int sm_count()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+    if (g_sm_count[dev] == 0) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        g_sm_count[dev] = n > 0 ? n : 148;
+    }
+    return g_sm_count[dev];
+}
+
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// ------------------------------------------------------------------ TMA maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (fn == nullptr) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 2D row-major [rows, inner] tensor of 1- or 2-byte elements; box of
+// box_rows x 128 bytes with the 128-byte swizzle; out-of-range reads are zero.
+bool make_map(CUtensorMap *m, const void *base, bool f16, int64_t inner, int64_t rows, uint32_t box_rows)
+{
+    auto fn = encode_fn();
+    if (fn == nullptr) return false;
+    const int elt = f16 ? 2 : 1;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(inner * elt)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elt), box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                          const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ GEMM launch
+template <int BN, int KIND, int EPI, bool SWAP>
+sq_status launch_gemm(gemm::Params p, const void *a, const void *b, cudaStream_t st)
+{
+    using C = gemm::TileCfg<BN>;
+    const bool f16 = (KIND == gemm::KIND_F16);
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, a, f16, p.K, p.rows_a, gemm::BM)) return SQ_ERR_CUDA;
+    if (!make_map(&mb, b, f16, p.K, p.rows_b, BN)) return SQ_ERR_CUDA;
+    auto kern = gemm::k_gemm<BN, KIND, EPI, SWAP>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return cuda_fail(e);
+    p.timeout_ns = g_timeout_ns;
+    const int grid = static_cast<int>(std::min<int64_t>(p.num_units, sm_count()));
+    kern<<<grid, gemm::NUM_THREADS, C::SMEM_BYTES, st>>>(ma, mb, p);
+    return check_launch();
+}
+
+void fill_tiles(gemm::Params &p, int bn, int64_t rows_a, int64_t rows_b)
+{
+    p.rows_a = static_cast<int>(rows_a);
+    p.rows_b = static_cast<int>(rows_b);
+    p.num_kb = static_cast<int>(cdiv(p.K, 128 / 1));
+    p.tiles_r = static_cast<int>(cdiv(rows_a, gemm::BM));
+    p.tiles_c = static_cast<int>(cdiv(rows_b, bn));
+    p.splits = 1;
+    p.kb_per_split = p.num_kb;
+    p.num_units = p.tiles_r * p.tiles_c;
+}
+
+constexpr int64_t kSwapMaxM = 128;
+
+int swap_bn(int64_t M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128; }
+
+int64_t swap_tiles(int64_t M, int64_t N) { return cdiv(N, gemm::BM) * cdiv(M, swap_bn(M)); }
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+size_t ws_bytes(int64_t M, int64_t N)
+{
+    if (M > kSwapMaxM) return 0;
+    return align_up(static_cast<size_t>(M * N) * 4, 256) + align_up(static_cast<size_t>(swap_tiles(M, N)) * 4, 256);
+}
+
+template <int EPI>
+sq_status dispatch_swap(gemm::Params &p, const int8_t *xq, const int8_t *wq, cudaStream_t st)
+{
+    const int bn = swap_bn(p.M);
+    fill_tiles(p, bn, p.N, p.M);
+    if (EPI == gemm::EPI_DEQUANT && p.ws_acc != nullptr) {
+        const int tiles = p.num_units;
+        const int sms = sm_count();
+        if (tiles < sms) {
+            int splits = std::max(1, sms / tiles);
+            splits = std::min(splits, std::max(1, p.num_kb / 2));
+            p.kb_per_split = static_cast<int>(cdiv(p.num_kb, splits));
+            p.splits = static_cast<int>(cdiv(p.num_kb, p.kb_per_split));
+            p.num_units = tiles * p.splits;
+        }
+    }
+    if (p.splits == 1) {
+        p.ws_acc = nullptr;
+        p.ws_cnt = nullptr;
+    }
+    switch (bn) {
+    case 16: return launch_gemm<16, gemm::KIND_I8, EPI, true>(p, wq, xq, st);
+    case 32: return launch_gemm<32, gemm::KIND_I8, EPI, true>(p, wq, xq, st);
+    case 64: return launch_gemm<64, gemm::KIND_I8, EPI, true>(p, wq, xq, st);
+    default: return launch_gemm<128, gemm::KIND_I8, EPI, true>(p, wq, xq, st);
+    }
+}
+
+// ------------------------------------------------------------------ row kernels
+template <int DT, int MODE>
+sq_status launch_rows_dt(RowArgs a, cudaStream_t st)
+{
+    constexpr int EPV = VecT<DT>::EPV;
+    const bool vec = aligned16(a.src0) && (a.src1 == nullptr || aligned16(a.src1)) && aligned16(a.out) &&
+                     (a.K % EPV) == 0;
+    const int64_t nvec = a.K / EPV;
+    const int64_t vpt = cdiv(nvec, ROW_T);
+    const size_t smem = static_cast<size_t>(a.K) * 4;
+    const int sms = sm_count();
+    if (vec && vpt <= 16 && smem <= 160 * 1024) {
+        void (*kern)(RowArgs) = nullptr;
+        if (vpt <= 1) kern = k_rows<DT, 1, MODE>;
+        else if (vpt <= 2) kern = k_rows<DT, 2, MODE>;
+        else if (vpt <= 4) kern = k_rows<DT, 4, MODE>;
+        else if (vpt <= 8) kern = k_rows<DT, 8, MODE>;
+        else kern = k_rows<DT, 16, MODE>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess) return cuda_fail(e);
+        int per_sm = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, ROW_T, smem);
+        if (e != cudaSuccess) return cuda_fail(e);
+        const int64_t grid = std::min<int64_t>(a.rows, static_cast<int64_t>(sms) * std::max(1, per_sm));
+        kern<<<static_cast<unsigned>(grid), ROW_T, smem, st>>>(a);
+    } else {
+        const int64_t grid = std::min<int64_t>(a.rows, static_cast<int64_t>(sms) * 8);
+        k_rows_scalar<MODE><<<static_cast<unsigned>(grid), ROW_T, 0, st>>>(a, DT);
+    }
+    return check_launch();
+}
+
+template <int MODE>
+sq_status launch_rows(RowArgs a, int dt, cudaStream_t st)
+{
+    if (a.rows == 0) return SQ_OK;
+    if (dt == SQ_F32) return launch_rows_dt<DT_F32, MODE>(a, st);
+    if (dt == SQ_F16) return launch_rows_dt<DT_F16, MODE>(a, st);
+    return launch_rows_dt<DT_BF16, MODE>(a, st);
+}
+
+}  // namespace
+
+// ============================================================================
+// C ABI
+// ============================================================================
+extern "C" {
+
+const char *sq_status_string(sq_status st)
+{
+    switch (st) {
+    case SQ_OK: return "SQ_OK";
+    case SQ_ERR_INVALID_ARG: return "SQ_ERR_INVALID_ARG";
+    case SQ_ERR_UNSUPPORTED: return "SQ_ERR_UNSUPPORTED";
+    case SQ_ERR_MISALIGNED: return "SQ_ERR_MISALIGNED";
+    case SQ_ERR_CUDA: return "SQ_ERR_CUDA";
+    case SQ_ERR_TIMEOUT: return "SQ_ERR_TIMEOUT";
+    case SQ_ERR_WORKSPACE: return "SQ_ERR_WORKSPACE";
+    }
+    return "SQ_ERR_UNKNOWN";
+}
+
+int sq_last_cuda_error(void) { return t_last_cuda_error; }
+
+void sq_set_wait_timeout_ns(unsigned long long ns) { g_timeout_ns = ns > 0 ? ns : 2000000000ull; }
+
+sq_status sq_sync_status(sq_stream stream)
+{
+    cudaError_t e = cudaStreamSynchronize(as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(e);
+    unsigned int word = 0;
+    e = cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word));
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (word != 0) {
+        const unsigned int zero = 0;
+        cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero));
+        return SQ_ERR_TIMEOUT;
+    }
+    return SQ_OK;
+}
+
+sq_status sq_calib_absmax(const void *x, sq_dtype dt, int64_t rows, int64_t cols, int64_t ld, float *absmax,
+                          sq_stream stream)
+{
+    if (x == nullptr || absmax == nullptr || !valid_dt(dt)) return SQ_ERR_INVALID_ARG;
+    if (rows < 0 || cols <= 0 || ld < cols || rows > (int64_t(1) << 40)) return SQ_ERR_INVALID_ARG;
+    if (rows == 0) return SQ_OK;
+    const cudaStream_t st = as_stream(stream);
+    const int elt = dtype_size(dt);
+    const int sms = sm_count();
+    const bool vec = aligned16(x) && (cols * elt) % 16 == 0 && (ld * elt) % 16 == 0;
+    if (vec) {
+        const int64_t nvec = cols * elt / 16;
+        const int64_t gx = cdiv(nvec, CALIB_TX);
+        const int64_t target = static_cast<int64_t>(sms) * 8;
+        int64_t gy = std::max<int64_t>(1, std::min<int64_t>(cdiv(rows, CALIB_TY * CALIB_UNROLL), cdiv(target, gx)));
+        gy = std::min<int64_t>(gy, 65535);
+        const int64_t slab = cdiv(rows, gy);
+        gy = cdiv(rows, slab);
+        dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), block(CALIB_TX, CALIB_TY);
+        const uint8_t *xb = static_cast<const uint8_t *>(x);
+        const int64_t ldb = ld * elt;
+        if (dt == SQ_F32) k_colabsmax<DT_F32><<<grid, block, 0, st>>>(xb, rows, nvec, ldb, slab, absmax);
+        else if (dt == SQ_F16) k_colabsmax<DT_F16><<<grid, block, 0, st>>>(xb, rows, nvec, ldb, slab, absmax);
+        else k_colabsmax<DT_BF16><<<grid, block, 0, st>>>(xb, rows, nvec, ldb, slab, absmax);
+    } else {
+        const int64_t gx = cdiv(cols, 256);
+        int64_t gy = std::max<int64_t>(1, std::min<int64_t>(cdiv(rows, 64), cdiv(static_cast<int64_t>(sms) * 8, gx)));
+        gy = std::min<int64_t>(gy, 65535);
+        const int64_t slab = cdiv(rows, gy);
+        gy = cdiv(rows, slab);
+        k_colabsmax_scalar<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), 256, 0, st>>>(
+            x, dt, rows, cols, ld, slab, absmax);
+    }
+    return check_launch();
+}
+
+sq_status sq_smooth_scales(const float *act_max, const float *w_max, int64_t K, float alpha, float *s,
+                           float *a_static, sq_stream stream)
+{
+    if (act_max == nullptr || w_max == nullptr || s == nullptr || K <= 0) return SQ_ERR_INVALID_ARG;
+    if (!(alpha >= 0.0f && alpha <= 1.0f)) return SQ_ERR_INVALID_ARG;
+    const cudaStream_t st = as_stream(stream);
+    if (a_static != nullptr) {
+        const cudaError_t e = cudaMemsetAsync(a_static, 0, sizeof(float), st);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(cdiv(K, 256), static_cast<int64_t>(sm_count()) * 4));
+    k_smooth_scales<<<static_cast<unsigned>(grid), 256, 0, st>>>(act_max, w_max, K, alpha, s, a_static);
+    return check_launch();
+}
+
+sq_status sq_quant_weight(const void *w, sq_dtype dt, int64_t N, int64_t K, const float *s, int8_t *wq,
+                          float *w_scale, sq_stream stream)
+{
+    if (w == nullptr || s == nullptr || wq == nullptr || w_scale == nullptr || !valid_dt(dt)) return SQ_ERR_INVALID_ARG;
+    if (N < 0 || K <= 0) return SQ_ERR_INVALID_ARG;
+    if (!aligned16(w) || !aligned16(wq)) return SQ_ERR_MISALIGNED;
+    RowArgs a{};
+    a.src0 = static_cast<const uint8_t *>(w);
+    a.rows = N;
+    a.K = K;
+    a.row_bytes = K * dtype_size(dt);
+    a.s = s;
+    a.scale_out = w_scale;
+    a.out = wq;
+    return launch_rows<ROW_WEIGHT>(a, dt, as_stream(stream));
+}
+
+sq_status sq_quant_weight_gateup(const void *w_gate, const void *w_up, sq_dtype dt, int64_t N_h, int64_t K,
+                                 const float *s, int8_t *wq_gu, float *w_scale_gu, sq_stream stream)
+{
+    if (w_gate == nullptr || w_up == nullptr || s == nullptr || wq_gu == nullptr || w_scale_gu == nullptr ||
+        !valid_dt(dt))
+        return SQ_ERR_INVALID_ARG;
+    if (N_h <= 0 || K <= 0 || (N_h % 32) != 0) return SQ_ERR_INVALID_ARG;
+    if (!aligned16(w_gate) || !aligned16(w_up) || !aligned16(wq_gu)) return SQ_ERR_MISALIGNED;
+    RowArgs a{};
+    a.src0 = static_cast<const uint8_t *>(w_gate);
+    a.src1 = static_cast<const uint8_t *>(w_up);
+    a.rows = 2 * N_h;
+    a.K = K;
+    a.row_bytes = K * dtype_size(dt);
+    a.s = s;
+    a.scale_out = w_scale_gu;
+    a.out = wq_gu;
+    return launch_rows<ROW_WEIGHT>(a, dt, as_stream(stream));
+}
+
+sq_status sq_smooth_quant_act(const void *x, sq_dtype dt, int64_t M, int64_t K, const float *s, sq_act_mode mode,
+                              float *a_scale, int8_t *xq, sq_stream stream)
+{
+    if (x == nullptr || s == nullptr || a_scale == nullptr || xq == nullptr || !valid_dt(dt)) return SQ_ERR_INVALID_ARG;
+    if (M < 0 || K <= 0 || (mode != SQ_ACT_STATIC && mode != SQ_ACT_PER_TOKEN)) return SQ_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(xq)) return SQ_ERR_MISALIGNED;
+    RowArgs a{};
+    a.src0 = static_cast<const uint8_t *>(x);
+    a.rows = M;
+    a.K = K;
+    a.row_bytes = K * dtype_size(dt);
+    a.s = s;
+    a.out = xq;
+    if (mode == SQ_ACT_STATIC) {
+        a.a_in = a_scale;
+        return launch_rows<ROW_ACT_STATIC>(a, dt, as_stream(stream));
+    }
+    a.scale_out = a_scale;
+    return launch_rows<ROW_ACT_TOKEN>(a, dt, as_stream(stream));
+}
+
+sq_status sq_rmsnorm_quant(const void *x, sq_dtype dt, int64_t M, int64_t d, const float *gamma, const float *s,
+                           float eps, const float *a_scale, int8_t *xq, float *rstd, sq_stream stream)
+{
+    if (x == nullptr || gamma == nullptr || s == nullptr || a_scale == nullptr || xq == nullptr || !valid_dt(dt))
+        return SQ_ERR_INVALID_ARG;
+    if (M < 0 || d <= 0 || !(eps >= 0.0f)) return SQ_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(xq)) return SQ_ERR_MISALIGNED;
+    RowArgs a{};
+    a.src0 = static_cast<const uint8_t *>(x);
+    a.rows = M;
+    a.K = d;
+    a.row_bytes = d * dtype_size(dt);
+    a.s = s;
+    a.gamma = gamma;
+    a.eps = eps;
+    a.a_in = a_scale;
+    a.rstd_out = rstd;
+    a.out = xq;
+    return launch_rows<ROW_RMSNORM>(a, dt, as_stream(stream));
+}
+
+size_t sq_linear_workspace_size(int64_t M, int64_t N, int64_t K)
+{
+    (void)K;
+    if (M <= 0 || N <= 0) return 0;
+    return ws_bytes(M, N);
+}
+
+static sq_status check_gemm_shape(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, int64_t K)
+{
+    if (xq == nullptr || wq == nullptr) return SQ_ERR_INVALID_ARG;
+    if (M < 1 || N < 16 || K < 16 || (N % 16) != 0 || (K % 16) != 0) return SQ_ERR_INVALID_ARG;
+    if (K >= 133144 || M > (int64_t(1) << 30) || N > (int64_t(1) << 30)) return SQ_ERR_UNSUPPORTED;
+    if (!aligned16(xq) || !aligned16(wq)) return SQ_ERR_MISALIGNED;
+    return SQ_OK;
+}
+
+sq_status sq_linear_w8a8(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, int64_t K, const float *a_scale,
+                         sq_act_mode mode, const float *w_scale, const void *bias, sq_dtype out_dt, void *y,
+                         void *workspace, size_t workspace_bytes, sq_stream stream)
+{
+    sq_status r = check_gemm_shape(xq, wq, M, N, K);
+    if (r != SQ_OK) return r;
+    if (a_scale == nullptr || w_scale == nullptr || y == nullptr || !valid_dt(out_dt)) return SQ_ERR_INVALID_ARG;
+    if (mode != SQ_ACT_STATIC && mode != SQ_ACT_PER_TOKEN) return SQ_ERR_INVALID_ARG;
+    if (!aligned16(y) || !aligned16(w_scale)) return SQ_ERR_MISALIGNED;
+    const cudaStream_t st = as_stream(stream);
+    gemm::Params p{};
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(N);
+    p.K = static_cast<int>(K);
+    p.a_scale = a_scale;
+    p.per_token = (mode == SQ_ACT_PER_TOKEN) ? 1 : 0;
+    p.w_scale = w_scale;
+    p.bias = bias;
+    p.out = y;
+    p.out_dt = out_dt;
+    if (M <= kSwapMaxM) {
+        const size_t need = ws_bytes(M, N);
+        if (workspace != nullptr && workspace_bytes >= need && aligned16(workspace)) {
+            p.ws_acc = static_cast<int32_t *>(workspace);
+            p.ws_cnt = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) +
+                                               align_up(static_cast<size_t>(M * N) * 4, 256));
+        }
+        return dispatch_swap<gemm::EPI_DEQUANT>(p, xq, wq, st);
+    }
+    fill_tiles(p, 256, M, N);
+    return launch_gemm<256, gemm::KIND_I8, gemm::EPI_DEQUANT, false>(p, xq, wq, st);
+}
+
+sq_status sq_gemm_s32(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, int64_t K, int32_t *acc,
+                      sq_stream stream)
+{
+    sq_status r = check_gemm_shape(xq, wq, M, N, K);
+    if (r != SQ_OK) return r;
+    if (acc == nullptr) return SQ_ERR_INVALID_ARG;
+    if (!aligned16(acc)) return SQ_ERR_MISALIGNED;
+    const cudaStream_t st = as_stream(stream);
+    gemm::Params p{};
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(N);
+    p.K = static_cast<int>(K);
+    p.out = acc;
+    if (M <= kSwapMaxM) return dispatch_swap<gemm::EPI_S32>(p, xq, wq, st);
+    fill_tiles(p, 256, M, N);
+    return launch_gemm<256, gemm::KIND_I8, gemm::EPI_S32, false>(p, xq, wq, st);
+}
+
+sq_status sq_linear_w8a8_gateup_silu(const int8_t *xq, const int8_t *wq_gu, int64_t M, int64_t N_h, int64_t K,
+                                     const float *a_scale, sq_act_mode mode, const float *w_scale_gu, void *h,
+                                     const float *s2, const float *a2, int8_t *hq, sq_stream stream)
+{
+    sq_status r = check_gemm_shape(xq, wq_gu, M, 2 * N_h, K);
+    if (r != SQ_OK) return r;
+    if (a_scale == nullptr || w_scale_gu == nullptr || (h == nullptr && hq == nullptr)) return SQ_ERR_INVALID_ARG;
+    if ((N_h % 128) != 0) return SQ_ERR_INVALID_ARG;
+    if (hq != nullptr && (s2 == nullptr || a2 == nullptr)) return SQ_ERR_INVALID_ARG;
+    if (mode != SQ_ACT_STATIC && mode != SQ_ACT_PER_TOKEN) return SQ_ERR_INVALID_ARG;
+    if ((h != nullptr && !aligned16(h)) || (hq != nullptr && !aligned16(hq))) return SQ_ERR_MISALIGNED;
+    gemm::Params p{};
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(2 * N_h);
+    p.K = static_cast<int>(K);
+    p.a_scale = a_scale;
+    p.per_token = (mode == SQ_ACT_PER_TOKEN) ? 1 : 0;
+    p.w_scale = w_scale_gu;
+    p.out = h;
+    p.out_dt = SQ_BF16;
+    p.s2 = s2;
+    p.a2 = a2;
+    p.hq = hq;
+    fill_tiles(p, 256, M, 2 * N_h);
+    return launch_gemm<256, gemm::KIND_I8, gemm::EPI_GATEUP, false>(p, xq, wq_gu, as_stream(stream));
+}
+
+sq_status sq_gemm_f16_ref(const void *x, const void *w, int64_t M, int64_t N, int64_t K, void *y, sq_stream stream)
+{
+    if (x == nullptr || w == nullptr || y == nullptr) return SQ_ERR_INVALID_ARG;
+    if (M < 1 || N < 16 || K < 8 || (N % 16) != 0 || (K % 8) != 0) return SQ_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w) || !aligned16(y)) return SQ_ERR_MISALIGNED;
+    gemm::Params p{};
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(N);
+    p.K = static_cast<int>(K);
+    p.out = y;
+    p.out_dt = SQ_F16;
+    fill_tiles(p, 256, M, N);
+    p.num_kb = static_cast<int>(cdiv(K, 64));   // 64 fp16 per 128-byte K block
+    p.kb_per_split = p.num_kb;
+    return launch_gemm<256, gemm::KIND_F16, gemm::EPI_F16, false>(p, x, w, as_stream(stream));
+}
+
+sq_status sq_sse_f16(const void *y, const void *y_ref, int64_t n, double *sse, sq_stream stream)
+{
+    if (y == nullptr || y_ref == nullptr || sse == nullptr || n < 0) return SQ_ERR_INVALID_ARG;
+    if (!aligned16(y) || !aligned16(y_ref)) return SQ_ERR_MISALIGNED;
+    if (n == 0) return SQ_OK;
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(cdiv(n, 8 * 256), static_cast<int64_t>(sm_count()) * 4));
+    k_sse_f16<<<static_cast<unsigned>(grid), 256, 0, as_stream(stream)>>>(static_cast<const __half *>(y),
+                                                                       static_cast<const __half *>(y_ref), n, sse);
+    return check_launch();
+}
+
+static size_t alpha_ws_layout(int64_t Mh, int64_t N, int64_t K, int n_alpha, size_t off[8])
+{
+    size_t o = 0;
+    off[0] = o; o = align_up(o + static_cast<size_t>(K) * 4, 256);          // s
+    off[1] = o; o = align_up(o + 4, 256);                                   // a
+    off[2] = o; o = align_up(o + static_cast<size_t>(N * K), 256);          // wq
+    off[3] = o; o = align_up(o + static_cast<size_t>(N) * 4, 256);          // w_scale
+    off[4] = o; o = align_up(o + static_cast<size_t>(Mh * K), 256);         // xq
+    off[5] = o; o = align_up(o + static_cast<size_t>(Mh * N) * 2, 256);     // y
+    off[6] = o; o = align_up(o + static_cast<size_t>(Mh * N) * 2, 256);     // y_ref
+    off[7] = o; o = align_up(o + static_cast<size_t>(n_alpha) * 8, 256);    // sse
+    const size_t lin = ws_bytes(Mh, N);
+    return o + lin;
+}
+
+size_t sq_alpha_search_workspace_size(int64_t M_held, int64_t N, int64_t K, int n_alpha)
+{
+    if (M_held <= 0 || N <= 0 || K <= 0 || n_alpha <= 0) return 0;
+    size_t off[8];
+    return alpha_ws_layout(M_held, N, K, n_alpha, off);
+}
+
+sq_status sq_alpha_search(const void *x_held, const void *w, int64_t M_held, int64_t N, int64_t K,
+                          const float *act_max, const float *w_max, const float *alphas, int n_alpha,
+                          void *workspace, size_t workspace_bytes, float *best_alpha, double *mse,
+                          sq_stream stream)
+{
+    if (x_held == nullptr || w == nullptr || act_max == nullptr || w_max == nullptr || alphas == nullptr ||
+        best_alpha == nullptr || workspace == nullptr)
+        return SQ_ERR_INVALID_ARG;
+    if (n_alpha < 1 || n_alpha > 16) return SQ_ERR_INVALID_ARG;
+    for (int i = 0; i < n_alpha; ++i)
+        if (!(alphas[i] >= 0.0f && alphas[i] <= 1.0f) || (i > 0 && !(alphas[i] > alphas[i - 1])))
+            return SQ_ERR_INVALID_ARG;
+    size_t off[8];
+    const size_t need = alpha_ws_layout(M_held, N, K, n_alpha, off);
+    if (workspace_bytes < need || !aligned16(workspace)) return SQ_ERR_WORKSPACE;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    float *s = reinterpret_cast<float *>(ws + off[0]);
+    float *a = reinterpret_cast<float *>(ws + off[1]);
+    int8_t *wq = reinterpret_cast<int8_t *>(ws + off[2]);
+    float *w_scale = reinterpret_cast<float *>(ws + off[3]);
+    int8_t *xq = reinterpret_cast<int8_t *>(ws + off[4]);
+    void *y = ws + off[5];
+    void *y_ref = ws + off[6];
+    double *sse = reinterpret_cast<double *>(ws + off[7]);
+    void *lin_ws = ws + (need - ws_bytes(M_held, N));
+    const size_t lin_bytes = ws_bytes(M_held, N);
+    const cudaStream_t st = as_stream(stream);
+
+    sq_status r = sq_gemm_f16_ref(x_held, w, M_held, N, K, y_ref, stream);
+    if (r != SQ_OK) return r;
+    cudaError_t e = cudaMemsetAsync(sse, 0, static_cast<size_t>(n_alpha) * 8, st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (lin_bytes > 0) {
+        e = cudaMemsetAsync(lin_ws, 0, lin_bytes, st);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    for (int i = 0; i < n_alpha; ++i) {
+        if ((r = sq_smooth_scales(act_max, w_max, K, alphas[i], s, a, stream)) != SQ_OK) return r;
+        if ((r = sq_quant_weight(w, SQ_F16, N, K, s, wq, w_scale, stream)) != SQ_OK) return r;
+        if ((r = sq_smooth_quant_act(x_held, SQ_F16, M_held, K, s, SQ_ACT_STATIC, a, xq, stream)) != SQ_OK) return r;
+        if ((r = sq_linear_w8a8(xq, wq, M_held, N, K, a, SQ_ACT_STATIC, w_scale, nullptr, SQ_F16, y, lin_ws,
+                                lin_bytes, stream)) != SQ_OK)
+            return r;
+        if ((r = sq_sse_f16(y, y_ref, M_held * N, sse + i, stream)) != SQ_OK) return r;
+    }
+    double host_sse[16];
+    e = cudaMemcpyAsync(host_sse, sse, static_cast<size_t>(n_alpha) * 8, cudaMemcpyDeviceToHost, st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    r = sq_sync_status(stream);
+    if (r != SQ_OK) return r;
+    const double n = static_cast<double>(M_held) * static_cast<double>(N);
+    int best = 0;
+    for (int i = 0; i < n_alpha; ++i) {
+        const double m = host_sse[i] / n;
+        if (mse != nullptr) mse[i] = m;
+        if (i > 0 && m < (host_sse[best] / n) * (1.0 - 1e-6)) best = i;
+    }
+    *best_alpha = alphas[best];
+    return SQ_OK;
+}
+
+}  // extern "C"

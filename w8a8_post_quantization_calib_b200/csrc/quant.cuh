@@ -1,0 +1,291 @@
+// quant.cuh -- smoothing factors, the offline weight transform + per-row INT8
+// quantisation, the runtime smooth + quantise of activations (static or
+// per-token), RMSNorm with 1/s folded into its gain, and the squared-error
+// reduction of the alpha search.
+//
+// Row kernels (HBM-bound): a block of ROW_T threads owns whole rows.  A row
+// is read once into registers as 16-byte vectors (vector i*ROW_T + tid), the
+// per-row statistic (absmax or sum of squares) is reduced across the block,
+// and the codes are written from the same registers, so every element moves
+// through HBM exactly once (16-bit in, 8-bit out).  The per-column constant
+// of the step (s_j, fl(1/s_j) or fl(gamma_j * fl(1/s_j))) is computed once
+// per block into shared memory.  Blocks loop over rows (grid <= rows).
+#pragma once
+
+#include "common.cuh"
+
+namespace sq {
+
+// ---------------------------------------------------------------------------
+// s_j = max(a_j,1e-5)^alpha / max(w_j,1e-5)^(1-alpha) in fp64, rounded once
+// (kwkr.cn blog 2.2; aiunderstanding.org technical insight; "010. SmoothQuant
+// Integration" context step 1; the 1e-5 clamp follows tbr8.org's example).
+// Optionally a_static = fl(max_j fl(act_max_j * recip(s_j)) / 127), the closed
+// form of "010. SmoothQuant Integration" key design point 1.  x -> fl(x/127)
+// is monotone, so max_b fl(m_b/127) = fl(max_b m_b / 127): blocks combine
+// with atomicMax on the (non-negative) float bits; *a_static is zeroed first.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+    k_smooth_scales(const float *__restrict__ act_max, const float *__restrict__ w_max, int64_t K,
+                    float alpha, float *__restrict__ s, float *__restrict__ a_static)
+{
+    __shared__ float red[32];
+    const double al = static_cast<double>(alpha);
+    float m = 0.0f;
+    for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < K;
+         j += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const double a = fmax(static_cast<double>(act_max[j]), 1e-5);
+        const double w = fmax(static_cast<double>(w_max[j]), 1e-5);
+        const float sj = static_cast<float>(pow(a, al) / pow(w, 1.0 - al));
+        s[j] = sj;
+        m = fmaxf(m, __fmul_rn(act_max[j], recip_or_zero(sj)));
+    }
+    if (a_static != nullptr) {
+        m = block_max(m, red);
+        if (threadIdx.x == 0) atomicMax(reinterpret_cast<int *>(a_static), __float_as_int(scale_from_absmax(m)));
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Row kernels
+// ---------------------------------------------------------------------------
+enum RowMode : int {
+    ROW_WEIGHT = 0,      // W' = fl(w*s_j); per-row scale; codes
+    ROW_ACT_STATIC = 1,  // x' = fl(x*fl(1/s_j)); codes with the given scale
+    ROW_ACT_TOKEN = 2,   // x' as above; per-row scale written; codes
+    ROW_RMSNORM = 3      // y = fl(fl(x*r)*fl(gamma_j*fl(1/s_j))); codes with the given scale
+};
+
+constexpr int ROW_T = 256;
+
+struct RowArgs {
+    const uint8_t *src0;     // input rows (row r at src0 + r*row_bytes)
+    const uint8_t *src1;     // gate/up: up rows (src0 = gate rows), else null
+    int64_t rows;            // rows to produce
+    int64_t K;               // elements per row
+    int64_t row_bytes;       // K * element size
+    const float *s;          // [K]
+    const float *gamma;      // [K] (RMSNorm)
+    float eps;
+    const float *a_in;       // static scale [1] (act static, RMSNorm)
+    float *scale_out;        // per-row scales [rows] (weight, per-token)
+    float *rstd_out;         // RMSNorm r_m [rows] or null
+    int8_t *out;             // codes [rows, K]
+};
+
+template <int DT>
+__device__ __forceinline__ void store_codes(int8_t *dst_row, int64_t v, const float (&f)[VecT<DT>::EPV])
+{
+    constexpr int EPV = VecT<DT>::EPV;
+    if constexpr (EPV == 8) {
+        uint2 o;
+        o.x = pack4(quant8(f[0]), quant8(f[1]), quant8(f[2]), quant8(f[3]));
+        o.y = pack4(quant8(f[4]), quant8(f[5]), quant8(f[6]), quant8(f[7]));
+        *reinterpret_cast<uint2 *>(dst_row + v * 8) = o;
+    } else {
+        *reinterpret_cast<uint32_t *>(dst_row + v * 4) =
+            pack4(quant8(f[0]), quant8(f[1]), quant8(f[2]), quant8(f[3]));
+    }
+}
+
+template <int DT, int VPT, int MODE>
+__global__ void __launch_bounds__(ROW_T) k_rows(RowArgs p)
+{
+    constexpr int EPV = VecT<DT>::EPV;
+    extern __shared__ float colv[];          // per-column constant, K floats
+    __shared__ float red[32];
+    __shared__ double red64[32];
+
+    const int tid = threadIdx.x;
+    const int64_t nvec = p.K / EPV;
+
+    // per-column constant of this step
+    for (int64_t j = tid; j < p.K; j += ROW_T) {
+        if constexpr (MODE == ROW_WEIGHT) colv[j] = p.s[j];
+        else if constexpr (MODE == ROW_RMSNORM) colv[j] = __fmul_rn(p.gamma[j], recip_or_zero(p.s[j]));
+        else colv[j] = recip_or_zero(p.s[j]);
+    }
+    float inv_a_static = 0.0f;
+    if constexpr (MODE == ROW_ACT_STATIC || MODE == ROW_RMSNORM) inv_a_static = recip_or_zero(p.a_in[0]);
+    __syncthreads();
+
+    for (int64_t row = blockIdx.x; row < p.rows; row += gridDim.x) {
+        const uint8_t *src;
+        if (p.src1 != nullptr) {          // gate/up interleave: blocks of 64 output rows
+            const int64_t b = row >> 6, w = row & 63;
+            src = (w < 32 ? p.src0 : p.src1) + ((b << 5) + (w & 31)) * p.row_bytes;
+        } else {
+            src = p.src0 + row * p.row_bytes;
+        }
+        uint4 raw[VPT];
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int64_t v = static_cast<int64_t>(i) * ROW_T + tid;
+            if (v < nvec) raw[i] = __ldcs(reinterpret_cast<const uint4 *>(src) + v);
+        }
+
+        // pass 1: the per-row statistic (absmax in fp32; sum of squares in fp64,
+        // where every square of a 16-bit or fp32 input is exact)
+        float stat = 0.0f;
+        double ss = 0.0;
+        if constexpr (MODE != ROW_ACT_STATIC) {
+#pragma unroll
+            for (int i = 0; i < VPT; ++i) {
+                const int64_t v = static_cast<int64_t>(i) * ROW_T + tid;
+                if (v < nvec) {
+                    float f[EPV];
+                    widen<DT>(raw[i], f);
+                    const float4 *cv = reinterpret_cast<const float4 *>(colv + v * EPV);
+#pragma unroll
+                    for (int e = 0; e < EPV; e += 4) {
+                        const float4 c = cv[e / 4];
+                        const float cc[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+                        for (int t = 0; t < 4; ++t) {
+                            if constexpr (MODE == ROW_RMSNORM)
+                                ss += static_cast<double>(f[e + t]) * static_cast<double>(f[e + t]);
+                            else
+                                stat = fmaxf(stat, fabsf(__fmul_rn(f[e + t], cc[t])));
+                        }
+                    }
+                }
+            }
+        }
+        float mul_a;          // multiplier applied before rounding
+        float r_m = 0.0f;     // RMSNorm row factor
+        if constexpr (MODE == ROW_ACT_STATIC) {
+            mul_a = inv_a_static;
+        } else if constexpr (MODE == ROW_RMSNORM) {
+            const double tot = block_sum_f64(ss, red64);
+            const float mean = __double2float_rn(tot / static_cast<double>(p.K));
+            r_m = __frcp_rn(__fsqrt_rn(__fadd_rn(mean, p.eps)));
+            mul_a = inv_a_static;
+            if (tid == 0 && p.rstd_out != nullptr) p.rstd_out[row] = r_m;
+        } else {
+            const float mx = block_max(stat, red);
+            const float sc = scale_from_absmax(mx);
+            mul_a = recip_or_zero(sc);
+            if (tid == 0) p.scale_out[row] = sc;
+        }
+
+        // pass 2: codes
+        int8_t *dst = p.out + row * p.K;
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int64_t v = static_cast<int64_t>(i) * ROW_T + tid;
+            if (v < nvec) {
+                float f[EPV];
+                widen<DT>(raw[i], f);
+                const float4 *cv = reinterpret_cast<const float4 *>(colv + v * EPV);
+#pragma unroll
+                for (int e = 0; e < EPV; e += 4) {
+                    const float4 c = cv[e / 4];
+                    const float cc[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        float y;
+                        if constexpr (MODE == ROW_RMSNORM) y = __fmul_rn(__fmul_rn(f[e + t], r_m), cc[t]);
+                        else y = __fmul_rn(f[e + t], cc[t]);
+                        f[e + t] = __fmul_rn(y, mul_a);
+                    }
+                }
+                store_codes<DT>(dst, v, f);
+            }
+        }
+    }
+}
+
+// Unaligned / very wide rows: one block per row, elementwise, two passes
+// over global memory (correct for any K; not tuned).
+template <int MODE>
+__global__ void __launch_bounds__(ROW_T) k_rows_scalar(RowArgs p, int dt)
+{
+    __shared__ float red[32];
+    __shared__ double red64[32];
+    const int tid = threadIdx.x;
+    float inv_a_static = 0.0f;
+    if constexpr (MODE == ROW_ACT_STATIC || MODE == ROW_RMSNORM) inv_a_static = recip_or_zero(p.a_in[0]);
+    for (int64_t row = blockIdx.x; row < p.rows; row += gridDim.x) {
+        const uint8_t *src;
+        if (p.src1 != nullptr) {
+            const int64_t b = row >> 6, w = row & 63;
+            src = (w < 32 ? p.src0 : p.src1) + ((b << 5) + (w & 31)) * p.row_bytes;
+        } else {
+            src = p.src0 + row * p.row_bytes;
+        }
+        auto colc = [&](int64_t j) -> float {
+            if constexpr (MODE == ROW_WEIGHT) return p.s[j];
+            else if constexpr (MODE == ROW_RMSNORM) return __fmul_rn(p.gamma[j], recip_or_zero(p.s[j]));
+            else return recip_or_zero(p.s[j]);
+        };
+        float stat = 0.0f;
+        double ss = 0.0;
+        if constexpr (MODE != ROW_ACT_STATIC) {
+            for (int64_t j = tid; j < p.K; j += ROW_T) {
+                const float x = load_elem_dt(src, dt, j);
+                if constexpr (MODE == ROW_RMSNORM) ss += static_cast<double>(x) * static_cast<double>(x);
+                else stat = fmaxf(stat, fabsf(__fmul_rn(x, colc(j))));
+            }
+        }
+        float mul_a, r_m = 0.0f;
+        if constexpr (MODE == ROW_ACT_STATIC) {
+            mul_a = inv_a_static;
+        } else if constexpr (MODE == ROW_RMSNORM) {
+            const double tot = block_sum_f64(ss, red64);
+            const float mean = __double2float_rn(tot / static_cast<double>(p.K));
+            r_m = __frcp_rn(__fsqrt_rn(__fadd_rn(mean, p.eps)));
+            mul_a = inv_a_static;
+            if (tid == 0 && p.rstd_out != nullptr) p.rstd_out[row] = r_m;
+        } else {
+            const float sc = scale_from_absmax(block_max(stat, red));
+            mul_a = recip_or_zero(sc);
+            if (tid == 0) p.scale_out[row] = sc;
+        }
+        for (int64_t j = tid; j < p.K; j += ROW_T) {
+            const float x = load_elem_dt(src, dt, j);
+            float y;
+            if constexpr (MODE == ROW_RMSNORM) y = __fmul_rn(__fmul_rn(x, r_m), colc(j));
+            else y = __fmul_rn(x, colc(j));
+            p.out[row * p.K + j] = static_cast<int8_t>(quant8(__fmul_rn(y, mul_a)));
+        }
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Sum of squared differences of two fp16 tensors, fp64 accumulation.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+    k_sse_f16(const __half *__restrict__ y, const __half *__restrict__ r, int64_t n, double *__restrict__ sse)
+{
+    __shared__ double red[8];
+    double acc = 0.0;
+    const int64_t nv = n / 8;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < nv; v += stride) {
+        const uint4 a = __ldg(reinterpret_cast<const uint4 *>(y) + v);
+        const uint4 b = __ldg(reinterpret_cast<const uint4 *>(r) + v);
+        const __half *ha = reinterpret_cast<const __half *>(&a);
+        const __half *hb = reinterpret_cast<const __half *>(&b);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const double d = static_cast<double>(__half2float(ha[e])) - static_cast<double>(__half2float(hb[e]));
+            acc += d * d;
+        }
+    }
+    for (int64_t i = nv * 8 + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride) {
+        const double d = static_cast<double>(__half2float(y[i])) - static_cast<double>(__half2float(r[i]));
+        acc += d * d;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double t = 0.0;
+        for (int i = 0; i < (blockDim.x >> 5); ++i) t += red[i];
+        atomicAdd(sse, t);
+    }
+}
+
+}  // namespace sq
