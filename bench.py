@@ -1,0 +1,436 @@
+#!/usr/bin/env python3
+"""Benchmark of the SmoothQuant W8A8 linear layer on B200.
+
+Workload: a Llama-7B-shaped QKV projection (K=4096 in, N=12288 out, M=2048
+runtime tokens, fp16 activations and weights with 0.5% seeded outlier
+channels x U(20,100), W ~ N(0, 0.02^2)), calibrated on 64 batches of 512
+tokens, alpha=0.5, per-tensor static activation scale, per-row weight scale,
+fp16 output.  Synthetic, seeded inputs.
+
+One step = the whole hot path over one batch, all through the C ABI:
+  calibration absmax over the 32768 calibration tokens (one launch) ->
+  weight column absmax -> smoothing factors + closed-form static scale ->
+  weight transform + per-row INT8 -> runtime smooth + INT8 quant of X ->
+  tcgen05 INT8 GEMM with the fp16 dequant epilogue.
+Under torchrun (N>1) each rank calibrates its own 64 x 512 token shard and
+runs its own runtime batch (weak scaling); the per-channel maxima are
+combined with one NCCL all-reduce(MAX) of K floats before the smoothing
+factors -- the only exchange the method has.
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle
+instead, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W8A8 linear INT8 TOPS & tokens/s at 1 B200; % of INT8 peak / HBM GB/s"
+WORKLOAD = ("Llama-7B QKV projection: K=4096, N=12288, M=2048 tokens, fp16 X/W with 0.5% outlier "
+            "channels, 64x512 calibration tokens, alpha=0.5, static per-tensor act scale, per-row "
+            "weight scale, fp16 out")
+M_TOK, K_IN, N_OUT, CALIB_B, CALIB_R = 2048, 4096, 12288, 64, 512
+ALPHA = 0.5
+
+
+def peaks():
+    """Measured roofline denominators (generated file) or the recipe's fallback."""
+    src = "measured"
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            mp = json.load(f)
+        hbm, bf16, bf16_s = float(mp["hbm_gbs"]), float(mp["bf16_tflops"]), float(mp["bf16_tflops_sustained"])
+    except Exception:
+        hbm, bf16, bf16_s, src = 6650.0, 1590.0, 1400.0, "fallback"
+    # INT8 dense tensor peak = measured bf16 x the nominal dense ratio 4.5 / 2.25
+    return {"hbm_gbs": hbm, "int8_tops": bf16 * 2.0, "int8_tops_sustained": bf16_s * 2.0, "source": src}
+
+
+def gemm_traffic():
+    """DRAM bytes per GEMM launch from the committed ncu summary, or None when the
+    kernel source changed after the counters were taken."""
+    import hashlib
+    tf = os.path.join(ROOT, "profiles", "linear_w8a8_qkv7b_traffic.json")
+    try:
+        d = json.load(open(tf))
+        h = hashlib.sha256()
+        for f in ("gemm.cuh", "ptx_sm100.cuh"):
+            h.update(open(os.path.join(ROOT, "w8a8_post_quantization_calib_b200", "csrc", f), "rb").read())
+        return d["dram_bytes_per_launch"] if h.hexdigest()[:16] == d["source_sha256_16"] else None
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """Polls SM clocks and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle"}
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            uuid = None
+            try:
+                import torch
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            except Exception:
+                pass
+            h = None
+            if uuid:
+                for cand in (uuid, "GPU-" + uuid):
+                    try:
+                        h = pynvml.nvmlDeviceGetHandleByUUID(cand)
+                        break
+                    except Exception:
+                        pass
+            self.h = h if h is not None else pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                fn = getattr(self.nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    self.nv.nvmlDeviceGetCurrentClocksThrottleReasons
+                r = fn(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.nv is not None:
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------
+# CPU oracle timing (reference arm and cpu_baseline)
+# --------------------------------------------------------------------------
+def oracle_sample(frac: float, wl=None):
+    """Run the oracle's full step on a fraction `frac` of every part of the workload.
+
+    Every part is linear in its row count (calibration rows, weight rows for
+    the statistic and the quantisation, runtime token rows for quantisation
+    and the INT8 GEMM over all N), so step time ~= sample time / frac.
+    Returns (seconds, description).
+    """
+    import numpy as np
+    import oracle
+    import synth
+    if wl is None:
+        wl = synth.qkv_7b()
+    calib = np.concatenate(wl.calib)
+    rc = max(1, int(round(calib.shape[0] * frac)))
+    rw = max(1, int(round(N_OUT * frac)))
+    rx = max(1, int(round(M_TOK * frac)))
+    t0 = time.perf_counter()
+    act_max = np.zeros(K_IN, np.float32)
+    oracle.calib_absmax(calib[:rc], synth.F16, act_max)
+    w_max = oracle.calib_absmax(wl.w[:rw], synth.F16)
+    s = oracle.smooth_scales(act_max, w_max, ALPHA)
+    a = oracle.static_scale(act_max, s)
+    wq, ws = oracle.quant_weight(wl.w[:rw], s, synth.F16)
+    xq, av = oracle.smooth_quant_act(wl.x[:rx], s, oracle.STATIC, a, synth.F16)
+    wq_full = np.resize(wq, (N_OUT, K_IN))          # GEMM over all N output channels
+    ws_full = np.resize(ws, N_OUT)
+    acc = oracle.gemm_s32(xq, wq_full)
+    oracle.dequant(acc, av, oracle.STATIC, ws_full, synth.F16)
+    dt = time.perf_counter() - t0
+    desc = (f"oracle full step on a {frac:.4f} fraction of every part: {rc} calibration rows, {rw} weight rows "
+            f"(statistic + quantisation), {rx} runtime tokens (quant + INT8 GEMM over all N={N_OUT}); "
+            f"step time extrapolated as sample time / fraction")
+    return dt, desc
+
+
+def cpu_cores():
+    n = os.environ.get("OMP_NUM_THREADS")
+    return int(n) if n and n.isdigit() else (os.cpu_count() or 1)
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    import synth
+    oracle.build()
+    wl = synth.qkv_7b()
+    ops = 2.0 * M_TOK * N_OUT * K_IN
+    # size one step so that warmup + steps stay within ~2 minutes
+    t_probe, _ = oracle_sample(1.0 / 512, wl)
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    frac = min(1.0, max(1.0 / 2048, (1.0 / 512) * budget / max(t_probe, 1e-3)))
+    for _ in range(args.warmup):
+        oracle_sample(frac, wl)
+    times, desc = [], ""
+    for _ in range(args.steps):
+        t, desc = oracle_sample(frac, wl)
+        times.append(t / frac)
+    ms = 1e3 * statistics.mean(times)
+    value = ops / (ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "s8", "data": "synthetic", "impl": "reference",
+        "config": {"workload": WORKLOAD, "M": M_TOK, "K": K_IN, "N": N_OUT, "calib_tokens": CALIB_B * CALIB_R,
+                   "parallelism": "host cores"},
+        "tokens_per_s": M_TOK / (ms * 1e-3),
+        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": cpu_cores(), "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------
+# GPU arm
+# --------------------------------------------------------------------------
+def run_gpu(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    import synth
+    import w8a8_post_quantization_calib_b200 as sq
+
+    P = peaks()
+    wl = synth.qkv_7b(shard=rank)
+    dev = torch.device("cuda", local)
+
+    def up(bits, dt=torch.float16):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(dt)
+
+    calib_h = up(np.concatenate(wl.calib)).pin_memory()
+    w_h = up(wl.w).pin_memory()
+    x_h = up(wl.x).pin_memory()
+    calib = calib_h.to(dev)
+    W = w_h.to(dev)
+    X = x_h.to(dev)
+    act_max = torch.zeros(K_IN, dtype=torch.float32, device=dev)
+    w_max = torch.zeros(K_IN, dtype=torch.float32, device=dev)
+    s = torch.empty(K_IN, dtype=torch.float32, device=dev)
+    a = torch.empty(1, dtype=torch.float32, device=dev)
+    wq = torch.empty(N_OUT, K_IN, dtype=torch.int8, device=dev)
+    ws = torch.empty(N_OUT, dtype=torch.float32, device=dev)
+    xq = torch.empty(M_TOK, K_IN, dtype=torch.int8, device=dev)
+    y = torch.empty(M_TOK, N_OUT, dtype=torch.float16, device=dev)
+    y_h = torch.empty(M_TOK, N_OUT, dtype=torch.float16).pin_memory()
+    stream = torch.cuda.current_stream()
+    names = ["calib_absmax", "weight_absmax", "smooth_scales", "quant_weight", "smooth_quant_act", "linear_w8a8"]
+    if world > 1:
+        names.insert(1, "allreduce_max")
+
+    def step(evs=None):
+        def mark(i):
+            if evs is not None:
+                evs[i].record(stream)
+        i = 0
+        mark(i)
+        act_max.zero_()
+        sq.calib_absmax(calib, act_max)
+        i += 1
+        mark(i)
+        if world > 1:
+            dist.all_reduce(act_max, op=dist.ReduceOp.MAX)
+            i += 1
+            mark(i)
+        w_max.zero_()
+        sq.calib_absmax(W, w_max)
+        i += 1
+        mark(i)
+        sq.smooth_scales(act_max, w_max, ALPHA, s, a)
+        i += 1
+        mark(i)
+        sq.quant_weight(W, s, wq, ws)
+        i += 1
+        mark(i)
+        sq.smooth_quant_act(X, s, sq.ACT_STATIC, a, xq)
+        i += 1
+        mark(i)
+        sq.linear_w8a8(xq, wq, a, sq.ACT_STATIC, ws, y)
+        i += 1
+        mark(i)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
+    if sq.sync_status() != 0:
+        raise RuntimeError("kernel error during warm-up")
+
+    # ---- timed region: K steps, per-kernel events on the launching stream
+    nk = len(names)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    with ClockSampler(local) as clk:
+        t_start.record(stream)
+        for k in range(args.steps):
+            step(evs[k])
+        t_end.record(stream)
+        barrier()
+    st = sq.sync_status()
+    if st != 0:
+        raise RuntimeError(f"kernel error in the timed region (status {st})")
+    ms_total = t_start.elapsed_time(t_end)
+    per_kernel = [statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps))
+                  for i in range(nk)]
+    ms_step = ms_total / args.steps
+    if world > 1:
+        t = torch.tensor([ms_step], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step = float(t.item())
+
+    ops = 2.0 * M_TOK * N_OUT * K_IN
+    value = world * ops / (ms_step * 1e-3) / 1e12
+    kt = dict(zip(names, per_kernel))
+
+    # algorithmic bytes / ops per launch
+    calib_bytes = CALIB_B * CALIB_R * K_IN * 2
+    kern = {
+        "calib_absmax": {"ms": kt["calib_absmax"], "bytes": calib_bytes},
+        "weight_absmax": {"ms": kt["weight_absmax"], "bytes": N_OUT * K_IN * 2},
+        "smooth_scales": {"ms": kt["smooth_scales"], "bytes": K_IN * 4 * 3},
+        "quant_weight": {"ms": kt["quant_weight"], "bytes": N_OUT * K_IN * 3 + N_OUT * 4},
+        "smooth_quant_act": {"ms": kt["smooth_quant_act"], "bytes": M_TOK * K_IN * 3},
+        "linear_w8a8": {"ms": kt["linear_w8a8"], "ops": ops,
+                        "bytes": M_TOK * K_IN + N_OUT * K_IN + M_TOK * N_OUT * 2 + N_OUT * 4},
+    }
+    for k, v in kern.items():
+        v["share"] = v["ms"] / ms_step
+        if "ops" in v:
+            v["tops"] = v["ops"] / (v["ms"] * 1e-3) / 1e12
+            v["frac_int8_peak"] = v["tops"] / P["int8_tops"]
+        v["gbs"] = v["bytes"] / (v["ms"] * 1e-3) / 1e9
+        v["frac_hbm"] = v["gbs"] / P["hbm_gbs"]
+    if world > 1:
+        kern["allreduce_max"] = {"ms": kt["allreduce_max"], "share": kt["allreduce_max"] / ms_step}
+
+    g = kern["linear_w8a8"]
+    traffic = gemm_traffic()
+    roofline = {"bound": "tensor", "kernel": "linear_w8a8 (tcgen05 kind::i8 GEMM + dequant)",
+                "achieved": g["tops"], "peak": P["int8_tops"], "unit": "TOPS", "frac": g["tops"] / P["int8_tops"],
+                "traffic": traffic,
+                "peak_note": f"INT8 dense = 2 x {P['source']} bf16 cuBLAS burst (nominal 4.5/2.25 ratio); "
+                             f"vs sustained {P['int8_tops_sustained']:.0f}: {g['tops'] / P['int8_tops_sustained']:.3f}"}
+
+    # ---- end to end: pinned host buffers, H2D of the step's inputs and D2H of the result in the region
+    e2e_steps = max(1, min(args.steps, 5))
+    h2d = calib_h.numel() * 2 + w_h.numel() * 2 + x_h.numel() * 2
+    d2h = y_h.numel() * 2
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        calib.copy_(calib_h, non_blocking=True)
+        W.copy_(w_h, non_blocking=True)
+        X.copy_(x_h, non_blocking=True)
+        step()
+        y_h.copy_(y, non_blocking=True)
+    e1.record(stream)
+    barrier()
+    ms_e2e = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([ms_e2e], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+    e2e = {"value": world * ops / (ms_e2e * 1e-3) / 1e12, "unit": "TOPS", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e, "steps": e2e_steps}
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        frac = args.cpu_frac
+        t, desc = oracle_sample(frac, wl)
+        cpu = {"value": ops / (t / frac) / 1e12, "unit": "TOPS", "cores": cpu_cores(), "kind": "oracle",
+               "sample": desc, "sample_seconds": t}
+
+    launches_per_step = 6
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "s8", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "M": M_TOK, "K": K_IN, "N": N_OUT, "calib_tokens": CALIB_B * CALIB_R,
+                       "alpha": ALPHA, "parallelism": f"dp{world} (token shards; all-reduce MAX of act_max)",
+                       "l2": "no flush: every step streams 384 MB of inputs (> 126 MB L2)"},
+            "tokens_per_s": world * M_TOK / (ms_step * 1e-3),
+            "roofline": roofline,
+            "kernels": kern,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "clocks": clk.summary(),
+            "gpu_launches": launches_per_step * args.steps,
+            "gpu_launches_note": "6 libsq kernels per step (+2 torch fills zeroing the running maxima, "
+                                 "+1 memset of the static scale)",
+            "peaks": P,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["sq", "reference"], default="sq")
+    ap.add_argument("--cpu-frac", type=float, default=0.25,
+                    help="fraction of the workload the CPU oracle baseline runs")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

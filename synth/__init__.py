@@ -107,8 +107,13 @@ def linear_toy(M: int = 16, K: int = 1024, N: int = 2048, calib_batches: int = 4
 def outlier_linear(M: int, K: int, N: int, calib_batches: int, calib_rows: int,
                    x_dt: int, w_dt: int, out_dt: int, workload: int, mode: int = 0,
                    frac: float = 0.005, lo: float = 20.0, hi: float | None = 100.0,
-                   heavy_tail: bool = False, w_sigma: float = 0.02) -> LinearWorkload:
-    """Llama-shaped linear with seeded, token-consistent outlier channels."""
+                   heavy_tail: bool = False, w_sigma: float = 0.02, shard: int = 0) -> LinearWorkload:
+    """Llama-shaped linear with seeded, token-consistent outlier channels.
+
+    ``shard`` selects an independent set of calibration and runtime token
+    batches (same layer, same weight, same outlier channels): one per rank
+    when the token batches are spread over several GPUs.
+    """
     idx, c = outlier_channels(rng(workload, 1), K, frac, lo, hi)
 
     def act(stream, rows):
@@ -120,17 +125,17 @@ def outlier_linear(M: int, K: int, N: int, calib_batches: int, calib_rows: int,
         return cast(apply_channels(x, idx, c), x_dt)
 
     wl = LinearWorkload("outlier linear", K, N, M, x_dt, w_dt, out_dt, mode=mode)
-    wl.calib = [act(100 + b, calib_rows) for b in range(calib_batches)]
-    wl.x = act(2, M)
+    wl.calib = [act(100 + b + 100000 * shard, calib_rows) for b in range(calib_batches)]
+    wl.x = act(2 + 100000 * shard, M)
     wl.w = cast(normal(rng(workload, 3), (N, K), w_sigma), w_dt)
     wl.outlier_idx = idx
     return wl
 
 
 def qkv_7b(M: int = 2048, K: int = 4096, N: int = 12288, calib_batches: int = 64,
-           calib_rows: int = 512) -> LinearWorkload:
+           calib_rows: int = 512, shard: int = 0) -> LinearWorkload:
     """Llama-7B-shaped QKV projection: fp16 X and W, static scale, fp16 out."""
-    return outlier_linear(M, K, N, calib_batches, calib_rows, F16, F16, F16, workload=2)
+    return outlier_linear(M, K, N, calib_batches, calib_rows, F16, F16, F16, workload=2, shard=shard)
 
 
 def mlp_7b(which: str, M: int, calib_batches: int = 64, calib_rows: int = 512,
