@@ -205,6 +205,35 @@ sq_status sq_linear_w8a8(const int8_t *xq, const int8_t *wq, int64_t M, int64_t 
                          const void *bias, sq_dtype out_dt, void *y, void *workspace,
                          size_t workspace_bytes, sq_stream stream);
 
+/* sq_linear_w8a8 for callers that cannot allocate device memory (the pages
+ * have no counterpart to this call).  Some callers cannot call cudaMalloc at
+ * all: a plugin running inside a host engine that owns every device buffer
+ * and hands it only inputs and outputs, or a latency-critical serving loop
+ * that must not pay cudaMalloc's implicit device-wide synchronisation.  This
+ * call takes no workspace: the small-M split-K path (M <= 128) keeps its
+ * int32 partial sums and per-tile counters in a fixed array inside the
+ * library (8 MiB of partial sums + 64 KiB of counters, held by every GPU that
+ * loads the library until the process exits).  M*N beyond
+ * sq_linear_w8a8_noalloc_max_elems() (2^21 = 2097152) on that path returns
+ * SQ_ERR_UNSUPPORTED without launching; M > 128 needs no scratch and runs the
+ * sq_linear_w8a8 launch.  The call allocates nothing: no cudaMalloc,
+ * cudaFree or allocating library routine.
+ *   - The first call on each device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - Each call zeroes the part of the array it uses (stream-ordered memsets)
+ *     before its kernel, since the array keeps the previous call's contents.
+ *   - All calls on a device share the one array: calls that overlap on the
+ *     GPU (different streams, no ordering between them) race and corrupt each
+ *     other's results.  Serialise them on one stream or order them with events.
+ * Arguments, layouts and results are those of sq_linear_w8a8. */
+sq_status sq_linear_w8a8_noalloc(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, int64_t K,
+                                 const float *a_scale, sq_act_mode mode, const float *w_scale,
+                                 const void *bias, sq_dtype out_dt, void *y, sq_stream stream);
+
+/* Largest M*N the fixed array of sq_linear_w8a8_noalloc holds on its small-M path. */
+size_t sq_linear_w8a8_noalloc_max_elems(void);
+
 /* Raw int32 accumulators acc[m,n] = sum_k xq[m,k] * wq[n,k] from the same
  * tensor-core mainloop (for exact INT32 checks).  acc: int32 [M, N]. */
 sq_status sq_gemm_s32(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, int64_t K,

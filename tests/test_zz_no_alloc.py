@@ -1,0 +1,113 @@
+"""sq_linear_w8a8_noalloc against sq_linear_w8a8 (GPU).
+
+sq_linear_w8a8_noalloc is the W8A8 linear for callers that cannot allocate
+device memory (a plugin that only receives its input and output buffers from
+a host engine, or a serving loop that must not pay cudaMalloc's device-wide
+synchronisation).  It takes no workspace: its small-M split-K path keeps the
+partial sums in a fixed array inside the library.  This file checks, through
+the C ABI, that it returns exactly what the workspace-taking entry point
+returns, on two calls in a row (the second call finds the first call's
+leftovers in the shared array), and that oversize requests are refused
+before any launch.  It is named so that pytest collects it last.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+sq = pytest.importorskip("w8a8_post_quantization_calib_b200")
+
+_OUT = {0: torch.float32, 1: torch.float16, 2: torch.bfloat16}
+
+
+def _operands(M, N, K, mode, out_dt, seed):
+    g = np.random.default_rng(seed)
+    xq = torch.from_numpy(g.integers(-127, 128, (M, K), dtype=np.int8)).cuda()
+    wq = torch.from_numpy(g.integers(-127, 128, (N, K), dtype=np.int8)).cuda()
+    a = torch.from_numpy((np.abs(g.standard_normal(1 if mode == 0 else M)) * 1e-2 + 1e-3).astype(np.float32)).cuda()
+    ws = torch.from_numpy((np.abs(g.standard_normal(N)) * 1e-4 + 1e-5).astype(np.float32)).cuda()
+    bias = torch.from_numpy(g.standard_normal(N).astype(np.float32)).cuda().to(_OUT[out_dt])
+    return xq, wq, a, ws, bias
+
+
+def _call_noalloc(xq, wq, a, mode, ws, bias, y):
+    M, K = xq.shape
+    N = wq.shape[0]
+    stream = torch.cuda.current_stream().cuda_stream
+    return sq.lib().sq_linear_w8a8_noalloc(
+        xq.data_ptr(), wq.data_ptr(), M, N, K, a.data_ptr(), mode, ws.data_ptr(),
+        bias.data_ptr() if bias is not None else None, {torch.float32: 0, torch.float16: 1,
+                                                        torch.bfloat16: 2}[y.dtype],
+        y.data_ptr(), stream)
+
+
+def _call_with_workspace(xq, wq, a, mode, ws, bias, y):
+    M, K = xq.shape
+    N = wq.shape[0]
+    n = sq.lib().sq_linear_workspace_size(M, N, K)
+    work = torch.zeros(max(n, 16), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    st = sq.lib().sq_linear_w8a8(
+        xq.data_ptr(), wq.data_ptr(), M, N, K, a.data_ptr(), mode, ws.data_ptr(),
+        bias.data_ptr() if bias is not None else None, {torch.float32: 0, torch.float16: 1,
+                                                        torch.bfloat16: 2}[y.dtype],
+        y.data_ptr(), work.data_ptr(), n, stream)
+    return st
+
+
+@pytest.mark.parametrize("M,N,K,mode,out_dt,with_bias", [
+    (16, 4096, 11008, 1, 2, False),     # decode-size down projection: split-K over the fixed array
+    (1, 11008, 4096, 1, 2, True),
+    (64, 2048, 1024, 0, 1, True),
+    (128, 1024, 4096, 0, 0, False),
+    (300, 528, 1040, 1, 1, True),       # large M: no scratch needed
+])
+def test_noalloc_matches_workspace_entry_point(M, N, K, mode, out_dt, with_bias):
+    xq, wq, a, ws, bias = _operands(M, N, K, mode, out_dt, M * 31 + N)
+    bias = bias if with_bias else None
+    y_ref = torch.empty(M, N, dtype=_OUT[out_dt], device="cuda")
+    assert _call_with_workspace(xq, wq, a, mode, ws, bias, y_ref) == 0
+    for _ in range(2):                  # two calls in a row share the library's array
+        y = torch.full((M, N), float("nan"), dtype=_OUT[out_dt], device="cuda")
+        assert _call_noalloc(xq, wq, a, mode, ws, bias, y) == 0
+        assert sq.sync_status() == 0
+        # same kernel, same exact int32 sums, same epilogue: bit-identical
+        assert torch.equal(y.view(torch.uint8), y_ref.view(torch.uint8))
+
+
+def test_noalloc_back_to_back_different_shapes():
+    """A smaller call after a larger one must not see the larger call's leftovers."""
+    big = _operands(64, 8192, 4096, 1, 2, 1)
+    small = _operands(16, 1024, 4096, 1, 2, 2)
+    outs = []
+    for ops in (big, small, big):
+        xq, wq, a, ws, _ = ops
+        y_ref = torch.empty(xq.shape[0], wq.shape[0], dtype=torch.bfloat16, device="cuda")
+        assert _call_with_workspace(xq, wq, a, 1, ws, None, y_ref) == 0
+        y = torch.empty_like(y_ref)
+        assert _call_noalloc(xq, wq, a, 1, ws, None, y) == 0
+        outs.append((y, y_ref))
+    assert sq.sync_status() == 0
+    for y, y_ref in outs:
+        assert torch.equal(y.view(torch.int16), y_ref.view(torch.int16))
+
+
+def test_noalloc_rejects_oversize_without_launch():
+    cap = sq.lib().sq_linear_w8a8_noalloc_max_elems()
+    assert cap == 2 ** 21
+    M, K = 128, 64
+    N = (cap // M) + 16                 # M*N just above the fixed array
+    N -= N % 16
+    while M * N <= cap:
+        N += 16
+    xq = torch.zeros(M, K, dtype=torch.int8, device="cuda")
+    wq = torch.zeros(N, K, dtype=torch.int8, device="cuda")
+    a = torch.ones(1, dtype=torch.float32, device="cuda")
+    ws = torch.ones(N, dtype=torch.float32, device="cuda")
+    y = torch.full((M, N), 7.0, dtype=torch.float16, device="cuda")
+    assert _call_noalloc(xq, wq, a, 0, ws, None, y) == 2            # SQ_ERR_UNSUPPORTED
+    assert sq.sync_status() == 0
+    assert torch.all(y == 7.0)                                        # nothing was launched

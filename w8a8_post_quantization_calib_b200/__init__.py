@@ -35,6 +35,7 @@ EXPORTS = (
     "sq_status_string", "sq_last_cuda_error", "sq_set_wait_timeout_ns", "sq_sync_status",
     "sq_calib_absmax", "sq_smooth_scales", "sq_quant_weight", "sq_quant_weight_gateup",
     "sq_smooth_quant_act", "sq_rmsnorm_quant", "sq_linear_workspace_size", "sq_linear_w8a8",
+    "sq_linear_w8a8_noalloc", "sq_linear_w8a8_noalloc_max_elems",
     "sq_gemm_s32", "sq_linear_w8a8_gateup_silu", "sq_gemm_f16_ref", "sq_sse_f16",
     "sq_alpha_search_workspace_size", "sq_alpha_search",
 )
@@ -68,6 +69,8 @@ def _load() -> ctypes.CDLL:
         "sq_rmsnorm_quant": (I, [P, I, I64, I64, P, P, F, P, P, P, P]),
         "sq_linear_workspace_size": (SZ, [I64, I64, I64]),
         "sq_linear_w8a8": (I, [P, P, I64, I64, I64, P, I, P, P, I, P, P, SZ, P]),
+        "sq_linear_w8a8_noalloc": (I, [P, P, I64, I64, I64, P, I, P, P, I, P, P]),
+        "sq_linear_w8a8_noalloc_max_elems": (SZ, []),
         "sq_gemm_s32": (I, [P, P, I64, I64, I64, P, P]),
         "sq_linear_w8a8_gateup_silu": (I, [P, P, I64, I64, I64, P, I, P, P, P, P, P, P]),
         "sq_gemm_f16_ref": (I, [P, P, I64, I64, I64, P, P]),
@@ -200,6 +203,20 @@ def linear_w8a8(xq, wq, a_scale, mode: int, w_scale, y, bias=None, workspace=Non
         _dev(a_scale, "a_scale", torch.float32), int(mode), _dev(w_scale, "w_scale", torch.float32),
         _dev(bias, "bias", y.dtype) if bias is not None else None, _dt(y), _dev(y, "y"),
         ws_ptr, ws_bytes, _stream(stream)))
+
+
+def linear_w8a8_noalloc(xq, wq, a_scale, mode: int, w_scale, y, bias=None, stream=None) -> None:
+    """linear_w8a8 without a workspace, for callers that cannot allocate device memory.
+
+    The small-M split-K path uses a fixed array inside the library instead
+    (calls on one device share it: do not overlap them on the GPU).
+    """
+    M, K = xq.shape
+    N = wq.shape[0]
+    _check("sq_linear_w8a8_noalloc", _lib.sq_linear_w8a8_noalloc(
+        _dev(xq, "xq", torch.int8), _dev(wq, "wq", torch.int8), M, N, K,
+        _dev(a_scale, "a_scale", torch.float32), int(mode), _dev(w_scale, "w_scale", torch.float32),
+        _dev(bias, "bias", y.dtype) if bias is not None else None, _dt(y), _dev(y, "y"), _stream(stream)))
 
 
 def gemm_s32(xq, wq, acc, stream=None) -> None:

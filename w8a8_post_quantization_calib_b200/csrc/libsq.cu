@@ -208,6 +208,45 @@ sq_status launch_rows(RowArgs a, int dt, cudaStream_t st)
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// Fixed device scratch for sq_linear_w8a8_noalloc.  Some callers cannot call
+// cudaMalloc at all: a plugin inside a host engine that owns every device
+// buffer and hands the plugin only its inputs and outputs, or a serving loop
+// that must never pay cudaMalloc's implicit device-wide synchronisation.  For
+// them the small-M split-K path keeps its int32 partial sums and per-tile
+// arrival counters in this file-scope array instead of a caller workspace.
+// Every GPU that loads the library holds it (8 MiB + 64 KiB) until exit.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocAccBytes = size_t(8) << 20;            // int32 partial sums
+constexpr size_t kNoAllocCntBytes = size_t(64) << 10;           // int32 tile counters
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocAccBytes + kNoAllocCntBytes];
+
+namespace {
+
+void *g_noalloc_ptr[kMaxDevices] = {nullptr};
+
+// Device address of g_noalloc_scratch for the current device.  In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+sq_status noalloc_scratch(void **out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= kMaxDevices) return SQ_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e);
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return SQ_OK;
+}
+
+}  // namespace
+
 // ============================================================================
 // C ABI
 // ============================================================================
@@ -423,6 +462,47 @@ sq_status sq_linear_w8a8(const int8_t *xq, const int8_t *wq, int64_t M, int64_t 
     }
     fill_tiles(p, 256, M, N);
     return launch_gemm<256, gemm::KIND_I8, gemm::EPI_DEQUANT, false>(p, xq, wq, st);
+}
+
+size_t sq_linear_w8a8_noalloc_max_elems(void) { return kNoAllocAccBytes / 4; }
+
+sq_status sq_linear_w8a8_noalloc(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, int64_t K,
+                                 const float *a_scale, sq_act_mode mode, const float *w_scale, const void *bias,
+                                 sq_dtype out_dt, void *y, sq_stream stream)
+{
+    sq_status r = check_gemm_shape(xq, wq, M, N, K);
+    if (r != SQ_OK) return r;
+    if (a_scale == nullptr || w_scale == nullptr || y == nullptr || !valid_dt(out_dt)) return SQ_ERR_INVALID_ARG;
+    if (mode != SQ_ACT_STATIC && mode != SQ_ACT_PER_TOKEN) return SQ_ERR_INVALID_ARG;
+    if (!aligned16(y) || !aligned16(w_scale)) return SQ_ERR_MISALIGNED;
+    if (M > kSwapMaxM)      // the large-M path needs no scratch: same launch as sq_linear_w8a8
+        return sq_linear_w8a8(xq, wq, M, N, K, a_scale, mode, w_scale, bias, out_dt, y, nullptr, 0, stream);
+    const size_t acc_bytes = static_cast<size_t>(M * N) * 4;
+    const size_t cnt_bytes = static_cast<size_t>(swap_tiles(M, N)) * 4;
+    if (acc_bytes > kNoAllocAccBytes || cnt_bytes > kNoAllocCntBytes) return SQ_ERR_UNSUPPORTED;
+    void *scratch = nullptr;
+    if ((r = noalloc_scratch(&scratch)) != SQ_OK) return r;
+    int32_t *acc = static_cast<int32_t *>(scratch);
+    int *cnt = reinterpret_cast<int *>(static_cast<unsigned char *>(scratch) + kNoAllocAccBytes);
+    const cudaStream_t st = as_stream(stream);
+    // the array keeps whatever the previous call left: zero the part this call uses
+    cudaError_t e = cudaMemsetAsync(acc, 0, acc_bytes, st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = cudaMemsetAsync(cnt, 0, cnt_bytes, st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    gemm::Params p{};
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(N);
+    p.K = static_cast<int>(K);
+    p.a_scale = a_scale;
+    p.per_token = (mode == SQ_ACT_PER_TOKEN) ? 1 : 0;
+    p.w_scale = w_scale;
+    p.bias = bias;
+    p.out = y;
+    p.out_dt = out_dt;
+    p.ws_acc = acc;
+    p.ws_cnt = cnt;
+    return dispatch_swap<gemm::EPI_DEQUANT>(p, xq, wq, st);
 }
 
 sq_status sq_gemm_s32(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, int64_t K, int32_t *acc,
