@@ -20,6 +20,13 @@ constexpr int CALIB_TX = 32;      // vectors per block strip
 constexpr int CALIB_TY = 8;       // row lanes per block
 constexpr int CALIB_UNROLL = 4;   // rows in flight per thread
 
+template <bool STREAM>
+__device__ __forceinline__ uint4 load16(const uint8_t *p)
+{
+    if constexpr (STREAM) return __ldcs(reinterpret_cast<const uint4 *>(p));
+    else return __ldg(reinterpret_cast<const uint4 *>(p));
+}
+
 template <int DT>
 struct AbsMaxAcc {
     static constexpr int EPV = VecT<DT>::EPV;
@@ -58,7 +65,10 @@ struct AbsMaxAcc {
     }
 };
 
-template <int DT>
+// STREAM: evict-first loads for tensors much larger than L2 (calibration
+// batches); otherwise normal loads, so that a tensor read again right after
+// (the weight: statistic, then transform) can still be found in L2.
+template <int DT, bool STREAM>
 __global__ void __launch_bounds__(CALIB_TX *CALIB_TY)
     k_colabsmax(const uint8_t *__restrict__ x, int64_t rows, int64_t nvec, int64_t ld_bytes,
                 int64_t row_slab, float *__restrict__ absmax)
@@ -80,11 +90,11 @@ __global__ void __launch_bounds__(CALIB_TX *CALIB_TY)
             uint4 t[CALIB_UNROLL];
 #pragma unroll
             for (int u = 0; u < CALIB_UNROLL; ++u)
-                t[u] = __ldcs(reinterpret_cast<const uint4 *>(col + (r + u * CALIB_TY) * ld_bytes));
+                t[u] = load16<STREAM>(col + (r + u * CALIB_TY) * ld_bytes);
 #pragma unroll
             for (int u = 0; u < CALIB_UNROLL; ++u) acc.add(t[u]);
         }
-        for (; r < r1; r += CALIB_TY) acc.add(__ldcs(reinterpret_cast<const uint4 *>(col + r * ld_bytes)));
+        for (; r < r1; r += CALIB_TY) acc.add(load16<STREAM>(col + r * ld_bytes));
     }
     float f[EPV];
     acc.to_float(f);

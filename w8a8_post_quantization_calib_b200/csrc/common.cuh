@@ -37,6 +37,23 @@ __device__ __forceinline__ int quant8(float v)
     return min(max(r, -127), 127);
 }
 
+// The same code as quant8, computed on the FMA/ALU pipes: clamp in fp32, then
+// add 1.5 * 2^23 so that the fp32 add itself rounds half to even to an
+// integer; the low byte of the sum's bit pattern is the two's-complement
+// code.  Clamping first gives the same result as rounding first (both ends of
+// [-127, 127] are integers), for every non-NaN v.
+__device__ __forceinline__ uint32_t quant8_bits(float v)
+{
+    const float c = fminf(fmaxf(v, -127.0f), 127.0f);
+    return __float_as_uint(__fadd_rn(c, 12582912.0f));
+}
+
+// low bytes of four quant8_bits results -> one packed word (byte 0 = a)
+__device__ __forceinline__ uint32_t pack4_bits(uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
 __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d)
 {
     return (uint32_t)(a & 0xff) | ((uint32_t)(b & 0xff) << 8) | ((uint32_t)(c & 0xff) << 16) |

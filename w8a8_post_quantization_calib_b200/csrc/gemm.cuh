@@ -44,6 +44,7 @@ constexpr int BKB = 128;           // bytes of K per stage (one swizzle row)
 constexpr int NUM_THREADS = 192;
 constexpr int GROUP_R = 16;        // raster group along A-row tiles (L2 reuse of B)
 constexpr int SMEM_BUDGET = 200 * 1024;
+constexpr int STG_BYTES = 4096;    // one epilogue staging buffer: 32 rows x up to 128 bytes
 
 // error codes recorded on a barrier timeout: 0x100 | role << 4 | where
 constexpr unsigned ERR_PRODUCER = 0x110, ERR_MMA = 0x120, ERR_EPI = 0x130, ERR_DRAIN = 0x140;
@@ -494,6 +495,321 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         __syncwarp();
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Epilogue of one 128-row accumulator with coalesced output: each warp packs
+// its 32 rows x 32 columns into a shared-memory staging buffer in the
+// tensor map's swizzled layout (64-byte rows for 16-bit outputs, 128-byte rows
+// for 32-bit ones) and one lane issues an asynchronous TMA store of the
+// 32 x 32 box; rows >= M and columns >= N of a box are not written.  Two
+// buffers per warp: a buffer is reused only after the store issued from it
+// two boxes earlier has finished reading shared memory.
+// ---------------------------------------------------------------------------
+template <int BN, int KIND, int EPI>
+__device__ __forceinline__ void epilogue_tma(const Params &p, const CUtensorMap *omap, uint32_t tbase, int tr,
+                                             int tc, int q, int lane, uint32_t stg, int &nstore,
+                                             const float *ws_tile, const float *bias_tile, float am)
+{
+    const int mrow0 = tr * BM + q * 32;
+    const bool wide = (EPI == EPI_S32) || (EPI == EPI_DEQUANT && p.out_dt == DT_F32);   // 4-byte outputs
+
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        ptx::tmem_ld32(tbase + c * 32, r);
+        ptx::tmem_ld_wait();
+        const int n0 = tc * BN + c * 32;
+        if (n0 >= p.N) continue;
+        const int nval = min(32, p.N - n0);
+        uint32_t w[32];                       // packed output words of this row's 32 columns
+        if constexpr (EPI == EPI_S32) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) w[i] = r[i];
+        } else {
+            float v[32];
+            if constexpr (EPI == EPI_F16) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; i += 4) {
+                    const float4 w4 = *reinterpret_cast<const float4 *>(ws_tile + c * 32 + i);     // broadcast
+                    const float4 b4 = *reinterpret_cast<const float4 *>(bias_tile + c * 32 + i);
+                    const float ws[4] = {w4.x, w4.y, w4.z, w4.w};
+                    const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+                    for (int t = 0; t < 4; ++t)
+                        v[i + t] = dequant(static_cast<int32_t>(r[i + t]), __fmul_rn(am, ws[t]), p.bias, bb[t]);
+                }
+            }
+            const int odt = (EPI == EPI_F16) ? DT_F16 : p.out_dt;
+            if (odt == DT_F32) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(v[i]);
+            } else if (odt == DT_F16) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    __half2 h = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
+                    w[i] = *reinterpret_cast<uint32_t *>(&h);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+                    w[i] = *reinterpret_cast<uint32_t *>(&h);
+                }
+            }
+        }
+        if (lane == 0 && nstore >= 2) ptx::bulk_wait_read_1();
+        __syncwarp();
+        const uint32_t buf = stg + static_cast<uint32_t>(nstore & 1) * STG_BYTES;
+        if (wide) {                           // 128-byte rows, 128-byte swizzle: chunk ^= row & 7
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const uint32_t a = buf + lane * 128 + ((k ^ (lane & 7)) << 4);
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(w[4 * k]), "r"(w[4 * k + 1]),
+                             "r"(w[4 * k + 2]), "r"(w[4 * k + 3])
+                             : "memory");
+            }
+        } else {                              // 64-byte rows, 64-byte swizzle: chunk ^= (row >> 1) & 3
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint32_t a = buf + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4);
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(w[4 * k]), "r"(w[4 * k + 1]),
+                             "r"(w[4 * k + 2]), "r"(w[4 * k + 3])
+                             : "memory");
+            }
+        }
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            ptx::tma_store_2d(omap, buf, n0, mrow0);
+            ptx::bulk_commit();
+        }
+        ++nstore;
+    }
+}
+
+// ===========================================================================
+// CTA-pair variant (cta_group::2): a cluster of two CTAs on two SMs computes a
+// 256 x BN tile.  Each CTA loads its own 128 rows of A and BN/2 rows of B
+// (32 KB per stage at BN = 256, so 6 stages fit), the leader CTA (rank 0)
+// issues tcgen05.mma.cta_group::2 (M = 256) that reads both CTAs' shared
+// memory and writes a 128 x BN int32 accumulator into each CTA's TMEM.  Half
+// the operand bytes per MAC of the single-CTA tile.
+//
+// Barriers: full[s] lives in the leader (its producer posts the transaction
+// bytes of both halves; both CTAs' TMA loads complete on it); empty[s] and
+// tfull[b] live in both CTAs and receive multicast tcgen05.commit arrivals
+// from the leader's MMA thread; tempty[b] lives in the leader and collects
+// one arrival per epilogue warp of both CTAs (8).
+// ===========================================================================
+template <int BN>
+struct PairCfg {
+    static constexpr int A_BYTES = BM * BKB;              // this CTA's 128 rows of A
+    static constexpr int B_BYTES = (BN / 2) * BKB;        // this CTA's BN/2 rows of B
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int STAGES_RAW = (188 * 1024) / STAGE_BYTES;
+    static constexpr int STAGES = STAGES_RAW > 10 ? 10 : STAGES_RAW;
+    static constexpr int TMEM_COLS = pow2_at_least(2 * BN, 32);
+    static constexpr int STG_TOTAL = 4 * 2 * STG_BYTES;   // 4 epilogue warps x 2 buffers
+    static constexpr int COLS_BYTES = 2 * 2 * 256 * 4;    // per accumulator buffer: w_scale + bias, 256 each
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STG_TOTAL + COLS_BYTES + 256;
+    static_assert(STAGE_BYTES % 1024 == 0, "stage must keep 1024-byte alignment");
+    static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "pair MMA N");
+    static_assert(TMEM_COLS <= 512, "two accumulators must fit TMEM");
+};
+
+template <int BN, int KIND, int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+    k_gemm2(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+            const __grid_constant__ CUtensorMap map_o, const Params p)
+{
+    using C = PairCfg<BN>;
+    constexpr int S = C::STAGES;
+    constexpr int BKE = (KIND == KIND_I8) ? BKB : BKB / 2;
+    constexpr uint32_t IDESC = (KIND == KIND_I8) ? ptx::idesc_i8_m256(BN) : ptx::idesc_f16_m256(BN);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + S * C::STAGE_BYTES + C::STG_TOTAL + C::COLS_BYTES);
+    const uint32_t bar0 = ptx::smem_addr(bars);
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
+    auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * S + b); };
+    auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * S + 2 + b); };
+    const uint32_t done_bar = bar0 + 8u * (2 * S + 4);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 5);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    volatile int *ok_flag = reinterpret_cast<volatile int *>(tmem_slot + 2);     // [2]
+    const uint32_t sbase = ptx::smem_addr(smem);
+    const uint32_t stg_base = sbase + S * C::STAGE_BYTES;      // 1024-aligned staging buffers
+    float *cols = reinterpret_cast<float *>(smem + S * C::STAGE_BYTES + C::STG_TOTAL);   // [2][w_scale 256 | bias 256]
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = ptx::cluster_ctarank();
+    const bool leader = (rank == 0);
+    const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            ptx::mbar_init(full_bar(s), 1);
+            ptx::mbar_init(empty_bar(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(tfull_bar(b), 1);
+            ptx::mbar_init(tempty_bar(b), 8);
+        }
+        ptx::mbar_init(done_bar, 1);
+        *abort_flag = 0;
+        ptx::fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        ptx::tma_prefetch_desc(&map_a);
+        ptx::tma_prefetch_desc(&map_b);
+        if constexpr (EPI != EPI_GATEUP) ptx::tma_prefetch_desc(&map_o);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc_pair(ptx::smem_addr(tmem_slot), C::TMEM_COLS);
+        ptx::tmem_relinquish_pair();
+    }
+    ptx::tc_fence_before();
+    ptx::cluster_sync();               // both CTAs' barriers exist before any remote use
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const uint64_t tmo = p.timeout_ns;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer (both CTAs)
+        if (lane == 0) {
+            int stage = 0, issued = 0;
+            uint32_t phase = 0;
+            for (int u = cluster; u < p.num_units && !*abort_flag; u += nclusters) {
+                int tr, tc, split, tile;
+                decode_unit(p, u, tr, tc, split, tile);
+                bool ok = true;
+                for (int kb = 0; kb < p.num_kb; ++kb) {
+                    if (!ptx::wait_bounded(empty_bar(stage), phase ^ 1u, tmo, abort_flag, ERR_PRODUCER)) {
+                        ok = false;
+                        break;
+                    }
+                    if (leader) ptx::mbar_arrive_expect_tx(full_bar(stage), 2 * C::STAGE_BYTES);
+                    const uint32_t fb = ptx::map_to_rank(full_bar(stage), 0);
+                    const uint32_t sa = sbase + stage * C::STAGE_BYTES;
+                    ptx::tma_load_2d_pair(sa, &map_a, fb, kb * BKE, tr * (2 * BM) + static_cast<int>(rank) * BM);
+                    ptx::tma_load_2d_pair(sa + C::A_BYTES, &map_b, fb, kb * BKE,
+                                          tc * BN + static_cast<int>(rank) * (BN / 2));
+                    ++issued;
+                    if (++stage == S) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+            }
+            // drain: the leader's full barriers count both CTAs' bytes
+            if (leader) {
+                const int n_wait = issued < S ? issued : S;
+                for (int i = 0; i < n_wait; ++i) {
+                    int s = stage - 1 - i;
+                    uint32_t ph = phase;
+                    if (s < 0) { s += S; ph ^= 1u; }
+                    volatile int no_abort = 0;
+                    ptx::wait_bounded(full_bar(s), ph, tmo, &no_abort, ERR_DRAIN);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer (leader only)
+        if (lane == 0 && leader) {
+            int stage = 0, local = 0;
+            uint32_t phase = 0;
+            for (int u = cluster; u < p.num_units; u += nclusters, ++local) {
+                const int b = local & 1;
+                const uint32_t use = static_cast<uint32_t>(local >> 1) & 1u;
+                if (!ptx::wait_bounded(tempty_bar(b), use ^ 1u, tmo, abort_flag, ERR_MMA)) break;
+                ptx::tc_fence_after();
+                const uint32_t d = tmem_base + static_cast<uint32_t>(b * BN);
+                bool ok = true;
+                for (int kb = 0; kb < p.num_kb; ++kb) {
+                    if (!ptx::wait_bounded(full_bar(stage), phase, tmo, abort_flag, ERR_MMA + 1)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint32_t sa = sbase + stage * C::STAGE_BYTES;
+                    const uint64_t ad = ptx::sdesc_kmajor_sw128(sa);
+                    const uint64_t bd = ptx::sdesc_kmajor_sw128(sa + C::A_BYTES);
+#pragma unroll
+                    for (int k = 0; k < BKB / 32; ++k) {
+                        const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
+                        if constexpr (KIND == KIND_I8)
+                            ptx::mma_i8_pair(d, ad + 2 * k, bd + 2 * k, IDESC, acc);
+                        else
+                            ptx::mma_f16_pair(d, ad + 2 * k, bd + 2 * k, IDESC, acc);
+                    }
+                    ptx::tc_commit_pair_mc(empty_bar(stage), 0x3);
+                    if (++stage == S) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                ptx::tc_commit_pair_mc(tfull_bar(b), 0x3);
+            }
+            ptx::tc_commit_pair(done_bar);
+            volatile int no_abort = 0;
+            ptx::wait_bounded(done_bar, 0u, tmo, &no_abort, ERR_DRAIN + 1);
+        }
+    } else {
+        // ------------------------------------------------ epilogue (warps 2..5, both CTAs)
+        const int q = warp & 3;
+        const uint32_t stg = stg_base + static_cast<uint32_t>((warp - 2) * 2 * STG_BYTES);
+        int nstore = 0;
+        int local = 0;
+        for (int u = cluster; u < p.num_units; u += nclusters, ++local) {
+            int tr, tc, split, tile;
+            decode_unit(p, u, tr, tc, split, tile);
+            const int b = local & 1;
+            const uint32_t use = static_cast<uint32_t>(local >> 1) & 1u;
+            // while the MMAs of this tile run: stage its per-column scales / bias
+            // and fetch this thread's row scale
+            float *ws_tile = cols + b * 512;
+            float *bias_tile = ws_tile + 256;
+            float am = 0.0f;
+            if constexpr (EPI == EPI_DEQUANT) {
+                const int et = threadIdx.x - 64;             // 0..127
+                for (int t = et; t < BN; t += 128) {
+                    const int n = tc * BN + t;
+                    ws_tile[t] = n < p.N ? p.w_scale[n] : 0.0f;
+                    bias_tile[t] = (n < p.N && p.bias != nullptr) ? load_bias(p.bias, p.out_dt, n) : 0.0f;
+                }
+                const int m = (2 * tr + static_cast<int>(rank)) * BM + q * 32 + lane;
+                if (m < p.M) am = p.per_token ? p.a_scale[m] : p.a_scale[0];
+            }
+            // one thread waits for the accumulator; the 128 epilogue threads
+            // then take the same decision (no warp is left at a barrier alone)
+            if (threadIdx.x == 64) ok_flag[b] = ptx::wait_bounded(tfull_bar(b), use, tmo, abort_flag, ERR_EPI) ? 1 : 0;
+            ptx::named_bar_sync(1, 128);
+            if (!ok_flag[b]) break;
+            ptx::tc_fence_after();
+            const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * BN);
+            // this CTA's accumulator rows are the tile's rows rank*128 .. rank*128+127
+            if constexpr (EPI == EPI_GATEUP)
+                epilogue_normal<BN, KIND, EPI>(p, tbase, 2 * tr + static_cast<int>(rank), tc, q, lane);
+            else
+                epilogue_tma<BN, KIND, EPI>(p, &map_o, tbase, 2 * tr + static_cast<int>(rank), tc, q, lane, stg,
+                                            nstore, ws_tile, bias_tile, am);
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive_cluster(ptx::map_to_rank(tempty_bar(b), 0));
+        }
+        if (lane == 0) ptx::bulk_wait_all();     // output stores complete before the CTA exits
+        __syncwarp();
+    }
+
+    ptx::tc_fence_before();
+    ptx::cluster_sync();               // no CTA leaves while its peer may still signal it
+    if (warp == 1) {
+        __syncwarp();
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
     }
 }
 

@@ -111,6 +111,110 @@ sq_status launch_gemm(gemm::Params p, const void *a, const void *b, cudaStream_t
     return check_launch();
 }
 
+// CTA-pair launch: grid = 2 x (co-resident clusters, at most one per unit).
+// Output map for the epilogue's TMA stores: [M, N] row-major, 32 x 32 boxes,
+// swizzle matching the staging layout (64-byte rows for 2-byte elements,
+// 128-byte rows for 4-byte ones).
+bool make_out_map(CUtensorMap *m, void *base, int out_dt, bool s32, int64_t M, int64_t N)
+{
+    auto fn = encode_fn();
+    if (fn == nullptr) return false;
+    CUtensorMapDataType t;
+    int elt;
+    if (s32) { t = CU_TENSOR_MAP_DATA_TYPE_INT32; elt = 4; }
+    else if (out_dt == SQ_F32) { t = CU_TENSOR_MAP_DATA_TYPE_FLOAT32; elt = 4; }
+    else if (out_dt == SQ_F16) { t = CU_TENSOR_MAP_DATA_TYPE_FLOAT16; elt = 2; }
+    else { t = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16; elt = 2; }
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(N * elt)};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(m, t, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          elt == 4 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                          CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int BN, int KIND, int EPI>
+sq_status launch_gemm2(gemm::Params p, const void *a, const void *b, cudaStream_t st)
+{
+    using C = gemm::PairCfg<BN>;
+    const bool f16 = (KIND == gemm::KIND_F16);
+    CUtensorMap ma, mb, mo;
+    if (!make_map(&ma, a, f16, p.K, p.rows_a, gemm::BM)) return SQ_ERR_CUDA;
+    if (!make_map(&mb, b, f16, p.K, p.rows_b, BN / 2)) return SQ_ERR_CUDA;
+    if constexpr (EPI == gemm::EPI_GATEUP) {
+        std::memset(&mo, 0, sizeof(mo));
+    } else {
+        const int odt = (EPI == gemm::EPI_F16) ? SQ_F16 : p.out_dt;
+        if (!make_out_map(&mo, p.out, odt, EPI == gemm::EPI_S32, p.M, p.N)) return SQ_ERR_CUDA;
+    }
+    auto kern = gemm::k_gemm2<BN, KIND, EPI>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return cuda_fail(e);
+    static int max_clusters[kMaxDevices] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= kMaxDevices) dev = 0;
+    if (max_clusters[dev] == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * (sm_count() / 2), 1, 1);
+        cfg.blockDim = dim3(gemm::NUM_THREADS, 1, 1);
+        cfg.dynamicSmemBytes = C::SMEM_BYTES;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void *>(kern), &cfg) != cudaSuccess || n <= 0)
+            n = sm_count() / 2;
+        cudaGetLastError();
+        max_clusters[dev] = n;
+    }
+    p.timeout_ns = g_timeout_ns;
+    const int clusters = static_cast<int>(std::min<int64_t>(p.num_units, max_clusters[dev]));
+    kern<<<2 * clusters, gemm::NUM_THREADS, C::SMEM_BYTES, st>>>(ma, mb, mo, p);
+    return check_launch();
+}
+
+void fill_tiles_pair(gemm::Params &p, int bn, int kb_bytes_per_elem)
+{
+    p.rows_a = p.M;
+    p.rows_b = p.N;
+    p.num_kb = static_cast<int>(cdiv(static_cast<int64_t>(p.K) * kb_bytes_per_elem, 128));
+    p.tiles_r = static_cast<int>(cdiv(p.M, 2 * gemm::BM));
+    p.tiles_c = static_cast<int>(cdiv(p.N, bn));
+    p.splits = 1;
+    p.kb_per_split = p.num_kb;
+    p.num_units = p.tiles_r * p.tiles_c;
+}
+
+// Pair-tile width with the fewest waves x tile width (ties to the wider tile).
+int pick_pair_bn(int64_t M, int64_t N)
+{
+    const int64_t clusters = std::max(1, sm_count() / 2);
+    const int cands[3] = {256, 192, 128};
+    int best = 256;
+    int64_t best_cost = -1;
+    for (int bn : cands) {
+        const int64_t tiles = cdiv(M, 2 * gemm::BM) * cdiv(N, bn);
+        const int64_t cost = cdiv(tiles, clusters) * bn;
+        if (best_cost < 0 || cost < best_cost) {
+            best = bn;
+            best_cost = cost;
+        }
+    }
+    return best;
+}
+
+template <int KIND, int EPI>
+sq_status dispatch_pair(gemm::Params &p, const void *a, const void *b, cudaStream_t st, int force_bn = 0)
+{
+    const int bn = force_bn ? force_bn : pick_pair_bn(p.M, p.N);
+    fill_tiles_pair(p, bn, KIND == gemm::KIND_F16 ? 2 : 1);
+    switch (bn) {
+    case 256: return launch_gemm2<256, KIND, EPI>(p, a, b, st);
+    case 192: return launch_gemm2<192, KIND, EPI>(p, a, b, st);
+    default: return launch_gemm2<128, KIND, EPI>(p, a, b, st);
+    }
+}
+
 void fill_tiles(gemm::Params &p, int bn, int64_t rows_a, int64_t rows_b)
 {
     p.rows_a = static_cast<int>(rows_a);
@@ -174,7 +278,8 @@ sq_status launch_rows_dt(RowArgs a, cudaStream_t st)
                      (a.K % EPV) == 0;
     const int64_t nvec = a.K / EPV;
     const int64_t vpt = cdiv(nvec, ROW_T);
-    const size_t smem = static_cast<size_t>(a.K) * 4;
+    // per-column constants in registers when VPT * EPV <= 32, else in shared memory
+    const size_t smem = (vpt * EPV <= 32) ? 0 : static_cast<size_t>(a.K) * 4;
     const int sms = sm_count();
     if (vec && vpt <= 16 && smem <= 160 * 1024) {
         void (*kern)(RowArgs) = nullptr;
@@ -183,8 +288,11 @@ sq_status launch_rows_dt(RowArgs a, cudaStream_t st)
         else if (vpt <= 4) kern = k_rows<DT, 4, MODE>;
         else if (vpt <= 8) kern = k_rows<DT, 8, MODE>;
         else kern = k_rows<DT, 16, MODE>;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-        if (e != cudaSuccess) return cuda_fail(e);
+        cudaError_t e = cudaSuccess;
+        if (smem > 48 * 1024) {
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+            if (e != cudaSuccess) return cuda_fail(e);
+        }
         int per_sm = 0;
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, ROW_T, smem);
         if (e != cudaSuccess) return cuda_fail(e);
@@ -306,9 +414,16 @@ sq_status sq_calib_absmax(const void *x, sq_dtype dt, int64_t rows, int64_t cols
         dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), block(CALIB_TX, CALIB_TY);
         const uint8_t *xb = static_cast<const uint8_t *>(x);
         const int64_t ldb = ld * elt;
-        if (dt == SQ_F32) k_colabsmax<DT_F32><<<grid, block, 0, st>>>(xb, rows, nvec, ldb, slab, absmax);
-        else if (dt == SQ_F16) k_colabsmax<DT_F16><<<grid, block, 0, st>>>(xb, rows, nvec, ldb, slab, absmax);
-        else k_colabsmax<DT_BF16><<<grid, block, 0, st>>>(xb, rows, nvec, ldb, slab, absmax);
+        const bool stream_hint = rows * ldb > (int64_t(100) << 20);     // much larger than L2 share
+        if (stream_hint) {
+            if (dt == SQ_F32) k_colabsmax<DT_F32, true><<<grid, block, 0, st>>>(xb, rows, nvec, ldb, slab, absmax);
+            else if (dt == SQ_F16) k_colabsmax<DT_F16, true><<<grid, block, 0, st>>>(xb, rows, nvec, ldb, slab, absmax);
+            else k_colabsmax<DT_BF16, true><<<grid, block, 0, st>>>(xb, rows, nvec, ldb, slab, absmax);
+        } else {
+            if (dt == SQ_F32) k_colabsmax<DT_F32, false><<<grid, block, 0, st>>>(xb, rows, nvec, ldb, slab, absmax);
+            else if (dt == SQ_F16) k_colabsmax<DT_F16, false><<<grid, block, 0, st>>>(xb, rows, nvec, ldb, slab, absmax);
+            else k_colabsmax<DT_BF16, false><<<grid, block, 0, st>>>(xb, rows, nvec, ldb, slab, absmax);
+        }
     } else {
         const int64_t gx = cdiv(cols, 256);
         int64_t gy = std::max<int64_t>(1, std::min<int64_t>(cdiv(rows, 64), cdiv(static_cast<int64_t>(sms) * 8, gx)));
@@ -327,12 +442,17 @@ sq_status sq_smooth_scales(const float *act_max, const float *w_max, int64_t K, 
     if (act_max == nullptr || w_max == nullptr || s == nullptr || K <= 0) return SQ_ERR_INVALID_ARG;
     if (!(alpha >= 0.0f && alpha <= 1.0f)) return SQ_ERR_INVALID_ARG;
     const cudaStream_t st = as_stream(stream);
+    if (K <= 256) {         // one block writes the static scale itself
+        k_smooth_scales<<<1, 256, 0, st>>>(act_max, w_max, K, alpha, s, a_static);
+        return check_launch();
+    }
     if (a_static != nullptr) {
         const cudaError_t e = cudaMemsetAsync(a_static, 0, sizeof(float), st);
         if (e != cudaSuccess) return cuda_fail(e);
     }
-    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(cdiv(K, 256), static_cast<int64_t>(sm_count()) * 4));
-    k_smooth_scales<<<static_cast<unsigned>(grid), 256, 0, st>>>(act_max, w_max, K, alpha, s, a_static);
+    // one channel per thread: the fp64 log2/exp2 chain is latency-bound
+    const int64_t grid = std::max<int64_t>(2, cdiv(K, 128));
+    k_smooth_scales<<<static_cast<unsigned>(grid), 128, 0, st>>>(act_max, w_max, K, alpha, s, a_static);
     return check_launch();
 }
 
@@ -460,8 +580,7 @@ sq_status sq_linear_w8a8(const int8_t *xq, const int8_t *wq, int64_t M, int64_t 
         }
         return dispatch_swap<gemm::EPI_DEQUANT>(p, xq, wq, st);
     }
-    fill_tiles(p, 256, M, N);
-    return launch_gemm<256, gemm::KIND_I8, gemm::EPI_DEQUANT, false>(p, xq, wq, st);
+    return dispatch_pair<gemm::KIND_I8, gemm::EPI_DEQUANT>(p, xq, wq, st);
 }
 
 size_t sq_linear_w8a8_noalloc_max_elems(void) { return kNoAllocAccBytes / 4; }
@@ -519,8 +638,7 @@ sq_status sq_gemm_s32(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, 
     p.K = static_cast<int>(K);
     p.out = acc;
     if (M <= kSwapMaxM) return dispatch_swap<gemm::EPI_S32>(p, xq, wq, st);
-    fill_tiles(p, 256, M, N);
-    return launch_gemm<256, gemm::KIND_I8, gemm::EPI_S32, false>(p, xq, wq, st);
+    return dispatch_pair<gemm::KIND_I8, gemm::EPI_S32>(p, xq, wq, st);
 }
 
 sq_status sq_linear_w8a8_gateup_silu(const int8_t *xq, const int8_t *wq_gu, int64_t M, int64_t N_h, int64_t K,
@@ -546,8 +664,7 @@ sq_status sq_linear_w8a8_gateup_silu(const int8_t *xq, const int8_t *wq_gu, int6
     p.s2 = s2;
     p.a2 = a2;
     p.hq = hq;
-    fill_tiles(p, 256, M, 2 * N_h);
-    return launch_gemm<256, gemm::KIND_I8, gemm::EPI_GATEUP, false>(p, xq, wq_gu, as_stream(stream));
+    return dispatch_pair<gemm::KIND_I8, gemm::EPI_GATEUP>(p, xq, wq_gu, as_stream(stream), 256);
 }
 
 sq_status sq_gemm_f16_ref(const void *x, const void *w, int64_t M, int64_t N, int64_t K, void *y, sq_stream stream)
@@ -561,10 +678,7 @@ sq_status sq_gemm_f16_ref(const void *x, const void *w, int64_t M, int64_t N, in
     p.K = static_cast<int>(K);
     p.out = y;
     p.out_dt = SQ_F16;
-    fill_tiles(p, 256, M, N);
-    p.num_kb = static_cast<int>(cdiv(K, 64));   // 64 fp16 per 128-byte K block
-    p.kb_per_split = p.num_kb;
-    return launch_gemm<256, gemm::KIND_F16, gemm::EPI_F16, false>(p, x, w, as_stream(stream));
+    return dispatch_pair<gemm::KIND_F16, gemm::EPI_F16>(p, x, w, as_stream(stream), 256);
 }
 
 sq_status sq_sse_f16(const void *y, const void *y_ref, int64_t n, double *sse, sq_stream stream)

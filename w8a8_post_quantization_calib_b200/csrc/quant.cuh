@@ -24,8 +24,9 @@ namespace sq {
 // form of "010. SmoothQuant Integration" key design point 1.  x -> fl(x/127)
 // is monotone, so max_b fl(m_b/127) = fl(max_b m_b / 127): blocks combine
 // with atomicMax on the (non-negative) float bits; *a_static is zeroed first.
+// A single-block launch (small K) writes the scale directly.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(1024)
     k_smooth_scales(const float *__restrict__ act_max, const float *__restrict__ w_max, int64_t K,
                     float alpha, float *__restrict__ s, float *__restrict__ a_static)
 {
@@ -36,13 +37,18 @@ __global__ void __launch_bounds__(256)
          j += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const double a = fmax(static_cast<double>(act_max[j]), 1e-5);
         const double w = fmax(static_cast<double>(w_max[j]), 1e-5);
-        const float sj = static_cast<float>(pow(a, al) / pow(w, 1.0 - al));
+        // a^alpha / w^(1-alpha) = 2^(alpha log2 a - (1-alpha) log2 w): fp64 log2/exp2
+        // carry ~1e-15 relative error, far below the one fp32 rounding that follows
+        const float sj = static_cast<float>(exp2(al * log2(a) - (1.0 - al) * log2(w)));
         s[j] = sj;
         m = fmaxf(m, __fmul_rn(act_max[j], recip_or_zero(sj)));
     }
     if (a_static != nullptr) {
         m = block_max(m, red);
-        if (threadIdx.x == 0) atomicMax(reinterpret_cast<int *>(a_static), __float_as_int(scale_from_absmax(m)));
+        if (threadIdx.x == 0) {
+            if (gridDim.x == 1) *a_static = scale_from_absmax(m);      // one block: no pre-zeroing needed
+            else atomicMax(reinterpret_cast<int *>(a_static), __float_as_int(scale_from_absmax(m)));
+        }
     }
 }
 
@@ -73,123 +79,200 @@ struct RowArgs {
     int8_t *out;             // codes [rows, K]
 };
 
-template <int DT>
-__device__ __forceinline__ void store_codes(int8_t *dst_row, int64_t v, const float (&f)[VecT<DT>::EPV])
+// Codes of EPV values (already multiplied by the scale reciprocal) -> global.
+template <int EPV>
+__device__ __forceinline__ void store_codes(int8_t *dst_row, int64_t v, const float *f)
 {
-    constexpr int EPV = VecT<DT>::EPV;
     if constexpr (EPV == 8) {
         uint2 o;
-        o.x = pack4(quant8(f[0]), quant8(f[1]), quant8(f[2]), quant8(f[3]));
-        o.y = pack4(quant8(f[4]), quant8(f[5]), quant8(f[6]), quant8(f[7]));
+        o.x = pack4_bits(quant8_bits(f[0]), quant8_bits(f[1]), quant8_bits(f[2]), quant8_bits(f[3]));
+        o.y = pack4_bits(quant8_bits(f[4]), quant8_bits(f[5]), quant8_bits(f[6]), quant8_bits(f[7]));
         *reinterpret_cast<uint2 *>(dst_row + v * 8) = o;
     } else {
         *reinterpret_cast<uint32_t *>(dst_row + v * 4) =
-            pack4(quant8(f[0]), quant8(f[1]), quant8(f[2]), quant8(f[3]));
+            pack4_bits(quant8_bits(f[0]), quant8_bits(f[1]), quant8_bits(f[2]), quant8_bits(f[3]));
     }
 }
 
+template <int MODE>
+__device__ __forceinline__ float column_constant(const RowArgs &p, int64_t j)
+{
+    if constexpr (MODE == ROW_WEIGHT) return p.s[j];
+    else if constexpr (MODE == ROW_RMSNORM) return __fmul_rn(p.gamma[j], recip_or_zero(p.s[j]));
+    else return recip_or_zero(p.s[j]);
+}
+
+// Thread `tid` owns the 16-byte vectors v = i*ROW_T + tid (i < VPT) of every
+// row it touches, so its per-column constants are row-invariant.  REG: they
+// (and the pass-1 products) live in registers; otherwise they are read from
+// shared memory laid out as EPV/4 planes of float4 (plane h holds elements
+// 4h..4h+3 of every vector), which makes the per-thread float4 reads
+// conflict-free.
 template <int DT, int VPT, int MODE>
 __global__ void __launch_bounds__(ROW_T) k_rows(RowArgs p)
 {
     constexpr int EPV = VecT<DT>::EPV;
-    extern __shared__ float colv[];          // per-column constant, K floats
+    constexpr bool REG = (VPT * EPV <= 32);
+    extern __shared__ float4 colv4[];
     __shared__ float red[32];
     __shared__ double red64[32];
 
     const int tid = threadIdx.x;
     const int64_t nvec = p.K / EPV;
+    const int64_t plane = nvec;            // float4 entries per plane
 
-    // per-column constant of this step
-    for (int64_t j = tid; j < p.K; j += ROW_T) {
-        if constexpr (MODE == ROW_WEIGHT) colv[j] = p.s[j];
-        else if constexpr (MODE == ROW_RMSNORM) colv[j] = __fmul_rn(p.gamma[j], recip_or_zero(p.s[j]));
-        else colv[j] = recip_or_zero(p.s[j]);
-    }
-    float inv_a_static = 0.0f;
-    if constexpr (MODE == ROW_ACT_STATIC || MODE == ROW_RMSNORM) inv_a_static = recip_or_zero(p.a_in[0]);
-    __syncthreads();
-
-    for (int64_t row = blockIdx.x; row < p.rows; row += gridDim.x) {
-        const uint8_t *src;
-        if (p.src1 != nullptr) {          // gate/up interleave: blocks of 64 output rows
-            const int64_t b = row >> 6, w = row & 63;
-            src = (w < 32 ? p.src0 : p.src1) + ((b << 5) + (w & 31)) * p.row_bytes;
-        } else {
-            src = p.src0 + row * p.row_bytes;
-        }
-        uint4 raw[VPT];
+    float creg[REG ? VPT : 1][REG ? EPV : 1];
+    if constexpr (REG) {
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
             const int64_t v = static_cast<int64_t>(i) * ROW_T + tid;
-            if (v < nvec) raw[i] = __ldcs(reinterpret_cast<const uint4 *>(src) + v);
+#pragma unroll
+            for (int e = 0; e < EPV; ++e) creg[i][e] = (v < nvec) ? column_constant<MODE>(p, v * EPV + e) : 0.0f;
+        }
+    } else {
+        float *cv = reinterpret_cast<float *>(colv4);
+        for (int64_t j = tid; j < p.K; j += ROW_T) {
+            const int64_t v = j / EPV;
+            const int e = static_cast<int>(j % EPV);
+            cv[((e >> 2) * plane + v) * 4 + (e & 3)] = column_constant<MODE>(p, j);
+        }
+        __syncthreads();
+    }
+    auto colc = [&](int i, int64_t v, float (&c)[EPV]) {
+        if constexpr (REG) {
+#pragma unroll
+            for (int e = 0; e < EPV; ++e) c[e] = creg[i][e];
+        } else {
+#pragma unroll
+            for (int h = 0; h < EPV / 4; ++h) {
+                const float4 t = colv4[h * plane + v];
+                c[4 * h] = t.x; c[4 * h + 1] = t.y; c[4 * h + 2] = t.z; c[4 * h + 3] = t.w;
+            }
+        }
+    };
+    float inv_a_static = 0.0f;
+    if constexpr (MODE == ROW_ACT_STATIC || MODE == ROW_RMSNORM) inv_a_static = recip_or_zero(p.a_in[0]);
+
+    auto row_src = [&](int64_t row) -> const uint8_t * {
+        if (p.src1 != nullptr) {          // gate/up interleave: blocks of 64 output rows
+            const int64_t b = row >> 6, w = row & 63;
+            return (w < 32 ? p.src0 : p.src1) + ((b << 5) + (w & 31)) * p.row_bytes;
+        }
+        return p.src0 + row * p.row_bytes;
+    };
+    auto load_row = [&](int64_t row, uint4 (&dst)[VPT]) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(row_src(row));
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int64_t v = static_cast<int64_t>(i) * ROW_T + tid;
+            if (v < nvec) dst[i] = __ldcs(src + v);
+        }
+    };
+    // REG rows are short: the next row's loads are issued before this row is
+    // processed, so each thread keeps two rows of loads in flight.
+    uint4 nxt[REG ? VPT : 1];
+    if constexpr (REG) {
+        if (blockIdx.x < p.rows) load_row(blockIdx.x, nxt);
+    }
+
+    for (int64_t row = blockIdx.x; row < p.rows; row += gridDim.x) {
+        uint4 raw[VPT];
+        if constexpr (REG) {
+#pragma unroll
+            for (int i = 0; i < VPT; ++i) raw[i] = nxt[i];
+            if (row + gridDim.x < p.rows) load_row(row + gridDim.x, nxt);
+        } else {
+            load_row(row, raw);
+        }
+        int8_t *dst = p.out + row * p.K;
+
+        if constexpr (MODE == ROW_ACT_STATIC) {
+#pragma unroll
+            for (int i = 0; i < VPT; ++i) {
+                const int64_t v = static_cast<int64_t>(i) * ROW_T + tid;
+                if (v < nvec) {
+                    float f[EPV], c[EPV];
+                    widen<DT>(raw[i], f);
+                    colc(i, v, c);
+#pragma unroll
+                    for (int e = 0; e < EPV; ++e) f[e] = __fmul_rn(__fmul_rn(f[e], c[e]), inv_a_static);
+                    store_codes<EPV>(dst, v, f);
+                }
+            }
+            continue;
         }
 
-        // pass 1: the per-row statistic (absmax in fp32; sum of squares in fp64,
-        // where every square of a 16-bit or fp32 input is exact)
-        float stat = 0.0f;
-        double ss = 0.0;
-        if constexpr (MODE != ROW_ACT_STATIC) {
+        if constexpr (MODE == ROW_RMSNORM) {
+            // pass 1: sum of squares in fp64 (exact squares)
+            double ss = 0.0;
 #pragma unroll
             for (int i = 0; i < VPT; ++i) {
                 const int64_t v = static_cast<int64_t>(i) * ROW_T + tid;
                 if (v < nvec) {
                     float f[EPV];
                     widen<DT>(raw[i], f);
-                    const float4 *cv = reinterpret_cast<const float4 *>(colv + v * EPV);
 #pragma unroll
-                    for (int e = 0; e < EPV; e += 4) {
-                        const float4 c = cv[e / 4];
-                        const float cc[4] = {c.x, c.y, c.z, c.w};
+                    for (int e = 0; e < EPV; ++e) ss += static_cast<double>(f[e]) * static_cast<double>(f[e]);
+                }
+            }
+            const double tot = block_sum_f64(ss, red64);
+            const float mean = __double2float_rn(tot / static_cast<double>(p.K));
+            const float r_m = __frcp_rn(__fsqrt_rn(__fadd_rn(mean, p.eps)));
+            if (tid == 0 && p.rstd_out != nullptr) p.rstd_out[row] = r_m;
 #pragma unroll
-                        for (int t = 0; t < 4; ++t) {
-                            if constexpr (MODE == ROW_RMSNORM)
-                                ss += static_cast<double>(f[e + t]) * static_cast<double>(f[e + t]);
-                            else
-                                stat = fmaxf(stat, fabsf(__fmul_rn(f[e + t], cc[t])));
-                        }
-                    }
+            for (int i = 0; i < VPT; ++i) {
+                const int64_t v = static_cast<int64_t>(i) * ROW_T + tid;
+                if (v < nvec) {
+                    float f[EPV], c[EPV];
+                    widen<DT>(raw[i], f);
+                    colc(i, v, c);
+#pragma unroll
+                    for (int e = 0; e < EPV; ++e)
+                        f[e] = __fmul_rn(__fmul_rn(__fmul_rn(f[e], r_m), c[e]), inv_a_static);
+                    store_codes<EPV>(dst, v, f);
+                }
+            }
+            continue;
+        }
+
+        // ROW_WEIGHT / ROW_ACT_TOKEN: pass 1 y = fl(x * c_j) and the row absmax,
+        // pass 2 codes of fl(y * recip(scale)).  REG keeps y in registers.
+        float ykeep[REG ? VPT : 1][REG ? EPV : 1];
+        float mx = 0.0f;
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int64_t v = static_cast<int64_t>(i) * ROW_T + tid;
+            if (v < nvec) {
+                float f[EPV], c[EPV];
+                widen<DT>(raw[i], f);
+                colc(i, v, c);
+#pragma unroll
+                for (int e = 0; e < EPV; ++e) {
+                    const float y = __fmul_rn(f[e], c[e]);
+                    mx = fmaxf(mx, fabsf(y));
+                    if constexpr (REG) ykeep[i][e] = y;
                 }
             }
         }
-        float mul_a;          // multiplier applied before rounding
-        float r_m = 0.0f;     // RMSNorm row factor
-        if constexpr (MODE == ROW_ACT_STATIC) {
-            mul_a = inv_a_static;
-        } else if constexpr (MODE == ROW_RMSNORM) {
-            const double tot = block_sum_f64(ss, red64);
-            const float mean = __double2float_rn(tot / static_cast<double>(p.K));
-            r_m = __frcp_rn(__fsqrt_rn(__fadd_rn(mean, p.eps)));
-            mul_a = inv_a_static;
-            if (tid == 0 && p.rstd_out != nullptr) p.rstd_out[row] = r_m;
-        } else {
-            const float mx = block_max(stat, red);
-            const float sc = scale_from_absmax(mx);
-            mul_a = recip_or_zero(sc);
-            if (tid == 0) p.scale_out[row] = sc;
-        }
-
-        // pass 2: codes
-        int8_t *dst = p.out + row * p.K;
+        const float sc = scale_from_absmax(block_max(mx, red));
+        const float inv = recip_or_zero(sc);
+        if (tid == 0) p.scale_out[row] = sc;
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
             const int64_t v = static_cast<int64_t>(i) * ROW_T + tid;
             if (v < nvec) {
                 float f[EPV];
-                widen<DT>(raw[i], f);
-                const float4 *cv = reinterpret_cast<const float4 *>(colv + v * EPV);
+                if constexpr (REG) {
 #pragma unroll
-                for (int e = 0; e < EPV; e += 4) {
-                    const float4 c = cv[e / 4];
-                    const float cc[4] = {c.x, c.y, c.z, c.w};
+                    for (int e = 0; e < EPV; ++e) f[e] = __fmul_rn(ykeep[i][e], inv);
+                } else {
+                    float c[EPV];
+                    widen<DT>(raw[i], f);
+                    colc(i, v, c);
 #pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        float y;
-                        if constexpr (MODE == ROW_RMSNORM) y = __fmul_rn(__fmul_rn(f[e + t], r_m), cc[t]);
-                        else y = __fmul_rn(f[e + t], cc[t]);
-                        f[e + t] = __fmul_rn(y, mul_a);
-                    }
+                    for (int e = 0; e < EPV; ++e) f[e] = __fmul_rn(__fmul_rn(f[e], c[e]), inv);
                 }
-                store_codes<DT>(dst, v, f);
+                store_codes<EPV>(dst, v, f);
             }
         }
     }
