@@ -179,6 +179,19 @@ sq_status sq_rmsnorm_quant(const void *x, sq_dtype dt, int64_t M, int64_t d, con
                            const float *s, float eps, const float *a_scale, int8_t *xq,
                            float *rstd, sq_stream stream);
 
+/* (3c) Calibration statistic of an RMSNorm output, for the linear that reads
+ * it (kwkr 3.1: statistics are taken per layer on the layer's own input; the
+ * gate/up projections of a decoder MLP read the normalised activations):
+ *
+ *   absmax[j] = max(absmax[j], max_m |fl(fl(x_mj * r_m) * gamma_j)|),  r_m as in sq_rmsnorm_quant
+ *
+ * x: [M, d] of `dt`, 16-byte aligned.  gamma: fp32 [d].  absmax: fp32 [d],
+ * a running max (the caller zeroes it once).  The per-thread column maxima
+ * stay in registers for d * sizeof(dt) <= 64 KiB; wider rows take a slow
+ * per-element path. */
+sq_status sq_rmsnorm_absmax(const void *x, sq_dtype dt, int64_t M, int64_t d, const float *gamma,
+                            float eps, float *absmax, sq_stream stream);
+
 /* -------------------------------------------------------------------------
  * (4) W8A8 GEMM with the dequant epilogue (pwwt 3.1: INT8 matmul with the
  * scale multiplications merged into it; adr-010 key design points 4-5 name

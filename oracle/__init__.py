@@ -32,6 +32,7 @@ Parity pins (tests/test_oracle_pins.py; tests/golden/ fixtures):
   dequant               -- fp64 product within one fp32 rounding + one output
                            rounding
   rmsnorm_quant         -- fp64 unfused RMSNorm then x/s, within rounding
+  rmsnorm_absmax        -- fp64 unfused RMSNorm column max, within rounding
   silu_mul_bf16         -- math.exp closed form; silu(0) = 0, silu(g) -> g
   mse_f16, gemm_f16_ref -- numpy fp64 mean / matmul
   identity              -- fp64 XW^T == (X diag(s)^-1)(W diag(s))^T, 1e-9
@@ -114,6 +115,7 @@ def lib():
             L.oracle_rmsnorm_quant.argtypes = [_P, ctypes.c_int, _I64, _I64, _P, _P, ctypes.c_float,
                                                _P, _P, _P, _P]
             L.oracle_silu_mul_bf16.argtypes = [_P, _P, _I64, _P]
+            L.oracle_rmsnorm_absmax.argtypes = [_P, ctypes.c_int, _I64, _I64, _P, ctypes.c_float, _P]
             L.oracle_mse_f16.restype = ctypes.c_double
             L.oracle_mse_f16.argtypes = [_P, _P, _I64]
             L.oracle_gemm_f16_ref.argtypes = [_P, _P, _I64, _I64, _I64, _P]
@@ -285,6 +287,16 @@ def rmsnorm_quant(x, gamma, s, eps, a_static, dt: int | None = None, r_given=Non
     lib().oracle_rmsnorm_quant(_ptr(x), dt, M, d, _ptr(g), _ptr(s), float(eps), _ptr(a),
                                _ptr(rg), _ptr(xq), _ptr(r))
     return xq, r
+
+
+def rmsnorm_absmax(x, gamma, eps, dt: int | None = None, absmax: np.ndarray | None = None) -> np.ndarray:
+    """Running column max of |RMSNorm(x) * gamma| (the gate/up layer's input statistic)."""
+    x, dt = _dtcode(x, dt)
+    M, d = x.shape
+    g = np.ascontiguousarray(gamma, np.float32)
+    out = np.zeros(d, np.float32) if absmax is None else absmax
+    lib().oracle_rmsnorm_absmax(_ptr(x), dt, M, d, _ptr(g), float(eps), _ptr(out))
+    return out
 
 
 def silu_mul_bf16(g: np.ndarray, u: np.ndarray) -> np.ndarray:

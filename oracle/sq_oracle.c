@@ -38,6 +38,7 @@
 #include <stddef.h>
 #include <string.h>
 #include <math.h>
+#include <stdlib.h>
 
 enum { OR_F32 = 0, OR_F16 = 1, OR_BF16 = 2 };
 enum { OR_STATIC = 0, OR_PER_TOKEN = 1 };
@@ -316,6 +317,28 @@ void oracle_rmsnorm_quant(const void *x, int dt, int64_t M, int64_t d, const flo
     }
 }
 
+/* Calibration statistic of the RMSNorm output (the activation that enters the  */
+/* gate/up linear): absmax_j = max(absmax_j, max_m |fl(fl(x_mj * r_m) * gamma_j)|), */
+/* r_m as in oracle_rmsnorm_quant ([KWKR] 3.1 statistic taken on the layer's     */
+/* actual input).                                                                */
+void oracle_rmsnorm_absmax(const void *x, int dt, int64_t M, int64_t d, const float *gamma, float eps,
+                           float *absmax)
+{
+    for (int64_t m = 0; m < M; ++m) {
+        double ss = 0.0;
+        for (int64_t j = 0; j < d; ++j) {
+            double v = (double)ld(x, dt, m * d + j);
+            ss += v * v;
+        }
+        float mean = (float)(ss / (double)d);
+        float r = 1.0f / sqrtf(mean + eps);
+        for (int64_t j = 0; j < d; ++j) {
+            float y = (ld(x, dt, m * d + j) * r) * gamma[j];
+            if (fabsf(y) > absmax[j]) absmax[j] = fabsf(y);
+        }
+    }
+}
+
 /* ---------------------------------------------------------------------- */
 /* a9: SiLU(gate) * up on the fp32 dequantised gate/up outputs, rounded to  */
 /* bf16.  silu(g) = g / (1 + exp(-g)), evaluated in fp64, rounded to fp32, */
@@ -352,14 +375,23 @@ double oracle_mse_f16(const uint16_t *y, const uint16_t *y_ref, int64_t n)
 void oracle_gemm_f16_ref(const uint16_t *x, const uint16_t *w, int64_t M, int64_t N, int64_t K,
                          uint16_t *y)
 {
+    /* both operands are widened once (exactly) to fp64, then summed in fp64 */
+    double *xd = (double *)malloc((size_t)(M * K) * sizeof(double));
+    double *wd = (double *)malloc((size_t)(N * K) * sizeof(double));
+    #pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < M * K; ++i) xd[i] = (double)oracle_f16_to_f32(x[i]);
+    #pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < N * K; ++i) wd[i] = (double)oracle_f16_to_f32(w[i]);
     #pragma omp parallel for collapse(2) schedule(static)
     for (int64_t m = 0; m < M; ++m)
         for (int64_t n = 0; n < N; ++n) {
             double a = 0.0;
             for (int64_t k = 0; k < K; ++k)
-                a += (double)oracle_f16_to_f32(x[m * K + k]) * (double)oracle_f16_to_f32(w[n * K + k]);
+                a += xd[m * K + k] * wd[n * K + k];
             y[m * N + n] = oracle_f32_to_f16((float)a);
         }
+    free(xd);
+    free(wd);
 }
 
 /* Array forms of the number-format conversions (used to widen / round whole

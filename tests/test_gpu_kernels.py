@@ -323,3 +323,19 @@ def test_alpha_search_small():
     best, mses = sq.alpha_search(dev(held, F16), dev(wl.w, F16), dev(am), dev(wm), work)
     assert best == best_ref
     assert rel_err(mses, mse_ref).max() < 1e-2
+
+
+# ------------------------------------------------------------------ a8 statistic
+@pytest.mark.parametrize("M,d,dt", [(300, 8192, BF16), (7, 4096, F16), (33, 1000, BF16), (5, 2048, F32),
+                                    (3, 11008, BF16)])
+def test_rmsnorm_absmax(M, d, dt):
+    X = rand_x(M * 5 + d, (M, d), dt, 1.0, outliers=max(1, d // 200))
+    gamma = np.random.default_rng(d + 1).uniform(0.5, 1.5, d).astype(np.float32)
+    am = torch.zeros(d, dtype=torch.float32, device="cuda")
+    half = M // 2
+    xt = dev(X, dt)
+    sq.rmsnorm_absmax(xt[:half] if half else xt[:0], dev(gamma), 1e-5, am)
+    sq.rmsnorm_absmax(xt[half:], dev(gamma), 1e-5, am)
+    _sync()
+    ref = oracle.rmsnorm_absmax(X, gamma, 1e-5, dt)
+    assert bits_equal(host(am), ref), mismatch_report(host(am), ref)

@@ -1,0 +1,349 @@
+"""End-to-end parity of the five SmoothQuant W8A8 workloads at their full sizes.
+
+Each workload runs through the C ABI exactly as bench.py launches it.  The
+oracle checks every output it can afford in full: calibration statistics,
+smoothing factors, static scales, weight codes and scales, activation codes
+and per-token scales, RMSNorm codes.  GEMM outputs, whose oracle cost is
+M*N*K int32 multiply-adds, are checked bit for bit on sampled token rows
+(every output channel of those rows).
+
+Staged parity: the smoothing factors come from fp64 log2/exp2 on the GPU and
+fp64 pow in the oracle, so they may differ in the last fp32 bit on a tiny
+fraction of channels.  Every downstream step is therefore also run on the GPU
+with the oracle's factors and scales uploaded, and those results must be
+bit-exact.  The GPU's own end-to-end chain is additionally checked to be
+bit-exact wherever its factors equal the oracle's.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from helpers import BF16, F16, F32, TORCH_DT, bits_equal, dev, host, mismatch_report, rel_err
+
+pytestmark = pytest.mark.gpu
+
+sq = pytest.importorskip("w8a8_post_quantization_calib_b200")
+
+
+def _sync():
+    assert sq.sync_status() == 0
+
+
+def _zeros(n):
+    return torch.zeros(n, dtype=torch.float32, device="cuda")
+
+
+def _check_scales(s_gpu, s_ref, a_gpu=None, a_ref=None):
+    assert rel_err(s_gpu, s_ref).max() <= 1e-6
+    assert (s_gpu != s_ref).mean() < 1e-3
+    if a_gpu is not None:
+        assert rel_err(a_gpu, a_ref).max() <= 1e-6
+
+
+def _sample_rows(M, n):
+    if M <= n:
+        return np.arange(M)
+    idx = np.unique(np.linspace(0, M - 1, n).astype(np.int64))
+    return idx
+
+
+def run_linear(wl, calib_concat=True, sample_rows=64, bias=None):
+    """GPU + oracle pipeline for one linear workload; returns the comparison record."""
+    K, N, M = wl.K, wl.N, wl.M
+    x_dt, w_dt, out_dt, mode = wl.x_dt, wl.w_dt, wl.out_dt, wl.mode
+    # ---------------- GPU: calibration -> scales -> weight -> activations -> GEMM
+    act_max = _zeros(K)
+    if calib_concat:
+        sq.calib_absmax(dev(np.concatenate(wl.calib), x_dt), act_max)
+    else:
+        for b in wl.calib:
+            sq.calib_absmax(dev(b, x_dt), act_max)
+    W = dev(wl.w, w_dt)
+    w_max = _zeros(K)
+    sq.calib_absmax(W, w_max)
+    s = torch.empty(K, dtype=torch.float32, device="cuda")
+    a = torch.empty(1, dtype=torch.float32, device="cuda")
+    sq.smooth_scales(act_max, w_max, wl.alpha, s, a)
+    wq = torch.empty(N, K, dtype=torch.int8, device="cuda")
+    ws = torch.empty(N, dtype=torch.float32, device="cuda")
+    sq.quant_weight(W, s, wq, ws)
+    X = dev(wl.x, x_dt)
+    xq = torch.empty(M, K, dtype=torch.int8, device="cuda")
+    at = a if mode == oracle.STATIC else torch.empty(M, dtype=torch.float32, device="cuda")
+    sq.smooth_quant_act(X, s, mode, at, xq)
+    y = torch.empty(M, N, dtype=TORCH_DT[out_dt], device="cuda")
+    work = torch.zeros(max(16, sq.linear_workspace_size(M, N, K)), dtype=torch.uint8, device="cuda")
+    bias_t = dev(bias, out_dt) if bias is not None else None
+    sq.linear_w8a8(xq, wq, at, mode, ws, y, bias=bias_t, workspace=work)
+    _sync()
+
+    # ---------------- oracle
+    ref = oracle.calibrate_and_quantize(wl.calib, wl.w, wl.alpha, x_dt, w_dt)
+    assert bits_equal(host(act_max), ref.act_max), mismatch_report(host(act_max), ref.act_max)
+    assert bits_equal(host(w_max), ref.w_max), mismatch_report(host(w_max), ref.w_max)
+    s_gpu = host(s)
+    _check_scales(s_gpu, ref.s, host(a), [ref.a_static])
+    same_s = bits_equal(s_gpu, ref.s) and host(a)[0] == ref.a_static
+
+    # ---------------- staged: GPU quantisation with the oracle's factors / scales
+    s_o = dev(ref.s)
+    a_o = dev(np.array([ref.a_static], np.float32))
+    wq2 = torch.empty_like(wq)
+    ws2 = torch.empty_like(ws)
+    sq.quant_weight(W, s_o, wq2, ws2)
+    xq2 = torch.empty_like(xq)
+    at2 = a_o if mode == oracle.STATIC else torch.empty(M, dtype=torch.float32, device="cuda")
+    sq.smooth_quant_act(X, s_o, mode, at2, xq2)
+    y2 = torch.empty_like(y)
+    sq.linear_w8a8(xq2, wq2, at2, mode, ws2, y2, bias=bias_t, workspace=work)
+    _sync()
+    assert bits_equal(host(ws2), ref.w_scale), mismatch_report(host(ws2), ref.w_scale)
+    assert bits_equal(host(wq2), ref.wq), mismatch_report(host(wq2), ref.wq)
+    if mode == oracle.STATIC:
+        xq_r, a_r = oracle.smooth_quant_act(wl.x, ref.s, oracle.STATIC, ref.a_static, x_dt)
+    else:
+        xq_r, a_r = oracle.smooth_quant_act(wl.x, ref.s, oracle.PER_TOKEN, None, x_dt)
+        assert bits_equal(host(at2), a_r), mismatch_report(host(at2), a_r)
+    assert bits_equal(host(xq2), xq_r), mismatch_report(host(xq2), xq_r)
+    rows = _sample_rows(M, sample_rows)
+    acc_r = oracle.gemm_s32(xq_r[rows], ref.wq)
+    a_rows = a_r if mode == oracle.STATIC else a_r[rows]
+    y_r = oracle.dequant(acc_r, a_rows, mode, ref.w_scale, out_dt, bias)
+    got = host(y2)[rows]
+    assert bits_equal(got, y_r), mismatch_report(got, y_r)
+    if same_s:        # the GPU's own chain reached the oracle's factors: everything is bit-exact
+        assert bits_equal(host(wq), ref.wq) and bits_equal(host(xq), xq_r)
+        assert bits_equal(host(y)[rows], y_r)
+    return {"same_s": same_s, "y": y, "rows": rows, "ref": ref}
+
+
+# ------------------------------------------------------------------ workload 1
+def test_linear_toy_fp32_full():
+    """tbr8.org toy layer: K=1024, N=2048, M=16, fp32, 4 calibration batches, static, fp32 out."""
+    wl = synth.linear_toy()
+    r = run_linear(wl, calib_concat=False, sample_rows=16)
+    # the smoothed W8A8 output reconstructs XW^T well below the unsmoothed error
+    Y = wl.x.astype(np.float64) @ wl.w.astype(np.float64).T
+    yq = host(r["y"]).astype(np.float64)
+    assert np.linalg.norm(yq - Y) / np.linalg.norm(Y) < 0.02
+
+
+# ------------------------------------------------------------------ workload 2
+def test_qkv_7b_full():
+    """Llama-7B QKV: K=4096, N=12288, M=2048, fp16, 64 x 512 calibration tokens, static, fp16 out."""
+    run_linear(synth.qkv_7b(), calib_concat=True, sample_rows=48)
+
+
+def test_qkv_7b_calibration_in_batches_equals_concatenated():
+    """Running max over 64 separate launches == one launch over the concatenated batches."""
+    wl = synth.qkv_7b(M=16)
+    a1 = _zeros(wl.K)
+    a2 = _zeros(wl.K)
+    for b in wl.calib:
+        sq.calib_absmax(dev(b, F16), a1)
+    sq.calib_absmax(dev(np.concatenate(wl.calib), F16), a2)
+    _sync()
+    assert torch.equal(a1, a2)
+
+
+# ------------------------------------------------------------------ workload 3
+_MLP7B = {}
+
+
+def _mlp_7b(which, M):
+    if which not in _MLP7B:
+        _MLP7B.clear()
+        _MLP7B[which] = synth.mlp_7b(which, M=4096)     # 64 x 512 calibration tokens
+    full = _MLP7B[which]
+    wl = synth.LinearWorkload(full.name, full.K, full.N, M, full.x_dt, full.w_dt, full.out_dt,
+                              calib=full.calib, x=full.x[:M], w=full.w, alpha=full.alpha, mode=full.mode)
+    return wl
+
+
+@pytest.mark.parametrize("M", [1, 16, 128, 4096])
+@pytest.mark.parametrize("which", ["up", "down"])
+def test_mlp_7b_per_token(which, M):
+    """Llama-7B MLP pair, per-token dynamic activation scales, bf16 in/out, decode to prefill."""
+    run_linear(_mlp_7b(which, M), calib_concat=True, sample_rows=24)
+
+
+# ------------------------------------------------------------------ workload 4
+def test_alpha_search_13b_full():
+    """13B linear: alpha grid search on the held batch (512 x 5120 x 13824), then the M=8192 run."""
+    wl = synth.heavy_13b()
+    am = _zeros(wl.K)
+    sq.calib_absmax(dev(np.concatenate(wl.calib), F16), am)
+    W = dev(wl.w, F16)
+    wm = _zeros(wl.K)
+    sq.calib_absmax(W, wm)
+    held = wl.calib[0]
+    work = torch.zeros(sq.alpha_search_workspace_size(held.shape[0], wl.N, wl.K, 4), dtype=torch.uint8,
+                       device="cuda")
+    best, mses = sq.alpha_search(dev(held, F16), W, am, wm, work)
+    am_r = np.zeros(wl.K, np.float32)
+    for b in wl.calib:
+        oracle.calib_absmax(b, F16, am_r)
+    wm_r = oracle.calib_absmax(wl.w, F16)
+    assert bits_equal(host(am), am_r) and bits_equal(host(wm), wm_r)
+    best_r, mses_r, _ = oracle.alpha_search(held, wl.w, am_r, wm_r)
+    # the reference product is accumulated in fp32 on the tensor cores and in fp64 in the oracle
+    assert rel_err(mses, mses_r).max() < 1e-2
+    assert best == best_r
+    assert mses[list(oracle.ALPHA_GRID).index(best)] <= min(mses[0], mses[-1])
+    # full-size run at the chosen alpha
+    wl.alpha = best
+    run_linear(wl, calib_concat=True, sample_rows=24)
+
+
+# ------------------------------------------------------------------ workload 5
+def _interleave(wg, wu):
+    Nh = wg.shape[0]
+    order = np.concatenate([np.concatenate([np.arange(b, b + 32), Nh + np.arange(b, b + 32)])
+                            for b in range(0, Nh, 32)])
+    return np.concatenate([wg, wu])[order], order
+
+
+def run_mlp_block(blk, sample_rows, exact_h_calibration):
+    d, f, M = blk.d, blk.f, blk.M
+    eps, al = blk.eps, blk.alpha
+    g = dev(blk.gamma)
+    # ---------------- GPU
+    am1 = _zeros(d)
+    for b in blk.calib:
+        sq.rmsnorm_absmax(dev(b, BF16), g, eps, am1)
+    Wg, Wu, Wd = dev(blk.w_gate, BF16), dev(blk.w_up, BF16), dev(blk.w_down, BF16)
+    wm1 = _zeros(d)
+    sq.calib_absmax(Wg, wm1)
+    sq.calib_absmax(Wu, wm1)
+    s1g = torch.empty(d, dtype=torch.float32, device="cuda")
+    a1g = torch.empty(1, dtype=torch.float32, device="cuda")
+    sq.smooth_scales(am1, wm1, al, s1g, a1g)
+    _sync()
+    # oracle statistics and factors of the first linear
+    am1_r = np.zeros(d, np.float32)
+    for b in blk.calib:
+        oracle.rmsnorm_absmax(b, blk.gamma, eps, BF16, am1_r)
+    assert bits_equal(host(am1), am1_r), mismatch_report(host(am1), am1_r)
+    wm1_r = oracle.calib_absmax(blk.w_gate, BF16)
+    oracle.calib_absmax(blk.w_up, BF16, wm1_r)
+    assert bits_equal(host(wm1), wm1_r)
+    s1_r = oracle.smooth_scales(am1_r, wm1_r, al)
+    a1_r = oracle.static_scale(am1_r, s1_r)
+    _check_scales(host(s1g), s1_r, host(a1g), [a1_r])
+    # staged from here on: the GPU continues with the oracle's factor and scale
+    s1 = dev(s1_r)
+    a1 = dev(np.array([a1_r], np.float32))
+    wq_gu = torch.empty(2 * f, d, dtype=torch.int8, device="cuda")
+    ws_gu = torch.empty(2 * f, dtype=torch.float32, device="cuda")
+    sq.quant_weight_gateup(Wg, Wu, s1, wq_gu, ws_gu)
+    # statistic of h (the down projection's input) on the calibration batches
+    am2 = _zeros(f)
+    for b in blk.calib:
+        xq_c = torch.empty(b.shape[0], d, dtype=torch.int8, device="cuda")
+        sq.rmsnorm_quant(dev(b, BF16), g, s1, eps, a1, xq_c)
+        h_c = torch.empty(b.shape[0], f, dtype=torch.bfloat16, device="cuda")
+        sq.linear_w8a8_gateup_silu(xq_c, wq_gu, a1, sq.ACT_STATIC, ws_gu, h=h_c)
+        sq.calib_absmax(h_c, am2)
+    wm2 = _zeros(f)
+    sq.calib_absmax(Wd, wm2)
+    s2 = torch.empty(f, dtype=torch.float32, device="cuda")
+    a2 = torch.empty(1, dtype=torch.float32, device="cuda")
+    sq.smooth_scales(am2, wm2, al, s2, a2)
+    wq_d = torch.empty(d, f, dtype=torch.int8, device="cuda")
+    ws_d = torch.empty(d, dtype=torch.float32, device="cuda")
+    sq.quant_weight(Wd, s2, wq_d, ws_d)
+    # runtime: RMSNorm+quant -> gate/up GEMM with SiLU*mul and requant -> down GEMM
+    X = dev(blk.x, BF16)
+    xq = torch.empty(M, d, dtype=torch.int8, device="cuda")
+    rstd = torch.empty(M, dtype=torch.float32, device="cuda")
+    sq.rmsnorm_quant(X, g, s1, eps, a1, xq, rstd)
+    hq = torch.empty(M, f, dtype=torch.int8, device="cuda")
+    h = torch.empty(M, f, dtype=torch.bfloat16, device="cuda")
+    sq.linear_w8a8_gateup_silu(xq, wq_gu, a1, sq.ACT_STATIC, ws_gu, h=h, s2=s2, a2=a2, hq=hq)
+    y = torch.empty(M, d, dtype=torch.bfloat16, device="cuda")
+    sq.linear_w8a8(hq, wq_d, a2, sq.ACT_STATIC, ws_d, y)
+    _sync()
+
+    # ---------------- oracle: weights and RMSNorm codes (full)
+    wcat, order = _interleave(blk.w_gate, blk.w_up)
+    wq_gu_r, ws_gu_r = oracle.quant_weight(wcat, s1_r, BF16)
+    assert bits_equal(host(ws_gu), ws_gu_r) and bits_equal(host(wq_gu), wq_gu_r)
+    xq_r, r_r = oracle.rmsnorm_quant(blk.x, blk.gamma, s1_r, eps, a1_r, BF16)
+    assert bits_equal(host(rstd), r_r), mismatch_report(host(rstd), r_r)
+    assert bits_equal(host(xq), xq_r), mismatch_report(host(xq), xq_r)
+
+    # h statistic: exact at reduced size; at full size every sampled calibration
+    # row's h (oracle) lies under it, and each channel's maximum is attained
+    h_stat = host(am2)
+    wg_q, wu_q = wq_gu_r[np.argsort(order)][:f], wq_gu_r[np.argsort(order)][f:]
+    wsg, wsu = ws_gu_r[np.argsort(order)][:f], ws_gu_r[np.argsort(order)][f:]
+
+    def oracle_h(xq_rows):
+        gv = oracle.dequant_f32(oracle.gemm_s32(xq_rows, wg_q), np.array([a1_r]), oracle.STATIC, wsg)
+        uv = oracle.dequant_f32(oracle.gemm_s32(xq_rows, wu_q), np.array([a1_r]), oracle.STATIC, wsu)
+        return oracle.silu_mul_bf16(gv, uv)
+
+    if exact_h_calibration:
+        am2_r = np.zeros(f, np.float32)
+        for b in blk.calib:
+            xq_c, _ = oracle.rmsnorm_quant(b, blk.gamma, s1_r, eps, a1_r, BF16)
+            oracle.calib_absmax(oracle_h(xq_c), BF16, am2_r)
+        # h itself is within 2 bf16 ulp of the oracle (CUDA expf), so is its column max
+        assert np.all(np.abs(h_stat - am2_r) <= np.abs(am2_r) * 2.0 ** -6 + 1e-30)
+        s2_ref_in = am2_r
+    else:
+        b0 = blk.calib[0]
+        rows_c = _sample_rows(b0.shape[0], 8)
+        xq_c, _ = oracle.rmsnorm_quant(b0[rows_c], blk.gamma, s1_r, eps, a1_r, BF16)
+        hc = np.abs(oracle.to_f32(oracle_h(xq_c), BF16))
+        assert np.all(hc <= h_stat[None, :] * (1 + 2.0 ** -6) + 1e-30)
+        s2_ref_in = h_stat          # downstream checks use the GPU statistic as a given input
+    wm2_r = oracle.calib_absmax(blk.w_down, BF16)
+    assert bits_equal(host(wm2), wm2_r)
+    s2_r = oracle.smooth_scales(s2_ref_in, wm2_r, al)
+    a2_r = oracle.static_scale(s2_ref_in, s2_r)
+    if exact_h_calibration:
+        _check_scales(host(s2), s2_r, host(a2), [a2_r])
+
+    # ---------------- staged downstream with the oracle's s2/a2 uploaded: bit-exact on sampled rows
+    s2_o, a2_o = dev(s2_r), dev(np.array([a2_r], np.float32))
+    wq_d2 = torch.empty_like(wq_d)
+    ws_d2 = torch.empty_like(ws_d)
+    sq.quant_weight(Wd, s2_o, wq_d2, ws_d2)
+    hq2 = torch.empty_like(hq)
+    h2 = torch.empty_like(h)
+    sq.linear_w8a8_gateup_silu(xq, wq_gu, a1, sq.ACT_STATIC, ws_gu, h=h2, s2=s2_o, a2=a2_o, hq=hq2)
+    y2 = torch.empty_like(y)
+    sq.linear_w8a8(hq2, wq_d2, a2_o, sq.ACT_STATIC, ws_d2, y2)
+    _sync()
+    wq_d_r, ws_d_r = oracle.quant_weight(blk.w_down, s2_r, BF16)
+    assert bits_equal(host(ws_d2), ws_d_r) and bits_equal(host(wq_d2), wq_d_r)
+    rows = _sample_rows(M, sample_rows)
+    h_r = oracle_h(xq_r[rows])
+    h_got = host(h2)[rows]
+    hf_got = oracle.to_f32(h_got, BF16).astype(np.float64)
+    hf_ref = oracle.to_f32(h_r, BF16).astype(np.float64)
+    assert np.all(np.abs(hf_got - hf_ref) <= 2 * np.abs(hf_ref) * 2.0 ** -7 + 1e-30)
+    hq_r, _ = oracle.smooth_quant_act(h_r, s2_r, oracle.STATIC, a2_r, BF16)
+    hq_got = host(hq2)[rows]
+    same = h_got == h_r
+    assert np.array_equal(hq_got[same], hq_r[same])
+    assert np.all(np.abs(hq_got.astype(int) - hq_r.astype(int)) <= 1)
+    # down projection on the GPU's own codes of the sampled rows (codes are compared above)
+    acc_d = oracle.gemm_s32(hq_got, wq_d_r)
+    y_r = oracle.dequant(acc_d, np.array([a2_r]), oracle.STATIC, ws_d_r, BF16)
+    assert bits_equal(host(y2)[rows], y_r), mismatch_report(host(y2)[rows], y_r)
+
+
+def test_mlp_block_reduced_exact():
+    """The whole MLP block, h calibration included, at a size the oracle can follow exactly."""
+    blk = synth.mlp_block_70b(M=512, d=1024, f=2048, calib_batches=2, calib_rows=256, gamma_random=True)
+    run_mlp_block(blk, sample_rows=64, exact_h_calibration=True)
+
+
+def test_mlp_block_70b_full():
+    """70B MLP block: M=16384, d=8192, f=28672, 8 x 2048 calibration tokens, bf16."""
+    blk = synth.mlp_block_70b()
+    run_mlp_block(blk, sample_rows=12, exact_h_calibration=False)

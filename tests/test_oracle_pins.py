@@ -440,6 +440,19 @@ def test_rmsnorm_fold_equals_unfused():
     assert np.array_equal(xq2, xq) and np.array_equal(rr2, rr)
 
 
+def test_rmsnorm_absmax_vs_fp64():
+    g = np.random.default_rng(22)
+    M, d = 40, 256
+    X = synth.cast(g.standard_normal((M, d)).astype(np.float32) * 3, BF16)
+    gamma = g.uniform(0.5, 1.5, d).astype(np.float32)
+    x = oracle.to_f32(X, BF16).astype(np.float64)
+    r = 1.0 / np.sqrt((x * x).mean(axis=1) + 1e-5)
+    ref = np.abs(x * r[:, None] * gamma[None, :]).max(axis=0)
+    half = oracle.rmsnorm_absmax(X[:20], gamma, 1e-5, BF16)
+    got = oracle.rmsnorm_absmax(X[20:], gamma, 1e-5, BF16, half)      # running max over two batches
+    assert _rel(got, ref).max() < 3e-7
+
+
 def test_silu_mul_closed_form():
     g = np.array([0.0, 1.0, -1.0, 20.0, -20.0, 3.5, -0.25], np.float32)
     u = np.array([5.0, 2.0, 2.0, 1.0, 1.0, -1.0, 4.0], np.float32)

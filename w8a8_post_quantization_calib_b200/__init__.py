@@ -34,7 +34,7 @@ _STATUS = {0: "SQ_OK", 1: "SQ_ERR_INVALID_ARG", 2: "SQ_ERR_UNSUPPORTED", 3: "SQ_
 EXPORTS = (
     "sq_status_string", "sq_last_cuda_error", "sq_set_wait_timeout_ns", "sq_sync_status",
     "sq_calib_absmax", "sq_smooth_scales", "sq_quant_weight", "sq_quant_weight_gateup",
-    "sq_smooth_quant_act", "sq_rmsnorm_quant", "sq_linear_workspace_size", "sq_linear_w8a8",
+    "sq_smooth_quant_act", "sq_rmsnorm_quant", "sq_rmsnorm_absmax", "sq_linear_workspace_size", "sq_linear_w8a8",
     "sq_linear_w8a8_noalloc", "sq_linear_w8a8_noalloc_max_elems",
     "sq_gemm_s32", "sq_linear_w8a8_gateup_silu", "sq_gemm_f16_ref", "sq_sse_f16",
     "sq_alpha_search_workspace_size", "sq_alpha_search",
@@ -67,6 +67,7 @@ def _load() -> ctypes.CDLL:
         "sq_quant_weight_gateup": (I, [P, P, I, I64, I64, P, P, P, P]),
         "sq_smooth_quant_act": (I, [P, I, I64, I64, P, I, P, P, P]),
         "sq_rmsnorm_quant": (I, [P, I, I64, I64, P, P, F, P, P, P, P]),
+        "sq_rmsnorm_absmax": (I, [P, I, I64, I64, P, F, P, P]),
         "sq_linear_workspace_size": (SZ, [I64, I64, I64]),
         "sq_linear_w8a8": (I, [P, P, I64, I64, I64, P, I, P, P, I, P, P, SZ, P]),
         "sq_linear_w8a8_noalloc": (I, [P, P, I64, I64, I64, P, I, P, P, I, P, P]),
@@ -187,6 +188,14 @@ def rmsnorm_quant(x, gamma, s, eps: float, a_scale, xq, rstd=None, stream=None) 
         _dev(x, "x"), _dt(x), M, d, _dev(gamma, "gamma", torch.float32), _dev(s, "s", torch.float32),
         float(eps), _dev(a_scale, "a_scale", torch.float32), _dev(xq, "xq", torch.int8),
         _dev(rstd, "rstd", torch.float32), _stream(stream)))
+
+
+def rmsnorm_absmax(x, gamma, eps: float, absmax, stream=None) -> None:
+    """absmax[j] = max(absmax[j], max_m |RMSNorm(x)[m, j] * gamma[j]|) (running max)."""
+    M, d = x.shape
+    _check("sq_rmsnorm_absmax", _lib.sq_rmsnorm_absmax(
+        _dev(x, "x"), _dt(x), M, d, _dev(gamma, "gamma", torch.float32), float(eps),
+        _dev(absmax, "absmax", torch.float32), _stream(stream)))
 
 
 def linear_workspace_size(M: int, N: int, K: int) -> int:

@@ -274,8 +274,9 @@ template <int DT, int MODE>
 sq_status launch_rows_dt(RowArgs a, cudaStream_t st)
 {
     constexpr int EPV = VecT<DT>::EPV;
-    const bool vec = aligned16(a.src0) && (a.src1 == nullptr || aligned16(a.src1)) && aligned16(a.out) &&
-                     (a.K % EPV) == 0;
+    const bool vec = aligned16(a.src0) && (a.src1 == nullptr || aligned16(a.src1)) &&
+                     (a.out == nullptr || aligned16(a.out)) && (a.K % EPV) == 0 &&
+                     (MODE != ROW_RMS_STAT || cdiv(a.K / EPV, ROW_T) * EPV <= 32);
     const int64_t nvec = a.K / EPV;
     const int64_t vpt = cdiv(nvec, ROW_T);
     // per-column constants in registers when VPT * EPV <= 32, else in shared memory
@@ -285,6 +286,7 @@ sq_status launch_rows_dt(RowArgs a, cudaStream_t st)
         void (*kern)(RowArgs) = nullptr;
         if (vpt <= 1) kern = k_rows<DT, 1, MODE>;
         else if (vpt <= 2) kern = k_rows<DT, 2, MODE>;
+        else if constexpr (MODE == ROW_RMS_STAT) kern = k_rows<DT, (DT == DT_F32 ? 8 : 4), MODE>;
         else if (vpt <= 4) kern = k_rows<DT, 4, MODE>;
         else if (vpt <= 8) kern = k_rows<DT, 8, MODE>;
         else kern = k_rows<DT, 16, MODE>;
@@ -533,6 +535,23 @@ sq_status sq_rmsnorm_quant(const void *x, sq_dtype dt, int64_t M, int64_t d, con
     a.rstd_out = rstd;
     a.out = xq;
     return launch_rows<ROW_RMSNORM>(a, dt, as_stream(stream));
+}
+
+sq_status sq_rmsnorm_absmax(const void *x, sq_dtype dt, int64_t M, int64_t d, const float *gamma, float eps,
+                            float *absmax, sq_stream stream)
+{
+    if (x == nullptr || gamma == nullptr || absmax == nullptr || !valid_dt(dt)) return SQ_ERR_INVALID_ARG;
+    if (M < 0 || d <= 0 || !(eps >= 0.0f)) return SQ_ERR_INVALID_ARG;
+    if (!aligned16(x)) return SQ_ERR_MISALIGNED;
+    RowArgs a{};
+    a.src0 = static_cast<const uint8_t *>(x);
+    a.rows = M;
+    a.K = d;
+    a.row_bytes = d * dtype_size(dt);
+    a.gamma = gamma;
+    a.eps = eps;
+    a.scale_out = absmax;
+    return launch_rows<ROW_RMS_STAT>(a, dt, as_stream(stream));
 }
 
 size_t sq_linear_workspace_size(int64_t M, int64_t N, int64_t K)

@@ -59,7 +59,8 @@ enum RowMode : int {
     ROW_WEIGHT = 0,      // W' = fl(w*s_j); per-row scale; codes
     ROW_ACT_STATIC = 1,  // x' = fl(x*fl(1/s_j)); codes with the given scale
     ROW_ACT_TOKEN = 2,   // x' as above; per-row scale written; codes
-    ROW_RMSNORM = 3      // y = fl(fl(x*r)*fl(gamma_j*fl(1/s_j))); codes with the given scale
+    ROW_RMSNORM = 3,     // y = fl(fl(x*r)*fl(gamma_j*fl(1/s_j))); codes with the given scale
+    ROW_RMS_STAT = 4     // running column max of |fl(fl(x*r)*gamma_j)| into scale_out[K] (no codes)
 };
 
 constexpr int ROW_T = 256;
@@ -99,6 +100,7 @@ __device__ __forceinline__ float column_constant(const RowArgs &p, int64_t j)
 {
     if constexpr (MODE == ROW_WEIGHT) return p.s[j];
     else if constexpr (MODE == ROW_RMSNORM) return __fmul_rn(p.gamma[j], recip_or_zero(p.s[j]));
+    else if constexpr (MODE == ROW_RMS_STAT) return p.gamma[j];
     else return recip_or_zero(p.s[j]);
 }
 
@@ -152,6 +154,14 @@ __global__ void __launch_bounds__(ROW_T) k_rows(RowArgs p)
     };
     float inv_a_static = 0.0f;
     if constexpr (MODE == ROW_ACT_STATIC || MODE == ROW_RMSNORM) inv_a_static = recip_or_zero(p.a_in[0]);
+    float cmax[MODE == ROW_RMS_STAT ? VPT : 1][MODE == ROW_RMS_STAT ? EPV : 1];
+    if constexpr (MODE == ROW_RMS_STAT) {
+        static_assert(REG, "the norm-output statistic keeps its column maxima in registers");
+#pragma unroll
+        for (int i = 0; i < VPT; ++i)
+#pragma unroll
+            for (int e = 0; e < EPV; ++e) cmax[i][e] = 0.0f;
+    }
 
     auto row_src = [&](int64_t row) -> const uint8_t * {
         if (p.src1 != nullptr) {          // gate/up interleave: blocks of 64 output rows
@@ -202,7 +212,7 @@ __global__ void __launch_bounds__(ROW_T) k_rows(RowArgs p)
             continue;
         }
 
-        if constexpr (MODE == ROW_RMSNORM) {
+        if constexpr (MODE == ROW_RMSNORM || MODE == ROW_RMS_STAT) {
             // pass 1: sum of squares in fp64 (exact squares)
             double ss = 0.0;
 #pragma unroll
@@ -226,10 +236,16 @@ __global__ void __launch_bounds__(ROW_T) k_rows(RowArgs p)
                     float f[EPV], c[EPV];
                     widen<DT>(raw[i], f);
                     colc(i, v, c);
+                    if constexpr (MODE == ROW_RMS_STAT) {
 #pragma unroll
-                    for (int e = 0; e < EPV; ++e)
-                        f[e] = __fmul_rn(__fmul_rn(__fmul_rn(f[e], r_m), c[e]), inv_a_static);
-                    store_codes<EPV>(dst, v, f);
+                        for (int e = 0; e < EPV; ++e)
+                            cmax[i][e] = fmaxf(cmax[i][e], fabsf(__fmul_rn(__fmul_rn(f[e], r_m), c[e])));
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < EPV; ++e)
+                            f[e] = __fmul_rn(__fmul_rn(__fmul_rn(f[e], r_m), c[e]), inv_a_static);
+                        store_codes<EPV>(dst, v, f);
+                    }
                 }
             }
             continue;
@@ -276,6 +292,17 @@ __global__ void __launch_bounds__(ROW_T) k_rows(RowArgs p)
             }
         }
     }
+    if constexpr (MODE == ROW_RMS_STAT) {
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int64_t v = static_cast<int64_t>(i) * ROW_T + tid;
+            if (v < nvec) {
+#pragma unroll
+                for (int e = 0; e < EPV; ++e)
+                    atomicMax(reinterpret_cast<int *>(p.scale_out + v * EPV + e), __float_as_int(cmax[i][e]));
+            }
+        }
+    }
 }
 
 // Unaligned / very wide rows: one block per row, elementwise, two passes
@@ -299,6 +326,7 @@ __global__ void __launch_bounds__(ROW_T) k_rows_scalar(RowArgs p, int dt)
         auto colc = [&](int64_t j) -> float {
             if constexpr (MODE == ROW_WEIGHT) return p.s[j];
             else if constexpr (MODE == ROW_RMSNORM) return __fmul_rn(p.gamma[j], recip_or_zero(p.s[j]));
+            else if constexpr (MODE == ROW_RMS_STAT) return p.gamma[j];
             else return recip_or_zero(p.s[j]);
         };
         float stat = 0.0f;
@@ -306,14 +334,15 @@ __global__ void __launch_bounds__(ROW_T) k_rows_scalar(RowArgs p, int dt)
         if constexpr (MODE != ROW_ACT_STATIC) {
             for (int64_t j = tid; j < p.K; j += ROW_T) {
                 const float x = load_elem_dt(src, dt, j);
-                if constexpr (MODE == ROW_RMSNORM) ss += static_cast<double>(x) * static_cast<double>(x);
+                if constexpr (MODE == ROW_RMSNORM || MODE == ROW_RMS_STAT)
+                    ss += static_cast<double>(x) * static_cast<double>(x);
                 else stat = fmaxf(stat, fabsf(__fmul_rn(x, colc(j))));
             }
         }
         float mul_a, r_m = 0.0f;
         if constexpr (MODE == ROW_ACT_STATIC) {
             mul_a = inv_a_static;
-        } else if constexpr (MODE == ROW_RMSNORM) {
+        } else if constexpr (MODE == ROW_RMSNORM || MODE == ROW_RMS_STAT) {
             const double tot = block_sum_f64(ss, red64);
             const float mean = __double2float_rn(tot / static_cast<double>(p.K));
             r_m = __frcp_rn(__fsqrt_rn(__fadd_rn(mean, p.eps)));
@@ -327,9 +356,12 @@ __global__ void __launch_bounds__(ROW_T) k_rows_scalar(RowArgs p, int dt)
         for (int64_t j = tid; j < p.K; j += ROW_T) {
             const float x = load_elem_dt(src, dt, j);
             float y;
-            if constexpr (MODE == ROW_RMSNORM) y = __fmul_rn(__fmul_rn(x, r_m), colc(j));
+            if constexpr (MODE == ROW_RMSNORM || MODE == ROW_RMS_STAT) y = __fmul_rn(__fmul_rn(x, r_m), colc(j));
             else y = __fmul_rn(x, colc(j));
-            p.out[row * p.K + j] = static_cast<int8_t>(quant8(__fmul_rn(y, mul_a)));
+            if constexpr (MODE == ROW_RMS_STAT)
+                atomicMax(reinterpret_cast<int *>(p.scale_out + j), __float_as_int(fabsf(y)));
+            else
+                p.out[row * p.K + j] = static_cast<int8_t>(quant8(__fmul_rn(y, mul_a)));
         }
         __syncthreads();
     }
