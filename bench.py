@@ -262,7 +262,7 @@ def run_gpu(args):
     def step(evs=None):
         def mark(i):
             if evs is not None:
-                evs[i].record(stream)
+                evs[i].record()          # the current stream: the capture stream while capturing
         i = 0
         mark(i)
         act_max.zero_()
@@ -300,15 +300,38 @@ def run_gpu(args):
     if sq.sync_status() != 0:
         raise RuntimeError("kernel error during warm-up")
 
-    # ---- timed region: K steps, per-kernel events on the launching stream
+    # ---- timed region: K steps, per-kernel events on the launching stream.
+    # The K steps are captured once into a CUDA graph (kernel nodes + event-record
+    # nodes) and launched as one graph, so host launch overhead is not on the
+    # device timeline; without --eager-steps a capture failure falls back to eager launches.
     nk = len(names)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(args.steps)]
+    graph = None
+    if not args.eager_steps:
+        try:
+            evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(nk + 1)]
+                   for _ in range(args.steps)]
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                for k in range(args.steps):
+                    step(evs[k])
+            graph.replay()                  # untimed: uploads the graph
+            torch.cuda.synchronize()
+            stream = torch.cuda.current_stream()
+        except Exception as exc:            # noqa: BLE001
+            print(f"graph capture failed ({exc}); timing eager launches", file=sys.stderr)
+            graph = None
+            torch.cuda.synchronize()
+    if graph is None:
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     with ClockSampler(local) as clk:
         t_start.record(stream)
-        for k in range(args.steps):
-            step(evs[k])
+        if graph is not None:
+            graph.replay()
+        else:
+            for k in range(args.steps):
+                step(evs[k])
         t_end.record(stream)
         barrier()
     st = sq.sync_status()
@@ -396,7 +419,8 @@ def run_gpu(args):
             "vs_baseline": None, "dtype": "s8", "data": "synthetic",
             "config": {"workload": WORKLOAD, "M": M_TOK, "K": K_IN, "N": N_OUT, "calib_tokens": CALIB_B * CALIB_R,
                        "alpha": ALPHA, "parallelism": f"dp{world} (token shards; all-reduce MAX of act_max)",
-                       "l2": "no flush: every step streams 384 MB of inputs (> 126 MB L2)"},
+                       "l2": "no flush: every step streams 384 MB of inputs (> 126 MB L2)",
+                       "launch": "K steps as one CUDA graph" if graph is not None else "eager"},
             "tokens_per_s": world * M_TOK / (ms_step * 1e-3),
             "roofline": roofline,
             "kernels": kern,
@@ -415,6 +439,181 @@ def run_gpu(args):
     return 0
 
 
+# --------------------------------------------------------------------------
+# Measurement of the other workloads (one JSON line each; not the bench line)
+# --------------------------------------------------------------------------
+def _time_ms(fn, iters, warmup=3, graph=True):
+    """Mean device time of fn() in ms.  With graph=True the call is captured once
+    in a CUDA graph and replayed, so host launch overhead is not counted."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    run = fn
+    if graph:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        run = g.replay
+        run()
+        torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(iters):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / iters
+
+
+def _dev16(bits, dt):
+    import numpy as np
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(dt).cuda()
+
+
+def run_workload(args):
+    import numpy as np
+    import torch
+    import synth
+    import w8a8_post_quantization_calib_b200 as sq
+
+    torch.cuda.set_device(0)
+    P = peaks()
+    out = {"workload": args.workload, "peaks": P}
+    bf16, f16 = torch.bfloat16, torch.float16
+    if args.workload == "mlp7b":
+        # per-token linear sweep, decode to prefill: the runtime quantisation + GEMM of one step
+        lines = []
+        for which in ("up", "down"):
+            wl = synth.mlp_7b(which, M=4096, calib_batches=4)
+            K, N = wl.K, wl.N
+            W = _dev16(wl.w, bf16)
+            am = torch.zeros(K, device="cuda")
+            sq.calib_absmax(_dev16(np.concatenate(wl.calib), bf16), am)
+            wm = torch.zeros(K, device="cuda")
+            sq.calib_absmax(W, wm)
+            s = torch.empty(K, device="cuda")
+            a = torch.empty(1, device="cuda")
+            sq.smooth_scales(am, wm, 0.5, s, a)
+            wq = torch.empty(N, K, dtype=torch.int8, device="cuda")
+            ws = torch.empty(N, device="cuda")
+            sq.quant_weight(W, s, wq, ws)
+            Xall = _dev16(wl.x, bf16)
+            for M in (1, 16, 128, 4096):
+                X = Xall[:M]
+                xq = torch.empty(M, K, dtype=torch.int8, device="cuda")
+                at = torch.empty(M, device="cuda")
+                y = torch.empty(M, N, dtype=bf16, device="cuda")
+                n = sq.linear_workspace_size(M, N, K)
+                work = torch.zeros(max(16, n), dtype=torch.uint8, device="cuda")
+                t_q = _time_ms(lambda: sq.smooth_quant_act(X, s, sq.ACT_PER_TOKEN, at, xq), 50)
+                t_g = _time_ms(lambda: sq.linear_w8a8(xq, wq, at, sq.ACT_PER_TOKEN, ws, y, workspace=work), 50)
+                ops = 2.0 * M * N * K
+                wbytes = N * K + N * 4 + M * K + M * N * 2
+                lines.append({"proj": which, "M": M, "K": K, "N": N,
+                              "act_quant_us": t_q * 1e3, "act_quant_gbs": M * K * 3 / (t_q * 1e-3) / 1e9,
+                              "gemm_us": t_g * 1e3, "gemm_tops": ops / (t_g * 1e-3) / 1e12,
+                              "gemm_frac_int8_peak": ops / (t_g * 1e-3) / 1e12 / P["int8_tops"],
+                              "gemm_gbs": wbytes / (t_g * 1e-3) / 1e9,
+                              "gemm_frac_hbm": wbytes / (t_g * 1e-3) / 1e9 / P["hbm_gbs"],
+                              "tokens_per_s": M / ((t_q + t_g) * 1e-3)})
+        out["lines"] = lines
+    elif args.workload == "alpha13b":
+        wl = synth.heavy_13b(M=8192)
+        K, N, M = wl.K, wl.N, wl.M
+        W = _dev16(wl.w, f16)
+        am = torch.zeros(K, device="cuda")
+        sq.calib_absmax(_dev16(np.concatenate(wl.calib), f16), am)
+        wm = torch.zeros(K, device="cuda")
+        sq.calib_absmax(W, wm)
+        held = _dev16(wl.calib[0], f16)
+        work = torch.zeros(sq.alpha_search_workspace_size(held.shape[0], N, K, 4), dtype=torch.uint8, device="cuda")
+        best = [None]
+
+        def search():
+            best[0] = sq.alpha_search(held, W, am, wm, work)
+        t_s = _time_ms(search, 5, warmup=1, graph=False)
+        al = best[0][0]
+        s = torch.empty(K, device="cuda")
+        a = torch.empty(1, device="cuda")
+        sq.smooth_scales(am, wm, al, s, a)
+        wq = torch.empty(N, K, dtype=torch.int8, device="cuda")
+        ws = torch.empty(N, device="cuda")
+        sq.quant_weight(W, s, wq, ws)
+        X = _dev16(wl.x, f16)
+        xq = torch.empty(M, K, dtype=torch.int8, device="cuda")
+        y = torch.empty(M, N, dtype=f16, device="cuda")
+        t_q = _time_ms(lambda: sq.smooth_quant_act(X, s, sq.ACT_STATIC, a, xq), 20)
+        t_g = _time_ms(lambda: sq.linear_w8a8(xq, wq, a, sq.ACT_STATIC, ws, y), 20)
+        yr = torch.empty(held.shape[0], N, dtype=f16, device="cuda")
+        t_r = _time_ms(lambda: sq.gemm_f16_ref(held, W, yr), 20)
+        ops = 2.0 * M * N * K
+        ops_h = 2.0 * held.shape[0] * N * K
+        out.update({"alpha": al, "mse": best[0][1], "search_ms": t_s,
+                    "search_note": "one f16 reference GEMM + 4 x (scales, weight quant, held-batch quant, INT8 GEMM, SSE) + host argmin",
+                    "ref_gemm_f16_us": t_r * 1e3, "ref_gemm_f16_tflops": ops_h / (t_r * 1e-3) / 1e12,
+                    "ref_gemm_f16_frac_bf16_peak": ops_h / (t_r * 1e-3) / 1e12 / (P["int8_tops"] / 2),
+                    "act_quant_us": t_q * 1e3, "act_quant_gbs": M * K * 3 / (t_q * 1e-3) / 1e9,
+                    "gemm_us": t_g * 1e3, "gemm_tops": ops / (t_g * 1e-3) / 1e12,
+                    "gemm_frac_int8_peak": ops / (t_g * 1e-3) / 1e12 / P["int8_tops"]})
+    elif args.workload == "mlp70b":
+        blk = synth.mlp_block_70b(calib_batches=1)
+        d, f, M = blk.d, blk.f, blk.M
+        g = torch.from_numpy(blk.gamma).cuda()
+        Wg, Wu, Wd = _dev16(blk.w_gate, bf16), _dev16(blk.w_up, bf16), _dev16(blk.w_down, bf16)
+        calib = _dev16(blk.calib[0], bf16)
+        am1 = torch.zeros(d, device="cuda")
+        t_stat = _time_ms(lambda: sq.rmsnorm_absmax(calib, g, blk.eps, am1), 10)
+        wm1 = torch.zeros(d, device="cuda")
+        sq.calib_absmax(Wg, wm1)
+        sq.calib_absmax(Wu, wm1)
+        s1 = torch.empty(d, device="cuda")
+        a1 = torch.empty(1, device="cuda")
+        sq.smooth_scales(am1, wm1, 0.5, s1, a1)
+        wq_gu = torch.empty(2 * f, d, dtype=torch.int8, device="cuda")
+        ws_gu = torch.empty(2 * f, device="cuda")
+        t_wgu = _time_ms(lambda: sq.quant_weight_gateup(Wg, Wu, s1, wq_gu, ws_gu), 5)
+        X = _dev16(blk.x, bf16)
+        xq = torch.empty(M, d, dtype=torch.int8, device="cuda")
+        h = torch.empty(M, f, dtype=bf16, device="cuda")
+        hq = torch.empty(M, f, dtype=torch.int8, device="cuda")
+        sq.rmsnorm_quant(X, g, s1, blk.eps, a1, xq)
+        sq.linear_w8a8_gateup_silu(xq[:2048], wq_gu, a1, sq.ACT_STATIC, ws_gu, h=h[:2048])
+        am2 = torch.zeros(f, device="cuda")
+        sq.calib_absmax(h[:2048], am2)
+        wm2 = torch.zeros(f, device="cuda")
+        sq.calib_absmax(Wd, wm2)
+        s2 = torch.empty(f, device="cuda")
+        a2 = torch.empty(1, device="cuda")
+        sq.smooth_scales(am2, wm2, 0.5, s2, a2)
+        wq_d = torch.empty(d, f, dtype=torch.int8, device="cuda")
+        ws_d = torch.empty(d, device="cuda")
+        sq.quant_weight(Wd, s2, wq_d, ws_d)
+        y = torch.empty(M, d, dtype=bf16, device="cuda")
+        t_n = _time_ms(lambda: sq.rmsnorm_quant(X, g, s1, blk.eps, a1, xq), 10)
+        t_gu = _time_ms(lambda: sq.linear_w8a8_gateup_silu(xq, wq_gu, a1, sq.ACT_STATIC, ws_gu, s2=s2, a2=a2, hq=hq), 5)
+        t_gu_h = _time_ms(lambda: sq.linear_w8a8_gateup_silu(xq, wq_gu, a1, sq.ACT_STATIC, ws_gu, h=h), 5)
+        t_d = _time_ms(lambda: sq.linear_w8a8(hq, wq_d, a2, sq.ACT_STATIC, ws_d, y), 5)
+        ops_gu, ops_d = 2.0 * M * 2 * f * d, 2.0 * M * d * f
+        t_blk = t_n + t_gu + t_d
+        out.update({"M": M, "d": d, "f": f,
+                    "block_ms": t_blk, "block_tokens_per_s": M / (t_blk * 1e-3),
+                    "block_tops": (ops_gu + ops_d) / (t_blk * 1e-3) / 1e12,
+                    "rmsnorm_quant_us": t_n * 1e3, "rmsnorm_quant_gbs": M * d * 3 / (t_n * 1e-3) / 1e9,
+                    "rmsnorm_absmax_us_per_2048_tokens": t_stat * 1e3,
+                    "rmsnorm_absmax_gbs": 2048 * d * 2 / (t_stat * 1e-3) / 1e9,
+                    "gateup_silu_requant_us": t_gu * 1e3, "gateup_tops": ops_gu / (t_gu * 1e-3) / 1e12,
+                    "gateup_frac_int8_peak": ops_gu / (t_gu * 1e-3) / 1e12 / P["int8_tops"],
+                    "gateup_silu_bf16_h_us": t_gu_h * 1e3,
+                    "down_us": t_d * 1e3, "down_tops": ops_d / (t_d * 1e-3) / 1e12,
+                    "down_frac_int8_peak": ops_d / (t_d * 1e-3) / 1e12 / P["int8_tops"],
+                    "weight_quant_gateup_us": t_wgu * 1e3,
+                    "weight_quant_gateup_gbs": 2 * f * d * 3 / (t_wgu * 1e-3) / 1e9})
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -424,11 +623,17 @@ def main():
     ap.add_argument("--cpu-frac", type=float, default=0.25,
                     help="fraction of the workload the CPU oracle baseline runs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager-steps", action="store_true",
+                    help="launch the timed steps one call at a time instead of as one captured CUDA graph")
+    ap.add_argument("--workload", choices=["qkv7b", "mlp7b", "alpha13b", "mlp70b"], default="qkv7b",
+                    help="qkv7b is the bench line; the others print per-kernel measurements of the other workloads")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload != "qkv7b":
+        return run_workload(args)
     return run_gpu(args)
 
 

@@ -205,11 +205,15 @@ sq_status sq_rmsnorm_absmax(const void *x, sq_dtype dt, int64_t M, int64_t d, co
  * w_scale: fp32 [N].  bias: [N] of out_dt, or NULL.  y: [M, N] of out_dt
  * (fp32/fp16/bf16), 16-byte aligned, N a multiple of 16.  M >= 1.
  * Runs on the 5th-generation tensor cores (tcgen05 kind::i8, TMA-fed shared
- * memory tiles, TMEM int32 accumulators).  Small M (<= 64 by default) takes a
- * weight-streaming path that may split K across CTAs; it then needs
- * `workspace` of sq_linear_workspace_size(M, N, K) bytes (16-byte aligned),
- * which it leaves zeroed for the next call.  The caller zeroes a new
- * workspace once (e.g. cudaMemsetAsync) before first use.
+ * memory tiles, TMEM int32 accumulators; CTA pairs with cta_group::2 for
+ * M > 128).  Small M (<= 128) takes a weight-streaming path (weights fill the
+ * 128-row MMA, tokens are its N) that splits K across CTAs when
+ * `workspace` holds sq_linear_workspace_size(M, N, K) bytes (16-byte
+ * aligned): one int32 partial-sum slice per split plus one arrival counter
+ * per tile.  The counters must be zero before the first use of a workspace
+ * (e.g. cudaMemsetAsync once) and are left zero by every call; the slices
+ * need no initialisation.  Without a workspace (NULL or too small) the small-M
+ * path runs unsplit.  Calls sharing one workspace must not overlap on the GPU.
  * ------------------------------------------------------------------------- */
 size_t sq_linear_workspace_size(int64_t M, int64_t N, int64_t K);
 
@@ -225,8 +229,9 @@ sq_status sq_linear_w8a8(const int8_t *xq, const int8_t *wq, int64_t M, int64_t 
  * that must not pay cudaMalloc's implicit device-wide synchronisation.  This
  * call takes no workspace: the small-M split-K path (M <= 128) keeps its
  * int32 partial sums and per-tile counters in a fixed array inside the
- * library (8 MiB of partial sums + 64 KiB of counters, held by every GPU that
- * loads the library until the process exits).  M*N beyond
+ * library (8 MiB of partial-sum slices + 64 KiB of counters, held by every
+ * GPU that loads the library until the process exits; the split count is
+ * capped by how many slices of M*N int32 fit).  M*N beyond
  * sq_linear_w8a8_noalloc_max_elems() (2^21 = 2097152) on that path returns
  * SQ_ERR_UNSUPPORTED without launching; M > 128 needs no scratch and runs the
  * sq_linear_w8a8 launch.  The call allocates nothing: no cudaMalloc,
@@ -234,8 +239,9 @@ sq_status sq_linear_w8a8(const int8_t *xq, const int8_t *wq, int64_t M, int64_t 
  *   - The first call on each device looks up the array's device address (with
  *     that device current) and caches it; make that first call before any
  *     stream capture.
- *   - Each call zeroes the part of the array it uses (stream-ordered memsets)
- *     before its kernel, since the array keeps the previous call's contents.
+ *   - Each call zeroes the arrival counters it uses (a stream-ordered memset)
+ *     before its kernel, since the array keeps the previous call's contents;
+ *     the partial-sum slices are fully rewritten by every call.
  *   - All calls on a device share the one array: calls that overlap on the
  *     GPU (different streams, no ordering between them) race and corrupt each
  *     other's results.  Serialise them on one stream or order them with events.

@@ -224,15 +224,14 @@ def test_linear_w8a8(M, N, K, out_dt, mode, with_bias, with_ws):
     if with_ws:
         n = sq.linear_workspace_size(M, N, K)
         work = torch.zeros(n, dtype=torch.uint8, device="cuda")
-    for _ in range(2):      # twice: the split-K workspace must come back zeroed
+    for _ in range(2):      # twice: the split-K arrival counters must come back reset
+        y.zero_()
         sq.linear_w8a8(dev(A), dev(B), dev(a), mode, dev(ws), y,
                        bias=dev(bias, out_dt) if with_bias else None, workspace=work)
-    _sync()
-    ref = oracle.dequant(acc_ref, a, mode, ws, out_dt, bias)
-    got = host(y)
-    assert bits_equal(got, ref), mismatch_report(got, ref)
-    if work is not None:
-        assert int(work.count_nonzero()) == 0
+        _sync()
+        ref = oracle.dequant(acc_ref, a, mode, ws, out_dt, bias)
+        got = host(y)
+        assert bits_equal(got, ref), mismatch_report(got, ref)
 
 
 # ------------------------------------------------------------------ a9
@@ -339,3 +338,28 @@ def test_rmsnorm_absmax(M, d, dt):
     _sync()
     ref = oracle.rmsnorm_absmax(X, gamma, 1e-5, dt)
     assert bits_equal(host(am), ref), mismatch_report(host(am), ref)
+
+
+@pytest.mark.parametrize("dt", [F32, BF16])
+def test_quant_tiny_rows_saturate_like_the_oracle(dt):
+    """Rows whose max gives a subnormal scale: codes still clamp to +-127 like the oracle's."""
+    K = 512
+    W = np.zeros((4, K), np.float32)
+    W[0, :] = 1e-39
+    W[0, 7] = -3e-39
+    W[1, 3] = 1e-44
+    W[2, :] = np.linspace(-1, 1, K)
+    Wd = synth.cast(W, dt)
+    s = np.ones(K, np.float32)
+    wq = torch.empty(4, K, dtype=torch.int8, device="cuda")
+    ws = torch.empty(4, dtype=torch.float32, device="cuda")
+    sq.quant_weight(dev(Wd, dt), dev(s), wq, ws)
+    xq = torch.empty(4, K, dtype=torch.int8, device="cuda")
+    at = torch.empty(4, dtype=torch.float32, device="cuda")
+    sq.smooth_quant_act(dev(Wd, dt), dev(s), oracle.PER_TOKEN, at, xq)
+    _sync()
+    wq_r, ws_r = oracle.quant_weight(Wd, s, dt)
+    xq_r, a_r = oracle.smooth_quant_act(Wd, s, oracle.PER_TOKEN, None, dt)
+    assert bits_equal(host(ws), ws_r) and bits_equal(host(at), a_r)
+    assert np.array_equal(host(wq), wq_r), mismatch_report(host(wq), wq_r)
+    assert np.array_equal(host(xq), xq_r), mismatch_report(host(xq), xq_r)

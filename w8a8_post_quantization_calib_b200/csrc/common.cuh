@@ -48,6 +48,12 @@ __device__ __forceinline__ uint32_t quant8_bits(float v)
     return __float_as_uint(__fadd_rn(c, 12582912.0f));
 }
 
+// quant8_bits for values already known to lie in [-127.5, 127.5): the
+// per-row (weight) and per-token codes, whose row maximum maps to
+// fl(m * fl(1 / fl(m / 127))) <= 127 * (1 + 3 * 2^-24) < 127.5, so the clamp
+// of quant8_bits cannot bind there.
+__device__ __forceinline__ uint32_t quant8_bits_inrange(float v) { return __float_as_uint(__fadd_rn(v, 12582912.0f)); }
+
 // low bytes of four quant8_bits results -> one packed word (byte 0 = a)
 __device__ __forceinline__ uint32_t pack4_bits(uint32_t a, uint32_t b, uint32_t c, uint32_t d)
 {

@@ -21,9 +21,10 @@
 // weights, B = activations (BN = 16..128 tokens), so the 128-row MMA is filled
 // with weight rows and the kernel streams the weight matrix; a TMEM lane is an
 // output channel, a column a token.  The swap path may split K across CTAs:
-// partial int32 sums are added (exact, order-free) into a workspace, and the
-// last CTA of a tile (a per-tile arrival counter) applies the epilogue and
-// re-zeroes the workspace.
+// each split stores its partial int32 sums into its own slice of a
+// workspace, and the last CTA of a tile (a per-tile arrival counter) adds the
+// slices in split order (exact integer sums), applies the epilogue and resets
+// the counter.
 //
 // Every mbarrier wait is bounded (ptx::wait_bounded): on expiry the kernel
 // records an error code, stops issuing, waits (bounded) for its own TMA loads
@@ -269,7 +270,7 @@ __device__ __forceinline__ void epilogue_normal(const Params &p, uint32_t tbase,
 // ---------------------------------------------------------------------------
 template <int BN, int EPI>
 __device__ __forceinline__ void epilogue_swap(const Params &p, uint32_t tbase, int tr, int tc, int tile,
-                                              int q, int lane, int *last_flag)
+                                              int split_idx, int q, int lane, int *last_flag)
 {
     constexpr int CW = TileCfg<BN>::CW;
     const int n = tr * BM + q * 32 + lane;
@@ -292,8 +293,8 @@ __device__ __forceinline__ void epilogue_swap(const Params &p, uint32_t tbase, i
             const int64_t o = static_cast<int64_t>(m) * p.N + n;
             if constexpr (EPI == EPI_S32) {
                 static_cast<int32_t *>(p.out)[o] = static_cast<int32_t>(r[i]);
-            } else if (split) {
-                ptx::red_add_s32(p.ws_acc + o, static_cast<int32_t>(r[i]));
+            } else if (split) {       // this split's partial sums: slice `split_idx` of the workspace
+                p.ws_acc[static_cast<int64_t>(split_idx) * p.M * p.N + o] = static_cast<int32_t>(r[i]);
             } else {
                 const float am = p.per_token ? p.a_scale[m] : p.a_scale[0];
                 store_out(p.out, p.out_dt, o, dequant(static_cast<int32_t>(r[i]), __fmul_rn(am, wsn), p.bias, bn));
@@ -314,13 +315,30 @@ __device__ __forceinline__ void epilogue_swap(const Params &p, uint32_t tbase, i
         if (*last_flag == 0) return;
         __threadfence();
         if (nok) {
+            // 8 tokens at a time so that 8 x splits independent loads are in flight
             const int mend = min(p.M, tc * BN + BN);
-            for (int m = tc * BN; m < mend; ++m) {
-                const int64_t o = static_cast<int64_t>(m) * p.N + n;
-                const int32_t acc = __ldcg(p.ws_acc + o);
-                p.ws_acc[o] = 0;
-                const float am = p.per_token ? p.a_scale[m] : p.a_scale[0];
-                store_out(p.out, p.out_dt, o, dequant(acc, __fmul_rn(am, wsn), p.bias, bn));
+            const int64_t slice = static_cast<int64_t>(p.M) * p.N;
+            for (int m0 = tc * BN; m0 < mend; m0 += 8) {
+                int32_t acc[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[j] = 0;
+                for (int sidx = 0; sidx < p.splits; ++sidx) {
+                    int32_t part[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        part[j] = (m0 + j < mend) ? __ldcg(p.ws_acc + sidx * slice + static_cast<int64_t>(m0 + j) * p.N + n) : 0;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) acc[j] += part[j];
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int m = m0 + j;
+                    if (m < mend) {
+                        const float am = p.per_token ? p.a_scale[m] : p.a_scale[0];
+                        store_out(p.out, p.out_dt, static_cast<int64_t>(m) * p.N + n,
+                                  dequant(acc[j], __fmul_rn(am, wsn), p.bias, bn));
+                    }
+                }
             }
         }
         ptx::named_bar_sync(1, 128);
@@ -481,7 +499,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ptx::tc_fence_after();
             const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * BN);
             if constexpr (SWAP)
-                epilogue_swap<BN, EPI>(p, tbase, tr, tc, tile, q, lane, last_flag);
+                epilogue_swap<BN, EPI>(p, tbase, tr, tc, tile, split, q, lane, last_flag);
             else
                 epilogue_normal<BN, KIND, EPI>(p, tbase, tr, tc, q, lane);
             ptx::tc_fence_before();

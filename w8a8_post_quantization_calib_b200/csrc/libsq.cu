@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <unordered_map>
 
 #include "sq.h"
 #include "common.cuh"
@@ -60,6 +61,34 @@ int sm_count()
 
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// Per (device, kernel): dynamic shared memory already granted, and the
+// occupancy figures the launch sizes its grid with.  Queried once.
+struct KernelInfo {
+    int smem_set = 0;
+    int per_sm = 0;
+    int clusters = 0;
+};
+std::unordered_map<uint64_t, KernelInfo> g_kinfo;
+
+KernelInfo &kinfo(const void *kern)
+{
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const uint64_t key = (static_cast<uint64_t>(dev) << 56) ^ reinterpret_cast<uint64_t>(kern);
+    return g_kinfo[key];
+}
+
+// Grants `smem` bytes of dynamic shared memory to `kern` (once per size increase).
+cudaError_t ensure_smem(const void *kern, int smem)
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    KernelInfo &ki = kinfo(kern);
+    if (ki.smem_set >= smem) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) ki.smem_set = smem;
+    return e;
+}
+
 // ------------------------------------------------------------------ TMA maps
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 {
@@ -103,7 +132,7 @@ sq_status launch_gemm(gemm::Params p, const void *a, const void *b, cudaStream_t
     if (!make_map(&ma, a, f16, p.K, p.rows_a, gemm::BM)) return SQ_ERR_CUDA;
     if (!make_map(&mb, b, f16, p.K, p.rows_b, BN)) return SQ_ERR_CUDA;
     auto kern = gemm::k_gemm<BN, KIND, EPI, SWAP>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), C::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_fail(e);
     p.timeout_ns = g_timeout_ns;
     const int grid = static_cast<int>(std::min<int64_t>(p.num_units, sm_count()));
@@ -150,13 +179,14 @@ sq_status launch_gemm2(gemm::Params p, const void *a, const void *b, cudaStream_
         if (!make_out_map(&mo, p.out, odt, EPI == gemm::EPI_S32, p.M, p.N)) return SQ_ERR_CUDA;
     }
     auto kern = gemm::k_gemm2<BN, KIND, EPI>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), C::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_fail(e);
-    static int max_clusters[kMaxDevices] = {0};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= kMaxDevices) dev = 0;
-    if (max_clusters[dev] == 0) {
+    int max_clusters = 0;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        max_clusters = kinfo(reinterpret_cast<const void *>(kern)).clusters;
+    }
+    if (max_clusters == 0) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2 * (sm_count() / 2), 1, 1);
         cfg.blockDim = dim3(gemm::NUM_THREADS, 1, 1);
@@ -165,10 +195,12 @@ sq_status launch_gemm2(gemm::Params p, const void *a, const void *b, cudaStream_
         if (cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void *>(kern), &cfg) != cudaSuccess || n <= 0)
             n = sm_count() / 2;
         cudaGetLastError();
-        max_clusters[dev] = n;
+        max_clusters = n;
+        std::lock_guard<std::mutex> lk(g_mu);
+        kinfo(reinterpret_cast<const void *>(kern)).clusters = n;
     }
     p.timeout_ns = g_timeout_ns;
-    const int clusters = static_cast<int>(std::min<int64_t>(p.num_units, max_clusters[dev]));
+    const int clusters = static_cast<int>(std::min<int64_t>(p.num_units, max_clusters));
     kern<<<2 * clusters, gemm::NUM_THREADS, C::SMEM_BYTES, st>>>(ma, mb, mo, p);
     return check_launch();
 }
@@ -190,11 +222,15 @@ int pick_pair_bn(int64_t M, int64_t N)
 {
     const int64_t clusters = std::max(1, sm_count() / 2);
     const int cands[3] = {256, 192, 128};
+    // measured time per output column of a full wave relative to the 256-wide
+    // tile (narrower tiles move more operand bytes per MAC)
+    const double eff[3] = {1.0, 0.93, 0.77};
     int best = 256;
-    int64_t best_cost = -1;
-    for (int bn : cands) {
+    double best_cost = -1.0;
+    for (int i = 0; i < 3; ++i) {
+        const int bn = cands[i];
         const int64_t tiles = cdiv(M, 2 * gemm::BM) * cdiv(N, bn);
-        const int64_t cost = cdiv(tiles, clusters) * bn;
+        const double cost = static_cast<double>(cdiv(tiles, clusters) * bn) / eff[i];
         if (best_cost < 0 || cost < best_cost) {
             best = bn;
             best_cost = cost;
@@ -235,27 +271,47 @@ int64_t swap_tiles(int64_t M, int64_t N) { return cdiv(N, gemm::BM) * cdiv(M, sw
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-size_t ws_bytes(int64_t M, int64_t N)
+// Split-K factor of the small-M path.  Every extra split costs a partial-sum
+// slice round trip and a short accumulator hand-off per unit, so K is split
+// only when the weight tiles alone leave most SMs idle (at most half as many
+// tiles as SMs) and the token tile is small (M <= 64); the units never exceed
+// the SM count.  Measured on the MLP-7B shapes: N=4096 (32 tiles) runs in
+// about half the time with 4 splits at M = 1..16; N=11008 (86 tiles) and
+// M = 128 are fastest unsplit.  max_splits caps it (fixed-size scratch).
+int choose_splits(int64_t M, int64_t N, int64_t K, int max_splits = 16)
+{
+    const int64_t tiles = swap_tiles(M, N);
+    const int64_t sms = sm_count();
+    const int64_t kb = cdiv(K, 128);
+    if (M > 64 || 2 * tiles > sms) return 1;
+    int64_t splits = std::min<int64_t>({sms / tiles, static_cast<int64_t>(max_splits), kb / 4, 8});
+    if (splits < 2) return 1;
+    const int64_t kps = cdiv(kb, splits);
+    return static_cast<int>(cdiv(kb, kps));
+}
+
+size_t ws_bytes_for(int64_t M, int64_t N, int splits)
+{
+    return align_up(static_cast<size_t>(splits) * static_cast<size_t>(M * N) * 4, 256) +
+           align_up(static_cast<size_t>(swap_tiles(M, N)) * 4, 256);
+}
+
+size_t ws_bytes(int64_t M, int64_t N, int64_t K)
 {
     if (M > kSwapMaxM) return 0;
-    return align_up(static_cast<size_t>(M * N) * 4, 256) + align_up(static_cast<size_t>(swap_tiles(M, N)) * 4, 256);
+    return ws_bytes_for(M, N, choose_splits(M, N, K));
 }
 
 template <int EPI>
-sq_status dispatch_swap(gemm::Params &p, const int8_t *xq, const int8_t *wq, cudaStream_t st)
+sq_status dispatch_swap(gemm::Params &p, const int8_t *xq, const int8_t *wq, cudaStream_t st, int splits = 1)
 {
     const int bn = swap_bn(p.M);
     fill_tiles(p, bn, p.N, p.M);
-    if (EPI == gemm::EPI_DEQUANT && p.ws_acc != nullptr) {
+    if (EPI == gemm::EPI_DEQUANT && p.ws_acc != nullptr && splits > 1) {
         const int tiles = p.num_units;
-        const int sms = sm_count();
-        if (tiles < sms) {
-            int splits = std::max(1, sms / tiles);
-            splits = std::min(splits, std::max(1, p.num_kb / 2));
-            p.kb_per_split = static_cast<int>(cdiv(p.num_kb, splits));
-            p.splits = static_cast<int>(cdiv(p.num_kb, p.kb_per_split));
-            p.num_units = tiles * p.splits;
-        }
+        p.kb_per_split = static_cast<int>(cdiv(p.num_kb, splits));
+        p.splits = static_cast<int>(cdiv(p.num_kb, p.kb_per_split));
+        p.num_units = tiles * p.splits;
     }
     if (p.splits == 1) {
         p.ws_acc = nullptr;
@@ -292,12 +348,22 @@ sq_status launch_rows_dt(RowArgs a, cudaStream_t st)
         else kern = k_rows<DT, 16, MODE>;
         cudaError_t e = cudaSuccess;
         if (smem > 48 * 1024) {
-            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+            e = ensure_smem(reinterpret_cast<const void *>(kern), static_cast<int>(smem));
             if (e != cudaSuccess) return cuda_fail(e);
         }
         int per_sm = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, ROW_T, smem);
-        if (e != cudaSuccess) return cuda_fail(e);
+        if (smem == 0) {      // occupancy does not depend on K: query once per kernel
+            std::lock_guard<std::mutex> lk(g_mu);
+            per_sm = kinfo(reinterpret_cast<const void *>(kern)).per_sm;
+        }
+        if (per_sm == 0) {
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, ROW_T, smem);
+            if (e != cudaSuccess) return cuda_fail(e);
+            if (smem == 0) {
+                std::lock_guard<std::mutex> lk(g_mu);
+                kinfo(reinterpret_cast<const void *>(kern)).per_sm = per_sm;
+            }
+        }
         const int64_t grid = std::min<int64_t>(a.rows, static_cast<int64_t>(sms) * std::max(1, per_sm));
         kern<<<static_cast<unsigned>(grid), ROW_T, smem, st>>>(a);
     } else {
@@ -444,8 +510,9 @@ sq_status sq_smooth_scales(const float *act_max, const float *w_max, int64_t K, 
     if (act_max == nullptr || w_max == nullptr || s == nullptr || K <= 0) return SQ_ERR_INVALID_ARG;
     if (!(alpha >= 0.0f && alpha <= 1.0f)) return SQ_ERR_INVALID_ARG;
     const cudaStream_t st = as_stream(stream);
-    if (K <= 256) {         // one block writes the static scale itself
-        k_smooth_scales<<<1, 256, 0, st>>>(act_max, w_max, K, alpha, s, a_static);
+    if (K <= 8 * 1024) {    // one cluster of 8 CTAs writes the static scale itself (no pre-zeroing)
+        const int threads = static_cast<int>(std::min<int64_t>(1024, ((cdiv(K, 8) + 31) / 32) * 32));
+        k_smooth_scales_cluster<<<8, threads, 0, st>>>(act_max, w_max, static_cast<int>(K), alpha, s, a_static);
         return check_launch();
     }
     if (a_static != nullptr) {
@@ -556,9 +623,8 @@ sq_status sq_rmsnorm_absmax(const void *x, sq_dtype dt, int64_t M, int64_t d, co
 
 size_t sq_linear_workspace_size(int64_t M, int64_t N, int64_t K)
 {
-    (void)K;
-    if (M <= 0 || N <= 0) return 0;
-    return ws_bytes(M, N);
+    if (M <= 0 || N <= 0 || K <= 0) return 0;
+    return ws_bytes(M, N, K);
 }
 
 static sq_status check_gemm_shape(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, int64_t K)
@@ -591,13 +657,15 @@ sq_status sq_linear_w8a8(const int8_t *xq, const int8_t *wq, int64_t M, int64_t 
     p.out = y;
     p.out_dt = out_dt;
     if (M <= kSwapMaxM) {
-        const size_t need = ws_bytes(M, N);
-        if (workspace != nullptr && workspace_bytes >= need && aligned16(workspace)) {
+        const int splits = choose_splits(M, N, K);
+        const size_t need = ws_bytes_for(M, N, splits);
+        if (splits > 1 && workspace != nullptr && workspace_bytes >= need && aligned16(workspace)) {
             p.ws_acc = static_cast<int32_t *>(workspace);
             p.ws_cnt = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) +
-                                               align_up(static_cast<size_t>(M * N) * 4, 256));
+                                               align_up(static_cast<size_t>(splits) * static_cast<size_t>(M * N) * 4, 256));
+            return dispatch_swap<gemm::EPI_DEQUANT>(p, xq, wq, st, splits);
         }
-        return dispatch_swap<gemm::EPI_DEQUANT>(p, xq, wq, st);
+        return dispatch_swap<gemm::EPI_DEQUANT>(p, xq, wq, st, 1);
     }
     return dispatch_pair<gemm::KIND_I8, gemm::EPI_DEQUANT>(p, xq, wq, st);
 }
@@ -615,18 +683,19 @@ sq_status sq_linear_w8a8_noalloc(const int8_t *xq, const int8_t *wq, int64_t M, 
     if (!aligned16(y) || !aligned16(w_scale)) return SQ_ERR_MISALIGNED;
     if (M > kSwapMaxM)      // the large-M path needs no scratch: same launch as sq_linear_w8a8
         return sq_linear_w8a8(xq, wq, M, N, K, a_scale, mode, w_scale, bias, out_dt, y, nullptr, 0, stream);
-    const size_t acc_bytes = static_cast<size_t>(M * N) * 4;
+    const size_t slice_bytes = static_cast<size_t>(M * N) * 4;
     const size_t cnt_bytes = static_cast<size_t>(swap_tiles(M, N)) * 4;
-    if (acc_bytes > kNoAllocAccBytes || cnt_bytes > kNoAllocCntBytes) return SQ_ERR_UNSUPPORTED;
+    if (slice_bytes > kNoAllocAccBytes || cnt_bytes > kNoAllocCntBytes) return SQ_ERR_UNSUPPORTED;
+    // as many K splits as the fixed array holds partial-sum slices for
+    const int splits = choose_splits(M, N, K, static_cast<int>(kNoAllocAccBytes / slice_bytes));
     void *scratch = nullptr;
     if ((r = noalloc_scratch(&scratch)) != SQ_OK) return r;
     int32_t *acc = static_cast<int32_t *>(scratch);
     int *cnt = reinterpret_cast<int *>(static_cast<unsigned char *>(scratch) + kNoAllocAccBytes);
     const cudaStream_t st = as_stream(stream);
-    // the array keeps whatever the previous call left: zero the part this call uses
-    cudaError_t e = cudaMemsetAsync(acc, 0, acc_bytes, st);
-    if (e != cudaSuccess) return cuda_fail(e);
-    e = cudaMemsetAsync(cnt, 0, cnt_bytes, st);
+    // the array keeps whatever the previous call left: the per-tile arrival
+    // counters must start at zero (the partial-sum slices are fully rewritten)
+    cudaError_t e = cudaMemsetAsync(cnt, 0, cnt_bytes, st);
     if (e != cudaSuccess) return cuda_fail(e);
     gemm::Params p{};
     p.M = static_cast<int>(M);
@@ -638,9 +707,9 @@ sq_status sq_linear_w8a8_noalloc(const int8_t *xq, const int8_t *wq, int64_t M, 
     p.bias = bias;
     p.out = y;
     p.out_dt = out_dt;
-    p.ws_acc = acc;
-    p.ws_cnt = cnt;
-    return dispatch_swap<gemm::EPI_DEQUANT>(p, xq, wq, st);
+    p.ws_acc = splits > 1 ? acc : nullptr;
+    p.ws_cnt = splits > 1 ? cnt : nullptr;
+    return dispatch_swap<gemm::EPI_DEQUANT>(p, xq, wq, st, splits);
 }
 
 sq_status sq_gemm_s32(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, int64_t K, int32_t *acc,
@@ -722,7 +791,7 @@ static size_t alpha_ws_layout(int64_t Mh, int64_t N, int64_t K, int n_alpha, siz
     off[5] = o; o = align_up(o + static_cast<size_t>(Mh * N) * 2, 256);     // y
     off[6] = o; o = align_up(o + static_cast<size_t>(Mh * N) * 2, 256);     // y_ref
     off[7] = o; o = align_up(o + static_cast<size_t>(n_alpha) * 8, 256);    // sse
-    const size_t lin = ws_bytes(Mh, N);
+    const size_t lin = ws_bytes(Mh, N, K);
     return o + lin;
 }
 
@@ -757,8 +826,8 @@ sq_status sq_alpha_search(const void *x_held, const void *w, int64_t M_held, int
     void *y = ws + off[5];
     void *y_ref = ws + off[6];
     double *sse = reinterpret_cast<double *>(ws + off[7]);
-    void *lin_ws = ws + (need - ws_bytes(M_held, N));
-    const size_t lin_bytes = ws_bytes(M_held, N);
+    void *lin_ws = ws + (need - ws_bytes(M_held, N, K));
+    const size_t lin_bytes = ws_bytes(M_held, N, K);
     const cudaStream_t st = as_stream(stream);
 
     sq_status r = sq_gemm_f16_ref(x_held, w, M_held, N, K, y_ref, stream);

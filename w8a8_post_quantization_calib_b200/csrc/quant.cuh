@@ -26,6 +26,51 @@ namespace sq {
 // with atomicMax on the (non-negative) float bits; *a_static is zeroed first.
 // A single-block launch (small K) writes the scale directly.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ float smoothing_factor(float act_max, float w_max, double al)
+{
+    const double a = fmax(static_cast<double>(act_max), 1e-5);
+    const double w = fmax(static_cast<double>(w_max), 1e-5);
+    // a^alpha / w^(1-alpha) = 2^(alpha log2 a - (1-alpha) log2 w): fp64 log2/exp2
+    // carry ~1e-15 relative error, far below the one fp32 rounding that follows
+    return static_cast<float>(exp2(al * log2(a) - (1.0 - al) * log2(w)));
+}
+
+// K <= 8 * 1024: one 8-CTA thread-block cluster, one channel per thread (the
+// fp64 log2/exp2 chains spread over 8 SMs).  Each CTA reduces its
+// fl(act_max_j * recip(s_j)) maximum into its shared memory; CTA 0 reads the 8
+// partial maxima through distributed shared memory and writes the static
+// scale, so no pre-zeroing and no atomics are needed.
+__global__ void __cluster_dims__(8, 1, 1) __launch_bounds__(1024)
+    k_smooth_scales_cluster(const float *__restrict__ act_max, const float *__restrict__ w_max, int K, float alpha,
+                            float *__restrict__ s, float *__restrict__ a_static)
+{
+    __shared__ float red[32];
+    __shared__ float cta_max;
+    const int j = blockIdx.x * blockDim.x + threadIdx.x;
+    float m = 0.0f;
+    if (j < K) {
+        const float am = act_max[j];
+        const float sj = smoothing_factor(am, w_max[j], static_cast<double>(alpha));
+        s[j] = sj;
+        m = __fmul_rn(am, recip_or_zero(sj));
+    }
+    m = block_max(m, red);
+    if (threadIdx.x == 0) cta_max = m;
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+    if (blockIdx.x == 0 && threadIdx.x < 32 && a_static != nullptr) {
+        float v = 0.0f;
+        if (threadIdx.x < 8) {
+            uint32_t local = static_cast<uint32_t>(__cvta_generic_to_shared(&cta_max)), remote;
+            asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(threadIdx.x));
+            asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+        }
+        v = warp_max(v);
+        if (threadIdx.x == 0) *a_static = scale_from_absmax(v);
+    }
+    // no CTA leaves while CTA 0 may still read its shared memory
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
 __global__ void __launch_bounds__(1024)
     k_smooth_scales(const float *__restrict__ act_max, const float *__restrict__ w_max, int64_t K,
                     float alpha, float *__restrict__ s, float *__restrict__ a_static)
@@ -35,11 +80,7 @@ __global__ void __launch_bounds__(1024)
     float m = 0.0f;
     for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < K;
          j += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const double a = fmax(static_cast<double>(act_max[j]), 1e-5);
-        const double w = fmax(static_cast<double>(w_max[j]), 1e-5);
-        // a^alpha / w^(1-alpha) = 2^(alpha log2 a - (1-alpha) log2 w): fp64 log2/exp2
-        // carry ~1e-15 relative error, far below the one fp32 rounding that follows
-        const float sj = static_cast<float>(exp2(al * log2(a) - (1.0 - al) * log2(w)));
+        const float sj = smoothing_factor(act_max[j], w_max[j], al);
         s[j] = sj;
         m = fmaxf(m, __fmul_rn(act_max[j], recip_or_zero(sj)));
     }
@@ -81,17 +122,18 @@ struct RowArgs {
 };
 
 // Codes of EPV values (already multiplied by the scale reciprocal) -> global.
-template <int EPV>
+// INRANGE: the values come from a per-row scale and cannot saturate.
+template <int EPV, bool INRANGE = false>
 __device__ __forceinline__ void store_codes(int8_t *dst_row, int64_t v, const float *f)
 {
+    auto q = [](float x) { return INRANGE ? quant8_bits_inrange(x) : quant8_bits(x); };
     if constexpr (EPV == 8) {
         uint2 o;
-        o.x = pack4_bits(quant8_bits(f[0]), quant8_bits(f[1]), quant8_bits(f[2]), quant8_bits(f[3]));
-        o.y = pack4_bits(quant8_bits(f[4]), quant8_bits(f[5]), quant8_bits(f[6]), quant8_bits(f[7]));
+        o.x = pack4_bits(q(f[0]), q(f[1]), q(f[2]), q(f[3]));
+        o.y = pack4_bits(q(f[4]), q(f[5]), q(f[6]), q(f[7]));
         *reinterpret_cast<uint2 *>(dst_row + v * 8) = o;
     } else {
-        *reinterpret_cast<uint32_t *>(dst_row + v * 4) =
-            pack4_bits(quant8_bits(f[0]), quant8_bits(f[1]), quant8_bits(f[2]), quant8_bits(f[3]));
+        *reinterpret_cast<uint32_t *>(dst_row + v * 4) = pack4_bits(q(f[0]), q(f[1]), q(f[2]), q(f[3]));
     }
 }
 
@@ -132,11 +174,24 @@ __global__ void __launch_bounds__(ROW_T) k_rows(RowArgs p)
             for (int e = 0; e < EPV; ++e) creg[i][e] = (v < nvec) ? column_constant<MODE>(p, v * EPV + e) : 0.0f;
         }
     } else {
+        // 8 columns per step: the loads of a step are independent and overlap
         float *cv = reinterpret_cast<float *>(colv4);
-        for (int64_t j = tid; j < p.K; j += ROW_T) {
-            const int64_t v = j / EPV;
-            const int e = static_cast<int>(j % EPV);
-            cv[((e >> 2) * plane + v) * 4 + (e & 3)] = column_constant<MODE>(p, j);
+        for (int64_t j0 = tid; j0 < p.K; j0 += 8 * ROW_T) {
+            float c[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int64_t j = j0 + static_cast<int64_t>(u) * ROW_T;
+                c[u] = (j < p.K) ? column_constant<MODE>(p, j) : 0.0f;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int64_t j = j0 + static_cast<int64_t>(u) * ROW_T;
+                if (j < p.K) {
+                    const int64_t v = j / EPV;
+                    const int e = static_cast<int>(j % EPV);
+                    cv[((e >> 2) * plane + v) * 4 + (e & 3)] = c[u];
+                }
+            }
         }
         __syncthreads();
     }
@@ -273,6 +328,8 @@ __global__ void __launch_bounds__(ROW_T) k_rows(RowArgs p)
         const float sc = scale_from_absmax(block_max(mx, red));
         const float inv = recip_or_zero(sc);
         if (tid == 0) p.scale_out[row] = sc;
+        // with a normal (or zero) scale the row's codes cannot saturate
+        const bool inrange = (sc == 0.0f) || (sc >= 1.17549435e-38f);
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
             const int64_t v = static_cast<int64_t>(i) * ROW_T + tid;
@@ -288,7 +345,8 @@ __global__ void __launch_bounds__(ROW_T) k_rows(RowArgs p)
 #pragma unroll
                     for (int e = 0; e < EPV; ++e) f[e] = __fmul_rn(__fmul_rn(f[e], c[e]), inv);
                 }
-                store_codes<EPV>(dst, v, f);
+                if (inrange) store_codes<EPV, true>(dst, v, f);
+                else store_codes<EPV, false>(dst, v, f);
             }
         }
     }
