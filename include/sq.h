@@ -81,6 +81,14 @@ int sq_last_cuda_error(void);
  * runs out records SQ_ERR_TIMEOUT and the kernel returns without hanging. */
 void sq_set_wait_timeout_ns(unsigned long long ns);
 
+/* Failure-detection test hook (off by default).  what = 1: in every GEMM
+ * launched afterwards, the producer warp of CTA 0 withholds its first
+ * pipeline stage (no arrival, no load), so the MMA warp's bounded wait on
+ * that stage runs out: the kernel records SQ_ERR_TIMEOUT, drains what it had
+ * in flight and returns, and the CUDA context stays usable.  what = 0 turns
+ * it off.  Nothing faults, traps or hangs. */
+void sq_debug_inject(int what);
+
 /* Synchronises `stream`, then returns SQ_ERR_TIMEOUT if any kernel of this
  * library recorded a barrier timeout on the current device since the last
  * check (and clears the record), SQ_ERR_CUDA if the stream reported an error,

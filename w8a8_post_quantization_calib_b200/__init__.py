@@ -32,7 +32,7 @@ _STATUS = {0: "SQ_OK", 1: "SQ_ERR_INVALID_ARG", 2: "SQ_ERR_UNSUPPORTED", 3: "SQ_
            4: "SQ_ERR_CUDA", 5: "SQ_ERR_TIMEOUT", 6: "SQ_ERR_WORKSPACE"}
 
 EXPORTS = (
-    "sq_status_string", "sq_last_cuda_error", "sq_set_wait_timeout_ns", "sq_sync_status",
+    "sq_status_string", "sq_last_cuda_error", "sq_set_wait_timeout_ns", "sq_debug_inject", "sq_sync_status",
     "sq_calib_absmax", "sq_smooth_scales", "sq_quant_weight", "sq_quant_weight_gateup",
     "sq_smooth_quant_act", "sq_rmsnorm_quant", "sq_rmsnorm_absmax", "sq_linear_workspace_size", "sq_linear_w8a8",
     "sq_linear_w8a8_noalloc", "sq_linear_w8a8_noalloc_max_elems",
@@ -60,6 +60,7 @@ def _load() -> ctypes.CDLL:
         "sq_status_string": (ctypes.c_char_p, [I]),
         "sq_last_cuda_error": (I, []),
         "sq_set_wait_timeout_ns": (None, [ctypes.c_ulonglong]),
+        "sq_debug_inject": (None, [I]),
         "sq_sync_status": (I, [P]),
         "sq_calib_absmax": (I, [P, I, I64, I64, I64, P, P]),
         "sq_smooth_scales": (I, [P, P, I64, F, P, P, P]),

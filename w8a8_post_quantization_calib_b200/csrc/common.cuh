@@ -20,6 +20,16 @@ __device__ unsigned int g_error_word;
 
 __device__ __forceinline__ void record_error(unsigned code) { atomicCAS(&g_error_word, 0u, code); }
 
+// Programmatic dependent launch.  Every kernel of this library is launched
+// with programmatic stream serialisation: it may start while the previous
+// kernel in the stream is finishing, runs its prologue, and must execute
+// pdl_wait() (all memory of the previous grid complete and visible) before
+// reading any global input.  pdl_launch_dependents() lets the next kernel
+// start its own prologue.  Both are no-ops when the launch was not
+// programmatic.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------------------
 // Canonical fp32 steps (round-to-nearest intrinsics so that nvcc never fuses
 // a product into a multiply-add).  Symmetric INT8 quantisation, zero point 0:

@@ -90,6 +90,7 @@ struct Params {
     const float *a2;           // gate/up: static scale of h [1]
     int8_t *hq;                // gate/up: codes of h [M, N/2] or null
     unsigned long long timeout_ns;
+    int inject;                // failure-detection test: 1 = CTA 0 withholds its first stage
 };
 
 __device__ __forceinline__ void decode_unit(const Params &p, int u, int &tr, int &tc, int &split, int &tile)
@@ -403,6 +404,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const uint64_t tmo = p.timeout_ns;
+    pdl_wait();                        // operands and scales come from the previous kernels
+    pdl_launch_dependents();
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
@@ -420,10 +423,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         ok = false;
                         break;
                     }
-                    ptx::mbar_arrive_expect_tx(full_bar(stage), C::STAGE_BYTES);
-                    const uint32_t sa = sbase + stage * C::STAGE_BYTES;
-                    ptx::tma_load_2d(sa, &map_a, full_bar(stage), kb * BKE, tr * BM);
-                    ptx::tma_load_2d(sa + C::A_BYTES, &map_b, full_bar(stage), kb * BKE, tc * BN);
+                    const bool withhold = p.inject == 1 && blockIdx.x == 0 && issued == 0;
+                    if (!withhold) {
+                        ptx::mbar_arrive_expect_tx(full_bar(stage), C::STAGE_BYTES);
+                        const uint32_t sa = sbase + stage * C::STAGE_BYTES;
+                        ptx::tma_load_2d(sa, &map_a, full_bar(stage), kb * BKE, tr * BM);
+                        ptx::tma_load_2d(sa + C::A_BYTES, &map_b, full_bar(stage), kb * BKE, tc * BN);
+                    }
                     ++issued;
                     if (++stage == S) { stage = 0; phase ^= 1u; }
                 }
@@ -698,6 +704,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const uint64_t tmo = p.timeout_ns;
+    pdl_wait();                        // operands and scales come from the previous kernels
+    pdl_launch_dependents();
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer (both CTAs)
@@ -713,12 +721,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                         ok = false;
                         break;
                     }
-                    if (leader) ptx::mbar_arrive_expect_tx(full_bar(stage), 2 * C::STAGE_BYTES);
-                    const uint32_t fb = ptx::map_to_rank(full_bar(stage), 0);
-                    const uint32_t sa = sbase + stage * C::STAGE_BYTES;
-                    ptx::tma_load_2d_pair(sa, &map_a, fb, kb * BKE, tr * (2 * BM) + static_cast<int>(rank) * BM);
-                    ptx::tma_load_2d_pair(sa + C::A_BYTES, &map_b, fb, kb * BKE,
-                                          tc * BN + static_cast<int>(rank) * (BN / 2));
+                    const bool withhold = p.inject == 1 && blockIdx.x == 0 && issued == 0;
+                    if (!withhold) {
+                        if (leader) ptx::mbar_arrive_expect_tx(full_bar(stage), 2 * C::STAGE_BYTES);
+                        const uint32_t fb = ptx::map_to_rank(full_bar(stage), 0);
+                        const uint32_t sa = sbase + stage * C::STAGE_BYTES;
+                        ptx::tma_load_2d_pair(sa, &map_a, fb, kb * BKE, tr * (2 * BM) + static_cast<int>(rank) * BM);
+                        ptx::tma_load_2d_pair(sa + C::A_BYTES, &map_b, fb, kb * BKE,
+                                              tc * BN + static_cast<int>(rank) * (BN / 2));
+                    }
                     ++issued;
                     if (++stage == S) { stage = 0; phase ^= 1u; }
                 }

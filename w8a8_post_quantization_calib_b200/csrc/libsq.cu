@@ -10,6 +10,7 @@
 #include <cstring>
 #include <mutex>
 #include <unordered_map>
+#include <utility>
 
 #include "sq.h"
 #include "common.cuh"
@@ -24,6 +25,7 @@ namespace {
 
 thread_local int t_last_cuda_error = 0;
 unsigned long long g_timeout_ns = 2000000000ull;   // bounded barrier waits: 2 s
+int g_inject = 0;                                  // failure-detection test knob
 
 constexpr int kMaxDevices = 64;
 int g_sm_count[kMaxDevices] = {0};
@@ -60,6 +62,24 @@ int sm_count()
 }
 
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Launch with programmatic stream serialisation (see pdl_wait in common.cuh):
+// the kernel may begin while the previous kernel of the stream drains.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // Per (device, kernel): dynamic shared memory already granted, and the
 // occupancy figures the launch sizes its grid with.  Queried once.
@@ -135,9 +155,10 @@ sq_status launch_gemm(gemm::Params p, const void *a, const void *b, cudaStream_t
     cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), C::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_fail(e);
     p.timeout_ns = g_timeout_ns;
+    p.inject = g_inject;
     const int grid = static_cast<int>(std::min<int64_t>(p.num_units, sm_count()));
-    kern<<<grid, gemm::NUM_THREADS, C::SMEM_BYTES, st>>>(ma, mb, p);
-    return check_launch();
+    e = launch_pdl(kern, dim3(grid), dim3(gemm::NUM_THREADS), C::SMEM_BYTES, st, ma, mb, p);
+    return e == cudaSuccess ? check_launch() : cuda_fail(e);
 }
 
 // CTA-pair launch: grid = 2 x (co-resident clusters, at most one per unit).
@@ -200,9 +221,10 @@ sq_status launch_gemm2(gemm::Params p, const void *a, const void *b, cudaStream_
         kinfo(reinterpret_cast<const void *>(kern)).clusters = n;
     }
     p.timeout_ns = g_timeout_ns;
+    p.inject = g_inject;
     const int clusters = static_cast<int>(std::min<int64_t>(p.num_units, max_clusters));
-    kern<<<2 * clusters, gemm::NUM_THREADS, C::SMEM_BYTES, st>>>(ma, mb, mo, p);
-    return check_launch();
+    e = launch_pdl(kern, dim3(2 * clusters), dim3(gemm::NUM_THREADS), C::SMEM_BYTES, st, ma, mb, mo, p);
+    return e == cudaSuccess ? check_launch() : cuda_fail(e);
 }
 
 void fill_tiles_pair(gemm::Params &p, int bn, int kb_bytes_per_elem)
@@ -365,10 +387,13 @@ sq_status launch_rows_dt(RowArgs a, cudaStream_t st)
             }
         }
         const int64_t grid = std::min<int64_t>(a.rows, static_cast<int64_t>(sms) * std::max(1, per_sm));
-        kern<<<static_cast<unsigned>(grid), ROW_T, smem, st>>>(a);
+        e = launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(ROW_T), smem, st, a);
+        if (e != cudaSuccess) return cuda_fail(e);
     } else {
         const int64_t grid = std::min<int64_t>(a.rows, static_cast<int64_t>(sms) * 8);
-        k_rows_scalar<MODE><<<static_cast<unsigned>(grid), ROW_T, 0, st>>>(a, DT);
+        const cudaError_t e = launch_pdl(k_rows_scalar<MODE>, dim3(static_cast<unsigned>(grid)), dim3(ROW_T), 0, st,
+                                         a, static_cast<int>(DT));
+        if (e != cudaSuccess) return cuda_fail(e);
     }
     return check_launch();
 }
@@ -446,6 +471,8 @@ int sq_last_cuda_error(void) { return t_last_cuda_error; }
 
 void sq_set_wait_timeout_ns(unsigned long long ns) { g_timeout_ns = ns > 0 ? ns : 2000000000ull; }
 
+void sq_debug_inject(int what) { g_inject = (what == 1) ? 1 : 0; }
+
 sq_status sq_sync_status(sq_stream stream)
 {
     cudaError_t e = cudaStreamSynchronize(as_stream(stream));
@@ -483,23 +510,26 @@ sq_status sq_calib_absmax(const void *x, sq_dtype dt, int64_t rows, int64_t cols
         const uint8_t *xb = static_cast<const uint8_t *>(x);
         const int64_t ldb = ld * elt;
         const bool stream_hint = rows * ldb > (int64_t(100) << 20);     // much larger than L2 share
+        cudaError_t e;
         if (stream_hint) {
-            if (dt == SQ_F32) k_colabsmax<DT_F32, true><<<grid, block, 0, st>>>(xb, rows, nvec, ldb, slab, absmax);
-            else if (dt == SQ_F16) k_colabsmax<DT_F16, true><<<grid, block, 0, st>>>(xb, rows, nvec, ldb, slab, absmax);
-            else k_colabsmax<DT_BF16, true><<<grid, block, 0, st>>>(xb, rows, nvec, ldb, slab, absmax);
+            if (dt == SQ_F32) e = launch_pdl(k_colabsmax<DT_F32, true>, grid, block, 0, st, xb, rows, nvec, ldb, slab, absmax);
+            else if (dt == SQ_F16) e = launch_pdl(k_colabsmax<DT_F16, true>, grid, block, 0, st, xb, rows, nvec, ldb, slab, absmax);
+            else e = launch_pdl(k_colabsmax<DT_BF16, true>, grid, block, 0, st, xb, rows, nvec, ldb, slab, absmax);
         } else {
-            if (dt == SQ_F32) k_colabsmax<DT_F32, false><<<grid, block, 0, st>>>(xb, rows, nvec, ldb, slab, absmax);
-            else if (dt == SQ_F16) k_colabsmax<DT_F16, false><<<grid, block, 0, st>>>(xb, rows, nvec, ldb, slab, absmax);
-            else k_colabsmax<DT_BF16, false><<<grid, block, 0, st>>>(xb, rows, nvec, ldb, slab, absmax);
+            if (dt == SQ_F32) e = launch_pdl(k_colabsmax<DT_F32, false>, grid, block, 0, st, xb, rows, nvec, ldb, slab, absmax);
+            else if (dt == SQ_F16) e = launch_pdl(k_colabsmax<DT_F16, false>, grid, block, 0, st, xb, rows, nvec, ldb, slab, absmax);
+            else e = launch_pdl(k_colabsmax<DT_BF16, false>, grid, block, 0, st, xb, rows, nvec, ldb, slab, absmax);
         }
+        if (e != cudaSuccess) return cuda_fail(e);
     } else {
         const int64_t gx = cdiv(cols, 256);
         int64_t gy = std::max<int64_t>(1, std::min<int64_t>(cdiv(rows, 64), cdiv(static_cast<int64_t>(sms) * 8, gx)));
         gy = std::min<int64_t>(gy, 65535);
         const int64_t slab = cdiv(rows, gy);
         gy = cdiv(rows, slab);
-        k_colabsmax_scalar<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), 256, 0, st>>>(
-            x, dt, rows, cols, ld, slab, absmax);
+        const cudaError_t e = launch_pdl(k_colabsmax_scalar, dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)),
+                                         dim3(256), 0, st, x, static_cast<int>(dt), rows, cols, ld, slab, absmax);
+        if (e != cudaSuccess) return cuda_fail(e);
     }
     return check_launch();
 }
@@ -512,8 +542,9 @@ sq_status sq_smooth_scales(const float *act_max, const float *w_max, int64_t K, 
     const cudaStream_t st = as_stream(stream);
     if (K <= 8 * 1024) {    // one cluster of 8 CTAs writes the static scale itself (no pre-zeroing)
         const int threads = static_cast<int>(std::min<int64_t>(1024, ((cdiv(K, 8) + 31) / 32) * 32));
-        k_smooth_scales_cluster<<<8, threads, 0, st>>>(act_max, w_max, static_cast<int>(K), alpha, s, a_static);
-        return check_launch();
+        const cudaError_t e = launch_pdl(k_smooth_scales_cluster, dim3(8), dim3(threads), 0, st, act_max, w_max,
+                                         static_cast<int>(K), alpha, s, a_static);
+        return e == cudaSuccess ? check_launch() : cuda_fail(e);
     }
     if (a_static != nullptr) {
         const cudaError_t e = cudaMemsetAsync(a_static, 0, sizeof(float), st);
@@ -521,7 +552,9 @@ sq_status sq_smooth_scales(const float *act_max, const float *w_max, int64_t K, 
     }
     // one channel per thread: the fp64 log2/exp2 chain is latency-bound
     const int64_t grid = std::max<int64_t>(2, cdiv(K, 128));
-    k_smooth_scales<<<static_cast<unsigned>(grid), 128, 0, st>>>(act_max, w_max, K, alpha, s, a_static);
+    const cudaError_t e = launch_pdl(k_smooth_scales, dim3(static_cast<unsigned>(grid)), dim3(128), 0, st, act_max,
+                                     w_max, K, alpha, s, a_static);
+    if (e != cudaSuccess) return cuda_fail(e);
     return check_launch();
 }
 
@@ -775,8 +808,9 @@ sq_status sq_sse_f16(const void *y, const void *y_ref, int64_t n, double *sse, s
     if (!aligned16(y) || !aligned16(y_ref)) return SQ_ERR_MISALIGNED;
     if (n == 0) return SQ_OK;
     const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(cdiv(n, 8 * 256), static_cast<int64_t>(sm_count()) * 4));
-    k_sse_f16<<<static_cast<unsigned>(grid), 256, 0, as_stream(stream)>>>(static_cast<const __half *>(y),
-                                                                       static_cast<const __half *>(y_ref), n, sse);
+    const cudaError_t e = launch_pdl(k_sse_f16, dim3(static_cast<unsigned>(grid)), dim3(256), 0, as_stream(stream),
+                                     static_cast<const __half *>(y), static_cast<const __half *>(y_ref), n, sse);
+    if (e != cudaSuccess) return cuda_fail(e);
     return check_launch();
 }
 

@@ -48,6 +48,8 @@ __global__ void __cluster_dims__(8, 1, 1) __launch_bounds__(1024)
     __shared__ float cta_max;
     const int j = blockIdx.x * blockDim.x + threadIdx.x;
     float m = 0.0f;
+    pdl_wait();
+    pdl_launch_dependents();
     if (j < K) {
         const float am = act_max[j];
         const float sj = smoothing_factor(am, w_max[j], static_cast<double>(alpha));
@@ -78,6 +80,8 @@ __global__ void __launch_bounds__(1024)
     __shared__ float red[32];
     const double al = static_cast<double>(alpha);
     float m = 0.0f;
+    pdl_wait();
+    pdl_launch_dependents();
     for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < K;
          j += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const float sj = smoothing_factor(act_max[j], w_max[j], al);
@@ -164,6 +168,8 @@ __global__ void __launch_bounds__(ROW_T) k_rows(RowArgs p)
     const int tid = threadIdx.x;
     const int64_t nvec = p.K / EPV;
     const int64_t plane = nvec;            // float4 entries per plane
+    pdl_wait();
+    pdl_launch_dependents();
 
     float creg[REG ? VPT : 1][REG ? EPV : 1];
     if constexpr (REG) {
@@ -371,6 +377,8 @@ __global__ void __launch_bounds__(ROW_T) k_rows_scalar(RowArgs p, int dt)
     __shared__ float red[32];
     __shared__ double red64[32];
     const int tid = threadIdx.x;
+    pdl_wait();
+    pdl_launch_dependents();
     float inv_a_static = 0.0f;
     if constexpr (MODE == ROW_ACT_STATIC || MODE == ROW_RMSNORM) inv_a_static = recip_or_zero(p.a_in[0]);
     for (int64_t row = blockIdx.x; row < p.rows; row += gridDim.x) {
@@ -434,6 +442,8 @@ __global__ void __launch_bounds__(256)
     __shared__ double red[8];
     double acc = 0.0;
     const int64_t nv = n / 8;
+    pdl_wait();
+    pdl_launch_dependents();
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < nv; v += stride) {
         const uint4 a = __ldg(reinterpret_cast<const uint4 *>(y) + v);
