@@ -23,6 +23,7 @@ instead, on a bounded sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import itertools
 import json
 import os
 import statistics
@@ -497,25 +498,30 @@ def run_gpu(args):
 # Measurement of the other workloads (one JSON line each; not the bench line)
 # --------------------------------------------------------------------------
 def _time_ms(fn, iters, warmup=3, graph=True):
-    """Mean device time of fn() in ms.  With graph=True the call is captured once
-    in a CUDA graph and replayed, so host launch overhead is not counted."""
+    """Mean device time of fn() in ms.  With graph=True, `iters` back-to-back calls
+    are captured into one CUDA graph (consecutive kernels overlap launch and
+    prologue through programmatic dependent launch, as a chain of layers would)
+    and the graph is launched once, so host launch overhead is not counted."""
     import torch
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
-    run = fn
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if graph:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            fn()
-        run = g.replay
-        run()
+            for _ in range(iters):
+                fn()
+        g.replay()
         torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(iters):
-        run()
-    e1.record()
+        e0.record()
+        g.replay()
+        e1.record()
+    else:
+        e0.record()
+        for _ in range(iters):
+            fn()
+        e1.record()
     torch.cuda.synchronize()
     return e0.elapsed_time(e1) / iters
 
@@ -539,7 +545,7 @@ def run_workload(args):
     if args.workload == "mlp7b":
         # per-token linear sweep, decode to prefill: the runtime quantisation + GEMM of one step
         lines = []
-        for which in ("up", "down"):
+        for which in args.proj.split(","):
             wl = synth.mlp_7b(which, M=4096, calib_batches=4)
             K, N = wl.K, wl.N
             W = _dev16(wl.w, bf16)
@@ -553,8 +559,12 @@ def run_workload(args):
             wq = torch.empty(N, K, dtype=torch.int8, device="cuda")
             ws = torch.empty(N, device="cuda")
             sq.quant_weight(W, s, wq, ws)
+            # a decode step reads each layer's weights once: the timed chain
+            # rotates over copies whose total exceeds the 126 MB L2, so every
+            # GEMM streams its weights from HBM
+            wcopies = [wq] + [wq.clone() for _ in range(max(1, -(-3 * 126 * 2**20 // (N * K))))]
             Xall = _dev16(wl.x, bf16)
-            for M in (1, 16, 128, 4096):
+            for M in (int(t) for t in args.tokens.split(",")):
                 X = Xall[:M]
                 xq = torch.empty(M, K, dtype=torch.int8, device="cuda")
                 at = torch.empty(M, device="cuda")
@@ -562,7 +572,9 @@ def run_workload(args):
                 n = sq.linear_workspace_size(M, N, K)
                 work = torch.zeros(max(16, n), dtype=torch.uint8, device="cuda")
                 t_q = _time_ms(lambda: sq.smooth_quant_act(X, s, sq.ACT_PER_TOKEN, at, xq), 50)
-                t_g = _time_ms(lambda: sq.linear_w8a8(xq, wq, at, sq.ACT_PER_TOKEN, ws, y, workspace=work), 50)
+                ctr = itertools.count()
+                t_g = _time_ms(lambda: sq.linear_w8a8(xq, wcopies[next(ctr) % len(wcopies)], at, sq.ACT_PER_TOKEN,
+                                                      ws, y, workspace=work), 50)
                 ops = 2.0 * M * N * K
                 wbytes = N * K + N * 4 + M * K + M * N * 2
                 lines.append({"proj": which, "M": M, "K": K, "N": N,
@@ -679,6 +691,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager-steps", action="store_true",
                     help="launch the timed steps one call at a time instead of as one captured CUDA graph")
+    ap.add_argument("--tokens", default="1,16,128,4096",
+                    help="mlp7b workload: comma-separated token counts M to sweep")
+    ap.add_argument("--proj", default="up,down", help="mlp7b workload: projections to sweep")
     ap.add_argument("--workload", choices=["qkv7b", "mlp7b", "alpha13b", "mlp70b"], default="qkv7b",
                     help="qkv7b is the bench line; the others print per-kernel measurements of the other workloads")
     args = ap.parse_args()

@@ -215,13 +215,17 @@ sq_status sq_rmsnorm_absmax(const void *x, sq_dtype dt, int64_t M, int64_t d, co
  * Runs on the 5th-generation tensor cores (tcgen05 kind::i8, TMA-fed shared
  * memory tiles, TMEM int32 accumulators; CTA pairs with cta_group::2 for
  * M > 128).  Small M (<= 128) takes a weight-streaming path (weights fill the
- * 128-row MMA, tokens are its N) that splits K across CTAs when
- * `workspace` holds sq_linear_workspace_size(M, N, K) bytes (16-byte
- * aligned): one int32 partial-sum slice per split plus one arrival counter
- * per tile.  The counters must be zero before the first use of a workspace
- * (e.g. cudaMemsetAsync once) and are left zero by every call; the slices
- * need no initialisation.  Without a workspace (NULL or too small) the small-M
- * path runs unsplit.  Calls sharing one workspace must not overlap on the GPU.
+ * 128-row MMA, tokens are its N).  When one 128-row weight tile per SM would
+ * leave many SMs idle, that path shares the (tile, K block) iterations evenly
+ * among the SMs (stream-K) if `workspace` holds sq_linear_workspace_size(M,
+ * N, K) bytes (16-byte aligned; the size depends on the current device's SM
+ * count and is 0 when no sharing is planned): one BM x BN int32 partial-sum
+ * slot per CTA plus one int32 arrival counter per weight tile.  The counters
+ * must be zero before the first use of a workspace (e.g. cudaMemsetAsync
+ * once) and are left zero by every call; the slots need no initialisation.
+ * Without a workspace (NULL or too small) the small-M path runs one tile per
+ * CTA.  Results are bit-identical either way (exact int32 sums).  Calls
+ * sharing one workspace must not overlap on the GPU.
  * ------------------------------------------------------------------------- */
 size_t sq_linear_workspace_size(int64_t M, int64_t N, int64_t K);
 
@@ -235,11 +239,12 @@ sq_status sq_linear_w8a8(const int8_t *xq, const int8_t *wq, int64_t M, int64_t 
  * all: a plugin running inside a host engine that owns every device buffer
  * and hands it only inputs and outputs, or a latency-critical serving loop
  * that must not pay cudaMalloc's implicit device-wide synchronisation.  This
- * call takes no workspace: the small-M split-K path (M <= 128) keeps its
+ * call takes no workspace: the small-M stream-K path (M <= 128) keeps its
  * int32 partial sums and per-tile counters in a fixed array inside the
- * library (8 MiB of partial-sum slices + 64 KiB of counters, held by every
- * GPU that loads the library until the process exits; the split count is
- * capped by how many slices of M*N int32 fit).  M*N beyond
+ * library (8 MiB of partial-sum slots + 64 KiB of counters, held by every
+ * GPU that loads the library until the process exits; the number of CTAs
+ * sharing the iterations is capped by how many slots fit, and the path runs
+ * one tile per CTA when too few fit).  M*N beyond
  * sq_linear_w8a8_noalloc_max_elems() (2^21 = 2097152) on that path returns
  * SQ_ERR_UNSUPPORTED without launching; M > 128 needs no scratch and runs the
  * sq_linear_w8a8 launch.  The call allocates nothing: no cudaMalloc,
@@ -247,9 +252,10 @@ sq_status sq_linear_w8a8(const int8_t *xq, const int8_t *wq, int64_t M, int64_t 
  *   - The first call on each device looks up the array's device address (with
  *     that device current) and caches it; make that first call before any
  *     stream capture.
- *   - Each call zeroes the arrival counters it uses (a stream-ordered memset)
- *     before its kernel, since the array keeps the previous call's contents;
- *     the partial-sum slices are fully rewritten by every call.
+ *   - Each call that shares tiles zeroes the arrival counters it uses (a
+ *     stream-ordered memset) before its kernel, since the array keeps the
+ *     previous call's contents; a partial-sum slot is always written before
+ *     it is read.
  *   - All calls on a device share the one array: calls that overlap on the
  *     GPU (different streams, no ordering between them) race and corrupt each
  *     other's results.  Serialise them on one stream or order them with events.

@@ -234,6 +234,39 @@ def test_linear_w8a8(M, N, K, out_dt, mode, with_bias, with_ws):
         assert bits_equal(got, ref), mismatch_report(got, ref)
 
 
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 11008), (16, 4096, 4096), (5, 1024, 4112), (32, 2048, 8192),
+                                   (17, 4096, 11008), (3, 256, 65536), (1, 11008, 4096), (33, 11008, 4112),
+                                   (100, 4096, 4096), (128, 18944, 256), (64, 1040, 528)])
+def test_linear_w8a8_stream_k(M, N, K):
+    """Small-M path with a workspace (the (tile, K block) iterations shared
+    evenly by the SMs, partial sums of shared tiles combined by the last CTA)
+    against the one-tile-per-CTA launch without one, bit for bit, twice (the
+    arrival counters must come back reset), and against the oracle on sampled
+    output channels (first, last and random rows of W)."""
+    g = np.random.default_rng(M * 5 + N + K)
+    A = g.integers(-127, 128, (M, K), dtype=np.int8)
+    B = g.integers(-127, 128, (N, K), dtype=np.int8)
+    a = (np.abs(g.standard_normal(M)) * 1e-2 + 1e-3).astype(np.float32)
+    ws = (np.abs(g.standard_normal(N)) * 1e-4 + 1e-5).astype(np.float32)
+    bias = synth.cast(g.standard_normal(N).astype(np.float32), BF16)
+    dA, dB, da, dws, db = dev(A), dev(B), dev(a), dev(ws), dev(bias, BF16)
+    y0 = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    sq.linear_w8a8(dA, dB, da, oracle.PER_TOKEN, dws, y0, bias=db)
+    n = sq.linear_workspace_size(M, N, K)
+    work = torch.zeros(max(16, n), dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        sq.linear_w8a8(dA, dB, da, oracle.PER_TOKEN, dws, y, bias=db, workspace=work)
+        _sync()
+        assert torch.equal(y.view(torch.int16), y0.view(torch.int16))
+    idx = np.unique(np.concatenate([np.arange(min(N, 160)), np.arange(max(0, N - 160), N),
+                                    g.integers(0, N, 64)]))
+    acc = oracle.gemm_s32(A, B[idx])
+    ref = oracle.dequant(acc, a, oracle.PER_TOKEN, ws[idx], BF16, bias[idx])
+    got = host(y)[:, idx]
+    assert bits_equal(got, ref), mismatch_report(got, ref)
+
+
 # ------------------------------------------------------------------ a9
 @pytest.mark.parametrize("M,Nh,K", [(300, 256, 512), (129, 384, 1040)])
 def test_gateup_silu(M, Nh, K):

@@ -16,15 +16,14 @@
 // TMEM holds two accumulators (2 x BN columns) so the epilogue of tile i
 // overlaps the mainloop of tile i+1.
 //
-// Orientation.  Normal: A = activations xq [M, K], B = weights wq [N, K]; a
-// TMEM lane is a token row, a column an output channel.  Swap (small M): A =
-// weights, B = activations (BN = 16..128 tokens), so the 128-row MMA is filled
-// with weight rows and the kernel streams the weight matrix; a TMEM lane is an
-// output channel, a column a token.  The swap path may split K across CTAs:
-// each split stores its partial int32 sums into its own slice of a
-// workspace, and the last CTA of a tile (a per-tile arrival counter) adds the
-// slices in split order (exact integer sums), applies the epilogue and resets
-// the counter.
+// Orientation.  Normal (CTA pairs, M > 128): A = activations xq [M, K], B =
+// weights wq [N, K]; a TMEM lane is a token row, a column an output channel.
+// Swap (small M): A = weights, B = activations (BN = 16..128 tokens), so the
+// 128-row MMA is filled with weight rows and the kernel streams the weight
+// matrix; a TMEM lane is an output channel, a column a token.  The swap kernel
+// spreads the (tile, K block) iterations evenly over the SMs (stream-K, see
+// k_gemm_swap), combining the partial sums of tiles shared by several CTAs
+// through a workspace.
 //
 // Every mbarrier wait is bounded (ptx::wait_bounded): on expiry the kernel
 // records an error code, stops issuing, waits (bounded) for its own TMA loads
@@ -57,10 +56,13 @@ __host__ __device__ constexpr int pow2_at_least(int v, int lo)
     return r;
 }
 
-template <int BN>
+// KBO: 128-byte K blocks per stage (one TMA load of each operand per stage)
+template <int BN, int KBO = 1>
 struct TileCfg {
-    static constexpr int A_BYTES = BM * BKB;
-    static constexpr int B_BYTES = BN * BKB;
+    static constexpr int A_KB = BM * BKB;          // one K block of A: a 128 x 128-byte swizzle tile
+    static constexpr int B_KB = BN * BKB;
+    static constexpr int A_BYTES = A_KB * KBO;
+    static constexpr int B_BYTES = B_KB * KBO;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int STAGES_RAW = SMEM_BUDGET / STAGE_BYTES;
     static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
@@ -76,16 +78,19 @@ struct Params {
     int rows_a, rows_b;        // rows of the A / B operand tensors
     int num_kb;                // K blocks of 128 bytes
     int tiles_r, tiles_c;      // tiles along A rows (BM) and B rows (BN)
-    int splits, kb_per_split;  // split-K (swap path only)
-    int num_units;             // tiles_r * tiles_c * splits
+    int splits, kb_per_split;  // CTA-pair path: always 1 / num_kb
+    int num_units;             // CTA-pair path: tiles_r * tiles_c
+    int sk_iters, sk_ctas;     // swap path: tiles * num_kb iterations shared by sk_ctas CTAs
+    int sk_slot;               // swap path: int32 per partial-sum slot (BM * BN)
+    int ring;                  // swap path: shared-memory stages in use (<= STAGES)
     const float *a_scale;      // [1] or [M]
     int per_token;
     const float *w_scale;      // [N]
     const void *bias;          // [N] of out_dt or null
     void *out;                 // [M, N] (gate/up: h [M, N/2] or null)
     int out_dt;
-    int32_t *ws_acc;           // split-K partial sums [M, N]
-    int *ws_cnt;               // split-K arrival counters [tiles]
+    int32_t *ws_acc;           // swap path: partial-sum slots [2 * sk_ctas][BN][BM]
+    int *ws_cnt;               // swap path: arrival counters [tiles]
     const float *s2;           // gate/up: smoothing of h [N/2]
     const float *a2;           // gate/up: static scale of h [1]
     int8_t *hq;                // gate/up: codes of h [M, N/2] or null
@@ -219,148 +224,232 @@ __device__ __forceinline__ void epilogue_normal(const Params &p, uint32_t tbase,
                 dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
             }
         }
-        return;
-    }
-
+    } else {
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        ptx::tmem_ld32(tbase + c * 32, r);
-        ptx::tmem_ld_wait();
-        const int n0 = tc * BN + c * 32;
-        if (n0 >= p.N || !mok) continue;
-        const int nval = min(32, p.N - n0);        // 16 or 32 (N is a multiple of 16)
-        const int64_t o = static_cast<int64_t>(m) * p.N + n0;
-        if constexpr (EPI == EPI_S32) {
-            int4 *dst = reinterpret_cast<int4 *>(static_cast<int32_t *>(p.out) + o);
+        for (int c = 0; c < BN / 32; ++c) {
+            uint32_t r[32];
+            ptx::tmem_ld32(tbase + c * 32, r);
+            ptx::tmem_ld_wait();
+            const int n0 = tc * BN + c * 32;
+            if (n0 >= p.N || !mok) continue;
+            const int nval = min(32, p.N - n0);        // 16 or 32 (N is a multiple of 16)
+            const int64_t o = static_cast<int64_t>(m) * p.N + n0;
+            if constexpr (EPI == EPI_S32) {
+                int4 *dst = reinterpret_cast<int4 *>(static_cast<int32_t *>(p.out) + o);
 #pragma unroll
-            for (int i = 0; i < 32; i += 4)
-                if (i < nval) dst[i / 4] = make_int4(r[i], r[i + 1], r[i + 2], r[i + 3]);
-        } else if constexpr (EPI == EPI_F16) {
-            float v[32];
+                for (int i = 0; i < 32; i += 4)
+                    if (i < nval) dst[i / 4] = make_int4(r[i], r[i + 1], r[i + 2], r[i + 3]);
+            } else if constexpr (EPI == EPI_F16) {
+                float v[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+                for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 #pragma unroll
-            for (int i = 0; i < 32; i += 8)
-                if (i < nval) store_out8(p.out, DT_F16, o + i, v + i);
-        } else {
-            float v[32];
+                for (int i = 0; i < 32; i += 8)
+                    if (i < nval) store_out8(p.out, DT_F16, o + i, v + i);
+            } else {
+                float v[32];
 #pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-                if (i < nval) {
-                    const float4 w4 = *reinterpret_cast<const float4 *>(p.w_scale + n0 + i);
-                    const float ws[4] = {w4.x, w4.y, w4.z, w4.w};
+                for (int i = 0; i < 32; i += 4) {
+                    if (i < nval) {
+                        const float4 w4 = *reinterpret_cast<const float4 *>(p.w_scale + n0 + i);
+                        const float ws[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        const float cc = __fmul_rn(am, ws[t]);
-                        v[i + t] = dequant(static_cast<int32_t>(r[i + t]), cc, p.bias,
-                                           load_bias(p.bias, p.out_dt, n0 + i + t));
+                        for (int t = 0; t < 4; ++t) {
+                            const float cc = __fmul_rn(am, ws[t]);
+                            v[i + t] = dequant(static_cast<int32_t>(r[i + t]), cc, p.bias,
+                                               load_bias(p.bias, p.out_dt, n0 + i + t));
+                        }
                     }
                 }
-            }
 #pragma unroll
-            for (int i = 0; i < 32; i += 8)
-                if (i < nval) store_out8(p.out, p.out_dt, o + i, v + i);
+                for (int i = 0; i < 32; i += 8)
+                    if (i < nval) store_out8(p.out, p.out_dt, o + i, v + i);
+            }
         }
     }
 }
 
 // ---------------------------------------------------------------------------
-// Epilogue of one unit, swap orientation (TMEM lane = output channel n,
-// column = token).  EPI_DEQUANT or EPI_S32 (no split for S32).
+// Small-M kernel: swap orientation (A = weights wq [N, K], B = activations
+// xq [M, K]; TMEM lane = output channel n, column = token), one persistent CTA
+// per SM on a stream-K schedule.
+//
+// The T = tiles * num_kb (tile, 128-byte K block) iterations are laid end to
+// end in tile order and CTA c of G takes iterations [floor(cT/G),
+// floor((c+1)T/G)), so every SM streams the same share of the weight bytes
+// whatever the tile count.  A CTA walks its share from the end to the start,
+// one segment per tile it touches.  A tile inside one CTA's share is finished
+// by that CTA.  A tile shared by CTAs c0 < ... < c1 is finished by its owner
+// c1, for which the tile's start is the start of its share, i.e. its last
+// segment; c0 reaches its part of the tile first and the middle CTAs (whose
+// whole share lies inside the tile) at their end.  Each non-owner stores its
+// int32 partial sums into its own slot of the workspace (a CTA is a non-owner
+// of at most one tile: the one its share ends in) and bumps the tile's
+// arrival counter with release semantics; the owner's epilogue warps, idle
+// while their own last segment streams, wait for the counter to reach
+// c1 - c0, add the slots into registers, and once their accumulator is ready
+// add it, apply the epilogue and reset the counter to zero.  A CTA waits only
+// for CTAs of lower index, which the hardware starts no later than itself, and
+// every wait is bounded.  The integer sums are exact, so the result does not
+// depend on G.  G = tiles gives the plain one-tile-per-CTA schedule, which
+// needs no workspace.
 // ---------------------------------------------------------------------------
-template <int BN, int EPI>
-__device__ __forceinline__ void epilogue_swap(const Params &p, uint32_t tbase, int tr, int tc, int tile,
-                                              int split_idx, int q, int lane, int *last_flag)
+__device__ __forceinline__ int sk_begin(const Params &p, int c)
+{
+    return static_cast<int>(static_cast<int64_t>(c) * p.sk_iters / p.sk_ctas);
+}
+
+// The CTA whose share holds iteration i: the largest c with sk_begin(c) <= i.
+__device__ __forceinline__ int sk_owner(const Params &p, int i)
+{
+    return static_cast<int>((static_cast<int64_t>(i + 1) * p.sk_ctas - 1) / p.sk_iters);
+}
+
+// One segment of a share walked backwards: iterations [lo, hi] of one tile.
+struct Seg {
+    int tile, kb_lo, kb_hi;
+};
+
+__device__ __forceinline__ Seg sk_segment(const Params &p, int it, int it_begin)
+{
+    Seg s;
+    s.tile = it / p.num_kb;
+    s.kb_hi = it - s.tile * p.num_kb;
+    s.kb_lo = max(0, s.kb_hi - (it - it_begin));
+    return s;
+}
+
+// acc[i] += slot_cc[(t0 + i) * BM + r] over the contributors' slots cc in
+// [c0, c1) for tokens t0 + i < mval; the loads of up to 64 / CW slots are in
+// flight together.
+template <int CW>
+__device__ __forceinline__ void add_slots(const Params &p, int32_t (&acc)[CW], int c0, int c1, int t0, int mval,
+                                          int r)
+{
+    constexpr int U = (64 / CW) > 1 ? 64 / CW : 1;
+    constexpr int64_t SLOT_STRIDE = BM;                // int32 per token row of a slot
+#pragma unroll 1
+    for (int cc = c0; cc < c1; cc += U) {
+        int32_t v[U][CW];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int32_t *sl = p.ws_acc + static_cast<int64_t>(cc + u) * p.sk_slot;
+#pragma unroll
+            for (int i = 0; i < CW; ++i)
+                v[u][i] = (cc + u < c1 && t0 + i < mval) ? __ldcg(sl + (t0 + i) * SLOT_STRIDE + r) : 0;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+#pragma unroll
+            for (int i = 0; i < CW; ++i) acc[i] += v[u][i];
+    }
+}
+
+// Epilogue of one segment.  q: TMEM lane quarter of this warp; row r = 32q +
+// lane of the weight tile is output channel n = tr*BM + r.  wsn / bn:
+// w_scale[n] and bias[n] (loaded before the accumulator is ready); s_am: the
+// token scales in shared memory.  tfull_wait() waits for the accumulator and
+// returns false on a timeout.
+template <int BN, int EPI, typename TfullWait>
+__device__ __forceinline__ bool epilogue_sk(const Params &p, uint32_t tbase, int tr, int tc, int tile, int q,
+                                            int lane, int *flag, volatile int *abort_flag, float wsn, float bn,
+                                            const float *s_am, TfullWait tfull_wait)
 {
     constexpr int CW = TileCfg<BN>::CW;
-    const int n = tr * BM + q * 32 + lane;
+    constexpr int64_t SLOT = static_cast<int64_t>(BM) * BN;
+    const int r = q * 32 + lane;
+    const int n = tr * BM + r;
     const bool nok = n < p.N;
-    const float wsn = nok ? p.w_scale[n] : 0.0f;
-    const float bn = (nok && p.bias != nullptr) ? load_bias(p.bias, p.out_dt, n) : 0.0f;
-    const bool split = p.splits > 1;
+    const int m0 = tc * BN;
+    const int mval = min(BN, p.M - m0);                 // valid tokens of this tile
+    auto emit = [&](int m, int32_t acc) {
+        const int64_t o = static_cast<int64_t>(m) * p.N + n;
+        if constexpr (EPI == EPI_S32) {
+            static_cast<int32_t *>(p.out)[o] = acc;
+        } else {
+            store_out(p.out, p.out_dt, o, dequant(acc, __fmul_rn(s_am[m - m0], wsn), p.bias, bn));
+        }
+    };
 
+    const int t0 = tile * p.num_kb;
+    const int c0 = sk_owner(p, t0), c1 = sk_owner(p, t0 + p.num_kb - 1);
+    const int me = static_cast<int>(blockIdx.x);
+    const bool shared = c0 != c1, owner = me == c1;
+
+    // the owner waits for the other contributors and pre-adds their slots
+    // for the first chunk while its own last segment is still streaming
+    int32_t pre[CW];
+#pragma unroll
+    for (int i = 0; i < CW; ++i) pre[i] = 0;
+    if (shared && owner) {
+        if (q == 2 && lane == 0) {
+            const bool ok = ptx::wait_count_bounded(p.ws_cnt + tile, c1 - c0, p.timeout_ns, abort_flag, ERR_EPI + 2);
+            if (ok) p.ws_cnt[tile] = 0;                 // every contributor has counted in: reset for the next call
+            *flag = ok ? 1 : 0;
+        }
+        ptx::named_bar_sync(1, 128);
+        if (*flag == 0) return tfull_wait();
+        ptx::fence_acq_rel_gpu();
+        add_slots<CW>(p, pre, c0, c1, 0, mval, r);
+    }
+    if (!tfull_wait()) return false;
+    ptx::tc_fence_after();
+
+    if (!shared || owner) {
+#pragma unroll 1
+        for (int c = 0; c < BN / CW; ++c) {
+            uint32_t v[32];
+            tmem_load_chunk(tbase + c * CW, v, CW);
+            ptx::tmem_ld_wait();
+            int32_t acc[CW];
+#pragma unroll
+            for (int i = 0; i < CW; ++i) acc[i] = static_cast<int32_t>(v[i]);
+            if (shared) {
+                if (c == 0) {
+#pragma unroll
+                    for (int i = 0; i < CW; ++i) acc[i] += pre[i];
+                } else {
+                    add_slots<CW>(p, acc, c0, c1, c * CW, mval, r);
+                }
+            }
+            if (!nok) continue;
+#pragma unroll
+            for (int i = 0; i < CW; ++i)
+                if (c * CW + i < mval) emit(m0 + c * CW + i, acc[i]);
+        }
+        return true;
+    }
+
+    // non-owner: publish the partial sums (slot layout [token][BM]) and count in
+    int32_t *mine = p.ws_acc + static_cast<int64_t>(me) * SLOT;
 #pragma unroll 1
     for (int c = 0; c < BN / CW; ++c) {
-        uint32_t r[32];
-        tmem_load_chunk(tbase + c * CW, r, CW);
+        uint32_t v[32];
+        tmem_load_chunk(tbase + c * CW, v, CW);
         ptx::tmem_ld_wait();
-        const int m0 = tc * BN + c * CW;
-        if (!nok) continue;
 #pragma unroll
-        for (int i = 0; i < CW; ++i) {
-            const int m = m0 + i;
-            if (m >= p.M) break;
-            const int64_t o = static_cast<int64_t>(m) * p.N + n;
-            if constexpr (EPI == EPI_S32) {
-                static_cast<int32_t *>(p.out)[o] = static_cast<int32_t>(r[i]);
-            } else if (split) {       // this split's partial sums: slice `split_idx` of the workspace
-                p.ws_acc[static_cast<int64_t>(split_idx) * p.M * p.N + o] = static_cast<int32_t>(r[i]);
-            } else {
-                const float am = p.per_token ? p.a_scale[m] : p.a_scale[0];
-                store_out(p.out, p.out_dt, o, dequant(static_cast<int32_t>(r[i]), __fmul_rn(am, wsn), p.bias, bn));
-            }
-        }
+        for (int i = 0; i < CW; ++i)
+            if (c * CW + i < mval) __stcg(mine + (c * CW + i) * BM + r, static_cast<int32_t>(v[i]));
     }
-    if constexpr (EPI == EPI_DEQUANT) {
-        if (!split) return;
-        // arrival: the last split of this tile applies the epilogue
-        __threadfence();
-        ptx::named_bar_sync(1, 128);
-        if (q == 2 && lane == 0) {       // first epilogue thread (warp 2)
-            __threadfence();
-            const int prev = atomicAdd(p.ws_cnt + tile, 1);
-            *last_flag = (prev == p.splits - 1) ? 1 : 0;
-        }
-        ptx::named_bar_sync(1, 128);
-        if (*last_flag == 0) return;
-        __threadfence();
-        if (nok) {
-            // 8 tokens at a time so that 8 x splits independent loads are in flight
-            const int mend = min(p.M, tc * BN + BN);
-            const int64_t slice = static_cast<int64_t>(p.M) * p.N;
-            for (int m0 = tc * BN; m0 < mend; m0 += 8) {
-                int32_t acc[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) acc[j] = 0;
-                for (int sidx = 0; sidx < p.splits; ++sidx) {
-                    int32_t part[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        part[j] = (m0 + j < mend) ? __ldcg(p.ws_acc + sidx * slice + static_cast<int64_t>(m0 + j) * p.N + n) : 0;
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) acc[j] += part[j];
-                }
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int m = m0 + j;
-                    if (m < mend) {
-                        const float am = p.per_token ? p.a_scale[m] : p.a_scale[0];
-                        store_out(p.out, p.out_dt, static_cast<int64_t>(m) * p.N + n,
-                                  dequant(acc[j], __fmul_rn(am, wsn), p.bias, bn));
-                    }
-                }
-            }
-        }
-        ptx::named_bar_sync(1, 128);
-        if (q == 2 && lane == 0) {
-            p.ws_cnt[tile] = 0;
-            *last_flag = 0;
-        }
-    }
+    ptx::fence_acq_rel_gpu();
+    ptx::named_bar_sync(1, 128);
+    if (q == 2 && lane == 0) ptx::red_add_release_gpu(p.ws_cnt + tile, 1);
+    return true;
 }
 
-// ---------------------------------------------------------------------------
-// The kernel
-// ---------------------------------------------------------------------------
-template <int BN, int KIND, int EPI, bool SWAP>
+// KBO = 1: 2D maps over wq [N, K] and xq [M, K] (any K, ragged last block
+// zero-filled); KBO > 1: 3D maps viewing them as [K/128][rows][128 bytes]
+// (K a multiple of 128), so that one TMA load brings KBO K blocks (one
+// 128-row swizzle tile each) -- a single CTA streams far more bytes per
+// second with fewer, larger loads.  An iteration is then a group of KBO
+// blocks; blocks past K are zero-filled.
+template <int BN, int EPI, int KBO>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-    k_gemm(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b, const Params p)
+    k_gemm_swap(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x, const Params p)
 {
-    using C = TileCfg<BN>;
+    using C = TileCfg<BN, KBO>;
     constexpr int S = C::STAGES;
-    constexpr int BKE = (KIND == KIND_I8) ? BKB : BKB / 2;       // K elements per stage
-    constexpr uint32_t IDESC = (KIND == KIND_I8) ? ptx::idesc_i8(BN) : ptx::idesc_f16(BN);
+    constexpr uint32_t IDESC = ptx::idesc_i8(BN);
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -373,8 +462,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t done_bar = bar0 + 8u * (2 * S + 4);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 5);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    int *last_flag = reinterpret_cast<int *>(tmem_slot + 2);
+    int *flag = reinterpret_cast<int *>(tmem_slot + 2);
+    __shared__ float s_am[BN];
     const uint32_t sbase = ptx::smem_addr(smem);
+    const int ring = (p.ring >= 2 && p.ring <= S) ? p.ring : S;   // stages in use
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -388,12 +479,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         ptx::mbar_init(done_bar, 1);
         *abort_flag = 0;
-        *last_flag = 0;
+        *flag = 0;
         ptx::fence_barrier_init();
     }
     if (warp == 0 && lane == 0) {
-        ptx::tma_prefetch_desc(&map_a);
-        ptx::tma_prefetch_desc(&map_b);
+        ptx::tma_prefetch_desc(&map_w);
+        ptx::tma_prefetch_desc(&map_x);
     }
     if (warp == 1) {
         ptx::tmem_alloc(ptx::smem_addr(tmem_slot), C::TMEM_COLS);
@@ -404,6 +495,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const uint64_t tmo = p.timeout_ns;
+    const int it_begin = sk_begin(p, blockIdx.x), it_end = sk_begin(p, blockIdx.x + 1);
     pdl_wait();                        // operands and scales come from the previous kernels
     pdl_launch_dependents();
 
@@ -412,35 +504,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (lane == 0) {
             int stage = 0, issued = 0;
             uint32_t phase = 0;
-            for (int u = blockIdx.x; u < p.num_units && !*abort_flag; u += gridDim.x) {
-                int tr, tc, split, tile;
-                decode_unit(p, u, tr, tc, split, tile);
-                const int kb0 = split * p.kb_per_split;
-                const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
-                bool ok = true;
-                for (int kb = kb0; kb < kb1; ++kb) {
-                    if (!ptx::wait_bounded(empty_bar(stage), phase ^ 1u, tmo, abort_flag, ERR_PRODUCER)) {
-                        ok = false;
-                        break;
+            for (int it = it_end - 1; it >= it_begin && !*abort_flag; --it) {
+                const int tile = it / p.num_kb, kb = it - tile * p.num_kb;
+                const int tr = tile / p.tiles_c, tc = tile - tr * p.tiles_c;
+                if (!ptx::wait_bounded(empty_bar(stage), phase ^ 1u, tmo, abort_flag, ERR_PRODUCER)) break;
+                const bool withhold = p.inject == 1 && blockIdx.x == 0 && issued == 0;
+                if (!withhold) {
+                    ptx::mbar_arrive_expect_tx(full_bar(stage), C::STAGE_BYTES);
+                    const uint32_t sa = sbase + stage * C::STAGE_BYTES;
+                    if constexpr (KBO == 1) {
+                        ptx::tma_load_2d(sa, &map_w, full_bar(stage), kb * BKB, tr * BM);
+                        ptx::tma_load_2d(sa + C::A_BYTES, &map_x, full_bar(stage), kb * BKB, tc * BN);
+                    } else {
+                        ptx::tma_load_3d(sa, &map_w, full_bar(stage), 0, tr * BM, kb * KBO);
+                        ptx::tma_load_3d(sa + C::A_BYTES, &map_x, full_bar(stage), 0, tc * BN, kb * KBO);
                     }
-                    const bool withhold = p.inject == 1 && blockIdx.x == 0 && issued == 0;
-                    if (!withhold) {
-                        ptx::mbar_arrive_expect_tx(full_bar(stage), C::STAGE_BYTES);
-                        const uint32_t sa = sbase + stage * C::STAGE_BYTES;
-                        ptx::tma_load_2d(sa, &map_a, full_bar(stage), kb * BKE, tr * BM);
-                        ptx::tma_load_2d(sa + C::A_BYTES, &map_b, full_bar(stage), kb * BKE, tc * BN);
-                    }
-                    ++issued;
-                    if (++stage == S) { stage = 0; phase ^= 1u; }
                 }
-                if (!ok) break;
+                ++issued;
+                if (++stage == ring) { stage = 0; phase ^= 1u; }
             }
             // drain: every issued load lands before the CTA exits
-            const int n_wait = issued < S ? issued : S;
+            const int n_wait = issued < ring ? issued : ring;
             for (int i = 0; i < n_wait; ++i) {
                 int s = stage - 1 - i;
                 uint32_t ph = phase;
-                if (s < 0) { s += S; ph ^= 1u; }
+                if (s < 0) { s += ring; ph ^= 1u; }
                 volatile int no_abort = 0;
                 ptx::wait_bounded(full_bar(s), ph, tmo, &no_abort, ERR_DRAIN);
             }
@@ -450,39 +538,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (lane == 0) {
             int stage = 0, local = 0;
             uint32_t phase = 0;
-            for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++local) {
-                int tr, tc, split, tile;
-                decode_unit(p, u, tr, tc, split, tile);
-                const int kb0 = split * p.kb_per_split;
-                const int kb1 = min(p.num_kb, kb0 + p.kb_per_split);
+            bool ok = true;
+            for (int it = it_end - 1; it >= it_begin && ok; ++local) {
+                const Seg sg = sk_segment(p, it, it_begin);
                 const int b = local & 1;
                 const uint32_t use = static_cast<uint32_t>(local >> 1) & 1u;
                 if (!ptx::wait_bounded(tempty_bar(b), use ^ 1u, tmo, abort_flag, ERR_MMA)) break;
                 ptx::tc_fence_after();
                 const uint32_t d = tmem_base + static_cast<uint32_t>(b * BN);
-                bool ok = true;
-                for (int kb = kb0; kb < kb1; ++kb) {
+                for (int kb = sg.kb_hi; kb >= sg.kb_lo; --kb) {
                     if (!ptx::wait_bounded(full_bar(stage), phase, tmo, abort_flag, ERR_MMA + 1)) {
                         ok = false;
                         break;
                     }
                     ptx::tc_fence_after();
                     const uint32_t sa = sbase + stage * C::STAGE_BYTES;
-                    const uint64_t ad = ptx::sdesc_kmajor_sw128(sa);
-                    const uint64_t bd = ptx::sdesc_kmajor_sw128(sa + C::A_BYTES);
 #pragma unroll
-                    for (int k = 0; k < BKB / 32; ++k) {
-                        const uint32_t acc = (kb > kb0 || k > 0) ? 1u : 0u;
-                        if constexpr (KIND == KIND_I8)
-                            ptx::mma_i8(d, ad + 2 * k, bd + 2 * k, IDESC, acc);
-                        else
-                            ptx::mma_f16(d, ad + 2 * k, bd + 2 * k, IDESC, acc);
+                    for (int j = 0; j < KBO; ++j) {
+                        const uint64_t ad = ptx::sdesc_kmajor_sw128(sa + j * C::A_KB);
+                        const uint64_t bd = ptx::sdesc_kmajor_sw128(sa + C::A_BYTES + j * C::B_KB);
+#pragma unroll
+                        for (int k = 0; k < BKB / 32; ++k)
+                            ptx::mma_i8(d, ad + 2 * k, bd + 2 * k, IDESC, (kb < sg.kb_hi || j > 0 || k > 0) ? 1u : 0u);
                     }
                     ptx::tc_commit(empty_bar(stage));
-                    if (++stage == S) { stage = 0; phase ^= 1u; }
+                    if (++stage == ring) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
                 ptx::tc_commit(tfull_bar(b));
+                it -= sg.kb_hi - sg.kb_lo + 1;
             }
             // drain: all issued MMAs complete before TMEM is released
             ptx::tc_commit(done_bar);
@@ -492,28 +576,48 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     } else {
         // ------------------------------------------------ epilogue (warps 2..5)
         const int q = warp & 3;
+        if constexpr (EPI == EPI_DEQUANT) {
+            // the token scales of the (single) token tile, staged once
+            const int t = threadIdx.x - 64;
+            for (int m = t; m < BN; m += 128) {
+                const int mg = min(m, p.M - 1);
+                s_am[m] = p.per_token ? p.a_scale[mg] : p.a_scale[0];
+            }
+            ptx::named_bar_sync(1, 128);
+        }
         int local = 0;
-        for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++local) {
-            int tr, tc, split, tile;
-            decode_unit(p, u, tr, tc, split, tile);
+        for (int it = it_end - 1; it >= it_begin; ++local) {
+            const Seg sg = sk_segment(p, it, it_begin);
+            const int tr = sg.tile / p.tiles_c, tc = sg.tile - tr * p.tiles_c;
             const int b = local & 1;
             const uint32_t use = static_cast<uint32_t>(local >> 1) & 1u;
-            int ok = 1;
-            if (lane == 0) ok = ptx::wait_bounded(tfull_bar(b), use, tmo, abort_flag, ERR_EPI) ? 1 : 0;
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) break;
-            ptx::tc_fence_after();
+            float wsn = 0.0f, bn = 0.0f;
+            if constexpr (EPI == EPI_DEQUANT) {
+                const int n = tr * BM + q * 32 + lane;
+                if (n < p.N) {
+                    wsn = p.w_scale[n];
+                    bn = load_bias(p.bias, p.out_dt, n);
+                }
+            }
+            auto tfull_wait = [&]() {
+                int ok = 1;
+                if (lane == 0) ok = ptx::wait_bounded(tfull_bar(b), use, tmo, abort_flag, ERR_EPI) ? 1 : 0;
+                return __shfl_sync(0xffffffffu, ok, 0) != 0;
+            };
             const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * BN);
-            if constexpr (SWAP)
-                epilogue_swap<BN, EPI>(p, tbase, tr, tc, tile, split, q, lane, last_flag);
-            else
-                epilogue_normal<BN, KIND, EPI>(p, tbase, tr, tc, q, lane);
+            if (!epilogue_sk<BN, EPI>(p, tbase, tr, tc, sg.tile, q, lane, flag, abort_flag, wsn, bn, s_am, tfull_wait))
+                break;
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(tempty_bar(b));
+            it -= sg.kb_hi - sg.kb_lo + 1;
         }
     }
 
+    // warps 0 and 1 ran their role on lane 0 alone: reconverge them first, so
+    // that the CTA barrier waits for every role to finish before TMEM is
+    // released
+    __syncwarp();
     __syncthreads();
     if (warp == 1) {
         __syncwarp();
@@ -521,7 +625,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ptx::tmem_dealloc(tmem_base, C::TMEM_COLS);
     }
 }
-
 // ---------------------------------------------------------------------------
 // Epilogue of one 128-row accumulator with coalesced output: each warp packs
 // its 32 rows x 32 columns into a shared-memory staging buffer in the

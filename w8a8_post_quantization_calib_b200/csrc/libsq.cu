@@ -142,22 +142,44 @@ bool make_map(CUtensorMap *m, const void *base, bool f16, int64_t inner, int64_t
     return r == CUDA_SUCCESS;
 }
 
-// ------------------------------------------------------------------ GEMM launch
-template <int BN, int KIND, int EPI, bool SWAP>
-sq_status launch_gemm(gemm::Params p, const void *a, const void *b, cudaStream_t st)
+// 3D view of a row-major [rows, K] int8 tensor (K a multiple of 128) as
+// [K/128][rows][128 bytes]: box = box_rows x 128 bytes x kbo blocks, each
+// block landing as its own 128-byte-swizzled tile.
+bool make_map3(CUtensorMap *m, const void *base, int64_t K, int64_t rows, uint32_t box_rows, uint32_t kbo)
 {
-    using C = gemm::TileCfg<BN>;
-    const bool f16 = (KIND == gemm::KIND_F16);
-    CUtensorMap ma, mb;
-    if (!make_map(&ma, a, f16, p.K, p.rows_a, gemm::BM)) return SQ_ERR_CUDA;
-    if (!make_map(&mb, b, f16, p.K, p.rows_b, BN)) return SQ_ERR_CUDA;
-    auto kern = gemm::k_gemm<BN, KIND, EPI, SWAP>;
+    auto fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(K / 128)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(K), 128};
+    cuuint32_t box[3] = {128, box_rows, kbo};
+    cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ GEMM launch
+// Small-M (swap) launch: map_w over the weights [N, K] in 128-row boxes, map_x
+// over the activations [M, K] in BN-row boxes; one CTA per stream-K share.
+template <int BN, int EPI, int KBO>
+sq_status launch_swap(gemm::Params p, const void *w, const void *x, cudaStream_t st)
+{
+    using C = gemm::TileCfg<BN, KBO>;
+    CUtensorMap mw, mx;
+    if constexpr (KBO == 1) {
+        if (!make_map(&mw, w, false, p.K, p.N, gemm::BM)) return SQ_ERR_CUDA;
+        if (!make_map(&mx, x, false, p.K, p.M, BN)) return SQ_ERR_CUDA;
+    } else {
+        if (!make_map3(&mw, w, p.K, p.N, gemm::BM, KBO)) return SQ_ERR_CUDA;
+        if (!make_map3(&mx, x, p.K, p.M, BN, KBO)) return SQ_ERR_CUDA;
+    }
+    auto kern = gemm::k_gemm_swap<BN, EPI, KBO>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), C::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_fail(e);
     p.timeout_ns = g_timeout_ns;
     p.inject = g_inject;
-    const int grid = static_cast<int>(std::min<int64_t>(p.num_units, sm_count()));
-    e = launch_pdl(kern, dim3(grid), dim3(gemm::NUM_THREADS), C::SMEM_BYTES, st, ma, mb, p);
+    e = launch_pdl(kern, dim3(p.sk_ctas), dim3(gemm::NUM_THREADS), C::SMEM_BYTES, st, mw, mx, p);
     return e == cudaSuccess ? check_launch() : cuda_fail(e);
 }
 
@@ -293,57 +315,81 @@ int64_t swap_tiles(int64_t M, int64_t N) { return cdiv(N, gemm::BM) * cdiv(M, sw
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Split-K factor of the small-M path.  Every extra split costs a partial-sum
-// slice round trip and a short accumulator hand-off per unit, so K is split
-// only when the weight tiles alone leave most SMs idle (at most half as many
-// tiles as SMs) and the token tile is small (M <= 64); the units never exceed
-// the SM count.  Measured on the MLP-7B shapes: N=4096 (32 tiles) runs in
-// about half the time with 4 splits at M = 1..16; N=11008 (86 tiles) and
-// M = 128 are fastest unsplit.  max_splits caps it (fixed-size scratch).
-int choose_splits(int64_t M, int64_t N, int64_t K, int max_splits = 16)
+// Stream-K CTA count of the small-M path.  Decode-size GEMMs are a stream of
+// the weight matrix, and one SM takes in only about 55 GB/s (measured with
+// TMA loads of two 16 KB blocks), so the weight bytes must be spread over
+// the SMs to reach the HBM rate: the 32 tiles of an 11008 -> 4096 projection
+// on 32 SMs cap near 2 TB/s.  The (tile, K block) iterations are then shared
+// evenly by min(SMs, iterations) CTAs.  Combining a shared tile costs a
+// partial-sum round trip (publish, arrival count, slot loads) of about 3 us
+// at the end of the owner's share, growing with the token tile, so sharing is
+// used only when one tile per CTA would leave more than half of the SMs idle
+// and the token tile is at most 32 (measured on the MLP-7B shapes: the
+// 32-tile projection gains from sharing at M = 1, 16 and loses at M = 64,
+// 128; the 86-tile one streams faster unshared at every M).  Otherwise, and
+// when the slots do not fit `slot_cap` bytes with at least min(tiles, SMs)
+// CTAs, the plain one-tile-per-CTA schedule runs: G = tiles.
+int64_t swap_grid(int64_t M, int64_t N, int64_t K, size_t slot_cap)
 {
     const int64_t tiles = swap_tiles(M, N);
+    const int64_t iters = tiles * ((K % 128) == 0 ? cdiv(K / 128, 2) : cdiv(K, 128));
     const int64_t sms = sm_count();
-    const int64_t kb = cdiv(K, 128);
-    if (M > 64 || 2 * tiles > sms) return 1;
-    int64_t splits = std::min<int64_t>({sms / tiles, static_cast<int64_t>(max_splits), kb / 4, 8});
-    if (splits < 2) return 1;
-    const int64_t kps = cdiv(kb, splits);
-    return static_cast<int>(cdiv(kb, kps));
+    if (tiles % sms == 0 || 2 * tiles > sms || swap_bn(M) > 32) return tiles;
+    int64_t g = std::min(sms, iters);
+    const size_t slot = static_cast<size_t>(gemm::BM) * swap_bn(M) * 4;
+    g = std::min<int64_t>(g, static_cast<int64_t>(slot_cap / slot));
+    if (g < std::min(tiles, sms)) return tiles;
+    return g;
 }
 
-size_t ws_bytes_for(int64_t M, int64_t N, int splits)
+// Workspace of a stream-K launch with G CTAs: G partial-sum slots of
+// BM x BN int32 (one per CTA), then one int32 arrival counter per tile.
+size_t swap_slot_bytes(int64_t M, int64_t G)
 {
-    return align_up(static_cast<size_t>(splits) * static_cast<size_t>(M * N) * 4, 256) +
-           align_up(static_cast<size_t>(swap_tiles(M, N)) * 4, 256);
+    return align_up(static_cast<size_t>(G) * gemm::BM * swap_bn(M) * 4, 256);
 }
 
 size_t ws_bytes(int64_t M, int64_t N, int64_t K)
 {
     if (M > kSwapMaxM) return 0;
-    return ws_bytes_for(M, N, choose_splits(M, N, K));
+    const int64_t g = swap_grid(M, N, K, SIZE_MAX);
+    if (g == swap_tiles(M, N)) return 0;
+    return swap_slot_bytes(M, g) + align_up(static_cast<size_t>(swap_tiles(M, N)) * 4, 256);
 }
 
+// p.ws_acc / p.ws_cnt must hold a workspace for `grid` CTAs unless grid is
+// the tile count (then they are ignored).
 template <int EPI>
-sq_status dispatch_swap(gemm::Params &p, const int8_t *xq, const int8_t *wq, cudaStream_t st, int splits = 1)
+sq_status dispatch_swap(gemm::Params &p, const int8_t *xq, const int8_t *wq, cudaStream_t st, int64_t grid)
 {
     const int bn = swap_bn(p.M);
     fill_tiles(p, bn, p.N, p.M);
-    if (EPI == gemm::EPI_DEQUANT && p.ws_acc != nullptr && splits > 1) {
-        const int tiles = p.num_units;
-        p.kb_per_split = static_cast<int>(cdiv(p.num_kb, splits));
-        p.splits = static_cast<int>(cdiv(p.num_kb, p.kb_per_split));
-        p.num_units = tiles * p.splits;
-    }
-    if (p.splits == 1) {
+    const bool kb2 = (p.K % 128) == 0;             // two K blocks per load (3D maps)
+    if (kb2) p.num_kb = static_cast<int>(cdiv(p.num_kb, 2));   // iterations: groups of 2 blocks
+    const int64_t tiles = static_cast<int64_t>(p.tiles_r) * p.tiles_c;
+    const int64_t iters = tiles * p.num_kb;
+    if (iters >= (int64_t(1) << 31)) return SQ_ERR_UNSUPPORTED;
+    p.sk_iters = static_cast<int>(iters);
+    p.sk_ctas = static_cast<int>(grid);
+    p.sk_slot = gemm::BM * bn;
+    p.ring = 0;                         // every stage of the ring
+    if (grid == tiles) {
         p.ws_acc = nullptr;
         p.ws_cnt = nullptr;
     }
+    if (kb2) {
+        switch (bn) {
+        case 16: return launch_swap<16, EPI, 2>(p, wq, xq, st);
+        case 32: return launch_swap<32, EPI, 2>(p, wq, xq, st);
+        case 64: return launch_swap<64, EPI, 2>(p, wq, xq, st);
+        default: return launch_swap<128, EPI, 2>(p, wq, xq, st);
+        }
+    }
     switch (bn) {
-    case 16: return launch_gemm<16, gemm::KIND_I8, EPI, true>(p, wq, xq, st);
-    case 32: return launch_gemm<32, gemm::KIND_I8, EPI, true>(p, wq, xq, st);
-    case 64: return launch_gemm<64, gemm::KIND_I8, EPI, true>(p, wq, xq, st);
-    default: return launch_gemm<128, gemm::KIND_I8, EPI, true>(p, wq, xq, st);
+    case 16: return launch_swap<16, EPI, 1>(p, wq, xq, st);
+    case 32: return launch_swap<32, EPI, 1>(p, wq, xq, st);
+    case 64: return launch_swap<64, EPI, 1>(p, wq, xq, st);
+    default: return launch_swap<128, EPI, 1>(p, wq, xq, st);
     }
 }
 
@@ -690,15 +736,15 @@ sq_status sq_linear_w8a8(const int8_t *xq, const int8_t *wq, int64_t M, int64_t 
     p.out = y;
     p.out_dt = out_dt;
     if (M <= kSwapMaxM) {
-        const int splits = choose_splits(M, N, K);
-        const size_t need = ws_bytes_for(M, N, splits);
-        if (splits > 1 && workspace != nullptr && workspace_bytes >= need && aligned16(workspace)) {
+        const int64_t tiles = swap_tiles(M, N);
+        const int64_t g = swap_grid(M, N, K, SIZE_MAX);
+        const size_t need = ws_bytes(M, N, K);
+        if (g != tiles && workspace != nullptr && workspace_bytes >= need && aligned16(workspace)) {
             p.ws_acc = static_cast<int32_t *>(workspace);
-            p.ws_cnt = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) +
-                                               align_up(static_cast<size_t>(splits) * static_cast<size_t>(M * N) * 4, 256));
-            return dispatch_swap<gemm::EPI_DEQUANT>(p, xq, wq, st, splits);
+            p.ws_cnt = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) + swap_slot_bytes(M, g));
+            return dispatch_swap<gemm::EPI_DEQUANT>(p, xq, wq, st, g);
         }
-        return dispatch_swap<gemm::EPI_DEQUANT>(p, xq, wq, st, 1);
+        return dispatch_swap<gemm::EPI_DEQUANT>(p, xq, wq, st, tiles);
     }
     return dispatch_pair<gemm::KIND_I8, gemm::EPI_DEQUANT>(p, xq, wq, st);
 }
@@ -716,20 +762,24 @@ sq_status sq_linear_w8a8_noalloc(const int8_t *xq, const int8_t *wq, int64_t M, 
     if (!aligned16(y) || !aligned16(w_scale)) return SQ_ERR_MISALIGNED;
     if (M > kSwapMaxM)      // the large-M path needs no scratch: same launch as sq_linear_w8a8
         return sq_linear_w8a8(xq, wq, M, N, K, a_scale, mode, w_scale, bias, out_dt, y, nullptr, 0, stream);
-    const size_t slice_bytes = static_cast<size_t>(M * N) * 4;
+    const size_t mn_bytes = static_cast<size_t>(M * N) * 4;
     const size_t cnt_bytes = static_cast<size_t>(swap_tiles(M, N)) * 4;
-    if (slice_bytes > kNoAllocAccBytes || cnt_bytes > kNoAllocCntBytes) return SQ_ERR_UNSUPPORTED;
-    // as many K splits as the fixed array holds partial-sum slices for
-    const int splits = choose_splits(M, N, K, static_cast<int>(kNoAllocAccBytes / slice_bytes));
+    if (mn_bytes > kNoAllocAccBytes || cnt_bytes > kNoAllocCntBytes) return SQ_ERR_UNSUPPORTED;
+    // as many stream-K CTAs as the fixed array holds partial-sum slots for
+    const int64_t g = swap_grid(M, N, K, kNoAllocAccBytes);
+    const bool shared = g != swap_tiles(M, N);
     void *scratch = nullptr;
     if ((r = noalloc_scratch(&scratch)) != SQ_OK) return r;
     int32_t *acc = static_cast<int32_t *>(scratch);
     int *cnt = reinterpret_cast<int *>(static_cast<unsigned char *>(scratch) + kNoAllocAccBytes);
     const cudaStream_t st = as_stream(stream);
     // the array keeps whatever the previous call left: the per-tile arrival
-    // counters must start at zero (the partial-sum slices are fully rewritten)
-    cudaError_t e = cudaMemsetAsync(cnt, 0, cnt_bytes, st);
-    if (e != cudaSuccess) return cuda_fail(e);
+    // counters must start at zero (a partial-sum slot is always written
+    // before it is read)
+    if (shared) {
+        cudaError_t e = cudaMemsetAsync(cnt, 0, cnt_bytes, st);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
     gemm::Params p{};
     p.M = static_cast<int>(M);
     p.N = static_cast<int>(N);
@@ -740,9 +790,9 @@ sq_status sq_linear_w8a8_noalloc(const int8_t *xq, const int8_t *wq, int64_t M, 
     p.bias = bias;
     p.out = y;
     p.out_dt = out_dt;
-    p.ws_acc = splits > 1 ? acc : nullptr;
-    p.ws_cnt = splits > 1 ? cnt : nullptr;
-    return dispatch_swap<gemm::EPI_DEQUANT>(p, xq, wq, st, splits);
+    p.ws_acc = shared ? acc : nullptr;
+    p.ws_cnt = shared ? cnt : nullptr;
+    return dispatch_swap<gemm::EPI_DEQUANT>(p, xq, wq, st, g);
 }
 
 sq_status sq_gemm_s32(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, int64_t K, int32_t *acc,
@@ -758,7 +808,7 @@ sq_status sq_gemm_s32(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, 
     p.N = static_cast<int>(N);
     p.K = static_cast<int>(K);
     p.out = acc;
-    if (M <= kSwapMaxM) return dispatch_swap<gemm::EPI_S32>(p, xq, wq, st);
+    if (M <= kSwapMaxM) return dispatch_swap<gemm::EPI_S32>(p, xq, wq, st, swap_tiles(M, N));
     return dispatch_pair<gemm::KIND_I8, gemm::EPI_S32>(p, xq, wq, st);
 }
 

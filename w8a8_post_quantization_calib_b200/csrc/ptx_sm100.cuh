@@ -77,6 +77,38 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, uint
     }
 }
 
+// Waits until the int at global address `cnt` (written by other CTAs with
+// release semantics) reaches `target`, reading it with acquire semantics.
+// Bounded like wait_bounded.
+__device__ __forceinline__ bool wait_count_bounded(const int *cnt, int target, uint64_t timeout_ns,
+                                                   volatile int *abort, unsigned code)
+{
+    auto load = [&]() {
+        int v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
+        return v;
+    };
+    if (load() >= target) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+        __nanosleep(64);
+        if (load() >= target) return true;
+        if (*abort) return false;
+        if (global_timer_ns() - t0 > timeout_ns) {
+            *abort = 1;
+            atomicCAS(&g_error_word, 0u, code);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
+__device__ __forceinline__ void red_add_release_gpu(int *p, int v)
+{
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const void *map)
 {
@@ -93,6 +125,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *map, uint3
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+
+// 3D tiled bulk-tensor load global -> shared (coordinates innermost first).
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *map, uint32_t bar, int x, int y, int z)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
         : "memory");
 }
 

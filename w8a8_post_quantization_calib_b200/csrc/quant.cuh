@@ -150,6 +150,29 @@ __device__ __forceinline__ float column_constant(const RowArgs &p, int64_t j)
     else return recip_or_zero(p.s[j]);
 }
 
+// The same constants for the four columns 4q..4q+3 from 16-byte loads
+// (caller checks that s and gamma are 16-byte aligned).
+template <int MODE>
+__device__ __forceinline__ float4 column_constant4(const RowArgs &p, int64_t q)
+{
+    if constexpr (MODE == ROW_WEIGHT) return __ldg(reinterpret_cast<const float4 *>(p.s) + q);
+    else if constexpr (MODE == ROW_RMS_STAT) return __ldg(reinterpret_cast<const float4 *>(p.gamma) + q);
+    else {
+        const float4 s = __ldg(reinterpret_cast<const float4 *>(p.s) + q);
+        float4 c = make_float4(recip_or_zero(s.x), recip_or_zero(s.y), recip_or_zero(s.z), recip_or_zero(s.w));
+        if constexpr (MODE == ROW_RMSNORM) {
+            const float4 g = __ldg(reinterpret_cast<const float4 *>(p.gamma) + q);
+            c = make_float4(__fmul_rn(g.x, c.x), __fmul_rn(g.y, c.y), __fmul_rn(g.z, c.z), __fmul_rn(g.w, c.w));
+        }
+        return c;
+    }
+}
+
+__device__ __forceinline__ bool constants_aligned16(const RowArgs &p)
+{
+    return ((reinterpret_cast<uintptr_t>(p.s) | reinterpret_cast<uintptr_t>(p.gamma)) & 15u) == 0;
+}
+
 // Thread `tid` owns the 16-byte vectors v = i*ROW_T + tid (i < VPT) of every
 // row it touches, so its per-column constants are row-invariant.  REG: they
 // (and the pass-1 products) live in registers; otherwise they are read from
@@ -171,14 +194,46 @@ __global__ void __launch_bounds__(ROW_T) k_rows(RowArgs p)
     pdl_wait();
     pdl_launch_dependents();
 
+    const bool c16 = constants_aligned16(p);
     float creg[REG ? VPT : 1][REG ? EPV : 1];
     if constexpr (REG) {
+        if (c16) {
 #pragma unroll
-        for (int i = 0; i < VPT; ++i) {
-            const int64_t v = static_cast<int64_t>(i) * ROW_T + tid;
+            for (int i = 0; i < VPT; ++i) {
+                const int64_t v = static_cast<int64_t>(i) * ROW_T + tid;
 #pragma unroll
-            for (int e = 0; e < EPV; ++e) creg[i][e] = (v < nvec) ? column_constant<MODE>(p, v * EPV + e) : 0.0f;
+                for (int h = 0; h < EPV / 4; ++h) {
+                    const float4 t = (v < nvec) ? column_constant4<MODE>(p, v * (EPV / 4) + h)
+                                                : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                    creg[i][4 * h] = t.x; creg[i][4 * h + 1] = t.y; creg[i][4 * h + 2] = t.z; creg[i][4 * h + 3] = t.w;
+                }
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < VPT; ++i) {
+                const int64_t v = static_cast<int64_t>(i) * ROW_T + tid;
+#pragma unroll
+                for (int e = 0; e < EPV; ++e) creg[i][e] = (v < nvec) ? column_constant<MODE>(p, v * EPV + e) : 0.0f;
+            }
         }
+    } else if (c16) {
+        // 16-byte loads, 8 per thread in flight: float4 q holds columns 4q..4q+3,
+        // i.e. plane q % (EPV/4) of vector q / (EPV/4)
+        const int64_t nq = p.K / 4;
+        for (int64_t q0 = tid; q0 < nq; q0 += 8 * ROW_T) {
+            float4 c[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int64_t q = q0 + static_cast<int64_t>(u) * ROW_T;
+                if (q < nq) c[u] = column_constant4<MODE>(p, q);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int64_t q = q0 + static_cast<int64_t>(u) * ROW_T;
+                if (q < nq) colv4[(q % (EPV / 4)) * plane + q / (EPV / 4)] = c[u];
+            }
+        }
+        __syncthreads();
     } else {
         // 8 columns per step: the loads of a step are independent and overlap
         float *cv = reinterpret_cast<float *>(colv4);
