@@ -676,6 +676,43 @@ def run_workload(args):
                     "down_frac_int8_peak": ops_d / (t_d * 1e-3) / 1e12 / P["int8_tops"],
                     "weight_quant_gateup_us": t_wgu * 1e3,
                     "weight_quant_gateup_gbs": 2 * f * d * 3 / (t_wgu * 1e-3) / 1e9})
+    elif args.workload == "rows":
+        # the HBM-bound kernels on inputs of 256 MiB (twice the L2), so that
+        # every call of a timed chain streams from HBM; bytes = algorithmic
+        # reads + writes
+        R = 1 << 27                                   # elements per input tensor
+        g16 = torch.Generator(device="cuda").manual_seed(7)
+        lines = []
+
+        only = set(args.only.split(",")) if args.only else None
+
+        def rec(name, fn, nbytes, shape, dt):
+            if only is not None and name not in only:
+                return
+            t_ms = _time_ms(fn, 10)
+            gbs = nbytes / (t_ms * 1e-3) / 1e9
+            lines.append({"kernel": name, "shape": shape, "dtype": dt, "us": t_ms * 1e3, "gbs": gbs,
+                          "frac_hbm": gbs / P["hbm_gbs"]})
+        for K, dt in ((4096, torch.float16), (8192, torch.bfloat16)):
+            M = R // K
+            X = torch.randn(M, K, generator=g16, device="cuda").to(dt)
+            name = "f16" if dt == torch.float16 else "bf16"
+            am = torch.zeros(K, device="cuda")
+            rec("calib_absmax", lambda: sq.calib_absmax(X, am), M * K * 2, [M, K], name)
+            s = torch.rand(K, device="cuda") + 0.5
+            a = torch.full((1,), 0.05, device="cuda")
+            xq = torch.empty(M, K, dtype=torch.int8, device="cuda")
+            at = torch.empty(M, device="cuda")
+            rec("act_static", lambda: sq.smooth_quant_act(X, s, sq.ACT_STATIC, a, xq), M * K * 3, [M, K], name)
+            rec("act_per_token", lambda: sq.smooth_quant_act(X, s, sq.ACT_PER_TOKEN, at, xq),
+                M * K * 3 + M * 4, [M, K], name)
+            rec("quant_weight", lambda: sq.quant_weight(X, s, xq, at), M * K * 3 + M * 4, [M, K], name)
+            gam = torch.rand(K, device="cuda") + 0.5
+            rec("rmsnorm_quant", lambda: sq.rmsnorm_quant(X, gam, s, 1e-5, a, xq), M * K * 3, [M, K], name)
+            rec("rmsnorm_absmax", lambda: sq.rmsnorm_absmax(X, gam, 1e-5, am), M * K * 2, [M, K], name)
+            del X, xq, at
+            torch.cuda.empty_cache()
+        out["lines"] = lines
     print(json.dumps(out), flush=True)
     return 0
 
@@ -694,7 +731,8 @@ def main():
     ap.add_argument("--tokens", default="1,16,128,4096",
                     help="mlp7b workload: comma-separated token counts M to sweep")
     ap.add_argument("--proj", default="up,down", help="mlp7b workload: projections to sweep")
-    ap.add_argument("--workload", choices=["qkv7b", "mlp7b", "alpha13b", "mlp70b"], default="qkv7b",
+    ap.add_argument("--only", default="", help="rows workload: comma-separated kernels to run (default all)")
+    ap.add_argument("--workload", choices=["qkv7b", "mlp7b", "alpha13b", "mlp70b", "rows"], default="qkv7b",
                     help="qkv7b is the bench line; the others print per-kernel measurements of the other workloads")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -733,10 +733,12 @@ __device__ __forceinline__ void epilogue_tma(const Params &p, const CUtensorMap 
 // from the leader's MMA thread; tempty[b] lives in the leader and collects
 // one arrival per epilogue warp of both CTAs (8).
 // ===========================================================================
-template <int BN>
+template <int BN, int KBO = 1>
 struct PairCfg {
-    static constexpr int A_BYTES = BM * BKB;              // this CTA's 128 rows of A
-    static constexpr int B_BYTES = (BN / 2) * BKB;        // this CTA's BN/2 rows of B
+    static constexpr int A_KB = BM * BKB;                 // this CTA's 128 rows of A, one K block
+    static constexpr int B_KB = (BN / 2) * BKB;           // this CTA's BN/2 rows of B, one K block
+    static constexpr int A_BYTES = A_KB * KBO;
+    static constexpr int B_BYTES = B_KB * KBO;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int STAGES_RAW = (188 * 1024) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_RAW > 10 ? 10 : STAGES_RAW;
@@ -749,12 +751,14 @@ struct PairCfg {
     static_assert(TMEM_COLS <= 512, "two accumulators must fit TMEM");
 };
 
-template <int BN, int KIND, int EPI>
+// KBO > 1 (kind::i8, K a multiple of 128): 3D operand maps, KBO K blocks per
+// TMA load (see k_gemm_swap); num_kb then counts groups of KBO blocks.
+template <int BN, int KIND, int EPI, int KBO = 1>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     k_gemm2(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
             const __grid_constant__ CUtensorMap map_o, const Params p)
 {
-    using C = PairCfg<BN>;
+    using C = PairCfg<BN, KBO>;
     constexpr int S = C::STAGES;
     constexpr int BKE = (KIND == KIND_I8) ? BKB : BKB / 2;
     constexpr uint32_t IDESC = (KIND == KIND_I8) ? ptx::idesc_i8_m256(BN) : ptx::idesc_f16_m256(BN);
@@ -829,9 +833,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                         if (leader) ptx::mbar_arrive_expect_tx(full_bar(stage), 2 * C::STAGE_BYTES);
                         const uint32_t fb = ptx::map_to_rank(full_bar(stage), 0);
                         const uint32_t sa = sbase + stage * C::STAGE_BYTES;
-                        ptx::tma_load_2d_pair(sa, &map_a, fb, kb * BKE, tr * (2 * BM) + static_cast<int>(rank) * BM);
-                        ptx::tma_load_2d_pair(sa + C::A_BYTES, &map_b, fb, kb * BKE,
-                                              tc * BN + static_cast<int>(rank) * (BN / 2));
+                        const int ya = tr * (2 * BM) + static_cast<int>(rank) * BM;
+                        const int yb = tc * BN + static_cast<int>(rank) * (BN / 2);
+                        if constexpr (KBO == 1) {
+                            ptx::tma_load_2d_pair(sa, &map_a, fb, kb * BKE, ya);
+                            ptx::tma_load_2d_pair(sa + C::A_BYTES, &map_b, fb, kb * BKE, yb);
+                        } else {
+                            ptx::tma_load_3d_pair(sa, &map_a, fb, 0, ya, kb * KBO);
+                            ptx::tma_load_3d_pair(sa + C::A_BYTES, &map_b, fb, 0, yb, kb * KBO);
+                        }
                     }
                     ++issued;
                     if (++stage == S) { stage = 0; phase ^= 1u; }
@@ -869,15 +879,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     }
                     ptx::tc_fence_after();
                     const uint32_t sa = sbase + stage * C::STAGE_BYTES;
-                    const uint64_t ad = ptx::sdesc_kmajor_sw128(sa);
-                    const uint64_t bd = ptx::sdesc_kmajor_sw128(sa + C::A_BYTES);
 #pragma unroll
-                    for (int k = 0; k < BKB / 32; ++k) {
-                        const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
-                        if constexpr (KIND == KIND_I8)
-                            ptx::mma_i8_pair(d, ad + 2 * k, bd + 2 * k, IDESC, acc);
-                        else
-                            ptx::mma_f16_pair(d, ad + 2 * k, bd + 2 * k, IDESC, acc);
+                    for (int j = 0; j < KBO; ++j) {
+                        const uint64_t ad = ptx::sdesc_kmajor_sw128(sa + j * C::A_KB);
+                        const uint64_t bd = ptx::sdesc_kmajor_sw128(sa + C::A_BYTES + j * C::B_KB);
+#pragma unroll
+                        for (int k = 0; k < BKB / 32; ++k) {
+                            const uint32_t acc = (kb > 0 || j > 0 || k > 0) ? 1u : 0u;
+                            if constexpr (KIND == KIND_I8)
+                                ptx::mma_i8_pair(d, ad + 2 * k, bd + 2 * k, IDESC, acc);
+                            else
+                                ptx::mma_f16_pair(d, ad + 2 * k, bd + 2 * k, IDESC, acc);
+                        }
                     }
                     ptx::tc_commit_pair_mc(empty_bar(stage), 0x3);
                     if (++stage == S) { stage = 0; phase ^= 1u; }

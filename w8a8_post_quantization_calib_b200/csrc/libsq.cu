@@ -81,6 +81,28 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
     return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
+// launch_pdl with a runtime cluster shape (cluster_x CTAs along x).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, unsigned cluster_x, cudaStream_t st,
+                               Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster_x;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // Per (device, kernel): dynamic shared memory already granted, and the
 // occupancy figures the launch sizes its grid with.  Queried once.
 struct KernelInfo {
@@ -207,21 +229,27 @@ bool make_out_map(CUtensorMap *m, void *base, int out_dt, bool s32, int64_t M, i
     return r == CUDA_SUCCESS;
 }
 
-template <int BN, int KIND, int EPI>
+template <int BN, int KIND, int EPI, int KBO>
 sq_status launch_gemm2(gemm::Params p, const void *a, const void *b, cudaStream_t st)
 {
-    using C = gemm::PairCfg<BN>;
+    using C = gemm::PairCfg<BN, KBO>;
     const bool f16 = (KIND == gemm::KIND_F16);
     CUtensorMap ma, mb, mo;
-    if (!make_map(&ma, a, f16, p.K, p.rows_a, gemm::BM)) return SQ_ERR_CUDA;
-    if (!make_map(&mb, b, f16, p.K, p.rows_b, BN / 2)) return SQ_ERR_CUDA;
+    if constexpr (KBO == 1) {
+        if (!make_map(&ma, a, f16, p.K, p.rows_a, gemm::BM)) return SQ_ERR_CUDA;
+        if (!make_map(&mb, b, f16, p.K, p.rows_b, BN / 2)) return SQ_ERR_CUDA;
+    } else {
+        static_assert(KIND == gemm::KIND_I8, "3D operand maps are int8");
+        if (!make_map3(&ma, a, p.K, p.rows_a, gemm::BM, KBO)) return SQ_ERR_CUDA;
+        if (!make_map3(&mb, b, p.K, p.rows_b, BN / 2, KBO)) return SQ_ERR_CUDA;
+    }
     if constexpr (EPI == gemm::EPI_GATEUP) {
         std::memset(&mo, 0, sizeof(mo));
     } else {
         const int odt = (EPI == gemm::EPI_F16) ? SQ_F16 : p.out_dt;
         if (!make_out_map(&mo, p.out, odt, EPI == gemm::EPI_S32, p.M, p.N)) return SQ_ERR_CUDA;
     }
-    auto kern = gemm::k_gemm2<BN, KIND, EPI>;
+    auto kern = gemm::k_gemm2<BN, KIND, EPI, KBO>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), C::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_fail(e);
     int max_clusters = 0;
@@ -267,8 +295,9 @@ int pick_pair_bn(int64_t M, int64_t N)
     const int64_t clusters = std::max(1, sm_count() / 2);
     const int cands[3] = {256, 192, 128};
     // measured time per output column of a full wave relative to the 256-wide
-    // tile (narrower tiles move more operand bytes per MAC)
-    const double eff[3] = {1.0, 0.93, 0.77};
+    // tile (narrower tiles move more operand bytes per MAC; the 192-wide one
+    // with two K blocks per load: Llama-7B QKV / MLP and 13B shapes)
+    const double eff[3] = {1.0, 0.89, 0.77};
     int best = 256;
     double best_cost = -1.0;
     for (int i = 0; i < 3; ++i) {
@@ -288,10 +317,19 @@ sq_status dispatch_pair(gemm::Params &p, const void *a, const void *b, cudaStrea
 {
     const int bn = force_bn ? force_bn : pick_pair_bn(p.M, p.N);
     fill_tiles_pair(p, bn, KIND == gemm::KIND_F16 ? 2 : 1);
+    if constexpr (KIND == gemm::KIND_I8) {
+        // 192-wide tiles: two K blocks per TMA load (3 stages of 56 KB hold
+        // the same 6 blocks as 6 single-block stages, with half the loads);
+        // the 256-wide tile would drop to 2 stages, so it keeps single blocks
+        if (bn == 192 && (p.K % 128) == 0) {
+            p.num_kb = static_cast<int>(cdiv(p.num_kb, 2));
+            return launch_gemm2<192, KIND, EPI, 2>(p, a, b, st);
+        }
+    }
     switch (bn) {
-    case 256: return launch_gemm2<256, KIND, EPI>(p, a, b, st);
-    case 192: return launch_gemm2<192, KIND, EPI>(p, a, b, st);
-    default: return launch_gemm2<128, KIND, EPI>(p, a, b, st);
+    case 256: return launch_gemm2<256, KIND, EPI, 1>(p, a, b, st);
+    case 192: return launch_gemm2<192, KIND, EPI, 1>(p, a, b, st);
+    default: return launch_gemm2<128, KIND, EPI, 1>(p, a, b, st);
     }
 }
 
@@ -402,18 +440,47 @@ sq_status launch_rows_dt(RowArgs a, cudaStream_t st)
                      (a.out == nullptr || aligned16(a.out)) && (a.K % EPV) == 0 &&
                      (MODE != ROW_RMS_STAT || cdiv(a.K / EPV, ROW_T) * EPV <= 32);
     const int64_t nvec = a.K / EPV;
-    const int64_t vpt = cdiv(nvec, ROW_T);
+    // 128 threads per row for rows of up to 512 vectors, else 256
+    const int nt = nvec <= 4 * 128 ? 128 : ROW_T;
+    const int64_t vpt = cdiv(nvec, nt);
     // per-column constants in registers when VPT * EPV <= 32, else in shared memory
     const size_t smem = (vpt * EPV <= 32) ? 0 : static_cast<size_t>(a.K) * 4;
     const int sms = sm_count();
+    // Fewer rows than SMs: the row kernel would run one latency-bound row per
+    // block on a few SMs; a cluster of CTAs per row (one vector per thread)
+    // spreads each row instead.  The cluster size is the smallest power of
+    // two up to 8 that divides the row's vectors into at most ROW_T each.
+    if (vec && a.rows < sms && a.src1 == nullptr) {
+        int cs = 0;
+        for (int c = 2; c <= 8; c *= 2)
+            if (nvec % c == 0 && nvec / c <= ROW_T) { cs = c; break; }
+        if (cs > 0) {
+            const cudaError_t e = launch_pdl_cluster(k_rows_split<DT, MODE>,
+                                                     dim3(static_cast<unsigned>(cs), static_cast<unsigned>(a.rows)),
+                                                     dim3(ROW_T), static_cast<unsigned>(cs), st, a);
+            if (e != cudaSuccess) return cuda_fail(e);
+            return check_launch();
+        }
+    }
     if (vec && vpt <= 16 && smem <= 160 * 1024) {
         void (*kern)(RowArgs) = nullptr;
-        if (vpt <= 1) kern = k_rows<DT, 1, MODE>;
-        else if (vpt <= 2) kern = k_rows<DT, 2, MODE>;
-        else if constexpr (MODE == ROW_RMS_STAT) kern = k_rows<DT, (DT == DT_F32 ? 8 : 4), MODE>;
-        else if (vpt <= 4) kern = k_rows<DT, 4, MODE>;
-        else if (vpt <= 8) kern = k_rows<DT, 8, MODE>;
-        else kern = k_rows<DT, 16, MODE>;
+        if (nt == 128) {
+            if (vpt <= 1) kern = k_rows<DT, 1, MODE, 128>;
+            else if (vpt <= 2) kern = k_rows<DT, 2, MODE, 128>;
+            else kern = k_rows<DT, 4, MODE, 128>;
+        } else if (vpt <= 1) {
+            kern = k_rows<DT, 1, MODE, ROW_T>;
+        } else if (vpt <= 2) {
+            kern = k_rows<DT, 2, MODE, ROW_T>;
+        } else if constexpr (MODE == ROW_RMS_STAT) {
+            kern = k_rows<DT, (DT == DT_F32 ? 8 : 4), MODE, ROW_T>;
+        } else if (vpt <= 4) {
+            kern = k_rows<DT, 4, MODE, ROW_T>;
+        } else if (vpt <= 8) {
+            kern = k_rows<DT, 8, MODE, ROW_T>;
+        } else {
+            kern = k_rows<DT, 16, MODE, ROW_T>;
+        }
         cudaError_t e = cudaSuccess;
         if (smem > 48 * 1024) {
             e = ensure_smem(reinterpret_cast<const void *>(kern), static_cast<int>(smem));
@@ -425,7 +492,7 @@ sq_status launch_rows_dt(RowArgs a, cudaStream_t st)
             per_sm = kinfo(reinterpret_cast<const void *>(kern)).per_sm;
         }
         if (per_sm == 0) {
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, ROW_T, smem);
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, nt, smem);
             if (e != cudaSuccess) return cuda_fail(e);
             if (smem == 0) {
                 std::lock_guard<std::mutex> lk(g_mu);
@@ -433,7 +500,7 @@ sq_status launch_rows_dt(RowArgs a, cudaStream_t st)
             }
         }
         const int64_t grid = std::min<int64_t>(a.rows, static_cast<int64_t>(sms) * std::max(1, per_sm));
-        e = launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(ROW_T), smem, st, a);
+        e = launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(nt), smem, st, a);
         if (e != cudaSuccess) return cuda_fail(e);
     } else {
         const int64_t grid = std::min<int64_t>(a.rows, static_cast<int64_t>(sms) * 8);
@@ -656,6 +723,33 @@ sq_status sq_smooth_quant_act(const void *x, sq_dtype dt, int64_t M, int64_t K, 
     a.out = xq;
     if (mode == SQ_ACT_STATIC) {
         a.a_in = a_scale;
+        const int elt = dtype_size(dt);
+        if (M > 0 && (K * elt) % 16 == 0) {
+            // elementwise: column strips x row slabs, like the calibration statistic
+            const int64_t nvec = K * elt / 16;
+            const int64_t gx = cdiv(nvec, QS_TX);
+            const int64_t target = static_cast<int64_t>(sm_count()) * 8;
+            int64_t gy = std::max<int64_t>(1, std::min<int64_t>(cdiv(M, QS_TY * QS_UNROLL), cdiv(target, gx)));
+            gy = std::min<int64_t>(gy, 65535);
+            const int64_t slab = cdiv(M, gy);
+            gy = cdiv(M, slab);
+            const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), block(QS_TX, QS_TY);
+            const uint8_t *xb = static_cast<const uint8_t *>(x);
+            const bool big = M * K * elt > (int64_t(100) << 20);
+            const cudaStream_t st = as_stream(stream);
+            cudaError_t e;
+            if (dt == SQ_F32)
+                e = big ? launch_pdl(k_quant_static<DT_F32, true>, grid, block, 0, st, xb, M, nvec, s, a_scale, slab, xq)
+                        : launch_pdl(k_quant_static<DT_F32, false>, grid, block, 0, st, xb, M, nvec, s, a_scale, slab, xq);
+            else if (dt == SQ_F16)
+                e = big ? launch_pdl(k_quant_static<DT_F16, true>, grid, block, 0, st, xb, M, nvec, s, a_scale, slab, xq)
+                        : launch_pdl(k_quant_static<DT_F16, false>, grid, block, 0, st, xb, M, nvec, s, a_scale, slab, xq);
+            else
+                e = big ? launch_pdl(k_quant_static<DT_BF16, true>, grid, block, 0, st, xb, M, nvec, s, a_scale, slab, xq)
+                        : launch_pdl(k_quant_static<DT_BF16, false>, grid, block, 0, st, xb, M, nvec, s, a_scale, slab, xq);
+            if (e != cudaSuccess) return cuda_fail(e);
+            return check_launch();
+        }
         return launch_rows<ROW_ACT_STATIC>(a, dt, as_stream(stream));
     }
     a.scale_out = a_scale;

@@ -307,6 +307,17 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void *map, 
         : "memory");
 }
 
+// 3D form of tma_load_2d_pair (coordinates innermost first).
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const void *map, uint32_t cluster_bar, int x, int y,
+                                                 int z)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(cluster_bar), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t slot_smem, uint32_t ncols)
 {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot_smem), "r"(ncols)

@@ -13,6 +13,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "ptx_sm100.cuh"
 
 namespace sq {
 
@@ -173,14 +174,18 @@ __device__ __forceinline__ bool constants_aligned16(const RowArgs &p)
     return ((reinterpret_cast<uintptr_t>(p.s) | reinterpret_cast<uintptr_t>(p.gamma)) & 15u) == 0;
 }
 
-// Thread `tid` owns the 16-byte vectors v = i*ROW_T + tid (i < VPT) of every
+// Thread `tid` owns the 16-byte vectors v = i*NT + tid (i < VPT) of every
 // row it touches, so its per-column constants are row-invariant.  REG: they
-// (and the pass-1 products) live in registers; otherwise they are read from
+// (and the pass-1 values) live in registers; otherwise they are read from
 // shared memory laid out as EPV/4 planes of float4 (plane h holds elements
 // 4h..4h+3 of every vector), which makes the per-thread float4 reads
-// conflict-free.
-template <int DT, int VPT, int MODE>
-__global__ void __launch_bounds__(ROW_T) k_rows(RowArgs p)
+// conflict-free.  The kernels are issue-bound rather than DRAM-bound at
+// these sizes, so vectors past the row end are computed on zeros and only
+// their stores are predicated (no divergent branches), and NT = 128 threads
+// per row for rows of up to 4096 16-bit elements halves the per-row cost of
+// the block reductions.
+template <int DT, int VPT, int MODE, int NT>
+__global__ void __launch_bounds__(NT) k_rows(RowArgs p)
 {
     constexpr int EPV = VecT<DT>::EPV;
     constexpr bool REG = (VPT * EPV <= 32);
@@ -194,13 +199,37 @@ __global__ void __launch_bounds__(ROW_T) k_rows(RowArgs p)
     pdl_wait();
     pdl_launch_dependents();
 
+    auto row_src = [&](int64_t row) -> const uint8_t * {
+        if (p.src1 != nullptr) {          // gate/up interleave: blocks of 64 output rows
+            const int64_t b = row >> 6, w = row & 63;
+            return (w < 32 ? p.src0 : p.src1) + ((b << 5) + (w & 31)) * p.row_bytes;
+        }
+        return p.src0 + row * p.row_bytes;
+    };
+    auto load_row = [&](int64_t row, uint4 (&dst)[VPT]) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(row_src(row));
+#pragma unroll
+        for (int i = 0; i < VPT; ++i) {
+            const int64_t v = static_cast<int64_t>(i) * NT + tid;
+            dst[i] = (v < nvec) ? __ldcs(src + v) : make_uint4(0u, 0u, 0u, 0u);
+        }
+    };
+    // Rows of up to 8 vectors per thread keep the next row's loads in flight
+    // while a row is processed; the first row is requested before the
+    // per-column constants, so that the two loads overlap.
+    constexpr bool PF = VPT <= 8;
+    uint4 nxt[PF ? VPT : 1];
+    if constexpr (PF) {
+        if (blockIdx.x < p.rows) load_row(blockIdx.x, nxt);
+    }
+
     const bool c16 = constants_aligned16(p);
     float creg[REG ? VPT : 1][REG ? EPV : 1];
     if constexpr (REG) {
         if (c16) {
 #pragma unroll
             for (int i = 0; i < VPT; ++i) {
-                const int64_t v = static_cast<int64_t>(i) * ROW_T + tid;
+                const int64_t v = static_cast<int64_t>(i) * NT + tid;
 #pragma unroll
                 for (int h = 0; h < EPV / 4; ++h) {
                     const float4 t = (v < nvec) ? column_constant4<MODE>(p, v * (EPV / 4) + h)
@@ -211,7 +240,7 @@ __global__ void __launch_bounds__(ROW_T) k_rows(RowArgs p)
         } else {
 #pragma unroll
             for (int i = 0; i < VPT; ++i) {
-                const int64_t v = static_cast<int64_t>(i) * ROW_T + tid;
+                const int64_t v = static_cast<int64_t>(i) * NT + tid;
 #pragma unroll
                 for (int e = 0; e < EPV; ++e) creg[i][e] = (v < nvec) ? column_constant<MODE>(p, v * EPV + e) : 0.0f;
             }
@@ -220,16 +249,16 @@ __global__ void __launch_bounds__(ROW_T) k_rows(RowArgs p)
         // 16-byte loads, 8 per thread in flight: float4 q holds columns 4q..4q+3,
         // i.e. plane q % (EPV/4) of vector q / (EPV/4)
         const int64_t nq = p.K / 4;
-        for (int64_t q0 = tid; q0 < nq; q0 += 8 * ROW_T) {
+        for (int64_t q0 = tid; q0 < nq; q0 += 8 * NT) {
             float4 c[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const int64_t q = q0 + static_cast<int64_t>(u) * ROW_T;
+                const int64_t q = q0 + static_cast<int64_t>(u) * NT;
                 if (q < nq) c[u] = column_constant4<MODE>(p, q);
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const int64_t q = q0 + static_cast<int64_t>(u) * ROW_T;
+                const int64_t q = q0 + static_cast<int64_t>(u) * NT;
                 if (q < nq) colv4[(q % (EPV / 4)) * plane + q / (EPV / 4)] = c[u];
             }
         }
@@ -237,16 +266,16 @@ __global__ void __launch_bounds__(ROW_T) k_rows(RowArgs p)
     } else {
         // 8 columns per step: the loads of a step are independent and overlap
         float *cv = reinterpret_cast<float *>(colv4);
-        for (int64_t j0 = tid; j0 < p.K; j0 += 8 * ROW_T) {
+        for (int64_t j0 = tid; j0 < p.K; j0 += 8 * NT) {
             float c[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const int64_t j = j0 + static_cast<int64_t>(u) * ROW_T;
+                const int64_t j = j0 + static_cast<int64_t>(u) * NT;
                 c[u] = (j < p.K) ? column_constant<MODE>(p, j) : 0.0f;
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const int64_t j = j0 + static_cast<int64_t>(u) * ROW_T;
+                const int64_t j = j0 + static_cast<int64_t>(u) * NT;
                 if (j < p.K) {
                     const int64_t v = j / EPV;
                     const int e = static_cast<int>(j % EPV);
@@ -256,14 +285,17 @@ __global__ void __launch_bounds__(ROW_T) k_rows(RowArgs p)
         }
         __syncthreads();
     }
+    // constants of vector slot i (vectors past the row end read a valid
+    // entry; their results are never stored)
     auto colc = [&](int i, int64_t v, float (&c)[EPV]) {
         if constexpr (REG) {
 #pragma unroll
             for (int e = 0; e < EPV; ++e) c[e] = creg[i][e];
         } else {
+            const int64_t vc = v < nvec ? v : nvec - 1;
 #pragma unroll
             for (int h = 0; h < EPV / 4; ++h) {
-                const float4 t = colv4[h * plane + v];
+                const float4 t = colv4[h * plane + vc];
                 c[4 * h] = t.x; c[4 * h + 1] = t.y; c[4 * h + 2] = t.z; c[4 * h + 3] = t.w;
             }
         }
@@ -279,31 +311,9 @@ __global__ void __launch_bounds__(ROW_T) k_rows(RowArgs p)
             for (int e = 0; e < EPV; ++e) cmax[i][e] = 0.0f;
     }
 
-    auto row_src = [&](int64_t row) -> const uint8_t * {
-        if (p.src1 != nullptr) {          // gate/up interleave: blocks of 64 output rows
-            const int64_t b = row >> 6, w = row & 63;
-            return (w < 32 ? p.src0 : p.src1) + ((b << 5) + (w & 31)) * p.row_bytes;
-        }
-        return p.src0 + row * p.row_bytes;
-    };
-    auto load_row = [&](int64_t row, uint4 (&dst)[VPT]) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(row_src(row));
-#pragma unroll
-        for (int i = 0; i < VPT; ++i) {
-            const int64_t v = static_cast<int64_t>(i) * ROW_T + tid;
-            if (v < nvec) dst[i] = __ldcs(src + v);
-        }
-    };
-    // REG rows are short: the next row's loads are issued before this row is
-    // processed, so each thread keeps two rows of loads in flight.
-    uint4 nxt[REG ? VPT : 1];
-    if constexpr (REG) {
-        if (blockIdx.x < p.rows) load_row(blockIdx.x, nxt);
-    }
-
     for (int64_t row = blockIdx.x; row < p.rows; row += gridDim.x) {
         uint4 raw[VPT];
-        if constexpr (REG) {
+        if constexpr (PF) {
 #pragma unroll
             for (int i = 0; i < VPT; ++i) raw[i] = nxt[i];
             if (row + gridDim.x < p.rows) load_row(row + gridDim.x, nxt);
@@ -315,30 +325,30 @@ __global__ void __launch_bounds__(ROW_T) k_rows(RowArgs p)
         if constexpr (MODE == ROW_ACT_STATIC) {
 #pragma unroll
             for (int i = 0; i < VPT; ++i) {
-                const int64_t v = static_cast<int64_t>(i) * ROW_T + tid;
-                if (v < nvec) {
-                    float f[EPV], c[EPV];
-                    widen<DT>(raw[i], f);
-                    colc(i, v, c);
+                const int64_t v = static_cast<int64_t>(i) * NT + tid;
+                float f[EPV], c[EPV];
+                widen<DT>(raw[i], f);
+                colc(i, v, c);
 #pragma unroll
-                    for (int e = 0; e < EPV; ++e) f[e] = __fmul_rn(__fmul_rn(f[e], c[e]), inv_a_static);
-                    store_codes<EPV>(dst, v, f);
-                }
+                for (int e = 0; e < EPV; ++e) f[e] = __fmul_rn(__fmul_rn(f[e], c[e]), inv_a_static);
+                if (v < nvec) store_codes<EPV>(dst, v, f);
             }
             continue;
         }
 
         if constexpr (MODE == ROW_RMSNORM || MODE == ROW_RMS_STAT) {
-            // pass 1: sum of squares in fp64 (exact squares)
+            // pass 1: sum of squares in fp64 (exact squares); REG keeps the
+            // widened row for pass 2
+            float fk[REG ? VPT : 1][REG ? EPV : 1];
             double ss = 0.0;
 #pragma unroll
             for (int i = 0; i < VPT; ++i) {
-                const int64_t v = static_cast<int64_t>(i) * ROW_T + tid;
-                if (v < nvec) {
-                    float f[EPV];
-                    widen<DT>(raw[i], f);
+                float f[EPV];
+                widen<DT>(raw[i], f);
 #pragma unroll
-                    for (int e = 0; e < EPV; ++e) ss += static_cast<double>(f[e]) * static_cast<double>(f[e]);
+                for (int e = 0; e < EPV; ++e) {
+                    ss += static_cast<double>(f[e]) * static_cast<double>(f[e]);
+                    if constexpr (REG) fk[i][e] = f[e];
                 }
             }
             const double tot = block_sum_f64(ss, red64);
@@ -347,21 +357,24 @@ __global__ void __launch_bounds__(ROW_T) k_rows(RowArgs p)
             if (tid == 0 && p.rstd_out != nullptr) p.rstd_out[row] = r_m;
 #pragma unroll
             for (int i = 0; i < VPT; ++i) {
-                const int64_t v = static_cast<int64_t>(i) * ROW_T + tid;
-                if (v < nvec) {
-                    float f[EPV], c[EPV];
+                const int64_t v = static_cast<int64_t>(i) * NT + tid;
+                float f[EPV], c[EPV];
+                if constexpr (REG) {
+#pragma unroll
+                    for (int e = 0; e < EPV; ++e) f[e] = fk[i][e];
+                } else {
                     widen<DT>(raw[i], f);
-                    colc(i, v, c);
-                    if constexpr (MODE == ROW_RMS_STAT) {
+                }
+                colc(i, v, c);
+                if constexpr (MODE == ROW_RMS_STAT) {
 #pragma unroll
-                        for (int e = 0; e < EPV; ++e)
-                            cmax[i][e] = fmaxf(cmax[i][e], fabsf(__fmul_rn(__fmul_rn(f[e], r_m), c[e])));
-                    } else {
+                    for (int e = 0; e < EPV; ++e)
+                        cmax[i][e] = fmaxf(cmax[i][e], fabsf(__fmul_rn(__fmul_rn(f[e], r_m), c[e])));
+                } else {
 #pragma unroll
-                        for (int e = 0; e < EPV; ++e)
-                            f[e] = __fmul_rn(__fmul_rn(__fmul_rn(f[e], r_m), c[e]), inv_a_static);
-                        store_codes<EPV>(dst, v, f);
-                    }
+                    for (int e = 0; e < EPV; ++e)
+                        f[e] = __fmul_rn(__fmul_rn(__fmul_rn(f[e], r_m), c[e]), inv_a_static);
+                    if (v < nvec) store_codes<EPV>(dst, v, f);
                 }
             }
             continue;
@@ -373,17 +386,15 @@ __global__ void __launch_bounds__(ROW_T) k_rows(RowArgs p)
         float mx = 0.0f;
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
-            const int64_t v = static_cast<int64_t>(i) * ROW_T + tid;
-            if (v < nvec) {
-                float f[EPV], c[EPV];
-                widen<DT>(raw[i], f);
-                colc(i, v, c);
+            const int64_t v = static_cast<int64_t>(i) * NT + tid;
+            float f[EPV], c[EPV];
+            widen<DT>(raw[i], f);
+            colc(i, v, c);
 #pragma unroll
-                for (int e = 0; e < EPV; ++e) {
-                    const float y = __fmul_rn(f[e], c[e]);
-                    mx = fmaxf(mx, fabsf(y));
-                    if constexpr (REG) ykeep[i][e] = y;
-                }
+            for (int e = 0; e < EPV; ++e) {
+                const float y = __fmul_rn(f[e], c[e]);
+                mx = fmaxf(mx, fabsf(y));
+                if constexpr (REG) ykeep[i][e] = y;
             }
         }
         const float sc = scale_from_absmax(block_max(mx, red));
@@ -393,19 +404,19 @@ __global__ void __launch_bounds__(ROW_T) k_rows(RowArgs p)
         const bool inrange = (sc == 0.0f) || (sc >= 1.17549435e-38f);
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
-            const int64_t v = static_cast<int64_t>(i) * ROW_T + tid;
+            const int64_t v = static_cast<int64_t>(i) * NT + tid;
+            float f[EPV];
+            if constexpr (REG) {
+#pragma unroll
+                for (int e = 0; e < EPV; ++e) f[e] = __fmul_rn(ykeep[i][e], inv);
+            } else {
+                float c[EPV];
+                widen<DT>(raw[i], f);
+                colc(i, v, c);
+#pragma unroll
+                for (int e = 0; e < EPV; ++e) f[e] = __fmul_rn(__fmul_rn(f[e], c[e]), inv);
+            }
             if (v < nvec) {
-                float f[EPV];
-                if constexpr (REG) {
-#pragma unroll
-                    for (int e = 0; e < EPV; ++e) f[e] = __fmul_rn(ykeep[i][e], inv);
-                } else {
-                    float c[EPV];
-                    widen<DT>(raw[i], f);
-                    colc(i, v, c);
-#pragma unroll
-                    for (int e = 0; e < EPV; ++e) f[e] = __fmul_rn(__fmul_rn(f[e], c[e]), inv);
-                }
                 if (inrange) store_codes<EPV, true>(dst, v, f);
                 else store_codes<EPV, false>(dst, v, f);
             }
@@ -414,12 +425,223 @@ __global__ void __launch_bounds__(ROW_T) k_rows(RowArgs p)
     if constexpr (MODE == ROW_RMS_STAT) {
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
-            const int64_t v = static_cast<int64_t>(i) * ROW_T + tid;
+            const int64_t v = static_cast<int64_t>(i) * NT + tid;
             if (v < nvec) {
 #pragma unroll
                 for (int e = 0; e < EPV; ++e)
                     atomicMax(reinterpret_cast<int *>(p.scale_out + v * EPV + e), __float_as_int(cmax[i][e]));
             }
+        }
+    }
+}
+
+// Static (per-tensor) activation quantisation is elementwise: code(x) =
+// q(fl(fl(x * recip(s_j)) * recip(a))).  It streams like the calibration
+// kernel: a block is a strip of 32 16-byte column vectors x 8 row lanes, each
+// thread keeps its vector's 1/s_j in registers and walks a slab of rows,
+// four rows at a time with the next four rows' loads in flight, writing 8
+// codes (16-bit inputs) or 4 (fp32) per vector: a warp reads 512 and writes
+// 256 contiguous bytes.
+constexpr int QS_TX = 32, QS_TY = 8, QS_UNROLL = 4;
+
+template <int DT, bool STREAM>
+__global__ void __launch_bounds__(QS_TX *QS_TY)
+    k_quant_static(const uint8_t *__restrict__ x, int64_t rows, int64_t nvec, const float *__restrict__ s,
+                   const float *__restrict__ a_in, int64_t row_slab, int8_t *__restrict__ out)
+{
+    constexpr int EPV = VecT<DT>::EPV;
+    const int tx = threadIdx.x, ty = threadIdx.y;
+    const int64_t v = static_cast<int64_t>(blockIdx.x) * QS_TX + tx;
+    const int64_t r0 = static_cast<int64_t>(blockIdx.y) * row_slab;
+    const int64_t r1 = min(rows, r0 + row_slab);
+    const int64_t K = nvec * EPV;
+    pdl_wait();
+    pdl_launch_dependents();
+    if (v >= nvec) return;
+    const uint8_t *col = x + v * 16;
+    auto load = [&](int64_t r) {
+        const uint4 *p = reinterpret_cast<const uint4 *>(col + r * nvec * 16);
+        if constexpr (STREAM) return __ldcs(p);
+        else return __ldg(p);
+    };
+    // first rows in flight before the constants
+    uint4 t[QS_UNROLL];
+    int64_t r = r0 + ty;
+#pragma unroll
+    for (int u = 0; u < QS_UNROLL; ++u)
+        if (r + u * QS_TY < r1) t[u] = load(r + u * QS_TY);
+    float c[EPV];
+    if ((reinterpret_cast<uintptr_t>(s) & 15u) == 0) {
+#pragma unroll
+        for (int h = 0; h < EPV / 4; ++h) {
+            const float4 w = __ldg(reinterpret_cast<const float4 *>(s) + v * (EPV / 4) + h);
+            c[4 * h] = recip_or_zero(w.x); c[4 * h + 1] = recip_or_zero(w.y);
+            c[4 * h + 2] = recip_or_zero(w.z); c[4 * h + 3] = recip_or_zero(w.w);
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) c[e] = recip_or_zero(s[v * EPV + e]);
+    }
+    const float inv_a = recip_or_zero(a_in[0]);
+    auto emit = [&](int64_t row, const uint4 &raw) {
+        float f[EPV];
+        widen<DT>(raw, f);
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) f[e] = __fmul_rn(__fmul_rn(f[e], c[e]), inv_a);
+        int8_t *dst = out + row * K;
+        if constexpr (EPV == 8) {
+            uint2 o;
+            o.x = pack4_bits(quant8_bits(f[0]), quant8_bits(f[1]), quant8_bits(f[2]), quant8_bits(f[3]));
+            o.y = pack4_bits(quant8_bits(f[4]), quant8_bits(f[5]), quant8_bits(f[6]), quant8_bits(f[7]));
+            __stcs(reinterpret_cast<uint2 *>(dst + v * 8), o);
+        } else {
+            __stcs(reinterpret_cast<uint32_t *>(dst + v * 4),
+                   pack4_bits(quant8_bits(f[0]), quant8_bits(f[1]), quant8_bits(f[2]), quant8_bits(f[3])));
+        }
+    };
+    // the next batch of rows is requested before this one is converted
+    for (;;) {
+        const int64_t rn = r + QS_UNROLL * QS_TY;
+        uint4 n[QS_UNROLL];
+#pragma unroll
+        for (int u = 0; u < QS_UNROLL; ++u)
+            if (rn + u * QS_TY < r1) n[u] = load(rn + u * QS_TY);
+#pragma unroll
+        for (int u = 0; u < QS_UNROLL; ++u)
+            if (r + u * QS_TY < r1) emit(r + u * QS_TY, t[u]);
+        if (rn >= r1) break;
+#pragma unroll
+        for (int u = 0; u < QS_UNROLL; ++u) t[u] = n[u];
+        r = rn;
+    }
+}
+
+// Few rows (decode-size activations): a cluster of CS CTAs shares each row,
+// CTA r of the cluster taking the 16-byte vectors [r*vpc, (r+1)*vpc) with
+// vpc = nvec / CS <= ROW_T, one vector per thread.  The row-wide reduction
+// (absmax, or the fp64 sum of squares of RMSNorm) combines the CTAs'
+// partials through distributed shared memory, in rank order, so that every
+// CTA of the cluster obtains the same value; the arithmetic per element is
+// that of k_rows.  grid = (CS, rows), cluster = (CS, 1, 1).
+__device__ __forceinline__ double ld_dsmem_f64(uint32_t addr)
+{
+    double v;
+    asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+template <int DT, int MODE>
+__global__ void __launch_bounds__(ROW_T) k_rows_split(RowArgs p)
+{
+    constexpr int EPV = VecT<DT>::EPV;
+    __shared__ float red[32];
+    __shared__ double red64[32];
+    __shared__ double part;            // this CTA's partial of the row reduction
+    __shared__ double total;           // the combined value
+    const int tid = threadIdx.x;
+    const int cs = static_cast<int>(gridDim.x);
+    const uint32_t rank = ptx::cluster_ctarank();
+    const int64_t row = blockIdx.y;
+    const int64_t nvec = p.K / EPV;
+    const int64_t vpc = nvec / cs;
+    const int64_t v = static_cast<int64_t>(rank) * vpc + tid;
+    const bool act = tid < vpc;
+    pdl_wait();
+    pdl_launch_dependents();
+
+    const uint8_t *src;
+    if (p.src1 != nullptr) {
+        const int64_t b = row >> 6, w = row & 63;
+        src = (w < 32 ? p.src0 : p.src1) + ((b << 5) + (w & 31)) * p.row_bytes;
+    } else {
+        src = p.src0 + row * p.row_bytes;
+    }
+    uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+    if (act) raw = __ldcs(reinterpret_cast<const uint4 *>(src) + v);
+    float c[EPV];
+    if (act) {
+        if (constants_aligned16(p)) {
+#pragma unroll
+            for (int h = 0; h < EPV / 4; ++h) {
+                const float4 t = column_constant4<MODE>(p, v * (EPV / 4) + h);
+                c[4 * h] = t.x; c[4 * h + 1] = t.y; c[4 * h + 2] = t.z; c[4 * h + 3] = t.w;
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < EPV; ++e) c[e] = column_constant<MODE>(p, v * EPV + e);
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) c[e] = 0.0f;
+    }
+    float f[EPV];
+    widen<DT>(raw, f);
+    int8_t *dst = p.out + row * p.K;
+
+    // row-wide value through the cluster: partials in rank order
+    auto cluster_combine = [&](double mine, bool is_max) -> double {
+        if (tid == 0) part = mine;
+        ptx::cluster_sync();                           // every partial written
+        if (tid == 0) {
+            const uint32_t local = ptx::smem_addr(&part);
+            double acc = 0.0;
+            for (int r = 0; r < cs; ++r) {
+                const double o = ld_dsmem_f64(ptx::map_to_rank(local, static_cast<uint32_t>(r)));
+                acc = is_max ? fmax(acc, o) : acc + o;
+            }
+            total = acc;
+        }
+        ptx::cluster_sync();                           // every partial read: peers may exit
+        return total;
+    };
+
+    if constexpr (MODE == ROW_ACT_STATIC) {
+        if (act) {
+            const float inv_a = recip_or_zero(p.a_in[0]);
+#pragma unroll
+            for (int e = 0; e < EPV; ++e) f[e] = __fmul_rn(__fmul_rn(f[e], c[e]), inv_a);
+            store_codes<EPV>(dst, v, f);
+        }
+    } else if constexpr (MODE == ROW_RMSNORM || MODE == ROW_RMS_STAT) {
+        double ss = 0.0;
+        if (act) {
+#pragma unroll
+            for (int e = 0; e < EPV; ++e) ss += static_cast<double>(f[e]) * static_cast<double>(f[e]);
+        }
+        const double tot = cluster_combine(block_sum_f64(ss, red64), false);
+        const float mean = __double2float_rn(tot / static_cast<double>(p.K));
+        const float r_m = __frcp_rn(__fsqrt_rn(__fadd_rn(mean, p.eps)));
+        if (rank == 0 && tid == 0 && p.rstd_out != nullptr) p.rstd_out[row] = r_m;
+        if (act) {
+            if constexpr (MODE == ROW_RMS_STAT) {
+#pragma unroll
+                for (int e = 0; e < EPV; ++e)
+                    atomicMax(reinterpret_cast<int *>(p.scale_out + v * EPV + e),
+                              __float_as_int(fabsf(__fmul_rn(__fmul_rn(f[e], r_m), c[e]))));
+            } else {
+                const float inv_a = recip_or_zero(p.a_in[0]);
+#pragma unroll
+                for (int e = 0; e < EPV; ++e) f[e] = __fmul_rn(__fmul_rn(__fmul_rn(f[e], r_m), c[e]), inv_a);
+                store_codes<EPV>(dst, v, f);
+            }
+        }
+    } else {
+        // ROW_WEIGHT / ROW_ACT_TOKEN: y = fl(x * c_j), row absmax, codes of fl(y * recip(scale))
+        float mx = 0.0f;
+#pragma unroll
+        for (int e = 0; e < EPV; ++e) {
+            f[e] = __fmul_rn(f[e], c[e]);
+            mx = fmaxf(mx, fabsf(f[e]));
+        }
+        const float rmax = static_cast<float>(cluster_combine(static_cast<double>(block_max(mx, red)), true));
+        const float sc = scale_from_absmax(rmax);
+        const float inv = recip_or_zero(sc);
+        if (rank == 0 && tid == 0) p.scale_out[row] = sc;
+        if (act) {
+#pragma unroll
+            for (int e = 0; e < EPV; ++e) f[e] = __fmul_rn(f[e], inv);
+            if ((sc == 0.0f) || (sc >= 1.17549435e-38f)) store_codes<EPV, true>(dst, v, f);
+            else store_codes<EPV, false>(dst, v, f);
         }
     }
 }
