@@ -277,14 +277,16 @@ sq_status sq_gemm_s32(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, 
  * g, u the fp32 dequant values (no bias) of the gate and up rows of output
  * channel c:
  *
- *   h[m,c] = RN_bf16(fl(fl(g / fl(1 + expf(-g))) * u))
+ *   h[m,c] = RN_bf16(fl(silu(g) * u)),  silu(g) = g / (1 + exp(-g))
  *
  * h: bf16 [M, N_h] or NULL.  If hq != NULL the epilogue also smooths and
  * quantises h for the next linear with a static scale:
  *   hq[m,c] = q(fl(fl(h[m,c] * recip(s2_c)) * recip(a2[0])))
  * using the bf16-rounded h (so it equals sq_smooth_quant_act on h).
  * s2: fp32 [N_h], a2: fp32 [1] (required with hq).  N_h a multiple of 128.
- * expf is CUDA's; h matches a correctly rounded SiLU within 2 bf16 ulp. */
+ * silu(g) is computed in fp32 with CUDA's fast exponential and division
+ * intrinsics (errors of a few fp32 ulp, far below bf16's 8 bits); h matches
+ * a correctly rounded SiLU within 2 bf16 ulp (or 1e-30 absolute). */
 sq_status sq_linear_w8a8_gateup_silu(const int8_t *xq, const int8_t *wq_gu, int64_t M,
                                      int64_t N_h, int64_t K, const float *a_scale,
                                      sq_act_mode mode, const float *w_scale_gu, void *h,

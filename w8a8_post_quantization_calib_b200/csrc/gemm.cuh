@@ -172,9 +172,14 @@ __device__ __forceinline__ float dequant(int32_t acc, float c, const void *bias,
 // ---------------------------------------------------------------------------
 // Epilogue of one tile, normal orientation (TMEM lane = token row m).
 // ---------------------------------------------------------------------------
+// Gate/up (EPI_GATEUP): ws_tile holds the tile's BN w_scale values and
+// s2inv_tile the BN/2 channels' fl(1/s2), staged in shared memory while the
+// tile's MMAs ran.  SiLU uses the fast exponential and division (h is
+// rounded to bf16 afterwards: a few fp32 ulp are far below its precision).
 template <int BN, int KIND, int EPI>
 __device__ __forceinline__ void epilogue_normal(const Params &p, uint32_t tbase, int tr, int tc, int q,
-                                                int lane)
+                                                int lane, const float *ws_tile = nullptr,
+                                                const float *s2inv_tile = nullptr)
 {
     const int m = tr * BM + q * 32 + lane;
     const bool mok = m < p.M;
@@ -198,9 +203,9 @@ __device__ __forceinline__ void epilogue_normal(const Params &p, uint32_t tbase,
             float h[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                const float g = __fmul_rn(__int2float_rn(static_cast<int32_t>(rg[i])), __fmul_rn(am, p.w_scale[row0 + i]));
-                const float u = __fmul_rn(__int2float_rn(static_cast<int32_t>(ru[i])), __fmul_rn(am, p.w_scale[row0 + 32 + i]));
-                const float sg = __fdiv_rn(g, __fadd_rn(1.0f, expf(-g)));
+                const float g = __fmul_rn(__int2float_rn(static_cast<int32_t>(rg[i])), __fmul_rn(am, ws_tile[c * 64 + i]));
+                const float u = __fmul_rn(__int2float_rn(static_cast<int32_t>(ru[i])), __fmul_rn(am, ws_tile[c * 64 + 32 + i]));
+                const float sg = __fdividef(g, __fadd_rn(1.0f, __expf(-g)));
                 h[i] = __bfloat162float(__float2bfloat16_rn(__fmul_rn(sg, u)));   // h as bf16
             }
             if (!mok) continue;
@@ -216,7 +221,7 @@ __device__ __forceinline__ void epilogue_normal(const Params &p, uint32_t tbase,
                     int qv[4];
 #pragma unroll
                     for (int t = 0; t < 4; ++t)
-                        qv[t] = quant8(__fmul_rn(__fmul_rn(h[i + t], recip_or_zero(p.s2[ch0 + i + t])), inv_a2));
+                        qv[t] = quant8(__fmul_rn(__fmul_rn(h[i + t], s2inv_tile[c * 32 + i + t]), inv_a2));
                     w[i / 4] = pack4(qv[0], qv[1], qv[2], qv[3]);
                 }
                 uint4 *dst = reinterpret_cast<uint4 *>(p.hq + o);
@@ -927,6 +932,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 }
                 const int m = (2 * tr + static_cast<int>(rank)) * BM + q * 32 + lane;
                 if (m < p.M) am = p.per_token ? p.a_scale[m] : p.a_scale[0];
+            } else if constexpr (EPI == EPI_GATEUP) {
+                // w_scale of the tile's gate/up rows, fl(1/s2) of its channels
+                const int et = threadIdx.x - 64;
+                for (int t = et; t < BN; t += 128) {
+                    const int n = tc * BN + t;
+                    ws_tile[t] = n < p.N ? p.w_scale[n] : 0.0f;
+                }
+                if (p.hq != nullptr) {
+                    for (int t = et; t < BN / 2; t += 128) {
+                        const int ch = (tc * BN) / 2 + t;
+                        bias_tile[t] = ch < (p.N >> 1) ? recip_or_zero(p.s2[ch]) : 0.0f;
+                    }
+                }
             }
             // one thread waits for the accumulator; the 128 epilogue threads
             // then take the same decision (no warp is left at a barrier alone)
@@ -937,7 +955,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * BN);
             // this CTA's accumulator rows are the tile's rows rank*128 .. rank*128+127
             if constexpr (EPI == EPI_GATEUP)
-                epilogue_normal<BN, KIND, EPI>(p, tbase, 2 * tr + static_cast<int>(rank), tc, q, lane);
+                epilogue_normal<BN, KIND, EPI>(p, tbase, 2 * tr + static_cast<int>(rank), tc, q, lane, ws_tile,
+                                               bias_tile);
             else
                 epilogue_tma<BN, KIND, EPI>(p, &map_o, tbase, 2 * tr + static_cast<int>(rank), tc, q, lane, stg,
                                             nstore, ws_tile, bias_tile, am);
