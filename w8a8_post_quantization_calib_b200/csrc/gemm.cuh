@@ -639,7 +639,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // buffers per warp: a buffer is reused only after the store issued from it
 // two boxes earlier has finished reading shared memory.
 // ---------------------------------------------------------------------------
-template <int BN, int KIND, int EPI>
+template <int BN, int KIND, int EPI, int NBUF>
 __device__ __forceinline__ void epilogue_tma(const Params &p, const CUtensorMap *omap, uint32_t tbase, int tr,
                                              int tc, int q, int lane, uint32_t stg, int &nstore,
                                              const float *ws_tile, const float *bias_tile, float am)
@@ -694,9 +694,15 @@ __device__ __forceinline__ void epilogue_tma(const Params &p, const CUtensorMap 
                 }
             }
         }
-        if (lane == 0 && nstore >= 2) ptx::bulk_wait_read_1();
+        // a staging buffer is rewritten only once the store issued from it has
+        // finished reading shared memory
+        if constexpr (NBUF == 2) {
+            if (lane == 0 && nstore >= 2) ptx::bulk_wait_read_1();
+        } else {
+            if (lane == 0 && nstore >= 1) ptx::bulk_wait_read_0();
+        }
         __syncwarp();
-        const uint32_t buf = stg + static_cast<uint32_t>(nstore & 1) * STG_BYTES;
+        const uint32_t buf = stg + static_cast<uint32_t>(NBUF == 2 ? (nstore & 1) : 0) * STG_BYTES;
         if (wide) {                           // 128-byte rows, 128-byte swizzle: chunk ^= row & 7
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
@@ -745,12 +751,16 @@ struct PairCfg {
     static constexpr int A_BYTES = A_KB * KBO;
     static constexpr int B_BYTES = B_KB * KBO;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int STAGES_RAW = (188 * 1024) / STAGE_BYTES;
+    // epilogue staging: 2 buffers per epilogue warp, 1 for the 256-wide
+    // two-block tile, which needs the room for a third stage
+    static constexpr int STG_BUFS = (KBO > 1 && BN == 256) ? 1 : 2;
+    static constexpr int STG_TOTAL = 4 * STG_BUFS * STG_BYTES;
+    static constexpr int COLS_BYTES = 2 * 2 * 256 * 4;    // per accumulator buffer: w_scale + bias, 256 each
+    static constexpr int FIXED_BYTES = 1024 + STG_TOTAL + COLS_BYTES + 256;
+    static constexpr int STAGES_RAW = (227 * 1024 - FIXED_BYTES) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_RAW > 10 ? 10 : STAGES_RAW;
     static constexpr int TMEM_COLS = pow2_at_least(2 * BN, 32);
-    static constexpr int STG_TOTAL = 4 * 2 * STG_BYTES;   // 4 epilogue warps x 2 buffers
-    static constexpr int COLS_BYTES = 2 * 2 * 256 * 4;    // per accumulator buffer: w_scale + bias, 256 each
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STG_TOTAL + COLS_BYTES + 256;
+    static constexpr int SMEM_BYTES = FIXED_BYTES + STAGES * STAGE_BYTES;
     static_assert(STAGE_BYTES % 1024 == 0, "stage must keep 1024-byte alignment");
     static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "pair MMA N");
     static_assert(TMEM_COLS <= 512, "two accumulators must fit TMEM");
@@ -910,7 +920,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     } else {
         // ------------------------------------------------ epilogue (warps 2..5, both CTAs)
         const int q = warp & 3;
-        const uint32_t stg = stg_base + static_cast<uint32_t>((warp - 2) * 2 * STG_BYTES);
+        const uint32_t stg = stg_base + static_cast<uint32_t>((warp - 2) * C::STG_BUFS * STG_BYTES);
         int nstore = 0;
         int local = 0;
         for (int u = cluster; u < p.num_units; u += nclusters, ++local) {
@@ -958,7 +968,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 epilogue_normal<BN, KIND, EPI>(p, tbase, 2 * tr + static_cast<int>(rank), tc, q, lane, ws_tile,
                                                bias_tile);
             else
-                epilogue_tma<BN, KIND, EPI>(p, &map_o, tbase, 2 * tr + static_cast<int>(rank), tc, q, lane, stg,
+                epilogue_tma<BN, KIND, EPI, C::STG_BUFS>(p, &map_o, tbase, 2 * tr + static_cast<int>(rank), tc, q, lane, stg,
                                             nstore, ws_tile, bias_tile, am);
             ptx::tc_fence_before();
             __syncwarp();

@@ -295,9 +295,10 @@ int pick_pair_bn(int64_t M, int64_t N)
     const int64_t clusters = std::max(1, sm_count() / 2);
     const int cands[3] = {256, 192, 128};
     // measured time per output column of a full wave relative to the 256-wide
-    // tile (narrower tiles move more operand bytes per MAC; the 192-wide one
-    // with two K blocks per load: Llama-7B QKV / MLP and 13B shapes)
-    const double eff[3] = {1.0, 0.89, 0.77};
+    // tile (narrower tiles move more operand bytes per MAC), both with two K
+    // blocks per load, on the Llama-7B QKV and MLP shapes; the 128-wide
+    // figure predates the two-block loads
+    const double eff[3] = {1.0, 0.85, 0.77};
     int best = 256;
     double best_cost = -1.0;
     for (int i = 0; i < 3; ++i) {
@@ -318,11 +319,13 @@ sq_status dispatch_pair(gemm::Params &p, const void *a, const void *b, cudaStrea
     const int bn = force_bn ? force_bn : pick_pair_bn(p.M, p.N);
     fill_tiles_pair(p, bn, KIND == gemm::KIND_F16 ? 2 : 1);
     if constexpr (KIND == gemm::KIND_I8) {
-        // 192-wide tiles: two K blocks per TMA load (3 stages of 56 KB hold
-        // the same 6 blocks as 6 single-block stages, with half the loads);
-        // the 256-wide tile would drop to 2 stages, so it keeps single blocks
-        if (bn == 192 && (p.K % 128) == 0) {
+        // two K blocks per TMA load: 3 stages of 56 KB (192-wide) hold the
+        // same 6 blocks as 6 single-block stages with half the loads; the
+        // 256-wide tile fits 3 stages of 64 KB with one epilogue staging
+        // buffer per warp
+        if ((bn == 192 || bn == 256) && (p.K % 128) == 0) {
             p.num_kb = static_cast<int>(cdiv(p.num_kb, 2));
+            if (bn == 256) return launch_gemm2<256, KIND, EPI, 2>(p, a, b, st);
             return launch_gemm2<192, KIND, EPI, 2>(p, a, b, st);
         }
     }
