@@ -693,7 +693,10 @@ def run_workload(args):
             gbs = nbytes / (t_ms * 1e-3) / 1e9
             lines.append({"kernel": name, "shape": shape, "dtype": dt, "us": t_ms * 1e3, "gbs": gbs,
                           "frac_hbm": gbs / P["hbm_gbs"]})
-        for K, dt in ((4096, torch.float16), (8192, torch.bfloat16)):
+        shapes = ((4096, torch.float16), (8192, torch.bfloat16))
+        if args.rows_k:
+            shapes = tuple(sh for sh in shapes if sh[0] in {int(k) for k in args.rows_k.split(",")})
+        for K, dt in shapes:
             M = R // K
             X = torch.randn(M, K, generator=g16, device="cuda").to(dt)
             name = "f16" if dt == torch.float16 else "bf16"
@@ -732,6 +735,7 @@ def main():
                     help="mlp7b workload: comma-separated token counts M to sweep")
     ap.add_argument("--proj", default="up,down", help="mlp7b workload: projections to sweep")
     ap.add_argument("--only", default="", help="rows workload: comma-separated kernels to run (default all)")
+    ap.add_argument("--rows-k", default="", help="rows workload: row lengths to run, of 4096 (fp16) and 8192 (bf16)")
     ap.add_argument("--workload", choices=["qkv7b", "mlp7b", "alpha13b", "mlp70b", "rows"], default="qkv7b",
                     help="qkv7b is the bench line; the others print per-kernel measurements of the other workloads")
     args = ap.parse_args()
