@@ -63,7 +63,7 @@ def gemm_traffic():
     try:
         d = json.load(open(tf))
         h = hashlib.sha256()
-        for f in ("gemm.cuh", "ptx_sm100.cuh"):
+        for f in ("gemm.cuh", "ptx_sm100.cuh", "libsq.cu"):
             h.update(open(os.path.join(ROOT, "w8a8_post_quantization_calib_b200", "csrc", f), "rb").read())
         return d["dram_bytes_per_launch"] if h.hexdigest()[:16] == d["source_sha256_16"] else None
     except Exception:

@@ -293,15 +293,15 @@ void fill_tiles_pair(gemm::Params &p, int bn, int kb_bytes_per_elem)
 int pick_pair_bn(int64_t M, int64_t N)
 {
     const int64_t clusters = std::max(1, sm_count() / 2);
-    const int cands[3] = {256, 192, 128};
+    const int cands[4] = {256, 224, 192, 128};
     // measured time per output column of a full wave relative to the 256-wide
-    // tile (narrower tiles move more operand bytes per MAC), both with two K
+    // tile (narrower tiles move more operand bytes per MAC), all with two K
     // blocks per load, on the Llama-7B QKV and MLP shapes; the 128-wide
     // figure predates the two-block loads
-    const double eff[3] = {1.0, 0.85, 0.77};
+    const double eff[4] = {1.0, 0.92, 0.85, 0.77};
     int best = 256;
     double best_cost = -1.0;
-    for (int i = 0; i < 3; ++i) {
+    for (int i = 0; i < 4; ++i) {
         const int bn = cands[i];
         const int64_t tiles = cdiv(M, 2 * gemm::BM) * cdiv(N, bn);
         const double cost = static_cast<double>(cdiv(tiles, clusters) * bn) / eff[i];
@@ -323,14 +323,16 @@ sq_status dispatch_pair(gemm::Params &p, const void *a, const void *b, cudaStrea
         // same 6 blocks as 6 single-block stages with half the loads; the
         // 256-wide tile fits 3 stages of 64 KB with one epilogue staging
         // buffer per warp
-        if ((bn == 192 || bn == 256) && (p.K % 128) == 0) {
+        if (bn >= 192 && (p.K % 128) == 0) {
             p.num_kb = static_cast<int>(cdiv(p.num_kb, 2));
             if (bn == 256) return launch_gemm2<256, KIND, EPI, 2>(p, a, b, st);
+            if (bn == 224) return launch_gemm2<224, KIND, EPI, 2>(p, a, b, st);
             return launch_gemm2<192, KIND, EPI, 2>(p, a, b, st);
         }
     }
     switch (bn) {
     case 256: return launch_gemm2<256, KIND, EPI, 1>(p, a, b, st);
+    case 224: return launch_gemm2<224, KIND, EPI, 1>(p, a, b, st);
     case 192: return launch_gemm2<192, KIND, EPI, 1>(p, a, b, st);
     default: return launch_gemm2<128, KIND, EPI, 1>(p, a, b, st);
     }
