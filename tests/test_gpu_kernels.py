@@ -157,6 +157,61 @@ def test_smooth_quant_act(dt, M, K, mode):
     assert bits_equal(host(xq), xq_ref), mismatch_report(host(xq), xq_ref)
 
 
+@pytest.mark.parametrize("M", [1, 3, 100, 147])
+@pytest.mark.parametrize("K,dt", [(2048, BF16), (4096, F16), (8192, BF16), (11008, BF16), (2048, F32)])
+def test_row_split_kernels(M, K, dt):
+    """Fewer rows than SMs take the cluster-split kernel (2, 4 or 8 CTAs per
+    row, row reductions through distributed shared memory): per-token
+    activation quant, weight transform and RMSNorm + quant, bit for bit."""
+    X = rand_x(M * 7 + K, (M, K), dt, 1.5, outliers=min(8, K // 100))
+    g = np.random.default_rng(M + K)
+    s = (np.abs(g.standard_normal(K)) + 0.3).astype(np.float32)
+    xq = torch.empty(M, K, dtype=torch.int8, device="cuda")
+    at = torch.empty(M, dtype=torch.float32, device="cuda")
+    sq.smooth_quant_act(dev(X, dt), dev(s), oracle.PER_TOKEN, at, xq)
+    _sync()
+    xq_ref, a_ref = oracle.smooth_quant_act(X, s, oracle.PER_TOKEN, None, dt)
+    assert bits_equal(host(at), a_ref), mismatch_report(host(at), a_ref)
+    assert bits_equal(host(xq), xq_ref), mismatch_report(host(xq), xq_ref)
+    ws = torch.empty(M, dtype=torch.float32, device="cuda")
+    sq.quant_weight(dev(X, dt), dev(s), xq, ws)
+    _sync()
+    wq_ref, ws_ref = oracle.quant_weight(X, s, dt)
+    assert bits_equal(host(ws), ws_ref), mismatch_report(host(ws), ws_ref)
+    assert bits_equal(host(xq), wq_ref), mismatch_report(host(xq), wq_ref)
+    if dt != F32:
+        gamma = g.uniform(0.5, 1.5, K).astype(np.float32)
+        a = np.float32(0.04)
+        r = torch.empty(M, dtype=torch.float32, device="cuda")
+        sq.rmsnorm_quant(dev(X, dt), dev(gamma), dev(s), 1e-5, dev(np.array([a])), xq, r)
+        _sync()
+        xq_ref, r_ref = oracle.rmsnorm_quant(X, gamma, s, 1e-5, a, dt)
+        assert bits_equal(host(r), r_ref), mismatch_report(host(r), r_ref)
+        assert bits_equal(host(xq), xq_ref), mismatch_report(host(xq), xq_ref)
+        am = torch.zeros(K, dtype=torch.float32, device="cuda")
+        sq.rmsnorm_absmax(dev(X, dt), dev(gamma), 1e-5, am)
+        _sync()
+        am_ref = oracle.rmsnorm_absmax(X, gamma, 1e-5, dt)
+        assert bits_equal(host(am), am_ref), mismatch_report(host(am), am_ref)
+
+
+@pytest.mark.parametrize("M,K,dt", [(1, 16, F16), (37, 4104, BF16), (2049, 520, F32), (600, 4096, F16)])
+def test_quant_static_streaming_misaligned_s(M, K, dt):
+    """Static-scale quantisation (column strips x row slabs) with a 1/s vector
+    that is not 16-byte aligned (scalar constant path) and ragged slabs."""
+    X = rand_x(M + K * 5, (M, K), dt, 2.0, outliers=min(8, K // 10))
+    s = (np.abs(np.random.default_rng(K).standard_normal(K)) + 0.2).astype(np.float32)
+    s_buf = torch.zeros(K + 1, dtype=torch.float32, device="cuda")
+    s_buf[1:] = dev(s)
+    s_view = s_buf[1:]                              # 4-byte offset
+    a = np.float32(20.0 / 127)
+    xq = torch.empty(M, K, dtype=torch.int8, device="cuda")
+    sq.smooth_quant_act(dev(X, dt), s_view, oracle.STATIC, dev(np.array([a], np.float32)), xq)
+    _sync()
+    xq_ref, _ = oracle.smooth_quant_act(X, s, oracle.STATIC, a, dt)
+    assert bits_equal(host(xq), xq_ref), mismatch_report(host(xq), xq_ref)
+
+
 # ------------------------------------------------------------------ a8
 @pytest.mark.parametrize("M,d", [(300, 8192), (5, 1000), (1, 4096)])
 @pytest.mark.parametrize("random_gamma", [False, True])
