@@ -81,12 +81,16 @@ int sq_last_cuda_error(void);
  * runs out records SQ_ERR_TIMEOUT and the kernel returns without hanging. */
 void sq_set_wait_timeout_ns(unsigned long long ns);
 
-/* Failure-detection test hook (off by default).  what = 1: in every GEMM
- * launched afterwards, the producer warp of CTA 0 withholds its first
- * pipeline stage (no arrival, no load), so the MMA warp's bounded wait on
- * that stage runs out: the kernel records SQ_ERR_TIMEOUT, drains what it had
- * in flight and returns, and the CUDA context stays usable.  what = 0 turns
- * it off.  Nothing faults, traps or hangs. */
+/* Test hooks (off by default), bit flags of `what`:
+ *   1: failure detection.  In every GEMM launched afterwards, the producer
+ *      warp of CTA 0 withholds its first pipeline stage (no arrival, no
+ *      load), so the MMA warp's bounded wait on that stage runs out: the
+ *      kernel records SQ_ERR_TIMEOUT, drains what it had in flight and
+ *      returns, and the CUDA context stays usable.  Nothing faults, traps or
+ *      hangs.
+ *   2: small-M GEMMs run without the cluster split (on the stream-K or
+ *      one-tile-per-CTA schedules), so that tests reach those paths.
+ * what = 0 turns both off. */
 void sq_debug_inject(int what);
 
 /* Synchronises `stream`, then returns SQ_ERR_TIMEOUT if any kernel of this
@@ -216,16 +220,20 @@ sq_status sq_rmsnorm_absmax(const void *x, sq_dtype dt, int64_t M, int64_t d, co
  * memory tiles, TMEM int32 accumulators; CTA pairs with cta_group::2 for
  * M > 128).  Small M (<= 128) takes a weight-streaming path (weights fill the
  * 128-row MMA, tokens are its N).  When one 128-row weight tile per SM would
- * leave many SMs idle, that path shares the (tile, K block) iterations evenly
- * among the SMs (stream-K) if `workspace` holds sq_linear_workspace_size(M,
- * N, K) bytes (16-byte aligned; the size depends on the current device's SM
- * count and is 0 when no sharing is planned): one BM x BN int32 partial-sum
- * slot per CTA plus one int32 arrival counter per weight tile.  The counters
- * must be zero before the first use of a workspace (e.g. cudaMemsetAsync
- * once) and are left zero by every call; the slots need no initialisation.
- * Without a workspace (NULL or too small) the small-M path runs one tile per
- * CTA.  Results are bit-identical either way (exact int32 sums).  Calls
- * sharing one workspace must not overlap on the GPU.
+ * leave more than half of the SMs idle, a cluster of 2 or 4 CTAs shares each
+ * tile's K range and combines the int32 partial sums in distributed shared
+ * memory; no workspace is needed.  The stream-K schedule (iterations shared
+ * evenly among the SMs, partial sums through global memory) is the fallback
+ * when the cluster split is off (sq_debug_inject bit 2); it needs
+ * `workspace` of sq_linear_workspace_size(M, N, K) bytes (16-byte aligned;
+ * the size depends on the current device's SM count and the test hooks, and
+ * is 0 when no workspace is used): one BM x BN int32 partial-sum slot per CTA
+ * plus one int32 arrival counter per weight tile.  The counters must be zero
+ * before the first use of a workspace (e.g. cudaMemsetAsync once) and are
+ * left zero by every call; the slots need no initialisation.  Without a
+ * workspace (NULL or too small) that path runs one tile per CTA.  Results are
+ * bit-identical on every schedule (exact int32 sums).  Calls sharing one
+ * workspace must not overlap on the GPU.
  * ------------------------------------------------------------------------- */
 size_t sq_linear_workspace_size(int64_t M, int64_t N, int64_t K);
 
@@ -239,12 +247,13 @@ sq_status sq_linear_w8a8(const int8_t *xq, const int8_t *wq, int64_t M, int64_t 
  * all: a plugin running inside a host engine that owns every device buffer
  * and hands it only inputs and outputs, or a latency-critical serving loop
  * that must not pay cudaMalloc's implicit device-wide synchronisation.  This
- * call takes no workspace: the small-M stream-K path (M <= 128) keeps its
- * int32 partial sums and per-tile counters in a fixed array inside the
- * library (8 MiB of partial-sum slots + 64 KiB of counters, held by every
- * GPU that loads the library until the process exits; the number of CTAs
- * sharing the iterations is capped by how many slots fit, and the path runs
- * one tile per CTA when too few fit).  M*N beyond
+ * call takes no workspace: the small-M cluster split needs none, and the
+ * small-M stream-K fallback (M <= 128, cluster split off) keeps its int32
+ * partial sums and per-tile counters in a fixed array inside the library
+ * (8 MiB of partial-sum slots + 64 KiB of counters, held by every GPU that
+ * loads the library until the process exits; the number of CTAs sharing the
+ * iterations is capped by how many slots fit, and the path runs one tile per
+ * CTA when too few fit).  M*N beyond
  * sq_linear_w8a8_noalloc_max_elems() (2^21 = 2097152) on that path returns
  * SQ_ERR_UNSUPPORTED without launching; M > 128 needs no scratch and runs the
  * sq_linear_w8a8 launch.  The call allocates nothing: no cudaMalloc,

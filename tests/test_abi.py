@@ -36,8 +36,14 @@ def test_host_only_entry_points_without_gpu():
     assert lib.sq_status_string(0) == b"SQ_OK"
     assert lib.sq_status_string(5) == b"SQ_ERR_TIMEOUT"
     # sizes are pure host arithmetic
-    assert sq.linear_workspace_size(16, 4096, 11008) >= 16 * 4096 * 4
+    # the small-M cluster split combines partial sums on chip: no workspace
+    assert sq.linear_workspace_size(16, 4096, 11008) == 0
     assert sq.linear_workspace_size(4096, 4096, 11008) == 0
+    lib.sq_debug_inject(2)                   # cluster split off: stream-K slots + counters
+    try:
+        assert sq.linear_workspace_size(16, 4096, 11008) >= 16 * 4096 * 4
+    finally:
+        lib.sq_debug_inject(0)
     assert sq.alpha_search_workspace_size(512, 13824, 5120, 4) > 13824 * 5120
 
 

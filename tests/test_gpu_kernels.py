@@ -289,15 +289,28 @@ def test_linear_w8a8(M, N, K, out_dt, mode, with_bias, with_ws):
         assert bits_equal(got, ref), mismatch_report(got, ref)
 
 
+@pytest.fixture
+def _no_cluster_split():
+    sq.lib().sq_debug_inject(2)
+    try:
+        yield
+    finally:
+        sq.lib().sq_debug_inject(0)
+
+
 @pytest.mark.parametrize("M,N,K", [(1, 4096, 11008), (16, 4096, 4096), (5, 1024, 4112), (32, 2048, 8192),
                                    (17, 4096, 11008), (3, 256, 65536), (1, 11008, 4096), (33, 11008, 4112),
-                                   (100, 4096, 4096), (128, 18944, 256), (64, 1040, 528)])
-def test_linear_w8a8_stream_k(M, N, K):
-    """Small-M path with a workspace (the (tile, K block) iterations shared
-    evenly by the SMs, partial sums of shared tiles combined by the last CTA)
-    against the one-tile-per-CTA launch without one, bit for bit, twice (the
-    arrival counters must come back reset), and against the oracle on sampled
-    output channels (first, last and random rows of W)."""
+                                   (100, 4096, 4096), (128, 18944, 256), (64, 1040, 528), (128, 2048, 11008)])
+@pytest.mark.parametrize("schedule", ["cluster", "stream_k"])
+def test_linear_w8a8_small_m_schedules(M, N, K, schedule, request):
+    """Small-M path on its schedules -- the cluster split (2 or 4 CTAs per
+    weight tile, partial sums combined in distributed shared memory) and,
+    with the cluster split off, the stream-K schedule with a workspace --
+    against the one-tile-per-CTA launch, bit for bit, twice (the stream-K
+    arrival counters must come back reset), and against the oracle on
+    sampled output channels (first, last and random rows of W)."""
+    if schedule == "stream_k":
+        request.getfixturevalue("_no_cluster_split")
     g = np.random.default_rng(M * 5 + N + K)
     A = g.integers(-127, 128, (M, K), dtype=np.int8)
     B = g.integers(-127, 128, (N, K), dtype=np.int8)
@@ -306,7 +319,11 @@ def test_linear_w8a8_stream_k(M, N, K):
     bias = synth.cast(g.standard_normal(N).astype(np.float32), BF16)
     dA, dB, da, dws, db = dev(A), dev(B), dev(a), dev(ws), dev(bias, BF16)
     y0 = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    hook = 2 if schedule == "stream_k" else 0
+    sq.lib().sq_debug_inject(2)                     # reference: one tile per CTA (no workspace)
     sq.linear_w8a8(dA, dB, da, oracle.PER_TOKEN, dws, y0, bias=db)
+    _sync()
+    sq.lib().sq_debug_inject(hook)
     n = sq.linear_workspace_size(M, N, K)
     work = torch.zeros(max(16, n), dtype=torch.uint8, device="cuda")
     for _ in range(2):

@@ -58,14 +58,26 @@ def _call_with_workspace(xq, wq, a, mode, ws, bias, y):
     return st
 
 
+@pytest.fixture(params=[0, 2], ids=["cluster_split", "stream_k_scratch"])
+def _hook(request):
+    """0: default schedules (the small-M cluster split needs no scratch);
+    2: cluster split off, so the small-M path shares tiles through the
+    library's fixed scratch array."""
+    sq.lib().sq_debug_inject(request.param)
+    try:
+        yield request.param
+    finally:
+        sq.lib().sq_debug_inject(0)
+
+
 @pytest.mark.parametrize("M,N,K,mode,out_dt,with_bias", [
-    (16, 4096, 11008, 1, 2, False),     # decode-size down projection: split-K over the fixed array
+    (16, 4096, 11008, 1, 2, False),     # decode-size down projection: tiles shared across CTAs
     (1, 11008, 4096, 1, 2, True),
     (64, 2048, 1024, 0, 1, True),
     (128, 1024, 4096, 0, 0, False),
     (300, 528, 1040, 1, 1, True),       # large M: no scratch needed
 ])
-def test_noalloc_matches_workspace_entry_point(M, N, K, mode, out_dt, with_bias):
+def test_noalloc_matches_workspace_entry_point(M, N, K, mode, out_dt, with_bias, _hook):
     xq, wq, a, ws, bias = _operands(M, N, K, mode, out_dt, M * 31 + N)
     bias = bias if with_bias else None
     y_ref = torch.empty(M, N, dtype=_OUT[out_dt], device="cuda")
@@ -78,7 +90,7 @@ def test_noalloc_matches_workspace_entry_point(M, N, K, mode, out_dt, with_bias)
         assert torch.equal(y.view(torch.uint8), y_ref.view(torch.uint8))
 
 
-def test_noalloc_back_to_back_different_shapes():
+def test_noalloc_back_to_back_different_shapes(_hook):
     """A smaller call after a larger one must not see the larger call's leftovers."""
     big = _operands(64, 8192, 4096, 1, 2, 1)
     small = _operands(16, 1024, 4096, 1, 2, 2)

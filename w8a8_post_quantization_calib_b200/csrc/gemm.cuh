@@ -68,9 +68,10 @@ struct TileCfg {
     static constexpr int STAGES = STAGES_RAW > 12 ? 12 : STAGES_RAW;
     static constexpr int TMEM_COLS = pow2_at_least(2 * BN, 32);
     static constexpr int CW = BN < 32 ? BN : 32;   // TMEM columns per epilogue load
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 512;
     static_assert(STAGE_BYTES % 1024 == 0, "stage must keep 1024-byte alignment");
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
+    static_assert((2 * STAGES + 7) * 8 + 16 <= 512, "barrier area");
 };
 
 struct Params {
@@ -448,11 +449,100 @@ __device__ __forceinline__ bool epilogue_sk(const Params &p, uint32_t tbase, int
 // 128-row swizzle tile each) -- a single CTA streams far more bytes per
 // second with fewer, larger loads.  An iteration is then a group of KBO
 // blocks; blocks past K are zero-filled.
-template <int BN, int EPI, int KBO>
+// Epilogue of the cluster split (CS > 1): the CS CTAs of a cluster share one
+// weight tile's K range equally (the stream-K partition with sk_ctas = tiles
+// x CS never crosses a tile).  Once its own MMAs are done, the leader (rank
+// 0) no longer needs its pipeline stages: it releases them to the others,
+// which store their int32 partial sums there through distributed shared
+// memory ([rank-1][BN][BM] int32) and arrive on its barrier; the leader adds
+// them to its own accumulator and applies the epilogue.  Every wait is
+// bounded.
+template <int BN, int EPI, int CS, typename TfullWait>
+__device__ __forceinline__ bool epilogue_cs(const Params &p, uint32_t tbase, int tr, int tc, int q, int lane,
+                                            uint32_t rank, float wsn, float bn, const float *s_am,
+                                            TfullWait tfull_wait, uint32_t go_bar, uint32_t part_bar,
+                                            uint32_t sbase, volatile int *abort_flag)
+{
+    constexpr int CW = TileCfg<BN>::CW;
+    const int r = q * 32 + lane;
+    const int n = tr * BM + r;
+    const bool nok = n < p.N;
+    const int m0 = tc * BN;
+    const int mval = min(BN, p.M - m0);
+    if (!tfull_wait()) return false;
+    ptx::tc_fence_after();
+    if (rank == 0) {
+        // this CTA's stages are no longer read: the others may write them
+        if (q == 2 && lane >= 1 && lane < CS) ptx::mbar_arrive_cluster(ptx::map_to_rank(go_bar, lane));
+        int ok = 1;
+        if (lane == 0) ok = ptx::wait_bounded_cluster(part_bar, 0u, p.timeout_ns, abort_flag, ERR_EPI + 3) ? 1 : 0;
+        if (__shfl_sync(0xffffffffu, ok, 0) == 0) return false;
+#pragma unroll 1
+        for (int c = 0; c < BN / CW; ++c) {
+            uint32_t v[32];
+            tmem_load_chunk(tbase + c * CW, v, CW);
+            ptx::tmem_ld_wait();
+            int32_t acc[CW];
+#pragma unroll
+            for (int i = 0; i < CW; ++i) acc[i] = static_cast<int32_t>(v[i]);
+#pragma unroll
+            for (int j = 1; j < CS; ++j) {
+#pragma unroll
+                for (int i = 0; i < CW; ++i) {
+                    if (c * CW + i < mval) {
+                        int32_t t;
+                        asm volatile("ld.shared.b32 %0, [%1];"
+                                     : "=r"(t)
+                                     : "r"(sbase + static_cast<uint32_t>((((j - 1) * BN + c * CW + i) * BM + r) * 4))
+                                     : "memory");
+                        acc[i] += t;
+                    }
+                }
+            }
+            if (!nok) continue;
+#pragma unroll
+            for (int i = 0; i < CW; ++i) {
+                if (c * CW + i < mval) {
+                    const int m = m0 + c * CW + i;
+                    const int64_t o = static_cast<int64_t>(m) * p.N + n;
+                    if constexpr (EPI == EPI_S32) {
+                        static_cast<int32_t *>(p.out)[o] = acc[i];
+                    } else {
+                        store_out(p.out, p.out_dt, o, dequant(acc[i], __fmul_rn(s_am[m - m0], wsn), p.bias, bn));
+                    }
+                }
+            }
+        }
+        return true;
+    }
+    // rank > 0: wait until the leader's stages are free, then send the partial sums
+    int ok = 1;
+    if (lane == 0) ok = ptx::wait_bounded_cluster(go_bar, 0u, p.timeout_ns, abort_flag, ERR_EPI + 4) ? 1 : 0;
+    if (__shfl_sync(0xffffffffu, ok, 0) == 0) return false;
+    const uint32_t remote = ptx::map_to_rank(sbase, 0);
+#pragma unroll 1
+    for (int c = 0; c < BN / CW; ++c) {
+        uint32_t v[32];
+        tmem_load_chunk(tbase + c * CW, v, CW);
+        ptx::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < CW; ++i)
+            if (c * CW + i < mval)
+                ptx::st_dsmem_u32(remote + static_cast<uint32_t>(((((int)rank - 1) * BN + c * CW + i) * BM + r) * 4), v[i]);
+    }
+    ptx::fence_acq_rel_cluster();
+    ptx::named_bar_sync(1, 128);
+    if (q == 2 && lane == 0) ptx::mbar_arrive_cluster(ptx::map_to_rank(part_bar, 0));
+    return true;
+}
+
+template <int BN, int EPI, int KBO, int CS>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_gemm_swap(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x, const Params p)
 {
     using C = TileCfg<BN, KBO>;
+    static_assert(CS >= 1 && CS <= 4, "cluster split of 1..4 CTAs");
+    static_assert((CS - 1) * BN * BM * 4 <= C::STAGES * C::STAGE_BYTES, "partial sums must fit the leader's stages");
     constexpr int S = C::STAGES;
     constexpr uint32_t IDESC = ptx::idesc_i8(BN);
 
@@ -465,7 +555,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * S + b); };
     auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * S + 2 + b); };
     const uint32_t done_bar = bar0 + 8u * (2 * S + 4);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 5);
+    const uint32_t go_bar = bar0 + 8u * (2 * S + 5);      // cluster split: leader's stages free
+    const uint32_t part_bar = bar0 + 8u * (2 * S + 6);    // cluster split: partial sums arrived
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * S + 7);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     int *flag = reinterpret_cast<int *>(tmem_slot + 2);
     __shared__ float s_am[BN];
@@ -483,6 +575,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ptx::mbar_init(tempty_bar(b), 4);
         }
         ptx::mbar_init(done_bar, 1);
+        if constexpr (CS > 1) {
+            ptx::mbar_init(go_bar, 1);
+            ptx::mbar_init(part_bar, CS - 1);
+        }
         *abort_flag = 0;
         *flag = 0;
         ptx::fence_barrier_init();
@@ -497,6 +593,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     ptx::tc_fence_before();
     __syncthreads();
+    if constexpr (CS > 1) ptx::cluster_sync();   // every CTA's barriers exist before any remote arrive
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const uint64_t tmo = p.timeout_ns;
@@ -610,8 +707,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 return __shfl_sync(0xffffffffu, ok, 0) != 0;
             };
             const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * BN);
-            if (!epilogue_sk<BN, EPI>(p, tbase, tr, tc, sg.tile, q, lane, flag, abort_flag, wsn, bn, s_am, tfull_wait))
+            if constexpr (CS > 1) {
+                if (!epilogue_cs<BN, EPI, CS>(p, tbase, tr, tc, q, lane, ptx::cluster_ctarank(), wsn, bn, s_am,
+                                              tfull_wait, go_bar, part_bar, sbase, abort_flag))
+                    break;
+            } else if (!epilogue_sk<BN, EPI>(p, tbase, tr, tc, sg.tile, q, lane, flag, abort_flag, wsn, bn, s_am,
+                                             tfull_wait)) {
                 break;
+            }
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(tempty_bar(b));

@@ -297,6 +297,48 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar)
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
 }
 
+// try_wait with cluster-scope acquire: writes that CTAs of the cluster made
+// before their release-arrive on this barrier are visible afterwards.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// wait_bounded for barriers that CTAs of the cluster arrive on remotely.
+__device__ __forceinline__ bool wait_bounded_cluster(uint32_t bar, uint32_t parity, uint64_t timeout_ns,
+                                                     volatile int *abort, unsigned code)
+{
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+#pragma unroll 1
+        for (int i = 0; i < 16; ++i)
+            if (mbar_try_wait_cluster(bar, parity)) return true;
+        if (*abort) return false;
+        if (global_timer_ns() - t0 > timeout_ns) {
+            *abort = 1;
+            atomicCAS(&g_error_word, 0u, code);
+            return false;
+        }
+    }
+}
+
+// 32-bit store to shared memory of a CTA of this cluster (address from mapa).
+__device__ __forceinline__ void st_dsmem_u32(uint32_t addr, uint32_t v)
+{
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void fence_acq_rel_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
+
 // TMA tile load into this CTA's shared memory whose completion is counted on
 // an mbarrier of either CTA of the pair (here: the leader's).
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void *map, uint32_t cluster_bar, int x, int y)
