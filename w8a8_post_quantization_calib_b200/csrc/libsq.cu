@@ -782,17 +782,19 @@ sq_status sq_smooth_quant_act(const void *x, sq_dtype dt, int64_t M, int64_t K, 
             const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), block(QS_TX, QS_TY);
             const uint8_t *xb = static_cast<const uint8_t *>(x);
             const bool big = M * K * elt > (int64_t(100) << 20);
+            const bool one = slab <= QS_UNROLL * QS_TY;
             const cudaStream_t st = as_stream(stream);
+            auto go = [&](auto kern) { return launch_pdl(kern, grid, block, 0, st, xb, M, nvec, s, a_scale, slab, xq); };
             cudaError_t e;
             if (dt == SQ_F32)
-                e = big ? launch_pdl(k_quant_static<DT_F32, true>, grid, block, 0, st, xb, M, nvec, s, a_scale, slab, xq)
-                        : launch_pdl(k_quant_static<DT_F32, false>, grid, block, 0, st, xb, M, nvec, s, a_scale, slab, xq);
+                e = big ? go(k_quant_static<DT_F32, true, false>)
+                        : one ? go(k_quant_static<DT_F32, false, true>) : go(k_quant_static<DT_F32, false, false>);
             else if (dt == SQ_F16)
-                e = big ? launch_pdl(k_quant_static<DT_F16, true>, grid, block, 0, st, xb, M, nvec, s, a_scale, slab, xq)
-                        : launch_pdl(k_quant_static<DT_F16, false>, grid, block, 0, st, xb, M, nvec, s, a_scale, slab, xq);
+                e = big ? go(k_quant_static<DT_F16, true, false>)
+                        : one ? go(k_quant_static<DT_F16, false, true>) : go(k_quant_static<DT_F16, false, false>);
             else
-                e = big ? launch_pdl(k_quant_static<DT_BF16, true>, grid, block, 0, st, xb, M, nvec, s, a_scale, slab, xq)
-                        : launch_pdl(k_quant_static<DT_BF16, false>, grid, block, 0, st, xb, M, nvec, s, a_scale, slab, xq);
+                e = big ? go(k_quant_static<DT_BF16, true, false>)
+                        : one ? go(k_quant_static<DT_BF16, false, true>) : go(k_quant_static<DT_BF16, false, false>);
             if (e != cudaSuccess) return cuda_fail(e);
             return check_launch();
         }

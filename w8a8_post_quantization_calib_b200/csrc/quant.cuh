@@ -444,7 +444,10 @@ __global__ void __launch_bounds__(NT) k_rows(RowArgs p)
 // 256 contiguous bytes.
 constexpr int QS_TX = 32, QS_TY = 8, QS_UNROLL = 4;
 
-template <int DT, bool STREAM>
+// ONE: every slab is at most one batch (QS_UNROLL x QS_TY rows), so no
+// second batch buffer is kept (fewer registers, more blocks resident: small
+// tensors are latency-bound).
+template <int DT, bool STREAM, bool ONE>
 __global__ void __launch_bounds__(QS_TX *QS_TY)
     k_quant_static(const uint8_t *__restrict__ x, int64_t rows, int64_t nvec, const float *__restrict__ s,
                    const float *__restrict__ a_in, int64_t row_slab, int8_t *__restrict__ out)
@@ -499,20 +502,26 @@ __global__ void __launch_bounds__(QS_TX *QS_TY)
                    pack4_bits(quant8_bits(f[0]), quant8_bits(f[1]), quant8_bits(f[2]), quant8_bits(f[3])));
         }
     };
-    // the next batch of rows is requested before this one is converted
-    for (;;) {
-        const int64_t rn = r + QS_UNROLL * QS_TY;
-        uint4 n[QS_UNROLL];
-#pragma unroll
-        for (int u = 0; u < QS_UNROLL; ++u)
-            if (rn + u * QS_TY < r1) n[u] = load(rn + u * QS_TY);
+    if constexpr (ONE) {
 #pragma unroll
         for (int u = 0; u < QS_UNROLL; ++u)
             if (r + u * QS_TY < r1) emit(r + u * QS_TY, t[u]);
-        if (rn >= r1) break;
+    } else {
+        // the next batch of rows is requested before this one is converted
+        for (;;) {
+            const int64_t rn = r + QS_UNROLL * QS_TY;
+            uint4 n[QS_UNROLL];
 #pragma unroll
-        for (int u = 0; u < QS_UNROLL; ++u) t[u] = n[u];
-        r = rn;
+            for (int u = 0; u < QS_UNROLL; ++u)
+                if (rn + u * QS_TY < r1) n[u] = load(rn + u * QS_TY);
+#pragma unroll
+            for (int u = 0; u < QS_UNROLL; ++u)
+                if (r + u * QS_TY < r1) emit(r + u * QS_TY, t[u]);
+            if (rn >= r1) break;
+#pragma unroll
+            for (int u = 0; u < QS_UNROLL; ++u) t[u] = n[u];
+            r = rn;
+        }
     }
 }
 
