@@ -489,8 +489,9 @@ sq_status launch_rows_dt(RowArgs a, cudaStream_t st)
     // 128 threads per row for rows of up to 512 vectors, else 256
     const int nt = nvec <= 4 * 128 ? 128 : ROW_T;
     const int64_t vpt = cdiv(nvec, nt);
-    // per-column constants in registers when VPT * EPV <= 32, else in shared memory
-    const size_t smem = (vpt * EPV <= 32) ? 0 : static_cast<size_t>(a.K) * 4;
+    // per-column constants in registers when VPT * EPV <= 32, else in shared
+    // memory; the norm-output statistic stages its column maxima there
+    const size_t smem = (vpt * EPV <= 32 && MODE != ROW_RMS_STAT) ? 0 : static_cast<size_t>(a.K) * 4;
     const int sms = sm_count();
     // Fewer rows than SMs: the row kernel would run one latency-bound row per
     // block on a few SMs; a cluster of CTAs per row (one vector per thread)
@@ -545,8 +546,15 @@ sq_status launch_rows_dt(RowArgs a, cudaStream_t st)
                 kinfo(reinterpret_cast<const void *>(kern)).per_sm = per_sm;
             }
         }
-        const int64_t grid = std::min<int64_t>(a.rows, static_cast<int64_t>(sms) * std::max(1, per_sm));
-        e = launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(nt), smem, st, a);
+        int64_t grid = std::min<int64_t>(a.rows, static_cast<int64_t>(sms) * std::max(1, per_sm));
+        if (MODE == ROW_RMS_STAT && a.rows <= 8 * grid) {
+            // few rows per block: the per-block column atomics dominate, so the
+            // blocks of a cluster combine their maxima first
+            grid = cdiv(grid, RMS_CL) * RMS_CL;       // whole clusters (blocks past the rows idle)
+            e = launch_pdl_cluster_smem(kern, dim3(static_cast<unsigned>(grid)), dim3(nt), RMS_CL, smem, st, a);
+        } else {
+            e = launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(nt), smem, st, a);
+        }
         if (e != cudaSuccess) return cuda_fail(e);
     } else {
         const int64_t grid = std::min<int64_t>(a.rows, static_cast<int64_t>(sms) * 8);

@@ -110,6 +110,7 @@ enum RowMode : int {
 };
 
 constexpr int ROW_T = 256;
+constexpr int RMS_CL = 8;          // cluster of the norm-output statistic (see k_rows)
 
 struct RowArgs {
     const uint8_t *src0;     // input rows (row r at src0 + r*row_bytes)
@@ -423,15 +424,38 @@ __global__ void __launch_bounds__(NT) k_rows(RowArgs p)
         }
     }
     if constexpr (MODE == ROW_RMS_STAT) {
+        // Launched in clusters (few rows per block, where the atomics would
+        // dominate), the blocks of a cluster first combine their column maxima
+        // through distributed shared memory: CTA r takes every n-th slice of
+        // the columns and issues the atomics for it, n times fewer atomics on
+        // the same addresses than one per column per block.
+        float *cm = reinterpret_cast<float *>(colv4);    // [K] (dynamic shared memory)
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
             const int64_t v = static_cast<int64_t>(i) * NT + tid;
             if (v < nvec) {
 #pragma unroll
-                for (int e = 0; e < EPV; ++e)
-                    atomicMax(reinterpret_cast<int *>(p.scale_out + v * EPV + e), __float_as_int(cmax[i][e]));
+                for (int e = 0; e < EPV; ++e) cm[v * EPV + e] = cmax[i][e];
             }
         }
+        ptx::cluster_sync();                            // every block's maxima written
+        const uint32_t rank = ptx::cluster_ctarank();
+        const int ncl = static_cast<int>(ptx::cluster_nctarank());   // 1 when launched without a cluster
+        const uint32_t local = ptx::smem_addr(cm);
+        for (int64_t j = static_cast<int64_t>(rank) * NT + tid; j < p.K; j += static_cast<int64_t>(ncl) * NT) {
+            float m = 0.0f;
+#pragma unroll 1
+            for (int c = 0; c < ncl; ++c) {
+                float o;
+                asm volatile("ld.shared::cluster.f32 %0, [%1];"
+                             : "=f"(o)
+                             : "r"(ptx::map_to_rank(local + static_cast<uint32_t>(j) * 4u, static_cast<uint32_t>(c)))
+                             : "memory");
+                m = fmaxf(m, o);
+            }
+            atomicMax(reinterpret_cast<int *>(p.scale_out + j), __float_as_int(m));
+        }
+        ptx::cluster_sync();                            // no block leaves while its maxima are read
     }
 }
 
