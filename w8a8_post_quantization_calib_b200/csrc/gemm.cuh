@@ -79,7 +79,6 @@ struct Params {
     int rows_a, rows_b;        // rows of the A / B operand tensors
     int num_kb;                // K blocks of 128 bytes
     int tiles_r, tiles_c;      // tiles along A rows (BM) and B rows (BN)
-    int splits, kb_per_split;  // CTA-pair path: always 1 / num_kb
     int num_units;             // CTA-pair path: tiles_r * tiles_c
     int sk_iters, sk_ctas;     // swap path: tiles * num_kb iterations shared by sk_ctas CTAs
     int sk_slot;               // swap path: int32 per partial-sum slot (BM * BN)
@@ -99,10 +98,11 @@ struct Params {
     int inject;                // failure-detection test: 1 = CTA 0 withholds its first stage
 };
 
-__device__ __forceinline__ void decode_unit(const Params &p, int u, int &tr, int &tc, int &split, int &tile)
+// Tile u of the CTA-pair grid in raster-group order (GROUP_R A-row tiles per
+// group, so that consecutive tiles share B tiles in L2).
+__device__ __forceinline__ void decode_unit(const Params &p, int u, int &tr, int &tc)
 {
-    split = u % p.splits;
-    tile = u / p.splits;
+    const int tile = u;
     const int group = tile / (GROUP_R * p.tiles_c);
     const int first = group * GROUP_R;
     const int gsz = min(GROUP_R, p.tiles_r - first);
@@ -171,106 +171,87 @@ __device__ __forceinline__ float dequant(int32_t acc, float c, const void *bias,
 }
 
 // ---------------------------------------------------------------------------
-// Epilogue of one tile, normal orientation (TMEM lane = token row m).
+// Gate/up epilogue of one 128-row accumulator (TMEM lane = token row m): the
+// columns come as 32 gate channels, then the same 32 channels' up rows,
+// repeated.  ws_tile holds the tile's BN w_scale values and s2inv_tile the
+// BN/2 channels' fl(1/s2), staged in shared memory while the tile's MMAs ran.
+// SiLU uses the fast exponential and division (h is rounded to bf16
+// afterwards: a few fp32 ulp are far below its precision).  h leaves through
+// the same swizzled staging + TMA store as epilogue_tma (a warp's 32 rows x
+// 32 channels of bf16 per box, rows >= M clipped by the tensor map); the
+// requantised codes go straight to global memory (one 32-byte sector per
+// row and chunk).
 // ---------------------------------------------------------------------------
-// Gate/up (EPI_GATEUP): ws_tile holds the tile's BN w_scale values and
-// s2inv_tile the BN/2 channels' fl(1/s2), staged in shared memory while the
-// tile's MMAs ran.  SiLU uses the fast exponential and division (h is
-// rounded to bf16 afterwards: a few fp32 ulp are far below its precision).
-template <int BN, int KIND, int EPI>
-__device__ __forceinline__ void epilogue_normal(const Params &p, uint32_t tbase, int tr, int tc, int q,
-                                                int lane, const float *ws_tile = nullptr,
-                                                const float *s2inv_tile = nullptr)
+template <int BN, int NBUF>
+__device__ __forceinline__ void epilogue_gateup(const Params &p, const CUtensorMap *omap_h, uint32_t tbase, int tr,
+                                                int tc, int q, int lane, const float *ws_tile,
+                                                const float *s2inv_tile, uint32_t stg, int &nstore)
 {
     const int m = tr * BM + q * 32 + lane;
+    const int mrow0 = tr * BM + q * 32;
     const bool mok = m < p.M;
-    float am = 0.0f;
-    if constexpr (EPI == EPI_DEQUANT || EPI == EPI_GATEUP)
-        if (mok) am = p.per_token ? p.a_scale[m] : p.a_scale[0];
-
-    if constexpr (EPI == EPI_GATEUP) {
-        // columns: 32 gate channels, then the same 32 channels' up rows, repeated
-        const int Nh = p.N >> 1;
-        const float inv_a2 = p.hq != nullptr ? recip_or_zero(p.a2[0]) : 0.0f;
+    const float am = mok ? (p.per_token ? p.a_scale[m] : p.a_scale[0]) : 0.0f;
+    const int Nh = p.N >> 1;
+    const float inv_a2 = p.hq != nullptr ? recip_or_zero(p.a2[0]) : 0.0f;
 #pragma unroll 1
-        for (int c = 0; c < BN / 64; ++c) {
-            uint32_t rg[32], ru[32];
-            ptx::tmem_ld32(tbase + c * 64, rg);
-            ptx::tmem_ld32(tbase + c * 64 + 32, ru);
-            ptx::tmem_ld_wait();
-            const int row0 = tc * BN + c * 64;         // first gate row of this pair of chunks
-            if (row0 >= p.N) continue;
-            const int ch0 = row0 >> 1;
-            float h[32];
+    for (int c = 0; c < BN / 64; ++c) {
+        uint32_t rg[32], ru[32];
+        ptx::tmem_ld32(tbase + c * 64, rg);
+        ptx::tmem_ld32(tbase + c * 64 + 32, ru);
+        ptx::tmem_ld_wait();
+        const int row0 = tc * BN + c * 64;             // first gate row of this pair of chunks
+        if (row0 >= p.N) continue;
+        const int ch0 = row0 >> 1;
+        float h[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const float g = __fmul_rn(__int2float_rn(static_cast<int32_t>(rg[i])), __fmul_rn(am, ws_tile[c * 64 + i]));
-                const float u = __fmul_rn(__int2float_rn(static_cast<int32_t>(ru[i])), __fmul_rn(am, ws_tile[c * 64 + 32 + i]));
-                const float sg = __fdividef(g, __fadd_rn(1.0f, __expf(-g)));
-                h[i] = __bfloat162float(__float2bfloat16_rn(__fmul_rn(sg, u)));   // h as bf16
-            }
-            if (!mok) continue;
-            const int64_t o = static_cast<int64_t>(m) * Nh + ch0;
-            if (p.out != nullptr) {
-#pragma unroll
-                for (int i = 0; i < 32; i += 8) store_out8(p.out, DT_BF16, o + i, h + i);
-            }
-            if (p.hq != nullptr) {
-                uint32_t w[8];
-#pragma unroll
-                for (int i = 0; i < 32; i += 4) {
-                    int qv[4];
-#pragma unroll
-                    for (int t = 0; t < 4; ++t)
-                        qv[t] = quant8(__fmul_rn(__fmul_rn(h[i + t], s2inv_tile[c * 32 + i + t]), inv_a2));
-                    w[i / 4] = pack4(qv[0], qv[1], qv[2], qv[3]);
-                }
-                uint4 *dst = reinterpret_cast<uint4 *>(p.hq + o);
-                dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-            }
+        for (int i = 0; i < 32; ++i) {
+            const float g = __fmul_rn(__int2float_rn(static_cast<int32_t>(rg[i])), __fmul_rn(am, ws_tile[c * 64 + i]));
+            const float u = __fmul_rn(__int2float_rn(static_cast<int32_t>(ru[i])), __fmul_rn(am, ws_tile[c * 64 + 32 + i]));
+            const float sg = __fdividef(g, __fadd_rn(1.0f, __expf(-g)));
+            h[i] = __bfloat162float(__float2bfloat16_rn(__fmul_rn(sg, u)));   // h as bf16
         }
-    } else {
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-            uint32_t r[32];
-            ptx::tmem_ld32(tbase + c * 32, r);
-            ptx::tmem_ld_wait();
-            const int n0 = tc * BN + c * 32;
-            if (n0 >= p.N || !mok) continue;
-            const int nval = min(32, p.N - n0);        // 16 or 32 (N is a multiple of 16)
-            const int64_t o = static_cast<int64_t>(m) * p.N + n0;
-            if constexpr (EPI == EPI_S32) {
-                int4 *dst = reinterpret_cast<int4 *>(static_cast<int32_t *>(p.out) + o);
+        if (p.out != nullptr) {
+            uint32_t w[16];
 #pragma unroll
-                for (int i = 0; i < 32; i += 4)
-                    if (i < nval) dst[i / 4] = make_int4(r[i], r[i + 1], r[i + 2], r[i + 3]);
-            } else if constexpr (EPI == EPI_F16) {
-                float v[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-#pragma unroll
-                for (int i = 0; i < 32; i += 8)
-                    if (i < nval) store_out8(p.out, DT_F16, o + i, v + i);
-            } else {
-                float v[32];
-#pragma unroll
-                for (int i = 0; i < 32; i += 4) {
-                    if (i < nval) {
-                        const float4 w4 = *reinterpret_cast<const float4 *>(p.w_scale + n0 + i);
-                        const float ws[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-                        for (int t = 0; t < 4; ++t) {
-                            const float cc = __fmul_rn(am, ws[t]);
-                            v[i + t] = dequant(static_cast<int32_t>(r[i + t]), cc, p.bias,
-                                               load_bias(p.bias, p.out_dt, n0 + i + t));
-                        }
-                    }
-                }
-#pragma unroll
-                for (int i = 0; i < 32; i += 8)
-                    if (i < nval) store_out8(p.out, p.out_dt, o + i, v + i);
+            for (int i = 0; i < 16; ++i) {
+                __nv_bfloat162 b2 = __floats2bfloat162_rn(h[2 * i], h[2 * i + 1]);   // exact: h is bf16 already
+                w[i] = *reinterpret_cast<uint32_t *>(&b2);
             }
+            if constexpr (NBUF == 2) {
+                if (lane == 0 && nstore >= 2) ptx::bulk_wait_read_1();
+            } else {
+                if (lane == 0 && nstore >= 1) ptx::bulk_wait_read_0();
+            }
+            __syncwarp();
+            const uint32_t buf = stg + static_cast<uint32_t>(NBUF == 2 ? (nstore & 1) : 0) * STG_BYTES;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {          // 64-byte rows, 64-byte swizzle: chunk ^= (row >> 1) & 3
+                const uint32_t a = buf + lane * 64 + ((k ^ ((lane >> 1) & 3)) << 4);
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(w[4 * k]), "r"(w[4 * k + 1]),
+                             "r"(w[4 * k + 2]), "r"(w[4 * k + 3])
+                             : "memory");
+            }
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                ptx::tma_store_2d(omap_h, buf, ch0, mrow0);
+                ptx::bulk_commit();
+            }
+            ++nstore;
+        }
+        if (p.hq != nullptr && mok) {
+            uint32_t w[8];
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+                int qv[4];
+#pragma unroll
+                for (int t = 0; t < 4; ++t)
+                    qv[t] = quant8(__fmul_rn(__fmul_rn(h[i + t], s2inv_tile[c * 32 + i + t]), inv_a2));
+                w[i / 4] = pack4(qv[0], qv[1], qv[2], qv[3]);
+            }
+            uint4 *dst = reinterpret_cast<uint4 *>(p.hq + static_cast<int64_t>(m) * Nh + ch0);
+            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
         }
     }
 }
@@ -938,8 +919,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             int stage = 0, issued = 0;
             uint32_t phase = 0;
             for (int u = cluster; u < p.num_units && !*abort_flag; u += nclusters) {
-                int tr, tc, split, tile;
-                decode_unit(p, u, tr, tc, split, tile);
+                int tr, tc;
+                decode_unit(p, u, tr, tc);
                 bool ok = true;
                 for (int kb = 0; kb < p.num_kb; ++kb) {
                     if (!ptx::wait_bounded(empty_bar(stage), phase ^ 1u, tmo, abort_flag, ERR_PRODUCER)) {
@@ -1027,8 +1008,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         int nstore = 0;
         int local = 0;
         for (int u = cluster; u < p.num_units; u += nclusters, ++local) {
-            int tr, tc, split, tile;
-            decode_unit(p, u, tr, tc, split, tile);
+            int tr, tc;
+            decode_unit(p, u, tr, tc);
             const int b = local & 1;
             const uint32_t use = static_cast<uint32_t>(local >> 1) & 1u;
             // while the MMAs of this tile run: stage its per-column scales / bias
@@ -1068,8 +1049,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * BN);
             // this CTA's accumulator rows are the tile's rows rank*128 .. rank*128+127
             if constexpr (EPI == EPI_GATEUP)
-                epilogue_normal<BN, KIND, EPI>(p, tbase, 2 * tr + static_cast<int>(rank), tc, q, lane, ws_tile,
-                                               bias_tile);
+                epilogue_gateup<BN, C::STG_BUFS>(p, &map_o, tbase, 2 * tr + static_cast<int>(rank), tc, q, lane,
+                                                 ws_tile, bias_tile, stg, nstore);
             else
                 epilogue_tma<BN, KIND, EPI, C::STG_BUFS>(p, &map_o, tbase, 2 * tr + static_cast<int>(rank), tc, q, lane, stg,
                                             nstore, ws_tile, bias_tile, am);

@@ -267,7 +267,9 @@ sq_status launch_gemm2(gemm::Params p, const void *a, const void *b, cudaStream_
         if (!make_map3(&mb, b, p.K, p.rows_b, BN / 2, KBO)) return SQ_ERR_CUDA;
     }
     if constexpr (EPI == gemm::EPI_GATEUP) {
+        // h [M, N/2] bf16, written with TMA stores when requested
         std::memset(&mo, 0, sizeof(mo));
+        if (p.out != nullptr && !make_out_map(&mo, p.out, SQ_BF16, false, p.M, p.N / 2)) return SQ_ERR_CUDA;
     } else {
         const int odt = (EPI == gemm::EPI_F16) ? SQ_F16 : p.out_dt;
         if (!make_out_map(&mo, p.out, odt, EPI == gemm::EPI_S32, p.M, p.N)) return SQ_ERR_CUDA;
@@ -307,8 +309,6 @@ void fill_tiles_pair(gemm::Params &p, int bn, int kb_bytes_per_elem)
     p.num_kb = static_cast<int>(cdiv(static_cast<int64_t>(p.K) * kb_bytes_per_elem, 128));
     p.tiles_r = static_cast<int>(cdiv(p.M, 2 * gemm::BM));
     p.tiles_c = static_cast<int>(cdiv(p.N, bn));
-    p.splits = 1;
-    p.kb_per_split = p.num_kb;
     p.num_units = p.tiles_r * p.tiles_c;
 }
 
@@ -368,8 +368,6 @@ void fill_tiles(gemm::Params &p, int bn, int64_t rows_a, int64_t rows_b)
     p.num_kb = static_cast<int>(cdiv(p.K, 128 / 1));
     p.tiles_r = static_cast<int>(cdiv(rows_a, gemm::BM));
     p.tiles_c = static_cast<int>(cdiv(rows_b, bn));
-    p.splits = 1;
-    p.kb_per_split = p.num_kb;
     p.num_units = p.tiles_r * p.tiles_c;
 }
 
@@ -581,8 +579,9 @@ sq_status launch_rows(RowArgs a, int dt, cudaStream_t st)
 // cudaMalloc at all: a plugin inside a host engine that owns every device
 // buffer and hands the plugin only its inputs and outputs, or a serving loop
 // that must never pay cudaMalloc's implicit device-wide synchronisation.  For
-// them the small-M split-K path keeps its int32 partial sums and per-tile
-// arrival counters in this file-scope array instead of a caller workspace.
+// them the small-M stream-K schedule (used when the cluster split is off)
+// keeps its int32 partial sums and per-tile arrival counters in this
+// file-scope array instead of a caller workspace.
 // Every GPU that loads the library holds it (8 MiB + 64 KiB) until exit.
 // ---------------------------------------------------------------------------
 constexpr size_t kNoAllocAccBytes = size_t(8) << 20;            // int32 partial sums
