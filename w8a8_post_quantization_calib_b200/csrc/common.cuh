@@ -170,4 +170,22 @@ __device__ __forceinline__ double block_sum_f64(double v, double *red)
     return r;
 }
 
+// block_sum_f64 for a compile-time warp count NW (a power of two): the
+// second level reduces only the NW warp sums, giving the same sum as
+// block_sum_f64 (whose lanes past NW add zeros).
+template <int NW>
+__device__ __forceinline__ double block_sum_f64_nw(double v, double *red)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    __syncthreads();
+    if (l == 0) red[w] = v;
+    __syncthreads();
+    double r = red[l & (NW - 1)];
+#pragma unroll
+    for (int o = NW / 2; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
+    return r;
+}
+
 }  // namespace sq

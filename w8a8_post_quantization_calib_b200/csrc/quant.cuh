@@ -303,6 +303,8 @@ __global__ void __launch_bounds__(NT) k_rows(RowArgs p)
     };
     float inv_a_static = 0.0f;
     if constexpr (MODE == ROW_ACT_STATIC || MODE == ROW_RMSNORM) inv_a_static = recip_or_zero(p.a_in[0]);
+    const bool k_pow2 = (p.K & (p.K - 1)) == 0;
+    const double k_recip = 1.0 / static_cast<double>(p.K);
     float cmax[MODE == ROW_RMS_STAT ? VPT : 1][MODE == ROW_RMS_STAT ? EPV : 1];
     if constexpr (MODE == ROW_RMS_STAT) {
         static_assert(REG, "the norm-output statistic keeps its column maxima in registers");
@@ -340,20 +342,25 @@ __global__ void __launch_bounds__(NT) k_rows(RowArgs p)
         if constexpr (MODE == ROW_RMSNORM || MODE == ROW_RMS_STAT) {
             // pass 1: sum of squares in fp64 (exact squares); REG keeps the
             // widened row for pass 2
+            // (four independent partial sums: the row's latency rather than
+            // the issue rate bounds this kernel, and a single chain of
+            // dependent fp64 adds per thread was a large part of it)
             float fk[REG ? VPT : 1][REG ? EPV : 1];
-            double ss = 0.0;
+            double ss4[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll
             for (int i = 0; i < VPT; ++i) {
                 float f[EPV];
                 widen<DT>(raw[i], f);
 #pragma unroll
                 for (int e = 0; e < EPV; ++e) {
-                    ss += static_cast<double>(f[e]) * static_cast<double>(f[e]);
+                    ss4[e & 3] += static_cast<double>(f[e]) * static_cast<double>(f[e]);
                     if constexpr (REG) fk[i][e] = f[e];
                 }
             }
-            const double tot = block_sum_f64(ss, red64);
-            const float mean = __double2float_rn(tot / static_cast<double>(p.K));
+            const double tot = block_sum_f64_nw<NT / 32>((ss4[0] + ss4[1]) + (ss4[2] + ss4[3]), red64);
+            // a power-of-two K divides exactly by its reciprocal (the same result as the division)
+            const double mean64 = k_pow2 ? tot * k_recip : tot / static_cast<double>(p.K);
+            const float mean = __double2float_rn(mean64);
             const float r_m = __frcp_rn(__fsqrt_rn(__fadd_rn(mean, p.eps)));
             if (tid == 0 && p.rstd_out != nullptr) p.rstd_out[row] = r_m;
 #pragma unroll
