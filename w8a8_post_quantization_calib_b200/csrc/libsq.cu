@@ -116,7 +116,8 @@ cudaError_t launch_pdl_cluster(void (*kern)(KArgs...), dim3 grid, dim3 block, un
 // occupancy figures the launch sizes its grid with.  Queried once.
 struct KernelInfo {
     int smem_set = 0;
-    int per_sm = 0;
+    int per_sm = 0;           // resident blocks per SM with per_sm_smem bytes of dynamic shared memory
+    int per_sm_smem = -1;
     int clusters = 0;
 };
 std::unordered_map<uint64_t, KernelInfo> g_kinfo;
@@ -489,8 +490,20 @@ sq_status launch_rows_dt(RowArgs a, cudaStream_t st)
     const int64_t vpt = cdiv(nvec, nt);
     // per-column constants in registers when VPT * EPV <= 32, else in shared
     // memory; the norm-output statistic stages its column maxima there
-    const size_t smem = (vpt * EPV <= 32 && MODE != ROW_RMS_STAT) ? 0 : static_cast<size_t>(a.K) * 4;
+    const bool reg_rows = vpt * EPV <= 32;
+    size_t smem = (reg_rows && MODE != ROW_RMS_STAT) ? 0 : static_cast<size_t>(a.K) * 4;
     const int sms = sm_count();
+    // Rows held in registers arrive through the shared-memory row ring where
+    // that measured faster (256 MiB inputs, 256-thread rows of 8192 16-bit
+    // elements: per-token 0.82 -> 0.88 of HBM, weight transform 0.86 -> 0.95;
+    // norm-output statistic 0.41 -> 0.56, and 0.56 -> 0.58 at 4096).  It was
+    // slower for the 128-thread rows of the weight transform and for RMSNorm
+    // + quant at both lengths, and for the statistic of a 2048-token batch.
+    constexpr bool kRingMode = MODE == ROW_WEIGHT || MODE == ROW_ACT_TOKEN || MODE == ROW_RMS_STAT;
+    const bool ring = kRingMode && reg_rows &&
+                      (MODE == ROW_RMS_STAT ? a.rows >= 64 * static_cast<int64_t>(sms) : nt == ROW_T);
+    if (ring) smem = ((smem + 127) & ~size_t(127)) + static_cast<size_t>(RING_ROWS) * a.row_bytes;
+    a.timeout_ns = g_timeout_ns;
     // Fewer rows than SMs: the row kernel would run one latency-bound row per
     // block on a few SMs; a cluster of CTAs per row (one vector per thread)
     // spreads each row instead.  The cluster size is the smallest power of
@@ -509,7 +522,27 @@ sq_status launch_rows_dt(RowArgs a, cudaStream_t st)
     }
     if (vec && vpt <= 16 && smem <= 160 * 1024) {
         void (*kern)(RowArgs) = nullptr;
-        if (nt == 128) {
+        if constexpr (kRingMode) {
+            if (ring) {
+                if (nt == 128) {
+                    if constexpr (MODE == ROW_RMS_STAT) {
+                        if (vpt <= 1) kern = k_rows<DT, 1, MODE, 128, true>;
+                        else if (vpt <= 2) kern = k_rows<DT, 2, MODE, 128, true>;
+                        else kern = k_rows<DT, 4, MODE, 128, true>;
+                    }
+                } else if (vpt <= 1) {
+                    kern = k_rows<DT, 1, MODE, ROW_T, true>;
+                } else if (vpt <= 2) {
+                    kern = k_rows<DT, 2, MODE, ROW_T, true>;
+                } else if (vpt <= 4) {
+                    kern = k_rows<DT, 4, MODE, ROW_T, true>;
+                } else {
+                    kern = k_rows<DT, (DT == DT_F32 ? 8 : 4), MODE, ROW_T, true>;
+                }
+            }
+        }
+        if (kern != nullptr) {
+        } else if (nt == 128) {
             if (vpt <= 1) kern = k_rows<DT, 1, MODE, 128>;
             else if (vpt <= 2) kern = k_rows<DT, 2, MODE, 128>;
             else kern = k_rows<DT, 4, MODE, 128>;
@@ -527,22 +560,23 @@ sq_status launch_rows_dt(RowArgs a, cudaStream_t st)
             kern = k_rows<DT, 16, MODE, ROW_T>;
         }
         cudaError_t e = cudaSuccess;
-        if (smem > 48 * 1024) {
+        if (smem > 0) {       // with the kernel's static shared memory it may pass the 48 KB default
             e = ensure_smem(reinterpret_cast<const void *>(kern), static_cast<int>(smem));
             if (e != cudaSuccess) return cuda_fail(e);
         }
         int per_sm = 0;
-        if (smem == 0) {      // occupancy does not depend on K: query once per kernel
+        {   // occupancy per kernel and shared-memory size, queried once
             std::lock_guard<std::mutex> lk(g_mu);
-            per_sm = kinfo(reinterpret_cast<const void *>(kern)).per_sm;
+            const KernelInfo &ki = kinfo(reinterpret_cast<const void *>(kern));
+            if (ki.per_sm_smem == static_cast<int>(smem)) per_sm = ki.per_sm;
         }
         if (per_sm == 0) {
             e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, nt, smem);
             if (e != cudaSuccess) return cuda_fail(e);
-            if (smem == 0) {
-                std::lock_guard<std::mutex> lk(g_mu);
-                kinfo(reinterpret_cast<const void *>(kern)).per_sm = per_sm;
-            }
+            std::lock_guard<std::mutex> lk(g_mu);
+            KernelInfo &ki = kinfo(reinterpret_cast<const void *>(kern));
+            ki.per_sm = per_sm;
+            ki.per_sm_smem = static_cast<int>(smem);
         }
         int64_t grid = std::min<int64_t>(a.rows, static_cast<int64_t>(sms) * std::max(1, per_sm));
         if (MODE == ROW_RMS_STAT && a.rows <= 8 * grid) {

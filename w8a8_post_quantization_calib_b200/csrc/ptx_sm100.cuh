@@ -138,6 +138,16 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *map, uint3
         : "memory");
 }
 
+// Untiled bulk copy global -> this CTA's shared memory of `bytes` (a multiple
+// of 16; both addresses 16-byte aligned), completion reported as transaction
+// bytes on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
 // 2D tiled bulk-tensor store shared -> global (out-of-range parts of the box
 // are not written).  x (inner, elements) * element size is a multiple of 16 B.
 __device__ __forceinline__ void tma_store_2d(const void *map, uint32_t src, int x, int y)

@@ -125,7 +125,13 @@ struct RowArgs {
     float *scale_out;        // per-row scales [rows] (weight, per-token)
     float *rstd_out;         // RMSNorm r_m [rows] or null
     int8_t *out;             // codes [rows, K]
+    unsigned long long timeout_ns;   // bound of the row-ring waits
 };
+
+// Rows in flight per block in the shared-memory row ring of k_rows, and the
+// error code a timed-out ring wait records.
+constexpr int RING_ROWS = 3;
+constexpr unsigned ERR_ROW_RING = 0x150;
 
 // Codes of EPV values (already multiplied by the scale reciprocal) -> global.
 // INRANGE: the values come from a per-row scale and cannot saturate.
@@ -185,18 +191,43 @@ __device__ __forceinline__ bool constants_aligned16(const RowArgs &p)
 // their stores are predicated (no divergent branches), and NT = 128 threads
 // per row for rows of up to 4096 16-bit elements halves the per-row cost of
 // the block reductions.
-template <int DT, int VPT, int MODE, int NT>
+//
+// RING (rows held in registers, modes with a per-row block reduction): the
+// rows come through a ring of RING_ROWS row buffers in shared memory filled
+// by bulk copies (one per row, issued by thread 0 on an mbarrier), so that
+// RING_ROWS rows per block are in flight from HBM whatever the registers
+// allow.  A buffer is refilled once every thread has moved its row into
+// registers, which the row's block reduction barrier guarantees.  The waits
+// are bounded: on expiry the kernel records the error and finishes on
+// whatever data it has (no thread leaves early, so no barrier is left short).
+template <int DT, int VPT, int MODE, int NT, bool RING = false>
 __global__ void __launch_bounds__(NT) k_rows(RowArgs p)
 {
     constexpr int EPV = VecT<DT>::EPV;
     constexpr bool REG = (VPT * EPV <= 32);
-    extern __shared__ float4 colv4[];
+    static_assert(!RING || (REG && MODE != ROW_ACT_STATIC), "the row ring needs register rows and a row barrier");
+    extern __shared__ __align__(128) float4 colv4[];
     __shared__ float red[32];
     __shared__ double red64[32];
+    __shared__ __align__(8) uint64_t ring_full[RING ? RING_ROWS : 1];
+    __shared__ int ring_abort;
 
     const int tid = threadIdx.x;
     const int64_t nvec = p.K / EPV;
     const int64_t plane = nvec;            // float4 entries per plane
+    // ring buffers after the statistic's column maxima (the other modes keep
+    // no per-column table in shared memory when the row is in registers)
+    uint8_t *ring = reinterpret_cast<uint8_t *>(colv4) +
+                    (MODE == ROW_RMS_STAT ? ((static_cast<size_t>(p.K) * 4 + 127) & ~size_t(127)) : 0);
+    const uint32_t row_bytes32 = static_cast<uint32_t>(p.row_bytes);
+    if constexpr (RING) {
+        if (tid == 0) {
+            for (int s = 0; s < RING_ROWS; ++s) ptx::mbar_init(ptx::smem_addr(&ring_full[s]), 1);
+            ring_abort = 0;
+            ptx::fence_barrier_init();
+        }
+        __syncthreads();
+    }
     pdl_wait();
     pdl_launch_dependents();
 
@@ -215,13 +246,40 @@ __global__ void __launch_bounds__(NT) k_rows(RowArgs p)
             dst[i] = (v < nvec) ? __ldcs(src + v) : make_uint4(0u, 0u, 0u, 0u);
         }
     };
-    // Rows of up to 8 vectors per thread keep the next row's loads in flight
-    // while a row is processed; the first row is requested before the
-    // per-column constants, so that the two loads overlap.
-    constexpr bool PF = VPT <= 8;
+    // local row i of this block -> ring buffer i % RING_ROWS
+    auto ring_issue = [&](int64_t i) {
+        const int64_t row = blockIdx.x + i * gridDim.x;
+        if (row < p.rows) {
+            const int sl = static_cast<int>(i % RING_ROWS);
+            const uint32_t bar = ptx::smem_addr(&ring_full[sl]);
+            ptx::mbar_arrive_expect_tx(bar, row_bytes32);
+            ptx::bulk_load(ptx::smem_addr(ring) + static_cast<uint32_t>(sl) * row_bytes32, row_src(row), row_bytes32,
+                           bar);
+        }
+    };
+    auto ring_take = [&](int64_t i, uint4 (&dst)[VPT]) {
+        const int sl = static_cast<int>(i % RING_ROWS);
+        const uint32_t par = static_cast<uint32_t>((i / RING_ROWS) & 1);
+        ptx::wait_bounded(ptx::smem_addr(&ring_full[sl]), par, p.timeout_ns, &ring_abort, ERR_ROW_RING);
+        const uint4 *src = reinterpret_cast<const uint4 *>(ring + static_cast<size_t>(sl) * p.row_bytes);
+#pragma unroll
+        for (int k = 0; k < VPT; ++k) {
+            const int64_t v = static_cast<int64_t>(k) * NT + tid;
+            dst[k] = (v < nvec) ? src[v] : make_uint4(0u, 0u, 0u, 0u);
+        }
+    };
+    // Without the ring, rows of up to 8 vectors per thread keep the next
+    // row's loads in flight while a row is processed; the first row is
+    // requested before the per-column constants, so that the two loads
+    // overlap.
+    constexpr bool PF = !RING && VPT <= 8;
     uint4 nxt[PF ? VPT : 1];
     if constexpr (PF) {
         if (blockIdx.x < p.rows) load_row(blockIdx.x, nxt);
+    }
+    if constexpr (RING) {
+        if (tid == 0)
+            for (int i = 0; i < RING_ROWS; ++i) ring_issue(i);
     }
 
     const bool c16 = constants_aligned16(p);
@@ -314,15 +372,28 @@ __global__ void __launch_bounds__(NT) k_rows(RowArgs p)
             for (int e = 0; e < EPV; ++e) cmax[i][e] = 0.0f;
     }
 
-    for (int64_t row = blockIdx.x; row < p.rows; row += gridDim.x) {
+    int64_t li = 0;                        // local row index (ring position)
+    for (int64_t row = blockIdx.x; row < p.rows; row += gridDim.x, ++li) {
         uint4 raw[VPT];
-        if constexpr (PF) {
+        if constexpr (RING) {
+            ring_take(li, raw);
+        } else if constexpr (PF) {
 #pragma unroll
             for (int i = 0; i < VPT; ++i) raw[i] = nxt[i];
             if (row + gridDim.x < p.rows) load_row(row + gridDim.x, nxt);
         } else {
             load_row(row, raw);
         }
+        // after the row's block barrier every thread holds its part of the
+        // row in registers: refill the buffer with the row RING_ROWS ahead
+        auto ring_refill = [&]() {
+            if constexpr (RING) {
+                if (tid == 0) {
+                    ptx::fence_proxy_async_smem();
+                    ring_issue(li + RING_ROWS);
+                }
+            }
+        };
         int8_t *dst = p.out + row * p.K;
 
         if constexpr (MODE == ROW_ACT_STATIC) {
@@ -358,6 +429,7 @@ __global__ void __launch_bounds__(NT) k_rows(RowArgs p)
                 }
             }
             const double tot = block_sum_f64_nw<NT / 32>((ss4[0] + ss4[1]) + (ss4[2] + ss4[3]), red64);
+            ring_refill();
             // a power-of-two K divides exactly by its reciprocal (the same result as the division)
             const double mean64 = k_pow2 ? tot * k_recip : tot / static_cast<double>(p.K);
             const float mean = __double2float_rn(mean64);
@@ -406,6 +478,7 @@ __global__ void __launch_bounds__(NT) k_rows(RowArgs p)
             }
         }
         const float sc = scale_from_absmax(block_max(mx, red));
+        ring_refill();
         const float inv = recip_or_zero(sc);
         if (tid == 0) p.scale_out[row] = sc;
         // with a normal (or zero) scale the row's codes cannot saturate
@@ -428,6 +501,16 @@ __global__ void __launch_bounds__(NT) k_rows(RowArgs p)
                 if (inrange) store_codes<EPV, true>(dst, v, f);
                 else store_codes<EPV, false>(dst, v, f);
             }
+        }
+    }
+    if constexpr (RING) {
+        // after a timed-out wait, no block leaves while a bulk copy may still
+        // be writing its shared memory
+        if (tid == 0 && ring_abort) {
+            volatile int no_abort = 0;
+            for (int64_t i = li > RING_ROWS ? li - RING_ROWS : 0; i < li; ++i)
+                ptx::wait_bounded(ptx::smem_addr(&ring_full[i % RING_ROWS]), static_cast<uint32_t>((i / RING_ROWS) & 1),
+                                  p.timeout_ns, &no_abort, ERR_ROW_RING);
         }
     }
     if constexpr (MODE == ROW_RMS_STAT) {
