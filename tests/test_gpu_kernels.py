@@ -445,6 +445,63 @@ def test_rmsnorm_absmax(M, d, dt):
     assert bits_equal(host(am), ref), mismatch_report(host(am), ref)
 
 
+# ------------------------------------------------------------------ row ring
+@pytest.mark.parametrize("case", ["token_bf16_8192", "token_f16_6144", "token_f32_8192", "weight_bf16_8192",
+                                  "gateup_bf16_8192", "stat_bf16_4096", "stat_f16_8192"])
+def test_row_ring_paths(case):
+    """Row kernels whose rows come through the shared-memory ring of bulk
+    copies (256-thread rows held in registers: per-token quant and the weight
+    transform; the norm-output statistic from 64 rows per SM up), at row
+    counts that are not a multiple of the grid and with a ragged last vector
+    group (6144 = 3 vectors per thread of 4), bit for bit against the oracle."""
+    kind, dname, k = case.split("_")
+    dt = {"bf16": BF16, "f16": F16, "f32": F32}[dname]
+    K = int(k)
+    g = np.random.default_rng(K + len(case))
+    s = (np.abs(g.standard_normal(K)) + 0.2).astype(np.float32)
+    if kind == "token":
+        M = 1000 if dt != F32 else 400
+        X = rand_x(M + K, (M, K), dt, 2.0, outliers=8)
+        xq = torch.empty(M, K, dtype=torch.int8, device="cuda")
+        at = torch.empty(M, dtype=torch.float32, device="cuda")
+        sq.smooth_quant_act(dev(X, dt), dev(s), oracle.PER_TOKEN, at, xq)
+        _sync()
+        xq_ref, a_ref = oracle.smooth_quant_act(X, s, oracle.PER_TOKEN, None, dt)
+        assert bits_equal(host(at), a_ref), mismatch_report(host(at), a_ref)
+        assert bits_equal(host(xq), xq_ref), mismatch_report(host(xq), xq_ref)
+    elif kind == "weight":
+        N = 1000
+        W = rand_x(N + K, (N, K), dt, 0.02)
+        wq = torch.empty(N, K, dtype=torch.int8, device="cuda")
+        ws = torch.empty(N, dtype=torch.float32, device="cuda")
+        sq.quant_weight(dev(W, dt), dev(s), wq, ws)
+        _sync()
+        wq_ref, ws_ref = oracle.quant_weight(W, s, dt)
+        assert bits_equal(host(ws), ws_ref), mismatch_report(host(ws), ws_ref)
+        assert bits_equal(host(wq), wq_ref), mismatch_report(host(wq), wq_ref)
+    elif kind == "gateup":
+        Nh = 160
+        Wg = rand_x(11, (Nh, K), dt, 0.02)
+        Wu = rand_x(12, (Nh, K), dt, 0.02)
+        wq = torch.empty(2 * Nh, K, dtype=torch.int8, device="cuda")
+        ws = torch.empty(2 * Nh, dtype=torch.float32, device="cuda")
+        sq.quant_weight_gateup(dev(Wg, dt), dev(Wu, dt), dev(s), wq, ws)
+        _sync()
+        order = np.concatenate([np.concatenate([np.arange(b, b + 32), Nh + np.arange(b, b + 32)])
+                                for b in range(0, Nh, 32)])
+        wq_ref, ws_ref = oracle.quant_weight(np.concatenate([Wg, Wu])[order], s, dt)
+        assert bits_equal(host(wq), wq_ref) and bits_equal(host(ws), ws_ref)
+    else:
+        M = 9500 if K == 4096 else 9600          # >= 64 rows per SM of a 148-SM part: ring path
+        X = rand_x(M + K, (M, K), dt, 1.0, outliers=max(1, K // 200))
+        gamma = g.uniform(0.5, 1.5, K).astype(np.float32)
+        am = torch.zeros(K, dtype=torch.float32, device="cuda")
+        sq.rmsnorm_absmax(dev(X, dt), dev(gamma), 1e-5, am)
+        _sync()
+        ref = oracle.rmsnorm_absmax(X, gamma, 1e-5, dt)
+        assert bits_equal(host(am), ref), mismatch_report(host(am), ref)
+
+
 @pytest.mark.parametrize("dt", [F32, BF16])
 def test_quant_tiny_rows_saturate_like_the_oracle(dt):
     """Rows whose max gives a subnormal scale: codes still clamp to +-127 like the oracle's."""
