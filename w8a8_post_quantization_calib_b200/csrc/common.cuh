@@ -18,8 +18,6 @@ __host__ __device__ constexpr int dtype_size(int dt) { return dt == DT_F32 ? 4 :
 // device (0 = none).  Read and cleared by sq_sync_status.
 __device__ unsigned int g_error_word;
 
-__device__ __forceinline__ void record_error(unsigned code) { atomicCAS(&g_error_word, 0u, code); }
-
 // Programmatic dependent launch.  Every kernel of this library is launched
 // with programmatic stream serialisation: it may start while the previous
 // kernel in the stream is finishing, runs its prologue, and must execute
@@ -127,13 +125,6 @@ __device__ __forceinline__ float warp_max(float v)
     return v;
 }
 
-__device__ __forceinline__ float warp_sum(float v)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
-    return v;
-}
-
 __device__ __forceinline__ float block_max(float v, float *red)
 {
     v = warp_max(v);
@@ -143,17 +134,6 @@ __device__ __forceinline__ float block_max(float v, float *red)
     __syncthreads();
     float r = (l < nw) ? red[l] : 0.0f;
     return warp_max(r);
-}
-
-__device__ __forceinline__ float block_sum(float v, float *red)
-{
-    v = warp_sum(v);
-    const int w = threadIdx.x >> 5, l = threadIdx.x & 31, nw = blockDim.x >> 5;
-    __syncthreads();
-    if (l == 0) red[w] = v;
-    __syncthreads();
-    float r = (l < nw) ? red[l] : 0.0f;
-    return warp_sum(r);
 }
 
 __device__ __forceinline__ double block_sum_f64(double v, double *red)
