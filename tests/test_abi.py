@@ -70,3 +70,72 @@ def test_gemm_validation():
     assert lib.sq_linear_w8a8(17, 16, 4, 32, 64, 16, 0, 16, None, 1, 16, None, 0, None) == 3
     assert lib.sq_smooth_scales(16, 16, 8, 1.5, 16, None, None) == 1
     assert lib.sq_smooth_scales(16, 16, 8, -0.1, 16, None, None) == 1
+
+
+# Every entry point validates its arguments on the host and returns before
+# any CUDA call, so these run without a GPU.  Pointers are fake addresses
+# (16 = aligned, 17 = misaligned); no call below reaches a launch.
+_A, _U = 16, 17
+
+
+def _alphas(*v):
+    import ctypes
+    return (ctypes.c_float * len(v))(*v)
+
+
+@pytest.mark.parametrize("fn,args,status", [
+    ("sq_quant_weight", (None, 1, 8, 64, _A, _A, _A, None), 1),
+    ("sq_quant_weight", (_A, 9, 8, 64, _A, _A, _A, None), 1),
+    ("sq_quant_weight", (_A, 1, -1, 64, _A, _A, _A, None), 1),
+    ("sq_quant_weight", (_U, 1, 8, 64, _A, _A, _A, None), 3),
+    ("sq_quant_weight_gateup", (_A, _A, 1, 48, 64, _A, _A, _A, None), 1),      # N_h not a multiple of 32
+    ("sq_quant_weight_gateup", (_A, _U, 1, 64, 64, _A, _A, _A, None), 3),
+    ("sq_smooth_quant_act", (_A, 1, 4, 64, _A, 2, _A, _A, None), 1),          # unknown mode
+    ("sq_smooth_quant_act", (_A, 1, 4, 0, _A, 0, _A, _A, None), 1),
+    ("sq_smooth_quant_act", (_A, 1, 4, 64, _A, 1, _A, _U, None), 3),
+    ("sq_smooth_quant_act", (_A, 1, 0, 64, _A, 1, _A, _A, None), 0),          # no rows: nothing to do
+    ("sq_rmsnorm_quant", (_A, 2, 4, 64, None, _A, 1e-5, _A, _A, None, None), 1),
+    ("sq_rmsnorm_quant", (_A, 2, 4, 64, _A, _A, -1.0, _A, _A, None, None), 1),
+    ("sq_rmsnorm_quant", (_A, 2, 4, 64, _A, _A, float("nan"), _A, _A, None, None), 1),
+    ("sq_rmsnorm_quant", (_U, 2, 4, 64, _A, _A, 1e-5, _A, _A, None, None), 3),
+    ("sq_rmsnorm_absmax", (_A, 2, 4, 0, _A, 1e-5, _A, None), 1),
+    ("sq_rmsnorm_absmax", (_U, 2, 4, 64, _A, 1e-5, _A, None), 3),
+    ("sq_rmsnorm_absmax", (_A, 2, 0, 64, _A, 1e-5, _A, None), 0),
+    ("sq_linear_w8a8_gateup_silu", (_A, _A, 300, 96, 512, _A, 0, _A, _A, None, None, None, None), 1),   # N_h % 128
+    ("sq_linear_w8a8_gateup_silu", (_A, _A, 300, 128, 512, _A, 0, _A, None, None, None, None, None), 1),  # no output
+    ("sq_linear_w8a8_gateup_silu", (_A, _A, 300, 128, 512, _A, 0, _A, None, None, None, _A, None), 1),   # hq without s2/a2
+    ("sq_linear_w8a8_gateup_silu", (_A, _A, 300, 128, 512, _A, 0, _A, _U, None, None, None, None), 3),
+    ("sq_gemm_f16_ref", (_A, _A, 4, 40, 64, _A, None), 1),                    # N % 16
+    ("sq_gemm_f16_ref", (_A, _A, 4, 32, 12, _A, None), 1),                    # K % 8
+    ("sq_gemm_f16_ref", (_A, _A, 4, 32, 64, _U, None), 3),
+    ("sq_sse_f16", (_A, _A, -1, _A, None), 1),
+    ("sq_sse_f16", (_A, _U, 8, _A, None), 3),
+    ("sq_sse_f16", (_A, _A, 0, _A, None), 0),
+    ("sq_gemm_s32", (_A, _A, 4, 32, 64, None, None), 1),
+    ("sq_gemm_s32", (_A, _A, 4, 32, 64, _U, None), 3),
+    ("sq_linear_w8a8_noalloc", (_A, _A, 128, 32768, 4096, _A, 1, _A, None, 2, _A, None), 2),   # M*N above the array
+    ("sq_linear_w8a8_noalloc", (_A, _A, 4, 32, 64, _A, 3, _A, None, 2, _A, None), 1),          # unknown mode
+    ("sq_calib_absmax", (_A, 1, 0, 64, 64, _A, None), 0),
+])
+def test_every_entry_point_validates_before_launch(fn, args, status):
+    import w8a8_post_quantization_calib_b200 as sq
+    assert getattr(sq.lib(), fn)(*args) == status
+
+
+def test_alpha_search_validation():
+    import ctypes
+    import w8a8_post_quantization_calib_b200 as sq
+    lib = sq.lib()
+    best = ctypes.c_float()
+    # alphas must be ascending and within [0, 1]; 1..16 of them; a workspace is required
+    assert lib.sq_alpha_search(_A, _A, 512, 256, 512, _A, _A, _alphas(0.5, 0.25), 2, _A, 1 << 30,
+                               ctypes.byref(best), None, None) == 1
+    assert lib.sq_alpha_search(_A, _A, 512, 256, 512, _A, _A, _alphas(0.5, 1.5), 2, _A, 1 << 30,
+                               ctypes.byref(best), None, None) == 1
+    assert lib.sq_alpha_search(_A, _A, 512, 256, 512, _A, _A, _alphas(0.5), 0, _A, 1 << 30,
+                               ctypes.byref(best), None, None) == 1
+    assert lib.sq_alpha_search(_A, _A, 512, 256, 512, _A, _A, _alphas(0.5), 1, None, 1 << 30,
+                               ctypes.byref(best), None, None) == 1
+    assert lib.sq_alpha_search(_A, _A, 512, 256, 512, _A, _A, _alphas(0.25, 0.5), 2, _A, 16,
+                               ctypes.byref(best), None, None) == 6          # workspace too small
+
