@@ -23,6 +23,13 @@ Parity pins (tests/test_oracle_pins.py; tests/golden/ fixtures):
   quant rule            -- [KWKR] 1.2 worked numbers (golden), RNE ties
   calib_absmax          -- numpy reduction, running-max == concatenated max,
                            outlier channel reads back exactly 100.0
+  calib_quantile        -- p = 1 equals calib_absmax; numpy's inverted-CDF
+                           quantile (the nearest-rank definition); a planted
+                           outlier token moves the max but not the 99.9 %
+                           quantile ([KWKR] 3.1)
+  calib_mean_of_max     -- equal batch maxima give the max; constructed
+                           per-batch maxima give their exact mean; bounded by
+                           the smallest and largest batch maximum
   smooth_scales         -- alpha = 0.5 / 1 / 0 closed forms, clamp at 1e-5
   static_scale          -- brute force over every smoothed calibration value
                            (bit-exact: fl() is monotone)
@@ -186,6 +193,41 @@ def calib_absmax(x: np.ndarray, dt: int | None = None, absmax: np.ndarray | None
     assert out.dtype == np.float32 and out.flags.c_contiguous
     lib().oracle_calib_absmax(_ptr(x), dt, rows, cols, cols, _ptr(out))
     return out
+
+
+def quantile_rank(p: float, count: int) -> int:
+    """1-based nearest rank of the p-quantile among `count` values: k = ceil(p * count)
+    (the product taken in fp64), at least 1 and at most count."""
+    import math
+    if not (0.0 < p <= 1.0) or count < 1:
+        raise ValueError("need 0 < p <= 1 and at least one value")
+    return min(count, max(1, math.ceil(float(p) * float(count))))
+
+
+def calib_quantile(batches, p: float, dt: int | None = None) -> np.ndarray:
+    """Robust calibration statistic, [KWKR] 3.1: a quantile of |X_j| over all the
+    calibration tokens (the page names 99.9 %) in place of the max, so that one
+    sample with an abnormally large activation does not set the channel's s.
+
+    Per channel j the p-quantile by nearest rank: with the T values |x_tj|
+    sorted ascending, the k-th smallest, k = quantile_rank(p, T).  It is one
+    of the data values (widened exactly to fp32); p = 1 gives the max."""
+    cols = [np.abs(to_f32(*_dtcode(b, dt))) for b in batches]
+    a = np.concatenate(cols, axis=0)                       # [T, K]
+    k = quantile_rank(p, a.shape[0])
+    return np.sort(a, axis=0)[k - 1].astype(np.float32)
+
+
+def calib_mean_of_max(batches, dt: int | None = None) -> np.ndarray:
+    """Robust calibration statistic, [KWKR] 3.1: the mean over calibration
+    samples of each sample's max|X_j| (a sample being one calibration batch).
+    The per-sample maxima are added in fp64 in sample order, the sum is divided
+    by the sample count in fp64 and rounded once to fp32."""
+    total = None
+    for b in batches:
+        m = calib_absmax(b, dt).astype(np.float64)
+        total = m if total is None else total + m
+    return (total / float(len(batches))).astype(np.float32)
 
 
 def smooth_scales(act_max: np.ndarray, w_max: np.ndarray, alpha: float = ALPHA_DEFAULT) -> np.ndarray:

@@ -114,6 +114,67 @@ def test_calib_absmax_vs_numpy(dt):
     assert np.array_equal(run, np.abs(allx).max(axis=0))
 
 
+@pytest.mark.parametrize("dt", [F32, F16, BF16])
+def test_calib_quantile_at_one_is_the_max(dt):
+    g = np.random.default_rng(40 + dt)
+    batches = [synth.cast(g.standard_normal((r, 53)).astype(np.float32) * 4, dt) for r in (7, 30, 1)]
+    run = np.zeros(53, np.float32)
+    for b in batches:
+        oracle.calib_absmax(b, dt, run)
+    assert np.array_equal(oracle.calib_quantile(batches, 1.0, dt), run)
+
+
+@pytest.mark.parametrize("p", [0.999, 0.9, 0.5, 0.013])
+def test_calib_quantile_is_numpy_inverted_cdf(p):
+    """Nearest rank k = ceil(pT) is numpy's inverted-CDF quantile (the smallest
+    value whose empirical CDF reaches p); T = 3001 keeps pT off the integers."""
+    g = np.random.default_rng(41)
+    batches = [synth.cast(g.standard_normal((r, 40)).astype(np.float32), BF16) for r in (1000, 2000, 1)]
+    a = np.abs(np.concatenate([oracle.to_f32(b, BF16) for b in batches]))
+    assert a.shape[0] == 3001 and abs(p * 3001 - round(p * 3001)) > 1e-6
+    ref = np.quantile(a, p, axis=0, method="inverted_cdf")
+    assert np.array_equal(oracle.calib_quantile(batches, p, BF16), ref.astype(np.float32))
+
+
+def test_calib_quantile_ignores_a_planted_outlier():
+    """[KWKR] 3.1: one sample with an abnormally large activation sets the max
+    of its channel; the 99.9 % quantile of 2000 tokens (rank 1998) stays with
+    the body of the distribution.  Channel 3: 1999 tokens with |x| = t/2000
+    (t = 1..1999) and one token at 5000."""
+    x = np.zeros((2000, 8), np.float32)
+    x[:1999, 3] = np.arange(1, 2000, dtype=np.float32) / 2000
+    x[1999, 3] = -5000.0
+    batches = [x[:700], x[700:]]
+    assert oracle.quantile_rank(0.999, 2000) == 1998
+    q = oracle.calib_quantile(batches, 0.999, F32)
+    assert q[3] == np.float32(1998) / 2000            # the 1998-th smallest |x|
+    assert oracle.calib_absmax(x, F32)[3] == 5000.0
+    assert np.all(q[np.arange(8) != 3] == 0.0)
+
+
+def test_calib_mean_of_max_closed_forms():
+    """[KWKR] 3.1 mean of per-sample maxima: batches whose channel maxima are
+    1, 2, 3, 4.5 (exact in every format) give 2.625; equal maxima give that max;
+    in general the mean lies between the smallest and largest batch maximum."""
+    B, K = 4, 6
+    peaks = np.array([1.0, 2.0, 3.0, 4.5], np.float32)
+    batches = []
+    for b in range(B):
+        x = np.full((5, K), 0.25, np.float32)
+        x[b + 1, 2] = -peaks[b]                     # channel 2: the planted per-batch maximum
+        x[0, 4] = 7.0                              # channel 4: the same maximum in every batch
+        batches.append(synth.cast(x, BF16))
+    m = oracle.calib_mean_of_max(batches, BF16)
+    assert m[2] == np.float32(2.625)
+    assert m[4] == np.float32(7.0)
+    assert m[0] == np.float32(0.25)
+    g = np.random.default_rng(42)
+    rb = [synth.cast(g.standard_normal((r, 31)).astype(np.float32) * 2, F16) for r in (3, 50, 9, 17)]
+    mm = oracle.calib_mean_of_max(rb, F16)
+    per = np.stack([oracle.calib_absmax(b, F16) for b in rb])
+    assert np.all(mm >= per.min(axis=0)) and np.all(mm <= per.max(axis=0))
+
+
 def test_toy_outlier_channel_statistic(golden_dir):
     spec = json.load(open(os.path.join(golden_dir, "tbr8_toy_layer.json")))
     wl = synth.linear_toy()
