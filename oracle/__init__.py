@@ -30,6 +30,13 @@ Parity pins (tests/test_oracle_pins.py; tests/golden/ fixtures):
   calib_mean_of_max     -- equal batch maxima give the max; constructed
                            per-batch maxima give their exact mean; bounded by
                            the smallest and largest batch maximum
+  e4m3_decode / encode  -- all 256 codes and in-range values (ties included)
+                           against torch's float8_e4m3fn casts; saturation
+                           to +-448 beyond (torch gives NaN there)
+  fp8 quantisers        -- the row maximum maps to +-448; every code within
+                           half an E4M3 spacing of its value
+  gemm_fp8_f64          -- exact: equals the int64 matmul of the codes'
+                           values scaled by 2^9
   smooth_scales         -- alpha = 0.5 / 1 / 0 closed forms, clamp at 1e-5
   static_scale          -- brute force over every smoothed calibration value
                            (bit-exact: fl() is monotone)
@@ -272,6 +279,85 @@ def smooth_quant_act(x: np.ndarray, s: np.ndarray, mode: int, a_scale=None, dt: 
         a = np.empty(M, np.float32)
     lib().oracle_smooth_quant_act(_ptr(x), dt, M, K, _ptr(s), mode, _ptr(a), _ptr(xq))
     return xq, a
+
+
+# --------------------------------------------------------------------------
+# FP8 (E4M3) variant: the same smoothing in front of an FP8 quantiser ([AIU]:
+# smoothing carries over to FP8 on Hopper / Blackwell).  E4M3: 1 sign, 4
+# exponent bits (bias 7), 3 mantissa bits, no infinities, code 0x7F / 0xFF
+# NaN, largest finite 448.
+# --------------------------------------------------------------------------
+E4M3_MAX = 448.0
+
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    """E4M3 codes (uint8) -> fp32 values (exact)."""
+    c = np.asarray(codes, np.uint8).astype(np.int64)
+    e, m = (c >> 3) & 0xF, c & 0x7
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    v = np.where(c & 0x80, -mag, mag)
+    v = np.where((c & 0x7F) == 0x7F, np.nan, v)
+    return v.astype(np.float32)
+
+
+_E4M3_POS = e4m3_decode(np.arange(0x7F, dtype=np.uint8)).astype(np.float64)   # codes 0..126, ascending
+
+
+def e4m3_encode(v: np.ndarray) -> np.ndarray:
+    """fp32 -> E4M3 codes: round to nearest, ties to the even code (even
+    mantissa), magnitudes beyond 448 saturate to +-448 (the finite-saturating
+    conversion), NaN -> 0x7F.  The nearest of the 127 non-negative finite
+    values is found by search over the ascending table."""
+    v = np.asarray(v, np.float32)
+    a = np.abs(v).astype(np.float64)
+    hi = np.clip(np.searchsorted(_E4M3_POS, a, side="left"), 0, 126)    # first value >= a
+    lo = np.clip(hi - 1, 0, 126)
+    dlo, dhi = a - _E4M3_POS[lo], _E4M3_POS[hi] - a
+    pick_hi = (dhi < dlo) | ((dhi == dlo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo)
+    code = np.where(a >= E4M3_MAX, 126, code)                             # saturate
+    code = code.astype(np.int64) | np.where(np.signbit(v), 0x80, 0)
+    code = np.where(np.isnan(v), 0x7F, code)
+    return code.astype(np.uint8)
+
+
+def _f32(x):
+    return np.asarray(x, np.float32)
+
+
+def _recip32(v: np.ndarray) -> np.ndarray:
+    """fl(1/v), 0 for v = 0 (the reciprocal rule of the INT8 path)."""
+    v = _f32(v)
+    with np.errstate(divide="ignore"):
+        return np.where(v > 0, np.float32(1.0) / np.where(v > 0, v, np.float32(1.0)), np.float32(0.0)).astype(np.float32)
+
+
+def smooth_quant_act_fp8(x: np.ndarray, s: np.ndarray, mode: int, a_scale=None, dt: int | None = None):
+    """x/s, then E4M3 with a per-tensor (static) or per-token scale a = max|x'|/448,
+    in the INT8 path's fp32 order: x' = fl(x * fl(1/s_j)); code = e4m3(fl(x' * fl(1/a)))."""
+    x, dt = _dtcode(x, dt)
+    xf = to_f32(x, dt)
+    xs = (xf * _recip32(s)[None, :]).astype(np.float32)
+    if mode == STATIC:
+        a = _f32([a_scale]).ravel()[:1]
+        inv = _recip32(a)[0]
+        return e4m3_encode((xs * inv).astype(np.float32)), a
+    a = (np.abs(xs).max(axis=1) / np.float32(E4M3_MAX)).astype(np.float32)
+    return e4m3_encode((xs * _recip32(a)[:, None]).astype(np.float32)), a
+
+
+def quant_weight_fp8(w: np.ndarray, s: np.ndarray, dt: int | None = None):
+    """W' = fl(W * s_j), per-row scale fl(max|W'_n| / 448), codes e4m3(fl(W' * fl(1/scale)))."""
+    w, dt = _dtcode(w, dt)
+    wf = (to_f32(w, dt) * _f32(s)[None, :]).astype(np.float32)
+    sc = (np.abs(wf).max(axis=1) / np.float32(E4M3_MAX)).astype(np.float32)
+    return e4m3_encode((wf * _recip32(sc)[:, None]).astype(np.float32)), sc
+
+
+def gemm_fp8_f64(xq: np.ndarray, wq: np.ndarray) -> np.ndarray:
+    """acc = dec(xq) . dec(wq)^T in fp64.  Every product of two E4M3 values is a
+    multiple of 2^-18 below 2^18, so for K < 2^16 the fp64 sum is exact in any order."""
+    return e4m3_decode(xq).astype(np.float64) @ e4m3_decode(wq).astype(np.float64).T
 
 
 def gemm_s32(xq: np.ndarray, wq: np.ndarray) -> np.ndarray:

@@ -536,3 +536,72 @@ def test_pipeline_output_close_to_fp64():
     Y = synth.as_f16(wl.x).astype(np.float64) @ synth.as_f16(wl.w).astype(np.float64).T
     rel = np.linalg.norm(y - Y) / np.linalg.norm(Y)
     assert rel < 0.05
+
+
+# --------------------------------------------------------------------------
+# FP8 (E4M3) variant ([AIU]: smoothing carries over to FP8)
+# --------------------------------------------------------------------------
+
+def test_e4m3_decode_all_codes_vs_torch():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float32).numpy()
+    got = oracle.e4m3_decode(codes)
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(got[ok].view(np.uint32), ref[ok].view(np.uint32))
+
+
+def test_e4m3_encode_vs_torch_in_range():
+    """Round to nearest, ties to even, on random values from the subnormals up
+    to 448 and on every exact midpoint between neighbouring codes."""
+    g = np.random.default_rng(50)
+    v = (g.standard_normal(200000) * np.exp2(g.uniform(-12, 8.7, 200000))).astype(np.float32)
+    v = v[np.abs(v) < 464]
+    pos = oracle.e4m3_decode(np.arange(0x7F, dtype=np.uint8)).astype(np.float64)
+    mids = ((pos[1:] + pos[:-1]) / 2).astype(np.float32)
+    assert np.array_equal(mids.astype(np.float64), (pos[1:] + pos[:-1]) / 2)   # midpoints exact in fp32
+    v = np.concatenate([v, mids, -mids, pos.astype(np.float32), np.float32([0.0, -0.0])])
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.e4m3_encode(v), ref)
+
+
+def test_e4m3_encode_saturates():
+    """Beyond the largest finite value the conversion saturates (the reading
+    taken for the quantiser; torch's cast gives NaN there)."""
+    v = np.float32([464.0, 480.0, 1e6, -500.0, np.inf, -np.inf])
+    assert list(oracle.e4m3_encode(v)) == [0x7E, 0x7E, 0x7E, 0xFE, 0x7E, 0xFE]
+    assert oracle.e4m3_encode(np.float32([np.nan]))[0] == 0x7F
+
+
+def test_fp8_quantisers_map_the_row_max_to_448():
+    g = np.random.default_rng(51)
+    X = synth.cast(g.standard_normal((37, 96)).astype(np.float32) * 3, BF16)
+    s = (np.abs(g.standard_normal(96)) + 0.2).astype(np.float32)
+    q, a = oracle.smooth_quant_act_fp8(X, s, PER_TOKEN, dt=BF16)
+    dec = oracle.e4m3_decode(q).astype(np.float64)
+    assert np.all(np.abs(dec).max(axis=1) == 448.0)
+    xs = oracle.to_f32(X, BF16).astype(np.float64) / s.astype(np.float64)[None, :]
+    v = xs / a.astype(np.float64)[:, None]
+    # nearest E4M3: within half a spacing (2^-4 relative for normals, 2^-10 absolute below 2^-6)
+    assert np.all(np.abs(dec - v) <= np.maximum(np.abs(v) * 2.0 ** -4, 2.0 ** -10) * (1 + 1e-6))
+    W = synth.cast(g.standard_normal((23, 96)).astype(np.float32) * 0.02, BF16)
+    qw, sw = oracle.quant_weight_fp8(W, s, BF16)
+    assert np.all(np.abs(oracle.e4m3_decode(qw)).max(axis=1) == 448.0)
+    # static: a scale that puts the outlier beyond 448 saturates it
+    qs, _ = oracle.smooth_quant_act_fp8(X, s, STATIC, a_scale=np.float32(a.min()), dt=BF16)
+    assert np.abs(oracle.e4m3_decode(qs)).max() == 448.0
+
+
+def test_gemm_fp8_f64_is_exact():
+    """E4M3 values are multiples of 2^-9, so their products scaled by 2^18 are
+    integers: the int64 matmul of the codes' values times 2^9 is the exact sum."""
+    g = np.random.default_rng(52)
+    xq = g.integers(0, 256, (9, 700), dtype=np.uint8)
+    wq = g.integers(0, 256, (13, 700), dtype=np.uint8)
+    xq[(xq & 0x7F) == 0x7F] = 0x7E                      # no NaN codes
+    wq[(wq & 0x7F) == 0x7F] = 0xFE
+    xi = np.rint(oracle.e4m3_decode(xq).astype(np.float64) * 512).astype(np.int64)
+    wi = np.rint(oracle.e4m3_decode(wq).astype(np.float64) * 512).astype(np.int64)
+    assert np.array_equal(xi.astype(np.float64) / 512, oracle.e4m3_decode(xq).astype(np.float64))
+    exact = xi @ wi.T
+    assert np.array_equal(oracle.gemm_fp8_f64(xq, wq) * 2.0 ** 18, exact.astype(np.float64))
