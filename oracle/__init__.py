@@ -37,6 +37,9 @@ Parity pins (tests/test_oracle_pins.py; tests/golden/ fixtures):
                            half an E4M3 spacing of its value
   gemm_fp8_f64          -- exact: equals the int64 matmul of the codes'
                            values scaled by 2^9
+  fold_into_previous    -- fp64 identity (X Wp'^T)(W diag(s))^T == (X Wp^T) W^T,
+                           also through the gated form silu(g) * u
+  scales_fp16           -- numpy's float16 round trip
   smooth_scales         -- alpha = 0.5 / 1 / 0 closed forms, clamp at 1e-5
   static_scale          -- brute force over every smoothed calibration value
                            (bit-exact: fl() is monotone)
@@ -469,6 +472,29 @@ def identity_residual(X: np.ndarray, W: np.ndarray, s: np.ndarray) -> float:
     Y = X @ W.T
     Ys = (X / s[None, :]) @ (W * s[None, :]).T
     return float(np.linalg.norm(Y - Ys) / np.linalg.norm(Y))
+
+
+# --------------------------------------------------------------------------
+# Follow-ups named by [ADR10]: cross-layer folding (Alternative C) and fp16
+# storage of the scales (Consequences, storage)
+# --------------------------------------------------------------------------
+
+def fold_into_previous(w_prev: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """Cross-layer folding: when the smoothed layer's input is a previous
+    linear's output (or depends linearly on it, as h = silu(g) * u does on the
+    up projection), 1/s_j moves into that layer's output row j,
+    W_prev'[j, :] = fl(W_prev[j, :] * fl(1/s_j)), and the runtime x/s step
+    disappears.  w_prev: fp32 [K, K_prev] (out x in); returns fp32."""
+    w = np.asarray(w_prev, np.float32)
+    return (w * _recip32(s)[:, None]).astype(np.float32)
+
+
+def scales_fp16(*scales):
+    """fp16 storage of scales ([ADR10] consequences: per-row weight scale,
+    per-tensor activation scale and input scales s in fp16): each fp32 scale
+    rounded to the nearest fp16 (RNE) and read back widened exactly to fp32,
+    the values every later step then uses."""
+    return tuple(to_f32(from_f32(np.asarray(v, np.float32), F16), F16) for v in scales)
 
 
 # --------------------------------------------------------------------------

@@ -605,3 +605,39 @@ def test_gemm_fp8_f64_is_exact():
     assert np.array_equal(xi.astype(np.float64) / 512, oracle.e4m3_decode(xq).astype(np.float64))
     exact = xi @ wi.T
     assert np.array_equal(oracle.gemm_fp8_f64(xq, wq) * 2.0 ** 18, exact.astype(np.float64))
+
+
+# --------------------------------------------------------------------------
+# follow-ups: cross-layer folding, fp16 scale storage ([ADR10])
+# --------------------------------------------------------------------------
+
+def test_fold_into_previous_identity():
+    """Folding 1/s into the previous layer's output rows leaves the product of
+    the two layers unchanged (fp64, up to the fp32 rounding of the folded
+    weights), directly and through the gated MLP form h = silu(g) * u."""
+    g = np.random.default_rng(60)
+    Kp, K, N, M = 48, 64, 40, 9
+    X = g.standard_normal((M, Kp)).astype(np.float32)
+    Wp = (g.standard_normal((K, Kp)) * 0.1).astype(np.float32)
+    Wg = (g.standard_normal((K, Kp)) * 0.1).astype(np.float32)
+    W = (g.standard_normal((N, K)) * 0.1).astype(np.float32)
+    s = (np.abs(g.standard_normal(K)) + 0.3).astype(np.float32)
+    Wp2 = oracle.fold_into_previous(Wp, s).astype(np.float64)
+    Ws = W.astype(np.float64) * s.astype(np.float64)[None, :]
+    x = X.astype(np.float64)
+    ref = (x @ Wp.astype(np.float64).T) @ W.astype(np.float64).T
+    got = (x @ Wp2.T) @ Ws.T
+    assert np.linalg.norm(got - ref) / np.linalg.norm(ref) < 1e-6
+    gate = x @ Wg.astype(np.float64).T
+    silu = gate / (1.0 + np.exp(-gate))
+    ref_h = (silu * (x @ Wp.astype(np.float64).T)) @ W.astype(np.float64).T
+    got_h = (silu * (x @ Wp2.T)) @ Ws.T
+    assert np.linalg.norm(got_h - ref_h) / np.linalg.norm(ref_h) < 1e-6
+
+
+def test_scales_fp16_round_trip():
+    g = np.random.default_rng(61)
+    v = (np.abs(g.standard_normal(1000)) * np.exp2(g.uniform(-14, 10, 1000))).astype(np.float32)
+    (got,) = oracle.scales_fp16(v)
+    assert np.array_equal(got, v.astype(np.float16).astype(np.float32))
+
