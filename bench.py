@@ -704,6 +704,24 @@ def run_workload(args):
             gbs = nbytes / (t_ms * 1e-3) / 1e9
             lines.append({"kernel": name, "shape": shape, "dtype": dt, "us": t_ms * 1e3, "gbs": gbs,
                           "frac_hbm": gbs / P["hbm_gbs"]})
+        if only is None or "calib_64_launches" in only:
+            # the QKV workload's calibration set (64 batches x 512 tokens, fp16,
+            # K = 4096) as 64 launches, one per batch, against the one launch
+            # over the concatenated batches
+            cb = torch.randn(64 * 512, 4096, generator=g16, device="cuda").to(torch.float16)
+            amc = torch.zeros(4096, device="cuda")
+            views = [cb[i * 512:(i + 1) * 512] for i in range(64)]
+
+            def per_batch():
+                for v in views:
+                    sq.calib_absmax(v, amc)
+            for name, fn in (("calib_64_launches", per_batch), ("calib_1_launch", lambda: sq.calib_absmax(cb, amc))):
+                t_ms = _time_ms(fn, 5)
+                gbs = cb.numel() * 2 / (t_ms * 1e-3) / 1e9
+                lines.append({"kernel": name, "shape": [64 * 512, 4096], "dtype": "f16", "us": t_ms * 1e3, "gbs": gbs,
+                              "frac_hbm": gbs / P["hbm_gbs"]})
+            del cb, views
+            torch.cuda.empty_cache()
         shapes = ((4096, torch.float16), (8192, torch.bfloat16))
         if args.rows_k:
             shapes = tuple(sh for sh in shapes if sh[0] in {int(k) for k in args.rows_k.split(",")})
