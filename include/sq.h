@@ -90,7 +90,10 @@ void sq_set_wait_timeout_ns(unsigned long long ns);
  *      hangs.
  *   2: small-M GEMMs run without the cluster split (on the stream-K or
  *      one-tile-per-CTA schedules), so that tests reach those paths.
- * what = 0 turns both off. */
+ *   4: sq_linear_w8a8_noalloc checks its requests against a capacity of
+ *      64 KiB of partial sums instead of its whole array, so that tests reach
+ *      its rejection of oversize requests.
+ * what = 0 turns them off. */
 void sq_debug_inject(int what);
 
 /* Synchronises `stream`, then returns SQ_ERR_TIMEOUT if any kernel of this
@@ -224,7 +227,7 @@ sq_status sq_rmsnorm_absmax(const void *x, sq_dtype dt, int64_t M, int64_t d, co
  * tile's K range and combines the int32 partial sums in distributed shared
  * memory; no workspace is needed.  The stream-K schedule (iterations shared
  * evenly among the SMs, partial sums through global memory) is the fallback
- * when the cluster split is off (sq_debug_inject bit 2); it needs
+ * when the cluster split is off (sq_debug_inject(2)); it needs
  * `workspace` of sq_linear_workspace_size(M, N, K) bytes (16-byte aligned;
  * the size depends on the current device's SM count and the test hooks, and
  * is 0 when no workspace is used): one BM x BN int32 partial-sum slot per CTA
@@ -247,24 +250,27 @@ sq_status sq_linear_w8a8(const int8_t *xq, const int8_t *wq, int64_t M, int64_t 
  * all: a plugin running inside a host engine that owns every device buffer
  * and hands it only inputs and outputs, or a latency-critical serving loop
  * that must not pay cudaMalloc's implicit device-wide synchronisation.  This
- * call takes no workspace: the small-M cluster split needs none, and the
- * small-M stream-K fallback (M <= 128, cluster split off) keeps its int32
- * partial sums and per-tile counters in a fixed array inside the library
- * (8 MiB of partial-sum slots + 64 KiB of counters, held by every GPU that
- * loads the library until the process exits; the number of CTAs sharing the
- * iterations is capped by how many slots fit, and the path runs one tile per
- * CTA when too few fit).  M*N beyond
- * sq_linear_w8a8_noalloc_max_elems() (2^21 = 2097152) on that path returns
- * SQ_ERR_UNSUPPORTED without launching; M > 128 needs no scratch and runs the
- * sq_linear_w8a8 launch.  The call allocates nothing: no cudaMalloc,
- * cudaFree or allocating library routine.
- *   - The first call on each device looks up the array's device address (with
- *     that device current) and caches it; make that first call before any
- *     stream capture.
+ * call takes no workspace and runs the same schedules as sq_linear_w8a8, so
+ * its results are bit-identical to that call's.  M > 128, and the small-M
+ * schedules that keep their partial sums on chip (the cluster split, one tile
+ * per CTA), use no scratch at all and accept any shape sq_linear_w8a8
+ * accepts.  Only the small-M stream-K schedule (the fallback when the cluster
+ * split is off, sq_debug_inject(2)) shares weight tiles between CTAs through
+ * scratch memory; here that scratch is a fixed array inside the library:
+ * 8 MiB of int32 partial-sum slots (sq_linear_w8a8_noalloc_max_elems() int32
+ * values) plus 64 KiB of per-tile arrival counters, held by every GPU that
+ * loads the library until the process exits.  The schedule needs one slot of
+ * 128 x (16 or 32) int32 per CTA, at most 2.4 MB with the 148 SMs of a B200;
+ * a request whose slots or counters would not fit (a device with many more
+ * SMs) returns SQ_ERR_UNSUPPORTED without launching anything.  The call
+ * allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ *   - The first call on each device that needs the array looks up its device
+ *     address (with that device current) and caches it; make that first call
+ *     before any stream capture.
  *   - Each call that shares tiles zeroes the arrival counters it uses (a
  *     stream-ordered memset) before its kernel, since the array keeps the
- *     previous call's contents; a partial-sum slot is always written before
- *     it is read.
+ *     previous call's contents (a call that timed out leaves its counters
+ *     raised); a partial-sum slot is always written before it is read.
  *   - All calls on a device share the one array: calls that overlap on the
  *     GPU (different streams, no ordering between them) race and corrupt each
  *     other's results.  Serialise them on one stream or order them with events.
@@ -273,7 +279,7 @@ sq_status sq_linear_w8a8_noalloc(const int8_t *xq, const int8_t *wq, int64_t M, 
                                  const float *a_scale, sq_act_mode mode, const float *w_scale,
                                  const void *bias, sq_dtype out_dt, void *y, sq_stream stream);
 
-/* Largest M*N the fixed array of sq_linear_w8a8_noalloc holds on its small-M path. */
+/* Capacity of the fixed partial-sum array of sq_linear_w8a8_noalloc, in int32 values (2^21). */
 size_t sq_linear_w8a8_noalloc_max_elems(void);
 
 /* Raw int32 accumulators acc[m,n] = sum_k xq[m,k] * wq[n,k] from the same
@@ -301,6 +307,51 @@ sq_status sq_linear_w8a8_gateup_silu(const int8_t *xq, const int8_t *wq_gu, int6
                                      sq_act_mode mode, const float *w_scale_gu, void *h,
                                      const float *s2, const float *a2, int8_t *hq,
                                      sq_stream stream);
+
+/* -------------------------------------------------------------------------
+ * FP8 (E4M3) variant.  aiunderstanding.org, "SmoothQuant 和激活量化" (on the
+ * method's future): the same smoothing carries over to FP8 formats on the
+ * Hopper / Blackwell tensor cores.  The calls mirror the INT8 ones with the
+ * same fp32 operation order; only the code format changes:
+ *
+ *   E4M3 code     = e4m3(v): round to nearest even, magnitudes beyond the
+ *                   largest finite value 448 saturate to +-448 (never NaN)
+ *   absmax scale  = fl(max |value| / 448)
+ *   act code      = e4m3(fl(fl(x * recip(s_j)) * recip(a)))
+ *   weight code   = e4m3(fl(fl(w * s_j) * recip(w_scale_n)))
+ *   acc[m,n]      = sum_k dec(xq8[m,k]) * dec(wq8[n,k])  in fp32 on the
+ *                   tensor cores (tcgen05 kind::f8f6f4; every product is
+ *                   exact, the sum is rounded in an unspecified order)
+ *   y[m,n]        = RN_out(fmaf(acc, fl(a_m * w_scale_n), bias_n))
+ *
+ * Codes are uint8 bit patterns (1 sign, 4 exponent bits with bias 7, 3
+ * mantissa bits).  Layouts, alignment and ownership are those of the INT8
+ * calls; the FP8 GEMM runs on the CTA-pair kernel for every M.
+ * ------------------------------------------------------------------------- */
+
+/* sq_smooth_scales with the static activation scale for E4M3 codes:
+ * a_static[0] = fl(max_j fl(act_max_j * recip(s_j)) / 448).  s is the same. */
+sq_status sq_smooth_scales_fp8(const float *act_max, const float *w_max, int64_t K, float alpha,
+                               float *s, float *a_static, sq_stream stream);
+
+/* W' = fl(W * s_j); w_scale[n] = fl(max_j |W'[n,j]| / 448); wq8 = e4m3 codes
+ * of fl(W' * recip(w_scale[n])).  wq8: uint8 [N, K]. */
+sq_status sq_quant_weight_fp8(const void *w, sq_dtype dt, int64_t N, int64_t K, const float *s,
+                              uint8_t *wq8, float *w_scale, sq_stream stream);
+
+/* x' = fl(x * recip(s_j)); static: a = a_scale[0] (read); per-token:
+ * a_scale[m] = fl(max_j |x'[m,j]| / 448) (written); xq8 = e4m3 codes of
+ * fl(x' * recip(a)).  xq8: uint8 [M, K]. */
+sq_status sq_smooth_quant_act_fp8(const void *x, sq_dtype dt, int64_t M, int64_t K, const float *s,
+                                  sq_act_mode mode, float *a_scale, uint8_t *xq8, sq_stream stream);
+
+/* y[m,n] = RN_out(fmaf(acc, fl(a_m * w_scale[n]), bias[n])) with the fp32
+ * tensor-core sum acc of the E4M3 products (see above).  Shapes and
+ * alignment as sq_linear_w8a8 (K a multiple of 16, N a multiple of 16);
+ * no workspace. */
+sq_status sq_linear_fp8(const uint8_t *xq8, const uint8_t *wq8, int64_t M, int64_t N, int64_t K,
+                        const float *a_scale, sq_act_mode mode, const float *w_scale,
+                        const void *bias, sq_dtype out_dt, void *y, sq_stream stream);
 
 /* -------------------------------------------------------------------------
  * Per-layer alpha search (adr-010 key design point 2: pick, per layer, the

@@ -48,11 +48,21 @@ Parity pins (tests/test_oracle_pins.py; tests/golden/ fixtures):
   gemm_s32              -- numpy int64 matmul (ragged shapes)
   dequant               -- fp64 product within one fp32 rounding + one output
                            rounding
+  dequant_f32           -- hand-computed values that each canonical rounding
+                           decides ((float)acc, fl(a_m * w_n), the product),
+                           per-token rows with distinct scales; fp64 bound;
+                           equal to dequant(..., F32, bias=None)
   rmsnorm_quant         -- fp64 unfused RMSNorm then x/s, within rounding
   rmsnorm_absmax        -- fp64 unfused RMSNorm column max, within rounding
-  silu_mul_bf16         -- math.exp closed form; silu(0) = 0, silu(g) -> g
+  silu_mul_bf16         -- math.exp closed form on a grid reaching the
+                           overflow range of exp (|g| up to 100); silu(0) = 0,
+                           silu(g) -> g, silu(-g) -> 0
   mse_f16, gemm_f16_ref -- numpy fp64 mean / matmul
-  identity              -- fp64 XW^T == (X diag(s)^-1)(W diag(s))^T, 1e-9
+  identity              -- fp64 XW^T == (X diag(s)^-1)(W diag(s))^T, 1e-9;
+                           smooth_operands on a hand-computed 2x2 case;
+                           rel_residual on a hand value; negative controls
+                           (s applied to one operand only) give residuals
+                           far above 1e-9
   quality gain          -- [ADR10] consequences: ~10x lower error with
                            smoothing on the outlier layer; not worse on normal
                            activations; smoothing after quantisation gives no
@@ -60,7 +70,9 @@ Parity pins (tests/test_oracle_pins.py; tests/golden/ fixtures):
                            "parity unpinned" (the page gives only "about an
                            order of magnitude"); the test bounds it below.
   alpha_search          -- argmin over the grid equals an fp64 numpy
-                           re-evaluation; the chosen MSE is <= both extremes.
+                           re-evaluation (fp64 dequant product) whose MSEs
+                           agree within 1e-4 relative; the chosen MSE is <=
+                           both extremes.
 """
 from __future__ import annotations
 
@@ -393,6 +405,8 @@ def dequant(acc: np.ndarray, a_scale: np.ndarray, mode: int, w_scale: np.ndarray
 
 
 def dequant_f32(acc, a_scale, mode, w_scale) -> np.ndarray:
+    """a9 -- the a6 epilogue values in fp32, no bias, no output rounding:
+    y = fl((float)acc * fl(a_m * w_n)) (the gate and up values of SiLU*mul)."""
     acc = np.ascontiguousarray(acc, np.int32)
     M, N = acc.shape
     a = np.ascontiguousarray(a_scale, np.float32).ravel()
@@ -461,17 +475,29 @@ def gemm_f16_ref(x_bits: np.ndarray, w_bits: np.ndarray) -> np.ndarray:
 # fp64 numpy checks of the mathematics
 # --------------------------------------------------------------------------
 
-def identity_residual(X: np.ndarray, W: np.ndarray, s: np.ndarray) -> float:
-    """[KWKR] 2.1: Y = XW = (X diag(s)^-1)(diag(s) W); relative Frobenius residual in fp64.
+def smooth_operands(X: np.ndarray, W: np.ndarray, s: np.ndarray):
+    """[KWKR] 2.1: the smoothed pair (X diag(s)^-1, W diag(s)) in fp64.
 
-    W is [N,K] (out x in), so diag(s) scales its columns.
-    """
+    X is [M,K]; W is [N,K] (out x in), so diag(s) scales its columns: both
+    operands are scaled along the shared input-channel index j."""
     X = np.asarray(X, np.float64)
     W = np.asarray(W, np.float64)
     s = np.asarray(s, np.float64)
-    Y = X @ W.T
-    Ys = (X / s[None, :]) @ (W * s[None, :]).T
+    return X / s[None, :], W * s[None, :]
+
+
+def rel_residual(Y: np.ndarray, Ys: np.ndarray) -> float:
+    """Relative Frobenius residual ||Y - Ys|| / ||Y|| in fp64."""
+    Y = np.asarray(Y, np.float64)
+    Ys = np.asarray(Ys, np.float64)
     return float(np.linalg.norm(Y - Ys) / np.linalg.norm(Y))
+
+
+def identity_residual(X: np.ndarray, W: np.ndarray, s: np.ndarray) -> float:
+    """[KWKR] 2.1: Y = X W^T = (X diag(s)^-1)(W diag(s))^T; relative residual in fp64."""
+    Xs, Ws = smooth_operands(X, W, s)
+    Y = np.asarray(X, np.float64) @ np.asarray(W, np.float64).T
+    return rel_residual(Y, Xs @ Ws.T)
 
 
 # --------------------------------------------------------------------------

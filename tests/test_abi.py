@@ -113,7 +113,6 @@ def _alphas(*v):
     ("sq_sse_f16", (_A, _A, 0, _A, None), 0),
     ("sq_gemm_s32", (_A, _A, 4, 32, 64, None, None), 1),
     ("sq_gemm_s32", (_A, _A, 4, 32, 64, _U, None), 3),
-    ("sq_linear_w8a8_noalloc", (_A, _A, 128, 32768, 4096, _A, 1, _A, None, 2, _A, None), 2),   # M*N above the array
     ("sq_linear_w8a8_noalloc", (_A, _A, 4, 32, 64, _A, 3, _A, None, 2, _A, None), 1),          # unknown mode
     ("sq_calib_absmax", (_A, 1, 0, 64, 64, _A, None), 0),
 ])
@@ -139,3 +138,16 @@ def test_alpha_search_validation():
     assert lib.sq_alpha_search(_A, _A, 512, 256, 512, _A, _A, _alphas(0.25, 0.5), 2, _A, 16,
                                ctypes.byref(best), None, None) == 6          # workspace too small
 
+
+
+def test_noalloc_refuses_oversize_before_launch():
+    """With the cluster split off (hook 2) the decode-size shape shares tiles
+    through the fixed array; hook 4 makes the size check assume a 64 KiB
+    array, which that schedule's partial sums do not fit."""
+    import w8a8_post_quantization_calib_b200 as sq
+    lib = sq.lib()
+    lib.sq_debug_inject(2 | 4)
+    try:
+        assert lib.sq_linear_w8a8_noalloc(_A, _A, 16, 4096, 11008, _A, 1, _A, None, 2, _A, None) == 2
+    finally:
+        lib.sq_debug_inject(0)

@@ -188,8 +188,10 @@ def test_alpha_search_13b_full():
     wm_r = oracle.calib_absmax(wl.w, F16)
     assert bits_equal(host(am), am_r) and bits_equal(host(wm), wm_r)
     best_r, mses_r, _ = oracle.alpha_search(held, wl.w, am_r, wm_r)
-    # the reference product is accumulated in fp32 on the tensor cores and in fp64 in the oracle
-    assert rel_err(mses, mses_r).max() < 1e-2
+    # the reference product is accumulated in fp32 on the tensor cores and in fp64 in the
+    # oracle, and s may differ in its last bit: one-ulp fp16 changes on a small fraction of
+    # the 7.1 M outputs, with no common sign (see test_gpu_paths.test_alpha_search_whole)
+    assert rel_err(mses, mses_r).max() < 1e-4
     assert best == best_r
     assert mses[list(oracle.ALPHA_GRID).index(best)] <= min(mses[0], mses[-1])
     # full-size run at the chosen alpha

@@ -7,8 +7,9 @@ synchronisation).  It takes no workspace: its small-M split-K path keeps the
 partial sums in a fixed array inside the library.  This file checks, through
 the C ABI, that it returns exactly what the workspace-taking entry point
 returns, on two calls in a row (the second call finds the first call's
-leftovers in the shared array), and that oversize requests are refused
-before any launch.  It is named so that pytest collects it last.
+leftovers in the shared array), after a call of another shape and after a
+call that timed out, and that oversize requests are refused before any
+launch.  It is named so that pytest collects it last.
 """
 import ctypes
 
@@ -91,9 +92,18 @@ def test_noalloc_matches_workspace_entry_point(M, N, K, mode, out_dt, with_bias,
 
 
 def test_noalloc_back_to_back_different_shapes(_hook):
-    """A smaller call after a larger one must not see the larger call's leftovers."""
-    big = _operands(64, 8192, 4096, 1, 2, 1)
-    small = _operands(16, 1024, 4096, 1, 2, 2)
+    """A smaller call after a larger one must not see the larger call's leftovers.
+
+    With the cluster split off both shapes share weight tiles between CTAs,
+    i.e. both go through the library's array (the workspace entry point asks
+    for a workspace exactly when its schedule shares tiles, and the no-alloc
+    entry point runs the same schedule)."""
+    big = _operands(32, 8192, 4096, 1, 2, 1)          # 64 weight tiles, 32-token tile
+    small = _operands(16, 1024, 4096, 1, 2, 2)        # 8 weight tiles
+    if _hook == 2:
+        for ops in (big, small):
+            M, N, K = ops[0].shape[0], ops[1].shape[0], ops[0].shape[1]
+            assert sq.lib().sq_linear_workspace_size(M, N, K) > 0
     outs = []
     for ops in (big, small, big):
         xq, wq, a, ws, _ = ops
@@ -108,18 +118,55 @@ def test_noalloc_back_to_back_different_shapes(_hook):
 
 
 def test_noalloc_rejects_oversize_without_launch():
-    cap = sq.lib().sq_linear_w8a8_noalloc_max_elems()
-    assert cap == 2 ** 21
-    M, K = 128, 64
-    N = (cap // M) + 16                 # M*N just above the fixed array
-    N -= N % 16
-    while M * N <= cap:
-        N += 16
-    xq = torch.zeros(M, K, dtype=torch.int8, device="cuda")
-    wq = torch.zeros(N, K, dtype=torch.int8, device="cuda")
-    a = torch.ones(1, dtype=torch.float32, device="cuda")
-    ws = torch.ones(N, dtype=torch.float32, device="cuda")
-    y = torch.full((M, N), 7.0, dtype=torch.float16, device="cuda")
-    assert _call_noalloc(xq, wq, a, 0, ws, None, y) == 2            # SQ_ERR_UNSUPPORTED
+    """A request whose tile-sharing schedule needs more partial-sum slots than
+    the array holds is refused before anything runs.  No B200 request is that
+    large (one 128 x 16 int32 slot per CTA, 148 CTAs: 1.2 MB here), so the
+    test hook 4 makes the size check assume a 64 KiB array."""
+    assert sq.lib().sq_linear_w8a8_noalloc_max_elems() == 2 ** 21
+    M, N, K = 16, 4096, 11008
+    xq, wq, a, ws, _ = _operands(M, N, K, 1, 1, 5)
+    sq.lib().sq_debug_inject(2 | 4)
+    try:
+        assert sq.lib().sq_linear_workspace_size(M, N, K) > 64 * 1024    # the schedule shares tiles
+        y = torch.full((M, N), 7.0, dtype=torch.float16, device="cuda")
+        assert _call_noalloc(xq, wq, a, 1, ws, None, y) == 2             # SQ_ERR_UNSUPPORTED
+        assert sq.sync_status() == 0
+        assert torch.all(y == 7.0)                                        # nothing was launched
+        # a shape whose schedule keeps its partial sums on chip is never refused,
+        # whatever its size (M*N here is 2.5 M values)
+        M2, N2, K2 = 128, 20480, 256
+        xq2, wq2, a2, ws2, _ = _operands(M2, N2, K2, 0, 2, 6)
+        assert sq.lib().sq_linear_workspace_size(M2, N2, K2) == 0
+        y_ref = torch.empty(M2, N2, dtype=torch.bfloat16, device="cuda")
+        assert _call_with_workspace(xq2, wq2, a2, 0, ws2, None, y_ref) == 0
+        y2 = torch.full((M2, N2), float("nan"), dtype=torch.bfloat16, device="cuda")
+        assert _call_noalloc(xq2, wq2, a2, 0, ws2, None, y2) == 0
+        assert sq.sync_status() == 0
+        assert torch.equal(y2.view(torch.int16), y_ref.view(torch.int16))
+    finally:
+        sq.lib().sq_debug_inject(0)
+
+
+def test_noalloc_after_a_timed_out_call():
+    """A call whose bounded wait ran out leaves tile counters raised in the
+    array; the next call clears the counters it uses and is exact again."""
+    M, N, K = 16, 4096, 11008
+    xq, wq, a, ws, _ = _operands(M, N, K, 1, 2, 9)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
     assert sq.sync_status() == 0
-    assert torch.all(y == 7.0)                                        # nothing was launched
+    sq.set_wait_timeout_ns(20_000_000)                  # 20 ms per barrier wait
+    sq.lib().sq_debug_inject(1 | 2)                     # withheld stage, stream-K schedule
+    try:
+        assert sq.lib().sq_linear_workspace_size(M, N, K) > 0
+        assert _call_noalloc(xq, wq, a, 1, ws, None, y) == 0           # launches; gives up inside
+        assert sq.sync_status() == 5                                    # SQ_ERR_TIMEOUT
+        sq.lib().sq_debug_inject(2)
+        y_ref = torch.empty_like(y)
+        assert _call_with_workspace(xq, wq, a, 1, ws, None, y_ref) == 0
+        y.fill_(float("nan"))
+        assert _call_noalloc(xq, wq, a, 1, ws, None, y) == 0
+        assert sq.sync_status() == 0
+        assert torch.equal(y.view(torch.int16), y_ref.view(torch.int16))
+    finally:
+        sq.lib().sq_debug_inject(0)
+        sq.set_wait_timeout_ns(0)

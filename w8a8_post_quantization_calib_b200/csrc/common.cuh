@@ -75,6 +75,37 @@ __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d)
 }
 
 // ---------------------------------------------------------------------------
+// FP8 (E4M3) codes for the FP8 variant of the layer (aiunderstanding.org,
+// "SmoothQuant 和激活量化": the smoothing carries over to FP8 tensor cores).
+// E4M3: 1 sign, 4 exponent bits (bias 7), 3 mantissa bits, largest finite
+// value 448.  The conversion rounds to nearest even and saturates magnitudes
+// beyond the largest finite value to +-448 (satfinite); the scale of a row or
+// tensor maps its absmax to 448.
+// ---------------------------------------------------------------------------
+constexpr float E4M3_MAX = 448.0f;
+
+// codes of (lo, hi) as two bytes: lo in bits 0..7, hi in bits 8..15
+__device__ __forceinline__ uint32_t e4m3x2_bits(float lo, float hi)
+{
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// four codes packed into one word (byte 0 = a)
+__device__ __forceinline__ uint32_t e4m3x4_bits(float a, float b, float c, float d)
+{
+    return e4m3x2_bits(a, b) | (e4m3x2_bits(c, d) << 16);
+}
+
+// the absmax scale of the code format: fl(m / 127) for INT8, fl(m / 448) for E4M3
+template <bool F8>
+__device__ __forceinline__ float scale_from_absmax_q(float m)
+{
+    return F8 ? __fdiv_rn(m, E4M3_MAX) : __fdiv_rn(m, 127.0f);
+}
+
+// ---------------------------------------------------------------------------
 // 16-byte vectors: EPV elements of dtype DT, widened exactly to fp32.
 // ---------------------------------------------------------------------------
 template <int DT> struct VecT { static constexpr int EPV = 16 / dtype_size(DT); };

@@ -36,7 +36,7 @@
 namespace sq {
 namespace gemm {
 
-enum Kind : int { KIND_I8 = 0, KIND_F16 = 1 };
+enum Kind : int { KIND_I8 = 0, KIND_F16 = 1, KIND_F8 = 2 };   // F8: E4M3 x E4M3 -> fp32
 enum Epi : int { EPI_DEQUANT = 0, EPI_S32 = 1, EPI_GATEUP = 2, EPI_F16 = 3 };
 
 constexpr int BM = 128;            // MMA M: rows of the A operand per tile
@@ -89,7 +89,7 @@ struct Params {
     const void *bias;          // [N] of out_dt or null
     void *out;                 // [M, N] (gate/up: h [M, N/2] or null)
     int out_dt;
-    int32_t *ws_acc;           // swap path: partial-sum slots [2 * sk_ctas][BN][BM]
+    int32_t *ws_acc;           // swap path: partial-sum slots [sk_ctas][BN][BM] (one per CTA, slot blockIdx.x)
     int *ws_cnt;               // swap path: arrival counters [tiles]
     const float *s2;           // gate/up: smoothing of h [N/2]
     const float *a2;           // gate/up: static scale of h [1]
@@ -168,6 +168,12 @@ __device__ __forceinline__ float dequant(int32_t acc, float c, const void *bias,
 {
     const float af = __int2float_rn(acc);
     return bias != nullptr ? __fmaf_rn(af, c, b) : __fmul_rn(af, c);
+}
+
+// The same epilogue on an fp32 accumulator (the FP8 GEMM).
+__device__ __forceinline__ float dequant_f(float acc, float c, const void *bias, float b)
+{
+    return bias != nullptr ? __fmaf_rn(acc, c, b) : __fmul_rn(acc, c);
 }
 
 // ---------------------------------------------------------------------------
@@ -756,8 +762,12 @@ __device__ __forceinline__ void epilogue_tma(const Params &p, const CUtensorMap 
                     const float ws[4] = {w4.x, w4.y, w4.z, w4.w};
                     const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
-                    for (int t = 0; t < 4; ++t)
-                        v[i + t] = dequant(static_cast<int32_t>(r[i + t]), __fmul_rn(am, ws[t]), p.bias, bb[t]);
+                    for (int t = 0; t < 4; ++t) {
+                        if constexpr (KIND == KIND_F8)
+                            v[i + t] = dequant_f(__uint_as_float(r[i + t]), __fmul_rn(am, ws[t]), p.bias, bb[t]);
+                        else
+                            v[i + t] = dequant(static_cast<int32_t>(r[i + t]), __fmul_rn(am, ws[t]), p.bias, bb[t]);
+                    }
                 }
             }
             const int odt = (EPI == EPI_F16) ? DT_F16 : p.out_dt;
@@ -859,8 +869,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 {
     using C = PairCfg<BN, KBO>;
     constexpr int S = C::STAGES;
-    constexpr int BKE = (KIND == KIND_I8) ? BKB : BKB / 2;
-    constexpr uint32_t IDESC = (KIND == KIND_I8) ? ptx::idesc_i8_m256(BN) : ptx::idesc_f16_m256(BN);
+    constexpr int BKE = (KIND == KIND_F16) ? BKB / 2 : BKB;          // K elements per 128-byte block
+    constexpr uint32_t IDESC = (KIND == KIND_I8)    ? ptx::idesc_i8_m256(BN)
+                               : (KIND == KIND_F8) ? ptx::idesc_e4m3_m256(BN)
+                                                   : ptx::idesc_f16_m256(BN);
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -987,6 +999,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                             const uint32_t acc = (kb > 0 || j > 0 || k > 0) ? 1u : 0u;
                             if constexpr (KIND == KIND_I8)
                                 ptx::mma_i8_pair(d, ad + 2 * k, bd + 2 * k, IDESC, acc);
+                            else if constexpr (KIND == KIND_F8)
+                                ptx::mma_f8_pair(d, ad + 2 * k, bd + 2 * k, IDESC, acc);
                             else
                                 ptx::mma_f16_pair(d, ad + 2 * k, bd + 2 * k, IDESC, acc);
                         }

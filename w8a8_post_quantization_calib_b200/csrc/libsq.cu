@@ -263,7 +263,7 @@ sq_status launch_gemm2(gemm::Params p, const void *a, const void *b, cudaStream_
         if (!make_map(&ma, a, f16, p.K, p.rows_a, gemm::BM)) return SQ_ERR_CUDA;
         if (!make_map(&mb, b, f16, p.K, p.rows_b, BN / 2)) return SQ_ERR_CUDA;
     } else {
-        static_assert(KIND == gemm::KIND_I8, "3D operand maps are int8");
+        static_assert(KIND != gemm::KIND_F16, "3D operand maps are of 1-byte elements");
         if (!make_map3(&ma, a, p.K, p.rows_a, gemm::BM, KBO)) return SQ_ERR_CUDA;
         if (!make_map3(&mb, b, p.K, p.rows_b, BN / 2, KBO)) return SQ_ERR_CUDA;
     }
@@ -342,7 +342,7 @@ sq_status dispatch_pair(gemm::Params &p, const void *a, const void *b, cudaStrea
 {
     const int bn = force_bn ? force_bn : pick_pair_bn(p.M, p.N);
     fill_tiles_pair(p, bn, KIND == gemm::KIND_F16 ? 2 : 1);
-    if constexpr (KIND == gemm::KIND_I8) {
+    if constexpr (KIND != gemm::KIND_F16) {
         // two K blocks per TMA load: 3 stages of 56 KB (192-wide) hold the
         // same 6 blocks as 6 single-block stages with half the loads; the
         // 256-wide tile fits 3 stages of 64 KB with one epilogue staging
@@ -431,7 +431,7 @@ size_t ws_bytes(int64_t M, int64_t N, int64_t K)
 // Measured on the MLP-7B 32-tile projection against the stream-K schedule
 // (whose combine goes through global memory): 14.1 -> 12.2 us at M = 1,
 // 15.1 -> 13.4 at M = 16, 25.3 -> 19.2 at M = 64, 34.3 -> 28.0 at M = 128.
-// sq_debug_inject bit 1 turns it off (tests of the other schedules).
+// sq_debug_inject(2) turns it off (tests of the other schedules).
 int swap_cluster_split(int64_t M, int64_t N, int64_t K)
 {
     if (g_inject & 2) return 1;
@@ -477,9 +477,10 @@ sq_status dispatch_swap(gemm::Params &p, const int8_t *xq, const int8_t *wq, cud
 }
 
 // ------------------------------------------------------------------ row kernels
-template <int DT, int MODE>
+template <int DT, int MODEF>
 sq_status launch_rows_dt(RowArgs a, cudaStream_t st)
 {
+    constexpr int MODE = MODEF & ROW_MODE_MASK;     // MODEF may carry ROW_FP8
     constexpr int EPV = VecT<DT>::EPV;
     const bool vec = aligned16(a.src0) && (a.src1 == nullptr || aligned16(a.src1)) &&
                      (a.out == nullptr || aligned16(a.out)) && (a.K % EPV) == 0 &&
@@ -513,7 +514,7 @@ sq_status launch_rows_dt(RowArgs a, cudaStream_t st)
         for (int c = 2; c <= 8; c *= 2)
             if (nvec % c == 0 && nvec / c <= ROW_T) { cs = c; break; }
         if (cs > 0) {
-            const cudaError_t e = launch_pdl_cluster(k_rows_split<DT, MODE>,
+            const cudaError_t e = launch_pdl_cluster(k_rows_split<DT, MODEF>,
                                                      dim3(static_cast<unsigned>(cs), static_cast<unsigned>(a.rows)),
                                                      dim3(ROW_T), static_cast<unsigned>(cs), st, a);
             if (e != cudaSuccess) return cuda_fail(e);
@@ -526,38 +527,38 @@ sq_status launch_rows_dt(RowArgs a, cudaStream_t st)
             if (ring) {
                 if (nt == 128) {
                     if constexpr (MODE == ROW_RMS_STAT) {
-                        if (vpt <= 1) kern = k_rows<DT, 1, MODE, 128, true>;
-                        else if (vpt <= 2) kern = k_rows<DT, 2, MODE, 128, true>;
-                        else kern = k_rows<DT, 4, MODE, 128, true>;
+                        if (vpt <= 1) kern = k_rows<DT, 1, MODEF, 128, true>;
+                        else if (vpt <= 2) kern = k_rows<DT, 2, MODEF, 128, true>;
+                        else kern = k_rows<DT, 4, MODEF, 128, true>;
                     }
                 } else if (vpt <= 1) {
-                    kern = k_rows<DT, 1, MODE, ROW_T, true>;
+                    kern = k_rows<DT, 1, MODEF, ROW_T, true>;
                 } else if (vpt <= 2) {
-                    kern = k_rows<DT, 2, MODE, ROW_T, true>;
+                    kern = k_rows<DT, 2, MODEF, ROW_T, true>;
                 } else if (vpt <= 4) {
-                    kern = k_rows<DT, 4, MODE, ROW_T, true>;
+                    kern = k_rows<DT, 4, MODEF, ROW_T, true>;
                 } else {
-                    kern = k_rows<DT, (DT == DT_F32 ? 8 : 4), MODE, ROW_T, true>;
+                    kern = k_rows<DT, (DT == DT_F32 ? 8 : 4), MODEF, ROW_T, true>;
                 }
             }
         }
         if (kern != nullptr) {
         } else if (nt == 128) {
-            if (vpt <= 1) kern = k_rows<DT, 1, MODE, 128>;
-            else if (vpt <= 2) kern = k_rows<DT, 2, MODE, 128>;
-            else kern = k_rows<DT, 4, MODE, 128>;
+            if (vpt <= 1) kern = k_rows<DT, 1, MODEF, 128>;
+            else if (vpt <= 2) kern = k_rows<DT, 2, MODEF, 128>;
+            else kern = k_rows<DT, 4, MODEF, 128>;
         } else if (vpt <= 1) {
-            kern = k_rows<DT, 1, MODE, ROW_T>;
+            kern = k_rows<DT, 1, MODEF, ROW_T>;
         } else if (vpt <= 2) {
-            kern = k_rows<DT, 2, MODE, ROW_T>;
+            kern = k_rows<DT, 2, MODEF, ROW_T>;
         } else if constexpr (MODE == ROW_RMS_STAT) {
-            kern = k_rows<DT, (DT == DT_F32 ? 8 : 4), MODE, ROW_T>;
+            kern = k_rows<DT, (DT == DT_F32 ? 8 : 4), MODEF, ROW_T>;
         } else if (vpt <= 4) {
-            kern = k_rows<DT, 4, MODE, ROW_T>;
+            kern = k_rows<DT, 4, MODEF, ROW_T>;
         } else if (vpt <= 8) {
-            kern = k_rows<DT, 8, MODE, ROW_T>;
+            kern = k_rows<DT, 8, MODEF, ROW_T>;
         } else {
-            kern = k_rows<DT, 16, MODE, ROW_T>;
+            kern = k_rows<DT, 16, MODEF, ROW_T>;
         }
         cudaError_t e = cudaSuccess;
         if (smem > 0) {       // with the kernel's static shared memory it may pass the 48 KB default
@@ -590,7 +591,7 @@ sq_status launch_rows_dt(RowArgs a, cudaStream_t st)
         if (e != cudaSuccess) return cuda_fail(e);
     } else {
         const int64_t grid = std::min<int64_t>(a.rows, static_cast<int64_t>(sms) * 8);
-        const cudaError_t e = launch_pdl(k_rows_scalar<MODE>, dim3(static_cast<unsigned>(grid)), dim3(ROW_T), 0, st,
+        const cudaError_t e = launch_pdl(k_rows_scalar<MODEF>, dim3(static_cast<unsigned>(grid)), dim3(ROW_T), 0, st,
                                          a, static_cast<int>(DT));
         if (e != cudaSuccess) return cuda_fail(e);
     }
@@ -620,6 +621,9 @@ sq_status launch_rows(RowArgs a, int dt, cudaStream_t st)
 // ---------------------------------------------------------------------------
 constexpr size_t kNoAllocAccBytes = size_t(8) << 20;            // int32 partial sums
 constexpr size_t kNoAllocCntBytes = size_t(64) << 10;           // int32 tile counters
+// sq_debug_inject(4): the partial-sum capacity the size check assumes, so
+// that tests reach the rejection (the whole array is always allocated)
+constexpr size_t kNoAllocTestCapBytes = size_t(64) << 10;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocAccBytes + kNoAllocCntBytes];
 
 namespace {
@@ -671,7 +675,7 @@ int sq_last_cuda_error(void) { return t_last_cuda_error; }
 
 void sq_set_wait_timeout_ns(unsigned long long ns) { g_timeout_ns = ns > 0 ? ns : 2000000000ull; }
 
-void sq_debug_inject(int what) { g_inject = what & 3; }
+void sq_debug_inject(int what) { g_inject = what & 7; }
 
 sq_status sq_sync_status(sq_stream stream)
 {
@@ -734,8 +738,8 @@ sq_status sq_calib_absmax(const void *x, sq_dtype dt, int64_t rows, int64_t cols
     return check_launch();
 }
 
-sq_status sq_smooth_scales(const float *act_max, const float *w_max, int64_t K, float alpha, float *s,
-                           float *a_static, sq_stream stream)
+static sq_status smooth_scales_q(const float *act_max, const float *w_max, int64_t K, float alpha, float *s,
+                                 float *a_static, float qmax, sq_stream stream)
 {
     if (act_max == nullptr || w_max == nullptr || s == nullptr || K <= 0) return SQ_ERR_INVALID_ARG;
     if (!(alpha >= 0.0f && alpha <= 1.0f)) return SQ_ERR_INVALID_ARG;
@@ -743,7 +747,7 @@ sq_status sq_smooth_scales(const float *act_max, const float *w_max, int64_t K, 
     if (K <= 8 * 1024) {    // one cluster of 8 CTAs writes the static scale itself (no pre-zeroing)
         const int threads = static_cast<int>(std::min<int64_t>(1024, ((cdiv(K, 8) + 31) / 32) * 32));
         const cudaError_t e = launch_pdl(k_smooth_scales_cluster, dim3(8), dim3(threads), 0, st, act_max, w_max,
-                                         static_cast<int>(K), alpha, s, a_static);
+                                         static_cast<int>(K), alpha, s, a_static, qmax);
         return e == cudaSuccess ? check_launch() : cuda_fail(e);
     }
     if (a_static != nullptr) {
@@ -753,13 +757,27 @@ sq_status sq_smooth_scales(const float *act_max, const float *w_max, int64_t K, 
     // one channel per thread: the fp64 log2/exp2 chain is latency-bound
     const int64_t grid = std::max<int64_t>(2, cdiv(K, 128));
     const cudaError_t e = launch_pdl(k_smooth_scales, dim3(static_cast<unsigned>(grid)), dim3(128), 0, st, act_max,
-                                     w_max, K, alpha, s, a_static);
+                                     w_max, K, alpha, s, a_static, qmax);
     if (e != cudaSuccess) return cuda_fail(e);
     return check_launch();
 }
 
-sq_status sq_quant_weight(const void *w, sq_dtype dt, int64_t N, int64_t K, const float *s, int8_t *wq,
-                          float *w_scale, sq_stream stream)
+sq_status sq_smooth_scales(const float *act_max, const float *w_max, int64_t K, float alpha, float *s,
+                           float *a_static, sq_stream stream)
+{
+    return smooth_scales_q(act_max, w_max, K, alpha, s, a_static, 127.0f, stream);
+}
+
+sq_status sq_smooth_scales_fp8(const float *act_max, const float *w_max, int64_t K, float alpha, float *s,
+                               float *a_static, sq_stream stream)
+{
+    return smooth_scales_q(act_max, w_max, K, alpha, s, a_static, E4M3_MAX, stream);
+}
+
+extern "C++" {
+template <int FMT>
+static sq_status quant_weight_impl(const void *w, sq_dtype dt, int64_t N, int64_t K, const float *s, int8_t *wq,
+                                   float *w_scale, sq_stream stream)
 {
     if (w == nullptr || s == nullptr || wq == nullptr || w_scale == nullptr || !valid_dt(dt)) return SQ_ERR_INVALID_ARG;
     if (N < 0 || K <= 0) return SQ_ERR_INVALID_ARG;
@@ -772,7 +790,20 @@ sq_status sq_quant_weight(const void *w, sq_dtype dt, int64_t N, int64_t K, cons
     a.s = s;
     a.scale_out = w_scale;
     a.out = wq;
-    return launch_rows<ROW_WEIGHT>(a, dt, as_stream(stream));
+    return launch_rows<ROW_WEIGHT | FMT>(a, dt, as_stream(stream));
+}
+}  // extern "C++"
+
+sq_status sq_quant_weight(const void *w, sq_dtype dt, int64_t N, int64_t K, const float *s, int8_t *wq,
+                          float *w_scale, sq_stream stream)
+{
+    return quant_weight_impl<0>(w, dt, N, K, s, wq, w_scale, stream);
+}
+
+sq_status sq_quant_weight_fp8(const void *w, sq_dtype dt, int64_t N, int64_t K, const float *s, uint8_t *wq8,
+                              float *w_scale, sq_stream stream)
+{
+    return quant_weight_impl<ROW_FP8>(w, dt, N, K, s, reinterpret_cast<int8_t *>(wq8), w_scale, stream);
 }
 
 sq_status sq_quant_weight_gateup(const void *w_gate, const void *w_up, sq_dtype dt, int64_t N_h, int64_t K,
@@ -795,9 +826,12 @@ sq_status sq_quant_weight_gateup(const void *w_gate, const void *w_up, sq_dtype 
     return launch_rows<ROW_WEIGHT>(a, dt, as_stream(stream));
 }
 
-sq_status sq_smooth_quant_act(const void *x, sq_dtype dt, int64_t M, int64_t K, const float *s, sq_act_mode mode,
-                              float *a_scale, int8_t *xq, sq_stream stream)
+extern "C++" {
+template <int FMT>
+static sq_status smooth_quant_act_impl(const void *x, sq_dtype dt, int64_t M, int64_t K, const float *s,
+                                       sq_act_mode mode, float *a_scale, int8_t *xq, sq_stream stream)
 {
+    constexpr bool F8 = FMT != 0;
     if (x == nullptr || s == nullptr || a_scale == nullptr || xq == nullptr || !valid_dt(dt)) return SQ_ERR_INVALID_ARG;
     if (M < 0 || K <= 0 || (mode != SQ_ACT_STATIC && mode != SQ_ACT_PER_TOKEN)) return SQ_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(xq)) return SQ_ERR_MISALIGNED;
@@ -828,22 +862,39 @@ sq_status sq_smooth_quant_act(const void *x, sq_dtype dt, int64_t M, int64_t K, 
             auto go = [&](auto kern) { return launch_pdl(kern, grid, block, 0, st, xb, M, nvec, s, a_scale, slab, xq); };
             cudaError_t e;
             if (dt == SQ_F32)
-                e = big ? go(k_quant_static<DT_F32, true, false>)
-                        : one ? go(k_quant_static<DT_F32, false, true>) : go(k_quant_static<DT_F32, false, false>);
+                e = big ? go(k_quant_static<DT_F32, true, false, F8>)
+                        : one ? go(k_quant_static<DT_F32, false, true, F8>)
+                              : go(k_quant_static<DT_F32, false, false, F8>);
             else if (dt == SQ_F16)
-                e = big ? go(k_quant_static<DT_F16, true, false>)
-                        : one ? go(k_quant_static<DT_F16, false, true>) : go(k_quant_static<DT_F16, false, false>);
+                e = big ? go(k_quant_static<DT_F16, true, false, F8>)
+                        : one ? go(k_quant_static<DT_F16, false, true, F8>)
+                              : go(k_quant_static<DT_F16, false, false, F8>);
             else
-                e = big ? go(k_quant_static<DT_BF16, true, false>)
-                        : one ? go(k_quant_static<DT_BF16, false, true>) : go(k_quant_static<DT_BF16, false, false>);
+                e = big ? go(k_quant_static<DT_BF16, true, false, F8>)
+                        : one ? go(k_quant_static<DT_BF16, false, true, F8>)
+                              : go(k_quant_static<DT_BF16, false, false, F8>);
             if (e != cudaSuccess) return cuda_fail(e);
             return check_launch();
         }
-        return launch_rows<ROW_ACT_STATIC>(a, dt, as_stream(stream));
+        return launch_rows<ROW_ACT_STATIC | FMT>(a, dt, as_stream(stream));
     }
     a.scale_out = a_scale;
-    return launch_rows<ROW_ACT_TOKEN>(a, dt, as_stream(stream));
+    return launch_rows<ROW_ACT_TOKEN | FMT>(a, dt, as_stream(stream));
 }
+}  // extern "C++"
+
+sq_status sq_smooth_quant_act(const void *x, sq_dtype dt, int64_t M, int64_t K, const float *s, sq_act_mode mode,
+                              float *a_scale, int8_t *xq, sq_stream stream)
+{
+    return smooth_quant_act_impl<0>(x, dt, M, K, s, mode, a_scale, xq, stream);
+}
+
+sq_status sq_smooth_quant_act_fp8(const void *x, sq_dtype dt, int64_t M, int64_t K, const float *s,
+                                  sq_act_mode mode, float *a_scale, uint8_t *xq8, sq_stream stream)
+{
+    return smooth_quant_act_impl<ROW_FP8>(x, dt, M, K, s, mode, a_scale, reinterpret_cast<int8_t *>(xq8), stream);
+}
+
 
 sq_status sq_rmsnorm_quant(const void *x, sq_dtype dt, int64_t M, int64_t d, const float *gamma, const float *s,
                            float eps, const float *a_scale, int8_t *xq, float *rstd, sq_stream stream)
@@ -934,6 +985,29 @@ sq_status sq_linear_w8a8(const int8_t *xq, const int8_t *wq, int64_t M, int64_t 
     return dispatch_pair<gemm::KIND_I8, gemm::EPI_DEQUANT>(p, xq, wq, st);
 }
 
+sq_status sq_linear_fp8(const uint8_t *xq8, const uint8_t *wq8, int64_t M, int64_t N, int64_t K,
+                        const float *a_scale, sq_act_mode mode, const float *w_scale, const void *bias,
+                        sq_dtype out_dt, void *y, sq_stream stream)
+{
+    sq_status r = check_gemm_shape(reinterpret_cast<const int8_t *>(xq8), reinterpret_cast<const int8_t *>(wq8), M,
+                                   N, K);
+    if (r != SQ_OK) return r;
+    if (a_scale == nullptr || w_scale == nullptr || y == nullptr || !valid_dt(out_dt)) return SQ_ERR_INVALID_ARG;
+    if (mode != SQ_ACT_STATIC && mode != SQ_ACT_PER_TOKEN) return SQ_ERR_INVALID_ARG;
+    if (!aligned16(y) || !aligned16(w_scale)) return SQ_ERR_MISALIGNED;
+    gemm::Params p{};
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(N);
+    p.K = static_cast<int>(K);
+    p.a_scale = a_scale;
+    p.per_token = (mode == SQ_ACT_PER_TOKEN) ? 1 : 0;
+    p.w_scale = w_scale;
+    p.bias = bias;
+    p.out = y;
+    p.out_dt = out_dt;
+    return dispatch_pair<gemm::KIND_F8, gemm::EPI_DEQUANT>(p, xq8, wq8, as_stream(stream));
+}
+
 size_t sq_linear_w8a8_noalloc_max_elems(void) { return kNoAllocAccBytes / 4; }
 
 sq_status sq_linear_w8a8_noalloc(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, int64_t K,
@@ -947,37 +1021,6 @@ sq_status sq_linear_w8a8_noalloc(const int8_t *xq, const int8_t *wq, int64_t M, 
     if (!aligned16(y) || !aligned16(w_scale)) return SQ_ERR_MISALIGNED;
     if (M > kSwapMaxM)      // the large-M path needs no scratch: same launch as sq_linear_w8a8
         return sq_linear_w8a8(xq, wq, M, N, K, a_scale, mode, w_scale, bias, out_dt, y, nullptr, 0, stream);
-    const size_t mn_bytes = static_cast<size_t>(M * N) * 4;
-    const size_t cnt_bytes = static_cast<size_t>(swap_tiles(M, N)) * 4;
-    if (mn_bytes > kNoAllocAccBytes || cnt_bytes > kNoAllocCntBytes) return SQ_ERR_UNSUPPORTED;
-    if (const int cs = swap_cluster_split(M, N, K); cs > 1) {   // partial sums stay on chip: no scratch
-        gemm::Params p{};
-        p.M = static_cast<int>(M);
-        p.N = static_cast<int>(N);
-        p.K = static_cast<int>(K);
-        p.a_scale = a_scale;
-        p.per_token = (mode == SQ_ACT_PER_TOKEN) ? 1 : 0;
-        p.w_scale = w_scale;
-        p.bias = bias;
-        p.out = y;
-        p.out_dt = out_dt;
-        return dispatch_swap<gemm::EPI_DEQUANT>(p, xq, wq, as_stream(stream), swap_tiles(M, N), cs);
-    }
-    // as many stream-K CTAs as the fixed array holds partial-sum slots for
-    const int64_t g = swap_grid(M, N, K, kNoAllocAccBytes);
-    const bool shared = g != swap_tiles(M, N);
-    void *scratch = nullptr;
-    if ((r = noalloc_scratch(&scratch)) != SQ_OK) return r;
-    int32_t *acc = static_cast<int32_t *>(scratch);
-    int *cnt = reinterpret_cast<int *>(static_cast<unsigned char *>(scratch) + kNoAllocAccBytes);
-    const cudaStream_t st = as_stream(stream);
-    // the array keeps whatever the previous call left: the per-tile arrival
-    // counters must start at zero (a partial-sum slot is always written
-    // before it is read)
-    if (shared) {
-        cudaError_t e = cudaMemsetAsync(cnt, 0, cnt_bytes, st);
-        if (e != cudaSuccess) return cuda_fail(e);
-    }
     gemm::Params p{};
     p.M = static_cast<int>(M);
     p.N = static_cast<int>(N);
@@ -988,8 +1031,27 @@ sq_status sq_linear_w8a8_noalloc(const int8_t *xq, const int8_t *wq, int64_t M, 
     p.bias = bias;
     p.out = y;
     p.out_dt = out_dt;
-    p.ws_acc = shared ? acc : nullptr;
-    p.ws_cnt = shared ? cnt : nullptr;
+    const cudaStream_t st = as_stream(stream);
+    const int64_t tiles = swap_tiles(M, N);
+    if (const int cs = swap_cluster_split(M, N, K); cs > 1)   // partial sums stay on chip: no scratch
+        return dispatch_swap<gemm::EPI_DEQUANT>(p, xq, wq, st, tiles, cs);
+    // the stream-K schedule of sq_linear_w8a8 (same CTAs, same partial sums):
+    // it is the only schedule that needs scratch, and only when tiles are shared
+    const int64_t g = swap_grid(M, N, K, SIZE_MAX);
+    if (g == tiles) return dispatch_swap<gemm::EPI_DEQUANT>(p, xq, wq, st, tiles);
+    const size_t acc_cap = (g_inject & 4) ? kNoAllocTestCapBytes : kNoAllocAccBytes;
+    const size_t cnt_bytes = static_cast<size_t>(tiles) * 4;
+    if (swap_slot_bytes(M, g) > acc_cap || cnt_bytes > kNoAllocCntBytes) return SQ_ERR_UNSUPPORTED;
+    void *scratch = nullptr;
+    if ((r = noalloc_scratch(&scratch)) != SQ_OK) return r;
+    int *cnt = reinterpret_cast<int *>(static_cast<unsigned char *>(scratch) + kNoAllocAccBytes);
+    // the array keeps whatever the previous call left (a call that timed out
+    // leaves its counters raised): the per-tile arrival counters must start at
+    // zero; a partial-sum slot is always written before it is read
+    cudaError_t e = cudaMemsetAsync(cnt, 0, cnt_bytes, st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    p.ws_acc = static_cast<int32_t *>(scratch);
+    p.ws_cnt = cnt;
     return dispatch_swap<gemm::EPI_DEQUANT>(p, xq, wq, st, g);
 }
 

@@ -432,6 +432,18 @@ __device__ __forceinline__ void mma_f16_pair(uint32_t d_tmem, uint64_t adesc, ui
         : "memory");
 }
 
+// FP8 pair MMA: E4M3 x E4M3 -> fp32 (kind::f8f6f4, 32 bytes of K per instruction)
+__device__ __forceinline__ void mma_f8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Instruction descriptors for the pair MMA (M = 256).
 __host__ __device__ constexpr uint32_t idesc_i8_m256(int n)
 {
@@ -442,6 +454,14 @@ __host__ __device__ constexpr uint32_t idesc_i8_m256(int n)
 __host__ __device__ constexpr uint32_t idesc_f16_m256(int n)
 {
     return (1u << 4) | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(256 >> 4) << 24);
+}
+
+// kind::f8f6f4: D fp32 (bits 4-5 = 1), A and B E4M3 (format code 0 in bits
+// 7-9 and 10-12), both K-major, N >> 3 at bit 17, M >> 4 at bit 24
+__host__ __device__ constexpr uint32_t idesc_e4m3_m256(int n)
+{
+    return (1u << 4) | (0u << 7) | (0u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
+           (static_cast<uint32_t>(256 >> 4) << 24);
 }
 
 }  // namespace ptx

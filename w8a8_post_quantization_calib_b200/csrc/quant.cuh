@@ -21,10 +21,11 @@ namespace sq {
 // s_j = max(a_j,1e-5)^alpha / max(w_j,1e-5)^(1-alpha) in fp64, rounded once
 // (kwkr.cn blog 2.2; aiunderstanding.org technical insight; "010. SmoothQuant
 // Integration" context step 1; the 1e-5 clamp follows tbr8.org's example).
-// Optionally a_static = fl(max_j fl(act_max_j * recip(s_j)) / 127), the closed
-// form of "010. SmoothQuant Integration" key design point 1.  x -> fl(x/127)
-// is monotone, so max_b fl(m_b/127) = fl(max_b m_b / 127): blocks combine
-// with atomicMax on the (non-negative) float bits; *a_static is zeroed first.
+// Optionally a_static = fl(max_j fl(act_max_j * recip(s_j)) / qmax), the closed
+// form of "010. SmoothQuant Integration" key design point 1 (qmax = 127 for
+// INT8 codes, 448 for E4M3).  x -> fl(x/qmax) is monotone, so max_b
+// fl(m_b/qmax) = fl(max_b m_b / qmax): blocks combine with atomicMax on the
+// (non-negative) float bits; *a_static is zeroed first.
 // A single-block launch (small K) writes the scale directly.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float smoothing_factor(float act_max, float w_max, double al)
@@ -43,7 +44,7 @@ __device__ __forceinline__ float smoothing_factor(float act_max, float w_max, do
 // scale, so no pre-zeroing and no atomics are needed.
 __global__ void __cluster_dims__(8, 1, 1) __launch_bounds__(1024)
     k_smooth_scales_cluster(const float *__restrict__ act_max, const float *__restrict__ w_max, int K, float alpha,
-                            float *__restrict__ s, float *__restrict__ a_static)
+                            float *__restrict__ s, float *__restrict__ a_static, float qmax)
 {
     __shared__ float red[32];
     __shared__ float cta_max;
@@ -68,7 +69,7 @@ __global__ void __cluster_dims__(8, 1, 1) __launch_bounds__(1024)
             asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
         }
         v = warp_max(v);
-        if (threadIdx.x == 0) *a_static = scale_from_absmax(v);
+        if (threadIdx.x == 0) *a_static = __fdiv_rn(v, qmax);
     }
     // no CTA leaves while CTA 0 may still read its shared memory
     asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
@@ -76,7 +77,7 @@ __global__ void __cluster_dims__(8, 1, 1) __launch_bounds__(1024)
 
 __global__ void __launch_bounds__(1024)
     k_smooth_scales(const float *__restrict__ act_max, const float *__restrict__ w_max, int64_t K,
-                    float alpha, float *__restrict__ s, float *__restrict__ a_static)
+                    float alpha, float *__restrict__ s, float *__restrict__ a_static, float qmax)
 {
     __shared__ float red[32];
     const double al = static_cast<double>(alpha);
@@ -92,8 +93,8 @@ __global__ void __launch_bounds__(1024)
     if (a_static != nullptr) {
         m = block_max(m, red);
         if (threadIdx.x == 0) {
-            if (gridDim.x == 1) *a_static = scale_from_absmax(m);      // one block: no pre-zeroing needed
-            else atomicMax(reinterpret_cast<int *>(a_static), __float_as_int(scale_from_absmax(m)));
+            if (gridDim.x == 1) *a_static = __fdiv_rn(m, qmax);      // one block: no pre-zeroing needed
+            else atomicMax(reinterpret_cast<int *>(a_static), __float_as_int(__fdiv_rn(m, qmax)));
         }
     }
 }
@@ -108,6 +109,10 @@ enum RowMode : int {
     ROW_RMSNORM = 3,     // y = fl(fl(x*r)*fl(gamma_j*fl(1/s_j))); codes with the given scale
     ROW_RMS_STAT = 4     // running column max of |fl(fl(x*r)*gamma_j)| into scale_out[K] (no codes)
 };
+// Added to ROW_WEIGHT / ROW_ACT_STATIC / ROW_ACT_TOKEN: E4M3 codes and
+// absmax / 448 scales instead of INT8 codes and absmax / 127.
+constexpr int ROW_FP8 = 8;
+constexpr int ROW_MODE_MASK = 7;
 
 constexpr int ROW_T = 256;
 constexpr int RMS_CL = 8;          // cluster of the norm-output statistic (see k_rows)
@@ -135,11 +140,20 @@ constexpr unsigned ERR_ROW_RING = 0x150;
 
 // Codes of EPV values (already multiplied by the scale reciprocal) -> global.
 // INRANGE: the values come from a per-row scale and cannot saturate.
-template <int EPV, bool INRANGE = false>
+template <int EPV, bool INRANGE = false, bool F8 = false>
 __device__ __forceinline__ void store_codes(int8_t *dst_row, int64_t v, const float *f)
 {
     auto q = [](float x) { return INRANGE ? quant8_bits_inrange(x) : quant8_bits(x); };
-    if constexpr (EPV == 8) {
+    if constexpr (F8) {
+        if constexpr (EPV == 8) {
+            uint2 o;
+            o.x = e4m3x4_bits(f[0], f[1], f[2], f[3]);
+            o.y = e4m3x4_bits(f[4], f[5], f[6], f[7]);
+            *reinterpret_cast<uint2 *>(dst_row + v * 8) = o;
+        } else {
+            *reinterpret_cast<uint32_t *>(dst_row + v * 4) = e4m3x4_bits(f[0], f[1], f[2], f[3]);
+        }
+    } else if constexpr (EPV == 8) {
         uint2 o;
         o.x = pack4_bits(q(f[0]), q(f[1]), q(f[2]), q(f[3]));
         o.y = pack4_bits(q(f[4]), q(f[5]), q(f[6]), q(f[7]));
@@ -200,9 +214,11 @@ __device__ __forceinline__ bool constants_aligned16(const RowArgs &p)
 // registers, which the row's block reduction barrier guarantees.  The waits
 // are bounded: on expiry the kernel records the error and finishes on
 // whatever data it has (no thread leaves early, so no barrier is left short).
-template <int DT, int VPT, int MODE, int NT, bool RING = false>
+template <int DT, int VPT, int MODEF, int NT, bool RING = false>
 __global__ void __launch_bounds__(NT) k_rows(RowArgs p)
 {
+    constexpr int MODE = MODEF & ROW_MODE_MASK;
+    constexpr bool F8 = (MODEF & ROW_FP8) != 0;
     constexpr int EPV = VecT<DT>::EPV;
     constexpr bool REG = (VPT * EPV <= 32);
     static_assert(!RING || (REG && MODE != ROW_ACT_STATIC), "the row ring needs register rows and a row barrier");
@@ -405,7 +421,7 @@ __global__ void __launch_bounds__(NT) k_rows(RowArgs p)
                 colc(i, v, c);
 #pragma unroll
                 for (int e = 0; e < EPV; ++e) f[e] = __fmul_rn(__fmul_rn(f[e], c[e]), inv_a_static);
-                if (v < nvec) store_codes<EPV>(dst, v, f);
+                if (v < nvec) store_codes<EPV, false, F8>(dst, v, f);
             }
             continue;
         }
@@ -477,7 +493,7 @@ __global__ void __launch_bounds__(NT) k_rows(RowArgs p)
                 if constexpr (REG) ykeep[i][e] = y;
             }
         }
-        const float sc = scale_from_absmax(block_max(mx, red));
+        const float sc = scale_from_absmax_q<F8>(block_max(mx, red));
         ring_refill();
         const float inv = recip_or_zero(sc);
         if (tid == 0) p.scale_out[row] = sc;
@@ -498,7 +514,8 @@ __global__ void __launch_bounds__(NT) k_rows(RowArgs p)
                 for (int e = 0; e < EPV; ++e) f[e] = __fmul_rn(__fmul_rn(f[e], c[e]), inv);
             }
             if (v < nvec) {
-                if (inrange) store_codes<EPV, true>(dst, v, f);
+                if (F8) store_codes<EPV, false, F8>(dst, v, f);
+                else if (inrange) store_codes<EPV, true>(dst, v, f);
                 else store_codes<EPV, false>(dst, v, f);
             }
         }
@@ -561,7 +578,7 @@ constexpr int QS_TX = 32, QS_TY = 8, QS_UNROLL = 4;
 // ONE: every slab is at most one batch (QS_UNROLL x QS_TY rows), so no
 // second batch buffer is kept (fewer registers, more blocks resident: small
 // tensors are latency-bound).
-template <int DT, bool STREAM, bool ONE>
+template <int DT, bool STREAM, bool ONE, bool F8 = false>
 __global__ void __launch_bounds__(QS_TX *QS_TY)
     k_quant_static(const uint8_t *__restrict__ x, int64_t rows, int64_t nvec, const float *__restrict__ s,
                    const float *__restrict__ a_in, int64_t row_slab, int8_t *__restrict__ out)
@@ -606,7 +623,14 @@ __global__ void __launch_bounds__(QS_TX *QS_TY)
 #pragma unroll
         for (int e = 0; e < EPV; ++e) f[e] = __fmul_rn(__fmul_rn(f[e], c[e]), inv_a);
         int8_t *dst = out + row * K;
-        if constexpr (EPV == 8) {
+        if constexpr (F8) {
+            if constexpr (EPV == 8) {
+                __stcs(reinterpret_cast<uint2 *>(dst + v * 8), make_uint2(e4m3x4_bits(f[0], f[1], f[2], f[3]),
+                                                                          e4m3x4_bits(f[4], f[5], f[6], f[7])));
+            } else {
+                __stcs(reinterpret_cast<uint32_t *>(dst + v * 4), e4m3x4_bits(f[0], f[1], f[2], f[3]));
+            }
+        } else if constexpr (EPV == 8) {
             uint2 o;
             o.x = pack4_bits(quant8_bits(f[0]), quant8_bits(f[1]), quant8_bits(f[2]), quant8_bits(f[3]));
             o.y = pack4_bits(quant8_bits(f[4]), quant8_bits(f[5]), quant8_bits(f[6]), quant8_bits(f[7]));
@@ -653,9 +677,11 @@ __device__ __forceinline__ double ld_dsmem_f64(uint32_t addr)
     return v;
 }
 
-template <int DT, int MODE>
+template <int DT, int MODEF>
 __global__ void __launch_bounds__(ROW_T) k_rows_split(RowArgs p)
 {
+    constexpr int MODE = MODEF & ROW_MODE_MASK;
+    constexpr bool F8 = (MODEF & ROW_FP8) != 0;
     constexpr int EPV = VecT<DT>::EPV;
     __shared__ float red[32];
     __shared__ double red64[32];
@@ -723,7 +749,7 @@ __global__ void __launch_bounds__(ROW_T) k_rows_split(RowArgs p)
             const float inv_a = recip_or_zero(p.a_in[0]);
 #pragma unroll
             for (int e = 0; e < EPV; ++e) f[e] = __fmul_rn(__fmul_rn(f[e], c[e]), inv_a);
-            store_codes<EPV>(dst, v, f);
+            store_codes<EPV, false, F8>(dst, v, f);
         }
     } else if constexpr (MODE == ROW_RMSNORM || MODE == ROW_RMS_STAT) {
         double ss = 0.0;
@@ -757,13 +783,14 @@ __global__ void __launch_bounds__(ROW_T) k_rows_split(RowArgs p)
             mx = fmaxf(mx, fabsf(f[e]));
         }
         const float rmax = static_cast<float>(cluster_combine(static_cast<double>(block_max(mx, red)), true));
-        const float sc = scale_from_absmax(rmax);
+        const float sc = scale_from_absmax_q<F8>(rmax);
         const float inv = recip_or_zero(sc);
         if (rank == 0 && tid == 0) p.scale_out[row] = sc;
         if (act) {
 #pragma unroll
             for (int e = 0; e < EPV; ++e) f[e] = __fmul_rn(f[e], inv);
-            if ((sc == 0.0f) || (sc >= 1.17549435e-38f)) store_codes<EPV, true>(dst, v, f);
+            if (F8) store_codes<EPV, false, F8>(dst, v, f);
+            else if ((sc == 0.0f) || (sc >= 1.17549435e-38f)) store_codes<EPV, true>(dst, v, f);
             else store_codes<EPV, false>(dst, v, f);
         }
     }
@@ -771,9 +798,11 @@ __global__ void __launch_bounds__(ROW_T) k_rows_split(RowArgs p)
 
 // Unaligned / very wide rows: one block per row, elementwise, two passes
 // over global memory (correct for any K; not tuned).
-template <int MODE>
+template <int MODEF>
 __global__ void __launch_bounds__(ROW_T) k_rows_scalar(RowArgs p, int dt)
 {
+    constexpr int MODE = MODEF & ROW_MODE_MASK;
+    constexpr bool F8 = (MODEF & ROW_FP8) != 0;
     __shared__ float red[32];
     __shared__ double red64[32];
     const int tid = threadIdx.x;
@@ -815,7 +844,7 @@ __global__ void __launch_bounds__(ROW_T) k_rows_scalar(RowArgs p, int dt)
             mul_a = inv_a_static;
             if (tid == 0 && p.rstd_out != nullptr) p.rstd_out[row] = r_m;
         } else {
-            const float sc = scale_from_absmax(block_max(stat, red));
+            const float sc = scale_from_absmax_q<F8>(block_max(stat, red));
             mul_a = recip_or_zero(sc);
             if (tid == 0) p.scale_out[row] = sc;
         }
@@ -826,6 +855,8 @@ __global__ void __launch_bounds__(ROW_T) k_rows_scalar(RowArgs p, int dt)
             else y = __fmul_rn(x, colc(j));
             if constexpr (MODE == ROW_RMS_STAT)
                 atomicMax(reinterpret_cast<int *>(p.scale_out + j), __float_as_int(fabsf(y)));
+            else if constexpr (F8)
+                p.out[row * p.K + j] = static_cast<int8_t>(e4m3x2_bits(__fmul_rn(y, mul_a), 0.0f) & 0xffu);
             else
                 p.out[row * p.K + j] = static_cast<int8_t>(quant8(__fmul_rn(y, mul_a)));
         }
