@@ -35,6 +35,7 @@ Parity pins (tests/test_oracle_pins.py; tests/golden/ fixtures):
                            to +-448 beyond (torch gives NaN there)
   fp8 quantisers        -- the row maximum maps to +-448; every code within
                            half an E4M3 spacing of its value
+  static_scale_fp8      -- brute force over every smoothed calibration value
   gemm_fp8_f64          -- exact: equals the int64 matmul of the codes'
                            values scaled by 2^9
   fold_into_previous    -- fp64 identity (X Wp'^T)(W diag(s))^T == (X Wp^T) W^T,
@@ -359,6 +360,13 @@ def smooth_quant_act_fp8(x: np.ndarray, s: np.ndarray, mode: int, a_scale=None, 
         return e4m3_encode((xs * inv).astype(np.float32)), a
     a = (np.abs(xs).max(axis=1) / np.float32(E4M3_MAX)).astype(np.float32)
     return e4m3_encode((xs * _recip32(a)[:, None]).astype(np.float32)), a
+
+
+def static_scale_fp8(act_max: np.ndarray, s: np.ndarray) -> np.float32:
+    """Closed-form per-tensor scale for E4M3 codes ([ADR10] key design point 1
+    with 448 in place of 127): fl(max_j fl(act_max_j * fl(1/s_j)) / 448)."""
+    m = (_f32(act_max) * _recip32(s)).astype(np.float32).max()
+    return np.float32(np.float32(m) / np.float32(E4M3_MAX))
 
 
 def quant_weight_fp8(w: np.ndarray, s: np.ndarray, dt: int | None = None):

@@ -115,6 +115,14 @@ def _alphas(*v):
     ("sq_gemm_s32", (_A, _A, 4, 32, 64, _U, None), 3),
     ("sq_linear_w8a8_noalloc", (_A, _A, 4, 32, 64, _A, 3, _A, None, 2, _A, None), 1),          # unknown mode
     ("sq_calib_absmax", (_A, 1, 0, 64, 64, _A, None), 0),
+    ("sq_smooth_scales_fp8", (_A, _A, 64, 1.5, _A, None, None), 1),           # alpha outside [0, 1]
+    ("sq_quant_weight_fp8", (_U, 1, 8, 64, _A, _A, _A, None), 3),
+    ("sq_quant_weight_fp8", (_A, 7, 8, 64, _A, _A, _A, None), 1),               # unknown dtype
+    ("sq_smooth_quant_act_fp8", (_A, 1, 4, 64, _A, 2, _A, _A, None), 1),        # unknown mode
+    ("sq_smooth_quant_act_fp8", (_A, 1, 4, 64, _A, 1, _A, _U, None), 3),
+    ("sq_linear_fp8", (_A, _A, 4, 40, 64, _A, 0, _A, None, 1, _A, None), 1),    # N % 16
+    ("sq_linear_fp8", (_A, _A, 4, 32, 64, _A, 0, _A, None, 1, _U, None), 3),
+    ("sq_linear_fp8", (_A, _A, 0, 32, 64, _A, 0, _A, None, 1, _A, None), 1),    # M = 0
 ])
 def test_every_entry_point_validates_before_launch(fn, args, status):
     import w8a8_post_quantization_calib_b200 as sq

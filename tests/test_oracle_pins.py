@@ -687,6 +687,25 @@ def test_fp8_quantisers_map_the_row_max_to_448():
     assert np.abs(oracle.e4m3_decode(qs)).max() == 448.0
 
 
+def test_static_scale_fp8_equals_brute_force():
+    """The FP8 closed form max_j(act_max_j / s_j) / 448 equals the largest
+    smoothed calibration value / 448 (fl() is monotone), bit for bit; the E4M3
+    code of that value at this scale is 448 (0x7E)."""
+    wl = synth.outlier_linear(M=16, K=256, N=64, calib_batches=3, calib_rows=32, x_dt=F16, w_dt=F16,
+                              out_dt=F16, workload=93)
+    am = np.zeros(wl.K, np.float32)
+    for b in wl.calib:
+        oracle.calib_absmax(b, F16, am)
+    s = oracle.smooth_scales(am, oracle.calib_absmax(wl.w, F16), 0.5)
+    a8 = oracle.static_scale_fp8(am, s)
+    inv_s = np.where(s > 0, np.float32(1) / s, np.float32(0)).astype(np.float32)
+    brute = max(float(np.abs((oracle.to_f32(b, F16) * inv_s[None, :]).astype(np.float32)).max()) for b in wl.calib)
+    assert a8 == np.float32(np.float32(brute) / np.float32(448.0))
+    assert np.float32(a8 * np.float32(448.0)) / np.float32(brute) == pytest.approx(1.0, abs=2 ** -22)
+    q, _ = oracle.smooth_quant_act_fp8(np.concatenate(wl.calib), s, STATIC, a8, F16)
+    assert (q & 0x7F).max() == 0x7E and oracle.e4m3_decode(np.array([0x7E], np.uint8))[0] == 448.0
+
+
 def test_gemm_fp8_f64_is_exact():
     """E4M3 values are multiples of 2^-9, so their products scaled by 2^18 are
     integers: the int64 matmul of the codes' values times 2^9 is the exact sum."""

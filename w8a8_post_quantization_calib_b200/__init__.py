@@ -12,7 +12,9 @@ library raises ``ImportError`` (build it with
 Names follow the C ABI: ``calib_absmax``, ``smooth_scales``,
 ``quant_weight``, ``smooth_quant_act``, ``linear_w8a8`` (+ ``gemm_s32``,
 ``quant_weight_gateup``, ``rmsnorm_quant``, ``linear_w8a8_gateup_silu``,
-``gemm_f16_ref``, ``sse_f16``, ``alpha_search``).
+``gemm_f16_ref``, ``sse_f16``, ``alpha_search``) and the FP8 (E4M3) variant
+``smooth_scales_fp8``, ``quant_weight_fp8``, ``smooth_quant_act_fp8``,
+``linear_fp8`` (codes are uint8 tensors holding E4M3 bit patterns).
 """
 from __future__ import annotations
 
@@ -38,6 +40,7 @@ EXPORTS = (
     "sq_linear_w8a8_noalloc", "sq_linear_w8a8_noalloc_max_elems",
     "sq_gemm_s32", "sq_linear_w8a8_gateup_silu", "sq_gemm_f16_ref", "sq_sse_f16",
     "sq_alpha_search_workspace_size", "sq_alpha_search",
+    "sq_smooth_scales_fp8", "sq_quant_weight_fp8", "sq_smooth_quant_act_fp8", "sq_linear_fp8",
 )
 
 
@@ -79,6 +82,10 @@ def _load() -> ctypes.CDLL:
         "sq_sse_f16": (I, [P, P, I64, P, P]),
         "sq_alpha_search_workspace_size": (SZ, [I64, I64, I64, I]),
         "sq_alpha_search": (I, [P, P, I64, I64, I64, P, P, P, I, P, SZ, P, P, P]),
+        "sq_smooth_scales_fp8": (I, [P, P, I64, F, P, P, P]),
+        "sq_quant_weight_fp8": (I, [P, I, I64, I64, P, P, P, P]),
+        "sq_smooth_quant_act_fp8": (I, [P, I, I64, I64, P, I, P, P, P]),
+        "sq_linear_fp8": (I, [P, P, I64, I64, I64, P, I, P, P, I, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -282,3 +289,34 @@ def alpha_search(x_held, w, act_max, w_max, workspace, alphas=ALPHA_GRID, stream
         _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
         ctypes.byref(best), mse, _stream(stream)))
     return float(best.value), [float(v) for v in mse]
+
+
+# ---------------------------------------------------------------- FP8 (E4M3) variant
+def smooth_scales_fp8(act_max, w_max, alpha: float, s, a_static=None, stream=None) -> None:
+    K = act_max.numel()
+    _check("sq_smooth_scales_fp8", _lib.sq_smooth_scales_fp8(
+        _dev(act_max, "act_max", torch.float32), _dev(w_max, "w_max", torch.float32), K, float(alpha),
+        _dev(s, "s", torch.float32), _dev(a_static, "a_static", torch.float32), _stream(stream)))
+
+
+def quant_weight_fp8(w, s, wq8, w_scale, stream=None) -> None:
+    N, K = w.shape
+    _check("sq_quant_weight_fp8", _lib.sq_quant_weight_fp8(
+        _dev(w, "w"), _dt(w), N, K, _dev(s, "s", torch.float32), _dev(wq8, "wq8", torch.uint8),
+        _dev(w_scale, "w_scale", torch.float32), _stream(stream)))
+
+
+def smooth_quant_act_fp8(x, s, mode: int, a_scale, xq8, stream=None) -> None:
+    M, K = x.shape
+    _check("sq_smooth_quant_act_fp8", _lib.sq_smooth_quant_act_fp8(
+        _dev(x, "x"), _dt(x), M, K, _dev(s, "s", torch.float32), int(mode),
+        _dev(a_scale, "a_scale", torch.float32), _dev(xq8, "xq8", torch.uint8), _stream(stream)))
+
+
+def linear_fp8(xq8, wq8, a_scale, mode: int, w_scale, y, bias=None, stream=None) -> None:
+    M, K = xq8.shape
+    N = wq8.shape[0]
+    _check("sq_linear_fp8", _lib.sq_linear_fp8(
+        _dev(xq8, "xq8", torch.uint8), _dev(wq8, "wq8", torch.uint8), M, N, K,
+        _dev(a_scale, "a_scale", torch.float32), int(mode), _dev(w_scale, "w_scale", torch.float32),
+        _dev(bias, "bias", y.dtype) if bias is not None else None, _dt(y), _dev(y, "y"), _stream(stream)))
