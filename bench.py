@@ -1,24 +1,31 @@
 #!/usr/bin/env python3
-"""Benchmark of the SmoothQuant W8A8 linear layer on B200.
+"""Benchmark of the SmoothQuant W8A8 layer on B200.
 
-Workload: a Llama-7B-shaped QKV projection (K=4096 in, N=12288 out, M=2048
-runtime tokens, fp16 activations and weights with 0.5% seeded outlier
-channels x U(20,100), W ~ N(0, 0.02^2)), calibrated on 64 batches of 512
-tokens, alpha=0.5, per-tensor static activation scale, per-row weight scale,
-fp16 output.  Synthetic, seeded inputs.
+Bench line (default, ``--workload mlp70b``): the 70B-shaped decoder MLP
+block, the largest single-GPU workload.  Inputs: bf16 X [16384, 8192]
+(runtime tokens) and 8 x 2048 calibration tokens, both N(0,1) with 41
+seeded outlier channels x U(20,100); W_gate, W_up [28672, 8192] and W_down
+[8192, 28672] ~ N(0, 0.02^2) bf16; RMSNorm gain 1, eps 1e-5; alpha 0.5.
+Synthetic, seeded.
 
 One step = the whole hot path over one batch, all through the C ABI:
-  calibration absmax over the 32768 calibration tokens (one launch) ->
-  weight column absmax -> smoothing factors + closed-form static scale ->
-  weight transform + per-row INT8 -> runtime smooth + INT8 quant of X ->
-  tcgen05 INT8 GEMM with the fp16 dequant epilogue.
-Under torchrun (N>1) each rank calibrates its own 64 x 512 token shard and
-runs its own runtime batch (weak scaling); the per-channel maxima are
-combined with one NCCL all-reduce(MAX) of K floats before the smoothing
-factors -- the only exchange the method has.
+  calibration statistic of the normalised input over the 16384
+  calibration tokens -> weight column statistics of W_gate, W_up -> smoothing
+  factors + static scale -> gate/up weight transform + per-row INT8 ->
+  calibration forward (RMSNorm + quant -> gate/up GEMM with SiLU*mul -> h)
+  and the statistic of h -> weight statistic of W_down -> smoothing factors
+  + static scale of h -> down weight transform -> runtime block:
+  RMSNorm with 1/s folded into its gain + INT8 quant -> gate/up GEMM with the
+  SiLU*mul epilogue and the smooth + requant of h -> down GEMM -> bf16 Y.
+Under torchrun (N>1) each rank calibrates on its own token shard and runs its
+own runtime tokens (weak scaling); the two per-channel statistics are
+combined with one NCCL all-reduce(MAX) each, the only exchanges the method
+has.
 
-Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle
-instead, on a bounded sample of the same workload.
+``--workload qkv7b`` prints the same kind of line for the Llama-7B QKV
+projection; the other workloads print per-kernel measurements.  Prints one
+JSON line (rank 0).  ``--impl reference`` times the CPU oracle instead, on a
+bounded sample of the same workload.
 """
 from __future__ import annotations
 
@@ -30,20 +37,23 @@ import statistics
 import sys
 import threading
 import time
+from dataclasses import dataclass, field
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "W8A8 linear INT8 TOPS & tokens/s at 1 B200; % of INT8 peak / HBM GB/s"
-WORKLOAD = ("Llama-7B QKV projection: K=4096, N=12288, M=2048 tokens, fp16 X/W with 0.5% outlier "
-            "channels, 64x512 calibration tokens, alpha=0.5, static per-tensor act scale, per-row "
-            "weight scale, fp16 out")
-M_TOK, K_IN, N_OUT, CALIB_B, CALIB_R = 2048, 4096, 12288, 64, 512
-ALPHA = 0.5
+LINES = ("mlp70b", "qkv7b")
+MLP70B_DESC = ("70B decoder MLP block: RMSNorm(d=8192, 1/s folded into the gain) + INT8 quant -> gate/up GEMM "
+               "K=8192, N=2x28672 + SiLU*mul + smooth/requant -> down GEMM K=28672, N=8192; M=16384 tokens, "
+               "8x2048 calibration tokens (h statistic from the calibration forward), alpha=0.5, static "
+               "per-tensor act scales, per-row weight scales, bf16 in/out, outlier channels")
+QKV_DESC = ("Llama-7B QKV projection: K=4096, N=12288, M=2048 tokens, fp16 X/W with 0.5% outlier channels, "
+            "64x512 calibration tokens, alpha=0.5, static per-tensor act scale, per-row weight scale, fp16 out")
 
 
 def peaks():
-    """Measured roofline denominators (generated file) or the recipe's fallback."""
+    """Measured HBM and bf16 denominators (generated file) or the recipe's fallback."""
     src = "measured"
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -51,21 +61,44 @@ def peaks():
         hbm, bf16, bf16_s = float(mp["hbm_gbs"]), float(mp["bf16_tflops"]), float(mp["bf16_tflops_sustained"])
     except Exception:
         hbm, bf16, bf16_s, src = 6650.0, 1590.0, 1400.0, "fallback"
-    # INT8 dense tensor peak = measured bf16 x the nominal dense ratio 4.5 / 2.25
-    return {"hbm_gbs": hbm, "int8_tops": bf16 * 2.0, "int8_tops_sustained": bf16_s * 2.0, "source": src}
+    return {"hbm_gbs": hbm, "bf16_tflops": bf16, "bf16_tflops_sustained": bf16_s, "source": src}
 
 
-def gemm_traffic():
-    """DRAM bytes per GEMM launch from the committed ncu summary, or None when the
-    kernel source changed after the counters were taken."""
+def tensor_peak(kind: str = "i8", clk=None) -> dict:
+    """Dense tensor-core peak measured on this GPU now (libsq_peak: the GEMM
+    mainloop on shared-memory operands): one ~100 ms launch (burst) and ~2 s of
+    back-to-back launches (sustained), with the SM clock sampled over each."""
+    from w8a8_post_quantization_calib_b200 import peak
+    out = {"kind": kind}
+    for name, kw in (("burst", {"ms": 100.0}), ("sustained", {"ms": 100.0, "seconds": 2.0})):
+        if clk is not None:
+            clk.begin()
+        r = peak.measure(kind, **kw)
+        if clk is not None:
+            clk.end()
+            c = clk.summary()
+            r["sm_mhz"] = c["sm_mhz"]
+            r["reasons"] = c["reasons"]
+            if c["sm_mhz"]:
+                r["tops_per_mhz"] = r["tops"] / c["sm_mhz"]
+        out[name] = r
+    return out
+
+
+def traffic_from_profile(name: str, sources=("gemm.cuh", "ptx_sm100.cuh", "libsq.cu")):
+    """DRAM bytes per launch of a kernel from a committed ncu summary
+    (profiles/<name>.json), or None when the kernel source changed after the
+    counters were taken."""
     import hashlib
-    tf = os.path.join(ROOT, "profiles", "linear_w8a8_qkv7b_traffic.json")
+    tf = os.path.join(ROOT, "profiles", name + ".json")
     try:
         d = json.load(open(tf))
         h = hashlib.sha256()
-        for f in ("gemm.cuh", "ptx_sm100.cuh", "libsq.cu"):
+        for f in sources:
             h.update(open(os.path.join(ROOT, "w8a8_post_quantization_calib_b200", "csrc", f), "rb").read())
-        return d["dram_bytes_per_launch"] if h.hexdigest()[:16] == d["source_sha256_16"] else None
+        if h.hexdigest()[:16] != d["source_sha256_16"]:
+            return None
+        return d["dram_bytes_per_launch"] * d.get("scale_to_bench", 1.0)
     except Exception:
         return None
 
@@ -148,14 +181,15 @@ class ClockSampler:
 # --------------------------------------------------------------------------
 # CPU oracle timing (reference arm and cpu_baseline)
 # --------------------------------------------------------------------------
-def oracle_sample(frac: float, wl=None):
-    """Run the oracle's full step on a fraction `frac` of every part of the workload.
+QKV_M, QKV_K, QKV_N, QKV_CB, QKV_CR = 2048, 4096, 12288, 64, 512
 
-    Every part is linear in its row count (calibration rows, weight rows for
-    the statistic and the quantisation, runtime token rows for quantisation
-    and the INT8 GEMM over all N), so step time ~= sample time / frac.
-    Returns (seconds, description).
-    """
+
+def oracle_sample_qkv(frac: float, wl=None):
+    """The oracle's full QKV step on a fraction `frac` of every part of the
+    workload: calibration rows, weight rows (statistic and quantisation),
+    runtime token rows (quantisation and the INT8 GEMM over all N).  Every
+    part is linear in its row count, so step time ~= sample time / frac.
+    Returns (seconds, description)."""
     import numpy as np
     import oracle
     import synth
@@ -163,25 +197,86 @@ def oracle_sample(frac: float, wl=None):
         wl = synth.qkv_7b()
     calib = np.concatenate(wl.calib)
     rc = max(1, int(round(calib.shape[0] * frac)))
-    rw = max(1, int(round(N_OUT * frac)))
-    rx = max(1, int(round(M_TOK * frac)))
+    rw = max(1, int(round(QKV_N * frac)))
+    rx = max(1, int(round(QKV_M * frac)))
     t0 = time.perf_counter()
-    act_max = np.zeros(K_IN, np.float32)
+    act_max = np.zeros(QKV_K, np.float32)
     oracle.calib_absmax(calib[:rc], synth.F16, act_max)
     w_max = oracle.calib_absmax(wl.w[:rw], synth.F16)
-    s = oracle.smooth_scales(act_max, w_max, ALPHA)
+    s = oracle.smooth_scales(act_max, w_max, 0.5)
     a = oracle.static_scale(act_max, s)
     wq, ws = oracle.quant_weight(wl.w[:rw], s, synth.F16)
     xq, av = oracle.smooth_quant_act(wl.x[:rx], s, oracle.STATIC, a, synth.F16)
-    wq_full = np.resize(wq, (N_OUT, K_IN))          # GEMM over all N output channels
-    ws_full = np.resize(ws, N_OUT)
+    wq_full = np.resize(wq, (QKV_N, QKV_K))          # GEMM over all N output channels
+    ws_full = np.resize(ws, QKV_N)
     acc = oracle.gemm_s32(xq, wq_full)
     oracle.dequant(acc, av, oracle.STATIC, ws_full, synth.F16)
     dt = time.perf_counter() - t0
-    desc = (f"oracle full step on a {frac:.4f} fraction of every part: {rc} calibration rows, {rw} weight rows "
-            f"(statistic + quantisation), {rx} runtime tokens (quant + INT8 GEMM over all N={N_OUT}); "
+    desc = (f"oracle QKV step on a {frac:.4f} fraction of every part: {rc} calibration rows, {rw} weight rows "
+            f"(statistic + quantisation), {rx} runtime tokens (quant + INT8 GEMM over all N={QKV_N}); "
             f"step time extrapolated as sample time / fraction")
     return dt, desc
+
+
+def oracle_sample_mlp70b(frac: float, blk=None):
+    """The oracle's full 70B MLP-block step on a fraction `frac` of every part:
+    calibration token rows (norm statistic, calibration forward through the
+    gate/up GEMM over all 2 x 28672 rows, h statistic), weight rows of W_gate,
+    W_up and W_down (statistics and quantisation), runtime token rows
+    (RMSNorm + quant, gate/up GEMM over all rows, SiLU*mul + requant, down GEMM
+    over all 8192 rows).  Step time ~= sample time / frac.  Returns
+    (seconds, description)."""
+    import numpy as np
+    import oracle
+    import synth
+    BF16 = synth.BF16
+    if blk is None:
+        blk = synth.mlp_block_70b()
+    d, f, eps = blk.d, blk.f, blk.eps
+    calib = np.concatenate(blk.calib)
+    rc = max(1, int(round(calib.shape[0] * frac)))
+    rf = max(32, int(round(f * frac)) // 32 * 32)
+    rd = max(1, int(round(d * frac)))
+    rx = max(1, int(round(blk.M * frac)))
+    one = np.array([1.0], np.float32)
+
+    def silu_h(xq, a, wg, wsg, wu, wsu):
+        gv = oracle.dequant_f32(oracle.gemm_s32(xq, wg), np.array([a], np.float32), oracle.STATIC, wsg)
+        uv = oracle.dequant_f32(oracle.gemm_s32(xq, wu), np.array([a], np.float32), oracle.STATIC, wsu)
+        return oracle.silu_mul_bf16(gv, uv)
+
+    t0 = time.perf_counter()
+    am1 = oracle.rmsnorm_absmax(calib[:rc], blk.gamma, eps, BF16)
+    wm1 = oracle.calib_absmax(blk.w_gate[:rf], BF16)
+    oracle.calib_absmax(blk.w_up[:rf], BF16, wm1)
+    s1 = oracle.smooth_scales(am1, wm1, blk.alpha)
+    a1 = oracle.static_scale(am1, s1)
+    wqg, wsg = oracle.quant_weight(blk.w_gate[:rf], s1, BF16)
+    wqu, wsu = oracle.quant_weight(blk.w_up[:rf], s1, BF16)
+    wqg, wsg = np.resize(wqg, (f, d)), np.resize(wsg, f)          # GEMMs over all f rows
+    wqu, wsu = np.resize(wqu, (f, d)), np.resize(wsu, f)
+    xq_c, _ = oracle.rmsnorm_quant(calib[:rc], blk.gamma, s1, eps, a1, BF16)
+    am2 = oracle.calib_absmax(silu_h(xq_c, a1, wqg, wsg, wqu, wsu), BF16)
+    wm2 = oracle.calib_absmax(blk.w_down[:rd], BF16)
+    s2 = oracle.smooth_scales(am2, wm2, blk.alpha)
+    a2 = oracle.static_scale(am2, s2)
+    wqd, wsd = oracle.quant_weight(blk.w_down[:rd], s2, BF16)
+    wqd, wsd = np.resize(wqd, (d, f)), np.resize(wsd, d)
+    xq, _ = oracle.rmsnorm_quant(blk.x[:rx], blk.gamma, s1, eps, a1, BF16)
+    h = silu_h(xq, a1, wqg, wsg, wqu, wsu)
+    hq, _ = oracle.smooth_quant_act(h, s2, oracle.STATIC, a2, BF16)
+    oracle.dequant(oracle.gemm_s32(hq, wqd), np.array([a2], np.float32), oracle.STATIC, wsd, BF16)
+    del one
+    dt = time.perf_counter() - t0
+    desc = (f"oracle 70B MLP-block step on a {frac:.5f} fraction of every part (a subset): {rc} calibration "
+            f"tokens (norm statistic, calibration forward over all {2 * f} gate/up rows, h statistic), "
+            f"{rf}+{rf} gate/up and {rd} down weight rows (statistics + quantisation), {rx} runtime tokens "
+            f"(RMSNorm+quant, gate/up over all rows, SiLU*mul+requant, down over all {d} rows); step time "
+            f"extrapolated as sample time / fraction")
+    return dt, desc
+
+
+ORACLE_SAMPLE = {"mlp70b": oracle_sample_mlp70b, "qkv7b": oracle_sample_qkv}
 
 
 def cpu_cores():
@@ -189,46 +284,42 @@ def cpu_cores():
     return int(n) if n and n.isdigit() else (os.cpu_count() or 1)
 
 
-def run_reference(args):
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
-        return 0
-    import oracle
-    import synth
-    oracle.build()
-    wl = synth.qkv_7b()
-    ops = 2.0 * M_TOK * N_OUT * K_IN
-    # size one step so that warmup + steps stay within ~2 minutes
-    t_probe, _ = oracle_sample(1.0 / 512, wl)
-    budget = 120.0 / max(1, args.steps + args.warmup)
-    frac = min(1.0, max(1.0 / 2048, (1.0 / 512) * budget / max(t_probe, 1e-3)))
-    for _ in range(args.warmup):
-        oracle_sample(frac, wl)
-    times, desc = [], ""
-    for _ in range(args.steps):
-        t, desc = oracle_sample(frac, wl)
-        times.append(t / frac)
-    ms = 1e3 * statistics.mean(times)
-    value = ops / (ms * 1e-3) / 1e12
-    line = {
-        "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": args.gpus, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "s8", "data": "synthetic", "impl": "reference",
-        "config": {"workload": WORKLOAD, "M": M_TOK, "K": K_IN, "N": N_OUT, "calib_tokens": CALIB_B * CALIB_R,
-                   "parallelism": "host cores"},
-        "tokens_per_s": M_TOK / (ms * 1e-3),
-        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": cpu_cores(), "kind": "oracle", "sample": desc},
-        "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-    }
-    print(json.dumps(line), flush=True)
-    return 0
+def oracle_baseline(workload: str, target_s: float, data=None):
+    """Times the oracle on a sample sized for about target_s seconds of CPU
+    work; returns (step seconds extrapolated, description, sample seconds)."""
+    fn = ORACLE_SAMPLE[workload]
+    probe = 1.0 / 1024
+    t_probe, _ = fn(probe, data)
+    frac = min(1.0, max(1.0 / 16384, probe * target_s / max(t_probe, 1e-3)))
+    t, desc = fn(frac, data)
+    return t / frac, desc, t, frac
 
 
 # --------------------------------------------------------------------------
-# GPU arm
+# GPU arm: one bench line
 # --------------------------------------------------------------------------
-def run_gpu(args):
-    import numpy as np
+@dataclass
+class Spec:
+    """What run_line needs from a workload."""
+    workload: str
+    config: dict
+    ops_per_step: float                 # INT8 tensor-core ops of one step (one rank)
+    tokens_per_step: int                # runtime tokens of one step (one rank)
+    names: list                         # kernels of a step, in order
+    step: object                        # step(mark): mark(i) before kernel i, mark(len(names)) after the last
+    dominant: str                       # the kernel the roofline line describes
+    work: dict                          # name -> {"bytes": algorithmic bytes, "ops": ops} per launch
+    solo: dict                          # name -> callable launching that kernel alone (same buffers)
+    e2e_in: list                        # (device tensor, pinned host tensor) copied in each e2e step
+    e2e_out: list                       # (pinned host tensor, device tensor) copied out each e2e step
+    launches_per_step: int
+    launches_note: str
+    traffic: object = None              # callable -> DRAM bytes per launch of the dominant kernel, or None
+    data: object = None                 # host-side workload object (for the oracle baseline)
+    extra: dict = field(default_factory=dict)
+
+
+def run_line(args, build):
     import torch
     import torch.distributed as dist
 
@@ -240,67 +331,15 @@ def run_gpu(args):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-
-    import synth
     import w8a8_post_quantization_calib_b200 as sq
-    from w8a8_post_quantization_calib_b200.dist import allreduce_absmax_
 
+    # a created stream: the library's kernels overlap their launches with
+    # programmatic dependent launch there (not on the default stream)
+    torch.cuda.set_stream(torch.cuda.Stream())
     P = peaks()
-    wl = synth.qkv_7b(shard=rank)
-    dev = torch.device("cuda", local)
-
-    def up(bits, dt=torch.float16):
-        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(dt)
-
-    calib_h = up(np.concatenate(wl.calib)).pin_memory()
-    w_h = up(wl.w).pin_memory()
-    x_h = up(wl.x).pin_memory()
-    calib = calib_h.to(dev)
-    W = w_h.to(dev)
-    X = x_h.to(dev)
-    stats = torch.zeros(2 * K_IN, dtype=torch.float32, device=dev)    # running maxima, zeroed per step
-    act_max, w_max = stats[:K_IN], stats[K_IN:]
-    s = torch.empty(K_IN, dtype=torch.float32, device=dev)
-    a = torch.empty(1, dtype=torch.float32, device=dev)
-    wq = torch.empty(N_OUT, K_IN, dtype=torch.int8, device=dev)
-    ws = torch.empty(N_OUT, dtype=torch.float32, device=dev)
-    xq = torch.empty(M_TOK, K_IN, dtype=torch.int8, device=dev)
-    y = torch.empty(M_TOK, N_OUT, dtype=torch.float16, device=dev)
-    y_h = torch.empty(M_TOK, N_OUT, dtype=torch.float16).pin_memory()
-    stream = torch.cuda.current_stream()
-    names = ["calib_absmax", "weight_absmax", "smooth_scales", "quant_weight", "smooth_quant_act", "linear_w8a8"]
-    if world > 1:
-        names.insert(1, "allreduce_max")
-
-    def step(evs=None):
-        def mark(i):
-            if evs is not None and evs[i] is not None:
-                evs[i].record()          # the current stream: the capture stream while capturing
-        i = 0
-        mark(i)
-        stats.zero_()                      # both running maxima start from zero each step
-        sq.calib_absmax(calib, act_max)
-        i += 1
-        mark(i)
-        if world > 1:
-            allreduce_absmax_(act_max)      # the one exchange: per-channel maxima of all token shards
-            i += 1
-            mark(i)
-        sq.calib_absmax(W, w_max)
-        i += 1
-        mark(i)
-        sq.smooth_scales(act_max, w_max, ALPHA, s, a)
-        i += 1
-        mark(i)
-        sq.quant_weight(W, s, wq, ws)
-        i += 1
-        mark(i)
-        sq.smooth_quant_act(X, s, sq.ACT_STATIC, a, xq)
-        i += 1
-        mark(i)
-        sq.linear_w8a8(xq, wq, a, sq.ACT_STATIC, ws, y)
-        i += 1
-        mark(i)
+    spec = build(args, rank, world)
+    names, nk = spec.names, len(spec.names)
+    steps = args.steps
 
     def barrier():
         if world > 1:
@@ -308,190 +347,396 @@ def run_gpu(args):
         torch.cuda.synchronize()
 
     for _ in range(args.warmup):
-        step()
+        spec.step(lambda i: None)
     if sq.sync_status() != 0:
         raise RuntimeError("kernel error during warm-up")
 
-    # ---- timed region: K steps captured once into a CUDA graph and launched as one
-    # graph.  Inside it, events bracket only each step's GEMM (the dominant kernel, for
-    # the roofline): an event between two kernels serialises them and cancels the
-    # programmatic-launch overlap, so the other kernels are timed in a second pass.
-    nk = len(names)
-    gi = names.index("linear_w8a8")
+    clk = ClockSampler(local).start()
+    # the INT8 dense tensor-core peak of this GPU, measured now
+    barrier()
+    tpk = tensor_peak("i8", clk)
+    barrier()
 
-    def capture(ev_sets):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            for k in range(args.steps):
-                step(ev_sets[k])
-        g.replay()                          # untimed: uploads the graph
-        torch.cuda.synchronize()
-        return g
+    # ---- timed region: the K steps captured once into a CUDA graph and launched
+    # as one graph; events bracket only each step's dominant kernel (an event
+    # between two kernels serialises them and cancels the programmatic-launch
+    # overlap).  The other kernels are timed alone below.
+    gi = names.index(spec.dominant)
 
-    def gemm_only_events():
+    def events_for_dominant():
         e = [None] * (nk + 1)
         e[gi] = torch.cuda.Event(enable_timing=True, external=not args.eager_steps)
         e[gi + 1] = torch.cuda.Event(enable_timing=True, external=not args.eager_steps)
         return e
 
-    ev_t = [gemm_only_events() for _ in range(args.steps)]
+    def run_steps(evsets):
+        for k in range(steps):
+            ev = evsets[k]
+
+            def mark(i, ev=ev):
+                if ev[i] is not None:
+                    ev[i].record()
+            spec.step(mark)
+
+    ev_t = [events_for_dominant() for _ in range(steps)]
     graph = None
     if not args.eager_steps:
         try:
-            graph = capture(ev_t)
-        except Exception as exc:            # noqa: BLE001
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                run_steps(ev_t)
+            graph.replay()                    # untimed: uploads the graph
+            torch.cuda.synchronize()
+        except Exception as exc:              # noqa: BLE001
             print(f"graph capture failed ({exc}); timing eager launches", file=sys.stderr)
             graph = None
             torch.cuda.synchronize()
-            ev_t = [gemm_only_events() for _ in range(args.steps)]
+            ev_t = [events_for_dominant() for _ in range(steps)]
     stream = torch.cuda.current_stream()
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clk = ClockSampler(local).start()
     barrier()
     clk.begin()
     t_start.record(stream)
     if graph is not None:
         graph.replay()
     else:
-        for k in range(args.steps):
-            step(ev_t[k])
+        run_steps(ev_t)
     t_end.record(stream)
     barrier()
     clk.end()
-    clk.stop()
+    clocks = clk.summary()
     st = sq.sync_status()
     if st != 0:
         raise RuntimeError(f"kernel error in the timed region (status {st})")
     ms_total = t_start.elapsed_time(t_end)
-    gemm_ms = statistics.mean(ev_t[k][gi].elapsed_time(ev_t[k][gi + 1]) for k in range(args.steps))
-    ms_step = ms_total / args.steps
+    dom_ms = statistics.mean(ev_t[k][gi].elapsed_time(ev_t[k][gi + 1]) for k in range(steps))
+    ms_step = ms_total / steps
     if world > 1:
-        t = torch.tensor([ms_step], dtype=torch.float64, device=dev)
+        t = torch.tensor([ms_step], dtype=torch.float64, device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_step = float(t.item())
     used_graph = graph is not None
     del graph
 
-    # ---- per-kernel breakdown: the same K steps with an event between every two kernels
-    ext = not args.eager_steps
-    evs = [[torch.cuda.Event(enable_timing=True, external=ext) for _ in range(nk + 1)] for _ in range(args.steps)]
-    g2 = None
-    if used_graph:
-        try:
-            g2 = capture(evs)
-        except Exception:                   # noqa: BLE001
-            g2 = None
-            evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(args.steps)]
-    barrier()
-    t2s, t2e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t2s.record(stream)
-    if g2 is not None:
-        g2.replay()
-    else:
-        for k in range(args.steps):
-            step(evs[k])
-    t2e.record(stream)
-    barrier()
-    ms_step_serial = t2s.elapsed_time(t2e) / args.steps
-    per_kernel = [statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps))
-                  for i in range(nk)]
-    del g2
+    # ---- every kernel alone: back-to-back launches of the same call in one
+    # graph (inputs larger than L2 stream from HBM on every launch)
+    kern = {}
+    for name in names:
+        fn = spec.solo.get(name)
+        if fn is None:
+            continue
+        reps = spec.extra.get("solo_reps", {}).get(name, 10)
+        time.sleep(0.3)        # let the clocks recover from the power cap of the previous measurement
+        ms = _time_ms(fn, reps, warmup=2, graph=not args.eager_steps)
+        v = {"ms": ms}
+        w = spec.work.get(name, {})
+        if "bytes" in w:
+            v["gbs"] = w["bytes"] / (ms * 1e-3) / 1e9
+            v["frac_hbm"] = v["gbs"] / P["hbm_gbs"]
+        if "ops" in w:
+            v["tops"] = w["ops"] / (ms * 1e-3) / 1e12
+            v["frac_int8_peak"] = v["tops"] / tpk["burst"]["tops"]
+        kern[name] = v
+    if sq.sync_status() != 0:
+        raise RuntimeError("kernel error in the per-kernel pass")
 
-    ops = 2.0 * M_TOK * N_OUT * K_IN
-    value = world * ops / (ms_step * 1e-3) / 1e12
-    kt = dict(zip(names, per_kernel))
+    value = world * spec.ops_per_step / (ms_step * 1e-3) / 1e12
+    dw = spec.work[spec.dominant]
+    dom_tops = dw["ops"] / (dom_ms * 1e-3) / 1e12
+    peak_b, peak_s = tpk["burst"]["tops"], tpk["sustained"]["tops"]
+    roofline = {"bound": "tensor", "kernel": spec.dominant, "achieved": dom_tops, "peak": peak_b, "unit": "TOPS",
+                "frac": dom_tops / peak_b, "traffic": spec.traffic() if spec.traffic else None,
+                "launch_us": dom_ms * 1e3, "ops_per_launch": dw["ops"],
+                "peak_note": ("measured on this GPU in this run (libsq_peak: tcgen05 kind::i8 mainloop on "
+                              "shared-memory operands, one ~100 ms launch); vs its ~2 s sustained figure "
+                              f"{peak_s:.0f}: {dom_tops / peak_s:.3f}; vs 2 x the {P['source']} bf16 cuBLAS burst "
+                              f"{2 * P['bf16_tflops']:.0f}: {dom_tops / (2 * P['bf16_tflops']):.3f}; vs the nominal "
+                              f"4500 dense INT8: {dom_tops / 4500.0:.3f}")}
 
-    # algorithmic bytes / ops per launch
-    calib_bytes = CALIB_B * CALIB_R * K_IN * 2
-    kern = {
-        "calib_absmax": {"ms": kt["calib_absmax"], "bytes": calib_bytes},
-        "weight_absmax": {"ms": kt["weight_absmax"], "bytes": N_OUT * K_IN * 2},
-        "smooth_scales": {"ms": kt["smooth_scales"], "bytes": K_IN * 4 * 3},
-        "quant_weight": {"ms": kt["quant_weight"], "bytes": N_OUT * K_IN * 3 + N_OUT * 4},
-        "smooth_quant_act": {"ms": kt["smooth_quant_act"], "bytes": M_TOK * K_IN * 3},
-        "linear_w8a8": {"ms": kt["linear_w8a8"], "ops": ops,
-                        "bytes": M_TOK * K_IN + N_OUT * K_IN + M_TOK * N_OUT * 2 + N_OUT * 4},
-    }
-    for k, v in kern.items():
-        v["share"] = v["ms"] / ms_step_serial
-        if "ops" in v:
-            v["tops"] = v["ops"] / (v["ms"] * 1e-3) / 1e12
-            v["frac_int8_peak"] = v["tops"] / P["int8_tops"]
-        v["gbs"] = v["bytes"] / (v["ms"] * 1e-3) / 1e9
-        v["frac_hbm"] = v["gbs"] / P["hbm_gbs"]
-    if world > 1:
-        kern["allreduce_max"] = {"ms": kt["allreduce_max"], "share": kt["allreduce_max"] / ms_step_serial}
-
-    gemm_tops = ops / (gemm_ms * 1e-3) / 1e12
-    traffic = gemm_traffic()
-    roofline = {"bound": "tensor", "kernel": "linear_w8a8 (tcgen05 kind::i8 GEMM + dequant)",
-                "achieved": gemm_tops, "peak": P["int8_tops"], "unit": "TOPS", "frac": gemm_tops / P["int8_tops"],
-                "launch_us": gemm_ms * 1e3,
-                "traffic": traffic,
-                "peak_note": f"INT8 dense = 2 x {P['source']} bf16 cuBLAS burst (nominal 4.5/2.25 ratio); "
-                             f"vs sustained {P['int8_tops_sustained']:.0f}: {gemm_tops / P['int8_tops_sustained']:.3f}; "
-                             f"vs the nominal 4500 dense INT8: {gemm_tops / 4500.0:.3f}"}
-
-    # ---- end to end: pinned host buffers, H2D of the step's inputs and D2H of the result in the region
-    e2e_steps = max(1, min(args.steps, 5))
-    h2d = calib_h.numel() * 2 + w_h.numel() * 2 + x_h.numel() * 2
-    d2h = y_h.numel() * 2
+    # ---- end to end: pinned host buffers, H2D of the step's inputs and D2H of
+    # the result inside the region
+    e2e_steps = max(1, min(steps, args.e2e_steps))
+    h2d = sum(h.numel() * h.element_size() for _, h in spec.e2e_in)
+    d2h = sum(h.numel() * h.element_size() for h, _ in spec.e2e_out)
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
-        calib.copy_(calib_h, non_blocking=True)
-        W.copy_(w_h, non_blocking=True)
-        X.copy_(x_h, non_blocking=True)
-        step()
-        y_h.copy_(y, non_blocking=True)
+        for dv, hv in spec.e2e_in:
+            dv.copy_(hv, non_blocking=True)
+        spec.step(lambda i: None)
+        for hv, dv in spec.e2e_out:
+            hv.copy_(dv, non_blocking=True)
     e1.record(stream)
     barrier()
     ms_e2e = e0.elapsed_time(e1) / e2e_steps
     if world > 1:
-        t = torch.tensor([ms_e2e], dtype=torch.float64, device=dev)
+        t = torch.tensor([ms_e2e], dtype=torch.float64, device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_e2e = float(t.item())
-    e2e = {"value": world * ops / (ms_e2e * 1e-3) / 1e12, "unit": "TOPS", "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e, "steps": e2e_steps}
+    clk.stop()
+    e2e = {"value": world * spec.ops_per_step / (ms_e2e * 1e-3) / 1e12, "unit": "TOPS",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e, "steps": e2e_steps,
+           "tokens_per_s": world * spec.tokens_per_step / (ms_e2e * 1e-3)}
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
-        frac = args.cpu_frac
-        t, desc = oracle_sample(frac, wl)
-        cpu = {"value": ops / (t / frac) / 1e12, "unit": "TOPS", "cores": cpu_cores(), "kind": "oracle",
-               "sample": desc, "sample_seconds": t}
+        t_step, desc, t_sample, frac = oracle_baseline(spec.workload, args.cpu_seconds, spec.data)
+        cpu = {"value": spec.ops_per_step / t_step / 1e12, "unit": "TOPS", "cores": cpu_cores(), "kind": "oracle",
+               "sample": desc, "sample_seconds": t_sample, "fraction": frac}
 
-    launches_per_step = 6
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+            "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "s8", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "M": M_TOK, "K": K_IN, "N": N_OUT, "calib_tokens": CALIB_B * CALIB_R,
-                       "alpha": ALPHA, "parallelism": f"dp{world} (token shards; all-reduce MAX of act_max)",
-                       "l2": "no flush: every step streams 384 MB of inputs (> 126 MB L2)",
-                       "launch": "K steps as one CUDA graph" if used_graph else "eager"},
-            "tokens_per_s": world * M_TOK / (ms_step * 1e-3),
+            "vs_baseline": None, "dtype": "s8", "data": "synthetic (seeded; shapes and laws of the workload)",
+            "config": dict(spec.config, parallelism=f"dp{world} (token shards; all-reduce MAX of the statistics)",
+                           launch="K steps as one CUDA graph" if used_graph else "eager"),
+            "tokens_per_s": world * spec.tokens_per_step / (ms_step * 1e-3),
             "roofline": roofline,
             "kernels": kern,
-            "kernels_note": "per-kernel times from a second pass of the same K steps with an event between every "
-                            f"two kernels (serialised: {ms_step_serial:.4f} ms/step); the timed region itself has "
-                            "events only around the GEMM, so consecutive kernels overlap their launch "
-                            "(programmatic dependent launch)",
+            "kernels_note": ("each kernel timed alone after a 0.3 s pause: back-to-back launches of the same "
+                             "call captured in one CUDA graph (CUDA events), fractions of the measured HBM copy / "
+                             "of this run's measured INT8 burst peak; inside the step the GEMMs hold the GPU at "
+                             "its power cap and lower clocks"),
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "clocks": clk.summary(),
-            "gpu_launches": launches_per_step * args.steps,
-            "gpu_launches_note": "6 libsq kernels per step (+1 torch fill zeroing the two running maxima)",
+            "clocks": clocks,
+            "int8_peak": tpk,
+            "gpu_launches": spec.launches_per_step * steps,
+            "gpu_launches_note": spec.launches_note,
             "peaks": P,
         }
+        line.update(spec.extra.get("line", {}))
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+    return 0
+
+
+def _pinned16(bits, dt):
+    import numpy as np
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(dt).pin_memory()
+
+
+def build_mlp70b(args, rank, world) -> Spec:
+    import numpy as np
+    import torch
+    import synth
+    import w8a8_post_quantization_calib_b200 as sq
+    from w8a8_post_quantization_calib_b200.dist import allreduce_absmax_
+
+    bf16 = torch.bfloat16
+    blk = synth.mlp_block_70b(shard=rank)
+    d, f, M, eps, al = blk.d, blk.f, blk.M, blk.eps, blk.alpha
+    calib_h = _pinned16(np.concatenate(blk.calib), bf16)
+    x_h = _pinned16(blk.x, bf16)
+    wg_h, wu_h, wd_h = _pinned16(blk.w_gate, bf16), _pinned16(blk.w_up, bf16), _pinned16(blk.w_down, bf16)
+    Mc = calib_h.shape[0]
+    dv = torch.device("cuda")
+    calib, X = calib_h.to(dv), x_h.to(dv)
+    Wg, Wu, Wd = wg_h.to(dv), wu_h.to(dv), wd_h.to(dv)
+    gamma = torch.from_numpy(blk.gamma).to(dv)
+    stats = torch.zeros(2 * d + 2 * f, dtype=torch.float32, device=dv)     # running maxima, zeroed each step
+    am1, wm1 = stats[:d], stats[d:2 * d]
+    am2, wm2 = stats[2 * d:2 * d + f], stats[2 * d + f:]
+    s1, s2 = torch.empty(d, device=dv), torch.empty(f, device=dv)
+    a1, a2 = torch.empty(1, device=dv), torch.empty(1, device=dv)
+    wq_gu = torch.empty(2 * f, d, dtype=torch.int8, device=dv)
+    ws_gu = torch.empty(2 * f, device=dv)
+    wq_d = torch.empty(d, f, dtype=torch.int8, device=dv)
+    ws_d = torch.empty(d, device=dv)
+    xq_c = torch.empty(Mc, d, dtype=torch.int8, device=dv)
+    h_c = torch.empty(Mc, f, dtype=bf16, device=dv)
+    xq = torch.empty(M, d, dtype=torch.int8, device=dv)
+    hq = torch.empty(M, f, dtype=torch.int8, device=dv)
+    y = torch.empty(M, d, dtype=bf16, device=dv)
+    y_h = torch.empty(M, d, dtype=bf16).pin_memory()
+    S = sq.ACT_STATIC
+
+    calls = [
+        ("calib_norm_absmax", lambda: sq.rmsnorm_absmax(calib, gamma, eps, am1)),
+        ("allreduce_norm_stat", lambda: allreduce_absmax_(am1)),
+        ("weight_absmax_gate", lambda: sq.calib_absmax(Wg, wm1)),
+        ("weight_absmax_up", lambda: sq.calib_absmax(Wu, wm1)),
+        ("smooth_scales_gateup", lambda: sq.smooth_scales(am1, wm1, al, s1, a1)),
+        ("quant_weight_gateup", lambda: sq.quant_weight_gateup(Wg, Wu, s1, wq_gu, ws_gu)),
+        ("calib_rmsnorm_quant", lambda: sq.rmsnorm_quant(calib, gamma, s1, eps, a1, xq_c)),
+        ("calib_gateup_h", lambda: sq.linear_w8a8_gateup_silu(xq_c, wq_gu, a1, S, ws_gu, h=h_c)),
+        ("calib_absmax_h", lambda: sq.calib_absmax(h_c, am2)),
+        ("allreduce_h_stat", lambda: allreduce_absmax_(am2)),
+        ("weight_absmax_down", lambda: sq.calib_absmax(Wd, wm2)),
+        ("smooth_scales_down", lambda: sq.smooth_scales(am2, wm2, al, s2, a2)),
+        ("quant_weight_down", lambda: sq.quant_weight(Wd, s2, wq_d, ws_d)),
+        ("rmsnorm_quant", lambda: sq.rmsnorm_quant(X, gamma, s1, eps, a1, xq)),
+        ("gateup_silu_requant", lambda: sq.linear_w8a8_gateup_silu(xq, wq_gu, a1, S, ws_gu, s2=s2, a2=a2, hq=hq)),
+        ("down", lambda: sq.linear_w8a8(hq, wq_d, a2, S, ws_d, y)),
+    ]
+    if world == 1:
+        calls = [c for c in calls if not c[0].startswith("allreduce")]
+    names = [c[0] for c in calls]
+
+    def step(mark):
+        stats.zero_()                        # the running maxima start from zero each step
+        for i, (_, fn) in enumerate(calls):
+            mark(i)
+            fn()
+        mark(len(calls))
+
+    gu_ops = 2.0 * M * 2 * f * d
+    work = {
+        "calib_norm_absmax": {"bytes": Mc * d * 2},
+        "weight_absmax_gate": {"bytes": f * d * 2},
+        "weight_absmax_up": {"bytes": f * d * 2},
+        "smooth_scales_gateup": {"bytes": d * 12},
+        "quant_weight_gateup": {"bytes": 2 * f * d * 3 + 2 * f * 4},
+        "calib_rmsnorm_quant": {"bytes": Mc * d * 3},
+        "calib_gateup_h": {"ops": 2.0 * Mc * 2 * f * d, "bytes": Mc * d + 2 * f * d + Mc * f * 2},
+        "calib_absmax_h": {"bytes": Mc * f * 2},
+        "weight_absmax_down": {"bytes": d * f * 2},
+        "smooth_scales_down": {"bytes": f * 12},
+        "quant_weight_down": {"bytes": d * f * 3 + d * 4},
+        "rmsnorm_quant": {"bytes": M * d * 3},
+        "gateup_silu_requant": {"ops": gu_ops, "bytes": M * d + 2 * f * d + M * f},
+        "down": {"ops": 2.0 * M * d * f, "bytes": M * f + d * f + M * d * 2},
+    }
+    solo = {n: fn for n, fn in calls if not n.startswith("allreduce")}
+    ops = 2.0 * Mc * 2 * f * d + gu_ops + 2.0 * M * d * f
+    nlaunch = len([n for n in names if not n.startswith("allreduce")])
+    return Spec(
+        workload="mlp70b",
+        config=dict(LINE_CONFIG["mlp70b"]),
+        ops_per_step=ops, tokens_per_step=M, names=names, step=step, dominant="gateup_silu_requant",
+        work=work, solo=solo,
+        e2e_in=[(calib, calib_h), (X, x_h), (Wg, wg_h), (Wu, wu_h), (Wd, wd_h)], e2e_out=[(y_h, y)],
+        launches_per_step=nlaunch,
+        launches_note=(f"{nlaunch} libsq kernels per step (+1 torch fill zeroing the four running maxima"
+                       + (", +2 NCCL all-reduces" if world > 1 else "") + ")"),
+        traffic=lambda: traffic_from_profile("linear_w8a8_gateup_mlp70b_traffic"),
+        data=blk if world == 1 else None,
+        extra={"solo_reps": {"calib_gateup_h": 3, "gateup_silu_requant": 3, "down": 3, "quant_weight_gateup": 5},
+               "line": {"ops_note": ("ops per step = the calibration forward's gate/up GEMM (16384 calibration "
+                                     "tokens) + the runtime gate/up and down GEMMs, 2*M*N*K each")}},
+    )
+
+
+def build_qkv7b(args, rank, world) -> Spec:
+    import numpy as np
+    import torch
+    import synth
+    import w8a8_post_quantization_calib_b200 as sq
+    from w8a8_post_quantization_calib_b200.dist import allreduce_absmax_
+
+    f16 = torch.float16
+    wl = synth.qkv_7b(shard=rank)
+    M, K, N = QKV_M, QKV_K, QKV_N
+    calib_h, w_h, x_h = _pinned16(np.concatenate(wl.calib), f16), _pinned16(wl.w, f16), _pinned16(wl.x, f16)
+    dv = torch.device("cuda")
+    calib, W, X = calib_h.to(dv), w_h.to(dv), x_h.to(dv)
+    stats = torch.zeros(2 * K, dtype=torch.float32, device=dv)
+    act_max, w_max = stats[:K], stats[K:]
+    s, a = torch.empty(K, device=dv), torch.empty(1, device=dv)
+    wq, ws = torch.empty(N, K, dtype=torch.int8, device=dv), torch.empty(N, device=dv)
+    xq = torch.empty(M, K, dtype=torch.int8, device=dv)
+    y = torch.empty(M, N, dtype=f16, device=dv)
+    y_h = torch.empty(M, N, dtype=f16).pin_memory()
+    calls = [
+        ("calib_absmax", lambda: sq.calib_absmax(calib, act_max)),
+        ("allreduce_max", lambda: allreduce_absmax_(act_max)),
+        ("weight_absmax", lambda: sq.calib_absmax(W, w_max)),
+        ("smooth_scales", lambda: sq.smooth_scales(act_max, w_max, 0.5, s, a)),
+        ("quant_weight", lambda: sq.quant_weight(W, s, wq, ws)),
+        ("smooth_quant_act", lambda: sq.smooth_quant_act(X, s, sq.ACT_STATIC, a, xq)),
+        ("linear_w8a8", lambda: sq.linear_w8a8(xq, wq, a, sq.ACT_STATIC, ws, y)),
+    ]
+    if world == 1:
+        calls = [c for c in calls if c[0] != "allreduce_max"]
+    names = [c[0] for c in calls]
+
+    def step(mark):
+        stats.zero_()
+        for i, (_, fn) in enumerate(calls):
+            mark(i)
+            fn()
+        mark(len(calls))
+
+    ops = 2.0 * M * N * K
+    Mc = calib_h.shape[0]
+    work = {"calib_absmax": {"bytes": Mc * K * 2}, "weight_absmax": {"bytes": N * K * 2},
+            "smooth_scales": {"bytes": K * 12}, "quant_weight": {"bytes": N * K * 3 + N * 4},
+            "smooth_quant_act": {"bytes": M * K * 3},
+            "linear_w8a8": {"ops": ops, "bytes": M * K + N * K + M * N * 2 + N * 4}}
+    return Spec(
+        workload="qkv7b",
+        config=dict(LINE_CONFIG["qkv7b"]),
+        ops_per_step=ops, tokens_per_step=M, names=names, step=step, dominant="linear_w8a8", work=work,
+        solo={n: fn for n, fn in calls if n != "allreduce_max"},
+        e2e_in=[(calib, calib_h), (W, w_h), (X, x_h)], e2e_out=[(y_h, y)],
+        launches_per_step=6, launches_note="6 libsq kernels per step (+1 torch fill zeroing the two running maxima)",
+        traffic=lambda: traffic_from_profile("linear_w8a8_qkv7b_traffic"),
+        data=wl if world == 1 else None,
+        extra={"solo_reps": {"linear_w8a8": 20, "calib_absmax": 10}})
+
+
+BUILDERS = {"mlp70b": build_mlp70b, "qkv7b": build_qkv7b}
+# the config of each line, shared by both arms (the reference arm reports the
+# same workload; "launch" is the GPU arm's default)
+LINE_CONFIG = {
+    "mlp70b": {"workload": MLP70B_DESC, "M": 16384, "d": 8192, "f": 28672, "calib_tokens": 16384, "alpha": 0.5,
+               "eps": 1e-5, "l2": "no flush: every step streams about 7 GB of inputs, weights and activations "
+                                  "(> 126 MB L2)"},
+    "qkv7b": {"workload": QKV_DESC, "M": QKV_M, "K": QKV_K, "N": QKV_N, "calib_tokens": QKV_CB * QKV_CR,
+              "alpha": 0.5, "l2": "no flush: every step streams 384 MB of inputs (> 126 MB L2)"},
+}
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle as it stands on a bounded sample of the
+    line workload, on this machine's host cores (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    import synth
+    oracle.build()
+    wl = args.workload
+    if wl == "mlp70b":
+        data = synth.mlp_block_70b()
+        ops, tokens = 2.0 * 16384 * 2 * 28672 * 8192 * 2 + 2.0 * 16384 * 8192 * 28672, 16384
+    else:
+        data = synth.qkv_7b()
+        ops, tokens = 2.0 * QKV_M * QKV_N * QKV_K, QKV_M
+    cfg = LINE_CONFIG[wl]
+    fn = ORACLE_SAMPLE[wl]
+    # size one step so that warm-up + steps stay within about two minutes
+    probe = 1.0 / 2048
+    t_probe, _ = fn(probe, data)
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    frac = min(1.0, max(1.0 / 16384, probe * budget / max(t_probe, 1e-3)))
+    for _ in range(args.warmup):
+        fn(frac, data)
+    times, sdesc = [], ""
+    for _ in range(args.steps):
+        t, sdesc = fn(frac, data)
+        times.append(t / frac)
+    ms = 1e3 * statistics.mean(times)
+    value = ops / (ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "s8", "data": "synthetic (seeded; shapes and laws of the workload)",
+        "impl": "reference",
+        "config": dict(cfg, parallelism=f"dp{args.gpus} (token shards; all-reduce MAX of the statistics)",
+                       launch="K steps as one CUDA graph"),
+        "tokens_per_s": tokens / (ms * 1e-3),
+        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": cpu_cores(), "kind": "oracle", "sample": sdesc},
+        "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
     return 0
 
 
@@ -540,7 +785,9 @@ def run_workload(args):
     import w8a8_post_quantization_calib_b200 as sq
 
     torch.cuda.set_device(0)
+    torch.cuda.set_stream(torch.cuda.Stream())
     P = peaks()
+    P["int8_tops"] = 2.0 * P["bf16_tflops"]        # per-kernel fractions below: 2 x bf16 (nominal ratio)
     out = {"workload": args.workload, "peaks": P}
     bf16, f16 = torch.bfloat16, torch.float16
     if args.workload == "mlp7b":
@@ -634,59 +881,83 @@ def run_workload(args):
                     "act_quant_us": t_q * 1e3, "act_quant_gbs": M * K * 3 / (t_q * 1e-3) / 1e9,
                     "gemm_us": t_g * 1e3, "gemm_tops": ops / (t_g * 1e-3) / 1e12,
                     "gemm_frac_int8_peak": ops / (t_g * 1e-3) / 1e12 / P["int8_tops"]})
-    elif args.workload == "mlp70b":
-        blk = synth.mlp_block_70b(calib_batches=1)
-        d, f, M = blk.d, blk.f, blk.M
-        g = torch.from_numpy(blk.gamma).cuda()
-        Wg, Wu, Wd = _dev16(blk.w_gate, bf16), _dev16(blk.w_up, bf16), _dev16(blk.w_down, bf16)
-        calib = _dev16(blk.calib[0], bf16)
-        am1 = torch.zeros(d, device="cuda")
-        t_stat = _time_ms(lambda: sq.rmsnorm_absmax(calib, g, blk.eps, am1), 10)
-        wm1 = torch.zeros(d, device="cuda")
-        sq.calib_absmax(Wg, wm1)
-        sq.calib_absmax(Wu, wm1)
-        s1 = torch.empty(d, device="cuda")
-        a1 = torch.empty(1, device="cuda")
-        sq.smooth_scales(am1, wm1, 0.5, s1, a1)
-        wq_gu = torch.empty(2 * f, d, dtype=torch.int8, device="cuda")
-        ws_gu = torch.empty(2 * f, device="cuda")
-        t_wgu = _time_ms(lambda: sq.quant_weight_gateup(Wg, Wu, s1, wq_gu, ws_gu), 5)
-        X = _dev16(blk.x, bf16)
-        xq = torch.empty(M, d, dtype=torch.int8, device="cuda")
-        h = torch.empty(M, f, dtype=bf16, device="cuda")
-        hq = torch.empty(M, f, dtype=torch.int8, device="cuda")
-        sq.rmsnorm_quant(X, g, s1, blk.eps, a1, xq)
-        sq.linear_w8a8_gateup_silu(xq[:2048], wq_gu, a1, sq.ACT_STATIC, ws_gu, h=h[:2048])
-        am2 = torch.zeros(f, device="cuda")
-        sq.calib_absmax(h[:2048], am2)
-        wm2 = torch.zeros(f, device="cuda")
-        sq.calib_absmax(Wd, wm2)
-        s2 = torch.empty(f, device="cuda")
-        a2 = torch.empty(1, device="cuda")
-        sq.smooth_scales(am2, wm2, 0.5, s2, a2)
-        wq_d = torch.empty(d, f, dtype=torch.int8, device="cuda")
-        ws_d = torch.empty(d, device="cuda")
-        sq.quant_weight(Wd, s2, wq_d, ws_d)
-        y = torch.empty(M, d, dtype=bf16, device="cuda")
-        t_n = _time_ms(lambda: sq.rmsnorm_quant(X, g, s1, blk.eps, a1, xq), 10)
-        t_gu = _time_ms(lambda: sq.linear_w8a8_gateup_silu(xq, wq_gu, a1, sq.ACT_STATIC, ws_gu, s2=s2, a2=a2, hq=hq), 5)
-        t_gu_h = _time_ms(lambda: sq.linear_w8a8_gateup_silu(xq, wq_gu, a1, sq.ACT_STATIC, ws_gu, h=h), 5)
-        t_d = _time_ms(lambda: sq.linear_w8a8(hq, wq_d, a2, sq.ACT_STATIC, ws_d, y), 5)
-        ops_gu, ops_d = 2.0 * M * 2 * f * d, 2.0 * M * d * f
-        t_blk = t_n + t_gu + t_d
-        out.update({"M": M, "d": d, "f": f,
-                    "block_ms": t_blk, "block_tokens_per_s": M / (t_blk * 1e-3),
-                    "block_tops": (ops_gu + ops_d) / (t_blk * 1e-3) / 1e12,
-                    "rmsnorm_quant_us": t_n * 1e3, "rmsnorm_quant_gbs": M * d * 3 / (t_n * 1e-3) / 1e9,
-                    "rmsnorm_absmax_us_per_2048_tokens": t_stat * 1e3,
-                    "rmsnorm_absmax_gbs": 2048 * d * 2 / (t_stat * 1e-3) / 1e9,
-                    "gateup_silu_requant_us": t_gu * 1e3, "gateup_tops": ops_gu / (t_gu * 1e-3) / 1e12,
-                    "gateup_frac_int8_peak": ops_gu / (t_gu * 1e-3) / 1e12 / P["int8_tops"],
-                    "gateup_silu_bf16_h_us": t_gu_h * 1e3,
-                    "down_us": t_d * 1e3, "down_tops": ops_d / (t_d * 1e-3) / 1e12,
-                    "down_frac_int8_peak": ops_d / (t_d * 1e-3) / 1e12 / P["int8_tops"],
-                    "weight_quant_gateup_us": t_wgu * 1e3,
-                    "weight_quant_gateup_gbs": 2 * f * d * 3 / (t_wgu * 1e-3) / 1e9})
+    elif args.workload == "peak":
+        clk = ClockSampler(0).start()
+        out["int8"] = tensor_peak("i8", clk)
+        out["e4m3"] = tensor_peak("e4m3", clk)
+        clk.stop()
+        out["nominal_dense_tops"] = 4500.0
+    elif args.workload == "fp8":
+        # the FP8 (E4M3) linear on the Llama-7B MLP shapes: per-token E4M3
+        # activation quant + kind::f8f6f4 GEMM, against the INT8 path
+        tpk = tensor_peak("e4m3")
+        lines = []
+        for which in args.proj.split(","):
+            wl = synth.mlp_7b(which, M=4096, calib_batches=4)
+            K, N = wl.K, wl.N
+            W = _dev16(wl.w, bf16)
+            am = torch.zeros(K, device="cuda")
+            sq.calib_absmax(_dev16(np.concatenate(wl.calib), bf16), am)
+            wm = torch.zeros(K, device="cuda")
+            sq.calib_absmax(W, wm)
+            s = torch.empty(K, device="cuda")
+            a = torch.empty(1, device="cuda")
+            sq.smooth_scales_fp8(am, wm, 0.5, s, a)
+            wq8 = torch.empty(N, K, dtype=torch.uint8, device="cuda")
+            ws = torch.empty(N, device="cuda")
+            sq.quant_weight_fp8(W, s, wq8, ws)
+            t_wq = _time_ms(lambda: sq.quant_weight_fp8(W, s, wq8, ws), 10)
+            Xall = _dev16(wl.x, bf16)
+            for M in (int(t) for t in args.tokens.split(",")):
+                X = Xall[:M]
+                xq8 = torch.empty(M, K, dtype=torch.uint8, device="cuda")
+                at = torch.empty(M, device="cuda")
+                y = torch.empty(M, N, dtype=bf16, device="cuda")
+                t_q = _time_ms(lambda: sq.smooth_quant_act_fp8(X, s, sq.ACT_PER_TOKEN, at, xq8), 50)
+                t_g = _time_ms(lambda: sq.linear_fp8(xq8, wq8, at, sq.ACT_PER_TOKEN, ws, y), 20)
+                ops = 2.0 * M * N * K
+                lines.append({"proj": which, "M": M, "K": K, "N": N,
+                              "act_quant_us": t_q * 1e3, "act_quant_gbs": M * K * 3 / (t_q * 1e-3) / 1e9,
+                              "gemm_us": t_g * 1e3, "gemm_tops": ops / (t_g * 1e-3) / 1e12,
+                              "gemm_frac_e4m3_peak": ops / (t_g * 1e-3) / 1e12 / tpk["burst"]["tops"],
+                              "weight_quant_us": t_wq * 1e3,
+                              "weight_quant_gbs": N * K * 3 / (t_wq * 1e-3) / 1e9})
+        out["e4m3_peak"] = tpk
+        out["lines"] = lines
+    elif args.workload == "gemm":
+        # one GEMM of the bench workloads on seeded INT8 operands, for timing
+        # and for targeted profiler captures: gateup (70B block, SiLU*mul +
+        # requant epilogue), down (70B block), qkv (Llama-7B QKV, fp16 out)
+        g8 = torch.Generator(device="cuda").manual_seed(11)
+
+        def codes(r, c):
+            return torch.randint(-127, 128, (r, c), generator=g8, device="cuda", dtype=torch.int8)
+        lines = []
+        for M in (int(t) for t in args.tokens.split(",")):
+            if args.gemm == "gateup":
+                d, f = 8192, 28672
+                xq, wq = codes(M, d), codes(2 * f, d)
+                a = torch.full((1,), 1e-2, device="cuda")
+                ws = torch.rand(2 * f, generator=g8, device="cuda") * 1e-3
+                s2 = torch.rand(f, generator=g8, device="cuda") + 0.5
+                a2 = torch.full((1,), 0.05, device="cuda")
+                hq = torch.empty(M, f, dtype=torch.int8, device="cuda")
+                fn = lambda: sq.linear_w8a8_gateup_silu(xq, wq, a, sq.ACT_STATIC, ws, s2=s2, a2=a2, hq=hq)
+                ops, nb = 2.0 * M * 2 * f * d, M * d + 2 * f * d + M * f
+            else:
+                K, N, odt = (28672, 8192, bf16) if args.gemm == "down" else (4096, 12288, f16)
+                xq, wq = codes(M, K), codes(N, K)
+                a = torch.full((1,), 1e-2, device="cuda")
+                ws = torch.rand(N, generator=g8, device="cuda") * 1e-3
+                y = torch.empty(M, N, dtype=odt, device="cuda")
+                fn = lambda: sq.linear_w8a8(xq, wq, a, sq.ACT_STATIC, ws, y)
+                ops, nb = 2.0 * M * N * K, M * K + N * K + M * N * 2
+            t_ms = _time_ms(fn, args.reps, warmup=3, graph=not args.eager_steps)
+            lines.append({"gemm": args.gemm, "M": M, "us": t_ms * 1e3, "tops": ops / (t_ms * 1e-3) / 1e12,
+                          "frac_int8_2xbf16": ops / (t_ms * 1e-3) / 1e12 / P["int8_tops"],
+                          "algorithmic_bytes": nb})
+            del xq, wq
+        out["lines"] = lines
     elif args.workload == "rows":
         # the HBM-bound kernels on inputs of 256 MiB (twice the L2), so that
         # every call of a timed chain streams from HBM; bytes = algorithmic
@@ -752,29 +1023,39 @@ def run_workload(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: 20 for mlp70b, 200 for qkv7b)")
+    ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["sq", "reference"], default="sq")
-    ap.add_argument("--cpu-frac", type=float, default=0.25,
-                    help="fraction of the workload the CPU oracle baseline runs")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0,
+                    help="CPU work the oracle baseline's sample is sized for")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--eager-steps", action="store_true",
                     help="launch the timed steps one call at a time instead of as one captured CUDA graph")
     ap.add_argument("--tokens", default="1,16,128,4096",
-                    help="mlp7b workload: comma-separated token counts M to sweep")
-    ap.add_argument("--proj", default="up,down", help="mlp7b workload: projections to sweep")
+                    help="mlp7b / fp8 workloads: comma-separated token counts M to sweep")
+    ap.add_argument("--proj", default="up,down", help="mlp7b / fp8 workloads: projections to sweep")
     ap.add_argument("--only", default="", help="rows workload: comma-separated kernels to run (default all)")
     ap.add_argument("--rows-k", default="", help="rows workload: row lengths to run, of 4096 (fp16) and 8192 (bf16)")
-    ap.add_argument("--workload", choices=["qkv7b", "mlp7b", "alpha13b", "mlp70b", "rows"], default="qkv7b",
-                    help="qkv7b is the bench line; the others print per-kernel measurements of the other workloads")
+    ap.add_argument("--gemm", choices=["gateup", "down", "qkv"], default="gateup",
+                    help="gemm workload: which GEMM of the bench workloads to run")
+    ap.add_argument("--reps", type=int, default=10, help="gemm workload: launches in the timed graph")
+    ap.add_argument("--workload", choices=list(LINES) + ["mlp7b", "alpha13b", "rows", "peak", "fp8", "gemm"],
+                    default="mlp70b",
+                    help="mlp70b (default) and qkv7b print a bench line; the others print per-kernel measurements")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.steps is None:
+        args.steps = 20 if args.workload == "mlp70b" else 200
     if args.impl == "reference":
+        if args.workload not in LINES:
+            ap.error("--impl reference times a bench-line workload")
         return run_reference(args)
-    if args.workload != "qkv7b":
+    if args.workload not in LINES:
         return run_workload(args)
-    return run_gpu(args)
+    return run_line(args, BUILDERS[args.workload])
 
 
 if __name__ == "__main__":

@@ -22,7 +22,10 @@
  *     says "host".  The library allocates no device memory; calls that need
  *     scratch take a caller-provided workspace.
  *   - Calls are asynchronous and stream-ordered on `stream` (a cudaStream_t;
- *     NULL is the legacy default stream) on the current CUDA device.
+ *     NULL is the legacy default stream) on the current CUDA device.  On a
+ *     created stream the kernels are launched with programmatic dependent
+ *     launch (no gap for launch processing between consecutive kernels); on
+ *     the default streams (legacy or per-thread) they are launched plainly.
  *   - Arguments are validated before any launch: null pointers, sizes, 16-byte
  *     alignment where vector or TMA access needs it, dtype support.  A bad
  *     argument returns an error status and launches nothing.  No call aborts,
@@ -120,6 +123,47 @@ sq_status sq_calib_absmax(const void *x, sq_dtype dt, int64_t rows, int64_t cols
                           float *absmax, sq_stream stream);
 
 /* -------------------------------------------------------------------------
+ * (1b) Robust calibration statistics.  kwkr 3.1: instead of the per-channel
+ * max, a high quantile of |X_j| (the page names 99.9 %) or the mean of the
+ * maxima of several calibration samples, so that one abnormal token does not
+ * set the channel's smoothing factor.  Either result stands in for act_max
+ * in sq_smooth_scales unchanged.
+ * ------------------------------------------------------------------------- */
+
+/* Nearest-rank p-quantile of |x| per column over all `rows` calibration
+ * tokens (the batches laid end to end, or strided with ld):
+ *
+ *   out[j] = the k-th smallest of |x[t * ld + j]|, t < rows,  k = ceil(p * rows)
+ *            (the product in fp64; 1 <= k <= rows)
+ *
+ * The result is one of the data values, widened exactly to fp32 (p = 1 gives
+ * the max).  Found by a radix select on the magnitude bit patterns: 2 passes
+ * over x for fp16/bf16, 4 for fp32.  x: [rows, ld] of `dt`, 16-byte aligned,
+ * cols * sizeof(dt) and ld * sizeof(dt) multiples of 16 (else
+ * SQ_ERR_MISALIGNED).  1 <= rows < 2^32; 0 < p <= 1.  out: fp32 [cols].
+ * workspace: sq_calib_quantile_workspace_size(cols) bytes, 16-byte aligned
+ * (per-column histograms of 256 bins, prefixes and ranks); no
+ * initialisation needed.  NaN inputs are not supported. */
+size_t sq_calib_quantile_workspace_size(int64_t cols);
+sq_status sq_calib_quantile(const void *x, sq_dtype dt, int64_t rows, int64_t cols, int64_t ld, double p,
+                            float *out, void *workspace, size_t workspace_bytes, sq_stream stream);
+
+/* Mean of per-sample maxima, one calibration batch (sample) per call:
+ *
+ *   batch max      m_j = max_r |x[r * ld + j]|                (exact, into batch_max)
+ *   running sum    sum_max[j] += (double) m_j;  batch_max[j] = 0
+ *
+ * then sq_calib_mean_of_max gives out[j] = fl32(sum_max[j] / n_batches) (fp64
+ * division).  The fp64 sum is taken in call order, one add per batch.
+ * batch_max: fp32 [cols], zero before the first call (every call leaves it
+ * zero).  sum_max: fp64 [cols], zeroed by the caller before the first batch.
+ * rows >= 1. */
+sq_status sq_calib_batchmax_accumulate(const void *x, sq_dtype dt, int64_t rows, int64_t cols, int64_t ld,
+                                       float *batch_max, double *sum_max, sq_stream stream);
+sq_status sq_calib_mean_of_max(const double *sum_max, int64_t cols, int64_t n_batches, float *out,
+                               sq_stream stream);
+
+/* -------------------------------------------------------------------------
  * (2a) Smoothing factors.  kwkr 2.2, aiu, adr-010 context step 1:
  *
  *   s_j = max(act_max_j, 1e-5)^alpha / max(w_max_j, 1e-5)^(1 - alpha)
@@ -161,6 +205,27 @@ sq_status sq_quant_weight(const void *w, sq_dtype dt, int64_t N, int64_t K, cons
 sq_status sq_quant_weight_gateup(const void *w_gate, const void *w_up, sq_dtype dt, int64_t N_h,
                                  int64_t K, const float *s, int8_t *wq_gu, float *w_scale_gu,
                                  sq_stream stream);
+
+/* Cross-layer folding ("010. SmoothQuant Integration", Alternative C; kwkr
+ * 3.2): when the smoothed layer's input is (or depends linearly on) a
+ * previous linear's output, 1/s of the smoothed layer moves into that
+ * previous layer's output rows, and the runtime x/s step disappears.  These
+ * calls transform the PREVIOUS layer's weight with the fold applied first:
+ *
+ *   W'[n,j] = fl(fl(W[n,j] * recip(s_next_n)) * s_j)     (then per-row INT8 as in sq_quant_weight)
+ *
+ * s: this layer's own smoothing factors [K]; s_next: the smoothing factors of
+ * the next layer's input channels, one per output row n [N].
+ * sq_quant_weight_gateup_fold folds only the up rows (h = silu(g) * u is
+ * linear in u, so h / s_next = silu(g) * (u / s_next)); s_next is [N_h],
+ * indexed by channel; the gate rows are those of sq_quant_weight_gateup.  A
+ * gate/up GEMM on folded weights is then called with s2 = NULL (its requant
+ * multiplies by recip(a2) only). */
+sq_status sq_quant_weight_fold(const void *w, sq_dtype dt, int64_t N, int64_t K, const float *s,
+                               const float *s_next, int8_t *wq, float *w_scale, sq_stream stream);
+sq_status sq_quant_weight_gateup_fold(const void *w_gate, const void *w_up, sq_dtype dt, int64_t N_h,
+                                      int64_t K, const float *s, const float *s_next, int8_t *wq_gu,
+                                      float *w_scale_gu, sq_stream stream);
 
 /* -------------------------------------------------------------------------
  * (3a) Runtime smoothing + INT8 activation quantisation.  The 1/s scaling
@@ -282,6 +347,20 @@ sq_status sq_linear_w8a8_noalloc(const int8_t *xq, const int8_t *wq, int64_t M, 
 /* Capacity of the fixed partial-sum array of sq_linear_w8a8_noalloc, in int32 values (2^21). */
 size_t sq_linear_w8a8_noalloc_max_elems(void);
 
+/* fp16 storage of the scales ("010. SmoothQuant Integration", consequences:
+ * storage).  sq_scales_to_f16 rounds fp32 scales to fp16 (nearest even;
+ * uint16 bit patterns), sq_scales_from_f16 widens them back exactly.
+ * sq_linear_w8a8_f16scales is sq_linear_w8a8 with a_scale and w_scale stored
+ * as fp16: the epilogue widens them exactly, so its result equals
+ * sq_linear_w8a8 given the widened fp32 scales, bit for bit.  w_scale_f16
+ * 16-byte aligned. */
+sq_status sq_scales_to_f16(const float *in, int64_t n, uint16_t *out, sq_stream stream);
+sq_status sq_scales_from_f16(const uint16_t *in, int64_t n, float *out, sq_stream stream);
+sq_status sq_linear_w8a8_f16scales(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, int64_t K,
+                                   const uint16_t *a_scale_f16, sq_act_mode mode,
+                                   const uint16_t *w_scale_f16, const void *bias, sq_dtype out_dt, void *y,
+                                   void *workspace, size_t workspace_bytes, sq_stream stream);
+
 /* Raw int32 accumulators acc[m,n] = sum_k xq[m,k] * wq[n,k] from the same
  * tensor-core mainloop (for exact INT32 checks).  acc: int32 [M, N]. */
 sq_status sq_gemm_s32(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, int64_t K,
@@ -298,7 +377,10 @@ sq_status sq_gemm_s32(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, 
  * quantises h for the next linear with a static scale:
  *   hq[m,c] = q(fl(fl(h[m,c] * recip(s2_c)) * recip(a2[0])))
  * using the bf16-rounded h (so it equals sq_smooth_quant_act on h).
- * s2: fp32 [N_h], a2: fp32 [1] (required with hq).  N_h a multiple of 128.
+ * s2: fp32 [N_h] or NULL, a2: fp32 [1] (required with hq).  s2 == NULL is
+ * the folded form (weights from sq_quant_weight_gateup_fold, h already
+ * divided by s2): hq[m,c] = q(fl(h[m,c] * recip(a2[0]))).  N_h a multiple
+ * of 128.
  * silu(g) is computed in fp32 with CUDA's fast exponential and division
  * intrinsics (errors of a few fp32 ulp, far below bf16's 8 bits); h matches
  * a correctly rounded SiLU within 2 bf16 ulp (or 1e-30 absolute). */

@@ -177,12 +177,15 @@ class MLPBlockWorkload:
 
 
 def mlp_block_70b(M: int = 16384, d: int = 8192, f: int = 28672, calib_batches: int = 8,
-                  calib_rows: int = 2048, gamma_random: bool = False) -> MLPBlockWorkload:
+                  calib_rows: int = 2048, gamma_random: bool = False, shard: int = 0) -> MLPBlockWorkload:
+    """``shard`` selects independent calibration and runtime token batches (same
+    block weights and outlier channels): one set per rank when the tokens are
+    spread over several GPUs."""
     wl = 5
     idx, c = outlier_channels(rng(wl, 1), d, 0.005, 20.0, 100.0)
 
     def act(stream, rows):
-        return cast(apply_channels(normal(rng(wl, stream), (rows, d)), idx, c), BF16)
+        return cast(apply_channels(normal(rng(wl, stream + 100000 * shard), (rows, d)), idx, c), BF16)
 
     gamma = (rng(wl, 4).uniform(0.5, 1.5, size=d).astype(np.float32) if gamma_random
              else np.ones(d, np.float32))

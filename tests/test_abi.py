@@ -103,7 +103,7 @@ def _alphas(*v):
     ("sq_rmsnorm_absmax", (_A, 2, 0, 64, _A, 1e-5, _A, None), 0),
     ("sq_linear_w8a8_gateup_silu", (_A, _A, 300, 96, 512, _A, 0, _A, _A, None, None, None, None), 1),   # N_h % 128
     ("sq_linear_w8a8_gateup_silu", (_A, _A, 300, 128, 512, _A, 0, _A, None, None, None, None, None), 1),  # no output
-    ("sq_linear_w8a8_gateup_silu", (_A, _A, 300, 128, 512, _A, 0, _A, None, None, None, _A, None), 1),   # hq without s2/a2
+    ("sq_linear_w8a8_gateup_silu", (_A, _A, 300, 128, 512, _A, 0, _A, None, _A, None, _A, None), 1),   # hq without a2
     ("sq_linear_w8a8_gateup_silu", (_A, _A, 300, 128, 512, _A, 0, _A, _U, None, None, None, None), 3),
     ("sq_gemm_f16_ref", (_A, _A, 4, 40, 64, _A, None), 1),                    # N % 16
     ("sq_gemm_f16_ref", (_A, _A, 4, 32, 12, _A, None), 1),                    # K % 8
@@ -123,6 +123,17 @@ def _alphas(*v):
     ("sq_linear_fp8", (_A, _A, 4, 40, 64, _A, 0, _A, None, 1, _A, None), 1),    # N % 16
     ("sq_linear_fp8", (_A, _A, 4, 32, 64, _A, 0, _A, None, 1, _U, None), 3),
     ("sq_linear_fp8", (_A, _A, 0, 32, 64, _A, 0, _A, None, 1, _A, None), 1),    # M = 0
+    ("sq_calib_quantile", (_A, 1, 8, 64, 64, 0.0, _A, _A, 1 << 20, None), 1),   # p outside (0, 1]
+    ("sq_calib_quantile", (_A, 1, 8, 64, 64, 0.5, _A, _A, 16, None), 6),        # workspace too small
+    ("sq_calib_quantile", (_U, 1, 8, 64, 64, 0.5, _A, _A, 1 << 20, None), 3),
+    ("sq_calib_quantile", (_A, 1, 8, 60, 60, 0.5, _A, _A, 1 << 20, None), 3),   # rows of 120 bytes
+    ("sq_calib_batchmax_accumulate", (_A, 1, 0, 64, 64, _A, _A, None), 1),      # an empty batch
+    ("sq_calib_mean_of_max", (_A, 64, 0, _A, None), 1),                          # no batches
+    ("sq_quant_weight_fold", (_A, 1, 8, 64, _A, None, _A, _A, None), 1),         # s_next required
+    ("sq_quant_weight_gateup_fold", (_A, _A, 1, 64, 64, _A, None, _A, _A, None), 1),
+    ("sq_scales_to_f16", (_A, -1, _A, None), 1),
+    ("sq_scales_from_f16", (None, 4, _A, None), 1),
+    ("sq_linear_w8a8_f16scales", (_A, _A, 4, 40, 64, _A, 0, _A, None, 1, _A, None, 0, None), 1),   # N % 16
 ])
 def test_every_entry_point_validates_before_launch(fn, args, status):
     import w8a8_post_quantization_calib_b200 as sq

@@ -9,7 +9,9 @@
   "SmoothQuant技术解析" 4.3: the statistic is combined across shards, every
   shard quantises and multiplies its own output rows, and the gathered
   columns equal the unsharded call bit for bit);
-- the layer driver (Calibrator -> QuantizedLinear) against the oracle pipeline.
+- the layer driver (Calibrator -> QuantizedLinear) against the oracle pipeline;
+- whole chains on a created stream (programmatic dependent launches) equal
+  to the same chains on the default stream (plain launches).
 """
 import numpy as np
 import pytest
@@ -17,7 +19,7 @@ import torch
 
 import oracle
 import synth
-from helpers import BF16, F16, bits_equal, dev, host, mismatch_report, rand_x, rel_err
+from helpers import BF16, F16, F32, bits_equal, dev, host, mismatch_report, rand_x, rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -227,3 +229,54 @@ def test_layer_driver_matches_oracle_pipeline(mode):
     assert bits_equal(host(layer.wq), st.wq) and bits_equal(host(layer.w_scale), st.w_scale)
     _, _, _, y_r = oracle.linear_forward(st, wl.x, mode, F16, F16)
     assert np.array_equal(host(y), y_r), mismatch_report(host(y), y_r)
+
+
+# ------------------------------------------------------------------ created streams (programmatic launches)
+def test_chains_on_a_created_stream_equal_the_default_stream():
+    """On a created stream the kernels are launched with programmatic
+    dependent launch (each one's prologue overlaps the previous kernel's
+    tail); the results of whole chains must equal the default stream's bit
+    for bit: the QKV-style linear (calibration -> scales -> weight codes ->
+    activation codes -> GEMM), the robust quantile's four dependent
+    passes, and the per-token small-M path."""
+    wl = synth.outlier_linear(M=300, K=1024, N=768, calib_batches=3, calib_rows=256, x_dt=F16, w_dt=F16,
+                              out_dt=F16, workload=63)
+    calib = dev(np.concatenate(wl.calib), F16)
+    W, X = dev(wl.w, F16), dev(wl.x, F16)
+
+    def chain():
+        am = torch.zeros(wl.K, dtype=torch.float32, device="cuda")
+        sq.calib_absmax(calib, am)
+        wm = torch.zeros(wl.K, dtype=torch.float32, device="cuda")
+        sq.calib_absmax(W, wm)
+        s = torch.empty(wl.K, dtype=torch.float32, device="cuda")
+        a = torch.empty(1, dtype=torch.float32, device="cuda")
+        sq.smooth_scales(am, wm, 0.5, s, a)
+        wq = torch.empty(wl.N, wl.K, dtype=torch.int8, device="cuda")
+        ws = torch.empty(wl.N, dtype=torch.float32, device="cuda")
+        sq.quant_weight(W, s, wq, ws)
+        outs = []
+        for M, mode in ((300, oracle.STATIC), (16, oracle.PER_TOKEN)):
+            xq = torch.empty(M, wl.K, dtype=torch.int8, device="cuda")
+            at = a if mode == oracle.STATIC else torch.empty(M, dtype=torch.float32, device="cuda")
+            sq.smooth_quant_act(X[:M], s, mode, at, xq)
+            y = torch.empty(M, wl.N, dtype=torch.float16, device="cuda")
+            sq.linear_w8a8(xq, wq, at, mode, ws, y)
+            outs.append(y)
+        q = torch.empty(wl.K, dtype=torch.float32, device="cuda")
+        work = torch.empty(sq.calib_quantile_workspace_size(wl.K), dtype=torch.uint8, device="cuda")
+        sq.calib_quantile(calib.float(), 0.999, q, work)       # fp32: four dependent digit passes
+        return [am, wm, s, a, wq, ws, q] + outs
+
+    ref = [t.clone() for t in chain()]
+    _sync()
+    side = torch.cuda.Stream()
+    for _ in range(3):
+        with torch.cuda.stream(side):
+            got = chain()
+        side.synchronize()
+        _sync()
+        for g, r in zip(got, ref):
+            assert torch.equal(g.view(torch.uint8), r.view(torch.uint8))
+    q_r = oracle.calib_quantile([oracle.to_f32(np.concatenate(wl.calib), F16)], 0.999, F32)
+    assert bits_equal(host(ref[6]), q_r)

@@ -14,7 +14,11 @@ Names follow the C ABI: ``calib_absmax``, ``smooth_scales``,
 ``quant_weight_gateup``, ``rmsnorm_quant``, ``linear_w8a8_gateup_silu``,
 ``gemm_f16_ref``, ``sse_f16``, ``alpha_search``) and the FP8 (E4M3) variant
 ``smooth_scales_fp8``, ``quant_weight_fp8``, ``smooth_quant_act_fp8``,
-``linear_fp8`` (codes are uint8 tensors holding E4M3 bit patterns).
+``linear_fp8`` (codes are uint8 tensors holding E4M3 bit patterns), and the
+robust calibration statistics ``calib_quantile``,
+``calib_batchmax_accumulate``, ``calib_mean_of_max``, and the cross-layer fold
+and fp16 scale storage ``quant_weight_fold``, ``quant_weight_gateup_fold``,
+``scales_to_f16``, ``scales_from_f16``, ``linear_w8a8_f16scales``.
 """
 from __future__ import annotations
 
@@ -41,6 +45,9 @@ EXPORTS = (
     "sq_gemm_s32", "sq_linear_w8a8_gateup_silu", "sq_gemm_f16_ref", "sq_sse_f16",
     "sq_alpha_search_workspace_size", "sq_alpha_search",
     "sq_smooth_scales_fp8", "sq_quant_weight_fp8", "sq_smooth_quant_act_fp8", "sq_linear_fp8",
+    "sq_calib_quantile_workspace_size", "sq_calib_quantile", "sq_calib_batchmax_accumulate", "sq_calib_mean_of_max",
+    "sq_quant_weight_fold", "sq_quant_weight_gateup_fold", "sq_scales_to_f16", "sq_scales_from_f16",
+    "sq_linear_w8a8_f16scales",
 )
 
 
@@ -86,6 +93,15 @@ def _load() -> ctypes.CDLL:
         "sq_quant_weight_fp8": (I, [P, I, I64, I64, P, P, P, P]),
         "sq_smooth_quant_act_fp8": (I, [P, I, I64, I64, P, I, P, P, P]),
         "sq_linear_fp8": (I, [P, P, I64, I64, I64, P, I, P, P, I, P, P]),
+        "sq_calib_quantile_workspace_size": (SZ, [I64]),
+        "sq_calib_quantile": (I, [P, I, I64, I64, I64, ctypes.c_double, P, P, SZ, P]),
+        "sq_calib_batchmax_accumulate": (I, [P, I, I64, I64, I64, P, P, P]),
+        "sq_calib_mean_of_max": (I, [P, I64, I64, P, P]),
+        "sq_quant_weight_fold": (I, [P, I, I64, I64, P, P, P, P, P]),
+        "sq_quant_weight_gateup_fold": (I, [P, P, I, I64, I64, P, P, P, P, P]),
+        "sq_scales_to_f16": (I, [P, I64, P, P]),
+        "sq_scales_from_f16": (I, [P, I64, P, P]),
+        "sq_linear_w8a8_f16scales": (I, [P, P, I64, I64, I64, P, I, P, P, I, P, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -320,3 +336,79 @@ def linear_fp8(xq8, wq8, a_scale, mode: int, w_scale, y, bias=None, stream=None)
         _dev(xq8, "xq8", torch.uint8), _dev(wq8, "wq8", torch.uint8), M, N, K,
         _dev(a_scale, "a_scale", torch.float32), int(mode), _dev(w_scale, "w_scale", torch.float32),
         _dev(bias, "bias", y.dtype) if bias is not None else None, _dt(y), _dev(y, "y"), _stream(stream)))
+
+
+# ---------------------------------------------------------------- robust calibration statistics
+def calib_quantile_workspace_size(cols: int) -> int:
+    return int(_lib.sq_calib_quantile_workspace_size(cols))
+
+
+def calib_quantile(x: torch.Tensor, p: float, out: torch.Tensor, workspace: torch.Tensor, rows=None, cols=None,
+                   ld=None, stream=None) -> None:
+    """out[j] = nearest-rank p-quantile of |x[:, j]| over the rows of a 2-D x."""
+    if x.dim() != 2 or x.stride(1) != 1 or not x.is_cuda:
+        raise ValueError("x must be a 2-D CUDA tensor with contiguous rows")
+    rows = x.shape[0] if rows is None else rows
+    cols = x.shape[1] if cols is None else cols
+    ld = x.stride(0) if ld is None else ld
+    _check("sq_calib_quantile", _lib.sq_calib_quantile(
+        x.data_ptr(), _dt(x), rows, cols, ld, float(p), _dev(out, "out", torch.float32),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def calib_batchmax_accumulate(x: torch.Tensor, batch_max: torch.Tensor, sum_max: torch.Tensor, stream=None) -> None:
+    """sum_max[j] += max_r |x[r, j]| (fp64, one calibration batch per call); batch_max is zeroed scratch."""
+    if x.dim() != 2 or x.stride(1) != 1 or not x.is_cuda:
+        raise ValueError("x must be a 2-D CUDA tensor with contiguous rows")
+    _check("sq_calib_batchmax_accumulate", _lib.sq_calib_batchmax_accumulate(
+        x.data_ptr(), _dt(x), x.shape[0], x.shape[1], x.stride(0), _dev(batch_max, "batch_max", torch.float32),
+        _dev(sum_max, "sum_max", torch.float64), _stream(stream)))
+
+
+def calib_mean_of_max(sum_max: torch.Tensor, n_batches: int, out: torch.Tensor, stream=None) -> None:
+    _check("sq_calib_mean_of_max", _lib.sq_calib_mean_of_max(
+        _dev(sum_max, "sum_max", torch.float64), sum_max.numel(), int(n_batches), _dev(out, "out", torch.float32),
+        _stream(stream)))
+
+
+# ---------------------------------------------------------------- cross-layer fold, fp16 scale storage
+def quant_weight_fold(w, s, s_next, wq, w_scale, stream=None) -> None:
+    """Per-row INT8 transform of a previous layer's weight with 1/s_next folded into its output rows."""
+    N, K = w.shape
+    _check("sq_quant_weight_fold", _lib.sq_quant_weight_fold(
+        _dev(w, "w"), _dt(w), N, K, _dev(s, "s", torch.float32), _dev(s_next, "s_next", torch.float32),
+        _dev(wq, "wq", torch.int8), _dev(w_scale, "w_scale", torch.float32), _stream(stream)))
+
+
+def quant_weight_gateup_fold(w_gate, w_up, s, s_next, wq_gu, w_scale_gu, stream=None) -> None:
+    N_h, K = w_gate.shape
+    if w_up.shape != w_gate.shape or w_up.dtype != w_gate.dtype:
+        raise ValueError("w_gate and w_up must match")
+    _check("sq_quant_weight_gateup_fold", _lib.sq_quant_weight_gateup_fold(
+        _dev(w_gate, "w_gate"), _dev(w_up, "w_up"), _dt(w_gate), N_h, K, _dev(s, "s", torch.float32),
+        _dev(s_next, "s_next", torch.float32), _dev(wq_gu, "wq_gu", torch.int8),
+        _dev(w_scale_gu, "w_scale_gu", torch.float32), _stream(stream)))
+
+
+def scales_to_f16(x, out, stream=None) -> None:
+    """fp32 scales -> fp16 storage (round to nearest even); out: float16 tensor."""
+    _check("sq_scales_to_f16", _lib.sq_scales_to_f16(
+        _dev(x, "x", torch.float32), x.numel(), _dev(out, "out", torch.float16), _stream(stream)))
+
+
+def scales_from_f16(x, out, stream=None) -> None:
+    _check("sq_scales_from_f16", _lib.sq_scales_from_f16(
+        _dev(x, "x", torch.float16), x.numel(), _dev(out, "out", torch.float32), _stream(stream)))
+
+
+def linear_w8a8_f16scales(xq, wq, a_scale, mode: int, w_scale, y, bias=None, workspace=None, stream=None) -> None:
+    """linear_w8a8 with a_scale and w_scale stored as float16."""
+    M, K = xq.shape
+    N = wq.shape[0]
+    ws_ptr = _dev(workspace, "workspace") if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("sq_linear_w8a8_f16scales", _lib.sq_linear_w8a8_f16scales(
+        _dev(xq, "xq", torch.int8), _dev(wq, "wq", torch.int8), M, N, K,
+        _dev(a_scale, "a_scale", torch.float16), int(mode), _dev(w_scale, "w_scale", torch.float16),
+        _dev(bias, "bias", y.dtype) if bias is not None else None, _dt(y), _dev(y, "y"),
+        ws_ptr, ws_bytes, _stream(stream)))

@@ -97,7 +97,6 @@ __global__ void __launch_bounds__(CALIB_TX *CALIB_TY)
         }
         for (; r < r1; r += CALIB_TY) acc.add(load16<STREAM>(col + r * ld_bytes));
     }
-    pdl_launch_dependents();
     float f[EPV];
     acc.to_float(f);
 #pragma unroll
@@ -122,7 +121,6 @@ __global__ void k_colabsmax_scalar(const void *__restrict__ x, int dt, int64_t r
                                    int64_t ld, int64_t row_slab, float *__restrict__ absmax)
 {
     pdl_wait();
-    pdl_launch_dependents();
     const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (j >= cols) return;
     const int64_t r0 = static_cast<int64_t>(blockIdx.y) * row_slab;

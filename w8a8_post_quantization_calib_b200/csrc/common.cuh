@@ -18,15 +18,17 @@ __host__ __device__ constexpr int dtype_size(int dt) { return dt == DT_F32 ? 4 :
 // device (0 = none).  Read and cleared by sq_sync_status.
 __device__ unsigned int g_error_word;
 
-// Programmatic dependent launch.  Every kernel of this library is launched
-// with programmatic stream serialisation: it may start while the previous
-// kernel in the stream is finishing, runs its prologue, and must execute
-// pdl_wait() (all memory of the previous grid complete and visible) before
-// reading any global input.  pdl_launch_dependents() lets the next kernel
-// start its own prologue.  Both are no-ops when the launch was not
-// programmatic.
+// Programmatic dependent launch.  On created streams every kernel of this
+// library is launched with programmatic stream serialisation and executes
+// pdl_wait() before it reads any global input; it may then be scheduled as
+// soon as the previous kernel of the stream completes (no gap for launch
+// processing).  No kernel here triggers its dependents early
+// (griddepcontrol.launch_dependents): measured on B200, global writes a
+// kernel made after that trigger were not visible to a dependent past its
+// griddepcontrol.wait -- a chain of small dependent kernels read stale
+// histograms and prefixes -- so a kernel could only trigger after its last
+// global write, which is no earlier than its completion.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
 // Canonical fp32 steps (round-to-nearest intrinsics so that nvcc never fuses

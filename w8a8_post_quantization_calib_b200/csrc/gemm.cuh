@@ -83,9 +83,10 @@ struct Params {
     int sk_iters, sk_ctas;     // swap path: tiles * num_kb iterations shared by sk_ctas CTAs
     int sk_slot;               // swap path: int32 per partial-sum slot (BM * BN)
     int ring;                  // swap path: shared-memory stages in use (<= STAGES)
-    const float *a_scale;      // [1] or [M]
+    const float *a_scale;      // [1] or [M] (fp16 values when scales_f16)
     int per_token;
-    const float *w_scale;      // [N]
+    const float *w_scale;      // [N] (fp16 values when scales_f16)
+    int scales_f16;            // a_scale / w_scale hold fp16 values (widened exactly on load)
     const void *bias;          // [N] of out_dt or null
     void *out;                 // [M, N] (gate/up: h [M, N/2] or null)
     int out_dt;
@@ -97,6 +98,17 @@ struct Params {
     unsigned long long timeout_ns;
     int inject;                // failure-detection test: 1 = CTA 0 withholds its first stage
 };
+
+// The dequant scales, stored as fp32 or as fp16 (widened exactly).
+__device__ __forceinline__ float load_scale(const float *p, int f16, int64_t i)
+{
+    return f16 ? __half2float(reinterpret_cast<const __half *>(p)[i]) : p[i];
+}
+
+__device__ __forceinline__ float a_scale_of(const Params &p, int64_t m)
+{
+    return load_scale(p.a_scale, p.scales_f16, p.per_token ? m : 0);
+}
 
 // Tile u of the CTA-pair grid in raster-group order (GROUP_R A-row tiles per
 // group, so that consecutive tiles share B tiles in L2).
@@ -196,7 +208,7 @@ __device__ __forceinline__ void epilogue_gateup(const Params &p, const CUtensorM
     const int m = tr * BM + q * 32 + lane;
     const int mrow0 = tr * BM + q * 32;
     const bool mok = m < p.M;
-    const float am = mok ? (p.per_token ? p.a_scale[m] : p.a_scale[0]) : 0.0f;
+    const float am = mok ? a_scale_of(p, m) : 0.0f;
     const int Nh = p.N >> 1;
     const float inv_a2 = p.hq != nullptr ? recip_or_zero(p.a2[0]) : 0.0f;
 #pragma unroll 1
@@ -246,13 +258,17 @@ __device__ __forceinline__ void epilogue_gateup(const Params &p, const CUtensorM
             ++nstore;
         }
         if (p.hq != nullptr && mok) {
+            // s2 == null: 1/s2 was folded into the up rows of the weight (the
+            // cross-layer fold), so h is already smoothed
+            const bool folded = p.s2 == nullptr;
             uint32_t w[8];
 #pragma unroll
             for (int i = 0; i < 32; i += 4) {
                 int qv[4];
 #pragma unroll
                 for (int t = 0; t < 4; ++t)
-                    qv[t] = quant8(__fmul_rn(__fmul_rn(h[i + t], s2inv_tile[c * 32 + i + t]), inv_a2));
+                    qv[t] = folded ? quant8(__fmul_rn(h[i + t], inv_a2))
+                                   : quant8(__fmul_rn(__fmul_rn(h[i + t], s2inv_tile[c * 32 + i + t]), inv_a2));
                 w[i / 4] = pack4(qv[0], qv[1], qv[2], qv[3]);
             }
             uint4 *dst = reinterpret_cast<uint4 *>(p.hq + static_cast<int64_t>(m) * Nh + ch0);
@@ -586,7 +602,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint64_t tmo = p.timeout_ns;
     const int it_begin = sk_begin(p, blockIdx.x), it_end = sk_begin(p, blockIdx.x + 1);
     pdl_wait();                        // operands and scales come from the previous kernels
-    pdl_launch_dependents();
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
@@ -670,7 +685,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const int t = threadIdx.x - 64;
             for (int m = t; m < BN; m += 128) {
                 const int mg = min(m, p.M - 1);
-                s_am[m] = p.per_token ? p.a_scale[mg] : p.a_scale[0];
+                s_am[m] = a_scale_of(p, mg);
             }
             ptx::named_bar_sync(1, 128);
         }
@@ -684,7 +699,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if constexpr (EPI == EPI_DEQUANT) {
                 const int n = tr * BM + q * 32 + lane;
                 if (n < p.N) {
-                    wsn = p.w_scale[n];
+                    wsn = load_scale(p.w_scale, p.scales_f16, n);
                     bn = load_bias(p.bias, p.out_dt, n);
                 }
             }
@@ -923,7 +938,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     const uint32_t tmem_base = *tmem_slot;
     const uint64_t tmo = p.timeout_ns;
     pdl_wait();                        // operands and scales come from the previous kernels
-    pdl_launch_dependents();
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer (both CTAs)
@@ -1035,19 +1049,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 const int et = threadIdx.x - 64;             // 0..127
                 for (int t = et; t < BN; t += 128) {
                     const int n = tc * BN + t;
-                    ws_tile[t] = n < p.N ? p.w_scale[n] : 0.0f;
+                    ws_tile[t] = n < p.N ? load_scale(p.w_scale, p.scales_f16, n) : 0.0f;
                     bias_tile[t] = (n < p.N && p.bias != nullptr) ? load_bias(p.bias, p.out_dt, n) : 0.0f;
                 }
                 const int m = (2 * tr + static_cast<int>(rank)) * BM + q * 32 + lane;
-                if (m < p.M) am = p.per_token ? p.a_scale[m] : p.a_scale[0];
+                if (m < p.M) am = a_scale_of(p, m);
             } else if constexpr (EPI == EPI_GATEUP) {
                 // w_scale of the tile's gate/up rows, fl(1/s2) of its channels
                 const int et = threadIdx.x - 64;
                 for (int t = et; t < BN; t += 128) {
                     const int n = tc * BN + t;
-                    ws_tile[t] = n < p.N ? p.w_scale[n] : 0.0f;
+                    ws_tile[t] = n < p.N ? load_scale(p.w_scale, p.scales_f16, n) : 0.0f;
                 }
-                if (p.hq != nullptr) {
+                if (p.hq != nullptr && p.s2 != nullptr) {
                     for (int t = et; t < BN / 2; t += 128) {
                         const int ch = (tc * BN) / 2 + t;
                         bias_tile[t] = ch < (p.N >> 1) ? recip_or_zero(p.s2[ch]) : 0.0f;

@@ -6,6 +6,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -16,6 +17,7 @@
 #include "common.cuh"
 #include "ptx_sm100.cuh"
 #include "calib.cuh"
+#include "robust.cuh"
 #include "quant.cuh"
 #include "gemm.cuh"
 
@@ -63,6 +65,15 @@ int sm_count()
 
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// Programmatic dependent launch is used only on explicitly created streams;
+// on the legacy and per-thread default streams launches go without the
+// attribute (plain stream order), which is where the chains that first showed
+// the early-trigger hazard (see pdl_wait in common.cuh) ran.
+inline bool pdl_stream(cudaStream_t st)
+{
+    return st != nullptr && st != cudaStreamLegacy && st != cudaStreamPerThread;
+}
+
 // Launch with programmatic stream serialisation (see pdl_wait in common.cuh):
 // the kernel may begin while the previous kernel of the stream drains.
 template <typename... KArgs, typename... Args>
@@ -77,7 +88,7 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl_stream(st) ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
@@ -93,14 +104,14 @@ cudaError_t launch_pdl_cluster_smem(void (*kern)(KArgs...), dim3 grid, dim3 bloc
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    attr[1].id = cudaLaunchAttributeClusterDimension;
-    attr[1].val.clusterDim.x = cluster_x;
-    attr[1].val.clusterDim.y = 1;
-    attr[1].val.clusterDim.z = 1;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cluster_x;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 2;
+    cfg.numAttrs = pdl_stream(st) ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
@@ -762,6 +773,104 @@ static sq_status smooth_scales_q(const float *act_max, const float *w_max, int64
     return check_launch();
 }
 
+sq_status sq_calib_batchmax_accumulate(const void *x, sq_dtype dt, int64_t rows, int64_t cols, int64_t ld,
+                                       float *batch_max, double *sum_max, sq_stream stream)
+{
+    if (x == nullptr || batch_max == nullptr || sum_max == nullptr || !valid_dt(dt)) return SQ_ERR_INVALID_ARG;
+    if (rows <= 0 || cols <= 0 || ld < cols) return SQ_ERR_INVALID_ARG;
+    sq_status r = sq_calib_absmax(x, dt, rows, cols, ld, batch_max, stream);
+    if (r != SQ_OK) return r;
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(cdiv(cols, 256), sm_count()));
+    const cudaError_t e = launch_pdl(k_batchmax_accumulate, dim3(static_cast<unsigned>(grid)), dim3(256), 0,
+                                     as_stream(stream), batch_max, sum_max, cols);
+    return e == cudaSuccess ? check_launch() : cuda_fail(e);
+}
+
+sq_status sq_calib_mean_of_max(const double *sum_max, int64_t cols, int64_t n_batches, float *out, sq_stream stream)
+{
+    if (sum_max == nullptr || out == nullptr || cols <= 0 || n_batches <= 0) return SQ_ERR_INVALID_ARG;
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(cdiv(cols, 256), sm_count()));
+    const cudaError_t e = launch_pdl(k_mean_of_max, dim3(static_cast<unsigned>(grid)), dim3(256), 0,
+                                     as_stream(stream), sum_max, cols, static_cast<double>(n_batches), out);
+    return e == cudaSuccess ? check_launch() : cuda_fail(e);
+}
+
+static size_t quantile_ws_layout(int64_t cols, size_t off[3])
+{
+    size_t o = 0;
+    off[0] = o; o = align_up(o + static_cast<size_t>(cols) * QH_BINS * 4, 256);    // histograms
+    off[1] = o; o = align_up(o + static_cast<size_t>(cols) * 4, 256);              // prefixes
+    off[2] = o; o = align_up(o + static_cast<size_t>(cols) * 4, 256);              // remaining ranks
+    return o;
+}
+
+size_t sq_calib_quantile_workspace_size(int64_t cols)
+{
+    if (cols <= 0) return 0;
+    size_t off[3];
+    return quantile_ws_layout(cols, off);
+}
+
+extern "C++" {
+template <int DT>
+static sq_status quantile_dt(const void *x, int64_t rows, int64_t cols, int64_t ld, uint32_t k, float *out,
+                             uint8_t *ws, const size_t off[3], cudaStream_t st)
+{
+    constexpr int EPV = VecT<DT>::EPV;
+    uint32_t *hist = reinterpret_cast<uint32_t *>(ws + off[0]);
+    uint32_t *prefix = reinterpret_cast<uint32_t *>(ws + off[1]);
+    uint32_t *krem = reinterpret_cast<uint32_t *>(ws + off[2]);
+    cudaError_t e = cudaMemsetAsync(hist, 0, static_cast<size_t>(cols) * QH_BINS * 4, st);
+    if (e != cudaSuccess) return cuda_fail(e);
+    auto hk = k_quantile_hist<DT>;
+    e = ensure_smem(reinterpret_cast<const void *>(hk), QH_SMEM);
+    if (e != cudaSuccess) return cuda_fail(e);
+    constexpr int LANES = QH_THREADS / (QH_COLS / EPV);
+    const int64_t gx = cdiv(cols, QH_COLS);
+    int64_t gy = std::max<int64_t>(1, std::min<int64_t>(cdiv(rows, LANES * QH_UNROLL), cdiv(2 * sm_count(), gx)));
+    gy = std::min<int64_t>(gy, 65535);
+    const int64_t slab = cdiv(rows, gy);
+    gy = cdiv(rows, slab);
+    const int64_t ldb = ld * dtype_size(DT);
+    // digits of the magnitude bits, most significant first: (shift, width)
+    const int nd = DT == DT_F32 ? 4 : 2;
+    const int shifts[4] = {DT == DT_F32 ? 23 : 7, DT == DT_F32 ? 15 : 0, 7, 0};
+    const int widths[4] = {8, DT == DT_F32 ? 8 : 7, 8, 7};
+    const unsigned sel_grid = static_cast<unsigned>(cdiv(cols * 32, 256));
+    for (int i = 0; i < nd; ++i) {
+        e = launch_pdl(hk, dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy)), dim3(QH_THREADS),
+                       static_cast<size_t>(QH_SMEM), st, static_cast<const uint8_t *>(x), rows, cols, ldb, slab,
+                       shifts[i], widths[i], i == 0 ? static_cast<const uint32_t *>(nullptr) : prefix, hist);
+        if (e != cudaSuccess) return cuda_fail(e);
+        e = launch_pdl(k_quantile_select<DT>, dim3(sel_grid), dim3(256), 0, st, hist, cols, widths[i], k,
+                       i == 0 ? 1 : 0, i == nd - 1 ? 1 : 0, prefix, krem, out);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    return check_launch();
+}
+}  // extern "C++"
+
+sq_status sq_calib_quantile(const void *x, sq_dtype dt, int64_t rows, int64_t cols, int64_t ld, double p, float *out,
+                            void *workspace, size_t workspace_bytes, sq_stream stream)
+{
+    if (x == nullptr || out == nullptr || !valid_dt(dt)) return SQ_ERR_INVALID_ARG;
+    if (rows <= 0 || rows >= (int64_t(1) << 32) || cols <= 0 || ld < cols) return SQ_ERR_INVALID_ARG;
+    if (!(p > 0.0 && p <= 1.0)) return SQ_ERR_INVALID_ARG;
+    size_t off[3];
+    const size_t need = quantile_ws_layout(cols, off);
+    if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)) return SQ_ERR_WORKSPACE;
+    const int elt = dtype_size(dt);
+    if (!aligned16(x) || (cols * elt) % 16 != 0 || (ld * elt) % 16 != 0) return SQ_ERR_MISALIGNED;
+    // nearest rank: k = ceil(p * T) in fp64, within [1, T]
+    const double kd = std::ceil(p * static_cast<double>(rows));
+    const uint32_t k = static_cast<uint32_t>(std::min<double>(static_cast<double>(rows), std::max(1.0, kd)));
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const cudaStream_t st = as_stream(stream);
+    if (dt == SQ_F32) return quantile_dt<DT_F32>(x, rows, cols, ld, k, out, ws, off, st);
+    if (dt == SQ_F16) return quantile_dt<DT_F16>(x, rows, cols, ld, k, out, ws, off, st);
+    return quantile_dt<DT_BF16>(x, rows, cols, ld, k, out, ws, off, st);
+}
+
 sq_status sq_smooth_scales(const float *act_max, const float *w_max, int64_t K, float alpha, float *s,
                            float *a_static, sq_stream stream)
 {
@@ -806,8 +915,46 @@ sq_status sq_quant_weight_fp8(const void *w, sq_dtype dt, int64_t N, int64_t K, 
     return quant_weight_impl<ROW_FP8>(w, dt, N, K, s, reinterpret_cast<int8_t *>(wq8), w_scale, stream);
 }
 
+sq_status sq_quant_weight_fold(const void *w, sq_dtype dt, int64_t N, int64_t K, const float *s, const float *s_next,
+                               int8_t *wq, float *w_scale, sq_stream stream)
+{
+    if (w == nullptr || s == nullptr || s_next == nullptr || wq == nullptr || w_scale == nullptr || !valid_dt(dt))
+        return SQ_ERR_INVALID_ARG;
+    if (N < 0 || K <= 0) return SQ_ERR_INVALID_ARG;
+    if (!aligned16(w) || !aligned16(wq)) return SQ_ERR_MISALIGNED;
+    RowArgs a{};
+    a.src0 = static_cast<const uint8_t *>(w);
+    a.rows = N;
+    a.K = K;
+    a.row_bytes = K * dtype_size(dt);
+    a.s = s;
+    a.fold_s = s_next;
+    a.scale_out = w_scale;
+    a.out = wq;
+    return launch_rows<ROW_WEIGHT | ROW_FOLD>(a, dt, as_stream(stream));
+}
+
+static sq_status quant_weight_gateup_impl(const void *w_gate, const void *w_up, sq_dtype dt, int64_t N_h, int64_t K,
+                                          const float *s, const float *s_next, int8_t *wq_gu, float *w_scale_gu,
+                                          sq_stream stream);
+
 sq_status sq_quant_weight_gateup(const void *w_gate, const void *w_up, sq_dtype dt, int64_t N_h, int64_t K,
                                  const float *s, int8_t *wq_gu, float *w_scale_gu, sq_stream stream)
+{
+    return quant_weight_gateup_impl(w_gate, w_up, dt, N_h, K, s, nullptr, wq_gu, w_scale_gu, stream);
+}
+
+sq_status sq_quant_weight_gateup_fold(const void *w_gate, const void *w_up, sq_dtype dt, int64_t N_h, int64_t K,
+                                      const float *s, const float *s_next, int8_t *wq_gu, float *w_scale_gu,
+                                      sq_stream stream)
+{
+    if (s_next == nullptr) return SQ_ERR_INVALID_ARG;
+    return quant_weight_gateup_impl(w_gate, w_up, dt, N_h, K, s, s_next, wq_gu, w_scale_gu, stream);
+}
+
+static sq_status quant_weight_gateup_impl(const void *w_gate, const void *w_up, sq_dtype dt, int64_t N_h, int64_t K,
+                                          const float *s, const float *s_next, int8_t *wq_gu, float *w_scale_gu,
+                                          sq_stream stream)
 {
     if (w_gate == nullptr || w_up == nullptr || s == nullptr || wq_gu == nullptr || w_scale_gu == nullptr ||
         !valid_dt(dt))
@@ -821,8 +968,10 @@ sq_status sq_quant_weight_gateup(const void *w_gate, const void *w_up, sq_dtype 
     a.K = K;
     a.row_bytes = K * dtype_size(dt);
     a.s = s;
+    a.fold_s = s_next;
     a.scale_out = w_scale_gu;
     a.out = wq_gu;
+    if (s_next != nullptr) return launch_rows<ROW_WEIGHT | ROW_FOLD>(a, dt, as_stream(stream));
     return launch_rows<ROW_WEIGHT>(a, dt, as_stream(stream));
 }
 
@@ -949,15 +1098,11 @@ static sq_status check_gemm_shape(const int8_t *xq, const int8_t *wq, int64_t M,
     return SQ_OK;
 }
 
-sq_status sq_linear_w8a8(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, int64_t K, const float *a_scale,
-                         sq_act_mode mode, const float *w_scale, const void *bias, sq_dtype out_dt, void *y,
-                         void *workspace, size_t workspace_bytes, sq_stream stream)
+static sq_status linear_w8a8_impl(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, int64_t K,
+                                  const float *a_scale, sq_act_mode mode, const float *w_scale, int scales_f16,
+                                  const void *bias, sq_dtype out_dt, void *y, void *workspace,
+                                  size_t workspace_bytes, sq_stream stream)
 {
-    sq_status r = check_gemm_shape(xq, wq, M, N, K);
-    if (r != SQ_OK) return r;
-    if (a_scale == nullptr || w_scale == nullptr || y == nullptr || !valid_dt(out_dt)) return SQ_ERR_INVALID_ARG;
-    if (mode != SQ_ACT_STATIC && mode != SQ_ACT_PER_TOKEN) return SQ_ERR_INVALID_ARG;
-    if (!aligned16(y) || !aligned16(w_scale)) return SQ_ERR_MISALIGNED;
     const cudaStream_t st = as_stream(stream);
     gemm::Params p{};
     p.M = static_cast<int>(M);
@@ -966,6 +1111,7 @@ sq_status sq_linear_w8a8(const int8_t *xq, const int8_t *wq, int64_t M, int64_t 
     p.a_scale = a_scale;
     p.per_token = (mode == SQ_ACT_PER_TOKEN) ? 1 : 0;
     p.w_scale = w_scale;
+    p.scales_f16 = scales_f16;
     p.bias = bias;
     p.out = y;
     p.out_dt = out_dt;
@@ -983,6 +1129,19 @@ sq_status sq_linear_w8a8(const int8_t *xq, const int8_t *wq, int64_t M, int64_t 
         return dispatch_swap<gemm::EPI_DEQUANT>(p, xq, wq, st, tiles);
     }
     return dispatch_pair<gemm::KIND_I8, gemm::EPI_DEQUANT>(p, xq, wq, st);
+}
+
+sq_status sq_linear_w8a8(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, int64_t K, const float *a_scale,
+                         sq_act_mode mode, const float *w_scale, const void *bias, sq_dtype out_dt, void *y,
+                         void *workspace, size_t workspace_bytes, sq_stream stream)
+{
+    sq_status r = check_gemm_shape(xq, wq, M, N, K);
+    if (r != SQ_OK) return r;
+    if (a_scale == nullptr || w_scale == nullptr || y == nullptr || !valid_dt(out_dt)) return SQ_ERR_INVALID_ARG;
+    if (mode != SQ_ACT_STATIC && mode != SQ_ACT_PER_TOKEN) return SQ_ERR_INVALID_ARG;
+    if (!aligned16(y) || !aligned16(w_scale)) return SQ_ERR_MISALIGNED;
+    return linear_w8a8_impl(xq, wq, M, N, K, a_scale, mode, w_scale, 0, bias, out_dt, y, workspace, workspace_bytes,
+                            stream);
 }
 
 sq_status sq_linear_fp8(const uint8_t *xq8, const uint8_t *wq8, int64_t M, int64_t N, int64_t K,
@@ -1006,6 +1165,42 @@ sq_status sq_linear_fp8(const uint8_t *xq8, const uint8_t *wq8, int64_t M, int64
     p.out = y;
     p.out_dt = out_dt;
     return dispatch_pair<gemm::KIND_F8, gemm::EPI_DEQUANT>(p, xq8, wq8, as_stream(stream));
+}
+
+sq_status sq_scales_to_f16(const float *in, int64_t n, uint16_t *out, sq_stream stream)
+{
+    if (in == nullptr || out == nullptr || n < 0) return SQ_ERR_INVALID_ARG;
+    if (n == 0) return SQ_OK;
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(cdiv(n, 256), 4 * sm_count()));
+    const cudaError_t e = launch_pdl(k_f32_to_f16, dim3(static_cast<unsigned>(grid)), dim3(256), 0, as_stream(stream),
+                                     in, n, reinterpret_cast<__half *>(out));
+    return e == cudaSuccess ? check_launch() : cuda_fail(e);
+}
+
+sq_status sq_scales_from_f16(const uint16_t *in, int64_t n, float *out, sq_stream stream)
+{
+    if (in == nullptr || out == nullptr || n < 0) return SQ_ERR_INVALID_ARG;
+    if (n == 0) return SQ_OK;
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(cdiv(n, 256), 4 * sm_count()));
+    const cudaError_t e = launch_pdl(k_f16_to_f32, dim3(static_cast<unsigned>(grid)), dim3(256), 0, as_stream(stream),
+                                     reinterpret_cast<const __half *>(in), n, out);
+    return e == cudaSuccess ? check_launch() : cuda_fail(e);
+}
+
+sq_status sq_linear_w8a8_f16scales(const int8_t *xq, const int8_t *wq, int64_t M, int64_t N, int64_t K,
+                                   const uint16_t *a_scale_f16, sq_act_mode mode, const uint16_t *w_scale_f16,
+                                   const void *bias, sq_dtype out_dt, void *y, void *workspace,
+                                   size_t workspace_bytes, sq_stream stream)
+{
+    sq_status r = check_gemm_shape(xq, wq, M, N, K);
+    if (r != SQ_OK) return r;
+    if (a_scale_f16 == nullptr || w_scale_f16 == nullptr || y == nullptr || !valid_dt(out_dt))
+        return SQ_ERR_INVALID_ARG;
+    if (mode != SQ_ACT_STATIC && mode != SQ_ACT_PER_TOKEN) return SQ_ERR_INVALID_ARG;
+    if (!aligned16(y) || !aligned16(w_scale_f16)) return SQ_ERR_MISALIGNED;
+    return linear_w8a8_impl(xq, wq, M, N, K, reinterpret_cast<const float *>(a_scale_f16), mode,
+                            reinterpret_cast<const float *>(w_scale_f16), 1, bias, out_dt, y, workspace,
+                            workspace_bytes, stream);
 }
 
 size_t sq_linear_w8a8_noalloc_max_elems(void) { return kNoAllocAccBytes / 4; }
@@ -1080,7 +1275,7 @@ sq_status sq_linear_w8a8_gateup_silu(const int8_t *xq, const int8_t *wq_gu, int6
     if (r != SQ_OK) return r;
     if (a_scale == nullptr || w_scale_gu == nullptr || (h == nullptr && hq == nullptr)) return SQ_ERR_INVALID_ARG;
     if ((N_h % 128) != 0) return SQ_ERR_INVALID_ARG;
-    if (hq != nullptr && (s2 == nullptr || a2 == nullptr)) return SQ_ERR_INVALID_ARG;
+    if (hq != nullptr && a2 == nullptr) return SQ_ERR_INVALID_ARG;     // s2 == null: folded into W_up
     if (mode != SQ_ACT_STATIC && mode != SQ_ACT_PER_TOKEN) return SQ_ERR_INVALID_ARG;
     if ((h != nullptr && !aligned16(h)) || (hq != nullptr && !aligned16(hq))) return SQ_ERR_MISALIGNED;
     gemm::Params p{};

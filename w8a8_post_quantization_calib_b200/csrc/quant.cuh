@@ -51,7 +51,6 @@ __global__ void __cluster_dims__(8, 1, 1) __launch_bounds__(1024)
     const int j = blockIdx.x * blockDim.x + threadIdx.x;
     float m = 0.0f;
     pdl_wait();
-    pdl_launch_dependents();
     if (j < K) {
         const float am = act_max[j];
         const float sj = smoothing_factor(am, w_max[j], static_cast<double>(alpha));
@@ -83,7 +82,6 @@ __global__ void __launch_bounds__(1024)
     const double al = static_cast<double>(alpha);
     float m = 0.0f;
     pdl_wait();
-    pdl_launch_dependents();
     for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < K;
          j += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const float sj = smoothing_factor(act_max[j], w_max[j], al);
@@ -112,6 +110,11 @@ enum RowMode : int {
 // Added to ROW_WEIGHT / ROW_ACT_STATIC / ROW_ACT_TOKEN: E4M3 codes and
 // absmax / 448 scales instead of INT8 codes and absmax / 127.
 constexpr int ROW_FP8 = 8;
+// Added to ROW_WEIGHT: the cross-layer fold.  Row n of the weight is first
+// multiplied by fl(1/s_next) of the channel it feeds in the next layer
+// (fold_s[n]; for the gate/up interleave only the up rows, fold_s indexed by
+// channel), W'[n,j] = fl(fl(W[n,j] * recip(s_next_n)) * s_j).
+constexpr int ROW_FOLD = 16;
 constexpr int ROW_MODE_MASK = 7;
 
 constexpr int ROW_T = 256;
@@ -131,7 +134,19 @@ struct RowArgs {
     float *rstd_out;         // RMSNorm r_m [rows] or null
     int8_t *out;             // codes [rows, K]
     unsigned long long timeout_ns;   // bound of the row-ring waits
+    const float *fold_s;     // ROW_FOLD: the next layer's smoothing factors of the folded rows
 };
+
+// fl(1/s_next) of output row `row` under ROW_FOLD (1 for the gate rows of the
+// gate/up interleave, which feed no smoothed layer directly: fl(x * 1) = x)
+__device__ __forceinline__ float row_fold_factor(const RowArgs &p, int64_t row)
+{
+    if (p.src1 != nullptr) {
+        const int64_t w = row & 63;
+        return w < 32 ? 1.0f : recip_or_zero(p.fold_s[((row >> 6) << 5) + (w & 31)]);
+    }
+    return recip_or_zero(p.fold_s[row]);
+}
 
 // Rows in flight per block in the shared-memory row ring of k_rows, and the
 // error code a timed-out ring wait records.
@@ -219,6 +234,7 @@ __global__ void __launch_bounds__(NT) k_rows(RowArgs p)
 {
     constexpr int MODE = MODEF & ROW_MODE_MASK;
     constexpr bool F8 = (MODEF & ROW_FP8) != 0;
+    constexpr bool FOLD = (MODEF & ROW_FOLD) != 0;
     constexpr int EPV = VecT<DT>::EPV;
     constexpr bool REG = (VPT * EPV <= 32);
     static_assert(!RING || (REG && MODE != ROW_ACT_STATIC), "the row ring needs register rows and a row barrier");
@@ -245,7 +261,6 @@ __global__ void __launch_bounds__(NT) k_rows(RowArgs p)
         __syncthreads();
     }
     pdl_wait();
-    pdl_launch_dependents();
 
     auto row_src = [&](int64_t row) -> const uint8_t * {
         if (p.src1 != nullptr) {          // gate/up interleave: blocks of 64 output rows
@@ -480,6 +495,7 @@ __global__ void __launch_bounds__(NT) k_rows(RowArgs p)
         // pass 2 codes of fl(y * recip(scale)).  REG keeps y in registers.
         float ykeep[REG ? VPT : 1][REG ? EPV : 1];
         float mx = 0.0f;
+        const float rf = FOLD ? row_fold_factor(p, row) : 1.0f;
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
             const int64_t v = static_cast<int64_t>(i) * NT + tid;
@@ -488,7 +504,7 @@ __global__ void __launch_bounds__(NT) k_rows(RowArgs p)
             colc(i, v, c);
 #pragma unroll
             for (int e = 0; e < EPV; ++e) {
-                const float y = __fmul_rn(f[e], c[e]);
+                const float y = __fmul_rn(FOLD ? __fmul_rn(f[e], rf) : f[e], c[e]);
                 mx = fmaxf(mx, fabsf(y));
                 if constexpr (REG) ykeep[i][e] = y;
             }
@@ -511,7 +527,7 @@ __global__ void __launch_bounds__(NT) k_rows(RowArgs p)
                 widen<DT>(raw[i], f);
                 colc(i, v, c);
 #pragma unroll
-                for (int e = 0; e < EPV; ++e) f[e] = __fmul_rn(__fmul_rn(f[e], c[e]), inv);
+                for (int e = 0; e < EPV; ++e) f[e] = __fmul_rn(__fmul_rn(FOLD ? __fmul_rn(f[e], rf) : f[e], c[e]), inv);
             }
             if (v < nvec) {
                 if (F8) store_codes<EPV, false, F8>(dst, v, f);
@@ -590,7 +606,6 @@ __global__ void __launch_bounds__(QS_TX *QS_TY)
     const int64_t r1 = min(rows, r0 + row_slab);
     const int64_t K = nvec * EPV;
     pdl_wait();
-    pdl_launch_dependents();
     if (v >= nvec) return;
     const uint8_t *col = x + v * 16;
     auto load = [&](int64_t r) {
@@ -682,6 +697,7 @@ __global__ void __launch_bounds__(ROW_T) k_rows_split(RowArgs p)
 {
     constexpr int MODE = MODEF & ROW_MODE_MASK;
     constexpr bool F8 = (MODEF & ROW_FP8) != 0;
+    constexpr bool FOLD = (MODEF & ROW_FOLD) != 0;
     constexpr int EPV = VecT<DT>::EPV;
     __shared__ float red[32];
     __shared__ double red64[32];
@@ -696,7 +712,6 @@ __global__ void __launch_bounds__(ROW_T) k_rows_split(RowArgs p)
     const int64_t v = static_cast<int64_t>(rank) * vpc + tid;
     const bool act = tid < vpc;
     pdl_wait();
-    pdl_launch_dependents();
 
     const uint8_t *src;
     if (p.src1 != nullptr) {
@@ -777,9 +792,10 @@ __global__ void __launch_bounds__(ROW_T) k_rows_split(RowArgs p)
     } else {
         // ROW_WEIGHT / ROW_ACT_TOKEN: y = fl(x * c_j), row absmax, codes of fl(y * recip(scale))
         float mx = 0.0f;
+        const float rf = FOLD ? row_fold_factor(p, row) : 1.0f;
 #pragma unroll
         for (int e = 0; e < EPV; ++e) {
-            f[e] = __fmul_rn(f[e], c[e]);
+            f[e] = __fmul_rn(FOLD ? __fmul_rn(f[e], rf) : f[e], c[e]);
             mx = fmaxf(mx, fabsf(f[e]));
         }
         const float rmax = static_cast<float>(cluster_combine(static_cast<double>(block_max(mx, red)), true));
@@ -803,11 +819,11 @@ __global__ void __launch_bounds__(ROW_T) k_rows_scalar(RowArgs p, int dt)
 {
     constexpr int MODE = MODEF & ROW_MODE_MASK;
     constexpr bool F8 = (MODEF & ROW_FP8) != 0;
+    constexpr bool FOLD = (MODEF & ROW_FOLD) != 0;
     __shared__ float red[32];
     __shared__ double red64[32];
     const int tid = threadIdx.x;
     pdl_wait();
-    pdl_launch_dependents();
     float inv_a_static = 0.0f;
     if constexpr (MODE == ROW_ACT_STATIC || MODE == ROW_RMSNORM) inv_a_static = recip_or_zero(p.a_in[0]);
     for (int64_t row = blockIdx.x; row < p.rows; row += gridDim.x) {
@@ -826,9 +842,10 @@ __global__ void __launch_bounds__(ROW_T) k_rows_scalar(RowArgs p, int dt)
         };
         float stat = 0.0f;
         double ss = 0.0;
+        const float rf = FOLD ? row_fold_factor(p, row) : 1.0f;
         if constexpr (MODE != ROW_ACT_STATIC) {
             for (int64_t j = tid; j < p.K; j += ROW_T) {
-                const float x = load_elem_dt(src, dt, j);
+                const float x = FOLD ? __fmul_rn(load_elem_dt(src, dt, j), rf) : load_elem_dt(src, dt, j);
                 if constexpr (MODE == ROW_RMSNORM || MODE == ROW_RMS_STAT)
                     ss += static_cast<double>(x) * static_cast<double>(x);
                 else stat = fmaxf(stat, fabsf(__fmul_rn(x, colc(j))));
@@ -849,7 +866,7 @@ __global__ void __launch_bounds__(ROW_T) k_rows_scalar(RowArgs p, int dt)
             if (tid == 0) p.scale_out[row] = sc;
         }
         for (int64_t j = tid; j < p.K; j += ROW_T) {
-            const float x = load_elem_dt(src, dt, j);
+            const float x = FOLD ? __fmul_rn(load_elem_dt(src, dt, j), rf) : load_elem_dt(src, dt, j);
             float y;
             if constexpr (MODE == ROW_RMSNORM || MODE == ROW_RMS_STAT) y = __fmul_rn(__fmul_rn(x, r_m), colc(j));
             else y = __fmul_rn(x, colc(j));
@@ -865,6 +882,26 @@ __global__ void __launch_bounds__(ROW_T) k_rows_scalar(RowArgs p, int dt)
 }
 
 // ---------------------------------------------------------------------------
+// fp16 storage of scales ("010. SmoothQuant Integration", consequences:
+// storage): fp32 -> fp16 round to nearest even, and the exact widening back.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_f32_to_f16(const float *__restrict__ in, int64_t n, __half *__restrict__ out)
+{
+    pdl_wait();
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+        out[i] = __float2half_rn(in[i]);
+}
+
+__global__ void __launch_bounds__(256) k_f16_to_f32(const __half *__restrict__ in, int64_t n, float *__restrict__ out)
+{
+    pdl_wait();
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+        out[i] = __half2float(in[i]);
+}
+
+// ---------------------------------------------------------------------------
 // Sum of squared differences of two fp16 tensors, fp64 accumulation.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
@@ -874,7 +911,6 @@ __global__ void __launch_bounds__(256)
     double acc = 0.0;
     const int64_t nv = n / 8;
     pdl_wait();
-    pdl_launch_dependents();
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < nv; v += stride) {
         const uint4 a = __ldg(reinterpret_cast<const uint4 *>(y) + v);
