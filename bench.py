@@ -85,16 +85,16 @@ def tensor_peak(kind: str = "i8", clk=None) -> dict:
     return out
 
 
-def traffic_from_profile(name: str, sources=("gemm.cuh", "ptx_sm100.cuh", "libsq.cu")):
+def traffic_from_profile(name: str):
     """DRAM bytes per launch of a kernel from a committed ncu summary
-    (profiles/<name>.json), or None when the kernel source changed after the
-    counters were taken."""
+    (profiles/<name>.json), or None when the kernel's source files (listed
+    there) changed after the counters were taken."""
     import hashlib
     tf = os.path.join(ROOT, "profiles", name + ".json")
     try:
         d = json.load(open(tf))
         h = hashlib.sha256()
-        for f in sources:
+        for f in d.get("sources", ("gemm.cuh", "ptx_sm100.cuh", "libsq.cu")):
             h.update(open(os.path.join(ROOT, "w8a8_post_quantization_calib_b200", "csrc", f), "rb").read())
         if h.hexdigest()[:16] != d["source_sha256_16"]:
             return None
