@@ -435,6 +435,19 @@ sq_status sq_linear_fp8(const uint8_t *xq8, const uint8_t *wq8, int64_t M, int64
                         const float *a_scale, sq_act_mode mode, const float *w_scale,
                         const void *bias, sq_dtype out_dt, void *y, sq_stream stream);
 
+/* The calibration statistic of h for the next linear, taken in the same
+ * epilogue instead of writing h (kwkr 3.1: statistics per layer on the
+ * layer's own input; h is the down projection's input):
+ *
+ *   h_absmax[c] = max(h_absmax[c], max_m |h[m,c]|),  h as in sq_linear_w8a8_gateup_silu
+ *
+ * (the bf16-rounded h, so the result equals sq_calib_absmax on the h that
+ * sq_linear_w8a8_gateup_silu writes).  h_absmax: fp32 [N_h], a running max
+ * the caller zeroes once.  Nothing else is written.  N_h a multiple of 128. */
+sq_status sq_linear_w8a8_gateup_silu_absmax(const int8_t *xq, const int8_t *wq_gu, int64_t M, int64_t N_h,
+                                            int64_t K, const float *a_scale, sq_act_mode mode,
+                                            const float *w_scale_gu, float *h_absmax, sq_stream stream);
+
 /* -------------------------------------------------------------------------
  * Per-layer alpha search (adr-010 key design point 2: pick, per layer, the
  * alpha of a small grid with the least output reconstruction error, using the

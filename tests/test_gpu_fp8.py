@@ -2,7 +2,8 @@
 "SmoothQuant 和激活量化": the smoothing carries over to FP8 tensor cores).
 
 Quantisers: given the oracle's s (and static scale), the E4M3 codes and the
-per-row / per-token scales are bit-exact.  GEMM: the tensor cores sum the
+per-row / per-token scales are bit-exact.  GEMM (CTA pairs for M > 128, the
+weight-streaming kernel with or without the cluster split below): the tensor cores sum the
 exact E4M3 products in fp32 in an unspecified order, so y is compared with
 the exact product (oracle.gemm_fp8_f64, fp64) within the fp32 summation
 bound K * 2^-24 * sum_k |x_k w_k| times the dequant factor, plus the
@@ -116,7 +117,8 @@ def _check_fp8_gemm(xq, wq, a, mode, ws, bias32, out_dt, y):
 
 
 @pytest.mark.parametrize("M,N,K", [(300, 528, 1040), (129, 256, 4096), (16, 1024, 2048), (1, 512, 1024),
-                                   (512, 768, 11008)])
+                                   (512, 768, 11008), (1, 4096, 11008), (64, 1024, 4096), (128, 2048, 2048),
+                                   (33, 11008, 4096)])
 @pytest.mark.parametrize("out_dt", [F32, F16, BF16])
 def test_linear_fp8(M, N, K, out_dt):
     g = np.random.default_rng(M * 7 + N + K + out_dt)

@@ -91,7 +91,8 @@ def test_smooth_scales(alpha, K):
 
 # ------------------------------------------------------------------ a4
 @pytest.mark.parametrize("dt", [F32, F16, BF16])
-@pytest.mark.parametrize("N,K", [(300, 4096), (64, 5120), (3, 40), (17, 28672), (130, 1000)])
+@pytest.mark.parametrize("N,K", [(300, 4096), (64, 5120), (3, 40), (17, 28672), (130, 1000), (300, 28672),
+                                 (150, 20000)])
 def test_quant_weight(dt, N, K):
     W = rand_x(N + K, (N, K), dt, 0.02)
     s = (np.abs(np.random.default_rng(K).standard_normal(K)) + 0.05).astype(np.float32)
@@ -136,7 +137,8 @@ def test_quant_weight_gateup_interleave(dt):
 
 # ------------------------------------------------------------------ a5 / a5'
 @pytest.mark.parametrize("dt", [F32, F16, BF16])
-@pytest.mark.parametrize("M,K", [(1, 4096), (300, 4096), (7, 11008), (5, 1024), (3, 40), (129, 5120)])
+@pytest.mark.parametrize("M,K", [(1, 4096), (300, 4096), (7, 11008), (5, 1024), (3, 40), (129, 5120),
+                                 (200, 20000)])
 @pytest.mark.parametrize("mode", [oracle.STATIC, oracle.PER_TOKEN])
 def test_smooth_quant_act(dt, M, K, mode):
     X = rand_x(M * 3 + K, (M, K), dt, 2.0, outliers=min(8, K // 10))

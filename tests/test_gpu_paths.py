@@ -280,3 +280,40 @@ def test_chains_on_a_created_stream_equal_the_default_stream():
             assert torch.equal(g.view(torch.uint8), r.view(torch.uint8))
     q_r = oracle.calib_quantile([oracle.to_f32(np.concatenate(wl.calib), F16)], 0.999, F32)
     assert bits_equal(host(ref[6]), q_r)
+
+
+# ------------------------------------------------------------------ the h statistic in the gate/up epilogue
+@pytest.mark.parametrize("M,Nh,K,mode", [(300, 256, 1024, oracle.STATIC), (1000, 384, 512, oracle.PER_TOKEN),
+                                         (4096, 128, 2048, oracle.STATIC)])
+def test_gateup_h_absmax_equals_the_statistic_of_h(M, Nh, K, mode):
+    """sq_linear_w8a8_gateup_silu_absmax keeps the column max of |h| in the
+    epilogue instead of writing h; it equals sq_calib_absmax over the h that
+    sq_linear_w8a8_gateup_silu writes, bit for bit (both see the same
+    bf16-rounded h), as a running max over two calls."""
+    g = np.random.default_rng(M + Nh)
+    A = g.integers(-127, 128, (M, K), dtype=np.int8)
+    B = g.integers(-127, 128, (2 * Nh, K), dtype=np.int8)
+    a = (np.abs(g.standard_normal(1 if mode == oracle.STATIC else M)) * 2e-3 + 1e-4).astype(np.float32)
+    ws = (np.abs(g.standard_normal(2 * Nh)) * 1e-3 + 1e-4).astype(np.float32)
+    At, Bt, at, wst = dev(A), dev(B), dev(a), dev(ws)
+    h = torch.empty(M, Nh, dtype=torch.bfloat16, device="cuda")
+    sq.linear_w8a8_gateup_silu(At, Bt, at, mode, wst, h=h)
+    ref = torch.zeros(Nh, dtype=torch.float32, device="cuda")
+    sq.calib_absmax(h, ref)
+    got = torch.zeros(Nh, dtype=torch.float32, device="cuda")
+    sq.linear_w8a8_gateup_silu_absmax(At, Bt, at, mode, wst, got)
+    _sync()
+    assert torch.equal(got, ref)
+    # a running max: a second batch (the first half of the rows) changes nothing, a scaled one raises it
+    half = M // 2
+    sq.linear_w8a8_gateup_silu_absmax(At[:half].contiguous(), Bt, at[:1] if mode == oracle.STATIC else at[:half],
+                                      mode, wst, got)
+    _sync()
+    assert torch.equal(got, ref)
+    # and against the oracle on the whole batch
+    order = _gateup_order(Nh)
+    inv = np.argsort(order)
+    gv = oracle.dequant_f32(oracle.gemm_s32(A, B[inv][:Nh]), a, mode, ws[inv][:Nh])
+    uv = oracle.dequant_f32(oracle.gemm_s32(A, B[inv][Nh:]), a, mode, ws[inv][Nh:])
+    h_ref = np.abs(oracle.to_f32(oracle.silu_mul_bf16(gv, uv), BF16)).max(axis=0)
+    assert np.all(np.abs(host(got) - h_ref) <= h_ref * 2.0 ** -6 + 1e-30)

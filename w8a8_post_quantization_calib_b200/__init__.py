@@ -47,7 +47,7 @@ EXPORTS = (
     "sq_smooth_scales_fp8", "sq_quant_weight_fp8", "sq_smooth_quant_act_fp8", "sq_linear_fp8",
     "sq_calib_quantile_workspace_size", "sq_calib_quantile", "sq_calib_batchmax_accumulate", "sq_calib_mean_of_max",
     "sq_quant_weight_fold", "sq_quant_weight_gateup_fold", "sq_scales_to_f16", "sq_scales_from_f16",
-    "sq_linear_w8a8_f16scales",
+    "sq_linear_w8a8_f16scales", "sq_linear_w8a8_gateup_silu_absmax",
 )
 
 
@@ -102,6 +102,7 @@ def _load() -> ctypes.CDLL:
         "sq_scales_to_f16": (I, [P, I64, P, P]),
         "sq_scales_from_f16": (I, [P, I64, P, P]),
         "sq_linear_w8a8_f16scales": (I, [P, P, I64, I64, I64, P, I, P, P, I, P, P, SZ, P]),
+        "sq_linear_w8a8_gateup_silu_absmax": (I, [P, P, I64, I64, I64, P, I, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -271,6 +272,16 @@ def linear_w8a8_gateup_silu(xq, wq_gu, a_scale, mode: int, w_scale_gu, h=None, s
         _dev(s2, "s2", torch.float32) if s2 is not None else None,
         _dev(a2, "a2", torch.float32) if a2 is not None else None,
         _dev(hq, "hq", torch.int8) if hq is not None else None, _stream(stream)))
+
+
+def linear_w8a8_gateup_silu_absmax(xq, wq_gu, a_scale, mode: int, w_scale_gu, h_absmax, stream=None) -> None:
+    """h_absmax[c] = max(h_absmax[c], max_m |h[m, c]|) for h = silu(g) * u of the gate/up GEMM; h is not written."""
+    M, K = xq.shape
+    N_h = wq_gu.shape[0] // 2
+    _check("sq_linear_w8a8_gateup_silu_absmax", _lib.sq_linear_w8a8_gateup_silu_absmax(
+        _dev(xq, "xq", torch.int8), _dev(wq_gu, "wq_gu", torch.int8), M, N_h, K,
+        _dev(a_scale, "a_scale", torch.float32), int(mode), _dev(w_scale_gu, "w_scale_gu", torch.float32),
+        _dev(h_absmax, "h_absmax", torch.float32), _stream(stream)))
 
 
 def gemm_f16_ref(x, w, y, stream=None) -> None:

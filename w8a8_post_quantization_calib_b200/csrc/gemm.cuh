@@ -95,6 +95,7 @@ struct Params {
     const float *s2;           // gate/up: smoothing of h [N/2]
     const float *a2;           // gate/up: static scale of h [1]
     int8_t *hq;                // gate/up: codes of h [M, N/2] or null
+    float *hmax;               // gate/up: running column max of |h| [N/2] or null
     unsigned long long timeout_ns;
     int inject;                // failure-detection test: 1 = CTA 0 withholds its first stage
 };
@@ -183,10 +184,21 @@ __device__ __forceinline__ float dequant(int32_t acc, float c, const void *bias,
 }
 
 // The same epilogue on an fp32 accumulator (the FP8 GEMM).
-__device__ __forceinline__ float dequant_f(float acc, float c, const void *bias, float b)
+__device__ __forceinline__ float dequant(float acc, float c, const void *bias, float b)
 {
     return bias != nullptr ? __fmaf_rn(acc, c, b) : __fmul_rn(acc, c);
 }
+
+// An accumulator element from its 32-bit pattern (TMEM, shared or global
+// memory): int32 for kind::i8, fp32 for kind::f8f6f4.
+template <int KIND> struct AccOf {
+    using T = int32_t;
+    __device__ __forceinline__ static T from(uint32_t b) { return static_cast<int32_t>(b); }
+};
+template <> struct AccOf<KIND_F8> {
+    using T = float;
+    __device__ __forceinline__ static T from(uint32_t b) { return __uint_as_float(b); }
+};
 
 // ---------------------------------------------------------------------------
 // Gate/up epilogue of one 128-row accumulator (TMEM lane = token row m): the
@@ -256,6 +268,19 @@ __device__ __forceinline__ void epilogue_gateup(const Params &p, const CUtensorM
                 ptx::bulk_commit();
             }
             ++nstore;
+        }
+        if (p.hmax != nullptr) {
+            // calibration statistic of h (the down projection's input): the
+            // column max of |h| over this warp's 32 rows, one warp max per
+            // channel (|h| >= 0 orders like its bit pattern), then one
+            // atomicMax per channel; h itself is not written
+            uint32_t mine = 0u;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const uint32_t mx = __reduce_max_sync(0xffffffffu, mok ? __float_as_uint(fabsf(h[i])) : 0u);
+                if (lane == i) mine = mx;
+            }
+            if (ch0 + lane < Nh) atomicMax(reinterpret_cast<unsigned int *>(p.hmax) + ch0 + lane, mine);
         }
         if (p.hq != nullptr && mok) {
             // s2 == null: 1/s2 was folded into the up rows of the weight (the
@@ -331,26 +356,26 @@ __device__ __forceinline__ Seg sk_segment(const Params &p, int it, int it_begin)
 // acc[i] += slot_cc[(t0 + i) * BM + r] over the contributors' slots cc in
 // [c0, c1) for tokens t0 + i < mval; the loads of up to 64 / CW slots are in
 // flight together.
-template <int CW>
-__device__ __forceinline__ void add_slots(const Params &p, int32_t (&acc)[CW], int c0, int c1, int t0, int mval,
-                                          int r)
+template <int CW, int KIND>
+__device__ __forceinline__ void add_slots(const Params &p, typename AccOf<KIND>::T (&acc)[CW], int c0, int c1, int t0,
+                                          int mval, int r)
 {
     constexpr int U = (64 / CW) > 1 ? 64 / CW : 1;
-    constexpr int64_t SLOT_STRIDE = BM;                // int32 per token row of a slot
+    constexpr int64_t SLOT_STRIDE = BM;                // 32-bit words per token row of a slot
 #pragma unroll 1
     for (int cc = c0; cc < c1; cc += U) {
-        int32_t v[U][CW];
+        uint32_t v[U][CW];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int32_t *sl = p.ws_acc + static_cast<int64_t>(cc + u) * p.sk_slot;
+            const uint32_t *sl = reinterpret_cast<const uint32_t *>(p.ws_acc) + static_cast<int64_t>(cc + u) * p.sk_slot;
 #pragma unroll
             for (int i = 0; i < CW; ++i)
-                v[u][i] = (cc + u < c1 && t0 + i < mval) ? __ldcg(sl + (t0 + i) * SLOT_STRIDE + r) : 0;
+                v[u][i] = (cc + u < c1 && t0 + i < mval) ? __ldcg(sl + (t0 + i) * SLOT_STRIDE + r) : 0u;
         }
 #pragma unroll
         for (int u = 0; u < U; ++u)
 #pragma unroll
-            for (int i = 0; i < CW; ++i) acc[i] += v[u][i];
+            for (int i = 0; i < CW; ++i) acc[i] += AccOf<KIND>::from(v[u][i]);
     }
 }
 
@@ -359,11 +384,12 @@ __device__ __forceinline__ void add_slots(const Params &p, int32_t (&acc)[CW], i
 // w_scale[n] and bias[n] (loaded before the accumulator is ready); s_am: the
 // token scales in shared memory.  tfull_wait() waits for the accumulator and
 // returns false on a timeout.
-template <int BN, int EPI, typename TfullWait>
+template <int BN, int EPI, int KIND, typename TfullWait>
 __device__ __forceinline__ bool epilogue_sk(const Params &p, uint32_t tbase, int tr, int tc, int tile, int q,
                                             int lane, int *flag, volatile int *abort_flag, float wsn, float bn,
                                             const float *s_am, TfullWait tfull_wait)
 {
+    using AT = typename AccOf<KIND>::T;
     constexpr int CW = TileCfg<BN>::CW;
     constexpr int64_t SLOT = static_cast<int64_t>(BM) * BN;
     const int r = q * 32 + lane;
@@ -371,10 +397,10 @@ __device__ __forceinline__ bool epilogue_sk(const Params &p, uint32_t tbase, int
     const bool nok = n < p.N;
     const int m0 = tc * BN;
     const int mval = min(BN, p.M - m0);                 // valid tokens of this tile
-    auto emit = [&](int m, int32_t acc) {
+    auto emit = [&](int m, AT acc) {
         const int64_t o = static_cast<int64_t>(m) * p.N + n;
         if constexpr (EPI == EPI_S32) {
-            static_cast<int32_t *>(p.out)[o] = acc;
+            static_cast<int32_t *>(p.out)[o] = static_cast<int32_t>(acc);
         } else {
             store_out(p.out, p.out_dt, o, dequant(acc, __fmul_rn(s_am[m - m0], wsn), p.bias, bn));
         }
@@ -387,7 +413,7 @@ __device__ __forceinline__ bool epilogue_sk(const Params &p, uint32_t tbase, int
 
     // the owner waits for the other contributors and pre-adds their slots
     // for the first chunk while its own last segment is still streaming
-    int32_t pre[CW];
+    AT pre[CW];
 #pragma unroll
     for (int i = 0; i < CW; ++i) pre[i] = 0;
     if (shared && owner) {
@@ -399,7 +425,7 @@ __device__ __forceinline__ bool epilogue_sk(const Params &p, uint32_t tbase, int
         ptx::named_bar_sync(1, 128);
         if (*flag == 0) return tfull_wait();
         ptx::fence_acq_rel_gpu();
-        add_slots<CW>(p, pre, c0, c1, 0, mval, r);
+        add_slots<CW, KIND>(p, pre, c0, c1, 0, mval, r);
     }
     if (!tfull_wait()) return false;
     ptx::tc_fence_after();
@@ -410,15 +436,15 @@ __device__ __forceinline__ bool epilogue_sk(const Params &p, uint32_t tbase, int
             uint32_t v[32];
             tmem_load_chunk(tbase + c * CW, v, CW);
             ptx::tmem_ld_wait();
-            int32_t acc[CW];
+            AT acc[CW];
 #pragma unroll
-            for (int i = 0; i < CW; ++i) acc[i] = static_cast<int32_t>(v[i]);
+            for (int i = 0; i < CW; ++i) acc[i] = AccOf<KIND>::from(v[i]);
             if (shared) {
                 if (c == 0) {
 #pragma unroll
                     for (int i = 0; i < CW; ++i) acc[i] += pre[i];
                 } else {
-                    add_slots<CW>(p, acc, c0, c1, c * CW, mval, r);
+                    add_slots<CW, KIND>(p, acc, c0, c1, c * CW, mval, r);
                 }
             }
             if (!nok) continue;
@@ -460,12 +486,13 @@ __device__ __forceinline__ bool epilogue_sk(const Params &p, uint32_t tbase, int
 // memory ([rank-1][BN][BM] int32) and arrive on its barrier; the leader adds
 // them to its own accumulator and applies the epilogue.  Every wait is
 // bounded.
-template <int BN, int EPI, int CS, typename TfullWait>
+template <int BN, int EPI, int CS, int KIND, typename TfullWait>
 __device__ __forceinline__ bool epilogue_cs(const Params &p, uint32_t tbase, int tr, int tc, int q, int lane,
                                             uint32_t rank, float wsn, float bn, const float *s_am,
                                             TfullWait tfull_wait, uint32_t go_bar, uint32_t part_bar,
                                             uint32_t sbase, volatile int *abort_flag)
 {
+    using AT = typename AccOf<KIND>::T;
     constexpr int CW = TileCfg<BN>::CW;
     const int r = q * 32 + lane;
     const int n = tr * BM + r;
@@ -485,20 +512,20 @@ __device__ __forceinline__ bool epilogue_cs(const Params &p, uint32_t tbase, int
             uint32_t v[32];
             tmem_load_chunk(tbase + c * CW, v, CW);
             ptx::tmem_ld_wait();
-            int32_t acc[CW];
+            AT acc[CW];
 #pragma unroll
-            for (int i = 0; i < CW; ++i) acc[i] = static_cast<int32_t>(v[i]);
+            for (int i = 0; i < CW; ++i) acc[i] = AccOf<KIND>::from(v[i]);
 #pragma unroll
             for (int j = 1; j < CS; ++j) {
 #pragma unroll
                 for (int i = 0; i < CW; ++i) {
                     if (c * CW + i < mval) {
-                        int32_t t;
+                        uint32_t t;
                         asm volatile("ld.shared.b32 %0, [%1];"
                                      : "=r"(t)
                                      : "r"(sbase + static_cast<uint32_t>((((j - 1) * BN + c * CW + i) * BM + r) * 4))
                                      : "memory");
-                        acc[i] += t;
+                        acc[i] += AccOf<KIND>::from(t);
                     }
                 }
             }
@@ -509,7 +536,7 @@ __device__ __forceinline__ bool epilogue_cs(const Params &p, uint32_t tbase, int
                     const int m = m0 + c * CW + i;
                     const int64_t o = static_cast<int64_t>(m) * p.N + n;
                     if constexpr (EPI == EPI_S32) {
-                        static_cast<int32_t *>(p.out)[o] = acc[i];
+                        static_cast<int32_t *>(p.out)[o] = static_cast<int32_t>(acc[i]);
                     } else {
                         store_out(p.out, p.out_dt, o, dequant(acc[i], __fmul_rn(s_am[m - m0], wsn), p.bias, bn));
                     }
@@ -539,15 +566,16 @@ __device__ __forceinline__ bool epilogue_cs(const Params &p, uint32_t tbase, int
     return true;
 }
 
-template <int BN, int EPI, int KBO, int CS>
+template <int BN, int EPI, int KBO, int CS, int KIND = KIND_I8>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     k_gemm_swap(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x, const Params p)
 {
     using C = TileCfg<BN, KBO>;
     static_assert(CS >= 1 && CS <= 4, "cluster split of 1..4 CTAs");
     static_assert((CS - 1) * BN * BM * 4 <= C::STAGES * C::STAGE_BYTES, "partial sums must fit the leader's stages");
+    static_assert(KIND == KIND_I8 || (KIND == KIND_F8 && EPI == EPI_DEQUANT), "the FP8 swap kernel dequantises");
     constexpr int S = C::STAGES;
-    constexpr uint32_t IDESC = ptx::idesc_i8(BN);
+    constexpr uint32_t IDESC = KIND == KIND_F8 ? ptx::idesc_e4m3(BN) : ptx::idesc_i8(BN);
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -662,8 +690,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         const uint64_t ad = ptx::sdesc_kmajor_sw128(sa + j * C::A_KB);
                         const uint64_t bd = ptx::sdesc_kmajor_sw128(sa + C::A_BYTES + j * C::B_KB);
 #pragma unroll
-                        for (int k = 0; k < BKB / 32; ++k)
-                            ptx::mma_i8(d, ad + 2 * k, bd + 2 * k, IDESC, (kb < sg.kb_hi || j > 0 || k > 0) ? 1u : 0u);
+                        for (int k = 0; k < BKB / 32; ++k) {
+                            const uint32_t acc = (kb < sg.kb_hi || j > 0 || k > 0) ? 1u : 0u;
+                            if constexpr (KIND == KIND_F8) ptx::mma_f8(d, ad + 2 * k, bd + 2 * k, IDESC, acc);
+                            else ptx::mma_i8(d, ad + 2 * k, bd + 2 * k, IDESC, acc);
+                        }
                     }
                     ptx::tc_commit(empty_bar(stage));
                     if (++stage == ring) { stage = 0; phase ^= 1u; }
@@ -710,11 +741,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             };
             const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * BN);
             if constexpr (CS > 1) {
-                if (!epilogue_cs<BN, EPI, CS>(p, tbase, tr, tc, q, lane, ptx::cluster_ctarank(), wsn, bn, s_am,
-                                              tfull_wait, go_bar, part_bar, sbase, abort_flag))
+                if (!epilogue_cs<BN, EPI, CS, KIND>(p, tbase, tr, tc, q, lane, ptx::cluster_ctarank(), wsn, bn,
+                                                    s_am, tfull_wait, go_bar, part_bar, sbase, abort_flag))
                     break;
-            } else if (!epilogue_sk<BN, EPI>(p, tbase, tr, tc, sg.tile, q, lane, flag, abort_flag, wsn, bn, s_am,
-                                             tfull_wait)) {
+            } else if (!epilogue_sk<BN, EPI, KIND>(p, tbase, tr, tc, sg.tile, q, lane, flag, abort_flag, wsn, bn,
+                                                   s_am, tfull_wait)) {
                 break;
             }
             ptx::tc_fence_before();
@@ -779,7 +810,7 @@ __device__ __forceinline__ void epilogue_tma(const Params &p, const CUtensorMap 
 #pragma unroll
                     for (int t = 0; t < 4; ++t) {
                         if constexpr (KIND == KIND_F8)
-                            v[i + t] = dequant_f(__uint_as_float(r[i + t]), __fmul_rn(am, ws[t]), p.bias, bb[t]);
+                            v[i + t] = dequant(__uint_as_float(r[i + t]), __fmul_rn(am, ws[t]), p.bias, bb[t]);
                         else
                             v[i + t] = dequant(static_cast<int32_t>(r[i + t]), __fmul_rn(am, ws[t]), p.bias, bb[t]);
                     }

@@ -205,7 +205,7 @@ bool make_map3(CUtensorMap *m, const void *base, int64_t K, int64_t rows, uint32
 // ------------------------------------------------------------------ GEMM launch
 // Small-M (swap) launch: map_w over the weights [N, K] in 128-row boxes, map_x
 // over the activations [M, K] in BN-row boxes; one CTA per stream-K share.
-template <int BN, int EPI, int KBO, int CS>
+template <int BN, int EPI, int KBO, int CS, int KIND = gemm::KIND_I8>
 sq_status launch_swap(gemm::Params p, const void *w, const void *x, cudaStream_t st)
 {
     using C = gemm::TileCfg<BN, KBO>;
@@ -217,7 +217,7 @@ sq_status launch_swap(gemm::Params p, const void *w, const void *x, cudaStream_t
         if (!make_map3(&mw, w, p.K, p.N, gemm::BM, KBO)) return SQ_ERR_CUDA;
         if (!make_map3(&mx, x, p.K, p.M, BN, KBO)) return SQ_ERR_CUDA;
     }
-    auto kern = gemm::k_gemm_swap<BN, EPI, KBO, CS>;
+    auto kern = gemm::k_gemm_swap<BN, EPI, KBO, CS, KIND>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), C::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_fail(e);
     p.timeout_ns = g_timeout_ns;
@@ -229,14 +229,14 @@ sq_status launch_swap(gemm::Params p, const void *w, const void *x, cudaStream_t
     return e == cudaSuccess ? check_launch() : cuda_fail(e);
 }
 
-template <int EPI, int KBO, int CS>
-sq_status launch_swap_bn(gemm::Params &p, int bn, const int8_t *wq, const int8_t *xq, cudaStream_t st)
+template <int EPI, int KBO, int CS, int KIND>
+sq_status launch_swap_bn(gemm::Params &p, int bn, const void *wq, const void *xq, cudaStream_t st)
 {
     switch (bn) {
-    case 16: return launch_swap<16, EPI, KBO, CS>(p, wq, xq, st);
-    case 32: return launch_swap<32, EPI, KBO, CS>(p, wq, xq, st);
-    case 64: return launch_swap<64, EPI, KBO, CS>(p, wq, xq, st);
-    default: return launch_swap<128, EPI, KBO, CS>(p, wq, xq, st);
+    case 16: return launch_swap<16, EPI, KBO, CS, KIND>(p, wq, xq, st);
+    case 32: return launch_swap<32, EPI, KBO, CS, KIND>(p, wq, xq, st);
+    case 64: return launch_swap<64, EPI, KBO, CS, KIND>(p, wq, xq, st);
+    default: return launch_swap<128, EPI, KBO, CS, KIND>(p, wq, xq, st);
     }
 }
 
@@ -457,8 +457,8 @@ int swap_cluster_split(int64_t M, int64_t N, int64_t K)
 // p.ws_acc / p.ws_cnt must hold a workspace for `grid` CTAs unless grid is
 // the tile count (then they are ignored).  cs > 1: cluster split, grid =
 // tiles x cs, no workspace.
-template <int EPI>
-sq_status dispatch_swap(gemm::Params &p, const int8_t *xq, const int8_t *wq, cudaStream_t st, int64_t grid,
+template <int EPI, int KIND = gemm::KIND_I8>
+sq_status dispatch_swap(gemm::Params &p, const void *xq, const void *wq, cudaStream_t st, int64_t grid,
                         int cs = 1)
 {
     const int bn = swap_bn(p.M);
@@ -478,13 +478,13 @@ sq_status dispatch_swap(gemm::Params &p, const int8_t *xq, const int8_t *wq, cud
         p.ws_cnt = nullptr;
     }
     if (kb2) {
-        if (cs == 4) return launch_swap_bn<EPI, 2, 4>(p, bn, wq, xq, st);
-        if (cs == 2) return launch_swap_bn<EPI, 2, 2>(p, bn, wq, xq, st);
-        return launch_swap_bn<EPI, 2, 1>(p, bn, wq, xq, st);
+        if (cs == 4) return launch_swap_bn<EPI, 2, 4, KIND>(p, bn, wq, xq, st);
+        if (cs == 2) return launch_swap_bn<EPI, 2, 2, KIND>(p, bn, wq, xq, st);
+        return launch_swap_bn<EPI, 2, 1, KIND>(p, bn, wq, xq, st);
     }
-    if (cs == 4) return launch_swap_bn<EPI, 1, 4>(p, bn, wq, xq, st);
-    if (cs == 2) return launch_swap_bn<EPI, 1, 2>(p, bn, wq, xq, st);
-    return launch_swap_bn<EPI, 1, 1>(p, bn, wq, xq, st);
+    if (cs == 4) return launch_swap_bn<EPI, 1, 4, KIND>(p, bn, wq, xq, st);
+    if (cs == 2) return launch_swap_bn<EPI, 1, 2, KIND>(p, bn, wq, xq, st);
+    return launch_swap_bn<EPI, 1, 1, KIND>(p, bn, wq, xq, st);
 }
 
 // ------------------------------------------------------------------ row kernels
@@ -528,6 +528,24 @@ sq_status launch_rows_dt(RowArgs a, cudaStream_t st)
             const cudaError_t e = launch_pdl_cluster(k_rows_split<DT, MODEF>,
                                                      dim3(static_cast<unsigned>(cs), static_cast<unsigned>(a.rows)),
                                                      dim3(ROW_T), static_cast<unsigned>(cs), st, a);
+            if (e != cudaSuccess) return cuda_fail(e);
+            return check_launch();
+        }
+    }
+    // Long rows (more than 8 vectors per thread of a 256-thread block, up to
+    // 4 of a 1024-thread one): 1024 threads per row, constants in shared
+    // memory, the next row's loads in flight -- 32 warps per SM where the
+    // 256-thread block with 16 vectors per thread ran 8 (the 28672-element
+    // rows of a 70B down projection: one block per SM either way, the
+    // constants taking 114 KB).
+    if constexpr (MODE == ROW_WEIGHT || MODE == ROW_ACT_TOKEN) {
+        const int64_t smem_long = static_cast<size_t>(a.K) * 4;
+        if (vec && nvec > 8 * ROW_T && cdiv(nvec, 1024) <= 4 && smem_long <= 200 * 1024) {
+            auto kern = k_rows<DT, 4, MODEF, 1024>;
+            cudaError_t e = ensure_smem(reinterpret_cast<const void *>(kern), static_cast<int>(smem_long));
+            if (e != cudaSuccess) return cuda_fail(e);
+            const int64_t grid = std::min<int64_t>(a.rows, static_cast<int64_t>(sms));
+            e = launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(1024), static_cast<size_t>(smem_long), st, a);
             if (e != cudaSuccess) return cuda_fail(e);
             return check_launch();
         }
@@ -1164,7 +1182,15 @@ sq_status sq_linear_fp8(const uint8_t *xq8, const uint8_t *wq8, int64_t M, int64
     p.bias = bias;
     p.out = y;
     p.out_dt = out_dt;
-    return dispatch_pair<gemm::KIND_F8, gemm::EPI_DEQUANT>(p, xq8, wq8, as_stream(stream));
+    const cudaStream_t st = as_stream(stream);
+    if (M <= kSwapMaxM) {
+        // weight streaming (the weights fill the 128-row MMA): the cluster
+        // split when one tile per CTA would leave most SMs idle, else one
+        // tile per CTA (the stream-K schedule needs a workspace: not used here)
+        const int cs = swap_cluster_split(M, N, K);
+        return dispatch_swap<gemm::EPI_DEQUANT, gemm::KIND_F8>(p, xq8, wq8, st, swap_tiles(M, N), cs);
+    }
+    return dispatch_pair<gemm::KIND_F8, gemm::EPI_DEQUANT>(p, xq8, wq8, st);
 }
 
 sq_status sq_scales_to_f16(const float *in, int64_t n, uint16_t *out, sq_stream stream)
@@ -1290,6 +1316,28 @@ sq_status sq_linear_w8a8_gateup_silu(const int8_t *xq, const int8_t *wq_gu, int6
     p.s2 = s2;
     p.a2 = a2;
     p.hq = hq;
+    return dispatch_pair<gemm::KIND_I8, gemm::EPI_GATEUP>(p, xq, wq_gu, as_stream(stream), 256);
+}
+
+sq_status sq_linear_w8a8_gateup_silu_absmax(const int8_t *xq, const int8_t *wq_gu, int64_t M, int64_t N_h,
+                                            int64_t K, const float *a_scale, sq_act_mode mode,
+                                            const float *w_scale_gu, float *h_absmax, sq_stream stream)
+{
+    sq_status r = check_gemm_shape(xq, wq_gu, M, 2 * N_h, K);
+    if (r != SQ_OK) return r;
+    if (a_scale == nullptr || w_scale_gu == nullptr || h_absmax == nullptr) return SQ_ERR_INVALID_ARG;
+    if ((N_h % 128) != 0) return SQ_ERR_INVALID_ARG;
+    if (mode != SQ_ACT_STATIC && mode != SQ_ACT_PER_TOKEN) return SQ_ERR_INVALID_ARG;
+    gemm::Params p{};
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(2 * N_h);
+    p.K = static_cast<int>(K);
+    p.a_scale = a_scale;
+    p.per_token = (mode == SQ_ACT_PER_TOKEN) ? 1 : 0;
+    p.w_scale = w_scale_gu;
+    p.out = nullptr;
+    p.out_dt = SQ_BF16;
+    p.hmax = h_absmax;
     return dispatch_pair<gemm::KIND_I8, gemm::EPI_GATEUP>(p, xq, wq_gu, as_stream(stream), 256);
 }
 

@@ -236,7 +236,9 @@ __global__ void __launch_bounds__(NT) k_rows(RowArgs p)
     constexpr bool F8 = (MODEF & ROW_FP8) != 0;
     constexpr bool FOLD = (MODEF & ROW_FOLD) != 0;
     constexpr int EPV = VecT<DT>::EPV;
-    constexpr bool REG = (VPT * EPV <= 32);
+    // per-column constants (and the pass-1 values) in registers; 1024-thread
+    // rows (long rows) keep them in shared memory to stay within 64 registers
+    constexpr bool REG = (VPT * EPV <= 32) && NT <= ROW_T;
     static_assert(!RING || (REG && MODE != ROW_ACT_STATIC), "the row ring needs register rows and a row barrier");
     extern __shared__ __align__(128) float4 colv4[];
     __shared__ float red[32];
