@@ -12,9 +12,10 @@ One step = the whole hot path over one batch, all through the C ABI:
   calibration statistic of the normalised input over the 16384
   calibration tokens -> weight column statistics of W_gate, W_up -> smoothing
   factors + static scale -> gate/up weight transform + per-row INT8 ->
-  calibration forward (RMSNorm + quant -> gate/up GEMM with SiLU*mul -> h)
-  and the statistic of h -> weight statistic of W_down -> smoothing factors
-  + static scale of h -> down weight transform -> runtime block:
+  calibration forward (RMSNorm + quant -> gate/up GEMM with SiLU*mul, the
+  column max of |h| kept in its epilogue) -> weight statistic of W_down ->
+  smoothing factors + static scale of h -> down weight transform -> runtime
+  block:
   RMSNorm with 1/s folded into its gain + INT8 quant -> gate/up GEMM with the
   SiLU*mul epilogue and the smooth + requant of h -> down GEMM -> bf16 Y.
 Under torchrun (N>1) each rank calibrates on its own token shard and runs its
@@ -310,8 +311,11 @@ class Spec:
     dominant: str                       # the kernel the roofline line describes
     work: dict                          # name -> {"bytes": algorithmic bytes, "ops": ops} per launch
     solo: dict                          # name -> callable launching that kernel alone (same buffers)
-    e2e_in: list                        # (device tensor, pinned host tensor) copied in each e2e step
-    e2e_out: list                       # (pinned host tensor, device tensor) copied out each e2e step
+    host_in: dict                       # name -> pinned host tensor: the step's inputs for the e2e leg
+    host_out: dict                      # name -> pinned host tensor: the step's result
+    io0: dict                           # name -> device tensor: the inputs and the result the step uses
+    alloc_io: object                    # () -> a second device set of the same inputs and result
+    make_step: object                   # io -> step(mark) on that set
     launches_per_step: int
     launches_note: str
     traffic: object = None              # callable -> DRAM bytes per launch of the dominant kernel, or None
@@ -453,31 +457,57 @@ def run_line(args, build):
                               f"{2 * P['bf16_tflops']:.0f}: {dom_tops / (2 * P['bf16_tflops']):.3f}; vs the nominal "
                               f"4500 dense INT8: {dom_tops / 4500.0:.3f}")}
 
-    # ---- end to end: pinned host buffers, H2D of the step's inputs and D2H of
-    # the result inside the region
-    e2e_steps = max(1, min(steps, args.e2e_steps))
-    h2d = sum(h.numel() * h.element_size() for _, h in spec.e2e_in)
-    d2h = sum(h.numel() * h.element_size() for h, _ in spec.e2e_out)
+    # ---- end to end: pinned host buffers, the H2D copy of every step's inputs
+    # and the D2H read of its result inside the region.  Two device sets of
+    # inputs and results, so that step k+1's inputs cross PCIe (copy stream)
+    # while step k computes (this stream) and step k-1's result returns (a
+    # third stream); every step still moves all of its bytes.
+    n2 = max(2, args.e2e_steps)
+    h2d = sum(h.numel() * h.element_size() for h in spec.host_in.values())
+    d2h = sum(h.numel() * h.element_size() for h in spec.host_out.values())
+    ios = [spec.io0, spec.alloc_io()]
+    steps_fn = [spec.make_step(io) for io in ios]
+    copy_s, back_s = torch.cuda.Stream(), torch.cuda.Stream()
+    copied = [torch.cuda.Event() for _ in range(n2)]
+    done = [torch.cuda.Event() for _ in range(n2)]
+    back = [torch.cuda.Event() for _ in range(n2)]
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        for dv, hv in spec.e2e_in:
-            dv.copy_(hv, non_blocking=True)
-        spec.step(lambda i: None)
-        for hv, dv in spec.e2e_out:
-            hv.copy_(dv, non_blocking=True)
+    copy_s.wait_event(e0)
+    for k in range(n2):
+        b = k & 1
+        with torch.cuda.stream(copy_s):
+            if k >= 2:
+                copy_s.wait_event(done[k - 2])          # set b is free once step k-2 has read it
+            for name, hv in spec.host_in.items():
+                ios[b][name].copy_(hv, non_blocking=True)
+            copied[k].record(copy_s)
+        stream.wait_event(copied[k])
+        if k >= 2:
+            stream.wait_event(back[k - 2])              # step k-2's result has left set b
+        steps_fn[b](lambda i: None)
+        done[k].record(stream)
+        with torch.cuda.stream(back_s):
+            back_s.wait_event(done[k])
+            for name, hv in spec.host_out.items():
+                hv.copy_(ios[b][name], non_blocking=True)
+            back[k].record(back_s)
+    stream.wait_event(back[n2 - 1])
     e1.record(stream)
     barrier()
-    ms_e2e = e0.elapsed_time(e1) / e2e_steps
+    ms_e2e = e0.elapsed_time(e1) / n2
+    del ios, steps_fn
     if world > 1:
         t = torch.tensor([ms_e2e], dtype=torch.float64, device="cuda")
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_e2e = float(t.item())
     clk.stop()
     e2e = {"value": world * spec.ops_per_step / (ms_e2e * 1e-3) / 1e12, "unit": "TOPS",
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e, "steps": e2e_steps,
-           "tokens_per_s": world * spec.tokens_per_step / (ms_e2e * 1e-3)}
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e, "steps": n2,
+           "tokens_per_s": world * spec.tokens_per_step / (ms_e2e * 1e-3),
+           "note": ("pinned host buffers through the C-ABI calls; every step copies its inputs in and its "
+                    "result out; two device sets, so step k+1's inputs cross PCIe while step k computes")}
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
@@ -538,8 +568,15 @@ def build_mlp70b(args, rank, world) -> Spec:
     wg_h, wu_h, wd_h = _pinned16(blk.w_gate, bf16), _pinned16(blk.w_up, bf16), _pinned16(blk.w_down, bf16)
     Mc = calib_h.shape[0]
     dv = torch.device("cuda")
-    calib, X = calib_h.to(dv), x_h.to(dv)
-    Wg, Wu, Wd = wg_h.to(dv), wu_h.to(dv), wd_h.to(dv)
+    host_in = {"calib": calib_h, "X": x_h, "Wg": wg_h, "Wu": wu_h, "Wd": wd_h}
+    io0 = {k: v.to(dv) for k, v in host_in.items()}
+    io0["y"] = torch.empty(M, d, dtype=bf16, device=dv)
+    y_h = torch.empty(M, d, dtype=bf16).pin_memory()
+
+    def alloc_io():
+        io = {k: torch.empty_like(v, device=dv) for k, v in host_in.items()}
+        io["y"] = torch.empty(M, d, dtype=bf16, device=dv)
+        return io
     gamma = torch.from_numpy(blk.gamma).to(dv)
     stats = torch.zeros(2 * d + 2 * f, dtype=torch.float32, device=dv)     # running maxima, zeroed each step
     am1, wm1 = stats[:d], stats[d:2 * d]
@@ -551,41 +588,48 @@ def build_mlp70b(args, rank, world) -> Spec:
     wq_d = torch.empty(d, f, dtype=torch.int8, device=dv)
     ws_d = torch.empty(d, device=dv)
     xq_c = torch.empty(Mc, d, dtype=torch.int8, device=dv)
-    h_c = torch.empty(Mc, f, dtype=bf16, device=dv)
     xq = torch.empty(M, d, dtype=torch.int8, device=dv)
     hq = torch.empty(M, f, dtype=torch.int8, device=dv)
-    y = torch.empty(M, d, dtype=bf16, device=dv)
-    y_h = torch.empty(M, d, dtype=bf16).pin_memory()
     S = sq.ACT_STATIC
 
-    calls = [
-        ("calib_norm_absmax", lambda: sq.rmsnorm_absmax(calib, gamma, eps, am1)),
-        ("allreduce_norm_stat", lambda: allreduce_absmax_(am1)),
-        ("weight_absmax_gate", lambda: sq.calib_absmax(Wg, wm1)),
-        ("weight_absmax_up", lambda: sq.calib_absmax(Wu, wm1)),
-        ("smooth_scales_gateup", lambda: sq.smooth_scales(am1, wm1, al, s1, a1)),
-        ("quant_weight_gateup", lambda: sq.quant_weight_gateup(Wg, Wu, s1, wq_gu, ws_gu)),
-        ("calib_rmsnorm_quant", lambda: sq.rmsnorm_quant(calib, gamma, s1, eps, a1, xq_c)),
-        ("calib_gateup_h", lambda: sq.linear_w8a8_gateup_silu(xq_c, wq_gu, a1, S, ws_gu, h=h_c)),
-        ("calib_absmax_h", lambda: sq.calib_absmax(h_c, am2)),
-        ("allreduce_h_stat", lambda: allreduce_absmax_(am2)),
-        ("weight_absmax_down", lambda: sq.calib_absmax(Wd, wm2)),
-        ("smooth_scales_down", lambda: sq.smooth_scales(am2, wm2, al, s2, a2)),
-        ("quant_weight_down", lambda: sq.quant_weight(Wd, s2, wq_d, ws_d)),
-        ("rmsnorm_quant", lambda: sq.rmsnorm_quant(X, gamma, s1, eps, a1, xq)),
-        ("gateup_silu_requant", lambda: sq.linear_w8a8_gateup_silu(xq, wq_gu, a1, S, ws_gu, s2=s2, a2=a2, hq=hq)),
-        ("down", lambda: sq.linear_w8a8(hq, wq_d, a2, S, ws_d, y)),
-    ]
-    if world == 1:
-        calls = [c for c in calls if not c[0].startswith("allreduce")]
-    names = [c[0] for c in calls]
+    def make_calls(io):
+        calib, X, Wg, Wu, Wd, y = io["calib"], io["X"], io["Wg"], io["Wu"], io["Wd"], io["y"]
+        calls = [
+            ("calib_norm_absmax", lambda: sq.rmsnorm_absmax(calib, gamma, eps, am1)),
+            ("allreduce_norm_stat", lambda: allreduce_absmax_(am1)),
+            ("weight_absmax_gate", lambda: sq.calib_absmax(Wg, wm1)),
+            ("weight_absmax_up", lambda: sq.calib_absmax(Wu, wm1)),
+            ("smooth_scales_gateup", lambda: sq.smooth_scales(am1, wm1, al, s1, a1)),
+            ("quant_weight_gateup", lambda: sq.quant_weight_gateup(Wg, Wu, s1, wq_gu, ws_gu)),
+            ("calib_rmsnorm_quant", lambda: sq.rmsnorm_quant(calib, gamma, s1, eps, a1, xq_c)),
+            ("calib_gateup_hmax", lambda: sq.linear_w8a8_gateup_silu_absmax(xq_c, wq_gu, a1, S, ws_gu, am2)),
+            ("allreduce_h_stat", lambda: allreduce_absmax_(am2)),
+            ("weight_absmax_down", lambda: sq.calib_absmax(Wd, wm2)),
+            ("smooth_scales_down", lambda: sq.smooth_scales(am2, wm2, al, s2, a2)),
+            ("quant_weight_down", lambda: sq.quant_weight(Wd, s2, wq_d, ws_d)),
+            ("rmsnorm_quant", lambda: sq.rmsnorm_quant(X, gamma, s1, eps, a1, xq)),
+            ("gateup_silu_requant", lambda: sq.linear_w8a8_gateup_silu(xq, wq_gu, a1, S, ws_gu, s2=s2, a2=a2,
+                                                                       hq=hq)),
+            ("down", lambda: sq.linear_w8a8(hq, wq_d, a2, S, ws_d, y)),
+        ]
+        if world == 1:
+            calls = [c for c in calls if not c[0].startswith("allreduce")]
+        return calls
 
-    def step(mark):
-        stats.zero_()                        # the running maxima start from zero each step
-        for i, (_, fn) in enumerate(calls):
-            mark(i)
-            fn()
-        mark(len(calls))
+    def make_step(io):
+        cl = make_calls(io)
+
+        def step(mark):
+            stats.zero_()                    # the running maxima start from zero each step
+            for i, (_, fn) in enumerate(cl):
+                mark(i)
+                fn()
+            mark(len(cl))
+        return step
+
+    calls = make_calls(io0)
+    names = [c[0] for c in calls]
+    step = make_step(io0)
 
     gu_ops = 2.0 * M * 2 * f * d
     work = {
@@ -595,8 +639,7 @@ def build_mlp70b(args, rank, world) -> Spec:
         "smooth_scales_gateup": {"bytes": d * 12},
         "quant_weight_gateup": {"bytes": 2 * f * d * 3 + 2 * f * 4},
         "calib_rmsnorm_quant": {"bytes": Mc * d * 3},
-        "calib_gateup_h": {"ops": 2.0 * Mc * 2 * f * d, "bytes": Mc * d + 2 * f * d + Mc * f * 2},
-        "calib_absmax_h": {"bytes": Mc * f * 2},
+        "calib_gateup_hmax": {"ops": 2.0 * Mc * 2 * f * d, "bytes": Mc * d + 2 * f * d + f * 4},
         "weight_absmax_down": {"bytes": d * f * 2},
         "smooth_scales_down": {"bytes": f * 12},
         "quant_weight_down": {"bytes": d * f * 3 + d * 4},
@@ -612,13 +655,13 @@ def build_mlp70b(args, rank, world) -> Spec:
         config=dict(LINE_CONFIG["mlp70b"]),
         ops_per_step=ops, tokens_per_step=M, names=names, step=step, dominant="gateup_silu_requant",
         work=work, solo=solo,
-        e2e_in=[(calib, calib_h), (X, x_h), (Wg, wg_h), (Wu, wu_h), (Wd, wd_h)], e2e_out=[(y_h, y)],
+        host_in=host_in, host_out={"y": y_h}, io0=io0, alloc_io=alloc_io, make_step=make_step,
         launches_per_step=nlaunch,
         launches_note=(f"{nlaunch} libsq kernels per step (+1 torch fill zeroing the four running maxima"
                        + (", +2 NCCL all-reduces" if world > 1 else "") + ")"),
         traffic=lambda: traffic_from_profile("linear_w8a8_gateup_mlp70b_traffic"),
         data=blk if world == 1 else None,
-        extra={"solo_reps": {"calib_gateup_h": 3, "gateup_silu_requant": 3, "down": 3, "quant_weight_gateup": 5},
+        extra={"solo_reps": {"calib_gateup_hmax": 3, "gateup_silu_requant": 3, "down": 3, "quant_weight_gateup": 5},
                "line": {"ops_note": ("ops per step = the calibration forward's gate/up GEMM (16384 calibration "
                                      "tokens) + the runtime gate/up and down GEMMs, 2*M*N*K each")}},
     )
@@ -636,33 +679,50 @@ def build_qkv7b(args, rank, world) -> Spec:
     M, K, N = QKV_M, QKV_K, QKV_N
     calib_h, w_h, x_h = _pinned16(np.concatenate(wl.calib), f16), _pinned16(wl.w, f16), _pinned16(wl.x, f16)
     dv = torch.device("cuda")
-    calib, W, X = calib_h.to(dv), w_h.to(dv), x_h.to(dv)
+    host_in = {"calib": calib_h, "W": w_h, "X": x_h}
+    io0 = {k: v.to(dv) for k, v in host_in.items()}
+    io0["y"] = torch.empty(M, N, dtype=f16, device=dv)
+    y_h = torch.empty(M, N, dtype=f16).pin_memory()
+
+    def alloc_io():
+        io = {k: torch.empty_like(v, device=dv) for k, v in host_in.items()}
+        io["y"] = torch.empty(M, N, dtype=f16, device=dv)
+        return io
     stats = torch.zeros(2 * K, dtype=torch.float32, device=dv)
     act_max, w_max = stats[:K], stats[K:]
     s, a = torch.empty(K, device=dv), torch.empty(1, device=dv)
     wq, ws = torch.empty(N, K, dtype=torch.int8, device=dv), torch.empty(N, device=dv)
     xq = torch.empty(M, K, dtype=torch.int8, device=dv)
-    y = torch.empty(M, N, dtype=f16, device=dv)
-    y_h = torch.empty(M, N, dtype=f16).pin_memory()
-    calls = [
-        ("calib_absmax", lambda: sq.calib_absmax(calib, act_max)),
-        ("allreduce_max", lambda: allreduce_absmax_(act_max)),
-        ("weight_absmax", lambda: sq.calib_absmax(W, w_max)),
-        ("smooth_scales", lambda: sq.smooth_scales(act_max, w_max, 0.5, s, a)),
-        ("quant_weight", lambda: sq.quant_weight(W, s, wq, ws)),
-        ("smooth_quant_act", lambda: sq.smooth_quant_act(X, s, sq.ACT_STATIC, a, xq)),
-        ("linear_w8a8", lambda: sq.linear_w8a8(xq, wq, a, sq.ACT_STATIC, ws, y)),
-    ]
-    if world == 1:
-        calls = [c for c in calls if c[0] != "allreduce_max"]
-    names = [c[0] for c in calls]
 
-    def step(mark):
-        stats.zero_()
-        for i, (_, fn) in enumerate(calls):
-            mark(i)
-            fn()
-        mark(len(calls))
+    def make_calls(io):
+        calib, W, X, y = io["calib"], io["W"], io["X"], io["y"]
+        calls = [
+            ("calib_absmax", lambda: sq.calib_absmax(calib, act_max)),
+            ("allreduce_max", lambda: allreduce_absmax_(act_max)),
+            ("weight_absmax", lambda: sq.calib_absmax(W, w_max)),
+            ("smooth_scales", lambda: sq.smooth_scales(act_max, w_max, 0.5, s, a)),
+            ("quant_weight", lambda: sq.quant_weight(W, s, wq, ws)),
+            ("smooth_quant_act", lambda: sq.smooth_quant_act(X, s, sq.ACT_STATIC, a, xq)),
+            ("linear_w8a8", lambda: sq.linear_w8a8(xq, wq, a, sq.ACT_STATIC, ws, y)),
+        ]
+        if world == 1:
+            calls = [c for c in calls if c[0] != "allreduce_max"]
+        return calls
+
+    def make_step(io):
+        cl = make_calls(io)
+
+        def step(mark):
+            stats.zero_()
+            for i, (_, fn) in enumerate(cl):
+                mark(i)
+                fn()
+            mark(len(cl))
+        return step
+
+    calls = make_calls(io0)
+    names = [c[0] for c in calls]
+    step = make_step(io0)
 
     ops = 2.0 * M * N * K
     Mc = calib_h.shape[0]
@@ -675,7 +735,7 @@ def build_qkv7b(args, rank, world) -> Spec:
         config=dict(LINE_CONFIG["qkv7b"]),
         ops_per_step=ops, tokens_per_step=M, names=names, step=step, dominant="linear_w8a8", work=work,
         solo={n: fn for n, fn in calls if n != "allreduce_max"},
-        e2e_in=[(calib, calib_h), (W, w_h), (X, x_h)], e2e_out=[(y_h, y)],
+        host_in=host_in, host_out={"y": y_h}, io0=io0, alloc_io=alloc_io, make_step=make_step,
         launches_per_step=6, launches_note="6 libsq kernels per step (+1 torch fill zeroing the two running maxima)",
         traffic=lambda: traffic_from_profile("linear_w8a8_qkv7b_traffic"),
         data=wl if world == 1 else None,
@@ -1030,7 +1090,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=20.0,
                     help="CPU work the oracle baseline's sample is sized for")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=6)
     ap.add_argument("--eager-steps", action="store_true",
                     help="launch the timed steps one call at a time instead of as one captured CUDA graph")
     ap.add_argument("--tokens", default="1,16,128,4096",

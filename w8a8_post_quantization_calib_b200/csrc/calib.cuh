@@ -113,6 +113,8 @@ __global__ void __launch_bounds__(CALIB_TX *CALIB_TY)
             atomicMax(reinterpret_cast<int *>(absmax + col), __float_as_int(m));
         }
     }
+    __syncthreads();
+    pdl_trigger();
 }
 
 // Fallback for tensors whose rows are not 16-byte aligned: one thread per
@@ -122,12 +124,15 @@ __global__ void k_colabsmax_scalar(const void *__restrict__ x, int dt, int64_t r
 {
     pdl_wait();
     const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (j >= cols) return;
-    const int64_t r0 = static_cast<int64_t>(blockIdx.y) * row_slab;
-    const int64_t r1 = min(rows, r0 + row_slab);
-    float m = 0.0f;
-    for (int64_t r = r0; r < r1; ++r) m = fmaxf(m, fabsf(load_elem_dt(x, dt, r * ld + j)));
-    atomicMax(reinterpret_cast<int *>(absmax + j), __float_as_int(m));
+    if (j < cols) {
+        const int64_t r0 = static_cast<int64_t>(blockIdx.y) * row_slab;
+        const int64_t r1 = min(rows, r0 + row_slab);
+        float m = 0.0f;
+        for (int64_t r = r0; r < r1; ++r) m = fmaxf(m, fabsf(load_elem_dt(x, dt, r * ld + j)));
+        atomicMax(reinterpret_cast<int *>(absmax + j), __float_as_int(m));
+    }
+    __syncthreads();
+    pdl_trigger();
 }
 
 }  // namespace sq

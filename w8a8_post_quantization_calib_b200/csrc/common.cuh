@@ -20,15 +20,16 @@ __device__ unsigned int g_error_word;
 
 // Programmatic dependent launch.  On created streams every kernel of this
 // library is launched with programmatic stream serialisation and executes
-// pdl_wait() before it reads any global input; it may then be scheduled as
-// soon as the previous kernel of the stream completes (no gap for launch
-// processing).  No kernel here triggers its dependents early
-// (griddepcontrol.launch_dependents): measured on B200, global writes a
-// kernel made after that trigger were not visible to a dependent past its
-// griddepcontrol.wait -- a chain of small dependent kernels read stale
-// histograms and prefixes -- so a kernel could only trigger after its last
-// global write, which is no earlier than its completion.
+// pdl_wait() before it reads any global input.  Each kernel triggers its
+// dependents (pdl_trigger) only at its very end: every thread of a CTA, after
+// a block-wide barrier that follows the CTA's last global write, so that the
+// next kernel's launch and prologue overlap this kernel's teardown.  Measured
+// on B200, global writes a kernel made AFTER its trigger were not visible to
+// the dependent past its griddepcontrol.wait (a chain of small dependent
+// kernels that triggered at their start read stale histograms and prefixes);
+// with the trigger after the last write the chain was exact.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
 // Canonical fp32 steps (round-to-nearest intrinsics so that nvcc never fuses

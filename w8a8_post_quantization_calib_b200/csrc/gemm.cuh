@@ -760,6 +760,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // released
     __syncwarp();
     __syncthreads();
+    pdl_trigger();                     // every output of this CTA is written
     if (warp == 1) {
         __syncwarp();
         ptx::tc_fence_after();
@@ -1123,6 +1124,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 
     ptx::tc_fence_before();
     ptx::cluster_sync();               // no CTA leaves while its peer may still signal it
+    pdl_trigger();                     // every output of this CTA is written (TMA stores waited for)
     if (warp == 1) {
         __syncwarp();
         ptx::tc_fence_after();

@@ -72,6 +72,8 @@ __global__ void __cluster_dims__(8, 1, 1) __launch_bounds__(1024)
     }
     // no CTA leaves while CTA 0 may still read its shared memory
     asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+    __syncthreads();
+    pdl_trigger();
 }
 
 __global__ void __launch_bounds__(1024)
@@ -95,6 +97,8 @@ __global__ void __launch_bounds__(1024)
             else atomicMax(reinterpret_cast<int *>(a_static), __float_as_int(__fdiv_rn(m, qmax)));
         }
     }
+    __syncthreads();
+    pdl_trigger();
 }
 
 // ---------------------------------------------------------------------------
@@ -582,6 +586,8 @@ __global__ void __launch_bounds__(NT) k_rows(RowArgs p)
         }
         ptx::cluster_sync();                            // no block leaves while its maxima are read
     }
+    __syncthreads();
+    pdl_trigger();
 }
 
 // Static (per-tensor) activation quantisation is elementwise: code(x) =
@@ -608,76 +614,79 @@ __global__ void __launch_bounds__(QS_TX *QS_TY)
     const int64_t r1 = min(rows, r0 + row_slab);
     const int64_t K = nvec * EPV;
     pdl_wait();
-    if (v >= nvec) return;
-    const uint8_t *col = x + v * 16;
-    auto load = [&](int64_t r) {
-        const uint4 *p = reinterpret_cast<const uint4 *>(col + r * nvec * 16);
-        if constexpr (STREAM) return __ldcs(p);
-        else return __ldg(p);
-    };
-    // first rows in flight before the constants
-    uint4 t[QS_UNROLL];
-    int64_t r = r0 + ty;
-#pragma unroll
-    for (int u = 0; u < QS_UNROLL; ++u)
-        if (r + u * QS_TY < r1) t[u] = load(r + u * QS_TY);
-    float c[EPV];
-    if ((reinterpret_cast<uintptr_t>(s) & 15u) == 0) {
-#pragma unroll
-        for (int h = 0; h < EPV / 4; ++h) {
-            const float4 w = __ldg(reinterpret_cast<const float4 *>(s) + v * (EPV / 4) + h);
-            c[4 * h] = recip_or_zero(w.x); c[4 * h + 1] = recip_or_zero(w.y);
-            c[4 * h + 2] = recip_or_zero(w.z); c[4 * h + 3] = recip_or_zero(w.w);
-        }
-    } else {
-#pragma unroll
-        for (int e = 0; e < EPV; ++e) c[e] = recip_or_zero(s[v * EPV + e]);
-    }
-    const float inv_a = recip_or_zero(a_in[0]);
-    auto emit = [&](int64_t row, const uint4 &raw) {
-        float f[EPV];
-        widen<DT>(raw, f);
-#pragma unroll
-        for (int e = 0; e < EPV; ++e) f[e] = __fmul_rn(__fmul_rn(f[e], c[e]), inv_a);
-        int8_t *dst = out + row * K;
-        if constexpr (F8) {
-            if constexpr (EPV == 8) {
-                __stcs(reinterpret_cast<uint2 *>(dst + v * 8), make_uint2(e4m3x4_bits(f[0], f[1], f[2], f[3]),
-                                                                          e4m3x4_bits(f[4], f[5], f[6], f[7])));
-            } else {
-                __stcs(reinterpret_cast<uint32_t *>(dst + v * 4), e4m3x4_bits(f[0], f[1], f[2], f[3]));
-            }
-        } else if constexpr (EPV == 8) {
-            uint2 o;
-            o.x = pack4_bits(quant8_bits(f[0]), quant8_bits(f[1]), quant8_bits(f[2]), quant8_bits(f[3]));
-            o.y = pack4_bits(quant8_bits(f[4]), quant8_bits(f[5]), quant8_bits(f[6]), quant8_bits(f[7]));
-            __stcs(reinterpret_cast<uint2 *>(dst + v * 8), o);
-        } else {
-            __stcs(reinterpret_cast<uint32_t *>(dst + v * 4),
-                   pack4_bits(quant8_bits(f[0]), quant8_bits(f[1]), quant8_bits(f[2]), quant8_bits(f[3])));
-        }
-    };
-    if constexpr (ONE) {
+    if (v < nvec) {
+        const uint8_t *col = x + v * 16;
+        auto load = [&](int64_t r) {
+            const uint4 *p = reinterpret_cast<const uint4 *>(col + r * nvec * 16);
+            if constexpr (STREAM) return __ldcs(p);
+            else return __ldg(p);
+        };
+        // first rows in flight before the constants
+        uint4 t[QS_UNROLL];
+        int64_t r = r0 + ty;
 #pragma unroll
         for (int u = 0; u < QS_UNROLL; ++u)
-            if (r + u * QS_TY < r1) emit(r + u * QS_TY, t[u]);
-    } else {
-        // the next batch of rows is requested before this one is converted
-        for (;;) {
-            const int64_t rn = r + QS_UNROLL * QS_TY;
-            uint4 n[QS_UNROLL];
+            if (r + u * QS_TY < r1) t[u] = load(r + u * QS_TY);
+        float c[EPV];
+        if ((reinterpret_cast<uintptr_t>(s) & 15u) == 0) {
 #pragma unroll
-            for (int u = 0; u < QS_UNROLL; ++u)
-                if (rn + u * QS_TY < r1) n[u] = load(rn + u * QS_TY);
+            for (int h = 0; h < EPV / 4; ++h) {
+                const float4 w = __ldg(reinterpret_cast<const float4 *>(s) + v * (EPV / 4) + h);
+                c[4 * h] = recip_or_zero(w.x); c[4 * h + 1] = recip_or_zero(w.y);
+                c[4 * h + 2] = recip_or_zero(w.z); c[4 * h + 3] = recip_or_zero(w.w);
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < EPV; ++e) c[e] = recip_or_zero(s[v * EPV + e]);
+        }
+        const float inv_a = recip_or_zero(a_in[0]);
+        auto emit = [&](int64_t row, const uint4 &raw) {
+            float f[EPV];
+            widen<DT>(raw, f);
+#pragma unroll
+            for (int e = 0; e < EPV; ++e) f[e] = __fmul_rn(__fmul_rn(f[e], c[e]), inv_a);
+            int8_t *dst = out + row * K;
+            if constexpr (F8) {
+                if constexpr (EPV == 8) {
+                    __stcs(reinterpret_cast<uint2 *>(dst + v * 8), make_uint2(e4m3x4_bits(f[0], f[1], f[2], f[3]),
+                                                                              e4m3x4_bits(f[4], f[5], f[6], f[7])));
+                } else {
+                    __stcs(reinterpret_cast<uint32_t *>(dst + v * 4), e4m3x4_bits(f[0], f[1], f[2], f[3]));
+                }
+            } else if constexpr (EPV == 8) {
+                uint2 o;
+                o.x = pack4_bits(quant8_bits(f[0]), quant8_bits(f[1]), quant8_bits(f[2]), quant8_bits(f[3]));
+                o.y = pack4_bits(quant8_bits(f[4]), quant8_bits(f[5]), quant8_bits(f[6]), quant8_bits(f[7]));
+                __stcs(reinterpret_cast<uint2 *>(dst + v * 8), o);
+            } else {
+                __stcs(reinterpret_cast<uint32_t *>(dst + v * 4),
+                       pack4_bits(quant8_bits(f[0]), quant8_bits(f[1]), quant8_bits(f[2]), quant8_bits(f[3])));
+            }
+        };
+        if constexpr (ONE) {
 #pragma unroll
             for (int u = 0; u < QS_UNROLL; ++u)
                 if (r + u * QS_TY < r1) emit(r + u * QS_TY, t[u]);
-            if (rn >= r1) break;
+        } else {
+            // the next batch of rows is requested before this one is converted
+            for (;;) {
+                const int64_t rn = r + QS_UNROLL * QS_TY;
+                uint4 n[QS_UNROLL];
 #pragma unroll
-            for (int u = 0; u < QS_UNROLL; ++u) t[u] = n[u];
-            r = rn;
+                for (int u = 0; u < QS_UNROLL; ++u)
+                    if (rn + u * QS_TY < r1) n[u] = load(rn + u * QS_TY);
+#pragma unroll
+                for (int u = 0; u < QS_UNROLL; ++u)
+                    if (r + u * QS_TY < r1) emit(r + u * QS_TY, t[u]);
+                if (rn >= r1) break;
+#pragma unroll
+                for (int u = 0; u < QS_UNROLL; ++u) t[u] = n[u];
+                r = rn;
+            }
         }
     }
+    __syncthreads();
+    pdl_trigger();
 }
 
 // Few rows (decode-size activations): a cluster of CS CTAs shares each row,
@@ -812,6 +821,8 @@ __global__ void __launch_bounds__(ROW_T) k_rows_split(RowArgs p)
             else store_codes<EPV, false>(dst, v, f);
         }
     }
+    __syncthreads();
+    pdl_trigger();
 }
 
 // Unaligned / very wide rows: one block per row, elementwise, two passes
@@ -881,6 +892,8 @@ __global__ void __launch_bounds__(ROW_T) k_rows_scalar(RowArgs p, int dt)
         }
         __syncthreads();
     }
+    __syncthreads();
+    pdl_trigger();
 }
 
 // ---------------------------------------------------------------------------
@@ -893,6 +906,8 @@ __global__ void __launch_bounds__(256) k_f32_to_f16(const float *__restrict__ in
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x)
         out[i] = __float2half_rn(in[i]);
+    __syncthreads();
+    pdl_trigger();
 }
 
 __global__ void __launch_bounds__(256) k_f16_to_f32(const __half *__restrict__ in, int64_t n, float *__restrict__ out)
@@ -901,6 +916,8 @@ __global__ void __launch_bounds__(256) k_f16_to_f32(const __half *__restrict__ i
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x)
         out[i] = __half2float(in[i]);
+    __syncthreads();
+    pdl_trigger();
 }
 
 // ---------------------------------------------------------------------------
@@ -938,6 +955,8 @@ __global__ void __launch_bounds__(256)
         for (int i = 0; i < (blockDim.x >> 5); ++i) t += red[i];
         atomicAdd(sse, t);
     }
+    __syncthreads();
+    pdl_trigger();
 }
 
 }  // namespace sq

@@ -36,6 +36,8 @@ __global__ void __launch_bounds__(256)
         sum_max[j] += static_cast<double>(batch_max[j]);
         batch_max[j] = 0.0f;
     }
+    __syncthreads();
+    pdl_trigger();
 }
 
 __global__ void __launch_bounds__(256)
@@ -45,6 +47,8 @@ __global__ void __launch_bounds__(256)
     for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < cols;
          j += static_cast<int64_t>(gridDim.x) * blockDim.x)
         out[j] = __double2float_rn(__ddiv_rn(sum_max[j], n_batches));
+    __syncthreads();
+    pdl_trigger();
 }
 
 // ------------------------------------------------------------- quantile
@@ -134,6 +138,8 @@ __global__ void __launch_bounds__(QH_THREADS)
         const uint32_t n = sh[c * QH_STRIDE + b];
         if (n != 0u && c0 + c < cols) atomicAdd(hist + (c0 + c) * QH_BINS + b, n);
     }
+    __syncthreads();
+    pdl_trigger();
 }
 
 // One warp per column: find the bin of the column's histogram that holds
@@ -142,11 +148,10 @@ __global__ void __launch_bounds__(QH_THREADS)
 // first: prefix 0 and krem = k for every column.  last: write the value
 // whose magnitude bits are the completed prefix.
 template <int DT>
-__global__ void __launch_bounds__(256)
-    k_quantile_select(uint32_t *__restrict__ hist, int64_t cols, int width, uint32_t k, int first, int last,
-                      uint32_t *__restrict__ prefix, uint32_t *__restrict__ krem, float *__restrict__ out)
+__device__ __forceinline__ void quantile_select_column(uint32_t *__restrict__ hist, int64_t cols, int width,
+                                                       uint32_t k, int first, int last, uint32_t *__restrict__ prefix,
+                                                       uint32_t *__restrict__ krem, float *__restrict__ out)
 {
-    pdl_wait();
     const int lane = threadIdx.x & 31;
     const int64_t j = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     if (j >= cols) return;
@@ -208,6 +213,17 @@ __global__ void __launch_bounds__(256)
             krem[j] = kr - below;
         }
     }
+}
+
+template <int DT>
+__global__ void __launch_bounds__(256)
+    k_quantile_select(uint32_t *__restrict__ hist, int64_t cols, int width, uint32_t k, int first, int last,
+                      uint32_t *__restrict__ prefix, uint32_t *__restrict__ krem, float *__restrict__ out)
+{
+    pdl_wait();
+    quantile_select_column<DT>(hist, cols, width, k, first, last, prefix, krem, out);
+    __syncthreads();
+    pdl_trigger();
 }
 
 }  // namespace sq
