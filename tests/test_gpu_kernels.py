@@ -232,6 +232,77 @@ def test_rmsnorm_quant(M, d, random_gamma):
     assert bits_equal(host(xq), xq_ref), mismatch_report(host(xq), xq_ref)
 
 
+@pytest.mark.parametrize("sign", [1, -1, 0])
+def test_rmsnorm_quant_saturation_boundary(sign):
+    """Codes at the edge of saturation.  The kernel skips the clamp for the
+    values of a thread whose magnitudes all lie below 127.5; a value of
+    magnitude >= 127.5 rounds to +-128 and must be clamped to +-127.  The
+    static scale is swept ulp by ulp so that row 0's largest value v =
+    fl(y * fl(1/a)) falls on both sides of 127.5 (and on it where the
+    rounding allows); the outlier of row 0 is positive, negative, or one of
+    each.  Every row is compared with the oracle at every scale (300 rows:
+    the many-row kernel; fewer rows than SMs take the split-row kernel)."""
+    M, d = 300, 4096
+    X = rand_x(40 + sign, (M, d), BF16, 1.0)
+    xf = oracle.to_f32(X, BF16).copy()
+    if sign >= 0:
+        xf[0, 100] = 12.0
+    if sign <= 0:
+        xf[0, 2000] = -12.0
+    X = synth.cast(xf, BF16)
+    g = np.random.default_rng(41)
+    gamma = g.uniform(0.5, 1.5, d).astype(np.float32)
+    s = (np.abs(g.standard_normal(d)) + 0.3).astype(np.float32)
+    s[[100, 2000]] = 1.0
+    gamma[[100, 2000]] = 1.0
+    # y of row 0 as the oracle computes it: fl(fl(x * r) * fl(gamma * fl(1/s)))
+    _, r0 = oracle.rmsnorm_quant(X[:1], gamma, s, 1e-5, np.float32(1.0), BF16)
+    c = (gamma * (np.float32(1.0) / s)).astype(np.float32)
+    y0 = ((oracle.to_f32(X[:1], BF16) * r0[0]).astype(np.float32) * c).astype(np.float32)
+    a0 = np.float32(np.abs(y0).max() / np.float32(127.5))
+    vs = []
+    for k in range(-6, 7):
+        a = np.float32(a0)
+        for _ in range(abs(k)):
+            a = np.nextafter(a, np.float32(np.inf if k > 0 else 0), dtype=np.float32)
+        vs.append(float(np.abs(y0 * (np.float32(1.0) / a)).max()))
+        xq = torch.empty(M, d, dtype=torch.int8, device="cuda")
+        sq.rmsnorm_quant(dev(X, BF16), dev(gamma), dev(s), 1e-5, dev(np.array([a], np.float32)), xq)
+        _sync()
+        xq_ref, _ = oracle.rmsnorm_quant(X, gamma, s, 1e-5, a, BF16)
+        assert bits_equal(host(xq), xq_ref), (k, mismatch_report(host(xq), xq_ref))
+        assert np.abs(xq_ref[0]).max() == 127
+    assert min(vs) < 127.5 <= max(vs)
+
+
+@pytest.mark.parametrize("dt", [BF16, F16])
+def test_quant_static_saturation_boundary(dt):
+    """Static-scale activation codes at the edge of saturation: the kernel
+    clamps only the vectors holding a value of magnitude >= 127.5.  Rows 0-2
+    carry +12, -12 and both; with s = 1 the scale is swept ulp by ulp around
+    12 / 127.5, so that fl(12 * fl(1/a)) falls on both sides of 127.5."""
+    M, K = 600, 4096
+    xf = oracle.to_f32(rand_x(50, (M, K), dt, 1.0), dt).copy()
+    xf[0, 8] = 12.0
+    xf[1, 4000] = -12.0
+    xf[2, 17], xf[2, 18] = 12.0, -12.0
+    X = synth.cast(xf, dt)
+    s = np.ones(K, np.float32)
+    a0 = np.float32(np.float32(12.0) / np.float32(127.5))
+    vs = []
+    for k in range(-6, 7):
+        a = np.float32(a0)
+        for _ in range(abs(k)):
+            a = np.nextafter(a, np.float32(np.inf if k > 0 else 0), dtype=np.float32)
+        vs.append(float(np.float32(12.0) * (np.float32(1.0) / a)))
+        xq = torch.empty(M, K, dtype=torch.int8, device="cuda")
+        sq.smooth_quant_act(dev(X, dt), dev(s), oracle.STATIC, dev(np.array([a], np.float32)), xq)
+        _sync()
+        xq_ref, _ = oracle.smooth_quant_act(X, s, oracle.STATIC, a, dt)
+        assert bits_equal(host(xq), xq_ref), (k, mismatch_report(host(xq), xq_ref))
+    assert min(vs) < 127.5 <= max(vs)
+
+
 # ------------------------------------------------------------------ a6
 GEMM_SHAPES = [(1, 16, 32), (16, 48, 48), (100, 272, 1040), (128, 528, 4096), (129, 256, 128),
                (300, 528, 1040), (64, 4096, 11008), (257, 768, 4096)]
@@ -445,6 +516,33 @@ def test_rmsnorm_absmax(M, d, dt):
     _sync()
     ref = oracle.rmsnorm_absmax(X, gamma, 1e-5, dt)
     assert bits_equal(host(am), ref), mismatch_report(host(am), ref)
+
+
+@pytest.mark.parametrize("M,K,dt", [(5000, 8192, BF16), (9001, 4096, F16), (3001, 6144, BF16), (2000, 3000, BF16),
+                                    (1500, 1032, F16)])
+def test_rmsnorm_pipelined_many_rows(M, K, dt):
+    """RMSNorm + quant and the norm-output statistic with many rows per block
+    (the software-pipelined kernel: row n's sum and r_m overlap row n - 1's
+    second pass through a ring of shared-memory row buffers), at row counts
+    that are not a multiple of the grid and row lengths with a ragged last
+    vector group, bit for bit against the oracle."""
+    X = rand_x(M + K + 3, (M, K), dt, 1.0, outliers=max(1, K // 200))
+    g = np.random.default_rng(M * 3 + K)
+    gamma = g.uniform(0.5, 1.5, K).astype(np.float32)
+    s = (np.abs(g.standard_normal(K)) + 0.3).astype(np.float32)
+    a = np.float32(0.04)
+    xq = torch.empty(M, K, dtype=torch.int8, device="cuda")
+    r = torch.empty(M, dtype=torch.float32, device="cuda")
+    xt = dev(X, dt)
+    sq.rmsnorm_quant(xt, dev(gamma), dev(s), 1e-5, dev(np.array([a])), xq, r)
+    am = torch.zeros(K, dtype=torch.float32, device="cuda")
+    sq.rmsnorm_absmax(xt, dev(gamma), 1e-5, am)
+    _sync()
+    xq_ref, r_ref = oracle.rmsnorm_quant(X, gamma, s, 1e-5, a, dt)
+    assert bits_equal(host(r), r_ref), mismatch_report(host(r), r_ref)
+    assert bits_equal(host(xq), xq_ref), mismatch_report(host(xq), xq_ref)
+    am_ref = oracle.rmsnorm_absmax(X, gamma, 1e-5, dt)
+    assert bits_equal(host(am), am_ref), mismatch_report(host(am), am_ref)
 
 
 # ------------------------------------------------------------------ row ring

@@ -65,6 +65,35 @@ __device__ __forceinline__ uint32_t quant8_bits(float v)
 // of quant8_bits cannot bind there.
 __device__ __forceinline__ uint32_t quant8_bits_inrange(float v) { return __float_as_uint(__fadd_rn(v, 12582912.0f)); }
 
+// quant8_bits (INRANGE: quant8_bits_inrange) of a pair of values with one
+// packed fp32 add (sm_100's f32x2 arithmetic rounds each lane like the
+// scalar instruction).
+template <bool INRANGE>
+__device__ __forceinline__ void quant8_bits2(float a, float b, uint32_t &qa, uint32_t &qb)
+{
+    const float2 c = INRANGE ? make_float2(a, b)
+                             : make_float2(fminf(fmaxf(a, -127.0f), 127.0f), fminf(fmaxf(b, -127.0f), 127.0f));
+    const float2 t = __fadd2_rn(c, make_float2(12582912.0f, 12582912.0f));
+    qa = __float_as_uint(t.x);
+    qb = __float_as_uint(t.y);
+}
+
+// max(m, |a|, |b|) in one instruction (sm_100's three-input max).  max3_abs
+// skips a NaN input like fmaxf; max3_abs_nan returns NaN when any input is
+// NaN, so that a range check on its result fails for NaN.
+__device__ __forceinline__ float max3_abs(float m, float a, float b)
+{
+    float r;
+    asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(m), "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ float max3_abs_nan(float m, float a, float b)
+{
+    float r;
+    asm("max.NaN.abs.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(m), "f"(a), "f"(b));
+    return r;
+}
+
 // low bytes of four quant8_bits results -> one packed word (byte 0 = a)
 __device__ __forceinline__ uint32_t pack4_bits(uint32_t a, uint32_t b, uint32_t c, uint32_t d)
 {

@@ -488,6 +488,41 @@ sq_status dispatch_swap(gemm::Params &p, const void *xq, const void *wq, cudaStr
 }
 
 // ------------------------------------------------------------------ row kernels
+// One row-kernel launch: opt-in shared memory, a grid of (blocks per SM, from
+// the occupancy calculator, cached per kernel and size) x SMs, and for the
+// norm-output statistic with few rows per block a cluster launch, so that the
+// blocks combine their column maxima before the atomics.
+template <int MODE>
+cudaError_t launch_row_kernel(void (*kern)(RowArgs), int nt, size_t smem, const RowArgs &a, cudaStream_t st)
+{
+    cudaError_t e = cudaSuccess;
+    if (smem > 0) {       // with the kernel's static shared memory it may pass the 48 KB default
+        e = ensure_smem(reinterpret_cast<const void *>(kern), static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+    }
+    int per_sm = 0;
+    {   // occupancy per kernel and shared-memory size, queried once
+        std::lock_guard<std::mutex> lk(g_mu);
+        const KernelInfo &ki = kinfo(reinterpret_cast<const void *>(kern));
+        if (ki.per_sm_smem == static_cast<int>(smem)) per_sm = ki.per_sm;
+    }
+    if (per_sm == 0) {
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, nt, smem);
+        if (e != cudaSuccess) return e;
+        std::lock_guard<std::mutex> lk(g_mu);
+        KernelInfo &ki = kinfo(reinterpret_cast<const void *>(kern));
+        ki.per_sm = per_sm;
+        ki.per_sm_smem = static_cast<int>(smem);
+    }
+    const int sms = sm_count();
+    int64_t grid = std::min<int64_t>(a.rows, static_cast<int64_t>(sms) * std::max(1, per_sm));
+    if (MODE == ROW_RMS_STAT && a.rows <= 8 * grid) {
+        grid = cdiv(grid, RMS_CL) * RMS_CL;       // whole clusters (blocks past the rows idle)
+        return launch_pdl_cluster_smem(kern, dim3(static_cast<unsigned>(grid)), dim3(nt), RMS_CL, smem, st, a);
+    }
+    return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(nt), smem, st, a);
+}
+
 template <int DT, int MODEF>
 sq_status launch_rows_dt(RowArgs a, cudaStream_t st)
 {
@@ -502,7 +537,7 @@ sq_status launch_rows_dt(RowArgs a, cudaStream_t st)
     const int64_t vpt = cdiv(nvec, nt);
     // per-column constants in registers when VPT * EPV <= 32, else in shared
     // memory; the norm-output statistic stages its column maxima there
-    const bool reg_rows = vpt * EPV <= 32;
+    const bool reg_rows = vpt * EPV <= 32 && MODE != ROW_RMSNORM;      // as k_rows' REG
     size_t smem = (reg_rows && MODE != ROW_RMS_STAT) ? 0 : static_cast<size_t>(a.K) * 4;
     const int sms = sm_count();
     // Rows held in registers arrive through the shared-memory row ring where
@@ -589,34 +624,7 @@ sq_status launch_rows_dt(RowArgs a, cudaStream_t st)
         } else {
             kern = k_rows<DT, 16, MODEF, ROW_T>;
         }
-        cudaError_t e = cudaSuccess;
-        if (smem > 0) {       // with the kernel's static shared memory it may pass the 48 KB default
-            e = ensure_smem(reinterpret_cast<const void *>(kern), static_cast<int>(smem));
-            if (e != cudaSuccess) return cuda_fail(e);
-        }
-        int per_sm = 0;
-        {   // occupancy per kernel and shared-memory size, queried once
-            std::lock_guard<std::mutex> lk(g_mu);
-            const KernelInfo &ki = kinfo(reinterpret_cast<const void *>(kern));
-            if (ki.per_sm_smem == static_cast<int>(smem)) per_sm = ki.per_sm;
-        }
-        if (per_sm == 0) {
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, nt, smem);
-            if (e != cudaSuccess) return cuda_fail(e);
-            std::lock_guard<std::mutex> lk(g_mu);
-            KernelInfo &ki = kinfo(reinterpret_cast<const void *>(kern));
-            ki.per_sm = per_sm;
-            ki.per_sm_smem = static_cast<int>(smem);
-        }
-        int64_t grid = std::min<int64_t>(a.rows, static_cast<int64_t>(sms) * std::max(1, per_sm));
-        if (MODE == ROW_RMS_STAT && a.rows <= 8 * grid) {
-            // few rows per block: the per-block column atomics dominate, so the
-            // blocks of a cluster combine their maxima first
-            grid = cdiv(grid, RMS_CL) * RMS_CL;       // whole clusters (blocks past the rows idle)
-            e = launch_pdl_cluster_smem(kern, dim3(static_cast<unsigned>(grid)), dim3(nt), RMS_CL, smem, st, a);
-        } else {
-            e = launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(nt), smem, st, a);
-        }
+        const cudaError_t e = launch_row_kernel<MODE>(kern, nt, smem, a, st);
         if (e != cudaSuccess) return cuda_fail(e);
     } else {
         const int64_t grid = std::min<int64_t>(a.rows, static_cast<int64_t>(sms) * 8);

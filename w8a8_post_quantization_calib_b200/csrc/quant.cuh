@@ -162,7 +162,6 @@ constexpr unsigned ERR_ROW_RING = 0x150;
 template <int EPV, bool INRANGE = false, bool F8 = false>
 __device__ __forceinline__ void store_codes(int8_t *dst_row, int64_t v, const float *f)
 {
-    auto q = [](float x) { return INRANGE ? quant8_bits_inrange(x) : quant8_bits(x); };
     if constexpr (F8) {
         if constexpr (EPV == 8) {
             uint2 o;
@@ -172,13 +171,42 @@ __device__ __forceinline__ void store_codes(int8_t *dst_row, int64_t v, const fl
         } else {
             *reinterpret_cast<uint32_t *>(dst_row + v * 4) = e4m3x4_bits(f[0], f[1], f[2], f[3]);
         }
-    } else if constexpr (EPV == 8) {
-        uint2 o;
-        o.x = pack4_bits(q(f[0]), q(f[1]), q(f[2]), q(f[3]));
-        o.y = pack4_bits(q(f[4]), q(f[5]), q(f[6]), q(f[7]));
-        *reinterpret_cast<uint2 *>(dst_row + v * 8) = o;
     } else {
-        *reinterpret_cast<uint32_t *>(dst_row + v * 4) = pack4_bits(q(f[0]), q(f[1]), q(f[2]), q(f[3]));
+        uint32_t b[EPV];
+#pragma unroll
+        for (int e = 0; e < EPV; e += 2) quant8_bits2<INRANGE>(f[e], f[e + 1], b[e], b[e + 1]);
+        if constexpr (EPV == 8) {
+            uint2 o;
+            o.x = pack4_bits(b[0], b[1], b[2], b[3]);
+            o.y = pack4_bits(b[4], b[5], b[6], b[7]);
+            *reinterpret_cast<uint2 *>(dst_row + v * 8) = o;
+        } else {
+            *reinterpret_cast<uint32_t *>(dst_row + v * 4) = pack4_bits(b[0], b[1], b[2], b[3]);
+        }
+    }
+}
+
+// y[e] = fl(x[e] * c[e]) for EPV (even) values, two per packed multiply
+template <int EPV>
+__device__ __forceinline__ void mul_rn_v(float (&y)[EPV], const float (&x)[EPV], const float (&c)[EPV])
+{
+#pragma unroll
+    for (int e = 0; e < EPV; e += 2) {
+        const float2 t = __fmul2_rn(make_float2(x[e], x[e + 1]), make_float2(c[e], c[e + 1]));
+        y[e] = t.x;
+        y[e + 1] = t.y;
+    }
+}
+
+// y[e] = fl(x[e] * k) for one multiplier k
+template <int EPV>
+__device__ __forceinline__ void mul_rn_s(float (&y)[EPV], const float (&x)[EPV], float k)
+{
+#pragma unroll
+    for (int e = 0; e < EPV; e += 2) {
+        const float2 t = __fmul2_rn(make_float2(x[e], x[e + 1]), make_float2(k, k));
+        y[e] = t.x;
+        y[e + 1] = t.y;
     }
 }
 
@@ -241,8 +269,12 @@ __global__ void __launch_bounds__(NT) k_rows(RowArgs p)
     constexpr bool FOLD = (MODEF & ROW_FOLD) != 0;
     constexpr int EPV = VecT<DT>::EPV;
     // per-column constants (and the pass-1 values) in registers; 1024-thread
-    // rows (long rows) keep them in shared memory to stay within 64 registers
-    constexpr bool REG = (VPT * EPV <= 32) && NT <= ROW_T;
+    // rows (long rows) keep them in shared memory to stay within 64 registers,
+    // and so does RMSNorm + quant, whose register row and constants would
+    // leave room for only 2 blocks per SM (80 registers and 3 blocks with the
+    // constants in shared memory: 0.60 -> 0.66 of HBM on 8192-element bf16
+    // rows, 0.67 -> 0.72 on 4096-element fp16 rows)
+    constexpr bool REG = (VPT * EPV <= 32) && NT <= ROW_T && MODE != ROW_RMSNORM;
     static_assert(!RING || (REG && MODE != ROW_ACT_STATIC), "the row ring needs register rows and a row barrier");
     extern __shared__ __align__(128) float4 colv4[];
     __shared__ float red[32];
@@ -440,8 +472,8 @@ __global__ void __launch_bounds__(NT) k_rows(RowArgs p)
                 float f[EPV], c[EPV];
                 widen<DT>(raw[i], f);
                 colc(i, v, c);
-#pragma unroll
-                for (int e = 0; e < EPV; ++e) f[e] = __fmul_rn(__fmul_rn(f[e], c[e]), inv_a_static);
+                mul_rn_v(f, f, c);
+                mul_rn_s(f, f, inv_a_static);
                 if (v < nvec) store_codes<EPV, false, F8>(dst, v, f);
             }
             continue;
@@ -472,6 +504,12 @@ __global__ void __launch_bounds__(NT) k_rows(RowArgs p)
             const float mean = __double2float_rn(mean64);
             const float r_m = __frcp_rn(__fsqrt_rn(__fadd_rn(mean, p.eps)));
             if (tid == 0 && p.rstd_out != nullptr) p.rstd_out[row] = r_m;
+            // pass 2: y = fl(fl(x * r_m) * c_j), then (RMSNorm) v = fl(y * recip(a)).
+            // With the row in registers the values v overwrite it until the
+            // thread's largest magnitude is known: below 127.5 (and not NaN)
+            // no code saturates and the clamp is skipped.  Otherwise the check
+            // is made per vector.
+            float vmax = 0.0f;
 #pragma unroll
             for (int i = 0; i < VPT; ++i) {
                 const int64_t v = static_cast<int64_t>(i) * NT + tid;
@@ -483,15 +521,39 @@ __global__ void __launch_bounds__(NT) k_rows(RowArgs p)
                     widen<DT>(raw[i], f);
                 }
                 colc(i, v, c);
+                mul_rn_s(f, f, r_m);
+                mul_rn_v(f, f, c);
                 if constexpr (MODE == ROW_RMS_STAT) {
 #pragma unroll
-                    for (int e = 0; e < EPV; ++e)
-                        cmax[i][e] = fmaxf(cmax[i][e], fabsf(__fmul_rn(__fmul_rn(f[e], r_m), c[e])));
+                    for (int e = 0; e < EPV; ++e) cmax[i][e] = fmaxf(cmax[i][e], fabsf(f[e]));
+                } else {
+                    mul_rn_s(f, f, inv_a_static);
+                    float m = 0.0f;
+#pragma unroll
+                    for (int e = 0; e < EPV; e += 2) m = max3_abs_nan(m, f[e], f[e + 1]);
+                    if constexpr (REG) {
+#pragma unroll
+                        for (int e = 0; e < EPV; ++e) fk[i][e] = f[e];
+                        vmax = max3_abs_nan(vmax, m, 0.0f);
+                    } else if (v < nvec) {
+                        if (m < 127.5f) store_codes<EPV, true>(dst, v, f);
+                        else store_codes<EPV, false>(dst, v, f);
+                    }
+                }
+            }
+            if constexpr (MODE == ROW_RMSNORM && REG) {
+                if (vmax < 127.5f) {
+#pragma unroll
+                    for (int i = 0; i < VPT; ++i) {
+                        const int64_t v = static_cast<int64_t>(i) * NT + tid;
+                        if (v < nvec) store_codes<EPV, true>(dst, v, fk[i]);
+                    }
                 } else {
 #pragma unroll
-                    for (int e = 0; e < EPV; ++e)
-                        f[e] = __fmul_rn(__fmul_rn(__fmul_rn(f[e], r_m), c[e]), inv_a_static);
-                    if (v < nvec) store_codes<EPV>(dst, v, f);
+                    for (int i = 0; i < VPT; ++i) {
+                        const int64_t v = static_cast<int64_t>(i) * NT + tid;
+                        if (v < nvec) store_codes<EPV, false>(dst, v, fk[i]);
+                    }
                 }
             }
             continue;
@@ -508,11 +570,15 @@ __global__ void __launch_bounds__(NT) k_rows(RowArgs p)
             float f[EPV], c[EPV];
             widen<DT>(raw[i], f);
             colc(i, v, c);
+            if constexpr (FOLD) mul_rn_s(f, f, rf);
+            mul_rn_v(f, f, c);
 #pragma unroll
-            for (int e = 0; e < EPV; ++e) {
-                const float y = __fmul_rn(FOLD ? __fmul_rn(f[e], rf) : f[e], c[e]);
-                mx = fmaxf(mx, fabsf(y));
-                if constexpr (REG) ykeep[i][e] = y;
+            for (int e = 0; e < EPV; e += 2) {
+                mx = max3_abs(mx, f[e], f[e + 1]);
+                if constexpr (REG) {
+                    ykeep[i][e] = f[e];
+                    ykeep[i][e + 1] = f[e + 1];
+                }
             }
         }
         const float sc = scale_from_absmax_q<F8>(block_max(mx, red));
@@ -526,14 +592,14 @@ __global__ void __launch_bounds__(NT) k_rows(RowArgs p)
             const int64_t v = static_cast<int64_t>(i) * NT + tid;
             float f[EPV];
             if constexpr (REG) {
-#pragma unroll
-                for (int e = 0; e < EPV; ++e) f[e] = __fmul_rn(ykeep[i][e], inv);
+                mul_rn_s(f, ykeep[i], inv);
             } else {
                 float c[EPV];
                 widen<DT>(raw[i], f);
                 colc(i, v, c);
-#pragma unroll
-                for (int e = 0; e < EPV; ++e) f[e] = __fmul_rn(__fmul_rn(FOLD ? __fmul_rn(f[e], rf) : f[e], c[e]), inv);
+                if constexpr (FOLD) mul_rn_s(f, f, rf);
+                mul_rn_v(f, f, c);
+                mul_rn_s(f, f, inv);
             }
             if (v < nvec) {
                 if (F8) store_codes<EPV, false, F8>(dst, v, f);
@@ -643,8 +709,8 @@ __global__ void __launch_bounds__(QS_TX *QS_TY)
         auto emit = [&](int64_t row, const uint4 &raw) {
             float f[EPV];
             widen<DT>(raw, f);
-#pragma unroll
-            for (int e = 0; e < EPV; ++e) f[e] = __fmul_rn(__fmul_rn(f[e], c[e]), inv_a);
+            mul_rn_v(f, f, c);
+            mul_rn_s(f, f, inv_a);
             int8_t *dst = out + row * K;
             if constexpr (F8) {
                 if constexpr (EPV == 8) {
@@ -653,14 +719,25 @@ __global__ void __launch_bounds__(QS_TX *QS_TY)
                 } else {
                     __stcs(reinterpret_cast<uint32_t *>(dst + v * 4), e4m3x4_bits(f[0], f[1], f[2], f[3]));
                 }
-            } else if constexpr (EPV == 8) {
-                uint2 o;
-                o.x = pack4_bits(quant8_bits(f[0]), quant8_bits(f[1]), quant8_bits(f[2]), quant8_bits(f[3]));
-                o.y = pack4_bits(quant8_bits(f[4]), quant8_bits(f[5]), quant8_bits(f[6]), quant8_bits(f[7]));
-                __stcs(reinterpret_cast<uint2 *>(dst + v * 8), o);
             } else {
-                __stcs(reinterpret_cast<uint32_t *>(dst + v * 4),
-                       pack4_bits(quant8_bits(f[0]), quant8_bits(f[1]), quant8_bits(f[2]), quant8_bits(f[3])));
+                // the clamp only where a value of the vector reaches 127.5 in
+                // magnitude (or is NaN)
+                float m = 0.0f;
+#pragma unroll
+                for (int e = 0; e < EPV; e += 2) m = max3_abs_nan(m, f[e], f[e + 1]);
+                uint32_t b[EPV];
+                if (m < 127.5f) {
+#pragma unroll
+                    for (int e = 0; e < EPV; e += 2) quant8_bits2<true>(f[e], f[e + 1], b[e], b[e + 1]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < EPV; e += 2) quant8_bits2<false>(f[e], f[e + 1], b[e], b[e + 1]);
+                }
+                if constexpr (EPV == 8)
+                    __stcs(reinterpret_cast<uint2 *>(dst + v * 8),
+                           make_uint2(pack4_bits(b[0], b[1], b[2], b[3]), pack4_bits(b[4], b[5], b[6], b[7])));
+                else
+                    __stcs(reinterpret_cast<uint32_t *>(dst + v * 4), pack4_bits(b[0], b[1], b[2], b[3]));
             }
         };
         if constexpr (ONE) {
