@@ -520,10 +520,10 @@ def test_rmsnorm_absmax(M, d, dt):
 
 @pytest.mark.parametrize("M,K,dt", [(5000, 8192, BF16), (9001, 4096, F16), (3001, 6144, BF16), (2000, 3000, BF16),
                                     (1500, 1032, F16)])
-def test_rmsnorm_pipelined_many_rows(M, K, dt):
+def test_rmsnorm_many_rows_per_block(M, K, dt):
     """RMSNorm + quant and the norm-output statistic with many rows per block
-    (the software-pipelined kernel: row n's sum and r_m overlap row n - 1's
-    second pass through a ring of shared-memory row buffers), at row counts
+    (each block walks rows with the next row's loads in flight; the
+    statistic's rows come through the shared-memory row ring), at row counts
     that are not a multiple of the grid and row lengths with a ragged last
     vector group, bit for bit against the oracle."""
     X = rand_x(M + K + 3, (M, K), dt, 1.0, outliers=max(1, K // 200))
