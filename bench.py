@@ -497,6 +497,20 @@ def run_line(args, build):
     e1.record(stream)
     barrier()
     ms_e2e = e0.elapsed_time(e1) / n2
+    # the PCIe ceiling of the same copies: the step's host inputs alone,
+    # back to back on the copy stream (no compute)
+    big = max(spec.host_in.values(), key=lambda h: h.numel() * h.element_size())
+    with torch.cuda.stream(copy_s):
+        ios[0][next(n for n, h in spec.host_in.items() if h is big)].copy_(big, non_blocking=True)
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    c0.record(copy_s)
+    with torch.cuda.stream(copy_s):
+        for name, hv in spec.host_in.items():
+            ios[0][name].copy_(hv, non_blocking=True)
+    c1.record(copy_s)
+    torch.cuda.synchronize()
+    ms_h2d = c0.elapsed_time(c1)
     del ios, steps_fn
     if world > 1:
         t = torch.tensor([ms_e2e], dtype=torch.float64, device="cuda")
@@ -506,8 +520,10 @@ def run_line(args, build):
     e2e = {"value": world * spec.ops_per_step / (ms_e2e * 1e-3) / 1e12, "unit": "TOPS",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e, "steps": n2,
            "tokens_per_s": world * spec.tokens_per_step / (ms_e2e * 1e-3),
+           "h2d_alone_ms": ms_h2d, "h2d_alone_gbs": h2d / (ms_h2d * 1e-3) / 1e9,
            "note": ("pinned host buffers through the C-ABI calls; every step copies its inputs in and its "
-                    "result out; two device sets, so step k+1's inputs cross PCIe while step k computes")}
+                    "result out; two device sets, so step k+1's inputs cross PCIe while step k computes; "
+                    "h2d_alone_ms: the same input copies alone, back to back (the PCIe floor of a step)")}
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
@@ -832,6 +848,19 @@ def _time_ms(fn, iters, warmup=3, graph=True):
     return e0.elapsed_time(e1) / iters
 
 
+def stream_ceiling_ms(bufs, iters=50):
+    """Device time of one launch that only reads one of `bufs` (rotated, so
+    that every launch streams from HBM): the ceiling of a GEMM that reads
+    the same weight bytes once per launch (libsq_peak's streaming read, 4
+    blocks of 512 threads per SM)."""
+    import torch
+    from w8a8_post_quantization_calib_b200 import peak
+    sink = torch.zeros(1, dtype=torch.int32, device="cuda")
+    blocks = 4 * torch.cuda.get_device_properties(0).multi_processor_count
+    ctr = itertools.count()
+    return _time_ms(lambda: peak.stream_read(bufs[next(ctr) % len(bufs)], blocks, sink), iters)
+
+
 def _dev16(bits, dt):
     import numpy as np
     import torch
@@ -892,6 +921,7 @@ def run_workload(args):
                     sq.linear_w8a8(xq, wcopies[next(ctr2) % len(wcopies)], at, sq.ACT_PER_TOKEN, ws, y,
                                    workspace=work)
                 t_p = _time_ms(pair, 50)
+                t_s = stream_ceiling_ms(wcopies)
                 ops = 2.0 * M * N * K
                 wbytes = N * K + N * 4 + M * K + M * N * 2
                 lines.append({"proj": which, "M": M, "K": K, "N": N,
@@ -900,6 +930,8 @@ def run_workload(args):
                               "gemm_frac_int8_peak": ops / (t_g * 1e-3) / 1e12 / P["int8_tops"],
                               "gemm_gbs": wbytes / (t_g * 1e-3) / 1e9,
                               "gemm_frac_hbm": wbytes / (t_g * 1e-3) / 1e9 / P["hbm_gbs"],
+                              "weight_stream_us": t_s * 1e3,
+                              "gemm_frac_weight_stream": t_s / t_g,
                               "tokens_per_s": M / ((t_q + t_g) * 1e-3),
                               "quant_gemm_chain_us": t_p * 1e3})
         out["lines"] = lines
@@ -967,6 +999,7 @@ def run_workload(args):
             ws = torch.empty(N, device="cuda")
             sq.quant_weight_fp8(W, s, wq8, ws)
             t_wq = _time_ms(lambda: sq.quant_weight_fp8(W, s, wq8, ws), 10)
+            wcopies = [wq8] + [wq8.clone() for _ in range(max(1, -(-3 * 126 * 2**20 // (N * K))))]
             Xall = _dev16(wl.x, bf16)
             for M in (int(t) for t in args.tokens.split(",")):
                 X = Xall[:M]
@@ -974,12 +1007,17 @@ def run_workload(args):
                 at = torch.empty(M, device="cuda")
                 y = torch.empty(M, N, dtype=bf16, device="cuda")
                 t_q = _time_ms(lambda: sq.smooth_quant_act_fp8(X, s, sq.ACT_PER_TOKEN, at, xq8), 50)
-                t_g = _time_ms(lambda: sq.linear_fp8(xq8, wq8, at, sq.ACT_PER_TOKEN, ws, y), 20)
+                ctr = itertools.count()
+                t_g = _time_ms(lambda: sq.linear_fp8(xq8, wcopies[next(ctr) % len(wcopies)], at, sq.ACT_PER_TOKEN,
+                                                     ws, y), 20)
+                t_s = stream_ceiling_ms(wcopies)
                 ops = 2.0 * M * N * K
                 lines.append({"proj": which, "M": M, "K": K, "N": N,
                               "act_quant_us": t_q * 1e3, "act_quant_gbs": M * K * 3 / (t_q * 1e-3) / 1e9,
                               "gemm_us": t_g * 1e3, "gemm_tops": ops / (t_g * 1e-3) / 1e12,
                               "gemm_frac_e4m3_peak": ops / (t_g * 1e-3) / 1e12 / tpk["burst"]["tops"],
+                              "weight_stream_us": t_s * 1e3,
+                              "gemm_frac_weight_stream": t_s / t_g,
                               "weight_quant_us": t_wq * 1e3,
                               "weight_quant_gbs": N * K * 3 / (t_wq * 1e-3) / 1e9})
         out["e4m3_peak"] = tpk

@@ -30,6 +30,23 @@ def test_library_exports_every_declared_symbol():
     assert sorted(EXPORTS) == names          # the binding wraps exactly the declared calls
 
 
+def test_measurement_library_loads_and_exports_its_calls():
+    """libsq_peak.so (the tensor-core peak and streaming-read ceiling used as
+    roofline denominators) loads without a GPU and exports its calls; the
+    streaming read validates its arguments before launching."""
+    from w8a8_post_quantization_calib_b200 import peak
+    lib = peak.lib()
+    for name in ("sqpeak_clusters", "sqpeak_launch", "sqpeak_error_word", "sqpeak_stream_read"):
+        assert hasattr(lib, name), name
+    inval = 1                                    # cudaErrorInvalidValue
+    assert lib.sqpeak_stream_read(None, 16, 1, None, None) == inval
+    assert lib.sqpeak_stream_read(16, 15, 1, None, None) == inval        # bytes not a multiple of 16
+    assert lib.sqpeak_stream_read(8, 16, 1, None, None) == inval         # misaligned
+    assert lib.sqpeak_stream_read(16, 16, 0, None, None) == inval        # no blocks
+    assert lib.sqpeak_launch(0, 0, 1, None) == inval
+    assert lib.sqpeak_launch(0, 1, (1 << 20) + 1, None) == inval
+
+
 def test_host_only_entry_points_without_gpu():
     import w8a8_post_quantization_calib_b200 as sq
     lib = sq.lib()

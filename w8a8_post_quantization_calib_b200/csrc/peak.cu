@@ -10,6 +10,13 @@
 // with CUDA events, so the rate is 2 * 256 * 256 * 128 * iters * clusters /
 // time.  Nothing is read from or written to global memory besides the error
 // word of the bounded wait.
+//
+// The second measurement is the read rate of one launch that streams a
+// buffer once: the ceiling of a decode-size GEMM, which reads its weights
+// once per launch.  Each block of 512 threads streams a contiguous share with
+// 16-byte evict-first loads, four in flight per thread; the loaded words are
+// folded into a value that is written only if it equals an impossible
+// constant, so the loads cannot be dropped.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -17,6 +24,29 @@
 #include "ptx_sm100.cuh"
 
 namespace {
+
+constexpr int SR_THREADS = 512;
+
+__global__ void __launch_bounds__(SR_THREADS) k_stream_read(const uint4 *__restrict__ buf, long long n16,
+                                                            unsigned int *sink)
+{
+    const long long per = (n16 + gridDim.x - 1) / gridDim.x;
+    const long long a = static_cast<long long>(blockIdx.x) * per;
+    const long long b = a + per < n16 ? a + per : n16;
+    uint32_t acc = 0;
+    long long i = a + threadIdx.x;
+    for (; i + 3 * SR_THREADS < b; i += 4 * SR_THREADS) {
+        const uint4 t0 = __ldcs(buf + i), t1 = __ldcs(buf + i + SR_THREADS);
+        const uint4 t2 = __ldcs(buf + i + 2 * SR_THREADS), t3 = __ldcs(buf + i + 3 * SR_THREADS);
+        acc ^= (t0.x ^ t0.y ^ t0.z ^ t0.w) + (t1.x ^ t1.y ^ t1.z ^ t1.w) + (t2.x ^ t2.y ^ t2.z ^ t2.w) +
+               (t3.x ^ t3.y ^ t3.z ^ t3.w);
+    }
+    for (; i < b; i += SR_THREADS) {
+        const uint4 t = __ldcs(buf + i);
+        acc ^= t.x ^ t.y ^ t.z ^ t.w;
+    }
+    if (acc == 0x9e3779b9u && sink != nullptr) *sink = acc;
+}
 
 constexpr int PK_THREADS = 128;
 constexpr int PK_TILE = 128 * 128;           // one 128-row x 128-byte operand tile per CTA
@@ -120,6 +150,19 @@ int sqpeak_launch(int kind, int clusters, int iters, void *stream)
                               : cudaLaunchKernelEx(&cfg, k_mma_peak<0>, iters, tmo);
     if (e == cudaSuccess) e = cudaGetLastError();
     return static_cast<int>(e);
+}
+
+// One launch of the streaming read over `bytes` bytes at `buf` (16-byte
+// aligned, bytes a multiple of 16) with `blocks` blocks of 512 threads on
+// `stream`; `sink` is a device word the kernel may write (never in practice).
+// Returns 0 or a cudaError_t.
+int sqpeak_stream_read(const void *buf, size_t bytes, int blocks, unsigned int *sink, void *stream)
+{
+    if (buf == nullptr || blocks <= 0 || (bytes % 16) != 0 || (reinterpret_cast<uintptr_t>(buf) % 16) != 0)
+        return static_cast<int>(cudaErrorInvalidValue);
+    k_stream_read<<<blocks, SR_THREADS, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint4 *>(buf), static_cast<long long>(bytes / 16), sink);
+    return static_cast<int>(cudaGetLastError());
 }
 
 // First barrier-timeout code recorded by the peak kernel (0 = none), cleared.

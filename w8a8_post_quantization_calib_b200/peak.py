@@ -7,6 +7,10 @@ its launches with CUDA events on the current stream.  ``burst`` is one launch
 of about ``ms`` milliseconds after a warm-up launch (the rate a kernel timed
 alone sees); ``sustained`` is back-to-back launches for about ``seconds``
 (the rate a kernel inside a long step sees under the power cap).
+
+``stream_read`` launches the library's streaming read of one buffer: the
+ceiling of a kernel that reads the same bytes once per launch (a decode-size
+GEMM's weights), against which the bench reports the small-M GEMMs.
 """
 from __future__ import annotations
 
@@ -35,6 +39,9 @@ def lib() -> ctypes.CDLL:
         L.sqpeak_launch.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
         L.sqpeak_error_word.restype = ctypes.c_int
         L.sqpeak_error_word.argtypes = []
+        L.sqpeak_stream_read.restype = ctypes.c_int
+        L.sqpeak_stream_read.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p,
+                                         ctypes.c_void_p]
         _lib = L
     return _lib
 
@@ -75,3 +82,12 @@ def measure(kind: str = "i8", ms: float = 100.0, seconds: float = 0.0) -> dict:
         raise RuntimeError("peak kernel: a bounded wait timed out")
     ops = 2.0 * MACS_PER_ITER * iters * clusters * launches
     return {"tops": ops / (t * 1e-3) / 1e12, "ms": t, "launches": launches, "iters": iters, "clusters": clusters}
+
+
+def stream_read(buf: torch.Tensor, blocks: int, sink: torch.Tensor) -> None:
+    """One launch reading every byte of the contiguous CUDA tensor `buf` once
+    (the ceiling of a kernel that streams it once) on the current stream."""
+    rc = lib().sqpeak_stream_read(buf.data_ptr(), buf.numel() * buf.element_size(), int(blocks), sink.data_ptr(),
+                                  torch.cuda.current_stream().cuda_stream)
+    if rc != 0:
+        raise RuntimeError(f"sqpeak_stream_read: cudaError {rc}")
