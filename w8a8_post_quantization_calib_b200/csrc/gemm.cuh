@@ -483,7 +483,7 @@ __device__ __forceinline__ bool epilogue_sk(const Params &p, uint32_t tbase, int
 // x CS never crosses a tile).  Once its own MMAs are done, the leader (rank
 // 0) no longer needs its pipeline stages: it releases them to the others,
 // which store their int32 partial sums there through distributed shared
-// memory ([rank-1][BN][BM] int32) and arrive on its barrier; the leader adds
+// memory ([rank-1][BN/4][BM][4] int32) and arrive on its barrier; the leader adds
 // them to its own accumulator and applies the epilogue.  Every wait is
 // bounded.
 template <int BN, int EPI, int CS, int KIND, typename TfullWait>
@@ -499,6 +499,12 @@ __device__ __forceinline__ bool epilogue_cs(const Params &p, uint32_t tbase, int
     const bool nok = n < p.N;
     const int m0 = tc * BN;
     const int mval = min(BN, p.M - m0);
+    // partial sums of CTA j + 1 in the leader's stages: [j][BN / 4][BM][4]
+    // int32 (four token columns of one row per 16 bytes), so that a warp's
+    // 16-byte stores and loads cover 512 contiguous bytes
+    auto part_off = [](int j, int g, int row) -> uint32_t {
+        return static_cast<uint32_t>(((j * (BN / 4) + g) * BM + row) * 16);
+    };
     if (!tfull_wait()) return false;
     ptx::tc_fence_after();
     if (rank == 0) {
@@ -518,14 +524,17 @@ __device__ __forceinline__ bool epilogue_cs(const Params &p, uint32_t tbase, int
 #pragma unroll
             for (int j = 1; j < CS; ++j) {
 #pragma unroll
-                for (int i = 0; i < CW; ++i) {
-                    if (c * CW + i < mval) {
-                        uint32_t t;
-                        asm volatile("ld.shared.b32 %0, [%1];"
-                                     : "=r"(t)
-                                     : "r"(sbase + static_cast<uint32_t>((((j - 1) * BN + c * CW + i) * BM + r) * 4))
+                for (int g = 0; g < CW / 4; ++g) {
+                    if (c * CW + 4 * g < mval) {
+                        uint32_t t0, t1, t2, t3;
+                        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(t0), "=r"(t1), "=r"(t2), "=r"(t3)
+                                     : "r"(sbase + part_off(j - 1, c * CW / 4 + g, r))
                                      : "memory");
-                        acc[i] += AccOf<KIND>::from(t);
+                        acc[4 * g] += AccOf<KIND>::from(t0);
+                        acc[4 * g + 1] += AccOf<KIND>::from(t1);
+                        acc[4 * g + 2] += AccOf<KIND>::from(t2);
+                        acc[4 * g + 3] += AccOf<KIND>::from(t3);
                     }
                 }
             }
@@ -556,9 +565,10 @@ __device__ __forceinline__ bool epilogue_cs(const Params &p, uint32_t tbase, int
         tmem_load_chunk(tbase + c * CW, v, CW);
         ptx::tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < CW; ++i)
-            if (c * CW + i < mval)
-                ptx::st_dsmem_u32(remote + static_cast<uint32_t>(((((int)rank - 1) * BN + c * CW + i) * BM + r) * 4), v[i]);
+        for (int g = 0; g < CW / 4; ++g)
+            if (c * CW + 4 * g < mval)
+                ptx::st_dsmem_v4(remote + part_off(static_cast<int>(rank) - 1, c * CW / 4 + g, r), v[4 * g],
+                                 v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
     }
     ptx::fence_acq_rel_cluster();
     ptx::named_bar_sync(1, 128);
