@@ -118,7 +118,7 @@ def _check_fp8_gemm(xq, wq, a, mode, ws, bias32, out_dt, y):
 
 @pytest.mark.parametrize("M,N,K", [(300, 528, 1040), (129, 256, 4096), (16, 1024, 2048), (1, 512, 1024),
                                    (512, 768, 11008), (1, 4096, 11008), (64, 1024, 4096), (128, 2048, 2048),
-                                   (33, 11008, 4096)])
+                                   (33, 11008, 4096), (100, 9600, 1040)])
 @pytest.mark.parametrize("out_dt", [F32, F16, BF16])
 def test_linear_fp8(M, N, K, out_dt):
     g = np.random.default_rng(M * 7 + N + K + out_dt)

@@ -412,6 +412,42 @@ def test_linear_w8a8_small_m_schedules(M, N, K, schedule, request):
     assert bits_equal(got, ref), mismatch_report(got, ref)
 
 
+@pytest.mark.parametrize("M,N,K", [(96, 11008, 4096), (80, 9728, 4112), (65, 12288, 2048), (100, 11008, 528),
+                                   (128, 19456, 4096), (128, 9600, 11008)])
+@pytest.mark.parametrize("out_dt,mode", [(BF16, oracle.PER_TOKEN), (F16, oracle.STATIC), (F32, oracle.PER_TOKEN)])
+def test_linear_w8a8_pair_swapped(M, N, K, out_dt, mode):
+    """64 < M <= 128 with many weight rows runs the CTA-pair kernel with the
+    weights as its A operand and the tokens as B (transposed epilogue):
+    bit-identical to the weight-streaming schedule (sq_debug_inject(2)) and
+    to the oracle on sampled output channels, with bias, per-token and static
+    scales, K a multiple of 128 and not, ragged token and channel tiles."""
+    g = np.random.default_rng(M * 11 + N + K)
+    A = g.integers(-127, 128, (M, K), dtype=np.int8)
+    B = g.integers(-127, 128, (N, K), dtype=np.int8)
+    a = (np.abs(g.standard_normal(1 if mode == oracle.STATIC else M)) * 1e-2 + 1e-3).astype(np.float32)
+    ws = (np.abs(g.standard_normal(N)) * 1e-4 + 1e-5).astype(np.float32)
+    bias = synth.cast(g.standard_normal(N).astype(np.float32), out_dt) if out_dt != F32 else None
+    dA, dB, da, dws = dev(A), dev(B), dev(a), dev(ws)
+    db = dev(bias, out_dt) if bias is not None else None
+    torch_dt = {BF16: torch.bfloat16, F16: torch.float16, F32: torch.float32}[out_dt]
+    y0 = torch.empty(M, N, dtype=torch_dt, device="cuda")
+    sq.lib().sq_debug_inject(2)
+    try:
+        sq.linear_w8a8(dA, dB, da, mode, dws, y0, bias=db)
+        _sync()
+    finally:
+        sq.lib().sq_debug_inject(0)
+    y = torch.full((M, N), float("nan"), dtype=torch_dt, device="cuda")
+    sq.linear_w8a8(dA, dB, da, mode, dws, y, bias=db)
+    _sync()
+    iv = torch.int32 if out_dt == F32 else torch.int16
+    assert torch.equal(y.view(iv), y0.view(iv))
+    idx = np.unique(np.concatenate([np.arange(160), np.arange(N - 160, N), g.integers(0, N, 64)]))
+    ref = oracle.dequant(oracle.gemm_s32(A, B[idx]), a, mode, ws[idx], out_dt,
+                         bias[idx] if bias is not None else None)
+    assert bits_equal(host(y)[:, idx], ref), mismatch_report(host(y)[:, idx], ref)
+
+
 # ------------------------------------------------------------------ a9
 @pytest.mark.parametrize("M,Nh,K", [(300, 256, 512), (129, 384, 1040)])
 def test_gateup_silu(M, Nh, K):

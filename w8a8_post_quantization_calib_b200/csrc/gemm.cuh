@@ -37,7 +37,9 @@ namespace sq {
 namespace gemm {
 
 enum Kind : int { KIND_I8 = 0, KIND_F16 = 1, KIND_F8 = 2 };   // F8: E4M3 x E4M3 -> fp32
-enum Epi : int { EPI_DEQUANT = 0, EPI_S32 = 1, EPI_GATEUP = 2, EPI_F16 = 3 };
+// EPI_DEQUANT_T: the CTA-pair kernel with the weights as its A operand and
+// the tokens as B (small M), writing the dequantised output transposed.
+enum Epi : int { EPI_DEQUANT = 0, EPI_S32 = 1, EPI_GATEUP = 2, EPI_F16 = 3, EPI_DEQUANT_T = 4 };
 
 constexpr int BM = 128;            // MMA M: rows of the A operand per tile
 constexpr int BKB = 128;           // bytes of K per stage (one swizzle row)
@@ -881,6 +883,42 @@ __device__ __forceinline__ void epilogue_tma(const Params &p, const CUtensorMap 
     }
 }
 
+// ---------------------------------------------------------------------------
+// Epilogue of the swapped CTA-pair tile (EPI_DEQUANT_T): TMEM lane = weight
+// row n (output channel), column = token m.  Each thread holds w_scale[n] and
+// bias[n]; the tile's token scales are staged in a_tile.  out[m, n] =
+// dequant(acc, fl(a_m * w_n), bias_n), stored directly: for each token the
+// warp's 32 lanes write 32 consecutive channels.
+// ---------------------------------------------------------------------------
+template <int BN, int KIND>
+__device__ __forceinline__ void epilogue_t(const Params &p, uint32_t tbase, int trow, int tc, int q, int lane,
+                                           const float *a_tile)
+{
+    using AT = typename AccOf<KIND>::T;
+    const int n = trow * BM + q * 32 + lane;
+    const bool nok = n < p.N;
+    const float wsn = nok ? load_scale(p.w_scale, p.scales_f16, n) : 0.0f;
+    const float bn = nok ? load_bias(p.bias, p.out_dt, n) : 0.0f;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+        const int m0 = tc * BN + c * 32;
+        if (m0 >= p.M) break;
+        uint32_t r[32];
+        ptx::tmem_ld32(tbase + c * 32, r);
+        ptx::tmem_ld_wait();
+        if (!nok) continue;
+        const int mval = min(32, p.M - m0);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            if (i < mval) {
+                const int64_t o = static_cast<int64_t>(m0 + i) * p.N + n;
+                store_out(p.out, p.out_dt, o,
+                          dequant(AccOf<KIND>::from(r[i]), __fmul_rn(a_tile[c * 32 + i], wsn), p.bias, bn));
+            }
+        }
+    }
+}
+
 // ===========================================================================
 // CTA-pair variant (cta_group::2): a cluster of two CTAs on two SMs computes a
 // 256 x BN tile.  Each CTA loads its own 128 rows of A and BN/2 rows of B
@@ -968,7 +1006,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     if (warp == 0 && lane == 0) {
         ptx::tma_prefetch_desc(&map_a);
         ptx::tma_prefetch_desc(&map_b);
-        if constexpr (EPI != EPI_GATEUP) ptx::tma_prefetch_desc(&map_o);
+        if constexpr (EPI != EPI_GATEUP && EPI != EPI_DEQUANT_T) ptx::tma_prefetch_desc(&map_o);
     }
     if (warp == 1) {
         ptx::tmem_alloc_pair(ptx::smem_addr(tmem_slot), C::TMEM_COLS);
@@ -1096,6 +1134,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 }
                 const int m = (2 * tr + static_cast<int>(rank)) * BM + q * 32 + lane;
                 if (m < p.M) am = a_scale_of(p, m);
+            } else if constexpr (EPI == EPI_DEQUANT_T) {
+                // the tile's token scales (its columns)
+                const int et = threadIdx.x - 64;
+                for (int t = et; t < BN; t += 128) {
+                    const int m = tc * BN + t;
+                    ws_tile[t] = a_scale_of(p, m < p.M ? m : p.M - 1);
+                }
             } else if constexpr (EPI == EPI_GATEUP) {
                 // w_scale of the tile's gate/up rows, fl(1/s2) of its channels
                 const int et = threadIdx.x - 64;
@@ -1121,6 +1166,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             if constexpr (EPI == EPI_GATEUP)
                 epilogue_gateup<BN, C::STG_BUFS>(p, &map_o, tbase, 2 * tr + static_cast<int>(rank), tc, q, lane,
                                                  ws_tile, bias_tile, stg, nstore);
+            else if constexpr (EPI == EPI_DEQUANT_T)
+                epilogue_t<BN, KIND>(p, tbase, 2 * tr + static_cast<int>(rank), tc, q, lane, ws_tile);
             else
                 epilogue_tma<BN, KIND, EPI, C::STG_BUFS>(p, &map_o, tbase, 2 * tr + static_cast<int>(rank), tc, q, lane, stg,
                                             nstore, ws_tile, bias_tile, am);

@@ -278,7 +278,9 @@ sq_status launch_gemm2(gemm::Params p, const void *a, const void *b, cudaStream_
         if (!make_map3(&ma, a, p.K, p.rows_a, gemm::BM, KBO)) return SQ_ERR_CUDA;
         if (!make_map3(&mb, b, p.K, p.rows_b, BN / 2, KBO)) return SQ_ERR_CUDA;
     }
-    if constexpr (EPI == gemm::EPI_GATEUP) {
+    if constexpr (EPI == gemm::EPI_DEQUANT_T) {
+        std::memset(&mo, 0, sizeof(mo));            // direct stores (see epilogue_t)
+    } else if constexpr (EPI == gemm::EPI_GATEUP) {
         // h [M, N/2] bf16, written with TMA stores when requested
         std::memset(&mo, 0, sizeof(mo));
         if (p.out != nullptr && !make_out_map(&mo, p.out, SQ_BF16, false, p.M, p.N / 2)) return SQ_ERR_CUDA;
@@ -373,6 +375,34 @@ sq_status dispatch_pair(gemm::Params &p, const void *a, const void *b, cudaStrea
     }
 }
 
+// Small M (64 < M <= 128) with many weight rows: the CTA-pair kernel with the
+// weights as its A operand (256 rows per pair, 128 per CTA) and the tokens as
+// B (BN = 128, half per CTA).  The pair's MMA reads the token tile from both
+// CTAs, so each CTA loads only half of it: with one weight tile per CTA, a
+// CTA of the weight-streaming kernel loads its 128 weight rows and the whole
+// token tile (the MLP-7B up projection at M = 128: 512 KB + 512 KB per CTA),
+// a pair CTA its 128 weight rows and half the tokens (768 KB).  Measured on
+// that projection: 22.7 -> 22.05 us at M = 128, 21.4 -> 20.9 at M = 100; at
+// M = 33 and 64 (BN = 64) it was no faster (14.9 -> 15.1, 16.7 -> 16.75 us),
+// so it serves only M > 64.  Its gain is small because a launch that streams
+// the 45 MB of weights once is itself bounded near 10 us.
+template <int KIND>
+sq_status dispatch_pair_t(gemm::Params &p, const void *xq, const void *wq, cudaStream_t st)
+{
+    constexpr int bn = 128;
+    p.rows_a = p.N;
+    p.rows_b = p.M;
+    p.num_kb = static_cast<int>(cdiv(p.K, 128));
+    p.tiles_r = static_cast<int>(cdiv(p.N, 2 * gemm::BM));
+    p.tiles_c = static_cast<int>(cdiv(p.M, bn));
+    p.num_units = p.tiles_r * p.tiles_c;
+    if ((p.K % 128) == 0) {
+        p.num_kb = static_cast<int>(cdiv(p.num_kb, 2));
+        return launch_gemm2<bn, KIND, gemm::EPI_DEQUANT_T, 2>(p, wq, xq, st);
+    }
+    return launch_gemm2<bn, KIND, gemm::EPI_DEQUANT_T, 1>(p, wq, xq, st);
+}
+
 void fill_tiles(gemm::Params &p, int bn, int64_t rows_a, int64_t rows_b)
 {
     p.rows_a = static_cast<int>(rows_a);
@@ -452,6 +482,18 @@ int swap_cluster_split(int64_t M, int64_t N, int64_t K)
     if (2 * tiles > sms) return 1;
     const int64_t c = std::min<int64_t>(sms / tiles, iters);
     return c >= 4 ? 4 : c >= 2 ? 2 : 1;
+}
+
+// The swapped CTA-pair kernel (dispatch_pair_t) serves 64 < M <= 128 where the
+// weight-streaming kernel would run one 128-row weight tile per CTA (no
+// cluster split) and the pair tiles fill at least half of the clusters.
+// Measured on the MLP-7B up projection (86 tiles): see dispatch_pair_t.  The
+// cluster split off (sq_debug_inject(2)) keeps the weight-streaming schedules.
+bool use_pair_t(int64_t M, int64_t N, int64_t K)
+{
+    if (M <= 64 || M > kSwapMaxM || (g_inject & 2)) return false;
+    if (swap_cluster_split(M, N, K) > 1) return false;
+    return 2 * cdiv(N, 2 * gemm::BM) >= sm_count() / 2;
 }
 
 // p.ws_acc / p.ws_cnt must hold a workspace for `grid` CTAs unless grid is
@@ -1141,6 +1183,7 @@ static sq_status linear_w8a8_impl(const int8_t *xq, const int8_t *wq, int64_t M,
     p.bias = bias;
     p.out = y;
     p.out_dt = out_dt;
+    if (use_pair_t(M, N, K)) return dispatch_pair_t<gemm::KIND_I8>(p, xq, wq, st);
     if (M <= kSwapMaxM) {
         const int64_t tiles = swap_tiles(M, N);
         if (const int cs = swap_cluster_split(M, N, K); cs > 1)
@@ -1191,6 +1234,7 @@ sq_status sq_linear_fp8(const uint8_t *xq8, const uint8_t *wq8, int64_t M, int64
     p.out = y;
     p.out_dt = out_dt;
     const cudaStream_t st = as_stream(stream);
+    if (use_pair_t(M, N, K)) return dispatch_pair_t<gemm::KIND_F8>(p, xq8, wq8, st);
     if (M <= kSwapMaxM) {
         // weight streaming (the weights fill the 128-row MMA): the cluster
         // split when one tile per CTA would leave most SMs idle, else one
@@ -1261,6 +1305,7 @@ sq_status sq_linear_w8a8_noalloc(const int8_t *xq, const int8_t *wq, int64_t M, 
     p.out = y;
     p.out_dt = out_dt;
     const cudaStream_t st = as_stream(stream);
+    if (use_pair_t(M, N, K)) return dispatch_pair_t<gemm::KIND_I8>(p, xq, wq, st);   // no scratch
     const int64_t tiles = swap_tiles(M, N);
     if (const int cs = swap_cluster_split(M, N, K); cs > 1)   // partial sums stay on chip: no scratch
         return dispatch_swap<gemm::EPI_DEQUANT>(p, xq, wq, st, tiles, cs);
