@@ -720,19 +720,12 @@ __global__ void __launch_bounds__(QS_TX *QS_TY)
                     __stcs(reinterpret_cast<uint32_t *>(dst + v * 4), e4m3x4_bits(f[0], f[1], f[2], f[3]));
                 }
             } else {
-                // the clamp only where a value of the vector reaches 127.5 in
-                // magnitude (or is NaN)
-                float m = 0.0f;
-#pragma unroll
-                for (int e = 0; e < EPV; e += 2) m = max3_abs_nan(m, f[e], f[e + 1]);
+                // always clamped: skipping the clamp behind a per-vector range
+                // check split the four unrolled rows into separate branches
+                // and measured 8 % slower (0.86 -> 0.79 of HBM)
                 uint32_t b[EPV];
-                if (m < 127.5f) {
 #pragma unroll
-                    for (int e = 0; e < EPV; e += 2) quant8_bits2<true>(f[e], f[e + 1], b[e], b[e + 1]);
-                } else {
-#pragma unroll
-                    for (int e = 0; e < EPV; e += 2) quant8_bits2<false>(f[e], f[e + 1], b[e], b[e + 1]);
-                }
+                for (int e = 0; e < EPV; e += 2) quant8_bits2<false>(f[e], f[e + 1], b[e], b[e + 1]);
                 if constexpr (EPV == 8)
                     __stcs(reinterpret_cast<uint2 *>(dst + v * 8),
                            make_uint2(pack4_bits(b[0], b[1], b[2], b[3]), pack4_bits(b[4], b[5], b[6], b[7])));
