@@ -122,7 +122,8 @@ def test_scales_f16_round_trip(n):
 
 
 @pytest.mark.parametrize("M,N,K,mode", [(300, 528, 1040, oracle.STATIC), (16, 1024, 2048, oracle.PER_TOKEN),
-                                        (1, 4096, 4096, oracle.PER_TOKEN), (512, 768, 4096, oracle.PER_TOKEN)])
+                                        (1, 4096, 4096, oracle.PER_TOKEN), (512, 768, 4096, oracle.PER_TOKEN),
+                                        (100, 11008, 4096, oracle.PER_TOKEN)])
 @pytest.mark.parametrize("out_dt", [F16, BF16])
 def test_linear_f16_scales(M, N, K, mode, out_dt):
     g = np.random.default_rng(M + N + K)

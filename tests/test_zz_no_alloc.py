@@ -76,6 +76,7 @@ def _hook(request):
     (1, 11008, 4096, 1, 2, True),
     (64, 2048, 1024, 0, 1, True),
     (128, 1024, 4096, 0, 0, False),
+    (100, 11008, 4096, 1, 2, True),     # swapped CTA pairs (64 < M <= 128, many weight rows)
     (300, 528, 1040, 1, 1, True),       # large M: no scratch needed
 ])
 def test_noalloc_matches_workspace_entry_point(M, N, K, mode, out_dt, with_bias, _hook):

@@ -2,28 +2,37 @@
 //
 //   acc[i, j] = sum_k A[i, k] * B[j, k]      (A, B K-major in global memory)
 //
-// kind::i8 (s8 x s8 -> s32) for the W8A8 linear, kind::f16 (f16 x f16 -> f32)
-// for the unquantised reference product of the alpha search.
+// kind::i8 (s8 x s8 -> s32) for the W8A8 linear, kind::f8f6f4 (E4M3 x E4M3 ->
+// f32) for its FP8 variant, kind::f16 (f16 x f16 -> f32) for the unquantised
+// reference product of the alpha search.
 //
-// One persistent CTA per SM (192 threads):
-//   warp 0      TMA producer: 128 x 128-byte A tile + BN x 128-byte B tile per
-//               stage, 128-byte swizzle, into a STAGES-deep shared-memory ring
-//   warp 1      MMA issuer: four 128 x BN x 32-byte tcgen05.mma per stage into
-//               a TMEM accumulator; tcgen05.commit frees the stage / hands a
+// Two kernels, each with 192 threads per CTA:
+//   warp 0      TMA producer: the stage's A and B tiles (128-byte swizzle,
+//               one or two 128-byte K blocks per load) into a ring of stages
+//   warp 1      MMA issuer: tcgen05.mma per 32-byte K step into a TMEM
+//               accumulator; tcgen05.commit frees the stage / hands a
 //               finished accumulator to the epilogue
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM lanes
-//               32*(w%4)..+31), dequant / SiLU*mul / requant, global stores
-// TMEM holds two accumulators (2 x BN columns) so the epilogue of tile i
-// overlaps the mainloop of tile i+1.
+//               32*(w%4)..+31), dequant / SiLU*mul / requant, stores
+// TMEM holds two accumulators (2 x BN columns) so that the epilogue of one
+// tile overlaps the mainloop of the next.
 //
-// Orientation.  Normal (CTA pairs, M > 128): A = activations xq [M, K], B =
-// weights wq [N, K]; a TMEM lane is a token row, a column an output channel.
-// Swap (small M): A = weights, B = activations (BN = 16..128 tokens), so the
-// 128-row MMA is filled with weight rows and the kernel streams the weight
-// matrix; a TMEM lane is an output channel, a column a token.  The swap kernel
-// spreads the (tile, K block) iterations evenly over the SMs (stream-K, see
-// k_gemm_swap), combining the partial sums of tiles shared by several CTAs
-// through a workspace.
+// k_gemm2 (M > 128, and the swapped form for 64 < M <= 128): clusters of two
+// CTAs on two SMs, one persistent cluster per SM pair walking tiles in
+// raster groups; the leader issues tcgen05.mma.cta_group::2 (M = 256), each
+// CTA loads its 128 rows of A and BN/2 rows of B.  Normal orientation: A =
+// activations xq [M, K], B = weights wq [N, K]; a TMEM lane is a token row, a
+// column an output channel; TMA stores of the outputs.  Swapped (EPI_DEQUANT_T):
+// A = weights, B = the token tile, output stored transposed.
+//
+// k_gemm_swap (M <= 128): A = weights, B = activations (BN = 16..128 tokens),
+// so the 128-row MMA is filled with weight rows and the kernel streams the
+// weight matrix; a TMEM lane is an output channel, a column a token.  One
+// weight tile per CTA, or, when that would leave most SMs idle, a cluster of
+// 2 or 4 CTAs sharing each tile's K range and combining their partial sums
+// through distributed shared memory.  With the cluster split off, the
+// (tile, K block) iterations may be spread evenly over the SMs (stream-K),
+// the partial sums of shared tiles going through a workspace.
 //
 // Every mbarrier wait is bounded (ptx::wait_bounded): on expiry the kernel
 // records an error code, stops issuing, waits (bounded) for its own TMA loads
