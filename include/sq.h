@@ -290,7 +290,10 @@ sq_status sq_rmsnorm_absmax(const void *x, sq_dtype dt, int64_t M, int64_t d, co
  * 128-row MMA, tokens are its N).  When one 128-row weight tile per SM would
  * leave more than half of the SMs idle, a cluster of 2 or 4 CTAs shares each
  * tile's K range and combines the int32 partial sums in distributed shared
- * memory; no workspace is needed.  The stream-K schedule (iterations shared
+ * memory; no workspace is needed.  For 64 < M <= 128 with more than 74
+ * weight tiles, CTA pairs (cta_group::2) take the weights as their 256-row
+ * operand and half the token tile each, writing the output transposed.  The
+ * stream-K schedule (iterations shared
  * evenly among the SMs, partial sums through global memory) is the fallback
  * when the cluster split is off (sq_debug_inject(2)); it needs
  * `workspace` of sq_linear_workspace_size(M, N, K) bytes (16-byte aligned;
@@ -318,7 +321,8 @@ sq_status sq_linear_w8a8(const int8_t *xq, const int8_t *wq, int64_t M, int64_t 
  * call takes no workspace and runs the same schedules as sq_linear_w8a8, so
  * its results are bit-identical to that call's.  M > 128, and the small-M
  * schedules that keep their partial sums on chip (the cluster split, one tile
- * per CTA), use no scratch at all and accept any shape sq_linear_w8a8
+ * per CTA, the swapped CTA pairs), use no scratch at all and accept any shape
+ * sq_linear_w8a8
  * accepts.  Only the small-M stream-K schedule (the fallback when the cluster
  * split is off, sq_debug_inject(2)) shares weight tiles between CTAs through
  * scratch memory; here that scratch is a fixed array inside the library:
